@@ -1,0 +1,416 @@
+"""Benchmark of the CCA / CCGQA prefill block on B200.
+
+    python bench.py [--gpus N] [--steps K] [--warmup W] [--impl ours|reference] [--workload NAME]
+
+One step = one pass of the whole block (down-projection, preprocessing,
+attention, output projection) over one batch of synthetic input, through the
+C ABI. Default workload: the CCGQA long prefill (B=1, S=16384, E=2048, C=4,
+4 query heads x 128, 2 KV heads, seq-conv kernel 4), the configuration the
+headline metric is quoted on. With N ranks (torchrun) every rank runs its own
+independent sequence batch (weak scaling, no data-path collective); the
+timing is the max over ranks.
+
+Prints one JSON line (rank 0). `--impl reference` times the float64 CPU
+oracle instead, on bounded samples of the same workload.
+"""
+from __future__ import annotations
+
+import argparse
+import datetime
+import hashlib
+import json
+import os
+import statistics
+import subprocess
+import sys
+import time
+
+import numpy as np
+import torch
+
+ROOT = os.path.dirname(os.path.abspath(__file__))
+sys.path.insert(0, ROOT)
+
+import workloads  # noqa: E402
+
+METRIC = "CCA prefill tokens/s and attention TFLOP/s (% bf16 peak) at S=16k, 1 B200"
+DEFAULT_WORKLOAD = "ccgqa_16k_bf16"
+DATASHEET_BF16_TFLOPS = 2250.0
+FALLBACK_PEAKS = {"hbm_gbs": 6650.0, "bf16_tflops": 1590.0, "bf16_tflops_sustained": 1400.0}
+L2_FLUSH_BYTES = 256 << 20
+ATTN_KERNEL_SRC = os.path.join(ROOT, "compressed_latent_space_cca_b200", "csrc", "attn_tc.cu")
+
+
+# ------------------------------------------------------------ host logic --
+def rank_workload(shape: workloads.BlockShape, rank: int) -> workloads.BlockShape:
+    """Weak scaling: each rank owns an independent batch of the same shape,
+    drawn with its own seed."""
+    return shape.replace(seed=shape.seed + 1000 * rank)
+
+
+def aggregate(elapsed_ms: float, tokens_per_rank: int, steps: int, world: int, reduce_max=None):
+    """Whole-job throughput from this rank's timed region: the max elapsed
+    time over ranks covers every rank's tokens."""
+    t = elapsed_ms
+    if reduce_max is not None:
+        t = reduce_max(t)
+    ms_per_step = t / steps
+    value = tokens_per_rank * world / (ms_per_step / 1e3)
+    return value, ms_per_step
+
+
+def algorithmic_work(shape: workloads.BlockShape):
+    B, S, E = shape.batch, shape.seq_len, shape.hidden
+    T = B * S
+    Lq, Lkv, d = shape.latent_q, shape.latent_kv, shape.head_dim
+    Nlat = Lq + 2 * Lkv
+    eb = 2 if shape.dtype == "bf16" else 4
+    return {
+        "down_proj_flops": 2.0 * T * E * Nlat,
+        "attention_flops": 2.0 * B * shape.n_q_heads * S * S * d,   # causal half, 2 GEMMs
+        "out_proj_flops": 2.0 * T * Lq * E,
+        "preproc_bytes": float(T * (Nlat + Lq + 2 * Lkv) * eb),     # read q~k~v~, write q, k, v
+    }
+
+
+def load_peaks():
+    p = os.path.join(ROOT, "MEASURED_PEAKS.json")
+    if os.path.exists(p):
+        with open(p) as f:
+            d = json.load(f)
+        return d, "measured"
+    return dict(FALLBACK_PEAKS), "fallback"
+
+
+def file_sha(path):
+    with open(path, "rb") as f:
+        return hashlib.sha256(f.read()).hexdigest()[:16]
+
+
+def traffic_record():
+    """DRAM bytes per attention launch from the committed ncu summary, valid only
+    while the kernel source is unchanged since the counters were taken."""
+    p = os.path.join(ROOT, "profiles", "traffic.json")
+    if not os.path.exists(p) or not os.path.exists(ATTN_KERNEL_SRC):
+        return None
+    with open(p) as f:
+        rec = json.load(f)
+    if rec.get("source_sha") != file_sha(ATTN_KERNEL_SRC):
+        return None
+    return rec
+
+
+class ClockSampler:
+    """nvidia-smi sampling of SM clocks and throttle reasons during timing."""
+
+    FIELDS = ["clocks.sm", "clocks.max.sm", "power.draw", "clocks_event_reasons.active",
+              "clocks_event_reasons.hw_slowdown", "clocks_event_reasons.hw_thermal_slowdown",
+              "clocks_event_reasons.sw_thermal_slowdown", "clocks_event_reasons.sw_power_cap"]
+
+    def __init__(self, index: int):
+        self.index = index
+        self.proc = None
+        self.path = os.path.join(ROOT, "gpurun_out", f"clocks_rank{index}.csv")
+
+    def start(self):
+        try:
+            os.makedirs(os.path.dirname(self.path), exist_ok=True)
+            self.fh = open(self.path, "w")
+            self.proc = subprocess.Popen(
+                ["nvidia-smi", f"--id={self.index}", "--query-gpu=" + ",".join(self.FIELDS),
+                 "--format=csv,noheader,nounits", "-lms", "100"], stdout=self.fh, stderr=subprocess.DEVNULL)
+        except Exception:
+            self.proc = None
+
+    def stop(self):
+        if self.proc is None:
+            return None
+        self.proc.terminate()
+        try:
+            self.proc.wait(timeout=5)
+        except Exception:
+            self.proc.kill()
+        self.fh.close()
+        sm, mx, reasons = [], None, set()
+        names = ["hw_slowdown", "hw_thermal_slowdown", "sw_thermal_slowdown", "sw_power_cap"]
+        with open(self.path) as f:
+            for line in f:
+                parts = [p.strip() for p in line.split(",")]
+                if len(parts) < len(self.FIELDS):
+                    continue
+                try:
+                    sm.append(float(parts[0]))
+                    mx = float(parts[1])
+                except ValueError:
+                    continue
+                for n, v in zip(names, parts[4:8]):
+                    if v.lower() == "active":
+                        reasons.add(n)
+        if not sm:
+            return None
+        return {"sm_mhz": statistics.median(sm), "sm_max_mhz": mx, "reasons": sorted(reasons),
+                "samples": len(sm)}
+
+
+# ---------------------------------------------------------- oracle timing --
+def oracle_threads():
+    try:
+        from threadpoolctl import threadpool_info
+        n = [p.get("num_threads", 0) for p in threadpool_info() if p.get("user_api") == "blas"]
+        if n:
+            return max(n)
+    except Exception:
+        pass
+    return len(os.sched_getaffinity(0))
+
+
+def oracle_call(shape, inp64, rows):
+    import oracle
+    t0 = time.perf_counter()
+    oracle.cca_block(inp64, shape.n_q_heads, shape.n_kv_heads, shape.head_dim, qk_mean_mode=shape.qk_mean_mode,
+                     use_value_shift=bool(shape.value_shift), use_rope=bool(shape.use_rope),
+                     rope_base=shape.rope_base, softmax_scale=shape.softmax_scale, rows=rows)
+    return time.perf_counter() - t0
+
+
+ROW_SAMPLES = (64, 512)
+
+
+def spaced_rows(S, n):
+    return np.unique(np.linspace(0, S - 1, n).round().astype(np.int64))
+
+
+def oracle_sample_text(shape):
+    return (f"oracle (numpy float64) on the {shape.name} inputs: every per-token stage over all "
+            f"{shape.tokens} tokens, attention and output projection for {ROW_SAMPLES[0]} and "
+            f"{ROW_SAMPLES[1]} evenly spaced query rows per sequence; full-block time extrapolated "
+            f"linearly in the number of query rows")
+
+
+def oracle_extrapolate(times_by_rows, S):
+    (r1, t1), (r2, t2) = times_by_rows
+    per_row = max(0.0, (t2 - t1) / (r2 - r1))
+    return t1 + per_row * (S - r1)
+
+
+def cpu_baseline(shape, inputs):
+    inp64 = workloads.as_float64(inputs)
+    pts = []
+    for r in ROW_SAMPLES:
+        rows = spaced_rows(shape.seq_len, r)
+        pts.append((len(rows), oracle_call(shape, inp64, rows)))
+    t_full = oracle_extrapolate(pts, shape.seq_len)
+    return {"value": shape.tokens / t_full, "unit": "tokens/s", "cores": oracle_threads(), "kind": "oracle",
+            "sample": oracle_sample_text(shape), "extrapolated": True,
+            "sample_seconds": round(sum(t for _, t in pts), 2)}
+
+
+def run_reference(args, shape):
+    rank = int(os.environ.get("RANK", "0"))
+    if rank != 0:
+        return 0
+    inputs = workloads.make_inputs(shape)
+    inp64 = workloads.as_float64(inputs)
+    samples = {r: [] for r in ROW_SAMPLES}
+    for i in range(args.warmup + args.steps):
+        r = ROW_SAMPLES[i % 2]
+        rows = spaced_rows(shape.seq_len, r)
+        t = oracle_call(shape, inp64, rows)
+        if i >= args.warmup:
+            samples[r].append(t)
+    if not samples[ROW_SAMPLES[1]]:  # a single timed step: take the other point from warm-up
+        rows = spaced_rows(shape.seq_len, ROW_SAMPLES[1])
+        samples[ROW_SAMPLES[1]].append(oracle_call(shape, inp64, rows))
+    if not samples[ROW_SAMPLES[0]]:
+        rows = spaced_rows(shape.seq_len, ROW_SAMPLES[0])
+        samples[ROW_SAMPLES[0]].append(oracle_call(shape, inp64, rows))
+    pts = [(len(spaced_rows(shape.seq_len, r)), statistics.mean(samples[r])) for r in ROW_SAMPLES]
+    t_full = oracle_extrapolate(pts, shape.seq_len)
+    value = shape.tokens / t_full
+    cores = oracle_threads()
+    line = {
+        "impl": "reference", "metric": METRIC, "value": value, "unit": "tokens/s", "n_gpus": args.gpus,
+        "steps": args.steps, "warmup": args.warmup, "ms_per_step": t_full * 1e3, "higher_is_better": True,
+        "scaling": "weak", "vs_baseline": None, "dtype": "f64", "data": "synthetic",
+        "config": config_dict(shape, "oracle"),
+        "cpu_baseline": {"value": value, "unit": "tokens/s", "cores": cores, "kind": "oracle",
+                         "sample": oracle_sample_text(shape), "extrapolated": True},
+        "e2e": {"value": value, "unit": "tokens/s", "h2d_bytes_per_step": 0, "d2h_bytes_per_step": 0},
+    }
+    print(json.dumps(line), flush=True)
+    return 0
+
+
+def config_dict(shape, path):
+    return {"workload": shape.name, "batch": shape.batch, "seq_len": shape.seq_len, "hidden": shape.hidden,
+            "C": shape.compression, "n_q_heads": shape.n_q_heads, "n_kv_heads": shape.n_kv_heads,
+            "head_dim": shape.head_dim, "conv_kernel": shape.conv_kernel, "qk_mean_mode": shape.qk_mean_mode,
+            "value_shift": shape.value_shift, "rope_base": shape.rope_base, "path": path,
+            "l2": "flushed between timed steps (256 MiB write)"}
+
+
+# ----------------------------------------------------------------- ours --
+def run_ours(args, shape):
+    import torch.distributed as dist
+
+    import compressed_latent_space_cca_b200 as cca
+
+    world = int(os.environ.get("WORLD_SIZE", "1"))
+    rank = int(os.environ.get("RANK", "0"))
+    local = int(os.environ.get("LOCAL_RANK", "0"))
+    if not torch.cuda.is_available():
+        raise SystemExit("bench.py needs a CUDA device")
+    torch.cuda.set_device(local)
+    dev = torch.device("cuda", local)
+    if world > 1:
+        dist.init_process_group("nccl", timeout=datetime.timedelta(seconds=120), device_id=dev)
+    my_shape = rank_workload(shape, rank)
+    inputs_cpu = workloads.make_inputs(my_shape)
+    cfg = cca.config_from_shape(my_shape)
+    inputs = {k: v.to(dev) for k, v in inputs_cpu.items()}
+    out = cca.alloc_outputs(cfg, dev)
+    ws = cca.alloc_workspace(cfg, dev)
+    flush = torch.empty(L2_FLUSH_BYTES, dtype=torch.uint8, device=dev)
+    stream = torch.cuda.current_stream(dev)
+
+    def barrier():
+        if world > 1:
+            dist.barrier()
+
+    def reduce_max(v):
+        if world == 1:
+            return v
+        t = torch.tensor([v], dtype=torch.float64, device=dev)
+        dist.all_reduce(t, op=dist.ReduceOp.MAX)
+        return float(t.item())
+
+    # which path runs (tensor cores or SIMT) and how many kernels a step launches
+    path_tensor = cca.validate(cfg) == 0 and _tensor_path_ok(cca, cfg, inputs, out, ws)
+    launches_per_step = 4 if path_tensor else 6
+
+    for _ in range(args.warmup):
+        flush.zero_()
+        cca.prefill(cfg, inputs, out=out, workspace=ws)
+    torch.cuda.synchronize()
+    st = cca.poll_device_status()
+    if st != 0:
+        raise SystemExit(f"device status {st} after warm-up")
+
+    evs = [[torch.cuda.Event(enable_timing=True) for _ in range(5)] for _ in range(args.steps)]
+    sampler = ClockSampler(local)
+    sampler.start()
+    time.sleep(0.3)
+    barrier()
+    torch.cuda.synchronize()
+    for i in range(args.steps):
+        flush.zero_()
+        cca.prefill(cfg, inputs, out=out, workspace=ws, stage_events=evs[i])
+    torch.cuda.synchronize()
+    barrier()
+    clocks = sampler.stop()
+    st = cca.poll_device_status()
+    if st != 0:
+        raise SystemExit(f"device status {st} after timing")
+
+    stage = np.array([[evs[i][j].elapsed_time(evs[i][j + 1]) for j in range(4)] for i in range(args.steps)])
+    elapsed = float(stage.sum())
+    value, ms_per_step = aggregate(elapsed, my_shape.tokens, args.steps, world, reduce_max)
+    stage_ms = stage.mean(axis=0)
+    work = algorithmic_work(my_shape)
+
+    # end to end: x from pinned host memory, y back to pinned host memory, one C call per step
+    x_host = inputs_cpu["x"].pin_memory()
+    y_host = torch.empty(tuple(out["y"].shape), dtype=out["y"].dtype).pin_memory()
+    x_dev = torch.empty_like(inputs["x"])
+    weights = {k: v for k, v in inputs.items() if k != "x"}
+    e2e_steps = max(3, min(args.steps, 20))
+    for _ in range(2):
+        cca.prefill_host(cfg, x_host, weights, x_dev, out["y"], y_host, out["k_cache"], out["v_cache"], ws)
+    torch.cuda.synchronize()
+    barrier()
+    e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    e0.record(stream)
+    for _ in range(e2e_steps):
+        cca.prefill_host(cfg, x_host, weights, x_dev, out["y"], y_host, out["k_cache"], out["v_cache"], ws)
+    e1.record(stream)
+    torch.cuda.synchronize()
+    barrier()
+    e2e_val, _ = aggregate(e0.elapsed_time(e1), my_shape.tokens, e2e_steps, world, reduce_max)
+
+    peaks, peak_src = load_peaks()
+    attn_s = stage_ms[2] / 1e3
+    attn_tflops = work["attention_flops"] / attn_s / 1e12
+    peak = float(peaks.get("bf16_tflops", FALLBACK_PEAKS["bf16_tflops"]))
+    traffic = traffic_record()
+    roofline = {
+        "kernel": "attention (tcgen05)" if path_tensor else "attention (SIMT)",
+        "bound": "tensor", "achieved": attn_tflops, "peak": peak, "unit": "TFLOP/s",
+        "frac": attn_tflops / peak, "peak_source": f"{peak_src} bf16 (burst)",
+        "frac_of_datasheet_2250": attn_tflops / DATASHEET_BF16_TFLOPS,
+        "traffic": traffic["dram_bytes_per_launch"] if traffic else None,
+        "algorithmic_flops_per_launch": work["attention_flops"],
+    }
+    hbm = float(peaks.get("hbm_gbs", FALLBACK_PEAKS["hbm_gbs"]))
+    kernels = {
+        "down_proj": {"ms": stage_ms[0], "tflops": work["down_proj_flops"] / (stage_ms[0] / 1e3) / 1e12,
+                      "frac": work["down_proj_flops"] / (stage_ms[0] / 1e3) / 1e12 / peak},
+        "preproc": {"ms": stage_ms[1], "gbs": work["preproc_bytes"] / (stage_ms[1] / 1e3) / 1e9,
+                    "frac": work["preproc_bytes"] / (stage_ms[1] / 1e3) / 1e9 / hbm},
+        "attention": {"ms": stage_ms[2], "tflops": attn_tflops, "frac": attn_tflops / peak},
+        "out_proj": {"ms": stage_ms[3], "tflops": work["out_proj_flops"] / (stage_ms[3] / 1e3) / 1e12,
+                     "frac": work["out_proj_flops"] / (stage_ms[3] / 1e3) / 1e12 / peak},
+    }
+    line = None
+    if rank == 0:
+        line = {
+            "metric": METRIC, "value": value, "unit": "tokens/s", "n_gpus": world, "steps": args.steps,
+            "warmup": args.warmup, "ms_per_step": ms_per_step, "higher_is_better": True, "scaling": "weak",
+            "vs_baseline": None, "dtype": "bf16", "data": "synthetic",
+            "config": config_dict(shape, "tensor" if path_tensor else "simt"),
+            "attention_tflops": attn_tflops,
+            "roofline": roofline,
+            "kernels": kernels,
+            "e2e": {"value": e2e_val, "unit": "tokens/s",
+                    "h2d_bytes_per_step": int(x_host.numel() * x_host.element_size()),
+                    "d2h_bytes_per_step": int(y_host.numel() * y_host.element_size())},
+            "gpu_launches": launches_per_step * args.steps,
+            "clocks": clocks,
+        }
+        if world == 1 and not args.no_cpu_baseline:
+            line["cpu_baseline"] = cpu_baseline(my_shape, inputs_cpu)
+        print(json.dumps(line, default=float), flush=True)
+    if world > 1:
+        dist.barrier()
+        dist.destroy_process_group()
+    return 0
+
+
+def _tensor_path_ok(cca, cfg, inputs, out, ws):
+    try:
+        cca.prefill(cfg, inputs, out=out, workspace=ws, path=cca.CCA_PATH_TENSOR)
+        return True
+    except cca.CcaError as e:
+        if e.status == cca.CCA_ERR_UNSUPPORTED:
+            return False
+        raise
+
+
+def main(argv=None):
+    ap = argparse.ArgumentParser(description=__doc__.split("\n")[0])
+    ap.add_argument("--gpus", type=int, default=1)
+    ap.add_argument("--steps", type=int, default=50)
+    ap.add_argument("--warmup", type=int, default=5)
+    ap.add_argument("--impl", choices=["ours", "reference"], default="ours")
+    ap.add_argument("--workload", default=DEFAULT_WORKLOAD, choices=sorted(workloads.WORKLOADS))
+    ap.add_argument("--no-cpu-baseline", action="store_true", help="skip the oracle timing (rank 0, N=1)")
+    args = ap.parse_args(argv)
+    if args.warmup < 3:
+        raise SystemExit("--warmup must be >= 3")
+    shape = workloads.WORKLOADS[args.workload]
+    if args.impl == "reference":
+        return run_reference(args, shape)
+    return run_ours(args, shape)
+
+
+if __name__ == "__main__":
+    sys.exit(main())

@@ -1,0 +1,231 @@
+"""B200 prefill of one Compressed Convolutional Attention (CCA / CCGQA) block.
+
+Thin Python binding over the C ABI in include/cca.h (libcca.so, built in-tree
+by `python -m compressed_latent_space_cca_b200.build`). This module only
+marshals arguments: shapes, dtypes and pointers are checked and passed
+through; every step of the block runs in the library's CUDA kernels. PyTorch
+is used for device memory and streams. If libcca.so is missing, every call
+raises: there is no CPU or PyTorch fallback.
+"""
+from __future__ import annotations
+
+import ctypes
+from typing import Dict, Optional, Sequence
+
+import torch
+
+from . import _capi
+from ._capi import (  # noqa: F401
+    CCA_BF16,
+    CCA_ERR_CUDA,
+    CCA_ERR_DEVICE_TIMEOUT,
+    CCA_ERR_INVALID_ARG,
+    CCA_ERR_UNSUPPORTED,
+    CCA_ERR_WORKSPACE,
+    CCA_F32,
+    CCA_OK,
+    CCA_PATH_AUTO,
+    CCA_PATH_SIMT,
+    CCA_PATH_TENSOR,
+    CcaConfig,
+    CcaWorkspaceLayout,
+)
+
+INPUT_NAMES = ("x", "W_q", "W_k", "W_v", "convq_seq", "convq_chan", "convk_seq", "convk_chan", "W_o")
+
+_DT = {CCA_F32: torch.float32, CCA_BF16: torch.bfloat16}
+_DT_CODE = {torch.float32: CCA_F32, torch.bfloat16: CCA_BF16, "f32": CCA_F32, "bf16": CCA_BF16}
+
+
+class CcaError(RuntimeError):
+    def __init__(self, status: int, where: str):
+        lib = _capi.load()
+        msg = lib.cca_last_error_message().decode()
+        super().__init__(f"{where}: {lib.cca_status_string(status).decode()} ({msg})")
+        self.status = status
+
+
+def library() -> ctypes.CDLL:
+    return _capi.load()
+
+
+def make_config(*, batch: int, seq_len: int, hidden: int, n_q_heads: int, n_kv_heads: int, head_dim: int,
+                conv_kernel: int = 4, dtype="bf16", out_dtype=None, qk_mean_mode: int = 3,
+                value_shift: int = 1, use_rope: int = 1, rope_base: float = 10000.0,
+                softmax_scale: float = 0.0, C: Optional[int] = None) -> CcaConfig:
+    """Build a cca_config_t. C defaults to hidden / (n_q_heads * head_dim)."""
+    dt = _DT_CODE[dtype]
+    odt = dt if out_dtype is None else _DT_CODE[out_dtype]
+    if C is None:
+        C = hidden // max(1, n_q_heads * head_dim)
+    return CcaConfig(batch, seq_len, hidden, C, n_q_heads, n_kv_heads, head_dim, conv_kernel, qk_mean_mode,
+                     value_shift, use_rope, rope_base, softmax_scale, dt, odt)
+
+
+def config_from_shape(shape, out_dtype=None) -> CcaConfig:
+    """cca_config_t from any object with the BlockShape attributes."""
+    return make_config(batch=shape.batch, seq_len=shape.seq_len, hidden=shape.hidden,
+                       n_q_heads=shape.n_q_heads, n_kv_heads=shape.n_kv_heads, head_dim=shape.head_dim,
+                       conv_kernel=shape.conv_kernel, dtype=shape.dtype, out_dtype=out_dtype,
+                       qk_mean_mode=shape.qk_mean_mode, value_shift=shape.value_shift,
+                       use_rope=shape.use_rope, rope_base=shape.rope_base, softmax_scale=shape.softmax_scale)
+
+
+def validate(cfg: CcaConfig) -> int:
+    return library().cca_validate(ctypes.byref(cfg))
+
+
+def workspace_size(cfg: CcaConfig) -> int:
+    return library().cca_workspace_size(ctypes.byref(cfg))
+
+
+def workspace_layout(cfg: CcaConfig) -> CcaWorkspaceLayout:
+    out = CcaWorkspaceLayout()
+    st = library().cca_workspace_layout(ctypes.byref(cfg), ctypes.byref(out))
+    if st != CCA_OK:
+        raise CcaError(st, "cca_workspace_layout")
+    return out
+
+
+def _shapes(cfg: CcaConfig) -> Dict[str, tuple]:
+    B, S, E = cfg.batch, cfg.seq_len, cfg.hidden
+    Lq, Lkv, K = cfg.n_q_heads * cfg.head_dim, cfg.n_kv_heads * cfg.head_dim, cfg.conv_kernel
+    d = cfg.head_dim
+    return {
+        "x": (B, S, E), "W_q": (Lq, E), "W_k": (Lkv, E), "W_v": (Lkv, E),
+        "convq_seq": (Lq, K), "convq_chan": (cfg.n_q_heads, d, d),
+        "convk_seq": (Lkv, K), "convk_chan": (cfg.n_kv_heads, d, d), "W_o": (E, Lq),
+        "y": (B, S, E), "k_cache": (B, S, cfg.n_kv_heads, d), "v_cache": (B, S, cfg.n_kv_heads, d),
+        "conv_state": (B, (K - 1) * (Lq + cfg.n_kv_heads * d) + cfg.n_kv_heads * d),
+    }
+
+
+def _check(t: torch.Tensor, name: str, shape: tuple, dtype: torch.dtype, device) -> int:
+    if not isinstance(t, torch.Tensor):
+        raise TypeError(f"{name} must be a torch.Tensor")
+    if t.device != device:
+        raise ValueError(f"{name} is on {t.device}, expected {device}")
+    if tuple(t.shape) != tuple(shape):
+        raise ValueError(f"{name} has shape {tuple(t.shape)}, expected {tuple(shape)}")
+    if t.dtype != dtype:
+        raise ValueError(f"{name} has dtype {t.dtype}, expected {dtype}")
+    if not t.is_contiguous():
+        raise ValueError(f"{name} must be contiguous")
+    return t.data_ptr()
+
+
+def alloc_outputs(cfg: CcaConfig, device, conv_state: bool = False) -> Dict[str, torch.Tensor]:
+    sh = _shapes(cfg)
+    dt, odt = _DT[cfg.dtype], _DT[cfg.out_dtype]
+    out = {
+        "y": torch.empty(sh["y"], dtype=odt, device=device),
+        "k_cache": torch.empty(sh["k_cache"], dtype=dt, device=device),
+        "v_cache": torch.empty(sh["v_cache"], dtype=dt, device=device),
+    }
+    if conv_state:
+        out["conv_state"] = torch.empty(sh["conv_state"], dtype=dt, device=device)
+    return out
+
+
+def alloc_workspace(cfg: CcaConfig, device) -> torch.Tensor:
+    n = workspace_size(cfg)
+    if n == 0:
+        raise CcaError(validate(cfg), "cca_workspace_size")
+    return torch.empty(n, dtype=torch.uint8, device=device)  # caching allocator: 512-byte aligned
+
+
+def prefill(cfg: CcaConfig, inputs: Dict[str, torch.Tensor], *, out: Optional[Dict[str, torch.Tensor]] = None,
+            workspace: Optional[torch.Tensor] = None, conv_state: bool = False, path: int = CCA_PATH_AUTO,
+            stage_events: Optional[Sequence[torch.cuda.Event]] = None,
+            stream: Optional[torch.cuda.Stream] = None) -> Dict[str, torch.Tensor]:
+    """Run cca_prefill_ex on `stream` (default: the current stream).
+
+    inputs: the nine tensors of INPUT_NAMES on one CUDA device, dtype cfg.dtype.
+    Returns {"y", "k_cache", "v_cache", ["conv_state"], "workspace"}.
+    """
+    x = inputs["x"]
+    device = x.device
+    if device.type != "cuda":
+        raise ValueError("inputs must be CUDA tensors")
+    sh = _shapes(cfg)
+    dt = _DT[cfg.dtype]
+    ptrs = [_check(inputs[n], n, sh[n], dt, device) for n in INPUT_NAMES]
+    if out is None:
+        out = alloc_outputs(cfg, device, conv_state)
+    y = _check(out["y"], "y", sh["y"], _DT[cfg.out_dtype], device)
+    kc = _check(out["k_cache"], "k_cache", sh["k_cache"], dt, device)
+    vc = _check(out["v_cache"], "v_cache", sh["v_cache"], dt, device)
+    cs = _check(out["conv_state"], "conv_state", sh["conv_state"], dt, device) if "conv_state" in out else None
+    if workspace is None:
+        workspace = alloc_workspace(cfg, device)
+    if stream is None:
+        stream = torch.cuda.current_stream(device)
+    opts = _capi.CcaPrefillOpts()
+    opts.path = path
+    if stage_events is not None:
+        if len(stage_events) != 5:
+            raise ValueError("stage_events needs 5 events")
+        arr = (ctypes.c_void_p * 5)(*[ev.cuda_event for ev in stage_events])
+        opts.stage_events = ctypes.cast(arr, ctypes.POINTER(ctypes.c_void_p))
+    st = library().cca_prefill_ex(ctypes.byref(cfg), *ptrs, y, kc, vc, cs, workspace.data_ptr(),
+                                  workspace.numel(), ctypes.c_void_p(stream.cuda_stream), ctypes.byref(opts))
+    if st != CCA_OK:
+        raise CcaError(st, "cca_prefill")
+    res = dict(out)
+    res["workspace"] = workspace
+    return res
+
+
+def prefill_host(cfg: CcaConfig, x_host: torch.Tensor, weights: Dict[str, torch.Tensor], x_dev: torch.Tensor,
+                 y_dev: torch.Tensor, y_host: torch.Tensor, k_cache: torch.Tensor, v_cache: torch.Tensor,
+                 workspace: torch.Tensor, stream: Optional[torch.cuda.Stream] = None) -> None:
+    """cca_prefill_host: x from (pinned) host memory, y back to (pinned) host memory."""
+    device = x_dev.device
+    sh = _shapes(cfg)
+    dt = _DT[cfg.dtype]
+    if x_host.device.type != "cpu" or y_host.device.type != "cpu":
+        raise ValueError("x_host and y_host must be host tensors")
+    if tuple(x_host.shape) != sh["x"] or x_host.dtype != dt or not x_host.is_contiguous():
+        raise ValueError("x_host shape/dtype mismatch")
+    if tuple(y_host.shape) != sh["y"] or y_host.dtype != _DT[cfg.out_dtype] or not y_host.is_contiguous():
+        raise ValueError("y_host shape/dtype mismatch")
+    wp = [_check(weights[n], n, sh[n], dt, device) for n in INPUT_NAMES[1:]]
+    xd = _check(x_dev, "x_dev", sh["x"], dt, device)
+    yd = _check(y_dev, "y_dev", sh["y"], _DT[cfg.out_dtype], device)
+    kc = _check(k_cache, "k_cache", sh["k_cache"], dt, device)
+    vc = _check(v_cache, "v_cache", sh["v_cache"], dt, device)
+    if stream is None:
+        stream = torch.cuda.current_stream(device)
+    st = library().cca_prefill_host(ctypes.byref(cfg), x_host.data_ptr(), xd, *wp, yd, y_host.data_ptr(), kc, vc,
+                                    None, workspace.data_ptr(), workspace.numel(),
+                                    ctypes.c_void_p(stream.cuda_stream))
+    if st != CCA_OK:
+        raise CcaError(st, "cca_prefill_host")
+
+
+def poll_device_status(stream: Optional[torch.cuda.Stream] = None) -> int:
+    """Synchronize and return the device status (CCA_OK or CCA_ERR_DEVICE_TIMEOUT ...)."""
+    s = stream.cuda_stream if stream is not None else torch.cuda.current_stream().cuda_stream
+    return library().cca_poll_device_status(ctypes.c_void_p(s))
+
+
+def selftest_wait_timeout(timeout_us: int, stream: Optional[torch.cuda.Stream] = None) -> int:
+    s = stream.cuda_stream if stream is not None else torch.cuda.current_stream().cuda_stream
+    return library().cca_selftest_wait_timeout(timeout_us, ctypes.c_void_p(s))
+
+
+def workspace_view(cfg: CcaConfig, workspace: torch.Tensor) -> Dict[str, torch.Tensor]:
+    """Views of the intermediates left in the workspace by the last call."""
+    L = workspace_layout(cfg)
+    dt = _DT[cfg.dtype]
+    T = cfg.batch * cfg.seq_len
+    Lq, Lkv = cfg.n_q_heads * cfg.head_dim, cfg.n_kv_heads * cfg.head_dim
+    eb = L.elem_bytes
+
+    def region(off, width):
+        return workspace[off:off + T * width * eb].view(dt).view(cfg.batch, cfg.seq_len, width)
+    return {
+        "qkv_lat": region(L.qkv_lat_offset, Lq + 2 * Lkv),
+        "q": region(L.q_offset, Lq),
+        "o": region(L.o_offset, Lq),
+    }

@@ -1,0 +1,447 @@
+// C ABI of the CCA / CCGQA prefill library: validation, workspace layout,
+// path choice and the launch sequence
+//   down-projection -> preprocessing -> attention -> output projection
+// of one block ("Compressed Convolutional Attention", gist.science/es/paper/
+// 2510.04476, section 2). Every step runs in this library's kernels.
+#include <math.h>
+#include <stdio.h>
+
+#include <mutex>
+#include <string>
+
+#include "../../include/cca.h"
+#include "cca_common.cuh"
+#include "launch.h"
+
+namespace cca {
+
+// Device error word, set by bounded waits that give up.
+__device__ unsigned g_device_error = 0;
+
+namespace {
+
+thread_local std::string t_last_error;
+
+cca_status_t fail(cca_status_t st, const std::string& msg) {
+  t_last_error = msg;
+  return st;
+}
+
+constexpr size_t kAlign = 256;
+size_t align_up(size_t v) { return (v + kAlign - 1) / kAlign * kAlign; }
+
+struct DeviceInfo {
+  bool init = false;
+  int major = 0, minor = 0, sms = 0;
+  unsigned* err_ptr = nullptr;
+};
+constexpr int kMaxDevices = 64;
+DeviceInfo g_dev[kMaxDevices];
+std::mutex g_dev_mu;
+
+cca_status_t device_info(DeviceInfo** out) {
+  int dev = 0;
+  cudaError_t e = cudaGetDevice(&dev);
+  if (e != cudaSuccess) return fail(CCA_ERR_CUDA, std::string("cudaGetDevice: ") + cudaGetErrorString(e));
+  if (dev < 0 || dev >= kMaxDevices) return fail(CCA_ERR_UNSUPPORTED, "device index out of range");
+  std::lock_guard<std::mutex> lk(g_dev_mu);
+  DeviceInfo& di = g_dev[dev];
+  if (!di.init) {
+    cudaDeviceProp prop;
+    if ((e = cudaGetDeviceProperties(&prop, dev)) != cudaSuccess)
+      return fail(CCA_ERR_CUDA, std::string("cudaGetDeviceProperties: ") + cudaGetErrorString(e));
+    void* p = nullptr;
+    if ((e = cudaGetSymbolAddress(&p, g_device_error)) != cudaSuccess)
+      return fail(CCA_ERR_CUDA, std::string("cudaGetSymbolAddress: ") + cudaGetErrorString(e));
+    di.major = prop.major;
+    di.minor = prop.minor;
+    di.sms = prop.multiProcessorCount;
+    di.err_ptr = static_cast<unsigned*>(p);
+    di.init = true;
+  }
+  *out = &di;
+  return CCA_OK;
+}
+
+bool is_dtype(int v) { return v == CCA_F32 || v == CCA_BF16; }
+
+cca_status_t check_config(const cca_config_t* c, BlockDims* dm) {
+  if (c == nullptr) return fail(CCA_ERR_INVALID_ARG, "cfg is NULL");
+  if (c->batch < 1 || c->seq_len < 1 || c->hidden < 1)
+    return fail(CCA_ERR_INVALID_ARG, "batch, seq_len and hidden must be >= 1");
+  if (c->n_q_heads < 1 || c->n_kv_heads < 1) return fail(CCA_ERR_INVALID_ARG, "head counts must be >= 1");
+  if (c->n_q_heads % c->n_kv_heads != 0)
+    return fail(CCA_ERR_INVALID_ARG, "n_q_heads must be a multiple of n_kv_heads");
+  if (c->head_dim < 2 || c->head_dim % 2 != 0) return fail(CCA_ERR_INVALID_ARG, "head_dim must be even and >= 2");
+  if (c->C < 1) return fail(CCA_ERR_INVALID_ARG, "C must be >= 1");
+  if ((long long)c->C * c->n_q_heads * c->head_dim != c->hidden)
+    return fail(CCA_ERR_INVALID_ARG, "hidden must equal C * n_q_heads * head_dim");
+  if (c->conv_kernel < 1 || c->conv_kernel > 64) return fail(CCA_ERR_INVALID_ARG, "conv_kernel must be in [1, 64]");
+  if (c->qk_mean_mode < 0 || c->qk_mean_mode > 3) return fail(CCA_ERR_INVALID_ARG, "qk_mean_mode must be in [0, 3]");
+  if (c->value_shift != 0 && c->value_shift != 1) return fail(CCA_ERR_INVALID_ARG, "value_shift must be 0 or 1");
+  if (c->use_rope != 0 && c->use_rope != 1) return fail(CCA_ERR_INVALID_ARG, "use_rope must be 0 or 1");
+  if (c->use_rope && !(c->rope_base > 1.0f && isfinite(c->rope_base)))
+    return fail(CCA_ERR_INVALID_ARG, "rope_base must be finite and > 1");
+  if (!(c->softmax_scale >= 0.0f) || !isfinite(c->softmax_scale))
+    return fail(CCA_ERR_INVALID_ARG, "softmax_scale must be finite and >= 0");
+  if (!is_dtype(c->dtype) || !is_dtype(c->out_dtype)) return fail(CCA_ERR_INVALID_ARG, "unknown dtype");
+  if (c->head_dim > 128) return fail(CCA_ERR_UNSUPPORTED, "head_dim > 128 is not supported");
+  const long long T = (long long)c->batch * c->seq_len;
+  const long long Nlat = (long long)(c->n_q_heads + 2 * c->n_kv_heads) * c->head_dim;
+  if (T > (1ll << 30) || Nlat > (1 << 20) || c->hidden > (1 << 20))
+    return fail(CCA_ERR_UNSUPPORTED, "tensor extent too large");
+  if (dm) {
+    dm->B = c->batch;
+    dm->S = c->seq_len;
+    dm->E = c->hidden;
+    dm->nq = c->n_q_heads;
+    dm->nkv = c->n_kv_heads;
+    dm->d = c->head_dim;
+    dm->K = c->conv_kernel;
+    dm->G = c->n_q_heads / c->n_kv_heads;
+    dm->Lq = c->n_q_heads * c->head_dim;
+    dm->Lkv = c->n_kv_heads * c->head_dim;
+    dm->Nlat = dm->Lq + 2 * dm->Lkv;
+    dm->T = T;
+    dm->qk_mean_mode = c->qk_mean_mode;
+    dm->value_shift = c->value_shift;
+    dm->use_rope = c->use_rope;
+    dm->rope_base = c->rope_base;
+    dm->scale = c->softmax_scale > 0.f ? c->softmax_scale : 1.0f / sqrtf((float)c->head_dim);
+    dm->bf16 = c->dtype == CCA_BF16;
+    dm->out_bf16 = c->out_dtype == CCA_BF16;
+  }
+  return CCA_OK;
+}
+
+cca_workspace_layout_t layout_of(const BlockDims& dm) {
+  cca_workspace_layout_t L;
+  const size_t eb = dm.bf16 ? 2 : 4;
+  L.elem_bytes = eb;
+  size_t off = 0;
+  L.qkv_lat_offset = off;
+  off = align_up(off + (size_t)dm.T * dm.Nlat * eb);
+  L.q_offset = off;
+  off = align_up(off + (size_t)dm.T * dm.Lq * eb);
+  L.o_offset = off;
+  off = align_up(off + (size_t)dm.T * dm.Lq * eb);
+  L.sched_offset = off;
+  off = align_up(off + 256);
+  L.total_bytes = off;
+  return L;
+}
+
+bool aligned16(const void* p) { return (reinterpret_cast<uintptr_t>(p) & 15u) == 0; }
+
+struct Resolved {
+  BlockDims dm;
+  bool tensor;  // tcgen05 path
+};
+
+cca_status_t resolve(const cca_config_t* cfg, int path, Resolved* r) {
+  cca_status_t st = check_config(cfg, &r->dm);
+  if (st != CCA_OK) return st;
+  DeviceInfo* di = nullptr;
+  if ((st = device_info(&di)) != CCA_OK) return st;
+  const BlockDims& dm = r->dm;
+  const bool tc_ok = di->major == 10 && dm.bf16 && dm.d == 128 && gemm_tc_supported(dm.T, dm.Nlat, dm.E) &&
+                     gemm_tc_supported(dm.T, dm.E, dm.Lq) && attention_tc_supported(dm);
+  if (path == CCA_PATH_TENSOR && !tc_ok)
+    return fail(CCA_ERR_UNSUPPORTED, "tensor-core path needs sm_100, bf16 and head_dim 128");
+  if (path != CCA_PATH_AUTO && path != CCA_PATH_SIMT && path != CCA_PATH_TENSOR)
+    return fail(CCA_ERR_INVALID_ARG, "unknown path");
+  r->tensor = (path == CCA_PATH_TENSOR) || (path == CCA_PATH_AUTO && tc_ok);
+  return CCA_OK;
+}
+
+cca_status_t cuda_fail(const char* what, cudaError_t e) {
+  return fail(CCA_ERR_CUDA, std::string(what) + ": " + cudaGetErrorString(e));
+}
+
+cca_status_t run_block(const Resolved& r, BlockPtrs p, cudaStream_t stream, void* const* ev) {
+  const BlockDims& dm = r.dm;
+  DeviceInfo* di = nullptr;
+  cca_status_t st = device_info(&di);
+  if (st != CCA_OK) return st;
+  p.dev_err = di->err_ptr;
+  cudaError_t e;
+  auto mark = [&](int i) -> cudaError_t {
+    return ev ? cudaEventRecord(static_cast<cudaEvent_t>(ev[i]), stream) : cudaSuccess;
+  };
+  const size_t eb = dm.bf16 ? 2 : 4;
+  if ((e = mark(0)) != cudaSuccess) return cuda_fail("event", e);
+  // 1. down-projection: q~ | k~ | v~ = x [W_q; W_k; W_v]^T
+  if (r.tensor) {
+    GemmTcArgs a{};
+    a.A = p.x;
+    a.M = dm.T;
+    a.K = dm.E;
+    a.B[0] = p.Wq;
+    a.B[1] = p.Wk;
+    a.B[2] = p.Wv;
+    a.nrows[0] = dm.Lq;
+    a.nrows[1] = dm.Lkv;
+    a.nrows[2] = dm.Lkv;
+    a.nb = 3;
+    a.C = p.qkv_lat;
+    a.ldc = dm.Nlat;
+    a.out_bf16 = true;
+    a.dev_err = p.dev_err;
+    if ((e = launch_gemm_tc(a, stream)) != cudaSuccess) return cuda_fail("down-projection (tcgen05)", e);
+  } else {
+    char* out = static_cast<char*>(p.qkv_lat);
+    const void* Ws[3] = {p.Wq, p.Wk, p.Wv};
+    const int ns[3] = {dm.Lq, dm.Lkv, dm.Lkv};
+    int col = 0;
+    for (int i = 0; i < 3; ++i) {
+      if ((e = launch_gemm_simt(dm.bf16, dm.bf16, p.x, dm.E, Ws[i], dm.E, out + (size_t)col * eb, dm.Nlat, dm.T,
+                                ns[i], dm.E, stream)) != cudaSuccess)
+        return cuda_fail("down-projection (SIMT)", e);
+      col += ns[i];
+    }
+  }
+  if ((e = mark(1)) != cudaSuccess) return cuda_fail("event", e);
+  // 2. seq conv, channel conv, QK-mean, RoPE, value shift; KV cache written here
+  if ((e = launch_preproc_simt(dm, p, stream)) != cudaSuccess) return cuda_fail("preprocessing", e);
+  if ((e = launch_conv_state(dm, p, stream)) != cudaSuccess) return cuda_fail("conv state", e);
+  if ((e = mark(2)) != cudaSuccess) return cuda_fail("event", e);
+  // 3. causal attention on the compressed heads
+  if (r.tensor) {
+    if ((e = launch_attention_tc(dm, p.q, p.k_cache, p.v_cache, p.o, p.sched, p.dev_err, stream)) != cudaSuccess)
+      return cuda_fail("attention (tcgen05)", e);
+  } else {
+    if ((e = launch_attention_simt(dm, p.q, p.k_cache, p.v_cache, p.o, stream)) != cudaSuccess)
+      return cuda_fail("attention (SIMT)", e);
+  }
+  if ((e = mark(3)) != cudaSuccess) return cuda_fail("event", e);
+  // 4. output projection y = o W_o^T
+  if (r.tensor) {
+    GemmTcArgs a{};
+    a.A = p.o;
+    a.M = dm.T;
+    a.K = dm.Lq;
+    a.B[0] = p.Wo;
+    a.nrows[0] = dm.E;
+    a.nb = 1;
+    a.C = p.y;
+    a.ldc = dm.E;
+    a.out_bf16 = dm.out_bf16;
+    a.dev_err = p.dev_err;
+    if ((e = launch_gemm_tc(a, stream)) != cudaSuccess) return cuda_fail("output projection (tcgen05)", e);
+  } else {
+    if ((e = launch_gemm_simt(dm.bf16, dm.out_bf16, p.o, dm.Lq, p.Wo, dm.Lq, p.y, dm.E, dm.T, dm.E, dm.Lq,
+                              stream)) != cudaSuccess)
+      return cuda_fail("output projection (SIMT)", e);
+  }
+  if ((e = mark(4)) != cudaSuccess) return cuda_fail("event", e);
+  return CCA_OK;
+}
+
+cca_status_t prepare(const cca_config_t* cfg, int path, const void* const* ins, void* const* outs, void* conv_state,
+                     void* workspace, size_t workspace_bytes, Resolved* r, BlockPtrs* p) {
+  cca_status_t st = resolve(cfg, path, r);
+  if (st != CCA_OK) return st;
+  static const char* in_names[9] = {"x", "W_q", "W_k", "W_v", "convq_seq", "convq_chan", "convk_seq", "convk_chan",
+                                    "W_o"};
+  for (int i = 0; i < 9; ++i) {
+    if (ins[i] == nullptr) return fail(CCA_ERR_INVALID_ARG, std::string(in_names[i]) + " is NULL");
+    if (!aligned16(ins[i])) return fail(CCA_ERR_INVALID_ARG, std::string(in_names[i]) + " is not 16-byte aligned");
+  }
+  static const char* out_names[3] = {"y", "k_cache", "v_cache"};
+  for (int i = 0; i < 3; ++i) {
+    if (outs[i] == nullptr) return fail(CCA_ERR_INVALID_ARG, std::string(out_names[i]) + " is NULL");
+    if (!aligned16(outs[i])) return fail(CCA_ERR_INVALID_ARG, std::string(out_names[i]) + " is not 16-byte aligned");
+  }
+  if (conv_state != nullptr && !aligned16(conv_state))
+    return fail(CCA_ERR_INVALID_ARG, "conv_state is not 16-byte aligned");
+  const cca_workspace_layout_t L = layout_of(r->dm);
+  if (workspace == nullptr) return fail(CCA_ERR_WORKSPACE, "workspace is NULL");
+  if ((reinterpret_cast<uintptr_t>(workspace) & (kAlign - 1)) != 0)
+    return fail(CCA_ERR_WORKSPACE, "workspace is not 256-byte aligned");
+  if (workspace_bytes < L.total_bytes)
+    return fail(CCA_ERR_WORKSPACE, "workspace smaller than cca_workspace_size()");
+  char* ws = static_cast<char*>(workspace);
+  p->x = ins[0];
+  p->Wq = ins[1];
+  p->Wk = ins[2];
+  p->Wv = ins[3];
+  p->cq_seq = ins[4];
+  p->cq_chan = ins[5];
+  p->ck_seq = ins[6];
+  p->ck_chan = ins[7];
+  p->Wo = ins[8];
+  p->y = outs[0];
+  p->k_cache = outs[1];
+  p->v_cache = outs[2];
+  p->conv_state = conv_state;
+  p->qkv_lat = ws + L.qkv_lat_offset;
+  p->q = ws + L.q_offset;
+  p->o = ws + L.o_offset;
+  p->sched = ws + L.sched_offset;
+  p->dev_err = nullptr;
+  return CCA_OK;
+}
+
+}  // namespace
+
+int num_sms() {
+  DeviceInfo* di = nullptr;
+  if (device_info(&di) != CCA_OK) return 148;
+  return di->sms;
+}
+
+EncodeTiledFn get_encode_tiled() {
+  static EncodeTiledFn fn = nullptr;
+  static std::once_flag once;
+  std::call_once(once, [] {
+    void* p = nullptr;
+    cudaDriverEntryPointQueryResult q;
+    if (cudaGetDriverEntryPoint("cuTensorMapEncodeTiled", &p, cudaEnableDefault, &q) == cudaSuccess &&
+        q == cudaDriverEntryPointSuccess)
+      fn = reinterpret_cast<EncodeTiledFn>(p);
+  });
+  return fn;
+}
+
+// -------------------------------------------------------- self-test kernel --
+namespace {
+__global__ void wait_timeout_selftest_kernel(unsigned* err, unsigned long long limit_ns) {
+  __shared__ __align__(8) uint64_t bar;
+  const uint32_t a = smem_u32(&bar);
+  if (threadIdx.x == 0) {
+    mbar_init(a, 1);
+    fence_mbar_init();
+  }
+  __syncthreads();
+  // Nothing ever arrives on this barrier: the bounded wait must give up.
+  if (threadIdx.x == 0) (void)mbar_wait_bounded(a, 0, err, nullptr, limit_ns);
+}
+}  // namespace
+
+cudaError_t launch_wait_timeout_selftest(unsigned* dev_err, unsigned long long limit_ns, cudaStream_t stream) {
+  wait_timeout_selftest_kernel<<<1, 32, 0, stream>>>(dev_err, limit_ns);
+  return cudaGetLastError();
+}
+
+}  // namespace cca
+
+// ============================================================== C ABI ==
+using namespace cca;
+
+extern "C" {
+
+int cca_version(void) { return CCA_VERSION; }
+
+const char* cca_status_string(cca_status_t s) {
+  switch (s) {
+    case CCA_OK: return "ok";
+    case CCA_ERR_INVALID_ARG: return "invalid argument";
+    case CCA_ERR_UNSUPPORTED: return "unsupported configuration";
+    case CCA_ERR_WORKSPACE: return "workspace missing or too small";
+    case CCA_ERR_CUDA: return "CUDA error";
+    case CCA_ERR_DEVICE_TIMEOUT: return "device-side wait timed out";
+  }
+  return "unknown status";
+}
+
+const char* cca_last_error_message(void) { return t_last_error.c_str(); }
+
+cca_status_t cca_validate(const cca_config_t* cfg) {
+  BlockDims dm;
+  cca_status_t st = check_config(cfg, &dm);
+  if (st == CCA_OK) t_last_error.clear();
+  return st;
+}
+
+size_t cca_workspace_size(const cca_config_t* cfg) {
+  BlockDims dm;
+  if (check_config(cfg, &dm) != CCA_OK) return 0;
+  return layout_of(dm).total_bytes;
+}
+
+cca_status_t cca_workspace_layout(const cca_config_t* cfg, cca_workspace_layout_t* out) {
+  if (out == nullptr) return fail(CCA_ERR_INVALID_ARG, "out is NULL");
+  BlockDims dm;
+  cca_status_t st = check_config(cfg, &dm);
+  if (st != CCA_OK) return st;
+  *out = layout_of(dm);
+  return CCA_OK;
+}
+
+cca_status_t cca_prefill_ex(const cca_config_t* cfg, const void* x, const void* W_q, const void* W_k,
+                            const void* W_v, const void* convq_seq, const void* convq_chan, const void* convk_seq,
+                            const void* convk_chan, const void* W_o, void* y, void* k_cache, void* v_cache,
+                            void* conv_state, void* workspace, size_t workspace_bytes, void* stream,
+                            const cca_prefill_opts_t* opts) {
+  const void* ins[9] = {x, W_q, W_k, W_v, convq_seq, convq_chan, convk_seq, convk_chan, W_o};
+  void* outs[3] = {y, k_cache, v_cache};
+  Resolved r;
+  BlockPtrs p;
+  const int path = opts ? opts->path : CCA_PATH_AUTO;
+  cca_status_t st = prepare(cfg, path, ins, outs, conv_state, workspace, workspace_bytes, &r, &p);
+  if (st != CCA_OK) return st;
+  return run_block(r, p, static_cast<cudaStream_t>(stream), opts ? opts->stage_events : nullptr);
+}
+
+cca_status_t cca_prefill(const cca_config_t* cfg, const void* x, const void* W_q, const void* W_k, const void* W_v,
+                         const void* convq_seq, const void* convq_chan, const void* convk_seq,
+                         const void* convk_chan, const void* W_o, void* y, void* k_cache, void* v_cache,
+                         void* conv_state, void* workspace, size_t workspace_bytes, void* stream) {
+  return cca_prefill_ex(cfg, x, W_q, W_k, W_v, convq_seq, convq_chan, convk_seq, convk_chan, W_o, y, k_cache,
+                        v_cache, conv_state, workspace, workspace_bytes, stream, nullptr);
+}
+
+cca_status_t cca_prefill_host(const cca_config_t* cfg, const void* x_host, void* x_dev, const void* W_q,
+                              const void* W_k, const void* W_v, const void* convq_seq, const void* convq_chan,
+                              const void* convk_seq, const void* convk_chan, const void* W_o, void* y_dev,
+                              void* y_host, void* k_cache, void* v_cache, void* conv_state, void* workspace,
+                              size_t workspace_bytes, void* stream) {
+  if (x_host == nullptr || y_host == nullptr) return fail(CCA_ERR_INVALID_ARG, "host buffer is NULL");
+  const void* ins[9] = {x_dev, W_q, W_k, W_v, convq_seq, convq_chan, convk_seq, convk_chan, W_o};
+  void* outs[3] = {y_dev, k_cache, v_cache};
+  Resolved r;
+  BlockPtrs p;
+  cca_status_t st = prepare(cfg, CCA_PATH_AUTO, ins, outs, conv_state, workspace, workspace_bytes, &r, &p);
+  if (st != CCA_OK) return st;
+  cudaStream_t s = static_cast<cudaStream_t>(stream);
+  const size_t xbytes = (size_t)r.dm.T * r.dm.E * (r.dm.bf16 ? 2 : 4);
+  const size_t ybytes = (size_t)r.dm.T * r.dm.E * (r.dm.out_bf16 ? 2 : 4);
+  cudaError_t e = cudaMemcpyAsync(x_dev, x_host, xbytes, cudaMemcpyHostToDevice, s);
+  if (e != cudaSuccess) return cuda_fail("copy x to device", e);
+  if ((st = run_block(r, p, s, nullptr)) != CCA_OK) return st;
+  e = cudaMemcpyAsync(y_host, y_dev, ybytes, cudaMemcpyDeviceToHost, s);
+  if (e != cudaSuccess) return cuda_fail("copy y to host", e);
+  return CCA_OK;
+}
+
+cca_status_t cca_poll_device_status(void* stream) {
+  DeviceInfo* di = nullptr;
+  cca_status_t st = device_info(&di);
+  if (st != CCA_OK) return st;
+  cudaStream_t s = static_cast<cudaStream_t>(stream);
+  cudaError_t e = cudaStreamSynchronize(s);
+  if (e != cudaSuccess) return cuda_fail("stream synchronize", e);
+  unsigned h = 0;
+  if ((e = cudaMemcpy(&h, di->err_ptr, sizeof(h), cudaMemcpyDeviceToHost)) != cudaSuccess)
+    return cuda_fail("read device error word", e);
+  if (h != 0) {
+    unsigned zero = 0;
+    if ((e = cudaMemcpy(di->err_ptr, &zero, sizeof(zero), cudaMemcpyHostToDevice)) != cudaSuccess)
+      return cuda_fail("clear device error word", e);
+    return fail(CCA_ERR_DEVICE_TIMEOUT, "a bounded device-side wait gave up");
+  }
+  return CCA_OK;
+}
+
+cca_status_t cca_selftest_wait_timeout(unsigned timeout_us, void* stream) {
+  if (timeout_us < 1 || timeout_us > 5000000u) return fail(CCA_ERR_INVALID_ARG, "timeout_us must be in [1, 5e6]");
+  DeviceInfo* di = nullptr;
+  cca_status_t st = device_info(&di);
+  if (st != CCA_OK) return st;
+  cudaError_t e = launch_wait_timeout_selftest(di->err_ptr, (unsigned long long)timeout_us * 1000ull,
+                                               static_cast<cudaStream_t>(stream));
+  if (e != cudaSuccess) return cuda_fail("self-test launch", e);
+  return CCA_OK;
+}
+
+}  // extern "C"

@@ -1,0 +1,77 @@
+// Internal launch interface between the C ABI (cca_api.cu) and the kernels.
+#pragma once
+
+#include <cuda.h>
+#include <cuda_runtime.h>
+#include <stddef.h>
+#include <stdint.h>
+
+namespace cca {
+
+// Shape and options of one block, resolved from cca_config_t.
+struct BlockDims {
+  int B, S, E, nq, nkv, d, K;
+  int G;        // nq / nkv
+  int Lq, Lkv;  // nq*d, nkv*d
+  int Nlat;     // Lq + 2*Lkv: width of the down-projection output
+  long long T;  // B*S
+  int qk_mean_mode, value_shift, use_rope;
+  float rope_base, scale;
+  bool bf16;      // element type of inputs, intermediates and the KV cache
+  bool out_bf16;  // element type of y
+};
+
+// Pointers of one call (all device memory).
+struct BlockPtrs {
+  const void *x, *Wq, *Wk, *Wv, *cq_seq, *cq_chan, *ck_seq, *ck_chan, *Wo;
+  void *y, *k_cache, *v_cache, *conv_state;
+  void *qkv_lat, *q, *o, *sched;
+  unsigned* dev_err;
+};
+
+// ---- SIMT path (any dtype, any even head_dim <= 128) ----
+// C[M, ldc] (cols [0,N)) = A[M,K] (row stride lda) * B[N,K]^T (row stride ldb)
+cudaError_t launch_gemm_simt(bool in_bf16, bool out_bf16, const void* A, long long lda, const void* Bm,
+                             long long ldb, void* C, long long ldc, long long M, int N, int K,
+                             cudaStream_t stream);
+cudaError_t launch_attention_simt(const BlockDims& dm, const void* q, const void* k, const void* v, void* o,
+                                  cudaStream_t stream);
+
+// ---- preprocessing (seq conv, channel conv, QK-mean, RoPE, value shift) ----
+cudaError_t launch_preproc_simt(const BlockDims& dm, const BlockPtrs& p, cudaStream_t stream);
+cudaError_t launch_conv_state(const BlockDims& dm, const BlockPtrs& p, cudaStream_t stream);
+
+// ---- tensor-core path (bf16, head_dim 128, sm_100a) ----
+bool gemm_tc_supported(long long M, int N, int K);
+// C[M, ldc] (cols [0,N)) = A[M,K] * [B0; B1; B2][N,K]^T, where the B operand
+// is split by rows into up to three separate matrices of n0, n1, n2 rows.
+struct GemmTcArgs {
+  const void* A;
+  long long M;
+  int K;
+  const void* B[3];
+  int nrows[3];
+  int nb;
+  void* C;
+  long long ldc;
+  bool out_bf16;
+  unsigned* dev_err;
+};
+cudaError_t launch_gemm_tc(const GemmTcArgs& a, cudaStream_t stream);
+
+bool attention_tc_supported(const BlockDims& dm);
+cudaError_t launch_attention_tc(const BlockDims& dm, const void* q, const void* k, const void* v, void* o,
+                                void* sched, unsigned* dev_err, cudaStream_t stream);
+
+// ---- misc ----
+cudaError_t launch_wait_timeout_selftest(unsigned* dev_err, unsigned long long limit_ns, cudaStream_t stream);
+
+// cuTensorMapEncodeTiled from the driver, fetched once through the runtime.
+typedef CUresult (*EncodeTiledFn)(CUtensorMap*, CUtensorMapDataType, cuuint32_t, void*, const cuuint64_t*,
+                                  const cuuint64_t*, const cuuint32_t*, const cuuint32_t*, CUtensorMapInterleave,
+                                  CUtensorMapSwizzle, CUtensorMapL2promotion, CUtensorMapFloatOOBfill);
+EncodeTiledFn get_encode_tiled();
+
+int num_sms();
+
+}  // namespace cca

@@ -1,0 +1,234 @@
+// Latent preprocessing of one CCA / CCGQA block, general SIMT version
+// (any even head_dim <= 128, fp32 or bf16 storage, fp32 arithmetic).
+//
+// "Compressed Convolutional Attention" (gist.science/es/paper/2510.04476),
+// section 2.B: on the compressed q~ and k~ a causal convolution along the
+// sequence, then a convolution across the channels of each head; the mean of
+// q and k taken before and after the convolutions is added; the value shift
+// gives half the value channels the previous token. Section 3 item 2: RoPE is
+// applied directly in the latent.
+//
+// One CTA handles TT tokens of one sequence for one KV group g: the G query
+// heads of the group and its K/V head, because the QK-mean couples exactly
+// those heads. The K-1 tokens before the tile are loaded as a halo.
+#include <math.h>
+
+#include "cca_common.cuh"
+#include "launch.h"
+
+namespace cca {
+namespace {
+
+constexpr int PP_TT = 8;       // tokens per CTA
+constexpr int PP_THREADS = 256;
+
+template <typename T>
+__global__ void __launch_bounds__(PP_THREADS) preproc_simt_kernel(
+    const T* __restrict__ qkv, const T* __restrict__ cq_seq, const T* __restrict__ cq_chan,
+    const T* __restrict__ ck_seq, const T* __restrict__ ck_chan, T* __restrict__ qout, T* __restrict__ kout,
+    T* __restrict__ vout, int S, int nq, int nkv, int d, int K, int mode, int vshift, int use_rope,
+    float rope_base) {
+  extern __shared__ float sm[];
+  const int G = nq / nkv;
+  const int H1 = G + 1;  // G query heads + the K head of the group
+  const int R = PP_TT + K - 1;
+  const int Lq = nq * d, Lkv = nkv * d, Nlat = Lq + 2 * Lkv;
+  const int half = d / 2;
+  float* zin = sm;                       // [H1][R][d]   latents incl. halo
+  float* sconv = zin + H1 * R * d;       // [H1][TT][d]  after the seq conv
+  float* cconv = sconv + H1 * PP_TT * d; // [H1][TT][d]  after the channel conv
+  float* rcos = cconv + H1 * PP_TT * d;  // [TT][d/2]
+  float* rsin = rcos + PP_TT * half;     // [TT][d/2]
+
+  const int tid = threadIdx.x;
+  const int t0 = blockIdx.x * PP_TT;
+  const int g = blockIdx.y, b = blockIdx.z;
+  const long long rowbase = (long long)b * S;
+
+  for (int e = tid; e < H1 * R * d; e += PP_THREADS) {
+    int hh = e / (R * d), rem = e % (R * d), row = rem / d, i = rem % d;
+    int t = t0 - (K - 1) + row;
+    int col = (hh < G) ? (g * G + hh) * d + i : Lq + g * d + i;
+    zin[e] = (t >= 0 && t < S) ? ld_f(qkv + (rowbase + t) * Nlat + col) : 0.f;
+  }
+  if (use_rope) {
+    const double two_pi = 6.283185307179586476925286766559;
+    for (int e = tid; e < PP_TT * half; e += PP_THREADS) {
+      int tt = e / half, i = e % half;
+      double theta = pow((double)rope_base, -2.0 * (double)i / (double)d);
+      double ang = (double)(t0 + tt) * theta;
+      double red = ang - two_pi * rint(ang / two_pi);  // exact enough: |ang| < 2^17
+      double sv, cv;
+      sincos(red, &sv, &cv);
+      rcos[e] = (float)cv;
+      rsin[e] = (float)sv;
+    }
+  }
+  __syncthreads();
+
+  // causal depthwise conv along the sequence; tap j reads token t-K+1+j
+  for (int e = tid; e < H1 * PP_TT * d; e += PP_THREADS) {
+    int hh = e / (PP_TT * d), rem = e % (PP_TT * d), tt = rem / d, i = rem % d;
+    const T* w = (hh < G) ? cq_seq + (long long)((g * G + hh) * d + i) * K : ck_seq + (long long)(g * d + i) * K;
+    const float* z = zin + (hh * R + tt) * d + i;
+    float acc = 0.f;
+    for (int j = 0; j < K; ++j) acc = fmaf(ld_f(w + j), z[j * d], acc);
+    sconv[e] = acc;
+  }
+  __syncthreads();
+
+  // per-head channel mix: one warp per output channel, lanes split the sum
+  {
+    const int warp = tid >> 5, lane = tid & 31, nwarps = PP_THREADS / 32;
+    for (int row = warp; row < H1 * d; row += nwarps) {
+      int hh = row / d, i = row % d;
+      const T* W = (hh < G) ? cq_chan + ((long long)(g * G + hh) * d + i) * d : ck_chan + ((long long)g * d + i) * d;
+      float wv[4];
+#pragma unroll
+      for (int m = 0; m < 4; ++m) {
+        int j = lane + 32 * m;
+        wv[m] = (j < d) ? ld_f(W + j) : 0.f;
+      }
+      for (int tt = 0; tt < PP_TT; ++tt) {
+        const float* s = sconv + (hh * PP_TT + tt) * d;
+        float part = 0.f;
+#pragma unroll
+        for (int m = 0; m < 4; ++m) {
+          int j = lane + 32 * m;
+          if (j < d) part = fmaf(wv[m], s[j], part);
+        }
+#pragma unroll
+        for (int off = 16; off > 0; off >>= 1) part += __shfl_xor_sync(0xffffffffu, part, off);
+        if (lane == 0) cconv[(hh * PP_TT + tt) * d + i] = part;
+      }
+    }
+  }
+  __syncthreads();
+
+  // QK-mean (before / after the convs), RoPE, store q and the K cache
+  const float invG = 1.f / (float)G;
+  auto combined = [&](int hh, int tt, int i) -> float {
+    const float c = cconv[(hh * PP_TT + tt) * d + i];
+    const float zc = zin[(hh * R + tt + K - 1) * d + i];
+    float r = c;
+    if (hh < G) {
+      if (mode & 1) r += 0.5f * (zc + zin[(G * R + tt + K - 1) * d + i]);
+      if (mode & 2) r += 0.5f * (c + cconv[(G * PP_TT + tt) * d + i]);
+    } else {
+      if (mode & 1) {
+        float mq = 0.f;
+        for (int h2 = 0; h2 < G; ++h2) mq += zin[(h2 * R + tt + K - 1) * d + i];
+        r += 0.5f * (mq * invG + zc);
+      }
+      if (mode & 2) {
+        float mc = 0.f;
+        for (int h2 = 0; h2 < G; ++h2) mc += cconv[(h2 * PP_TT + tt) * d + i];
+        r += 0.5f * (mc * invG + c);
+      }
+    }
+    return r;
+  };
+  for (int e = tid; e < H1 * PP_TT * half; e += PP_THREADS) {
+    int hh = e / (PP_TT * half), rem = e % (PP_TT * half), tt = rem / half, i = rem % half;
+    int t = t0 + tt;
+    if (t >= S) continue;
+    float x1 = combined(hh, tt, i), x2 = combined(hh, tt, i + half);
+    float o1 = x1, o2 = x2;
+    if (use_rope) {
+      float c = rcos[tt * half + i], s = rsin[tt * half + i];
+      o1 = x1 * c - x2 * s;
+      o2 = x2 * c + x1 * s;
+    }
+    T* dst = (hh < G) ? qout + (rowbase + t) * Lq + (long long)(g * G + hh) * d
+                      : kout + (rowbase + t) * Lkv + (long long)g * d;
+    st_f(dst + i, o1);
+    st_f(dst + i + half, o2);
+  }
+
+  // value shift: channels [Lkv/2, Lkv) come from the previous token
+  for (int e = tid; e < PP_TT * d; e += PP_THREADS) {
+    int tt = e / d, i = e % d;
+    int t = t0 + tt;
+    if (t >= S) continue;
+    int gc = g * d + i;
+    int src = (vshift && gc >= Lkv / 2) ? t - 1 : t;
+    T* dst = vout + (rowbase + t) * Lkv + gc;
+    if (src >= 0)
+      *dst = qkv[(rowbase + src) * Nlat + Lq + Lkv + gc];
+    else
+      st_f(dst, 0.f);
+  }
+}
+
+// Conv state per sequence: the last K-1 rows of q~ and of k~ and the last row
+// of v~, zero rows before the sequence start.
+template <typename T>
+__global__ void conv_state_kernel(const T* __restrict__ qkv, T* __restrict__ state, int S, int Lq, int Lkv,
+                                  int K) {
+  const int b = blockIdx.x;
+  const int Nlat = Lq + 2 * Lkv;
+  const long long per = (long long)(K - 1) * (Lq + Lkv) + Lkv;
+  T* dst = state + b * per;
+  const long long rowbase = (long long)b * S;
+  for (long long e = threadIdx.x; e < per; e += blockDim.x) {
+    int t, col;
+    if (e < (long long)(K - 1) * Lq) {
+      t = S - (K - 1) + (int)(e / Lq);
+      col = (int)(e % Lq);
+    } else if (e < (long long)(K - 1) * (Lq + Lkv)) {
+      long long e2 = e - (long long)(K - 1) * Lq;
+      t = S - (K - 1) + (int)(e2 / Lkv);
+      col = Lq + (int)(e2 % Lkv);
+    } else {
+      t = S - 1;
+      col = Lq + Lkv + (int)(e - (long long)(K - 1) * (Lq + Lkv));
+    }
+    if (t >= 0)
+      dst[e] = qkv[(rowbase + t) * Nlat + col];
+    else
+      st_f(dst + e, 0.f);
+  }
+}
+
+}  // namespace
+
+cudaError_t launch_preproc_simt(const BlockDims& dm, const BlockPtrs& p, cudaStream_t stream) {
+  const int H1 = dm.G + 1, R = PP_TT + dm.K - 1;
+  size_t smem = sizeof(float) * ((size_t)H1 * R * dm.d + 2 * (size_t)H1 * PP_TT * dm.d + (size_t)PP_TT * dm.d);
+  dim3 grid((dm.S + PP_TT - 1) / PP_TT, dm.nkv, dm.B);
+  cudaError_t e;
+  if (dm.bf16) {
+    using T = __nv_bfloat16;
+    auto kern = preproc_simt_kernel<T>;
+    if ((e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem)) != cudaSuccess)
+      return e;
+    kern<<<grid, PP_THREADS, smem, stream>>>((const T*)p.qkv_lat, (const T*)p.cq_seq, (const T*)p.cq_chan,
+                                             (const T*)p.ck_seq, (const T*)p.ck_chan, (T*)p.q, (T*)p.k_cache,
+                                             (T*)p.v_cache, dm.S, dm.nq, dm.nkv, dm.d, dm.K, dm.qk_mean_mode,
+                                             dm.value_shift, dm.use_rope, dm.rope_base);
+  } else {
+    using T = float;
+    auto kern = preproc_simt_kernel<T>;
+    if ((e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem)) != cudaSuccess)
+      return e;
+    kern<<<grid, PP_THREADS, smem, stream>>>((const T*)p.qkv_lat, (const T*)p.cq_seq, (const T*)p.cq_chan,
+                                             (const T*)p.ck_seq, (const T*)p.ck_chan, (T*)p.q, (T*)p.k_cache,
+                                             (T*)p.v_cache, dm.S, dm.nq, dm.nkv, dm.d, dm.K, dm.qk_mean_mode,
+                                             dm.value_shift, dm.use_rope, dm.rope_base);
+  }
+  return cudaGetLastError();
+}
+
+cudaError_t launch_conv_state(const BlockDims& dm, const BlockPtrs& p, cudaStream_t stream) {
+  if (p.conv_state == nullptr) return cudaSuccess;
+  if (dm.bf16)
+    conv_state_kernel<__nv_bfloat16><<<dm.B, 256, 0, stream>>>((const __nv_bfloat16*)p.qkv_lat,
+                                                                (__nv_bfloat16*)p.conv_state, dm.S, dm.Lq,
+                                                                dm.Lkv, dm.K);
+  else
+    conv_state_kernel<float><<<dm.B, 256, 0, stream>>>((const float*)p.qkv_lat, (float*)p.conv_state, dm.S,
+                                                        dm.Lq, dm.Lkv, dm.K);
+  return cudaGetLastError();
+}
+
+}  // namespace cca

@@ -1,0 +1,213 @@
+/*
+ * cca.h - C ABI of the B200 prefill library for one Compressed Convolutional
+ * Attention (CCA) / CCGQA block.
+ *
+ * The operation is the block described in "Compressed Convolutional
+ * Attention: Efficient Attention in a Compressed Latent Space"
+ * (gist.science/es/paper/2510.04476, section 2; French twin
+ * gist.science/fr/paper/2510.04476, section 2):
+ *
+ *   q~, k~, v~ = x W_q^T, x W_k^T, x W_v^T        latent width E/C  (es 2.A)
+ *   q, k       = causal seq conv -> per-head channel conv of q~, k~ (es 2.B.1)
+ *                + QK-mean before and after the convs             (es 2.B.2)
+ *                then RoPE in the latent                          (es 3, item 2)
+ *   v          = value shift of v~: the upper half of the latent
+ *                channels comes from the previous token           (es 2.B.3)
+ *   o          = causal softmax(q k^T / sqrt(d)) v, K/V head g serves the
+ *                query heads g*G .. g*G+G-1 (G = n_q / n_kv)      (es 2.A, 2.C)
+ *   y          = o W_o^T                                           (implied)
+ *
+ * and the compressed KV cache (k after RoPE, v after the shift).
+ *
+ * Conventions for every call below:
+ *   - Pointers named *_host are host memory; every other data pointer is
+ *     device memory of the current CUDA device. The caller allocates and owns
+ *     all of it. The library allocates nothing per call.
+ *   - All tensors are dense and row-major (the last index is contiguous) and
+ *     start on a 16-byte boundary. Element type is cfg->dtype unless noted.
+ *   - Work is enqueued on `stream` (a cudaStream_t; NULL = legacy default
+ *     stream) and nothing synchronizes except cca_poll_device_status.
+ *   - Invalid arguments are rejected before any launch; outputs are then left
+ *     untouched. cca_last_error_message() gives a one-line reason.
+ *   - Calls on distinct streams may run concurrently if they use distinct
+ *     workspaces and outputs.
+ */
+#ifndef CCA_H_
+#define CCA_H_
+
+#include <stddef.h>
+#include <stdint.h>
+
+#ifdef __cplusplus
+extern "C" {
+#endif
+
+#define CCA_VERSION 1
+
+typedef enum cca_status {
+  CCA_OK = 0,
+  CCA_ERR_INVALID_ARG = 1,    /* a shape, pointer, mode or alignment is invalid */
+  CCA_ERR_UNSUPPORTED = 2,    /* valid block, but no kernel for this shape/dtype */
+  CCA_ERR_WORKSPACE = 3,      /* workspace missing or smaller than cca_workspace_size */
+  CCA_ERR_CUDA = 4,           /* a CUDA runtime call or launch failed */
+  CCA_ERR_DEVICE_TIMEOUT = 5  /* a bounded device-side wait gave up (see cca_poll_device_status) */
+} cca_status_t;
+
+typedef enum cca_dtype {
+  CCA_F32 = 0,   /* float32 */
+  CCA_BF16 = 1   /* bfloat16 */
+} cca_dtype_t;
+
+/* QK-mean mode bits (es 2.B item 2: the mean of q and k taken before and
+ * after the convolution is added to the conv outputs). */
+#define CCA_QK_MEAN_PRE 1
+#define CCA_QK_MEAN_POST 2
+
+/* Block shape and options. Field order is part of the ABI. */
+typedef struct cca_config {
+  int batch;         /* B >= 1 independent sequences */
+  int seq_len;       /* S >= 1 tokens per sequence */
+  int hidden;        /* E */
+  int C;             /* compression factor: hidden == C * n_q_heads * head_dim */
+  int n_q_heads;     /* query heads in the latent */
+  int n_kv_heads;    /* K/V heads; n_q_heads % n_kv_heads == 0 (CCGQA when <) */
+  int head_dim;      /* d, even */
+  int conv_kernel;   /* K >= 1 taps of the causal sequence conv */
+  int qk_mean_mode;  /* OR of CCA_QK_MEAN_*; 3 is the method as described */
+  int value_shift;   /* 1 = shift the upper half of v's channels by one token */
+  int use_rope;      /* 1 = rotate-half RoPE on q and k */
+  float rope_base;   /* RoPE base, e.g. 10000 */
+  float softmax_scale; /* 0 => 1/sqrt(head_dim) */
+  int dtype;         /* cca_dtype_t of every input, the KV cache and the conv state */
+  int out_dtype;     /* cca_dtype_t of y (CCA_F32 allowed for bf16 inputs) */
+} cca_config_t;
+
+/* Kernel path selection (cca_prefill_ex). AUTO takes the tensor-core path
+ * (tcgen05/TMEM, TMA) for bf16 with head_dim 128 and the SIMT path
+ * otherwise. */
+typedef enum cca_path {
+  CCA_PATH_AUTO = 0,
+  CCA_PATH_SIMT = 1,
+  CCA_PATH_TENSOR = 2   /* CCA_ERR_UNSUPPORTED if the shape does not allow it */
+} cca_path_t;
+
+typedef struct cca_prefill_opts {
+  int path;              /* cca_path_t */
+  /* If non-NULL: five cudaEvent_t recorded on `stream` before the down-
+   * projection, before preprocessing, before attention, before the output
+   * projection and after it. Owned by the caller. */
+  void* const* stage_events;
+} cca_prefill_opts_t;
+
+/* Byte offsets of the intermediates inside the workspace, for inspection
+ * after a call has completed. Each region is [T, width] row-major of the
+ * element type `elem_bytes`, T = batch * seq_len. */
+typedef struct cca_workspace_layout {
+  size_t total_bytes;
+  size_t elem_bytes;        /* 4 for CCA_F32, 2 for CCA_BF16 */
+  size_t qkv_lat_offset;    /* [T, Lq + 2*Lkv]: q~ | k~ | v~ (down-projection) */
+  size_t q_offset;          /* [T, Lq]: q after convs, QK-mean and RoPE */
+  size_t o_offset;          /* [T, Lq]: attention output, heads concatenated */
+  size_t sched_offset;      /* small scheduling scratch of the attention kernel */
+} cca_workspace_layout_t;
+
+/* Checks a configuration. CCA_OK if some kernel path accepts it. */
+cca_status_t cca_validate(const cca_config_t* cfg);
+
+/* Workspace bytes that cca_prefill needs for cfg (0 if cfg is invalid). */
+size_t cca_workspace_size(const cca_config_t* cfg);
+
+/* Fills *out with the workspace layout for cfg. */
+cca_status_t cca_workspace_layout(const cca_config_t* cfg, cca_workspace_layout_t* out);
+
+/*
+ * Prefill forward of one CCA / CCGQA block over B sequences of S tokens.
+ *
+ * Inputs (device, cfg->dtype, Lq = n_q*d, Lkv = n_kv*d, T = B*S):
+ *   x          [B, S, E]         hidden states
+ *   W_q        [Lq, E]           down-projections (torch Linear layout)
+ *   W_k, W_v   [Lkv, E]
+ *   convq_seq  [Lq, K]           causal seq-conv taps per q channel; tap K-1
+ *                                multiplies the current token
+ *   convq_chan [n_q, d, d]       per-head channel mix: out_i = sum_j W[i][j] in_j
+ *   convk_seq  [Lkv, K], convk_chan [n_kv, d, d]   the same for k
+ *   W_o        [E, Lq]           output projection
+ * Outputs (device):
+ *   y          [B, S, E]         cfg->out_dtype
+ *   k_cache    [B, S, n_kv, d]   k after convs, QK-mean and RoPE
+ *   v_cache    [B, S, n_kv, d]   v after the value shift
+ *   conv_state optional (NULL to skip), [B, (K-1)*(Lq+Lkv) + Lkv]: per
+ *              sequence the last K-1 rows of q~ (each Lq wide), then of k~
+ *              (Lkv wide), then the last row of v~; rows before the sequence
+ *              start are zero. It is what a later decode step would resume
+ *              from.
+ *   workspace  >= cca_workspace_size(cfg) bytes, 256-byte aligned; holds the
+ *              intermediates listed in cca_workspace_layout_t.
+ * Errors: INVALID_ARG / UNSUPPORTED / WORKSPACE before any launch; CUDA if a
+ * launch fails. A device-side wait that gives up is reported later by
+ * cca_poll_device_status.
+ */
+cca_status_t cca_prefill(const cca_config_t* cfg,
+                         const void* x,
+                         const void* W_q, const void* W_k, const void* W_v,
+                         const void* convq_seq, const void* convq_chan,
+                         const void* convk_seq, const void* convk_chan,
+                         const void* W_o,
+                         void* y, void* k_cache, void* v_cache, void* conv_state,
+                         void* workspace, size_t workspace_bytes, void* stream);
+
+/* cca_prefill with options (path choice, per-stage events); opts may be NULL. */
+cca_status_t cca_prefill_ex(const cca_config_t* cfg,
+                            const void* x,
+                            const void* W_q, const void* W_k, const void* W_v,
+                            const void* convq_seq, const void* convq_chan,
+                            const void* convk_seq, const void* convk_chan,
+                            const void* W_o,
+                            void* y, void* k_cache, void* v_cache, void* conv_state,
+                            void* workspace, size_t workspace_bytes, void* stream,
+                            const cca_prefill_opts_t* opts);
+
+/*
+ * End-to-end variant for callers whose hidden states live in host memory:
+ * copies x_host (B*S*E elements, pinned host memory for a truly asynchronous
+ * copy) into the device buffer x_dev, runs cca_prefill, and copies y back
+ * from y_dev into y_host (pinned). The KV cache stays on the device. All
+ * three steps are enqueued on `stream`; y_host is valid once the stream has
+ * been synchronized.
+ */
+cca_status_t cca_prefill_host(const cca_config_t* cfg,
+                              const void* x_host, void* x_dev,
+                              const void* W_q, const void* W_k, const void* W_v,
+                              const void* convq_seq, const void* convq_chan,
+                              const void* convk_seq, const void* convk_chan,
+                              const void* W_o,
+                              void* y_dev, void* y_host,
+                              void* k_cache, void* v_cache, void* conv_state,
+                              void* workspace, size_t workspace_bytes, void* stream);
+
+/* Synchronizes `stream`, then reports and clears the device error word:
+ * CCA_ERR_DEVICE_TIMEOUT if a bounded wait in a kernel gave up since the last
+ * poll, CCA_ERR_CUDA if the stream reports a CUDA error, else CCA_OK. */
+cca_status_t cca_poll_device_status(void* stream);
+
+/* Self-test of the bounded-wait machinery: launches one kernel that waits on
+ * an mbarrier nothing will ever complete, with a limit of `timeout_us`
+ * microseconds (1..5000000). The kernel gives up, records the timeout in the
+ * device error word and exits; cca_poll_device_status then returns
+ * CCA_ERR_DEVICE_TIMEOUT. */
+cca_status_t cca_selftest_wait_timeout(unsigned timeout_us, void* stream);
+
+/* Static description of a status code. */
+const char* cca_status_string(cca_status_t status);
+
+/* One-line reason for the last non-OK status returned on this host thread. */
+const char* cca_last_error_message(void);
+
+/* CCA_VERSION of the built library. */
+int cca_version(void);
+
+#ifdef __cplusplus
+}  /* extern "C" */
+#endif
+
+#endif  /* CCA_H_ */

@@ -1,0 +1,100 @@
+"""Host-side checks of the C ABI: the library loads, exports every function
+declared in include/cca.h, and validates configurations. No kernel runs."""
+import ctypes
+import os
+import re
+
+import pytest
+
+import compressed_latent_space_cca_b200 as cca
+from compressed_latent_space_cca_b200 import _capi
+
+ROOT = os.path.dirname(os.path.dirname(os.path.abspath(__file__)))
+
+
+def declared_functions():
+    src = open(os.path.join(ROOT, "include", "cca.h")).read()
+    src = re.sub(r"/\*.*?\*/", "", src, flags=re.S)
+    return sorted(set(re.findall(r"^[A-Za-z_][\w\s\*]*?\b(cca_\w+)\s*\(", src, flags=re.M)))
+
+
+def test_library_exports_every_declared_function():
+    lib = _capi.load()
+    names = declared_functions()
+    assert len(names) >= 11, names
+    for n in names:
+        assert hasattr(lib, n), n
+        assert n in _capi.SIGNATURES, f"{n} has no ctypes signature"
+    assert lib.cca_version() == 1
+
+
+def test_struct_layouts():
+    assert ctypes.sizeof(cca.CcaConfig) == 15 * 4
+    assert ctypes.sizeof(cca.CcaWorkspaceLayout) == 6 * 8
+
+
+def good(**kw):
+    base = dict(batch=1, seq_len=16384, hidden=2048, n_q_heads=4, n_kv_heads=2, head_dim=128, dtype="bf16")
+    base.update(kw)
+    return cca.make_config(**base)
+
+
+def test_valid_configs_and_workspace():
+    assert cca.validate(good()) == cca.CCA_OK
+    cfg = good()
+    T, Lq, Lkv = 16384, 512, 256
+    lay = cca.workspace_layout(cfg)
+    assert lay.elem_bytes == 2
+    assert lay.q_offset >= T * (Lq + 2 * Lkv) * 2
+    assert lay.o_offset - lay.q_offset >= T * Lq * 2
+    assert cca.workspace_size(cfg) == lay.total_bytes
+    for off in (lay.qkv_lat_offset, lay.q_offset, lay.o_offset, lay.sched_offset, lay.total_bytes):
+        assert off % 256 == 0
+    tiny = cca.make_config(batch=1, seq_len=64, hidden=128, n_q_heads=2, n_kv_heads=2, head_dim=16, dtype="f32")
+    assert cca.validate(tiny) == cca.CCA_OK
+    assert cca.workspace_layout(tiny).elem_bytes == 4
+
+
+@pytest.mark.parametrize("bad,code", [
+    (dict(batch=0), cca.CCA_ERR_INVALID_ARG),
+    (dict(seq_len=0), cca.CCA_ERR_INVALID_ARG),
+    (dict(n_kv_heads=3), cca.CCA_ERR_INVALID_ARG),
+    (dict(head_dim=127, hidden=4 * 127), cca.CCA_ERR_INVALID_ARG),
+    (dict(C=3), cca.CCA_ERR_INVALID_ARG),
+    (dict(conv_kernel=0), cca.CCA_ERR_INVALID_ARG),
+    (dict(qk_mean_mode=4), cca.CCA_ERR_INVALID_ARG),
+    (dict(value_shift=2), cca.CCA_ERR_INVALID_ARG),
+    (dict(rope_base=0.5), cca.CCA_ERR_INVALID_ARG),
+    (dict(softmax_scale=-1.0), cca.CCA_ERR_INVALID_ARG),
+    (dict(head_dim=256, hidden=4096), cca.CCA_ERR_UNSUPPORTED),
+])
+def test_invalid_configs_rejected(bad, code):
+    cfg = good(**bad)
+    assert cca.validate(cfg) == code
+    assert cca.workspace_size(cfg) == 0
+    assert cca.library().cca_last_error_message().decode()
+
+
+def test_bad_dtype_and_null_config():
+    cfg = good()
+    cfg.dtype = 7
+    assert cca.validate(cfg) == cca.CCA_ERR_INVALID_ARG
+    lib = cca.library()
+    assert lib.cca_validate(None) == cca.CCA_ERR_INVALID_ARG
+    assert lib.cca_workspace_size(None) == 0
+    assert lib.cca_status_string(cca.CCA_ERR_DEVICE_TIMEOUT) == b"device-side wait timed out"
+
+
+def test_prefill_without_device_fails_cleanly():
+    """No GPU here: the call must return an error status, never fall back."""
+    import torch
+    if torch.cuda.is_available():
+        pytest.skip("a GPU is present")
+    cfg = good(seq_len=128)
+    lib = cca.library()
+    null = [ctypes.c_void_p(16)] * 9
+    outs = [ctypes.c_void_p(16)] * 3
+    st = lib.cca_prefill(ctypes.byref(cfg), *null, *outs, None, ctypes.c_void_p(256), 1 << 40, None)
+    assert st in (cca.CCA_ERR_CUDA, cca.CCA_ERR_UNSUPPORTED)
+    st = lib.cca_prefill(ctypes.byref(cfg), *null, *outs, None, None, 0, None)
+    assert st != cca.CCA_OK

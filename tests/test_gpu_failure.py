@@ -1,0 +1,42 @@
+"""Failure detection on the GPU without faulting it: a kernel waits on an
+mbarrier that nothing will complete, with a 20 ms limit. The bounded wait must
+give up, record the timeout in the device error word and return, leaving the
+context usable for the next call."""
+import pytest
+import torch
+
+import compressed_latent_space_cca_b200 as cca
+import workloads
+from parity import run_gpu, run_oracle, assert_close
+
+pytestmark = pytest.mark.gpu
+
+
+def test_bounded_wait_reports_timeout_and_context_survives():
+    assert cca.poll_device_status() == cca.CCA_OK
+    assert cca.selftest_wait_timeout(20000) == cca.CCA_OK
+    assert cca.poll_device_status() == cca.CCA_ERR_DEVICE_TIMEOUT
+    assert cca.poll_device_status() == cca.CCA_OK  # the word is cleared by the poll
+    sh = workloads.WORKLOADS["tiny_cca_fp32"]
+    inp = workloads.make_inputs(sh)
+    gpu = run_gpu(sh, inp)
+    assert_close("y", gpu["y"], run_oracle(sh, inp)["y"], "f32")
+
+
+def test_invalid_calls_rejected_before_launch():
+    sh = workloads.WORKLOADS["tiny_cca_fp32"]
+    cfg = cca.config_from_shape(sh)
+    inp = {k: v.cuda() for k, v in workloads.make_inputs(sh).items()}
+    out = cca.alloc_outputs(cfg, torch.device("cuda"))
+    sentinel = out["y"].fill_(7.0).clone()
+    small_ws = torch.empty(64, dtype=torch.uint8, device="cuda")
+    with pytest.raises(cca.CcaError) as ei:
+        cca.prefill(cfg, inp, out=out, workspace=small_ws)
+    assert ei.value.status == cca.CCA_ERR_WORKSPACE
+    bad = cca.config_from_shape(sh)
+    bad.n_kv_heads = 3
+    with pytest.raises(cca.CcaError) as ei:
+        cca.alloc_workspace(bad, torch.device("cuda"))
+    assert ei.value.status == cca.CCA_ERR_INVALID_ARG
+    torch.cuda.synchronize()
+    assert torch.equal(out["y"], sentinel)  # outputs untouched

@@ -1,0 +1,142 @@
+"""GPU parity: the CUDA path (through the C ABI) against the float64 oracle on
+the same seeded inputs, element by element, per row-normalised error."""
+import numpy as np
+import pytest
+import torch
+
+import compressed_latent_space_cca_b200 as cca
+import workloads
+from parity import assert_close, run_gpu, run_oracle, sample_rows
+
+pytestmark = pytest.mark.gpu
+
+SIMT, TENSOR = cca.CCA_PATH_SIMT, cca.CCA_PATH_TENSOR
+
+
+def shape(**kw):
+    base = dict(name="case", batch=1, seq_len=300, hidden=512, n_q_heads=4, n_kv_heads=2, head_dim=128,
+                conv_kernel=4, dtype="bf16", seed=11)
+    base.update(kw)
+    return workloads.BlockShape(**base)
+
+
+def check_all(sh, gpu, ref, stages=True):
+    dt = sh.dtype
+    assert_close("k_cache", gpu["k_cache"], ref["k_cache"], dt)
+    assert_close("v_cache", gpu["v_cache"], ref["v_cache"], dt)
+    if stages:
+        T = sh.seq_len
+        lq, lkv = sh.latent_q, sh.latent_kv
+        lat = gpu["qkv_lat"]
+        assert_close("q_lat", lat[..., :lq], ref["q_lat"], dt)
+        assert_close("k_lat", lat[..., lq:lq + lkv], ref["k_lat"], dt)
+        assert_close("v_lat", lat[..., lq + lkv:], ref["v_lat"], dt)
+        assert_close("q", gpu["q"], ref["q"], dt)
+        assert_close("o", gpu["o"], ref["o"], dt)
+    return assert_close("y", gpu["y"], ref["y"], dt)
+
+
+# --------------------------------------------------------------- fp32 tiny --
+def test_tiny_fp32_block():
+    sh = workloads.WORKLOADS["tiny_cca_fp32"]
+    inp = workloads.make_inputs(sh)
+    check_all(sh, run_gpu(sh, inp), run_oracle(sh, inp))
+
+
+@pytest.mark.parametrize("S,nq,nkv,d,K", [(1, 2, 2, 16, 4), (65, 4, 1, 32, 4), (130, 4, 2, 64, 1),
+                                          (97, 6, 3, 8, 7)])
+def test_fp32_shapes(S, nq, nkv, d, K):
+    sh = shape(dtype="f32", seq_len=S, n_q_heads=nq, n_kv_heads=nkv, head_dim=d, hidden=2 * nq * d,
+               conv_kernel=K, batch=2)
+    inp = workloads.make_inputs(sh)
+    check_all(sh, run_gpu(sh, inp), run_oracle(sh, inp))
+
+
+# ------------------------------------------------------------ bf16, small --
+BF16_CASES = [
+    dict(seq_len=300, n_q_heads=4, n_kv_heads=2, hidden=512),             # CCGQA, ragged tail
+    dict(seq_len=256, n_q_heads=4, n_kv_heads=4, hidden=1024, batch=2),   # CCA, C=2
+    dict(seq_len=1, n_q_heads=4, n_kv_heads=2, hidden=512),               # one token
+    dict(seq_len=129, n_q_heads=8, n_kv_heads=2, hidden=1024, batch=3),   # G=4
+    dict(seq_len=200, n_q_heads=2, n_kv_heads=1, hidden=512),             # n_kv=1: shift within the head
+    dict(seq_len=383, n_q_heads=2, n_kv_heads=2, hidden=256),             # C=1
+]
+
+
+@pytest.mark.parametrize("path", [SIMT, TENSOR], ids=["simt", "tensor"])
+@pytest.mark.parametrize("case", range(len(BF16_CASES)))
+def test_bf16_small(path, case):
+    sh = shape(**BF16_CASES[case])
+    inp = workloads.make_inputs(sh)
+    check_all(sh, run_gpu(sh, inp, path=path), run_oracle(sh, inp))
+
+
+@pytest.mark.parametrize("path", [SIMT, TENSOR], ids=["simt", "tensor"])
+@pytest.mark.parametrize("mode,vshift,rope", [(0, 0, 0), (1, 0, 1), (2, 1, 0), (3, 1, 1), (0, 1, 1)])
+def test_bf16_modes(path, mode, vshift, rope):
+    sh = shape(seq_len=257, qk_mean_mode=mode, value_shift=vshift, use_rope=rope, batch=2)
+    inp = workloads.make_inputs(sh)
+    check_all(sh, run_gpu(sh, inp, path=path), run_oracle(sh, inp))
+
+
+@pytest.mark.parametrize("path", [SIMT, TENSOR], ids=["simt", "tensor"])
+def test_fp32_output_and_conv_state(path):
+    sh = shape(seq_len=190, batch=2)
+    inp = workloads.make_inputs(sh)
+    gpu = run_gpu(sh, inp, path=path, conv_state=True, out_dtype="f32")
+    ref = run_oracle(sh, inp)
+    check_all(sh, gpu, ref, stages=False)
+    K = sh.conv_kernel
+    lq, lkv = sh.latent_q, sh.latent_kv
+    cs = gpu["conv_state"]
+    nq_part = (K - 1) * lq
+    np.testing.assert_allclose(cs[:, :nq_part].reshape(2, K - 1, lq), ref["conv_state_q"], rtol=1e-2, atol=1e-2)
+    np.testing.assert_allclose(cs[:, nq_part:nq_part + (K - 1) * lkv].reshape(2, K - 1, lkv), ref["conv_state_k"],
+                               rtol=1e-2, atol=1e-2)
+    np.testing.assert_allclose(cs[:, nq_part + (K - 1) * lkv:].reshape(2, 1, lkv), ref["conv_state_v"],
+                               rtol=1e-2, atol=1e-2)
+    # the conv state is a copy of the workspace latents: exact
+    lat = gpu["qkv_lat"]
+    np.testing.assert_array_equal(cs[:, :nq_part].reshape(2, K - 1, lq), lat[:, -(K - 1):, :lq])
+
+
+@pytest.mark.parametrize("path", [SIMT, TENSOR], ids=["simt", "tensor"])
+def test_deterministic_and_causal(path):
+    """Three runs are bit-identical; perturbing x[t0] leaves every output row
+    before t0 bit-identical (nothing reads the future)."""
+    sh = shape(seq_len=520, batch=2)
+    inp = workloads.make_inputs(sh)
+    a = run_gpu(sh, inp, path=path)
+    for _ in range(2):
+        b = run_gpu(sh, inp, path=path)
+        for k in ("y", "k_cache", "v_cache", "q", "o"):
+            assert np.array_equal(a[k], b[k]), k
+    t0 = 300
+    inp2 = dict(inp)
+    x = inp["x"].clone()
+    x[1, t0] += 1.0
+    inp2["x"] = x
+    c = run_gpu(sh, inp2, path=path)
+    for k in ("y", "k_cache", "v_cache"):
+        assert np.array_equal(c[k][1, :t0], a[k][1, :t0]), k
+        assert np.array_equal(c[k][0], a[k][0]), k
+        assert not np.array_equal(c[k][1, t0], a[k][1, t0]), k
+
+
+# ------------------------------------------------- the five named workloads --
+@pytest.mark.parametrize("name", ["cca_dense_bf16", "ccgqa_16k_bf16", "ccgqa_8x_bf16", "ccgqa_64k_bf16"])
+def test_named_workload_full_size(name):
+    """Full-size run in the bench's launch configuration (auto path); the
+    KV cache is compared in full, y and the attention output on sampled rows
+    the oracle computes one by one."""
+    sh = workloads.WORKLOADS[name]
+    inp = workloads.make_inputs(sh)
+    rows = sample_rows(sh.seq_len, 40, seed=sh.seed)
+    gpu = run_gpu(sh, inp, rows=rows, stages=False)
+    ref = run_oracle(sh, inp, rows=rows)
+    assert_close("k_cache", gpu["k_cache"], ref["k_cache"], "bf16")
+    assert_close("v_cache", gpu["v_cache"], ref["v_cache"], "bf16")
+    assert_close("o", gpu["o"], ref["o"], "bf16")
+    assert_close("y", gpu["y"], ref["y"], "bf16")
+    del gpu
+    torch.cuda.empty_cache()
