@@ -284,9 +284,10 @@ def run_ours(args, shape):
         dist.all_reduce(t, op=dist.ReduceOp.MAX)
         return float(t.item())
 
-    # which path runs (tensor cores or SIMT) and how many kernels a step launches
-    path_tensor = cca.validate(cfg) == 0 and _tensor_path_ok(cca, cfg, inputs, out, ws)
-    launches_per_step = 4 if path_tensor else 6
+    # which kernels run (tcgen05 or SIMT per stage) and how many launches a step makes
+    plan = cca.plan(cfg)
+    path_tensor = plan["attention_tensor"]
+    launches_per_step = plan["launches"]
 
     for _ in range(args.warmup):
         flush.zero_()
@@ -366,7 +367,7 @@ def run_ours(args, shape):
             "metric": METRIC, "value": value, "unit": "tokens/s", "n_gpus": world, "steps": args.steps,
             "warmup": args.warmup, "ms_per_step": ms_per_step, "higher_is_better": True, "scaling": "weak",
             "vs_baseline": None, "dtype": "bf16", "data": "synthetic",
-            "config": config_dict(shape, "tensor" if path_tensor else "simt"),
+            "config": config_dict(shape, plan_name(plan)),
             "attention_tflops": attn_tflops,
             "roofline": roofline,
             "kernels": kernels,
@@ -385,14 +386,10 @@ def run_ours(args, shape):
     return 0
 
 
-def _tensor_path_ok(cca, cfg, inputs, out, ws):
-    try:
-        cca.prefill(cfg, inputs, out=out, workspace=ws, path=cca.CCA_PATH_TENSOR)
-        return True
-    except cca.CcaError as e:
-        if e.status == cca.CCA_ERR_UNSUPPORTED:
-            return False
-        raise
+def plan_name(plan):
+    k = lambda b: "tcgen05" if b else "simt"  # noqa: E731
+    return (f"down_proj={k(plan['down_proj_tensor'])},attention={k(plan['attention_tensor'])},"
+            f"out_proj={k(plan['out_proj_tensor'])}")
 
 
 def main(argv=None):

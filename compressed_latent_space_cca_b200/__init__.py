@@ -20,20 +20,23 @@ from ._capi import (  # noqa: F401
     CCA_ERR_CUDA,
     CCA_ERR_DEVICE_TIMEOUT,
     CCA_ERR_INVALID_ARG,
+    CCA_ERR_NUMERIC_RANGE,
     CCA_ERR_UNSUPPORTED,
     CCA_ERR_WORKSPACE,
+    CCA_F16,
     CCA_F32,
     CCA_OK,
     CCA_PATH_AUTO,
     CCA_PATH_SIMT,
     CCA_PATH_TENSOR,
+    CCA_PATH_TENSOR_MASK,
     CcaConfig,
     CcaWorkspaceLayout,
 )
 
 INPUT_NAMES = ("x", "W_q", "W_k", "W_v", "convq_seq", "convq_chan", "convk_seq", "convk_chan", "W_o")
 
-_DT = {CCA_F32: torch.float32, CCA_BF16: torch.bfloat16}
+_DT = {CCA_F32: torch.float32, CCA_BF16: torch.bfloat16, CCA_F16: torch.float16}
 _DT_CODE = {torch.float32: CCA_F32, torch.bfloat16: CCA_BF16, "f32": CCA_F32, "bf16": CCA_BF16}
 
 
@@ -85,6 +88,16 @@ def workspace_layout(cfg: CcaConfig) -> CcaWorkspaceLayout:
     if st != CCA_OK:
         raise CcaError(st, "cca_workspace_layout")
     return out
+
+
+def plan(cfg: CcaConfig, path: int = CCA_PATH_AUTO) -> dict:
+    """Which kernels cca_prefill_ex would launch on the current device."""
+    out = _capi.CcaPlan()
+    st = library().cca_plan(ctypes.byref(cfg), path, ctypes.byref(out))
+    if st != CCA_OK:
+        raise CcaError(st, "cca_plan")
+    return {"down_proj_tensor": bool(out.down_proj_tensor), "attention_tensor": bool(out.attention_tensor),
+            "out_proj_tensor": bool(out.out_proj_tensor), "launches": out.launches}
 
 
 def _shapes(cfg: CcaConfig) -> Dict[str, tuple]:
@@ -165,6 +178,9 @@ def prefill(cfg: CcaConfig, inputs: Dict[str, torch.Tensor], *, out: Optional[Di
     if stage_events is not None:
         if len(stage_events) != 5:
             raise ValueError("stage_events needs 5 events")
+        for ev in stage_events:  # torch creates the CUDA event on its first record
+            if ev.cuda_event == 0:
+                ev.record(stream)
         arr = (ctypes.c_void_p * 5)(*[ev.cuda_event for ev in stage_events])
         opts.stage_events = ctypes.cast(arr, ctypes.POINTER(ctypes.c_void_p))
     st = library().cca_prefill_ex(ctypes.byref(cfg), *ptrs, y, kc, vc, cs, workspace.data_ptr(),
@@ -217,15 +233,19 @@ def selftest_wait_timeout(timeout_us: int, stream: Optional[torch.cuda.Stream] =
 def workspace_view(cfg: CcaConfig, workspace: torch.Tensor) -> Dict[str, torch.Tensor]:
     """Views of the intermediates left in the workspace by the last call."""
     L = workspace_layout(cfg)
-    dt = _DT[cfg.dtype]
+    dt = _DT[L.lat_dtype]
     T = cfg.batch * cfg.seq_len
     Lq, Lkv = cfg.n_q_heads * cfg.head_dim, cfg.n_kv_heads * cfg.head_dim
     eb = L.elem_bytes
 
     def region(off, width):
         return workspace[off:off + T * width * eb].view(dt).view(cfg.batch, cfg.seq_len, width)
-    return {
+    out = {
         "qkv_lat": region(L.qkv_lat_offset, Lq + 2 * Lkv),
         "q": region(L.q_offset, Lq),
         "o": region(L.o_offset, Lq),
     }
+    if L.v_att_offset > L.k_att_offset:
+        out["k_att"] = region(L.k_att_offset, Lkv)
+        out["v_att"] = region(L.v_att_offset, Lkv)
+    return out

@@ -13,13 +13,20 @@ CCA_ERR_UNSUPPORTED = 2
 CCA_ERR_WORKSPACE = 3
 CCA_ERR_CUDA = 4
 CCA_ERR_DEVICE_TIMEOUT = 5
+CCA_ERR_NUMERIC_RANGE = 6
 
 CCA_F32 = 0
 CCA_BF16 = 1
+CCA_F16 = 2
 
 CCA_PATH_AUTO = 0
 CCA_PATH_SIMT = 1
 CCA_PATH_TENSOR = 2
+
+
+def CCA_PATH_TENSOR_MASK(bits: int) -> int:
+    """bit0 down-projection, bit1 attention, bit2 output projection on tcgen05."""
+    return 0x100 | (bits & 7)
 
 
 class CcaConfig(Structure):
@@ -50,11 +57,21 @@ class CcaWorkspaceLayout(Structure):
     _fields_ = [
         ("total_bytes", c_size_t),
         ("elem_bytes", c_size_t),
+        ("lat_dtype", c_int),
+        ("reserved", c_int),
         ("qkv_lat_offset", c_size_t),
         ("q_offset", c_size_t),
+        ("k_att_offset", c_size_t),
+        ("v_att_offset", c_size_t),
         ("o_offset", c_size_t),
+        ("wo_offset", c_size_t),
         ("sched_offset", c_size_t),
     ]
+
+
+class CcaPlan(Structure):
+    _fields_ = [("down_proj_tensor", c_int), ("attention_tensor", c_int), ("out_proj_tensor", c_int),
+                ("launches", c_int)]
 
 
 _PREFILL_ARGS = [POINTER(CcaConfig)] + [c_void_p] * 9 + [c_void_p] * 4 + [c_void_p, c_size_t, c_void_p]
@@ -64,6 +81,7 @@ SIGNATURES = {
     "cca_validate": (c_int, [POINTER(CcaConfig)]),
     "cca_workspace_size": (c_size_t, [POINTER(CcaConfig)]),
     "cca_workspace_layout": (c_int, [POINTER(CcaConfig), POINTER(CcaWorkspaceLayout)]),
+    "cca_plan": (c_int, [POINTER(CcaConfig), c_int, POINTER(CcaPlan)]),
     "cca_prefill": (c_int, _PREFILL_ARGS),
     "cca_prefill_ex": (c_int, _PREFILL_ARGS + [POINTER(CcaPrefillOpts)]),
     "cca_prefill_host": (c_int, [POINTER(CcaConfig), c_void_p, c_void_p] + [c_void_p] * 8

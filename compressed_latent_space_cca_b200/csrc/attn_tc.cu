@@ -1,9 +1,425 @@
-// placeholder, replaced by the tcgen05 attention kernel
+// Causal flash attention on the compressed heads, tcgen05 / TMEM / TMA for
+// sm_100a, head_dim 128, fp16 q / k / v / P / O, fp32 softmax and accumulation.
+//
+// "Compressed Convolutional Attention" (gist.science/es/paper/2510.04476):
+// attention runs entirely in the compressed latent (section 2.A) and, in
+// CCGQA, one K/V head serves a group of G query heads (section 2.C):
+//   O[t, h] = sum_{s <= t} softmax_s(q[t,h] . k[s,g(h)] * scale) v[s,g(h)],
+//   g(h) = h / G.
+//
+// One CTA owns a pair of 128-query tiles of one KV group (for G >= 2 two
+// query heads at the same positions, for G = 1 two consecutive query tiles
+// of one head), so every K/V tile it loads serves both. Roles:
+//   warp 0      TMA: Q tiles once per pair, then K and V tiles (2-stage ring)
+//   warp 1      one thread issues tcgen05.mma: S_j = Q_j K^T (SS form) into
+//               TMEM, then O_j += P_j V (TS form, P read from TMEM)
+//   warps 2-5   softmax of tile 0, warps 6-9 softmax of tile 1: each thread
+//               owns one query row, reads its S row from TMEM, keeps the
+//               running max / sum, writes P (fp16) back over S in TMEM,
+//               rescales its O row in TMEM when the max grows by more than
+//               2^8, and finally normalises O and stores it.
+// TMEM (512 columns): S0 | S1 | O0 | O1, 128 fp32 columns each; P_j overlays
+// the first 64 columns of S_j. The two tiles ping-pong: while one softmax
+// group works, the tensor core runs the other tile's MMAs. Key tiles above
+// the diagonal are never loaded (causal tile skipping); the diagonal tile is
+// masked per element. Pairs are scheduled longest first over persistent
+// CTAs. Every mbarrier wait is bounded.
+#include "cca_common.cuh"
 #include "launch.h"
+
 namespace cca {
-bool attention_tc_supported(const BlockDims&) { return false; }
-cudaError_t launch_attention_tc(const BlockDims&, const void*, const void*, const void*, void*, void*, unsigned*,
-                                cudaStream_t) {
-  return cudaErrorNotSupported;
+namespace {
+
+constexpr int D = 128;           // head dim
+constexpr int TQ = 128;          // queries per tile
+constexpr int TK = 128;          // keys per tile
+constexpr int KV_STAGES = 2;
+constexpr int HALF_BYTES = 128 * 64 * 2;  // 128 rows x 64 fp16 (one 128-byte swizzle span)
+constexpr int TILE_BYTES = 2 * HALF_BYTES;  // 128 x 128 fp16
+constexpr int NUM_THREADS = 320;
+constexpr int TMEM_COLS = 512;
+constexpr uint32_t COL_S0 = 0, COL_O0 = 256;
+constexpr float RESCALE_THRESHOLD = 8.0f;  // log2 units: rescale O only if the max grows by > 2^8
+
+// shared memory: Q0 | Q1 | K[2] | V[2] | barriers
+constexpr int OFF_Q = 0;
+constexpr int OFF_K = 2 * TILE_BYTES;
+constexpr int OFF_V = OFF_K + KV_STAGES * TILE_BYTES;
+constexpr int OFF_BAR = OFF_V + KV_STAGES * TILE_BYTES;
+constexpr size_t SMEM_BYTES = OFF_BAR + 256 + 1024;
+
+struct AttnMaps {
+  CUtensorMap q, k, v;
+};
+
+struct AttnParams {
+  int B, S, nq, nkv, G;
+  int num_qt;  // query tiles per sequence
+  int pairs;   // tile pairs per (sequence, KV group)
+  int items;   // B * nkv * pairs
+  int Lq;
+  float scale_log2;  // softmax scale * log2(e)
+  __half* o;
+  unsigned* err;
+};
+
+struct Item {
+  int b, g, nkv_tiles;
+  int h[2], qt[2];
+  bool active[2];
+};
+
+__device__ __forceinline__ Item get_item(const AttnParams& p, int w) {
+  const int bgc = p.B * p.nkv;
+  const int pr = p.pairs - 1 - w / bgc;  // longest pairs first
+  const int bg = w % bgc;
+  Item it;
+  it.b = bg / p.nkv;
+  it.g = bg % p.nkv;
+  const int U = p.num_qt * p.G;  // (query tile, head) units of this group, tile-major
+  it.nkv_tiles = 0;
+#pragma unroll
+  for (int j = 0; j < 2; ++j) {
+    const int u = 2 * pr + j;
+    it.active[j] = u < U;
+    const int uu = it.active[j] ? u : 2 * pr;
+    it.qt[j] = uu / p.G;
+    it.h[j] = it.g * p.G + uu % p.G;
+    if (it.active[j] && it.qt[j] + 1 > it.nkv_tiles) it.nkv_tiles = it.qt[j] + 1;
+  }
+  return it;
 }
+
+// Work item of this CTA in round r (serpentine order over the CTAs).
+__device__ __forceinline__ int item_index(int r, int cta, int grid) {
+  return r * grid + ((r & 1) ? (grid - 1 - cta) : cta);
+}
+
+__global__ void __launch_bounds__(NUM_THREADS, 1) attn_tc_kernel(const __grid_constant__ AttnMaps maps,
+                                                                 const AttnParams p) {
+  extern __shared__ uint8_t smem_raw[];
+  uint8_t* smem = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
+  uint64_t* bars = reinterpret_cast<uint64_t*>(smem + OFF_BAR);
+  uint64_t* q_full = bars + 0;
+  uint64_t* q_empty = bars + 1;
+  uint64_t* k_full = bars + 2;             // [KV_STAGES]
+  uint64_t* k_empty = k_full + KV_STAGES;  // [KV_STAGES]
+  uint64_t* v_full = k_empty + KV_STAGES;  // [KV_STAGES]
+  uint64_t* v_empty = v_full + KV_STAGES;  // [KV_STAGES]
+  uint64_t* s_full = v_empty + KV_STAGES;  // [2]
+  uint64_t* p_full = s_full + 2;           // [2]
+  uint64_t* o_full = p_full + 2;           // [2]
+  uint64_t* o_empty = o_full + 2;          // [2]
+  uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(o_empty + 2);
+  volatile int* abort_flag = reinterpret_cast<volatile int*>(tmem_slot + 1);
+
+  const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+  if (threadIdx.x == 0) {
+    mbar_init(smem_u32(q_full), 1);
+    mbar_init(smem_u32(q_empty), 1);
+    for (int s = 0; s < KV_STAGES; ++s) {
+      mbar_init(smem_u32(&k_full[s]), 1);
+      mbar_init(smem_u32(&k_empty[s]), 1);
+      mbar_init(smem_u32(&v_full[s]), 1);
+      mbar_init(smem_u32(&v_empty[s]), 1);
+    }
+    for (int j = 0; j < 2; ++j) {
+      mbar_init(smem_u32(&s_full[j]), 1);
+      mbar_init(smem_u32(&p_full[j]), 4);
+      mbar_init(smem_u32(&o_full[j]), 1);
+      mbar_init(smem_u32(&o_empty[j]), 4);
+    }
+    *abort_flag = 0;
+    fence_mbar_init();
+  }
+  if (warp == 0 && lane == 0) {
+    prefetch_tmap(&maps.q);
+    prefetch_tmap(&maps.k);
+    prefetch_tmap(&maps.v);
+  }
+  if (warp == 1) {
+    tmem_alloc(smem_u32(tmem_slot), TMEM_COLS);
+    tmem_relinquish();
+  }
+  tc_fence_before();
+  __syncthreads();
+  tc_fence_after();
+  const uint32_t tmem = *tmem_slot;
+  const int cta = blockIdx.x, grid = gridDim.x;
+
+  if (warp == 0) {
+    if (lane == 0) {
+      // ------------------------------------------------------------ TMA --
+      int stage = 0;
+      uint32_t phase = 0;
+      for (int r = 0;; ++r) {
+        const int w = item_index(r, cta, grid);
+        if (w >= p.items) break;
+        const Item it = get_item(p, w);
+        if (!mbar_wait_bounded(smem_u32(q_empty), (r & 1) ^ 1, p.err, abort_flag, wait_site(kSiteAttn, 1, 1))) goto done;
+        mbar_arrive_expect_tx(smem_u32(q_full), 2 * TILE_BYTES);
+#pragma unroll
+        for (int j = 0; j < 2; ++j)
+#pragma unroll
+          for (int hf = 0; hf < 2; ++hf)
+            tma_load_3d(smem_u32(smem + OFF_Q + j * TILE_BYTES + hf * HALF_BYTES), &maps.q, smem_u32(q_full),
+                        it.h[j] * D + hf * 64, it.qt[j] * TQ, it.b);
+        for (int jj = 0; jj < it.nkv_tiles; ++jj) {
+          if (!mbar_wait_bounded(smem_u32(&k_empty[stage]), phase ^ 1, p.err, abort_flag, wait_site(kSiteAttn, 1, 2))) goto done;
+          mbar_arrive_expect_tx(smem_u32(&k_full[stage]), TILE_BYTES);
+#pragma unroll
+          for (int hf = 0; hf < 2; ++hf)
+            tma_load_3d(smem_u32(smem + OFF_K + stage * TILE_BYTES + hf * HALF_BYTES), &maps.k,
+                        smem_u32(&k_full[stage]), it.g * D + hf * 64, jj * TK, it.b);
+          if (!mbar_wait_bounded(smem_u32(&v_empty[stage]), phase ^ 1, p.err, abort_flag, wait_site(kSiteAttn, 1, 3))) goto done;
+          mbar_arrive_expect_tx(smem_u32(&v_full[stage]), TILE_BYTES);
+#pragma unroll
+          for (int hf = 0; hf < 2; ++hf)
+            tma_load_3d(smem_u32(smem + OFF_V + stage * TILE_BYTES + hf * HALF_BYTES), &maps.v,
+                        smem_u32(&v_full[stage]), it.g * D + hf * 64, jj * TK, it.b);
+          if (++stage == KV_STAGES) {
+            stage = 0;
+            phase ^= 1;
+          }
+        }
+      }
+    }
+  } else if (warp == 1) {
+    if (lane == 0) {
+      // ------------------------------------------------------------ MMA --
+      const uint32_t idesc_qk = idesc_f32acc(TQ, TK, 0, 0, kFmtF16);  // Q, K both K-major (d contiguous)
+      const uint32_t idesc_pv = idesc_f32acc(TQ, D, 0, 1, kFmtF16);   // P from TMEM, V MN-major (d contiguous)
+      int stage = 0;
+      uint32_t phase = 0;
+      uint32_t pcount[2] = {0, 0};
+      for (int r = 0;; ++r) {
+        const int w = item_index(r, cta, grid);
+        if (w >= p.items) break;
+        const Item it = get_item(p, w);
+        if (!mbar_wait_bounded(smem_u32(q_full), r & 1, p.err, abort_flag, wait_site(kSiteAttn, 2, 4))) goto done;
+        for (int j = 0; j < 2; ++j)
+          if (!mbar_wait_bounded(smem_u32(&o_empty[j]), (r & 1) ^ 1, p.err, abort_flag, wait_site(kSiteAttn, 2, 5))) goto done;
+        tc_fence_after();
+        const uint32_t q_base[2] = {smem_u32(smem + OFF_Q), smem_u32(smem + OFF_Q + TILE_BYTES)};
+        auto issue_qk = [&](int j, int st) {
+          const uint32_t kb = smem_u32(smem + OFF_K + st * TILE_BYTES);
+#pragma unroll
+          for (int kk = 0; kk < D / 16; ++kk) {
+            const uint32_t off = (kk >> 2) * HALF_BYTES + (kk & 3) * 32;
+            umma_ss(tmem + COL_S0 + j * TK, smem_desc_sw128(q_base[j] + off, 16, 1024),
+                    smem_desc_sw128(kb + off, 16, 1024), idesc_qk, kk > 0);
+          }
+          umma_commit(smem_u32(&s_full[j]));
+        };
+        // first key tile: S_j = Q_j K_0^T for both tiles
+        if (!mbar_wait_bounded(smem_u32(&k_full[stage]), phase, p.err, abort_flag, wait_site(kSiteAttn, 2, 6))) goto done;
+        tc_fence_after();
+        for (int j = 0; j < 2; ++j)
+          if (it.active[j]) issue_qk(j, stage);
+        umma_commit(smem_u32(&k_empty[stage]));
+        for (int jj = 0; jj < it.nkv_tiles; ++jj) {
+          const int nst = (stage + 1 == KV_STAGES) ? 0 : stage + 1;
+          const uint32_t nph = (stage + 1 == KV_STAGES) ? phase ^ 1 : phase;
+          bool next_k_ready = false;
+          if (!mbar_wait_bounded(smem_u32(&v_full[stage]), phase, p.err, abort_flag, wait_site(kSiteAttn, 2, 7))) goto done;
+          tc_fence_after();
+          const uint32_t vb = smem_u32(smem + OFF_V + stage * TILE_BYTES);
+          for (int j = 0; j < 2; ++j) {
+            if (!it.active[j] || jj > it.qt[j]) continue;
+            if (!mbar_wait_bounded(smem_u32(&p_full[j]), pcount[j] & 1, p.err, abort_flag, wait_site(kSiteAttn, 2, 8))) goto done;
+            ++pcount[j];
+            tc_fence_after();
+            // O_j += P_j V_jj
+#pragma unroll
+            for (int kk = 0; kk < TK / 16; ++kk)
+              umma_ts(tmem + COL_O0 + j * D, tmem + COL_S0 + j * TK + kk * 8,
+                      smem_desc_sw128(vb + kk * 16 * 128, HALF_BYTES, 1024), idesc_pv, (jj > 0 || kk > 0));
+            if (jj + 1 <= it.qt[j]) {
+              if (!next_k_ready) {
+                if (!mbar_wait_bounded(smem_u32(&k_full[nst]), nph, p.err, abort_flag, wait_site(kSiteAttn, 2, 9))) goto done;
+                tc_fence_after();
+                next_k_ready = true;
+              }
+              issue_qk(j, nst);  // S_j = Q_j K_{jj+1}^T, overwrites P_j after the PV above
+            } else {
+              umma_commit(smem_u32(&o_full[j]));
+            }
+          }
+          umma_commit(smem_u32(&v_empty[stage]));
+          if (next_k_ready) umma_commit(smem_u32(&k_empty[nst]));
+          stage = nst;
+          phase = nph;
+        }
+        umma_commit(smem_u32(q_empty));
+      }
+    }
+  } else {
+    // -------------------------------------------------------- softmax --
+    const int j = (warp - 2) >> 2;  // tile of this warpgroup
+    const int quad = warp & 3;      // TMEM lanes [32*quad, 32*quad + 32)
+    const int row = quad * 32 + lane;
+    const uint32_t lane_off = (uint32_t)(quad * 32) << 16;
+    const uint32_t s_col = tmem + lane_off + COL_S0 + j * TK;
+    const uint32_t o_col = tmem + lane_off + COL_O0 + j * D;
+    uint32_t scount = 0, ocount = 0;
+    for (int r = 0;; ++r) {
+      const int w = item_index(r, cta, grid);
+      if (w >= p.items) break;
+      const Item it = get_item(p, w);
+      if (it.active[j]) {
+        const int qt = it.qt[j];
+        float m = -INFINITY;  // running max of scaled scores (log2 domain)
+        float l = 0.f;        // running row sum
+        for (int jj = 0; jj <= qt; ++jj) {
+          if (!mbar_wait_bounded(smem_u32(&s_full[j]), scount & 1, p.err, abort_flag, wait_site(kSiteAttn, 3, 10))) goto done;
+          ++scount;
+          tc_fence_after();
+          uint32_t s[128];
+#pragma unroll
+          for (int c = 0; c < 4; ++c) tmem_ld_32x32b_x32(s_col + c * 32, s + c * 32);
+          tmem_ld_wait();
+          float tmax = -INFINITY;
+          if (jj == qt) {  // diagonal tile: key c is visible to query row iff c <= row
+#pragma unroll
+            for (int c = 0; c < 128; ++c) {
+              float v = (c <= row) ? u2f(s[c]) * p.scale_log2 : -INFINITY;
+              s[c] = __float_as_uint(v);
+              tmax = fmaxf(tmax, v);
+            }
+          } else {
+#pragma unroll
+            for (int c = 0; c < 128; ++c) {
+              float v = u2f(s[c]) * p.scale_log2;
+              s[c] = __float_as_uint(v);
+              tmax = fmaxf(tmax, v);
+            }
+          }
+          // lazy rescale: keep the stale max unless it grew by more than 2^8
+          const bool need = tmax > m + RESCALE_THRESHOLD;
+          float f = 1.f;  // factor for the O row and the sum
+          bool rescale = false;
+          if (jj == 0) {
+            m = tmax;
+          } else if (__any_sync(0xffffffffu, need)) {
+            const float mnew = fmaxf(m, tmax);
+            f = fast_exp2(m - mnew);
+            m = mnew;
+            rescale = true;
+          }
+          float sum = 0.f;
+#pragma unroll
+          for (int c2 = 0; c2 < 2; ++c2) {
+            uint32_t pk[32];
+#pragma unroll
+            for (int e = 0; e < 32; ++e) {
+              const float p0 = fast_exp2(u2f(s[c2 * 64 + 2 * e]) - m);
+              const float p1 = fast_exp2(u2f(s[c2 * 64 + 2 * e + 1]) - m);
+              sum += p0 + p1;
+              pk[e] = pack_f16x2(p0, p1);
+            }
+            tmem_st_32x32b_x32(s_col + c2 * 32, pk);
+          }
+          l = l * f + sum;
+          if (rescale) {
+            // O_j is stable: the commit behind s_full covered the previous PV
+#pragma unroll 1
+            for (int c = 0; c < 4; ++c) {
+              uint32_t o[32];
+              tmem_ld_32x32b_x32(o_col + c * 32, o);
+              tmem_ld_wait();
+#pragma unroll
+              for (int e = 0; e < 32; ++e) o[e] = __float_as_uint(u2f(o[e]) * f);
+              tmem_st_32x32b_x32(o_col + c * 32, o);
+            }
+          }
+          tmem_st_wait();
+          tc_fence_before();
+          __syncwarp();
+          if (lane == 0) mbar_arrive(smem_u32(&p_full[j]));
+        }
+        // epilogue: O / l -> fp16 -> global
+        if (!mbar_wait_bounded(smem_u32(&o_full[j]), ocount & 1, p.err, abort_flag, wait_site(kSiteAttn, 3, 11))) goto done;
+        ++ocount;
+        tc_fence_after();
+        const int t = qt * TQ + row;
+        const float inv = 1.f / l;
+        __half* dst = p.o + ((long long)it.b * p.S + t) * p.Lq + (long long)it.h[j] * D;
+#pragma unroll 1
+        for (int c = 0; c < 4; ++c) {
+          uint32_t o[32];
+          tmem_ld_32x32b_x32(o_col + c * 32, o);
+          tmem_ld_wait();
+          if (t < p.S) {
+            uint4* d4 = reinterpret_cast<uint4*>(dst + c * 32);
+#pragma unroll
+            for (int v = 0; v < 4; ++v) {
+              uint4 wv;
+              wv.x = pack_f16x2(u2f(o[8 * v + 0]) * inv, u2f(o[8 * v + 1]) * inv);
+              wv.y = pack_f16x2(u2f(o[8 * v + 2]) * inv, u2f(o[8 * v + 3]) * inv);
+              wv.z = pack_f16x2(u2f(o[8 * v + 4]) * inv, u2f(o[8 * v + 5]) * inv);
+              wv.w = pack_f16x2(u2f(o[8 * v + 6]) * inv, u2f(o[8 * v + 7]) * inv);
+              d4[v] = wv;
+            }
+          }
+        }
+        tc_fence_before();
+      }
+      __syncwarp();
+      if (lane == 0) mbar_arrive(smem_u32(&o_empty[j]));
+    }
+  }
+done:
+  tc_fence_before();
+  __syncthreads();
+  tc_fence_after();
+  if (warp == 1) tmem_dealloc(tmem, TMEM_COLS);
+}
+
+bool encode_3d(CUtensorMap* m, const void* ptr, uint64_t width, uint64_t S, uint64_t B) {
+  EncodeTiledFn enc = get_encode_tiled();
+  if (enc == nullptr) return false;
+  cuuint64_t dims[3] = {width, S, B};
+  cuuint64_t strides[2] = {width * 2, width * S * 2};
+  cuuint32_t box[3] = {64, 128, 1};
+  cuuint32_t estr[3] = {1, 1, 1};
+  return enc(m, CU_TENSOR_MAP_DATA_TYPE_FLOAT16, 3, const_cast<void*>(ptr), dims, strides, box, estr,
+             CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B, CU_TENSOR_MAP_L2_PROMOTION_L2_256B,
+             CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) == CUDA_SUCCESS;
+}
+
+}  // namespace
+
+bool attention_tc_supported(const BlockDims& dm) {
+  return dm.lat == DType::F16 && dm.d == D && dm.S >= 1 && (long long)dm.Lq * dm.S * 2 < (1ll << 40);
+}
+
+cudaError_t launch_attention_tc(const BlockDims& dm, const void* q, const void* k, const void* v, void* o,
+                                void* sched, unsigned* dev_err, cudaStream_t stream) {
+  (void)sched;
+  if (!attention_tc_supported(dm)) return cudaErrorInvalidValue;
+  AttnMaps maps;
+  if (!encode_3d(&maps.q, q, (uint64_t)dm.Lq, (uint64_t)dm.S, (uint64_t)dm.B) ||
+      !encode_3d(&maps.k, k, (uint64_t)dm.Lkv, (uint64_t)dm.S, (uint64_t)dm.B) ||
+      !encode_3d(&maps.v, v, (uint64_t)dm.Lkv, (uint64_t)dm.S, (uint64_t)dm.B))
+    return cudaErrorInvalidValue;
+  AttnParams p;
+  p.B = dm.B;
+  p.S = dm.S;
+  p.nq = dm.nq;
+  p.nkv = dm.nkv;
+  p.G = dm.G;
+  p.num_qt = (dm.S + TQ - 1) / TQ;
+  p.pairs = (p.num_qt * dm.G + 1) / 2;
+  p.items = dm.B * dm.nkv * p.pairs;
+  p.Lq = dm.Lq;
+  p.scale_log2 = dm.scale * 1.4426950408889634f;
+  p.o = static_cast<__half*>(o);
+  p.err = dev_err;
+  const int grid = p.items < num_sms() ? p.items : num_sms();
+  cudaError_t e = cudaFuncSetAttribute(attn_tc_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)SMEM_BYTES);
+  if (e != cudaSuccess) return e;
+  attn_tc_kernel<<<grid, NUM_THREADS, SMEM_BYTES, stream>>>(maps, p);
+  return cudaGetLastError();
+}
+
 }  // namespace cca

@@ -108,23 +108,32 @@ cca_status_t check_config(const cca_config_t* c, BlockDims* dm) {
     dm->use_rope = c->use_rope;
     dm->rope_base = c->rope_base;
     dm->scale = c->softmax_scale > 0.f ? c->softmax_scale : 1.0f / sqrtf((float)c->head_dim);
-    dm->bf16 = c->dtype == CCA_BF16;
-    dm->out_bf16 = c->out_dtype == CCA_BF16;
+    dm->io = c->dtype == CCA_BF16 ? DType::BF16 : DType::F32;
+    dm->lat = c->dtype == CCA_BF16 ? DType::F16 : DType::F32;
+    dm->out = c->out_dtype == CCA_BF16 ? DType::BF16 : DType::F32;
   }
   return CCA_OK;
 }
 
 cca_workspace_layout_t layout_of(const BlockDims& dm) {
   cca_workspace_layout_t L;
-  const size_t eb = dm.bf16 ? 2 : 4;
+  const size_t eb = dtype_bytes(dm.lat);
+  const bool sep = dm.lat != dm.io;  // attention K/V and W_o need their own copies
   L.elem_bytes = eb;
+  L.lat_dtype = dm.lat == DType::F16 ? CCA_F16 : (dm.lat == DType::BF16 ? CCA_BF16 : CCA_F32);
   size_t off = 0;
   L.qkv_lat_offset = off;
   off = align_up(off + (size_t)dm.T * dm.Nlat * eb);
   L.q_offset = off;
   off = align_up(off + (size_t)dm.T * dm.Lq * eb);
+  L.k_att_offset = off;
+  if (sep) off = align_up(off + (size_t)dm.T * dm.Lkv * eb);
+  L.v_att_offset = off;
+  if (sep) off = align_up(off + (size_t)dm.T * dm.Lkv * eb);
   L.o_offset = off;
   off = align_up(off + (size_t)dm.T * dm.Lq * eb);
+  L.wo_offset = off;
+  if (sep) off = align_up(off + (size_t)dm.E * dm.Lq * eb);
   L.sched_offset = off;
   off = align_up(off + 256);
   L.total_bytes = off;
@@ -135,7 +144,7 @@ bool aligned16(const void* p) { return (reinterpret_cast<uintptr_t>(p) & 15u) ==
 
 struct Resolved {
   BlockDims dm;
-  bool tensor;  // tcgen05 path
+  bool tc_down, tc_attn, tc_out;  // tcgen05 kernels per stage
 };
 
 cca_status_t resolve(const cca_config_t* cfg, int path, Resolved* r) {
@@ -144,13 +153,23 @@ cca_status_t resolve(const cca_config_t* cfg, int path, Resolved* r) {
   DeviceInfo* di = nullptr;
   if ((st = device_info(&di)) != CCA_OK) return st;
   const BlockDims& dm = r->dm;
-  const bool tc_ok = di->major == 10 && dm.bf16 && dm.d == 128 && gemm_tc_supported(dm.T, dm.Nlat, dm.E) &&
-                     gemm_tc_supported(dm.T, dm.E, dm.Lq) && attention_tc_supported(dm);
-  if (path == CCA_PATH_TENSOR && !tc_ok)
-    return fail(CCA_ERR_UNSUPPORTED, "tensor-core path needs sm_100, bf16 and head_dim 128");
-  if (path != CCA_PATH_AUTO && path != CCA_PATH_SIMT && path != CCA_PATH_TENSOR)
+  const bool masked = (path & ~7) == CCA_PATH_TENSOR_MASK(0);
+  if (path != CCA_PATH_AUTO && path != CCA_PATH_SIMT && path != CCA_PATH_TENSOR && !masked)
     return fail(CCA_ERR_INVALID_ARG, "unknown path");
-  r->tensor = (path == CCA_PATH_TENSOR) || (path == CCA_PATH_AUTO && tc_ok);
+  const bool sm100 = di->major == 10;
+  const bool b16 = dm.io == DType::BF16;
+  const bool down = sm100 && b16 && gemm_tc_supported(dm.T, dm.Nlat, dm.E) && dm.Lq % 128 == 0 &&
+                    dm.Lkv % 128 == 0;
+  const bool attn = sm100 && b16 && dm.d == 128 && attention_tc_supported(dm);
+  const bool out = sm100 && b16 && gemm_tc_supported(dm.T, dm.E, dm.Lq);
+  if (path == CCA_PATH_TENSOR && !(down && attn && out))
+    return fail(CCA_ERR_UNSUPPORTED, "tensor-core path needs sm_100, bf16, head_dim 128 and 128-aligned widths");
+  if (masked && (((path & 1) && !down) || ((path & 2) && !attn) || ((path & 4) && !out)))
+    return fail(CCA_ERR_UNSUPPORTED, "a stage asked for the tensor-core kernel cannot use it");
+  const bool use = path != CCA_PATH_SIMT;
+  r->tc_down = masked ? (path & 1) != 0 : use && down;
+  r->tc_attn = masked ? (path & 2) != 0 : use && attn;
+  r->tc_out = masked ? (path & 4) != 0 : use && out;
   return CCA_OK;
 }
 
@@ -168,10 +187,10 @@ cca_status_t run_block(const Resolved& r, BlockPtrs p, cudaStream_t stream, void
   auto mark = [&](int i) -> cudaError_t {
     return ev ? cudaEventRecord(static_cast<cudaEvent_t>(ev[i]), stream) : cudaSuccess;
   };
-  const size_t eb = dm.bf16 ? 2 : 4;
+  const size_t eb = dtype_bytes(dm.lat);
   if ((e = mark(0)) != cudaSuccess) return cuda_fail("event", e);
   // 1. down-projection: q~ | k~ | v~ = x [W_q; W_k; W_v]^T
-  if (r.tensor) {
+  if (r.tc_down) {
     GemmTcArgs a{};
     a.A = p.x;
     a.M = dm.T;
@@ -185,7 +204,8 @@ cca_status_t run_block(const Resolved& r, BlockPtrs p, cudaStream_t stream, void
     a.nb = 3;
     a.C = p.qkv_lat;
     a.ldc = dm.Nlat;
-    a.out_bf16 = true;
+    a.in = dm.io;
+    a.out = dm.lat;
     a.dev_err = p.dev_err;
     if ((e = launch_gemm_tc(a, stream)) != cudaSuccess) return cuda_fail("down-projection (tcgen05)", e);
   } else {
@@ -194,7 +214,7 @@ cca_status_t run_block(const Resolved& r, BlockPtrs p, cudaStream_t stream, void
     const int ns[3] = {dm.Lq, dm.Lkv, dm.Lkv};
     int col = 0;
     for (int i = 0; i < 3; ++i) {
-      if ((e = launch_gemm_simt(dm.bf16, dm.bf16, p.x, dm.E, Ws[i], dm.E, out + (size_t)col * eb, dm.Nlat, dm.T,
+      if ((e = launch_gemm_simt(dm.io, dm.lat, p.x, dm.E, Ws[i], dm.E, out + (size_t)col * eb, dm.Nlat, dm.T,
                                 ns[i], dm.E, stream)) != cudaSuccess)
         return cuda_fail("down-projection (SIMT)", e);
       col += ns[i];
@@ -206,30 +226,31 @@ cca_status_t run_block(const Resolved& r, BlockPtrs p, cudaStream_t stream, void
   if ((e = launch_conv_state(dm, p, stream)) != cudaSuccess) return cuda_fail("conv state", e);
   if ((e = mark(2)) != cudaSuccess) return cuda_fail("event", e);
   // 3. causal attention on the compressed heads
-  if (r.tensor) {
-    if ((e = launch_attention_tc(dm, p.q, p.k_cache, p.v_cache, p.o, p.sched, p.dev_err, stream)) != cudaSuccess)
+  if (r.tc_attn) {
+    if ((e = launch_attention_tc(dm, p.q, p.k_att, p.v_att, p.o, p.sched, p.dev_err, stream)) != cudaSuccess)
       return cuda_fail("attention (tcgen05)", e);
   } else {
-    if ((e = launch_attention_simt(dm, p.q, p.k_cache, p.v_cache, p.o, stream)) != cudaSuccess)
+    if ((e = launch_attention_simt(dm, p.q, p.k_att, p.v_att, p.o, stream)) != cudaSuccess)
       return cuda_fail("attention (SIMT)", e);
   }
   if ((e = mark(3)) != cudaSuccess) return cuda_fail("event", e);
   // 4. output projection y = o W_o^T
-  if (r.tensor) {
+  if (r.tc_out) {
     GemmTcArgs a{};
     a.A = p.o;
     a.M = dm.T;
     a.K = dm.Lq;
-    a.B[0] = p.Wo;
+    a.B[0] = p.wo_lat;
     a.nrows[0] = dm.E;
     a.nb = 1;
     a.C = p.y;
     a.ldc = dm.E;
-    a.out_bf16 = dm.out_bf16;
+    a.in = dm.lat;
+    a.out = dm.out;
     a.dev_err = p.dev_err;
     if ((e = launch_gemm_tc(a, stream)) != cudaSuccess) return cuda_fail("output projection (tcgen05)", e);
   } else {
-    if ((e = launch_gemm_simt(dm.bf16, dm.out_bf16, p.o, dm.Lq, p.Wo, dm.Lq, p.y, dm.E, dm.T, dm.E, dm.Lq,
+    if ((e = launch_gemm_simt(dm.lat, dm.out, p.o, dm.Lq, p.wo_lat, dm.Lq, p.y, dm.E, dm.T, dm.E, dm.Lq,
                               stream)) != cudaSuccess)
       return cuda_fail("output projection (SIMT)", e);
   }
@@ -274,9 +295,13 @@ cca_status_t prepare(const cca_config_t* cfg, int path, const void* const* ins, 
   p->k_cache = outs[1];
   p->v_cache = outs[2];
   p->conv_state = conv_state;
+  const bool sep = r->dm.lat != r->dm.io;
   p->qkv_lat = ws + L.qkv_lat_offset;
   p->q = ws + L.q_offset;
+  p->k_att = sep ? ws + L.k_att_offset : outs[1];
+  p->v_att = sep ? ws + L.v_att_offset : outs[2];
   p->o = ws + L.o_offset;
+  p->wo_lat = sep ? ws + L.wo_offset : const_cast<void*>(ins[8]);
   p->sched = ws + L.sched_offset;
   p->dev_err = nullptr;
   return CCA_OK;
@@ -314,7 +339,7 @@ __global__ void wait_timeout_selftest_kernel(unsigned* err, unsigned long long l
   }
   __syncthreads();
   // Nothing ever arrives on this barrier: the bounded wait must give up.
-  if (threadIdx.x == 0) (void)mbar_wait_bounded(a, 0, err, nullptr, limit_ns);
+  if (threadIdx.x == 0) (void)mbar_wait_bounded(a, 0, err, nullptr, wait_site(kSiteSelftest, 0, 0), limit_ns);
 }
 }  // namespace
 
@@ -340,6 +365,7 @@ const char* cca_status_string(cca_status_t s) {
     case CCA_ERR_WORKSPACE: return "workspace missing or too small";
     case CCA_ERR_CUDA: return "CUDA error";
     case CCA_ERR_DEVICE_TIMEOUT: return "device-side wait timed out";
+    case CCA_ERR_NUMERIC_RANGE: return "intermediate out of fp16 range";
   }
   return "unknown status";
 }
@@ -357,6 +383,18 @@ size_t cca_workspace_size(const cca_config_t* cfg) {
   BlockDims dm;
   if (check_config(cfg, &dm) != CCA_OK) return 0;
   return layout_of(dm).total_bytes;
+}
+
+cca_status_t cca_plan(const cca_config_t* cfg, int path, cca_plan_t* out) {
+  if (out == nullptr) return fail(CCA_ERR_INVALID_ARG, "out is NULL");
+  Resolved r;
+  cca_status_t st = resolve(cfg, path, &r);
+  if (st != CCA_OK) return st;
+  out->down_proj_tensor = r.tc_down;
+  out->attention_tensor = r.tc_attn;
+  out->out_proj_tensor = r.tc_out;
+  out->launches = (r.tc_down ? 1 : 3) + 1 + 1 + 1;
+  return CCA_OK;
 }
 
 cca_status_t cca_workspace_layout(const cca_config_t* cfg, cca_workspace_layout_t* out) {
@@ -404,8 +442,8 @@ cca_status_t cca_prefill_host(const cca_config_t* cfg, const void* x_host, void*
   cca_status_t st = prepare(cfg, CCA_PATH_AUTO, ins, outs, conv_state, workspace, workspace_bytes, &r, &p);
   if (st != CCA_OK) return st;
   cudaStream_t s = static_cast<cudaStream_t>(stream);
-  const size_t xbytes = (size_t)r.dm.T * r.dm.E * (r.dm.bf16 ? 2 : 4);
-  const size_t ybytes = (size_t)r.dm.T * r.dm.E * (r.dm.out_bf16 ? 2 : 4);
+  const size_t xbytes = (size_t)r.dm.T * r.dm.E * dtype_bytes(r.dm.io);
+  const size_t ybytes = (size_t)r.dm.T * r.dm.E * dtype_bytes(r.dm.out);
   cudaError_t e = cudaMemcpyAsync(x_dev, x_host, xbytes, cudaMemcpyHostToDevice, s);
   if (e != cudaSuccess) return cuda_fail("copy x to device", e);
   if ((st = run_block(r, p, s, nullptr)) != CCA_OK) return st;
@@ -428,7 +466,13 @@ cca_status_t cca_poll_device_status(void* stream) {
     unsigned zero = 0;
     if ((e = cudaMemcpy(di->err_ptr, &zero, sizeof(zero), cudaMemcpyHostToDevice)) != cudaSuccess)
       return cuda_fail("clear device error word", e);
-    return fail(CCA_ERR_DEVICE_TIMEOUT, "a bounded device-side wait gave up");
+    if ((h & 0xffu) == kDevErrRange)
+      return fail(CCA_ERR_NUMERIC_RANGE, "an intermediate exceeded the fp16 range (|value| > 65504)");
+    static const char* kernels[4] = {"?", "gemm", "attention", "self-test"};
+    char msg[160];
+    snprintf(msg, sizeof(msg), "a bounded device-side wait gave up (kernel %s, role %u, barrier %u)",
+             kernels[((h >> 8) & 0xffu) < 4 ? ((h >> 8) & 0xffu) : 0], (h >> 16) & 0xffu, (h >> 24) & 0xffu);
+    return fail(CCA_ERR_DEVICE_TIMEOUT, msg);
   }
   return CCA_OK;
 }

@@ -5,6 +5,7 @@
 
 #include <cuda.h>
 #include <cuda_bf16.h>
+#include <cuda_fp16.h>
 #include <cuda_runtime.h>
 #include <stdint.h>
 
@@ -14,7 +15,8 @@ namespace cca {
 // Codes written to the device error word (first writer wins).
 enum DeviceError : unsigned {
   kDevErrNone = 0,
-  kDevErrWaitTimeout = 1,
+  kDevErrWaitTimeout = 1,  // a bounded wait gave up
+  kDevErrRange = 2,        // a finite value did not fit the fp16 range of an intermediate
 };
 
 // A bounded wait gives up after this many nanoseconds of %globaltimer.
@@ -31,12 +33,30 @@ template <> struct Elem<__nv_bfloat16> {
   static __device__ __forceinline__ void store(__nv_bfloat16* p, float v) { *p = __float2bfloat16_rn(v); }
 };
 
+template <> struct Elem<__half> {
+  static __device__ __forceinline__ float load(const __half* p) { return __half2float(*p); }
+  static __device__ __forceinline__ void store(__half* p, float v) { *p = __float2half_rn(v); }
+};
+
 template <typename T> __device__ __forceinline__ float ld_f(const T* p) { return Elem<T>::load(p); }
 template <typename T> __device__ __forceinline__ void st_f(T* p, float v) { Elem<T>::store(p, v); }
 
 __device__ __forceinline__ uint32_t pack_bf16x2(float lo, float hi) {
   __nv_bfloat162 h = __floats2bfloat162_rn(lo, hi);  // .x = lo (low 16 bits)
   return *reinterpret_cast<uint32_t*>(&h);
+}
+__device__ __forceinline__ uint32_t pack_f16x2(float lo, float hi) {
+  __half2 h = __floats2half2_rn(lo, hi);  // .x = lo (low 16 bits)
+  return *reinterpret_cast<uint32_t*>(&h);
+}
+
+// True if v is finite but beyond the largest finite fp16 (65504).
+__device__ __forceinline__ bool f16_overflow(float v) { return fabsf(v) > 65504.0f && isfinite(v); }
+
+// Records kDevErrRange once per warp that saw an overflow (all lanes call).
+__device__ __forceinline__ void report_range(bool bad, unsigned* err) {
+  if (__any_sync(0xffffffffu, bad) && (threadIdx.x & 31) == 0 && err != nullptr)
+    atomicCAS(err, 0u, (unsigned)kDevErrRange);
 }
 
 // --------------------------------------------------------------- timing --
@@ -77,11 +97,18 @@ __device__ __forceinline__ bool mbar_try_wait(uint32_t bar, uint32_t parity) {
   return ok != 0;
 }
 
+// Where a bounded wait gave up, stored above the code in the error word:
+// bits [8,16) kernel, [16,24) role, [24,32) barrier.
+__host__ __device__ constexpr unsigned wait_site(unsigned kernel, unsigned role, unsigned barrier) {
+  return (kernel << 8) | (role << 16) | (barrier << 24);
+}
+enum WaitKernel : unsigned { kSiteGemm = 1, kSiteAttn = 2, kSiteSelftest = 3 };
+
 // Waits for phase `parity` of the mbarrier to complete. Gives up after
 // kWaitTimeoutNs (or as soon as *abort is set by another warp of the CTA),
-// records kDevErrWaitTimeout in *err, raises *abort and returns false.
+// records kDevErrWaitTimeout | site in *err, raises *abort and returns false.
 __device__ __forceinline__ bool mbar_wait_bounded(uint32_t bar, uint32_t parity, unsigned* err,
-                                                  volatile int* abort,
+                                                  volatile int* abort, unsigned site = 0,
                                                   unsigned long long limit_ns = kWaitTimeoutNs) {
 #pragma unroll 1
   for (int i = 0; i < 32; ++i)
@@ -94,7 +121,7 @@ __device__ __forceinline__ bool mbar_wait_bounded(uint32_t bar, uint32_t parity,
     if ((++n & 63u) == 0) {
       if (abort != nullptr && *abort) return false;
       if (globaltimer_ns() - t0 > limit_ns) {
-        atomicCAS(err, 0u, (unsigned)kDevErrWaitTimeout);
+        atomicCAS(err, 0u, (unsigned)kDevErrWaitTimeout | site);
         if (abort != nullptr) *abort = 1;
         return false;
       }
@@ -141,7 +168,7 @@ __device__ __forceinline__ void tc_fence_after() {
   asm volatile("tcgen05.fence::after_thread_sync;" ::: "memory");
 }
 
-// D[tmem] (+)= A[smem] * B[smem]^T, kind::f16 (bf16 in, fp32 accumulate).
+// D[tmem] (+)= A[smem] * B[smem]^T, kind::f16 (16-bit in, fp32 accumulate).
 __device__ __forceinline__ void umma_ss(uint32_t d_tmem, uint64_t a_desc, uint64_t b_desc, uint32_t idesc,
                                         uint32_t accumulate) {
   asm volatile(
@@ -177,15 +204,17 @@ __device__ __forceinline__ uint64_t smem_desc_sw128(uint32_t saddr, uint32_t lbo
   return d;
 }
 
-// Instruction descriptor for kind::f16: bf16 x bf16 -> fp32, dense.
-// a_mn / b_mn: 0 = K-major, 1 = MN-major.
-__host__ __device__ constexpr uint32_t idesc_bf16_f32(int M, int N, int a_mn, int b_mn) {
-  return (1u << 4)                       // D format fp32
-         | (1u << 7)                     // A format bf16
-         | (1u << 10)                    // B format bf16
+// Instruction descriptor for kind::f16 with fp32 accumulation, dense.
+// fmt: 0 = fp16, 1 = bf16 (A and B share it). a_mn / b_mn: 0 = K-major,
+// 1 = MN-major.
+__host__ __device__ constexpr uint32_t idesc_f32acc(int M, int N, int a_mn, int b_mn, int fmt) {
+  return (1u << 4)                                 // D format fp32
+         | ((uint32_t)fmt << 7)                    // A format
+         | ((uint32_t)fmt << 10)                   // B format
          | ((uint32_t)a_mn << 15) | ((uint32_t)b_mn << 16) | ((uint32_t)(N >> 3) << 17) |
          ((uint32_t)(M >> 4) << 24);
 }
+constexpr int kFmtF16 = 0, kFmtBF16 = 1;
 
 // 32 lanes x 32 columns of 32-bit: thread i of the warp gets lane (base+i),
 // columns [col, col+32).

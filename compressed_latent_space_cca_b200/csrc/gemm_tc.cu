@@ -1,6 +1,281 @@
-// placeholder, replaced by the tcgen05 GEMM
+// Tensor-core GEMM for sm_100a: C[M, N] = A[M, K] * B[N, K]^T, 16-bit inputs
+// (bf16 or fp16), fp32 accumulation in tensor memory, fp32 / bf16 / fp16
+// output.
+//
+// Used for the two dense projections of a CCA block ("Compressed
+// Convolutional Attention", gist.science/es/paper/2510.04476, section 2.A):
+// the down-projection of the hidden states to the q~ | k~ | v~ latents (the B
+// operand is W_q, W_k, W_v stacked by rows, each in its own buffer) and the
+// output projection o W_o^T.
+//
+// Design: persistent CTAs (one per SM) walk 128 x 256 output tiles. Warp 0
+// issues TMA loads of 128 x 64 A tiles and 256 x 64 B tiles (128-byte swizzle)
+// into a 4-stage shared-memory ring; one thread of warp 1 issues
+// tcgen05.mma (M=128, N=256, K=16) into one of two 256-column fp32
+// accumulators in tensor memory; warps 2-5 drain the other accumulator
+// (tcgen05.ld -> convert -> global store) so the epilogue of tile i overlaps
+// the main loop of tile i+1. Every mbarrier wait is bounded.
+#include "cca_common.cuh"
 #include "launch.h"
+
 namespace cca {
-bool gemm_tc_supported(long long, int, int) { return false; }
-cudaError_t launch_gemm_tc(const GemmTcArgs&, cudaStream_t) { return cudaErrorNotSupported; }
+namespace {
+
+constexpr int BM = 128, BN = 256, BK = 64, STAGES = 4;
+constexpr int A_BYTES = BM * BK * 2;  // 16 KB
+constexpr int B_BYTES = BN * BK * 2;  // 32 KB
+constexpr int STAGE_BYTES = A_BYTES + B_BYTES;
+constexpr int NUM_THREADS = 192;
+constexpr int TMEM_COLS = 512;  // two 128 x 256 fp32 accumulators
+constexpr size_t SMEM_BYTES = (size_t)STAGES * STAGE_BYTES + 1024 /*align slack*/ + 256 /*barriers*/;
+
+struct GemmMaps {
+  CUtensorMap a;
+  CUtensorMap b[3];
+};
+
+struct GemmParams {
+  long long M;
+  int N, K;
+  int nb;
+  int row_start[3];  // first row of B matrix i in the stacked operand
+  int nrows[3];
+  void* C;
+  long long ldc;
+  int out_type;  // DType of C
+  int in_fmt;    // kFmtBF16 or kFmtF16
+  unsigned* err;
+  int num_tiles;
+  int n_tiles_n;
+};
+
+// Stores 32 fp32 accumulators of one row; returns true if an fp16 output overflowed.
+__device__ __forceinline__ bool store_row_chunk(const GemmParams& p, long long row, int col0, const uint32_t* r) {
+  bool bad = false;
+  if (p.out_type == (int)DType::BF16 || p.out_type == (int)DType::F16) {
+    const bool h = p.out_type == (int)DType::F16;
+    uint4* dst = reinterpret_cast<uint4*>(static_cast<uint16_t*>(p.C) + row * p.ldc + col0);
+#pragma unroll
+    for (int v = 0; v < 4; ++v) {
+      uint32_t w[4];
+#pragma unroll
+      for (int e = 0; e < 4; ++e) {
+        const float a = u2f(r[8 * v + 2 * e]), b = u2f(r[8 * v + 2 * e + 1]);
+        if (h) {
+          w[e] = pack_f16x2(a, b);
+          bad |= f16_overflow(a) || f16_overflow(b);
+        } else {
+          w[e] = pack_bf16x2(a, b);
+        }
+      }
+      dst[v] = make_uint4(w[0], w[1], w[2], w[3]);
+    }
+  } else {
+    uint4* dst = reinterpret_cast<uint4*>(static_cast<float*>(p.C) + row * p.ldc + col0);
+#pragma unroll
+    for (int v = 0; v < 8; ++v) dst[v] = make_uint4(r[4 * v], r[4 * v + 1], r[4 * v + 2], r[4 * v + 3]);
+  }
+  return bad;
+}
+
+__global__ void __launch_bounds__(NUM_THREADS, 1) gemm_tc_kernel(const __grid_constant__ GemmMaps maps,
+                                                                 const GemmParams p) {
+  extern __shared__ uint8_t smem_raw[];
+  uint8_t* smem = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
+  uint64_t* bars = reinterpret_cast<uint64_t*>(smem + STAGES * STAGE_BYTES);
+  uint64_t* full = bars;                 // [STAGES] TMA -> MMA
+  uint64_t* empty = bars + STAGES;       // [STAGES] MMA -> TMA
+  uint64_t* tfull = bars + 2 * STAGES;   // [2] MMA -> epilogue
+  uint64_t* tempty = bars + 2 * STAGES + 2;  // [2] epilogue -> MMA
+  uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(bars + 2 * STAGES + 4);
+  volatile int* abort_flag = reinterpret_cast<volatile int*>(tmem_slot + 1);
+
+  const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+  if (threadIdx.x == 0) {
+    for (int s = 0; s < STAGES; ++s) {
+      mbar_init(smem_u32(&full[s]), 1);
+      mbar_init(smem_u32(&empty[s]), 1);
+    }
+    for (int a = 0; a < 2; ++a) {
+      mbar_init(smem_u32(&tfull[a]), 1);
+      mbar_init(smem_u32(&tempty[a]), 4);
+    }
+    *abort_flag = 0;
+    fence_mbar_init();
+  }
+  if (warp == 0 && lane == 0) {
+    prefetch_tmap(&maps.a);
+    for (int i = 0; i < p.nb; ++i) prefetch_tmap(&maps.b[i]);
+  }
+  if (warp == 1) {
+    tmem_alloc(smem_u32(tmem_slot), TMEM_COLS);
+    tmem_relinquish();
+  }
+  tc_fence_before();
+  __syncthreads();
+  tc_fence_after();
+  const uint32_t tmem_base = *tmem_slot;
+  const int kblocks = p.K / BK;
+
+  if (warp == 0) {
+    if (lane == 0) {
+      // ---------------------------------------------------- TMA producer --
+      int stage = 0;
+      uint32_t phase = 0;
+      for (int t = blockIdx.x; t < p.num_tiles; t += gridDim.x) {
+        const int m0 = (t / p.n_tiles_n) * BM;
+        const int n0 = (t % p.n_tiles_n) * BN;
+        for (int kb = 0; kb < kblocks; ++kb) {
+          if (!mbar_wait_bounded(smem_u32(&empty[stage]), phase ^ 1, p.err, abort_flag, wait_site(kSiteGemm, 1, 1))) goto producer_done;
+          const uint32_t fb = smem_u32(&full[stage]);
+          mbar_arrive_expect_tx(fb, STAGE_BYTES);
+          uint8_t* sa = smem + stage * STAGE_BYTES;
+          tma_load_2d(smem_u32(sa), &maps.a, fb, kb * BK, m0);
+#pragma unroll
+          for (int h = 0; h < 2; ++h) {
+            const int row = n0 + h * 128;
+            int mi = p.nb - 1, r = p.nrows[p.nb - 1];  // past the end: zero fill
+            if (row < p.N) {
+              mi = 0;
+              while (mi + 1 < p.nb && row >= p.row_start[mi + 1]) ++mi;
+              r = row - p.row_start[mi];
+            }
+            tma_load_2d(smem_u32(sa + A_BYTES + h * (128 * BK * 2)), &maps.b[mi], fb, kb * BK, r);
+          }
+          if (++stage == STAGES) {
+            stage = 0;
+            phase ^= 1;
+          }
+        }
+      }
+    producer_done:;
+    }
+  } else if (warp == 1) {
+    if (lane == 0) {
+      // ------------------------------------------------------ MMA issuer --
+      const uint32_t idesc = idesc_f32acc(BM, BN, 0, 0, p.in_fmt);
+      int stage = 0;
+      uint32_t phase = 0;
+      int i = 0;
+      for (int t = blockIdx.x; t < p.num_tiles; t += gridDim.x, ++i) {
+        const int acc = i & 1;
+        const uint32_t tph = (i >> 1) & 1;
+        if (!mbar_wait_bounded(smem_u32(&tempty[acc]), tph ^ 1, p.err, abort_flag, wait_site(kSiteGemm, 2, 2))) goto mma_done;
+        tc_fence_after();
+        const uint32_t d_tmem = tmem_base + acc * BN;
+        for (int kb = 0; kb < kblocks; ++kb) {
+          if (!mbar_wait_bounded(smem_u32(&full[stage]), phase, p.err, abort_flag, wait_site(kSiteGemm, 2, 3))) goto mma_done;
+          tc_fence_after();
+          const uint32_t a_base = smem_u32(smem + stage * STAGE_BYTES);
+          const uint32_t b_base = a_base + A_BYTES;
+#pragma unroll
+          for (int k = 0; k < BK / 16; ++k) {
+            const uint64_t ad = smem_desc_sw128(a_base + k * 32, 16, 1024);
+            const uint64_t bd = smem_desc_sw128(b_base + k * 32, 16, 1024);
+            umma_ss(d_tmem, ad, bd, idesc, (kb | k) != 0);
+          }
+          umma_commit(smem_u32(&empty[stage]));
+          if (++stage == STAGES) {
+            stage = 0;
+            phase ^= 1;
+          }
+        }
+        umma_commit(smem_u32(&tfull[acc]));
+      }
+    mma_done:;
+    }
+  } else {
+    // --------------------------------------------------------- epilogue --
+    const int quad = warp & 3;  // this warp may touch TMEM lanes [32*quad, 32*quad+32)
+    bool bad = false;
+    int i = 0;
+    for (int t = blockIdx.x; t < p.num_tiles; t += gridDim.x, ++i) {
+      const int acc = i & 1;
+      const uint32_t tph = (i >> 1) & 1;
+      if (!mbar_wait_bounded(smem_u32(&tfull[acc]), tph, p.err, abort_flag, wait_site(kSiteGemm, 3, 4))) break;
+      tc_fence_after();
+      const long long m0 = (long long)(t / p.n_tiles_n) * BM;
+      const int n0 = (t % p.n_tiles_n) * BN;
+      const long long row = m0 + quad * 32 + lane;
+#pragma unroll 1
+      for (int c = 0; c < BN / 32; ++c) {
+        uint32_t r[32];
+        tmem_ld_32x32b_x32(tmem_base + ((uint32_t)(quad * 32) << 16) + acc * BN + c * 32, r);
+        tmem_ld_wait();
+        const int col0 = n0 + c * 32;
+        if (row < p.M && col0 < p.N) bad |= store_row_chunk(p, row, col0, r);
+      }
+      tc_fence_before();
+      __syncwarp();
+      if (lane == 0) mbar_arrive(smem_u32(&tempty[acc]));
+    }
+    report_range(bad, p.err);
+  }
+  tc_fence_before();
+  __syncthreads();
+  tc_fence_after();
+  if (warp == 1) tmem_dealloc(tmem_base, TMEM_COLS);
+}
+
+bool encode_2d(CUtensorMap* m, const void* ptr, CUtensorMapDataType dt, uint64_t inner, uint64_t outer,
+               uint32_t box_inner, uint32_t box_outer) {
+  EncodeTiledFn enc = get_encode_tiled();
+  if (enc == nullptr) return false;
+  cuuint64_t dims[2] = {inner, outer};
+  cuuint64_t strides[1] = {inner * 2};
+  cuuint32_t box[2] = {box_inner, box_outer};
+  cuuint32_t estr[2] = {1, 1};
+  return enc(m, dt, 2, const_cast<void*>(ptr), dims, strides, box, estr,
+             CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B, CU_TENSOR_MAP_L2_PROMOTION_L2_256B,
+             CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) == CUDA_SUCCESS;
+}
+
+}  // namespace
+
+bool gemm_tc_supported(long long M, int N, int K) {
+  return M >= 1 && M < (1ll << 31) && K >= BK && K % BK == 0 && N >= 128 && N % 128 == 0;
+}
+
+cudaError_t launch_gemm_tc(const GemmTcArgs& a, cudaStream_t stream) {
+  int N = 0;
+  for (int i = 0; i < a.nb; ++i) {
+    if (a.nrows[i] % 128 != 0) return cudaErrorInvalidValue;
+    N += a.nrows[i];
+  }
+  if (!gemm_tc_supported(a.M, N, a.K) || a.nb < 1 || a.nb > 3) return cudaErrorInvalidValue;
+  if (a.ldc % 8 != 0 || (reinterpret_cast<uintptr_t>(a.C) & 15) != 0) return cudaErrorInvalidValue;
+  if (a.in != DType::BF16 && a.in != DType::F16) return cudaErrorInvalidValue;
+  const CUtensorMapDataType dt =
+      a.in == DType::F16 ? CU_TENSOR_MAP_DATA_TYPE_FLOAT16 : CU_TENSOR_MAP_DATA_TYPE_BFLOAT16;
+  GemmMaps maps;
+  GemmParams p{};
+  if (!encode_2d(&maps.a, a.A, dt, (uint64_t)a.K, (uint64_t)a.M, BK, BM)) return cudaErrorInvalidValue;
+  int start = 0;
+  for (int i = 0; i < 3; ++i) {
+    const int src = i < a.nb ? i : 0;
+    if (!encode_2d(&maps.b[i], a.B[src], dt, (uint64_t)a.K, (uint64_t)a.nrows[src], BK, 128))
+      return cudaErrorInvalidValue;
+    p.row_start[i] = i < a.nb ? start : N;
+    p.nrows[i] = a.nrows[src];
+    if (i < a.nb) start += a.nrows[i];
+  }
+  p.M = a.M;
+  p.N = N;
+  p.K = a.K;
+  p.nb = a.nb;
+  p.C = a.C;
+  p.ldc = a.ldc;
+  p.out_type = (int)a.out;
+  p.in_fmt = a.in == DType::F16 ? kFmtF16 : kFmtBF16;
+  p.err = a.dev_err;
+  p.n_tiles_n = (N + BN - 1) / BN;
+  const long long m_tiles = (a.M + BM - 1) / BM;
+  p.num_tiles = (int)(m_tiles * p.n_tiles_n);
+  const int grid = p.num_tiles < num_sms() ? p.num_tiles : num_sms();
+  cudaError_t e = cudaFuncSetAttribute(gemm_tc_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)SMEM_BYTES);
+  if (e != cudaSuccess) return e;
+  gemm_tc_kernel<<<grid, NUM_THREADS, SMEM_BYTES, stream>>>(maps, p);
+  return cudaGetLastError();
+}
+
 }  // namespace cca

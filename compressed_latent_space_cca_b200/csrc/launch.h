@@ -8,7 +8,18 @@
 
 namespace cca {
 
+// Element types that move between stages.
+enum class DType : int { F32 = 0, BF16 = 1, F16 = 2 };
+
+inline size_t dtype_bytes(DType t) { return t == DType::F32 ? 4 : 2; }
+
 // Shape and options of one block, resolved from cca_config_t.
+//
+// Storage types: `io` is the type of the inputs and of the KV cache; `lat`
+// the type of every intermediate (latents, attention q/k/v, attention
+// output, the output-projection weight copy); `out` the type of y. For bf16
+// blocks the intermediates are fp16: same tensor-core rate, 8x finer
+// rounding, which keeps the chain of roundings inside the parity budget.
 struct BlockDims {
   int B, S, E, nq, nkv, d, K;
   int G;        // nq / nkv
@@ -17,23 +28,28 @@ struct BlockDims {
   long long T;  // B*S
   int qk_mean_mode, value_shift, use_rope;
   float rope_base, scale;
-  bool bf16;      // element type of inputs, intermediates and the KV cache
-  bool out_bf16;  // element type of y
+  DType io, lat, out;
 };
 
 // Pointers of one call (all device memory).
 struct BlockPtrs {
   const void *x, *Wq, *Wk, *Wv, *cq_seq, *cq_chan, *ck_seq, *ck_chan, *Wo;
   void *y, *k_cache, *v_cache, *conv_state;
-  void *qkv_lat, *q, *o, *sched;
+  // workspace
+  void* qkv_lat;  // [T, Nlat] lat
+  void* q;        // [T, Lq]  lat: attention queries
+  void* k_att;    // [T, Lkv] lat: attention keys (== k_cache when lat == io)
+  void* v_att;    // [T, Lkv] lat: attention values (== v_cache when lat == io)
+  void* o;        // [T, Lq]  lat: attention output
+  void* wo_lat;   // [E, Lq]  lat copy of W_o (== Wo when lat == io)
+  void* sched;
   unsigned* dev_err;
 };
 
 // ---- SIMT path (any dtype, any even head_dim <= 128) ----
 // C[M, ldc] (cols [0,N)) = A[M,K] (row stride lda) * B[N,K]^T (row stride ldb)
-cudaError_t launch_gemm_simt(bool in_bf16, bool out_bf16, const void* A, long long lda, const void* Bm,
-                             long long ldb, void* C, long long ldc, long long M, int N, int K,
-                             cudaStream_t stream);
+cudaError_t launch_gemm_simt(DType in, DType out, const void* A, long long lda, const void* Bm, long long ldb,
+                             void* C, long long ldc, long long M, int N, int K, cudaStream_t stream);
 cudaError_t launch_attention_simt(const BlockDims& dm, const void* q, const void* k, const void* v, void* o,
                                   cudaStream_t stream);
 
@@ -41,10 +57,11 @@ cudaError_t launch_attention_simt(const BlockDims& dm, const void* q, const void
 cudaError_t launch_preproc_simt(const BlockDims& dm, const BlockPtrs& p, cudaStream_t stream);
 cudaError_t launch_conv_state(const BlockDims& dm, const BlockPtrs& p, cudaStream_t stream);
 
-// ---- tensor-core path (bf16, head_dim 128, sm_100a) ----
+// ---- tensor-core path (16-bit operands, sm_100a) ----
 bool gemm_tc_supported(long long M, int N, int K);
 // C[M, ldc] (cols [0,N)) = A[M,K] * [B0; B1; B2][N,K]^T, where the B operand
-// is split by rows into up to three separate matrices of n0, n1, n2 rows.
+// is split by rows into up to three separate matrices. A and B share `in`
+// (BF16 or F16); C is `out`.
 struct GemmTcArgs {
   const void* A;
   long long M;
@@ -54,7 +71,7 @@ struct GemmTcArgs {
   int nb;
   void* C;
   long long ldc;
-  bool out_bf16;
+  DType in, out;
   unsigned* dev_err;
 };
 cudaError_t launch_gemm_tc(const GemmTcArgs& a, cudaStream_t stream);

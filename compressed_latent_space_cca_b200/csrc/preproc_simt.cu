@@ -1,5 +1,6 @@
 // Latent preprocessing of one CCA / CCGQA block, general SIMT version
-// (any even head_dim <= 128, fp32 or bf16 storage, fp32 arithmetic).
+// (any even head_dim <= 128; fp32 blocks, or bf16 blocks with fp16
+// intermediates; fp32 arithmetic).
 //
 // "Compressed Convolutional Attention" (gist.science/es/paper/2510.04476),
 // section 2.B: on the compressed q~ and k~ a causal convolution along the
@@ -22,12 +23,14 @@ namespace {
 constexpr int PP_TT = 8;       // tokens per CTA
 constexpr int PP_THREADS = 256;
 
-template <typename T>
+// Tl: intermediates (latents in, attention q/k/v out); Tc: weights and KV cache.
+template <typename Tl, typename Tc>
 __global__ void __launch_bounds__(PP_THREADS) preproc_simt_kernel(
-    const T* __restrict__ qkv, const T* __restrict__ cq_seq, const T* __restrict__ cq_chan,
-    const T* __restrict__ ck_seq, const T* __restrict__ ck_chan, T* __restrict__ qout, T* __restrict__ kout,
-    T* __restrict__ vout, int S, int nq, int nkv, int d, int K, int mode, int vshift, int use_rope,
-    float rope_base) {
+    const Tl* __restrict__ qkv, const Tc* __restrict__ cq_seq, const Tc* __restrict__ cq_chan,
+    const Tc* __restrict__ ck_seq, const Tc* __restrict__ ck_chan, Tl* __restrict__ qout, Tc* __restrict__ kout,
+    Tc* __restrict__ vout, Tl* __restrict__ katt, Tl* __restrict__ vatt, const Tc* __restrict__ wo,
+    Tl* __restrict__ wo_lat, long long wo_n, unsigned* __restrict__ err, int S, int nq, int nkv, int d, int K,
+    int mode, int vshift, int use_rope, float rope_base) {
   extern __shared__ float sm[];
   const int G = nq / nkv;
   const int H1 = G + 1;  // G query heads + the K head of the group
@@ -69,7 +72,7 @@ __global__ void __launch_bounds__(PP_THREADS) preproc_simt_kernel(
   // causal depthwise conv along the sequence; tap j reads token t-K+1+j
   for (int e = tid; e < H1 * PP_TT * d; e += PP_THREADS) {
     int hh = e / (PP_TT * d), rem = e % (PP_TT * d), tt = rem / d, i = rem % d;
-    const T* w = (hh < G) ? cq_seq + (long long)((g * G + hh) * d + i) * K : ck_seq + (long long)(g * d + i) * K;
+    const Tc* w = (hh < G) ? cq_seq + (long long)((g * G + hh) * d + i) * K : ck_seq + (long long)(g * d + i) * K;
     const float* z = zin + (hh * R + tt) * d + i;
     float acc = 0.f;
     for (int j = 0; j < K; ++j) acc = fmaf(ld_f(w + j), z[j * d], acc);
@@ -82,7 +85,7 @@ __global__ void __launch_bounds__(PP_THREADS) preproc_simt_kernel(
     const int warp = tid >> 5, lane = tid & 31, nwarps = PP_THREADS / 32;
     for (int row = warp; row < H1 * d; row += nwarps) {
       int hh = row / d, i = row % d;
-      const T* W = (hh < G) ? cq_chan + ((long long)(g * G + hh) * d + i) * d : ck_chan + ((long long)g * d + i) * d;
+      const Tc* W = (hh < G) ? cq_chan + ((long long)(g * G + hh) * d + i) * d : ck_chan + ((long long)g * d + i) * d;
       float wv[4];
 #pragma unroll
       for (int m = 0; m < 4; ++m) {
@@ -128,21 +131,35 @@ __global__ void __launch_bounds__(PP_THREADS) preproc_simt_kernel(
     }
     return r;
   };
-  for (int e = tid; e < H1 * PP_TT * half; e += PP_THREADS) {
+  bool bad = false;
+  for (int e0 = 0; e0 < H1 * PP_TT * half; e0 += PP_THREADS) {
+    const int e = e0 + tid;
     int hh = e / (PP_TT * half), rem = e % (PP_TT * half), tt = rem / half, i = rem % half;
     int t = t0 + tt;
-    if (t >= S) continue;
-    float x1 = combined(hh, tt, i), x2 = combined(hh, tt, i + half);
-    float o1 = x1, o2 = x2;
-    if (use_rope) {
-      float c = rcos[tt * half + i], s = rsin[tt * half + i];
-      o1 = x1 * c - x2 * s;
-      o2 = x2 * c + x1 * s;
+    if (e < H1 * PP_TT * half && t < S) {
+      float x1 = combined(hh, tt, i), x2 = combined(hh, tt, i + half);
+      float o1 = x1, o2 = x2;
+      if (use_rope) {
+        float c = rcos[tt * half + i], s = rsin[tt * half + i];
+        o1 = x1 * c - x2 * s;
+        o2 = x2 * c + x1 * s;
+      }
+      if (hh < G) {
+        Tl* dst = qout + (rowbase + t) * Lq + (long long)(g * G + hh) * d;
+        st_f(dst + i, o1);
+        st_f(dst + i + half, o2);
+      } else {
+        Tc* dst = kout + (rowbase + t) * Lkv + (long long)g * d;
+        st_f(dst + i, o1);
+        st_f(dst + i + half, o2);
+        if (katt != nullptr) {
+          Tl* da = katt + (rowbase + t) * Lkv + (long long)g * d;
+          st_f(da + i, o1);
+          st_f(da + i + half, o2);
+        }
+      }
+      if (sizeof(Tl) == 2) bad |= f16_overflow(o1) || f16_overflow(o2);
     }
-    T* dst = (hh < G) ? qout + (rowbase + t) * Lq + (long long)(g * G + hh) * d
-                      : kout + (rowbase + t) * Lkv + (long long)g * d;
-    st_f(dst + i, o1);
-    st_f(dst + i + half, o2);
   }
 
   // value shift: channels [Lkv/2, Lkv) come from the previous token
@@ -152,23 +169,35 @@ __global__ void __launch_bounds__(PP_THREADS) preproc_simt_kernel(
     if (t >= S) continue;
     int gc = g * d + i;
     int src = (vshift && gc >= Lkv / 2) ? t - 1 : t;
-    T* dst = vout + (rowbase + t) * Lkv + gc;
-    if (src >= 0)
-      *dst = qkv[(rowbase + src) * Nlat + Lq + Lkv + gc];
-    else
-      st_f(dst, 0.f);
+    const float val = (src >= 0) ? ld_f(qkv + (rowbase + src) * Nlat + Lq + Lkv + gc) : 0.f;
+    st_f(vout + (rowbase + t) * Lkv + gc, val);
+    if (vatt != nullptr) st_f(vatt + (rowbase + t) * Lkv + gc, val);
   }
+
+  // side job: this CTA's slice of the W_o copy in the intermediate type
+  if (wo_lat != nullptr) {
+    const long long nct = (long long)gridDim.x * gridDim.y * gridDim.z;
+    const long long cid = ((long long)blockIdx.z * gridDim.y + blockIdx.y) * gridDim.x + blockIdx.x;
+    const long long chunk = (wo_n + nct - 1) / nct;
+    const long long lo = cid * chunk, hi = lo + chunk < wo_n ? lo + chunk : wo_n;
+    for (long long e = lo + tid; e < hi; e += PP_THREADS) {
+      const float w = ld_f(wo + e);
+      st_f(wo_lat + e, w);
+      bad |= f16_overflow(w);
+    }
+  }
+  report_range(bad, err);
 }
 
 // Conv state per sequence: the last K-1 rows of q~ and of k~ and the last row
 // of v~, zero rows before the sequence start.
-template <typename T>
-__global__ void conv_state_kernel(const T* __restrict__ qkv, T* __restrict__ state, int S, int Lq, int Lkv,
+template <typename Tl, typename Tc>
+__global__ void conv_state_kernel(const Tl* __restrict__ qkv, Tc* __restrict__ state, int S, int Lq, int Lkv,
                                   int K) {
   const int b = blockIdx.x;
   const int Nlat = Lq + 2 * Lkv;
   const long long per = (long long)(K - 1) * (Lq + Lkv) + Lkv;
-  T* dst = state + b * per;
+  Tc* dst = state + b * per;
   const long long rowbase = (long long)b * S;
   for (long long e = threadIdx.x; e < per; e += blockDim.x) {
     int t, col;
@@ -183,51 +212,47 @@ __global__ void conv_state_kernel(const T* __restrict__ qkv, T* __restrict__ sta
       t = S - 1;
       col = Lq + Lkv + (int)(e - (long long)(K - 1) * (Lq + Lkv));
     }
-    if (t >= 0)
-      dst[e] = qkv[(rowbase + t) * Nlat + col];
-    else
-      st_f(dst + e, 0.f);
+    st_f(dst + e, t >= 0 ? ld_f(qkv + (rowbase + t) * Nlat + col) : 0.f);
   }
 }
 
 }  // namespace
 
-cudaError_t launch_preproc_simt(const BlockDims& dm, const BlockPtrs& p, cudaStream_t stream) {
+namespace {
+template <typename Tl, typename Tc>
+cudaError_t preproc_typed(const BlockDims& dm, const BlockPtrs& p, cudaStream_t stream) {
   const int H1 = dm.G + 1, R = PP_TT + dm.K - 1;
   size_t smem = sizeof(float) * ((size_t)H1 * R * dm.d + 2 * (size_t)H1 * PP_TT * dm.d + (size_t)PP_TT * dm.d);
   dim3 grid((dm.S + PP_TT - 1) / PP_TT, dm.nkv, dm.B);
-  cudaError_t e;
-  if (dm.bf16) {
-    using T = __nv_bfloat16;
-    auto kern = preproc_simt_kernel<T>;
-    if ((e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem)) != cudaSuccess)
-      return e;
-    kern<<<grid, PP_THREADS, smem, stream>>>((const T*)p.qkv_lat, (const T*)p.cq_seq, (const T*)p.cq_chan,
-                                             (const T*)p.ck_seq, (const T*)p.ck_chan, (T*)p.q, (T*)p.k_cache,
-                                             (T*)p.v_cache, dm.S, dm.nq, dm.nkv, dm.d, dm.K, dm.qk_mean_mode,
-                                             dm.value_shift, dm.use_rope, dm.rope_base);
-  } else {
-    using T = float;
-    auto kern = preproc_simt_kernel<T>;
-    if ((e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem)) != cudaSuccess)
-      return e;
-    kern<<<grid, PP_THREADS, smem, stream>>>((const T*)p.qkv_lat, (const T*)p.cq_seq, (const T*)p.cq_chan,
-                                             (const T*)p.ck_seq, (const T*)p.ck_chan, (T*)p.q, (T*)p.k_cache,
-                                             (T*)p.v_cache, dm.S, dm.nq, dm.nkv, dm.d, dm.K, dm.qk_mean_mode,
-                                             dm.value_shift, dm.use_rope, dm.rope_base);
-  }
+  auto kern = preproc_simt_kernel<Tl, Tc>;
+  cudaError_t e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
+  if (e != cudaSuccess) return e;
+  const bool sep = dm.lat != dm.io;  // separate attention K/V and W_o copies
+  kern<<<grid, PP_THREADS, smem, stream>>>(
+      (const Tl*)p.qkv_lat, (const Tc*)p.cq_seq, (const Tc*)p.cq_chan, (const Tc*)p.ck_seq, (const Tc*)p.ck_chan,
+      (Tl*)p.q, (Tc*)p.k_cache, (Tc*)p.v_cache, sep ? (Tl*)p.k_att : nullptr, sep ? (Tl*)p.v_att : nullptr,
+      (const Tc*)p.Wo, sep ? (Tl*)p.wo_lat : nullptr, (long long)dm.E * dm.Lq, p.dev_err, dm.S, dm.nq, dm.nkv, dm.d,
+      dm.K, dm.qk_mean_mode, dm.value_shift, dm.use_rope, dm.rope_base);
   return cudaGetLastError();
+}
+}  // namespace
+
+cudaError_t launch_preproc_simt(const BlockDims& dm, const BlockPtrs& p, cudaStream_t stream) {
+  if (dm.io == DType::BF16 && dm.lat == DType::F16) return preproc_typed<__half, __nv_bfloat16>(dm, p, stream);
+  if (dm.io == DType::F32 && dm.lat == DType::F32) return preproc_typed<float, float>(dm, p, stream);
+  return cudaErrorInvalidValue;
 }
 
 cudaError_t launch_conv_state(const BlockDims& dm, const BlockPtrs& p, cudaStream_t stream) {
   if (p.conv_state == nullptr) return cudaSuccess;
-  if (dm.bf16)
-    conv_state_kernel<__nv_bfloat16><<<dm.B, 256, 0, stream>>>((const __nv_bfloat16*)p.qkv_lat,
-                                                                (__nv_bfloat16*)p.conv_state, dm.S, dm.Lq,
-                                                                dm.Lkv, dm.K);
+  if (dm.io == DType::BF16 && dm.lat == DType::F16)
+    conv_state_kernel<__half, __nv_bfloat16><<<dm.B, 256, 0, stream>>>(
+        (const __half*)p.qkv_lat, (__nv_bfloat16*)p.conv_state, dm.S, dm.Lq, dm.Lkv, dm.K);
+  else if (dm.io == DType::F32 && dm.lat == DType::F32)
+    conv_state_kernel<float, float><<<dm.B, 256, 0, stream>>>((const float*)p.qkv_lat, (float*)p.conv_state, dm.S,
+                                                              dm.Lq, dm.Lkv, dm.K);
   else
-    conv_state_kernel<float><<<dm.B, 256, 0, stream>>>((const float*)p.qkv_lat, (float*)p.conv_state, dm.S,
-                                                        dm.Lq, dm.Lkv, dm.K);
+    return cudaErrorInvalidValue;
   return cudaGetLastError();
 }
 

@@ -160,26 +160,32 @@ __global__ void __launch_bounds__(128) attention_simt_kernel(const T* __restrict
 
 }  // namespace
 
-cudaError_t launch_gemm_simt(bool in_bf16, bool out_bf16, const void* A, long long lda, const void* Bm,
-                             long long ldb, void* C, long long ldc, long long M, int N, int K,
-                             cudaStream_t stream) {
+namespace {
+template <typename Tin, typename Tout>
+void gemm_simt_typed(const void* A, long long lda, const void* Bm, long long ldb, void* C, long long ldc,
+                     long long M, int N, int K, dim3 grid, cudaStream_t stream) {
+  gemm_simt_kernel<Tin, Tout><<<grid, 256, 0, stream>>>((const Tin*)A, lda, (const Tin*)Bm, ldb, (Tout*)C, ldc, M,
+                                                         N, K);
+}
+template <typename Tin>
+void gemm_simt_out(DType out, const void* A, long long lda, const void* Bm, long long ldb, void* C, long long ldc,
+                   long long M, int N, int K, dim3 grid, cudaStream_t stream) {
+  switch (out) {
+    case DType::F32: gemm_simt_typed<Tin, float>(A, lda, Bm, ldb, C, ldc, M, N, K, grid, stream); break;
+    case DType::BF16: gemm_simt_typed<Tin, __nv_bfloat16>(A, lda, Bm, ldb, C, ldc, M, N, K, grid, stream); break;
+    case DType::F16: gemm_simt_typed<Tin, __half>(A, lda, Bm, ldb, C, ldc, M, N, K, grid, stream); break;
+  }
+}
+}  // namespace
+
+cudaError_t launch_gemm_simt(DType in, DType out, const void* A, long long lda, const void* Bm, long long ldb,
+                             void* C, long long ldc, long long M, int N, int K, cudaStream_t stream) {
   if (M <= 0 || N <= 0) return cudaSuccess;
   dim3 grid((N + GT_N - 1) / GT_N, (unsigned)((M + GT_M - 1) / GT_M));
-  if (in_bf16) {
-    using Ti = __nv_bfloat16;
-    if (out_bf16)
-      gemm_simt_kernel<Ti, __nv_bfloat16><<<grid, 256, 0, stream>>>((const Ti*)A, lda, (const Ti*)Bm, ldb,
-                                                                     (__nv_bfloat16*)C, ldc, M, N, K);
-    else
-      gemm_simt_kernel<Ti, float><<<grid, 256, 0, stream>>>((const Ti*)A, lda, (const Ti*)Bm, ldb, (float*)C,
-                                                             ldc, M, N, K);
-  } else {
-    if (out_bf16)
-      gemm_simt_kernel<float, __nv_bfloat16><<<grid, 256, 0, stream>>>((const float*)A, lda, (const float*)Bm,
-                                                                        ldb, (__nv_bfloat16*)C, ldc, M, N, K);
-    else
-      gemm_simt_kernel<float, float><<<grid, 256, 0, stream>>>((const float*)A, lda, (const float*)Bm, ldb,
-                                                                (float*)C, ldc, M, N, K);
+  switch (in) {
+    case DType::F32: gemm_simt_out<float>(out, A, lda, Bm, ldb, C, ldc, M, N, K, grid, stream); break;
+    case DType::BF16: gemm_simt_out<__nv_bfloat16>(out, A, lda, Bm, ldb, C, ldc, M, N, K, grid, stream); break;
+    case DType::F16: gemm_simt_out<__half>(out, A, lda, Bm, ldb, C, ldc, M, N, K, grid, stream); break;
   }
   return cudaGetLastError();
 }
@@ -191,19 +197,20 @@ cudaError_t launch_attention_simt(const BlockDims& dm, const void* q, const void
                                  (size_t)AT_Q * (AT_K + 1));
   dim3 grid((dm.S + AT_Q - 1) / AT_Q, dm.nq, dm.B);
   cudaError_t e;
-  if (dm.bf16) {
-    auto kern = attention_simt_kernel<__nv_bfloat16>;
+  if (dm.lat == DType::F16) {
+    auto kern = attention_simt_kernel<__half>;
     if ((e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem)) != cudaSuccess)
       return e;
-    kern<<<grid, 128, smem, stream>>>((const __nv_bfloat16*)q, (const __nv_bfloat16*)k,
-                                      (const __nv_bfloat16*)v, (__nv_bfloat16*)o, dm.S, dm.nq, dm.nkv, d,
-                                      dm.scale);
-  } else {
+    kern<<<grid, 128, smem, stream>>>((const __half*)q, (const __half*)k, (const __half*)v, (__half*)o, dm.S,
+                                      dm.nq, dm.nkv, d, dm.scale);
+  } else if (dm.lat == DType::F32) {
     auto kern = attention_simt_kernel<float>;
     if ((e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem)) != cudaSuccess)
       return e;
     kern<<<grid, 128, smem, stream>>>((const float*)q, (const float*)k, (const float*)v, (float*)o, dm.S, dm.nq,
                                       dm.nkv, d, dm.scale);
+  } else {
+    return cudaErrorInvalidValue;
   }
   return cudaGetLastError();
 }

@@ -50,12 +50,14 @@ typedef enum cca_status {
   CCA_ERR_UNSUPPORTED = 2,    /* valid block, but no kernel for this shape/dtype */
   CCA_ERR_WORKSPACE = 3,      /* workspace missing or smaller than cca_workspace_size */
   CCA_ERR_CUDA = 4,           /* a CUDA runtime call or launch failed */
-  CCA_ERR_DEVICE_TIMEOUT = 5  /* a bounded device-side wait gave up (see cca_poll_device_status) */
+  CCA_ERR_DEVICE_TIMEOUT = 5, /* a bounded device-side wait gave up (see cca_poll_device_status) */
+  CCA_ERR_NUMERIC_RANGE = 6   /* an fp16 intermediate overflowed (see cca_poll_device_status) */
 } cca_status_t;
 
 typedef enum cca_dtype {
   CCA_F32 = 0,   /* float32 */
-  CCA_BF16 = 1   /* bfloat16 */
+  CCA_BF16 = 1,  /* bfloat16 */
+  CCA_F16 = 2    /* float16: only as the type of bf16 blocks' intermediates */
 } cca_dtype_t;
 
 /* QK-mean mode bits (es 2.B item 2: the mean of q and k taken before and
@@ -82,14 +84,27 @@ typedef struct cca_config {
   int out_dtype;     /* cca_dtype_t of y (CCA_F32 allowed for bf16 inputs) */
 } cca_config_t;
 
-/* Kernel path selection (cca_prefill_ex). AUTO takes the tensor-core path
- * (tcgen05/TMEM, TMA) for bf16 with head_dim 128 and the SIMT path
- * otherwise. */
+/* Kernel path selection (cca_prefill_ex). AUTO runs each stage on its
+ * tensor-core kernel (tcgen05/TMEM fed by TMA, sm_100 only) when that kernel
+ * takes the shape (bf16; head_dim 128 for attention) and on its SIMT kernel
+ * otherwise. SIMT forces every stage onto the SIMT kernels; TENSOR requires
+ * the tensor-core kernels for both projections and attention. */
 typedef enum cca_path {
   CCA_PATH_AUTO = 0,
   CCA_PATH_SIMT = 1,
   CCA_PATH_TENSOR = 2   /* CCA_ERR_UNSUPPORTED if the shape does not allow it */
 } cca_path_t;
+/* Per-stage choice: bit0 down-projection, bit1 attention, bit2 output
+ * projection on the tensor-core kernel, the other stages on SIMT. */
+#define CCA_PATH_TENSOR_MASK(bits) (0x100 | ((bits) & 7))
+
+/* Which kernels a call would launch (cca_plan). */
+typedef struct cca_plan {
+  int down_proj_tensor;   /* 1: tcgen05 GEMM, 0: SIMT GEMM (three launches) */
+  int attention_tensor;   /* 1: tcgen05 flash attention, 0: SIMT attention */
+  int out_proj_tensor;    /* 1: tcgen05 GEMM, 0: SIMT GEMM */
+  int launches;           /* kernel launches of one cca_prefill without conv_state */
+} cca_plan_t;
 
 typedef struct cca_prefill_opts {
   int path;              /* cca_path_t */
@@ -100,14 +115,23 @@ typedef struct cca_prefill_opts {
 } cca_prefill_opts_t;
 
 /* Byte offsets of the intermediates inside the workspace, for inspection
- * after a call has completed. Each region is [T, width] row-major of the
- * element type `elem_bytes`, T = batch * seq_len. */
+ * after a call has completed. Each region is row-major of type lat_dtype,
+ * T = batch * seq_len. Intermediates of fp32 blocks are fp32; those of bf16
+ * blocks are fp16 (same tensor-core rate as bf16, 8x finer rounding), which
+ * keeps the block's chain of roundings small; inputs, the KV cache and y keep
+ * cfg->dtype / cfg->out_dtype. For fp32 blocks the k_att / v_att / W_o
+ * regions are empty (the attention reads the KV cache and W_o directly). */
 typedef struct cca_workspace_layout {
   size_t total_bytes;
-  size_t elem_bytes;        /* 4 for CCA_F32, 2 for CCA_BF16 */
+  size_t elem_bytes;        /* bytes per intermediate element */
+  int lat_dtype;            /* cca_dtype_t of the intermediates */
+  int reserved;
   size_t qkv_lat_offset;    /* [T, Lq + 2*Lkv]: q~ | k~ | v~ (down-projection) */
   size_t q_offset;          /* [T, Lq]: q after convs, QK-mean and RoPE */
+  size_t k_att_offset;      /* [T, Lkv]: k as the attention reads it */
+  size_t v_att_offset;      /* [T, Lkv]: v as the attention reads it */
   size_t o_offset;          /* [T, Lq]: attention output, heads concatenated */
+  size_t wo_offset;         /* [E, Lq]: W_o in the intermediate type */
   size_t sched_offset;      /* small scheduling scratch of the attention kernel */
 } cca_workspace_layout_t;
 
@@ -116,6 +140,9 @@ cca_status_t cca_validate(const cca_config_t* cfg);
 
 /* Workspace bytes that cca_prefill needs for cfg (0 if cfg is invalid). */
 size_t cca_workspace_size(const cca_config_t* cfg);
+
+/* Kernel choice of cca_prefill_ex(cfg, ..., path) on the current device. */
+cca_status_t cca_plan(const cca_config_t* cfg, int path, cca_plan_t* out);
 
 /* Fills *out with the workspace layout for cfg. */
 cca_status_t cca_workspace_layout(const cca_config_t* cfg, cca_workspace_layout_t* out);
@@ -187,7 +214,9 @@ cca_status_t cca_prefill_host(const cca_config_t* cfg,
 
 /* Synchronizes `stream`, then reports and clears the device error word:
  * CCA_ERR_DEVICE_TIMEOUT if a bounded wait in a kernel gave up since the last
- * poll, CCA_ERR_CUDA if the stream reports a CUDA error, else CCA_OK. */
+ * poll, CCA_ERR_NUMERIC_RANGE if a finite fp16 intermediate overflowed (its
+ * stored value is then +-inf), CCA_ERR_CUDA if the stream reports a CUDA
+ * error, else CCA_OK. */
 cca_status_t cca_poll_device_status(void* stream);
 
 /* Self-test of the bounded-wait machinery: launches one kernel that waits on

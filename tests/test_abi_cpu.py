@@ -30,7 +30,7 @@ def test_library_exports_every_declared_function():
 
 def test_struct_layouts():
     assert ctypes.sizeof(cca.CcaConfig) == 15 * 4
-    assert ctypes.sizeof(cca.CcaWorkspaceLayout) == 6 * 8
+    assert ctypes.sizeof(cca.CcaWorkspaceLayout) == 2 * 8 + 2 * 4 + 7 * 8
 
 
 def good(**kw):
@@ -44,15 +44,22 @@ def test_valid_configs_and_workspace():
     cfg = good()
     T, Lq, Lkv = 16384, 512, 256
     lay = cca.workspace_layout(cfg)
-    assert lay.elem_bytes == 2
+    assert lay.elem_bytes == 2 and lay.lat_dtype == cca.CCA_F16
     assert lay.q_offset >= T * (Lq + 2 * Lkv) * 2
-    assert lay.o_offset - lay.q_offset >= T * Lq * 2
+    assert lay.k_att_offset - lay.q_offset >= T * Lq * 2
+    assert lay.v_att_offset - lay.k_att_offset >= T * Lkv * 2
+    assert lay.o_offset - lay.v_att_offset >= T * Lkv * 2
+    assert lay.wo_offset - lay.o_offset >= T * Lq * 2
+    assert lay.sched_offset - lay.wo_offset >= 2048 * Lq * 2
     assert cca.workspace_size(cfg) == lay.total_bytes
-    for off in (lay.qkv_lat_offset, lay.q_offset, lay.o_offset, lay.sched_offset, lay.total_bytes):
+    for off in (lay.qkv_lat_offset, lay.q_offset, lay.k_att_offset, lay.v_att_offset, lay.o_offset,
+                lay.wo_offset, lay.sched_offset, lay.total_bytes):
         assert off % 256 == 0
     tiny = cca.make_config(batch=1, seq_len=64, hidden=128, n_q_heads=2, n_kv_heads=2, head_dim=16, dtype="f32")
     assert cca.validate(tiny) == cca.CCA_OK
-    assert cca.workspace_layout(tiny).elem_bytes == 4
+    lt = cca.workspace_layout(tiny)
+    assert lt.elem_bytes == 4 and lt.lat_dtype == cca.CCA_F32
+    assert lt.k_att_offset == lt.v_att_offset == lt.o_offset  # fp32 blocks read the cache directly
 
 
 @pytest.mark.parametrize("bad,code", [
@@ -78,6 +85,8 @@ def test_invalid_configs_rejected(bad, code):
 def test_bad_dtype_and_null_config():
     cfg = good()
     cfg.dtype = 7
+    assert cca.validate(cfg) == cca.CCA_ERR_INVALID_ARG
+    cfg.dtype = cca.CCA_F16  # fp16 is only an intermediate type
     assert cca.validate(cfg) == cca.CCA_ERR_INVALID_ARG
     lib = cca.library()
     assert lib.cca_validate(None) == cca.CCA_ERR_INVALID_ARG

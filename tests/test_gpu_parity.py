@@ -10,7 +10,7 @@ from parity import assert_close, run_gpu, run_oracle, sample_rows
 
 pytestmark = pytest.mark.gpu
 
-SIMT, TENSOR = cca.CCA_PATH_SIMT, cca.CCA_PATH_TENSOR
+SIMT, AUTO, TENSOR = cca.CCA_PATH_SIMT, cca.CCA_PATH_AUTO, cca.CCA_PATH_TENSOR
 
 
 def shape(**kw):
@@ -32,6 +32,9 @@ def check_all(sh, gpu, ref, stages=True):
         assert_close("k_lat", lat[..., lq:lq + lkv], ref["k_lat"], dt)
         assert_close("v_lat", lat[..., lq + lkv:], ref["v_lat"], dt)
         assert_close("q", gpu["q"], ref["q"], dt)
+        if "k_att" in gpu:
+            assert_close("k_att", gpu["k_att"], ref["k_cache"].reshape(gpu["k_att"].shape), dt)
+            assert_close("v_att", gpu["v_att"], ref["v_cache"].reshape(gpu["v_att"].shape), dt)
         assert_close("o", gpu["o"], ref["o"], dt)
     return assert_close("y", gpu["y"], ref["y"], dt)
 
@@ -63,7 +66,7 @@ BF16_CASES = [
 ]
 
 
-@pytest.mark.parametrize("path", [SIMT, TENSOR], ids=["simt", "tensor"])
+@pytest.mark.parametrize("path", [SIMT, AUTO, TENSOR], ids=["simt", "auto", "tensor"])
 @pytest.mark.parametrize("case", range(len(BF16_CASES)))
 def test_bf16_small(path, case):
     sh = shape(**BF16_CASES[case])
@@ -71,7 +74,7 @@ def test_bf16_small(path, case):
     check_all(sh, run_gpu(sh, inp, path=path), run_oracle(sh, inp))
 
 
-@pytest.mark.parametrize("path", [SIMT, TENSOR], ids=["simt", "tensor"])
+@pytest.mark.parametrize("path", [SIMT, AUTO, TENSOR], ids=["simt", "auto", "tensor"])
 @pytest.mark.parametrize("mode,vshift,rope", [(0, 0, 0), (1, 0, 1), (2, 1, 0), (3, 1, 1), (0, 1, 1)])
 def test_bf16_modes(path, mode, vshift, rope):
     sh = shape(seq_len=257, qk_mean_mode=mode, value_shift=vshift, use_rope=rope, batch=2)
@@ -79,7 +82,7 @@ def test_bf16_modes(path, mode, vshift, rope):
     check_all(sh, run_gpu(sh, inp, path=path), run_oracle(sh, inp))
 
 
-@pytest.mark.parametrize("path", [SIMT, TENSOR], ids=["simt", "tensor"])
+@pytest.mark.parametrize("path", [SIMT, AUTO, TENSOR], ids=["simt", "auto", "tensor"])
 def test_fp32_output_and_conv_state(path):
     sh = shape(seq_len=190, batch=2)
     inp = workloads.make_inputs(sh)
@@ -100,7 +103,7 @@ def test_fp32_output_and_conv_state(path):
     np.testing.assert_array_equal(cs[:, :nq_part].reshape(2, K - 1, lq), lat[:, -(K - 1):, :lq])
 
 
-@pytest.mark.parametrize("path", [SIMT, TENSOR], ids=["simt", "tensor"])
+@pytest.mark.parametrize("path", [SIMT, AUTO, TENSOR], ids=["simt", "auto", "tensor"])
 def test_deterministic_and_causal(path):
     """Three runs are bit-identical; perturbing x[t0] leaves every output row
     before t0 bit-identical (nothing reads the future)."""
