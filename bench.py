@@ -388,7 +388,8 @@ def run_ours(args, shape):
 
 def plan_name(plan):
     k = lambda b: "tcgen05" if b else "simt"  # noqa: E731
-    return (f"down_proj={k(plan['down_proj_tensor'])},attention={k(plan['attention_tensor'])},"
+    return (f"down_proj={k(plan['down_proj_tensor'])},"
+            f"preproc={'mma' if plan['preproc_tensor'] else 'simt'},attention={k(plan['attention_tensor'])},"
             f"out_proj={k(plan['out_proj_tensor'])}")
 
 

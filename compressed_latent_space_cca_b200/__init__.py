@@ -97,7 +97,8 @@ def plan(cfg: CcaConfig, path: int = CCA_PATH_AUTO) -> dict:
     if st != CCA_OK:
         raise CcaError(st, "cca_plan")
     return {"down_proj_tensor": bool(out.down_proj_tensor), "attention_tensor": bool(out.attention_tensor),
-            "out_proj_tensor": bool(out.out_proj_tensor), "launches": out.launches}
+            "out_proj_tensor": bool(out.out_proj_tensor), "preproc_tensor": bool(out.preproc_tensor),
+            "launches": out.launches}
 
 
 def _shapes(cfg: CcaConfig) -> Dict[str, tuple]:

@@ -25,8 +25,8 @@ CCA_PATH_TENSOR = 2
 
 
 def CCA_PATH_TENSOR_MASK(bits: int) -> int:
-    """bit0 down-projection, bit1 attention, bit2 output projection on tcgen05."""
-    return 0x100 | (bits & 7)
+    """bit0 down-projection, bit1 attention, bit2 output projection, bit3 preprocessing."""
+    return 0x100 | (bits & 15)
 
 
 class CcaConfig(Structure):
@@ -71,7 +71,7 @@ class CcaWorkspaceLayout(Structure):
 
 class CcaPlan(Structure):
     _fields_ = [("down_proj_tensor", c_int), ("attention_tensor", c_int), ("out_proj_tensor", c_int),
-                ("launches", c_int)]
+                ("preproc_tensor", c_int), ("launches", c_int)]
 
 
 _PREFILL_ARGS = [POINTER(CcaConfig)] + [c_void_p] * 9 + [c_void_p] * 4 + [c_void_p, c_size_t, c_void_p]

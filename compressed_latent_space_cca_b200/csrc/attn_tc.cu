@@ -109,8 +109,7 @@ __global__ void __launch_bounds__(NUM_THREADS, 1) attn_tc_kernel(const __grid_co
   uint64_t* s_full = v_empty + KV_STAGES;  // [2]
   uint64_t* p_full = s_full + 2;           // [2]
   uint64_t* o_full = p_full + 2;           // [2]
-  uint64_t* o_empty = o_full + 2;          // [2]
-  uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(o_empty + 2);
+  uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(o_full + 2);
   volatile int* abort_flag = reinterpret_cast<volatile int*>(tmem_slot + 1);
 
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
@@ -127,7 +126,6 @@ __global__ void __launch_bounds__(NUM_THREADS, 1) attn_tc_kernel(const __grid_co
       mbar_init(smem_u32(&s_full[j]), 1);
       mbar_init(smem_u32(&p_full[j]), 4);
       mbar_init(smem_u32(&o_full[j]), 1);
-      mbar_init(smem_u32(&o_empty[j]), 4);
     }
     *abort_flag = 0;
     fence_mbar_init();
@@ -197,8 +195,8 @@ __global__ void __launch_bounds__(NUM_THREADS, 1) attn_tc_kernel(const __grid_co
         if (w >= p.items) break;
         const Item it = get_item(p, w);
         if (!mbar_wait_bounded(smem_u32(q_full), r & 1, p.err, abort_flag, wait_site(kSiteAttn, 2, 4))) goto done;
-        for (int j = 0; j < 2; ++j)
-          if (!mbar_wait_bounded(smem_u32(&o_empty[j]), (r & 1) ^ 1, p.err, abort_flag, wait_site(kSiteAttn, 2, 5))) goto done;
+        // O_j of the previous pair needs no guard: the first PV of this pair waits for p_full[j],
+        // which the softmax group raises only after its epilogue has read O_j back.
         tc_fence_after();
         const uint32_t q_base[2] = {smem_u32(smem + OFF_Q), smem_u32(smem + OFF_Q + TILE_BYTES)};
         auto issue_qk = [&](int j, int st) {
@@ -364,8 +362,6 @@ __global__ void __launch_bounds__(NUM_THREADS, 1) attn_tc_kernel(const __grid_co
         }
         tc_fence_before();
       }
-      __syncwarp();
-      if (lane == 0) mbar_arrive(smem_u32(&o_empty[j]));
     }
   }
 done:

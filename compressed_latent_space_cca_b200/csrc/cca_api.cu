@@ -145,6 +145,7 @@ bool aligned16(const void* p) { return (reinterpret_cast<uintptr_t>(p) & 15u) ==
 struct Resolved {
   BlockDims dm;
   bool tc_down, tc_attn, tc_out;  // tcgen05 kernels per stage
+  bool tc_pre;                    // tensor-core preprocessing kernel
 };
 
 cca_status_t resolve(const cca_config_t* cfg, int path, Resolved* r) {
@@ -153,7 +154,7 @@ cca_status_t resolve(const cca_config_t* cfg, int path, Resolved* r) {
   DeviceInfo* di = nullptr;
   if ((st = device_info(&di)) != CCA_OK) return st;
   const BlockDims& dm = r->dm;
-  const bool masked = (path & ~7) == CCA_PATH_TENSOR_MASK(0);
+  const bool masked = (path & ~15) == CCA_PATH_TENSOR_MASK(0);
   if (path != CCA_PATH_AUTO && path != CCA_PATH_SIMT && path != CCA_PATH_TENSOR && !masked)
     return fail(CCA_ERR_INVALID_ARG, "unknown path");
   const bool sm100 = di->major == 10;
@@ -162,14 +163,16 @@ cca_status_t resolve(const cca_config_t* cfg, int path, Resolved* r) {
                     dm.Lkv % 128 == 0;
   const bool attn = sm100 && b16 && dm.d == 128 && attention_tc_supported(dm);
   const bool out = sm100 && b16 && gemm_tc_supported(dm.T, dm.E, dm.Lq);
-  if (path == CCA_PATH_TENSOR && !(down && attn && out))
+  const bool pre = preproc_tc_supported(dm);
+  if (path == CCA_PATH_TENSOR && !(down && attn && out && pre))
     return fail(CCA_ERR_UNSUPPORTED, "tensor-core path needs sm_100, bf16, head_dim 128 and 128-aligned widths");
-  if (masked && (((path & 1) && !down) || ((path & 2) && !attn) || ((path & 4) && !out)))
+  if (masked && (((path & 1) && !down) || ((path & 2) && !attn) || ((path & 4) && !out) || ((path & 8) && !pre)))
     return fail(CCA_ERR_UNSUPPORTED, "a stage asked for the tensor-core kernel cannot use it");
   const bool use = path != CCA_PATH_SIMT;
   r->tc_down = masked ? (path & 1) != 0 : use && down;
   r->tc_attn = masked ? (path & 2) != 0 : use && attn;
   r->tc_out = masked ? (path & 4) != 0 : use && out;
+  r->tc_pre = masked ? (path & 8) != 0 : use && pre;
   return CCA_OK;
 }
 
@@ -222,7 +225,11 @@ cca_status_t run_block(const Resolved& r, BlockPtrs p, cudaStream_t stream, void
   }
   if ((e = mark(1)) != cudaSuccess) return cuda_fail("event", e);
   // 2. seq conv, channel conv, QK-mean, RoPE, value shift; KV cache written here
-  if ((e = launch_preproc_simt(dm, p, stream)) != cudaSuccess) return cuda_fail("preprocessing", e);
+  if (r.tc_pre) {
+    if ((e = launch_preproc_tc(dm, p, stream)) != cudaSuccess) return cuda_fail("preprocessing (mma)", e);
+  } else {
+    if ((e = launch_preproc_simt(dm, p, stream)) != cudaSuccess) return cuda_fail("preprocessing (SIMT)", e);
+  }
   if ((e = launch_conv_state(dm, p, stream)) != cudaSuccess) return cuda_fail("conv state", e);
   if ((e = mark(2)) != cudaSuccess) return cuda_fail("event", e);
   // 3. causal attention on the compressed heads
@@ -393,6 +400,7 @@ cca_status_t cca_plan(const cca_config_t* cfg, int path, cca_plan_t* out) {
   out->down_proj_tensor = r.tc_down;
   out->attention_tensor = r.tc_attn;
   out->out_proj_tensor = r.tc_out;
+  out->preproc_tensor = r.tc_pre;
   out->launches = (r.tc_down ? 1 : 3) + 1 + 1 + 1;
   return CCA_OK;
 }

@@ -86,23 +86,25 @@ typedef struct cca_config {
 
 /* Kernel path selection (cca_prefill_ex). AUTO runs each stage on its
  * tensor-core kernel (tcgen05/TMEM fed by TMA, sm_100 only) when that kernel
- * takes the shape (bf16; head_dim 128 for attention) and on its SIMT kernel
- * otherwise. SIMT forces every stage onto the SIMT kernels; TENSOR requires
- * the tensor-core kernels for both projections and attention. */
+ * takes the shape (bf16; head_dim 128 for attention and preprocessing) and on
+ * its SIMT kernel otherwise. SIMT forces every stage onto the SIMT kernels;
+ * TENSOR requires the tensor-core kernels for every stage. */
 typedef enum cca_path {
   CCA_PATH_AUTO = 0,
   CCA_PATH_SIMT = 1,
   CCA_PATH_TENSOR = 2   /* CCA_ERR_UNSUPPORTED if the shape does not allow it */
 } cca_path_t;
 /* Per-stage choice: bit0 down-projection, bit1 attention, bit2 output
- * projection on the tensor-core kernel, the other stages on SIMT. */
-#define CCA_PATH_TENSOR_MASK(bits) (0x100 | ((bits) & 7))
+ * projection, bit3 preprocessing on the tensor-core kernel, the other stages
+ * on SIMT. */
+#define CCA_PATH_TENSOR_MASK(bits) (0x100 | ((bits) & 15))
 
 /* Which kernels a call would launch (cca_plan). */
 typedef struct cca_plan {
   int down_proj_tensor;   /* 1: tcgen05 GEMM, 0: SIMT GEMM (three launches) */
   int attention_tensor;   /* 1: tcgen05 flash attention, 0: SIMT attention */
   int out_proj_tensor;    /* 1: tcgen05 GEMM, 0: SIMT GEMM */
+  int preproc_tensor;     /* 1: preprocessing with the channel mix on tensor cores (mma.sync) */
   int launches;           /* kernel launches of one cca_prefill without conv_state */
 } cca_plan_t;
 

@@ -98,9 +98,9 @@ def test_fp32_output_and_conv_state(path):
                                rtol=1e-2, atol=1e-2)
     np.testing.assert_allclose(cs[:, nq_part + (K - 1) * lkv:].reshape(2, 1, lkv), ref["conv_state_v"],
                                rtol=1e-2, atol=1e-2)
-    # the conv state is a copy of the workspace latents: exact
-    lat = gpu["qkv_lat"]
-    np.testing.assert_array_equal(cs[:, :nq_part].reshape(2, K - 1, lq), lat[:, -(K - 1):, :lq])
+    # the conv state is the workspace latents converted to the block dtype: exact
+    lat = torch.from_numpy(gpu["qkv_lat"][:, -(K - 1):, :lq]).to(torch.bfloat16).double().numpy()
+    np.testing.assert_array_equal(cs[:, :nq_part].reshape(2, K - 1, lq), lat)
 
 
 @pytest.mark.parametrize("path", [SIMT, AUTO, TENSOR], ids=["simt", "auto", "tensor"])
