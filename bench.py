@@ -320,7 +320,10 @@ def run_ours(args, shape):
     work = algorithmic_work(my_shape)
 
     # end to end: x from pinned host memory, y back to pinned host memory, one C call per step
-    x_host = inputs_cpu["x"].pin_memory()
+    e2e = None
+    if not args.no_e2e:
+        e2e = run_e2e(cca, cfg, args, inputs_cpu, inputs, out, ws, stream, my_shape, world, barrier, reduce_max)
+    _unused = 
     y_host = torch.empty(tuple(out["y"].shape), dtype=out["y"].dtype).pin_memory()
     x_dev = torch.empty_like(inputs["x"])
     weights = {k: v for k, v in inputs.items() if k != "x"}
@@ -371,9 +374,7 @@ def run_ours(args, shape):
             "attention_tflops": attn_tflops,
             "roofline": roofline,
             "kernels": kernels,
-            "e2e": {"value": e2e_val, "unit": "tokens/s",
-                    "h2d_bytes_per_step": int(x_host.numel() * x_host.element_size()),
-                    "d2h_bytes_per_step": int(y_host.numel() * y_host.element_size())},
+            "e2e": e2e,
             "gpu_launches": launches_per_step * args.steps,
             "clocks": clocks,
         }
@@ -384,6 +385,31 @@ def run_ours(args, shape):
         dist.barrier()
         dist.destroy_process_group()
     return 0
+
+
+def run_e2e(cca, cfg, args, inputs_cpu, inputs, out, ws, stream, shape, world, barrier, reduce_max):
+    """Same metric through cca_prefill_host: x from pinned host memory, y back to
+    pinned host memory inside the timed region (the KV cache stays on the device)."""
+    x_host = inputs_cpu["x"].pin_memory()
+    y_host = torch.empty(tuple(out["y"].shape), dtype=out["y"].dtype).pin_memory()
+    x_dev = torch.empty_like(inputs["x"])
+    weights = {k: v for k, v in inputs.items() if k != "x"}
+    steps = max(3, min(args.steps, 20))
+    for _ in range(2):
+        cca.prefill_host(cfg, x_host, weights, x_dev, out["y"], y_host, out["k_cache"], out["v_cache"], ws)
+    torch.cuda.synchronize()
+    barrier()
+    e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    e0.record(stream)
+    for _ in range(steps):
+        cca.prefill_host(cfg, x_host, weights, x_dev, out["y"], y_host, out["k_cache"], out["v_cache"], ws)
+    e1.record(stream)
+    torch.cuda.synchronize()
+    barrier()
+    value, _ = aggregate(e0.elapsed_time(e1), shape.tokens, steps, world, reduce_max)
+    return {"value": value, "unit": "tokens/s", "steps": steps,
+            "h2d_bytes_per_step": int(x_host.numel() * x_host.element_size()),
+            "d2h_bytes_per_step": int(y_host.numel() * y_host.element_size())}
 
 
 def plan_name(plan):
@@ -401,10 +427,16 @@ def main(argv=None):
     ap.add_argument("--impl", choices=["ours", "reference"], default="ours")
     ap.add_argument("--workload", default=DEFAULT_WORKLOAD, choices=sorted(workloads.WORKLOADS))
     ap.add_argument("--no-cpu-baseline", action="store_true", help="skip the oracle timing (rank 0, N=1)")
+    ap.add_argument("--no-e2e", action="store_true", help="skip the host-buffer end-to-end timing")
+    ap.add_argument("--batch", type=int, default=None, help="override the workload's batch (profiling cases)")
+    ap.add_argument("--seq-len", type=int, default=None, help="override the workload's sequence length")
     args = ap.parse_args(argv)
     if args.warmup < 3:
         raise SystemExit("--warmup must be >= 3")
     shape = workloads.WORKLOADS[args.workload]
+    if args.batch is not None or args.seq_len is not None:
+        shape = shape.replace(batch=args.batch or shape.batch, seq_len=args.seq_len or shape.seq_len,
+                              name=f"{shape.name}(B={args.batch or shape.batch},S={args.seq_len or shape.seq_len})")
     if args.impl == "reference":
         return run_reference(args, shape)
     return run_ours(args, shape)
