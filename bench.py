@@ -323,23 +323,6 @@ def run_ours(args, shape):
     e2e = None
     if not args.no_e2e:
         e2e = run_e2e(cca, cfg, args, inputs_cpu, inputs, out, ws, stream, my_shape, world, barrier, reduce_max)
-    _unused = 
-    y_host = torch.empty(tuple(out["y"].shape), dtype=out["y"].dtype).pin_memory()
-    x_dev = torch.empty_like(inputs["x"])
-    weights = {k: v for k, v in inputs.items() if k != "x"}
-    e2e_steps = max(3, min(args.steps, 20))
-    for _ in range(2):
-        cca.prefill_host(cfg, x_host, weights, x_dev, out["y"], y_host, out["k_cache"], out["v_cache"], ws)
-    torch.cuda.synchronize()
-    barrier()
-    e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
-    e0.record(stream)
-    for _ in range(e2e_steps):
-        cca.prefill_host(cfg, x_host, weights, x_dev, out["y"], y_host, out["k_cache"], out["v_cache"], ws)
-    e1.record(stream)
-    torch.cuda.synchronize()
-    barrier()
-    e2e_val, _ = aggregate(e0.elapsed_time(e1), my_shape.tokens, e2e_steps, world, reduce_max)
 
     peaks, peak_src = load_peaks()
     attn_s = stage_ms[2] / 1e3
