@@ -188,7 +188,11 @@ def oracle_sample_text(shape):
 
 
 def oracle_extrapolate(times_by_rows, S):
+    """Full-block time from two row counts (linear in the rows evaluated). When the
+    sequence is shorter than the samples both calls already ran the full block."""
     (r1, t1), (r2, t2) = times_by_rows
+    if r2 <= r1:
+        return 0.5 * (t1 + t2)
     per_row = max(0.0, (t2 - t1) / (r2 - r1))
     return t1 + per_row * (S - r1)
 

@@ -48,6 +48,22 @@ constexpr int OFF_V = OFF_K + KV_STAGES * TILE_BYTES;
 constexpr int OFF_BAR = OFF_V + KV_STAGES * TILE_BYTES;
 constexpr size_t SMEM_BYTES = OFF_BAR + 256 + 1024;
 
+// 2^x on the FMA and integer pipes, for x in [-inf, 126]: x = n + f with
+// n = round(x) (found by adding 1.5 * 2^23, which leaves n in the low
+// mantissa bits) and |f| <= 1/2; 2^f from a cubic fitted to 2^f on
+// [-1/2, 1/2] by iteratively reweighted least squares (max relative error
+// 1.0e-4, below the fp16 rounding of P); 2^n is added to the exponent field.
+// Used for a share of the probabilities so that the special-function unit,
+// which the tensor core otherwise waits on, is not the only exp2 source.
+__device__ __forceinline__ float exp2_fma(float x) {
+  x = fmaxf(x, -126.0f);
+  const float t = x + 12582912.0f;
+  const float f = x - (t - 12582912.0f);
+  const float p = fmaf(fmaf(fmaf(0.05500893f, f, 0.24221097f), f, 0.69328290f), f, 1.0f);
+  return __int_as_float(__float_as_int(p) + (__float_as_int(t) << 23));
+}
+constexpr int POLY_EVERY = 4;  // one pair in POLY_EVERY takes exp2_fma
+
 struct AttnMaps {
   CUtensorMap q, k, v;
 };
@@ -310,8 +326,10 @@ __global__ void __launch_bounds__(NUM_THREADS, 1) attn_tc_kernel(const __grid_co
             uint32_t pk[32];
 #pragma unroll
             for (int e = 0; e < 32; ++e) {
-              const float p0 = fast_exp2(u2f(s[c2 * 64 + 2 * e]) - m);
-              const float p1 = fast_exp2(u2f(s[c2 * 64 + 2 * e + 1]) - m);
+              const bool poly = (e % POLY_EVERY) == POLY_EVERY - 1;
+              const float x0 = u2f(s[c2 * 64 + 2 * e]) - m, x1 = u2f(s[c2 * 64 + 2 * e + 1]) - m;
+              const float p0 = poly ? exp2_fma(x0) : fast_exp2(x0);
+              const float p1 = poly ? exp2_fma(x1) : fast_exp2(x1);
               sum += p0 + p1;
               pk[e] = pack_f16x2(p0, p1);
             }

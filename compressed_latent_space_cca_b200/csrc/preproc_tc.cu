@@ -10,17 +10,20 @@
 // shifted by one token).
 //
 // One CTA = 32 tokens of one sequence x one KV group (its G query heads and
-// its K/V head). Per head: the fp16 latents of the 32 tokens plus a K-1
-// token halo are staged in shared memory, the causal seq conv runs on CUDA
-// cores in fp32 and writes an fp16 tile, and the 32x128x128 channel mix runs
-// on the tensor cores (mma.sync m16n8k16, fp16 x fp16 -> fp32) against the
-// head's weights, converted from bf16 to fp16 while staged. Each thread owns
-// the same accumulator positions for every head, so the cross-head QK-mean
-// sums stay in registers, and since its columns come in pairs (c, c+64) RoPE
-// is applied in registers too. Output tiles are staged in shared memory and
-// written with 16-byte coalesced stores: q (fp16), the bf16 K cache and the
-// fp16 attention copy of k; then the value shift copies v (bf16 cache and
-// fp16 attention copy).
+// its K/V head). The fp16 latents of all G+1 heads (32 tokens plus a K-1
+// token halo) arrive in shared memory by cp.async. Per head, the head's bf16
+// channel-mix weights stream in by cp.async, the causal seq conv runs on CUDA
+// cores in fp32, and its output s is split into bf16 s_hi + s_lo so that the
+// 32x128x128 channel mix runs on the tensor cores (mma.sync m16n8k16 bf16,
+// fp32 accumulate, two products per step) on the exact bf16 weights with a
+// relative error near 2^-18. Each thread owns the same accumulator positions
+// for every head, so c_k and the sum of the c_q stay in registers, and its
+// columns come in pairs (c, c+64), so RoPE is applied in registers. Output
+// tiles are staged in shared memory and written with 16-byte coalesced
+// stores: q (fp16), the bf16 K cache and the fp16 attention copy of k; then
+// the value shift copies v (bf16 cache and fp16 attention copy). Every
+// shared-memory row is padded to 272 bytes, which keeps ldmatrix, the
+// per-thread reads and the staging stores free of bank conflicts.
 #include <math.h>
 
 #include "cca_common.cuh"
@@ -33,25 +36,35 @@ constexpr int D = 128;
 constexpr int TT = 32;          // tokens per CTA
 constexpr int NT = 256;         // threads
 constexpr int KMAX = 8;         // largest seq-conv kernel of this path
-constexpr int ROWH = D + 8;     // padded row (halves) of the MMA operand tiles: 272 B, ldmatrix conflict-free
+constexpr int GMAX = 8;         // largest group (query heads per KV head) of this path
+constexpr int ROWH = D + 8;     // padded row, in 16-bit elements (272 bytes)
 constexpr int ZROWS = TT + KMAX - 1;
+constexpr int KSTR = D + 4;     // padded fp32 row of the k stage
 
 struct Theta {
   double v[D / 2];  // base^(-2i/d)
 };
 
 struct PreParams {
-  const __half* lat;       // [T, Nlat] q~ | k~ | v~
+  const __half* lat;  // [T, Nlat] q~ | k~ | v~
   const __nv_bfloat16 *cq_seq, *cq_chan, *ck_seq, *ck_chan;
-  __half* q;               // [T, Lq]
-  __nv_bfloat16 *k_cache, *v_cache;  // [T, Lkv]
-  __half *k_att, *v_att;   // [T, Lkv]
-  const __nv_bfloat16* wo;  // [E, Lq] (converted by a side job)
+  __half* q;                          // [T, Lq]
+  __nv_bfloat16 *k_cache, *v_cache;   // [T, Lkv]
+  __half *k_att, *v_att;              // [T, Lkv]
+  const __nv_bfloat16* wo;            // [E, Lq] (converted by a side job)
   __half* wo_lat;
   long long wo_n;
   unsigned* err;
   int S, nq, nkv, K, mode, vshift, use_rope;
 };
+
+__device__ __forceinline__ void cp_async16(uint32_t dst, const void* src, bool valid) {
+  const int n = valid ? 16 : 0;  // 0 source bytes: the 16 destination bytes are zero-filled
+  asm volatile("cp.async.cg.shared.global [%0], [%1], 16, %2;" ::"r"(dst), "l"(src), "r"(n) : "memory");
+}
+__device__ __forceinline__ void cp_async_wait_all() {
+  asm volatile("cp.async.commit_group;\ncp.async.wait_group 0;" ::: "memory");
+}
 
 __device__ __forceinline__ void ldsm_x4(uint32_t addr, uint32_t& r0, uint32_t& r1, uint32_t& r2, uint32_t& r3) {
   asm volatile("ldmatrix.sync.aligned.m8n8.x4.shared.b16 {%0,%1,%2,%3}, [%4];"
@@ -59,49 +72,18 @@ __device__ __forceinline__ void ldsm_x4(uint32_t addr, uint32_t& r0, uint32_t& r
                : "r"(addr));
 }
 
-__device__ __forceinline__ void mma_f16_16816(float* c, uint32_t a0, uint32_t a1, uint32_t a2, uint32_t a3,
-                                              uint32_t b0, uint32_t b1) {
+__device__ __forceinline__ void mma_bf16_16816(float* c, uint32_t a0, uint32_t a1, uint32_t a2, uint32_t a3,
+                                               uint32_t b0, uint32_t b1) {
   asm volatile(
-      "mma.sync.aligned.m16n8k16.row.col.f32.f16.f16.f32 {%0,%1,%2,%3}, {%4,%5,%6,%7}, {%8,%9}, "
+      "mma.sync.aligned.m16n8k16.row.col.f32.bf16.bf16.f32 {%0,%1,%2,%3}, {%4,%5,%6,%7}, {%8,%9}, "
       "{%0,%1,%2,%3};"
       : "+f"(c[0]), "+f"(c[1]), "+f"(c[2]), "+f"(c[3])
       : "r"(a0), "r"(a1), "r"(a2), "r"(a3), "r"(b0), "r"(b1));
 }
 
-// Stage the latents of one head (rows t0-K+1 .. t0+TT-1, zero outside the
-// sequence) into zbuf [ZROWS][D] fp16.
-__device__ __forceinline__ void load_latents(const PreParams& p, __half* zbuf, long long rowbase, int t0, int col,
-                                             int Nlat) {
-  const int rows = TT + p.K - 1;
-  for (int e = threadIdx.x; e < rows * (D / 8); e += NT) {
-    const int r = e / (D / 8), v = e % (D / 8);
-    const int t = t0 - (p.K - 1) + r;
-    uint4 val = make_uint4(0, 0, 0, 0);
-    if (t >= 0 && t < p.S) val = *reinterpret_cast<const uint4*>(p.lat + (rowbase + t) * Nlat + col + v * 8);
-    *reinterpret_cast<uint4*>(zbuf + r * D + v * 8) = val;
-  }
-}
-
-// Stage one head's channel-mix weights [out i][in j] (bf16) as fp16 rows of ROWH.
-__device__ __forceinline__ void load_weights(const __nv_bfloat16* W, __half* wbuf, bool& bad) {
-  for (int e = threadIdx.x; e < D * (D / 8); e += NT) {
-    const int r = e / (D / 8), v = e % (D / 8);
-    const uint4 raw = *reinterpret_cast<const uint4*>(W + (long long)r * D + v * 8);
-    const __nv_bfloat162* b2 = reinterpret_cast<const __nv_bfloat162*>(&raw);
-    uint32_t h[4];
-#pragma unroll
-    for (int k = 0; k < 4; ++k) {
-      const float2 f = __bfloat1622float2(b2[k]);
-      bad |= f16_overflow(f.x) || f16_overflow(f.y);
-      h[k] = pack_f16x2(f.x, f.y);
-    }
-    *reinterpret_cast<uint4*>(wbuf + r * ROWH + v * 8) = make_uint4(h[0], h[1], h[2], h[3]);
-  }
-}
-
-// Causal depthwise seq conv of the staged head into sbuf [TT][ROWH] fp16.
-__device__ __forceinline__ void seq_conv(const PreParams& p, const __half* zbuf, __half* sbuf,
-                                         const __nv_bfloat16* wseq) {
+// Causal depthwise seq conv of one staged head into the bf16 hi / lo tiles.
+__device__ __forceinline__ void seq_conv(const PreParams& p, const __half* zbuf, __nv_bfloat16* shi,
+                                         __nv_bfloat16* slo, const __nv_bfloat16* wseq) {
   const int cp = threadIdx.x % (D / 2);  // column pair
   float w0[KMAX], w1[KMAX];
 #pragma unroll
@@ -114,63 +96,72 @@ __device__ __forceinline__ void seq_conv(const PreParams& p, const __half* zbuf,
 #pragma unroll
     for (int j = 0; j < KMAX; ++j) {
       if (j < p.K) {
-        const float2 z = __half22float2(*reinterpret_cast<const __half2*>(zbuf + (t + j) * D + 2 * cp));
+        const float2 z = __half22float2(*reinterpret_cast<const __half2*>(zbuf + (t + j) * ROWH + 2 * cp));
         a0 = fmaf(w0[j], z.x, a0);
         a1 = fmaf(w1[j], z.y, a1);
       }
     }
-    *reinterpret_cast<__half2*>(sbuf + t * ROWH + 2 * cp) = __floats2half2_rn(a0, a1);
+    const __nv_bfloat162 hi = __floats2bfloat162_rn(a0, a1);
+    const float2 hf = __bfloat1622float2(hi);
+    *reinterpret_cast<__nv_bfloat162*>(shi + t * ROWH + 2 * cp) = hi;
+    *reinterpret_cast<__nv_bfloat162*>(slo + t * ROWH + 2 * cp) = __floats2bfloat162_rn(a0 - hf.x, a1 - hf.y);
   }
 }
 
-// Channel mix of the warp's 16 rows x 4 n-tiles: acc[nt][0..3] (m16n8 layout).
-__device__ __forceinline__ void channel_mix(const __half* sbuf, const __half* wbuf, int rb, const int* ncol,
+// Channel mix of the warp's 16 rows x 4 n-tiles: acc[nt][0..3] (m16n8 layout),
+// acc = (s_hi + s_lo) W^T.
+__device__ __forceinline__ void channel_mix(const __nv_bfloat16* shi, const __nv_bfloat16* slo,
+                                            const __nv_bfloat16* wbuf, int rb, const int* ncol,
                                             float (&acc)[4][4]) {
   const int lane = threadIdx.x & 31;
 #pragma unroll
   for (int nt = 0; nt < 4; ++nt)
 #pragma unroll
     for (int e = 0; e < 4; ++e) acc[nt][e] = 0.f;
-  // ldmatrix addresses: A rows rb + (lane % 16), column block (lane / 16) * 8
-  const uint32_t a_base = smem_u32(sbuf + (rb + (lane & 15)) * ROWH + (lane >> 4) * 8);
-  // B x4 covers two n-tiles: matrix m = lane / 8 -> n offset (m / 2) * 8, k offset (m % 2) * 8
+  const int arow = (rb + (lane & 15)) * ROWH + (lane >> 4) * 8;
+  const uint32_t ahi = smem_u32(shi + arow), alo = smem_u32(slo + arow);
   const int m = lane >> 3, rr = lane & 7;
-  const uint32_t b_base0 = smem_u32(wbuf + (ncol[0] + (m >> 1) * 8 + rr) * ROWH + (m & 1) * 8);
-  const uint32_t b_base1 = smem_u32(wbuf + (ncol[2] + (m >> 1) * 8 + rr) * ROWH + (m & 1) * 8);
+  const uint32_t b0base = smem_u32(wbuf + (ncol[0] + (m >> 1) * 8 + rr) * ROWH + (m & 1) * 8);
+  const uint32_t b1base = smem_u32(wbuf + (ncol[2] + (m >> 1) * 8 + rr) * ROWH + (m & 1) * 8);
 #pragma unroll
   for (int ks = 0; ks < D / 16; ++ks) {
-    uint32_t a0, a1, a2, a3, b0, b1, b2, b3, c0, c1, c2, c3;
-    ldsm_x4(a_base + ks * 32, a0, a1, a2, a3);
-    ldsm_x4(b_base0 + ks * 32, b0, b1, b2, b3);
-    ldsm_x4(b_base1 + ks * 32, c0, c1, c2, c3);
-    mma_f16_16816(acc[0], a0, a1, a2, a3, b0, b1);
-    mma_f16_16816(acc[1], a0, a1, a2, a3, b2, b3);
-    mma_f16_16816(acc[2], a0, a1, a2, a3, c0, c1);
-    mma_f16_16816(acc[3], a0, a1, a2, a3, c2, c3);
+    uint32_t h0, h1, h2, h3, l0, l1, l2, l3, b0, b1, b2, b3, c0, c1, c2, c3;
+    ldsm_x4(ahi + ks * 32, h0, h1, h2, h3);
+    ldsm_x4(alo + ks * 32, l0, l1, l2, l3);
+    ldsm_x4(b0base + ks * 32, b0, b1, b2, b3);
+    ldsm_x4(b1base + ks * 32, c0, c1, c2, c3);
+    mma_bf16_16816(acc[0], h0, h1, h2, h3, b0, b1);
+    mma_bf16_16816(acc[1], h0, h1, h2, h3, b2, b3);
+    mma_bf16_16816(acc[2], h0, h1, h2, h3, c0, c1);
+    mma_bf16_16816(acc[3], h0, h1, h2, h3, c2, c3);
+    mma_bf16_16816(acc[0], l0, l1, l2, l3, b0, b1);
+    mma_bf16_16816(acc[1], l0, l1, l2, l3, b2, b3);
+    mma_bf16_16816(acc[2], l0, l1, l2, l3, c0, c1);
+    mma_bf16_16816(acc[3], l0, l1, l2, l3, c2, c3);
   }
 }
 
-// Coalesced copy of a staged [TT][ROWH] fp16 tile to rows [t0, t0+TT) of dst (row stride ld).
-__device__ __forceinline__ void store_tile_f16(const __half* stage, __half* dst, long long rowbase, int t0, int S,
-                                               long long ld) {
-  for (int e = threadIdx.x; e < TT * (D / 8); e += NT) {
+// Stream one head's channel-mix weights [out i][in j] (bf16) into wbuf rows of ROWH.
+__device__ __forceinline__ void load_weights_async(const __nv_bfloat16* W, __nv_bfloat16* wbuf) {
+  for (int e = threadIdx.x; e < D * (D / 8); e += NT) {
     const int r = e / (D / 8), v = e % (D / 8);
-    if (t0 + r < S)
-      *reinterpret_cast<uint4*>(dst + (rowbase + t0 + r) * ld + v * 8) =
-          *reinterpret_cast<const uint4*>(stage + r * ROWH + v * 8);
+    cp_async16(smem_u32(wbuf + r * ROWH + v * 8), W + (long long)r * D + v * 8, true);
   }
 }
 
 __global__ void __launch_bounds__(NT, 2) preproc_tc_kernel(const __grid_constant__ PreParams p,
                                                           const __grid_constant__ Theta th) {
   extern __shared__ __align__(16) uint8_t smem_raw[];
-  __half* kbuf = reinterpret_cast<__half*>(smem_raw);  // [ZROWS][D]  k~ latents (kept)
-  __half* zbuf = kbuf + ZROWS * D;                      // [ZROWS][D]  q~ latents of the current head
-  __half* wbuf = zbuf + ZROWS * D;                      // [D][ROWH]   channel weights (fp16)
-  __half* sbuf = wbuf + D * ROWH;                       // [TT][ROWH]  seq-conv output / output staging
-  float* kst = reinterpret_cast<float*>(wbuf);          // [TT][D]     final k (fp32), reuses wbuf
-
   const int G = p.nq / p.nkv;
+  const int H1 = G + 1;
+  const int ZR = TT + p.K - 1;  // staged rows per head
+  __nv_bfloat16* wbuf = reinterpret_cast<__nv_bfloat16*>(smem_raw);  // [D][ROWH] channel weights
+  __nv_bfloat16* shi = wbuf + D * ROWH;                               // [TT][ROWH] s, bf16 high part
+  __nv_bfloat16* slo = shi + TT * ROWH;                               // [TT][ROWH] s, bf16 low part
+  __half* zall = reinterpret_cast<__half*>(slo + TT * ROWH);          // [H1][ZR][ROWH] latents; head G = k
+  __half* stage = reinterpret_cast<__half*>(shi);                     // [TT][ROWH] q output stage
+  float* kst = reinterpret_cast<float*>(wbuf);                        // [TT][KSTR] k stage (fp32)
+
   const int Lq = p.nq * D, Lkv = p.nkv * D, Nlat = Lq + 2 * Lkv;
   const int t0 = blockIdx.x * TT, g = blockIdx.y, b = blockIdx.z;
   const long long rowbase = (long long)b * p.S;
@@ -183,6 +174,17 @@ __global__ void __launch_bounds__(NT, 2) preproc_tc_kernel(const __grid_constant
   const int zr0 = r0 + p.K - 1, zr1 = r1 + p.K - 1;  // current-token rows in the latent tiles
   bool bad = false;
 
+  // ---- all latents of the group (query heads 0..G-1, then the K head) and the K head's weights
+  for (int e = threadIdx.x; e < H1 * ZR * (D / 8); e += NT) {
+    const int hh = e / (ZR * (D / 8)), rem = e % (ZR * (D / 8)), r = rem / (D / 8), v = rem % (D / 8);
+    const int t = t0 - (p.K - 1) + r;
+    const int col = (hh < G) ? (g * G + hh) * D : Lq + g * D;
+    const bool ok = t >= 0 && t < p.S;
+    cp_async16(smem_u32(zall + (hh * ZR + r) * ROWH + v * 8), p.lat + (rowbase + (ok ? t : 0)) * Nlat + col + v * 8,
+               ok);
+  }
+  load_weights_async(p.ck_chan + (long long)g * D * D, wbuf);
+
   // RoPE factors of this thread's (row, column < 64) positions: [nt<2][e]
   float rc[2][4], rs[2][4];
 #pragma unroll
@@ -194,7 +196,7 @@ __global__ void __launch_bounds__(NT, 2) preproc_tc_kernel(const __grid_constant
       float c = 1.f, s = 0.f;
       if (p.use_rope) {
         const double a = (double)pos * th.v[i];
-        // reduce a modulo 2 pi in two steps (2 pi split into a high and a low part)
+        // reduce a modulo 2 pi with 2 pi split into a high and a low double
         const double k = rint(a * 0.15915494309189535);
         double r = fma(-k, 6.283185307179586, a);
         r = fma(-k, 2.4492935982947064e-16, r);
@@ -203,78 +205,73 @@ __global__ void __launch_bounds__(NT, 2) preproc_tc_kernel(const __grid_constant
       rc[nt][e] = c;
       rs[nt][e] = s;
     }
-
-  auto rope_pair = [&](float x1, float x2, int nt, int e, float& o1, float& o2) {
-    o1 = x1 * rc[nt][e] - x2 * rs[nt][e];
-    o2 = x2 * rc[nt][e] + x1 * rs[nt][e];
-  };
-
-  // ---- the K head of the group: conv + channel mix, result kept in registers
-  float ck[4][4];
-  load_latents(p, kbuf, rowbase, t0, Lq + g * D, Nlat);
-  load_weights(p.ck_chan + (long long)g * D * D, wbuf, bad);
-  __syncthreads();
-  seq_conv(p, kbuf, sbuf, p.ck_seq + (long long)g * D * p.K);
-  __syncthreads();
-  channel_mix(sbuf, wbuf, rb, ncol, ck);
-
-  float csum[4][4], mq[4][4];
-#pragma unroll
-  for (int nt = 0; nt < 4; ++nt)
-#pragma unroll
-    for (int e = 0; e < 4; ++e) csum[nt][e] = mq[nt][e] = 0.f;
-
-  // ---- the G query heads
-  for (int hh = 0; hh < G; ++hh) {
-    const int h = g * G + hh;
-    __syncthreads();  // previous users of zbuf / wbuf / sbuf are done
-    load_latents(p, zbuf, rowbase, t0, h * D, Nlat);
-    load_weights(p.cq_chan + (long long)h * D * D, wbuf, bad);
-    __syncthreads();
-    seq_conv(p, zbuf, sbuf, p.cq_seq + (long long)h * D * p.K);
-    __syncthreads();
-    float acc[4][4];
-    channel_mix(sbuf, wbuf, rb, ncol, acc);
-    __syncthreads();  // sbuf becomes the output stage
-    float val[4][4];
-#pragma unroll
-    for (int nt = 0; nt < 4; ++nt)
-#pragma unroll
-      for (int e = 0; e < 4; ++e) {
-        const int col = ncol[nt] + cq + (e & 1);
-        const int zr = (e < 2) ? zr0 : zr1;
-        const float zq = __half2float(zbuf[zr * D + col]);
-        const float zk = __half2float(kbuf[zr * D + col]);
-        float v = acc[nt][e];
-        if (p.mode & 1) v += 0.5f * (zq + zk);
-        if (p.mode & 2) v += 0.5f * (acc[nt][e] + ck[nt][e]);
-        val[nt][e] = v;
-        csum[nt][e] += acc[nt][e];
-        mq[nt][e] += zq;
-      }
+  auto rope = [&](float (&v)[4][4]) {
 #pragma unroll
     for (int nt = 0; nt < 2; ++nt)
 #pragma unroll
       for (int e = 0; e < 4; ++e) {
-        float o1 = val[nt][e], o2 = val[nt + 2][e];
-        if (p.use_rope) rope_pair(val[nt][e], val[nt + 2][e], nt, e, o1, o2);
-        val[nt][e] = o1;
-        val[nt + 2][e] = o2;
+        const float x1 = v[nt][e], x2 = v[nt + 2][e];
+        v[nt][e] = x1 * rc[nt][e] - x2 * rs[nt][e];
+        v[nt + 2][e] = x2 * rc[nt][e] + x1 * rs[nt][e];
       }
+  };
+  auto zval = [&](int hh, int nt, int e) -> float {
+    return __half2float(zall[(hh * ZR + ((e < 2) ? zr0 : zr1)) * ROWH + ncol[nt] + cq + (e & 1)]);
+  };
+
+  // ---- the K head: conv + channel mix, c_k kept in registers
+  cp_async_wait_all();
+  __syncthreads();
+  seq_conv(p, zall + G * ZR * ROWH, shi, slo, p.ck_seq + (long long)g * D * p.K);
+  __syncthreads();
+  float ck[4][4];
+  channel_mix(shi, slo, wbuf, rb, ncol, ck);
+  float csum[4][4];
+#pragma unroll
+  for (int nt = 0; nt < 4; ++nt)
+#pragma unroll
+    for (int e = 0; e < 4; ++e) csum[nt][e] = 0.f;
+
+  // ---- the G query heads
+  for (int hh = 0; hh < G; ++hh) {
+    const int h = g * G + hh;
+    __syncthreads();  // wbuf, shi, slo are free
+    load_weights_async(p.cq_chan + (long long)h * D * D, wbuf);
+    seq_conv(p, zall + hh * ZR * ROWH, shi, slo, p.cq_seq + (long long)h * D * p.K);
+    cp_async_wait_all();
+    __syncthreads();
+    float acc[4][4];
+    channel_mix(shi, slo, wbuf, rb, ncol, acc);
+#pragma unroll
+    for (int nt = 0; nt < 4; ++nt)
+#pragma unroll
+      for (int e = 0; e < 4; ++e) {
+        float v = acc[nt][e];
+        if (p.mode & 1) v += 0.5f * (zval(hh, nt, e) + zval(G, nt, e));
+        if (p.mode & 2) v += 0.5f * (acc[nt][e] + ck[nt][e]);
+        csum[nt][e] += acc[nt][e];
+        acc[nt][e] = v;
+      }
+    if (p.use_rope) rope(acc);
+    __syncthreads();  // shi becomes the q stage
 #pragma unroll
     for (int nt = 0; nt < 4; ++nt) {
       const int col = ncol[nt] + cq;
-      *reinterpret_cast<__half2*>(sbuf + r0 * ROWH + col) = __floats2half2_rn(val[nt][0], val[nt][1]);
-      *reinterpret_cast<__half2*>(sbuf + r1 * ROWH + col) = __floats2half2_rn(val[nt][2], val[nt][3]);
+      *reinterpret_cast<__half2*>(stage + r0 * ROWH + col) = __floats2half2_rn(acc[nt][0], acc[nt][1]);
+      *reinterpret_cast<__half2*>(stage + r1 * ROWH + col) = __floats2half2_rn(acc[nt][2], acc[nt][3]);
 #pragma unroll
-      for (int e = 0; e < 4; ++e) bad |= f16_overflow(val[nt][e]);
+      for (int e = 0; e < 4; ++e) bad |= f16_overflow(acc[nt][e]);
     }
     __syncthreads();
-    store_tile_f16(sbuf, p.q + (long long)h * D, rowbase, t0, p.S, Lq);
+    for (int e = threadIdx.x; e < TT * (D / 8); e += NT) {
+      const int r = e / (D / 8), v = e % (D / 8);
+      if (t0 + r < p.S)
+        *reinterpret_cast<uint4*>(p.q + (rowbase + t0 + r) * Lq + (long long)h * D + v * 8) =
+            *reinterpret_cast<const uint4*>(stage + r * ROWH + v * 8);
+    }
   }
 
-  // ---- k = c_k + means, RoPE; staged in fp32, written as bf16 cache and fp16 copy
-  __syncthreads();  // wbuf is free: it becomes the fp32 k stage
+  // ---- k = c_k + means, RoPE; staged in fp32, written as the bf16 cache and the fp16 copy
   {
     const float invG = 1.f / (float)G;
     float val[4][4];
@@ -282,28 +279,22 @@ __global__ void __launch_bounds__(NT, 2) preproc_tc_kernel(const __grid_constant
     for (int nt = 0; nt < 4; ++nt)
 #pragma unroll
       for (int e = 0; e < 4; ++e) {
-        const int col = ncol[nt] + cq + (e & 1);
-        const int zr = (e < 2) ? zr0 : zr1;
-        const float zk = __half2float(kbuf[zr * D + col]);
         float v = ck[nt][e];
-        if (p.mode & 1) v += 0.5f * (mq[nt][e] * invG + zk);
+        if (p.mode & 1) {
+          float mq = 0.f;
+          for (int hh = 0; hh < G; ++hh) mq += zval(hh, nt, e);
+          v += 0.5f * (mq * invG + zval(G, nt, e));
+        }
         if (p.mode & 2) v += 0.5f * (csum[nt][e] * invG + ck[nt][e]);
         val[nt][e] = v;
       }
-#pragma unroll
-    for (int nt = 0; nt < 2; ++nt)
-#pragma unroll
-      for (int e = 0; e < 4; ++e) {
-        float o1 = val[nt][e], o2 = val[nt + 2][e];
-        if (p.use_rope) rope_pair(val[nt][e], val[nt + 2][e], nt, e, o1, o2);
-        val[nt][e] = o1;
-        val[nt + 2][e] = o2;
-      }
+    if (p.use_rope) rope(val);
+    __syncthreads();  // wbuf becomes the k stage
 #pragma unroll
     for (int nt = 0; nt < 4; ++nt) {
       const int col = ncol[nt] + cq;
-      *reinterpret_cast<float2*>(kst + r0 * D + col) = make_float2(val[nt][0], val[nt][1]);
-      *reinterpret_cast<float2*>(kst + r1 * D + col) = make_float2(val[nt][2], val[nt][3]);
+      *reinterpret_cast<float2*>(kst + r0 * KSTR + col) = make_float2(val[nt][0], val[nt][1]);
+      *reinterpret_cast<float2*>(kst + r1 * KSTR + col) = make_float2(val[nt][2], val[nt][3]);
 #pragma unroll
       for (int e = 0; e < 4; ++e) bad |= f16_overflow(val[nt][e]);
     }
@@ -312,16 +303,13 @@ __global__ void __launch_bounds__(NT, 2) preproc_tc_kernel(const __grid_constant
   for (int e = threadIdx.x; e < TT * (D / 8); e += NT) {
     const int r = e / (D / 8), v = e % (D / 8);
     if (t0 + r >= p.S) continue;
-    const float* src = kst + r * D + v * 8;
-    uint32_t hb[4], hh[4];
-#pragma unroll
-    for (int k = 0; k < 4; ++k) {
-      hb[k] = pack_bf16x2(src[2 * k], src[2 * k + 1]);
-      hh[k] = pack_f16x2(src[2 * k], src[2 * k + 1]);
-    }
+    const float4 lo = *reinterpret_cast<const float4*>(kst + r * KSTR + v * 8);
+    const float4 hi = *reinterpret_cast<const float4*>(kst + r * KSTR + v * 8 + 4);
     const long long off = (rowbase + t0 + r) * Lkv + (long long)g * D + v * 8;
-    *reinterpret_cast<uint4*>(p.k_cache + off) = make_uint4(hb[0], hb[1], hb[2], hb[3]);
-    *reinterpret_cast<uint4*>(p.k_att + off) = make_uint4(hh[0], hh[1], hh[2], hh[3]);
+    *reinterpret_cast<uint4*>(p.k_cache + off) =
+        make_uint4(pack_bf16x2(lo.x, lo.y), pack_bf16x2(lo.z, lo.w), pack_bf16x2(hi.x, hi.y), pack_bf16x2(hi.z, hi.w));
+    *reinterpret_cast<uint4*>(p.k_att + off) =
+        make_uint4(pack_f16x2(lo.x, lo.y), pack_f16x2(lo.z, lo.w), pack_f16x2(hi.x, hi.y), pack_f16x2(hi.z, hi.w));
   }
 
   // ---- value shift: channels [Lkv/2, Lkv) from the previous token (8-channel vectors never straddle)
@@ -368,12 +356,15 @@ __global__ void __launch_bounds__(NT, 2) preproc_tc_kernel(const __grid_constant
   report_range(bad, p.err);
 }
 
-constexpr size_t SMEM_BYTES = sizeof(__half) * (2 * ZROWS * D + D * ROWH + TT * ROWH);
+size_t smem_bytes(int G, int K) {
+  return sizeof(__nv_bfloat16) * ((size_t)D * ROWH + 2 * (size_t)TT * ROWH) +
+         sizeof(__half) * (size_t)(G + 1) * (TT + K - 1) * ROWH;
+}
 
 }  // namespace
 
 bool preproc_tc_supported(const BlockDims& dm) {
-  return dm.io == DType::BF16 && dm.lat == DType::F16 && dm.d == D && dm.K >= 1 && dm.K <= KMAX &&
+  return dm.io == DType::BF16 && dm.lat == DType::F16 && dm.d == D && dm.K >= 1 && dm.K <= KMAX && dm.G <= GMAX &&
          ((long long)dm.E * dm.Lq) % 8 == 0;
 }
 
@@ -403,10 +394,11 @@ cudaError_t launch_preproc_tc(const BlockDims& dm, const BlockPtrs& p, cudaStrea
   q.use_rope = dm.use_rope;
   Theta th;
   for (int i = 0; i < D / 2; ++i) th.v[i] = pow((double)dm.rope_base, -2.0 * (double)i / (double)D);
-  cudaError_t e = cudaFuncSetAttribute(preproc_tc_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)SMEM_BYTES);
+  const size_t smem = smem_bytes(dm.G, dm.K);
+  cudaError_t e = cudaFuncSetAttribute(preproc_tc_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
   if (e != cudaSuccess) return e;
   dim3 grid((dm.S + TT - 1) / TT, dm.nkv, dm.B);
-  preproc_tc_kernel<<<grid, NT, SMEM_BYTES, stream>>>(q, th);
+  preproc_tc_kernel<<<grid, NT, smem, stream>>>(q, th);
   return cudaGetLastError();
 }
 

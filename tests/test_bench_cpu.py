@@ -1,0 +1,39 @@
+"""bench.py on the CPU: the reference arm (the oracle on bounded samples) runs
+and prints one well-formed JSON line; the host helpers give the documented
+work counts."""
+import json
+import os
+import subprocess
+import sys
+
+import bench
+import workloads
+
+ROOT = os.path.dirname(os.path.dirname(os.path.abspath(__file__)))
+
+
+def test_reference_arm_prints_one_json_line():
+    out = subprocess.run([sys.executable, "bench.py", "--impl", "reference", "--workload", "tiny_cca_fp32",
+                          "--steps", "2", "--warmup", "3"], cwd=ROOT, capture_output=True, text=True, timeout=300)
+    assert out.returncode == 0, out.stderr
+    lines = [l for l in out.stdout.splitlines() if l.startswith("{")]
+    assert len(lines) == 1
+    line = json.loads(lines[0])
+    assert line["impl"] == "reference" and line["unit"] == "tokens/s" and line["value"] > 0
+    assert line["cpu_baseline"]["kind"] == "oracle" and line["cpu_baseline"]["cores"] >= 1
+    assert line["e2e"]["h2d_bytes_per_step"] == 0 and line["e2e"]["value"] == line["value"]
+    assert line["config"]["workload"] == "tiny_cca_fp32"
+
+
+def test_algorithmic_work_of_the_headline_workload():
+    w = bench.algorithmic_work(workloads.WORKLOADS["ccgqa_16k_bf16"])
+    assert w["attention_flops"] == 2.0 * 4 * 16384 ** 2 * 128          # 274.9 GFLOP, causal half
+    assert w["down_proj_flops"] == 2.0 * 16384 * 2048 * 1024           # 68.7 GFLOP
+    assert w["out_proj_flops"] == 2.0 * 16384 * 512 * 2048             # 34.4 GFLOP
+    assert w["preproc_bytes"] == 16384 * (1024 + 512 + 512) * 2.0      # 67.1 MB
+
+
+def test_warmup_floor():
+    r = subprocess.run([sys.executable, "bench.py", "--warmup", "2"], cwd=ROOT, capture_output=True, text=True,
+                       timeout=120)
+    assert r.returncode != 0
