@@ -48,21 +48,50 @@ constexpr int OFF_V = OFF_K + KV_STAGES * TILE_BYTES;
 constexpr int OFF_BAR = OFF_V + KV_STAGES * TILE_BYTES;
 constexpr size_t SMEM_BYTES = OFF_BAR + 256 + 1024;
 
-// 2^x on the FMA and integer pipes, for x in [-inf, 126]: x = n + f with
-// n = round(x) (found by adding 1.5 * 2^23, which leaves n in the low
-// mantissa bits) and |f| <= 1/2; 2^f from a cubic fitted to 2^f on
-// [-1/2, 1/2] by iteratively reweighted least squares (max relative error
-// 1.0e-4, below the fp16 rounding of P); 2^n is added to the exponent field.
-// Used for a share of the probabilities so that the special-function unit,
-// which the tensor core otherwise waits on, is not the only exp2 source.
-__device__ __forceinline__ float exp2_fma(float x) {
-  x = fmaxf(x, -126.0f);
-  const float t = x + 12582912.0f;
-  const float f = x - (t - 12582912.0f);
-  const float p = fmaf(fmaf(fmaf(0.05500893f, f, 0.24221097f), f, 0.69328290f), f, 1.0f);
-  return __int_as_float(__float_as_int(p) + (__float_as_int(t) << 23));
+// Packed fp32 pair arithmetic of sm_100 (one instruction for two lanes of work).
+__device__ __forceinline__ void fma2(float& d0, float& d1, float a0, float a1, float b0, float b1, float c0,
+                                     float c1) {
+  asm("{\n .reg .b64 ra, rb, rc, rd;\n mov.b64 ra, {%2, %3};\n mov.b64 rb, {%4, %5};\n"
+      " mov.b64 rc, {%6, %7};\n fma.rn.f32x2 rd, ra, rb, rc;\n mov.b64 {%0, %1}, rd;\n}\n"
+      : "=f"(d0), "=f"(d1)
+      : "f"(a0), "f"(a1), "f"(b0), "f"(b1), "f"(c0), "f"(c1));
 }
-constexpr int POLY_EVERY = 4;  // one pair in POLY_EVERY takes exp2_fma
+__device__ __forceinline__ void add2(float& d0, float& d1, float a0, float a1, float b0, float b1) {
+  asm("{\n .reg .b64 ra, rb, rd;\n mov.b64 ra, {%2, %3};\n mov.b64 rb, {%4, %5};\n"
+      " add.rn.f32x2 rd, ra, rb;\n mov.b64 {%0, %1}, rd;\n}\n"
+      : "=f"(d0), "=f"(d1)
+      : "f"(a0), "f"(a1), "f"(b0), "f"(b1));
+}
+__device__ __forceinline__ float max3f(float a, float b, float c) {
+  float d;
+  asm("max.f32 %0, %1, %2, %3;" : "=f"(d) : "f"(a), "f"(b), "f"(c));
+  return d;
+}
+
+// 2^x for a pair, on the FMA and integer pipes, for x in [-inf, 126]:
+// x = n + f with n = round(x) (adding 1.5 * 2^23 leaves n in the low mantissa
+// bits) and |f| <= 1/2; 2^f from a cubic fitted to 2^f on [-1/2, 1/2] by
+// iteratively reweighted least squares (max relative error 1.0e-4, below the
+// fp16 rounding of P); 2^n is added to the exponent field. A share of the
+// probabilities takes this path so that the special-function unit, which
+// otherwise paces the tensor core at head_dim 128, does less of the work.
+__device__ __forceinline__ void exp2_fma_x2(float x0, float x1, float& p0, float& p1) {
+  constexpr float kMagic = 12582912.0f;
+  x0 = fmaxf(x0, -126.0f);
+  x1 = fmaxf(x1, -126.0f);
+  float t0, t1, r0, r1, f0, f1, q0, q1;
+  add2(t0, t1, x0, x1, kMagic, kMagic);
+  add2(r0, r1, t0, t1, -kMagic, -kMagic);
+  fma2(f0, f1, r0, r1, -1.0f, -1.0f, x0, x1);
+  fma2(q0, q1, 0.05500893f, 0.05500893f, f0, f1, 0.24221097f, 0.24221097f);
+  fma2(q0, q1, q0, q1, f0, f1, 0.69328290f, 0.69328290f);
+  fma2(q0, q1, q0, q1, f0, f1, 1.0f, 1.0f);
+  p0 = __int_as_float(__float_as_int(q0) + (__float_as_int(t0) << 23));
+  p1 = __int_as_float(__float_as_int(q1) + (__float_as_int(t1) << 23));
+}
+#ifndef CCA_POLY_EVERY
+#define CCA_POLY_EVERY 4  // one pair in CCA_POLY_EVERY takes exp2_fma_x2 (0: none)
+#endif
 
 struct AttnMaps {
   CUtensorMap q, k, v;
@@ -292,22 +321,21 @@ __global__ void __launch_bounds__(NUM_THREADS, 1) attn_tc_kernel(const __grid_co
 #pragma unroll
           for (int c = 0; c < 4; ++c) tmem_ld_32x32b_x32(s_col + c * 32, s + c * 32);
           tmem_ld_wait();
-          float tmax = -INFINITY;
           if (jj == qt) {  // diagonal tile: key c is visible to query row iff c <= row
 #pragma unroll
-            for (int c = 0; c < 128; ++c) {
-              float v = (c <= row) ? u2f(s[c]) * p.scale_log2 : -INFINITY;
-              s[c] = __float_as_uint(v);
-              tmax = fmaxf(tmax, v);
-            }
-          } else {
-#pragma unroll
-            for (int c = 0; c < 128; ++c) {
-              float v = u2f(s[c]) * p.scale_log2;
-              s[c] = __float_as_uint(v);
-              tmax = fmaxf(tmax, v);
-            }
+            for (int c = 0; c < 128; ++c)
+              if (c > row) s[c] = __float_as_uint(-INFINITY);
           }
+          // row max of the raw scores (the scale is positive), four independent chains
+          float mx0 = -INFINITY, mx1 = -INFINITY, mx2 = -INFINITY, mx3 = -INFINITY;
+#pragma unroll
+          for (int c = 0; c < 128; c += 8) {
+            mx0 = max3f(mx0, u2f(s[c + 0]), u2f(s[c + 1]));
+            mx1 = max3f(mx1, u2f(s[c + 2]), u2f(s[c + 3]));
+            mx2 = max3f(mx2, u2f(s[c + 4]), u2f(s[c + 5]));
+            mx3 = max3f(mx3, u2f(s[c + 6]), u2f(s[c + 7]));
+          }
+          const float tmax = fmaxf(fmaxf(mx0, mx1), fmaxf(mx2, mx3)) * p.scale_log2;
           // lazy rescale: keep the stale max unless it grew by more than 2^8
           const bool need = tmax > m + RESCALE_THRESHOLD;
           float f = 1.f;  // factor for the O row and the sum
@@ -320,21 +348,30 @@ __global__ void __launch_bounds__(NUM_THREADS, 1) attn_tc_kernel(const __grid_co
             m = mnew;
             rescale = true;
           }
-          float sum = 0.f;
+          const float sc = p.scale_log2, nm = -m;
+          float sa0 = 0.f, sa1 = 0.f, sb0 = 0.f, sb1 = 0.f;  // packed partial row sums
 #pragma unroll
           for (int c2 = 0; c2 < 2; ++c2) {
             uint32_t pk[32];
 #pragma unroll
             for (int e = 0; e < 32; ++e) {
-              const bool poly = (e % POLY_EVERY) == POLY_EVERY - 1;
-              const float x0 = u2f(s[c2 * 64 + 2 * e]) - m, x1 = u2f(s[c2 * 64 + 2 * e + 1]) - m;
-              const float p0 = poly ? exp2_fma(x0) : fast_exp2(x0);
-              const float p1 = poly ? exp2_fma(x1) : fast_exp2(x1);
-              sum += p0 + p1;
+              float x0, x1, p0, p1;
+              fma2(x0, x1, u2f(s[c2 * 64 + 2 * e]), u2f(s[c2 * 64 + 2 * e + 1]), sc, sc, nm, nm);
+              if (CCA_POLY_EVERY > 0 && (e % (CCA_POLY_EVERY > 0 ? CCA_POLY_EVERY : 1)) == CCA_POLY_EVERY - 1) {
+                exp2_fma_x2(x0, x1, p0, p1);
+              } else {
+                p0 = fast_exp2(x0);
+                p1 = fast_exp2(x1);
+              }
+              if (e & 1)
+                add2(sb0, sb1, sb0, sb1, p0, p1);
+              else
+                add2(sa0, sa1, sa0, sa1, p0, p1);
               pk[e] = pack_f16x2(p0, p1);
             }
             tmem_st_32x32b_x32(s_col + c2 * 32, pk);
           }
+          const float sum = (sa0 + sa1) + (sb0 + sb1);
           l = l * f + sum;
           if (rescale) {
             // O_j is stable: the commit behind s_full covered the previous PV
