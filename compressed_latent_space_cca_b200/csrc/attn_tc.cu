@@ -10,7 +10,8 @@
 // One CTA owns a pair of 128-query tiles of one KV group (for G >= 2 two
 // query heads at the same positions, for G = 1 two consecutive query tiles
 // of one head), so every K/V tile it loads serves both. Roles:
-//   warp 0      TMA: Q tiles once per pair, then K and V tiles (2-stage ring)
+//   warp 0      TMA: Q tiles once per pair, then K tiles (3-stage ring) and V
+//               tiles (2-stage ring)
 //   warp 1      one thread issues tcgen05.mma: S_j = Q_j K^T (SS form) into
 //               TMEM, then O_j += P_j V (TS form, P read from TMEM)
 //   warps 2-5   softmax of tile 0, warps 6-9 softmax of tile 1: each thread
@@ -22,8 +23,13 @@
 // the first 64 columns of S_j. The two tiles ping-pong: while one softmax
 // group works, the tensor core runs the other tile's MMAs. Key tiles above
 // the diagonal are never loaded (causal tile skipping); the diagonal tile is
-// masked per element. Pairs are scheduled longest first over persistent
-// CTAs. Every mbarrier wait is bounded.
+// masked per element. Pairs are assigned to the persistent CTAs by a host-side
+// longest-processing-time schedule (largest pair to the least-loaded CTA),
+// passed in the kernel parameters. Every mbarrier wait is bounded.
+#include <queue>
+#include <utility>
+#include <vector>
+
 #include "cca_common.cuh"
 #include "launch.h"
 
@@ -33,7 +39,7 @@ namespace {
 constexpr int D = 128;           // head dim
 constexpr int TQ = 128;          // queries per tile
 constexpr int TK = 128;          // keys per tile
-constexpr int KV_STAGES = 2;
+constexpr int K_STAGES = 3, V_STAGES = 2;
 constexpr int HALF_BYTES = 128 * 64 * 2;  // 128 rows x 64 fp16 (one 128-byte swizzle span)
 constexpr int TILE_BYTES = 2 * HALF_BYTES;  // 128 x 128 fp16
 constexpr int NUM_THREADS = 320;
@@ -41,11 +47,13 @@ constexpr int TMEM_COLS = 512;
 constexpr uint32_t COL_S0 = 0, COL_O0 = 256;
 constexpr float RESCALE_THRESHOLD = 8.0f;  // log2 units: rescale O only if the max grows by > 2^8
 
-// shared memory: Q0 | Q1 | K[2] | V[2] | barriers
+// shared memory: Q0 | Q1 | K[3] | V[2] | barriers
 constexpr int OFF_Q = 0;
 constexpr int OFF_K = 2 * TILE_BYTES;
-constexpr int OFF_V = OFF_K + KV_STAGES * TILE_BYTES;
-constexpr int OFF_BAR = OFF_V + KV_STAGES * TILE_BYTES;
+constexpr int OFF_V = OFF_K + K_STAGES * TILE_BYTES;
+constexpr int OFF_BAR = OFF_V + V_STAGES * TILE_BYTES;
+constexpr int MAX_CTAS = 160;
+constexpr int MAX_LIST = 4096;  // pairs a host schedule can hold in the kernel parameters
 constexpr size_t SMEM_BYTES = OFF_BAR + 256 + 1024;
 
 // Packed fp32 pair arithmetic of sm_100 (one instruction for two lanes of work).
@@ -90,7 +98,7 @@ __device__ __forceinline__ void exp2_fma_x2(float x0, float x1, float& p0, float
   p1 = __int_as_float(__float_as_int(q1) + (__float_as_int(t1) << 23));
 }
 #ifndef CCA_POLY_EVERY
-#define CCA_POLY_EVERY 4  // one pair in CCA_POLY_EVERY takes exp2_fma_x2 (0: none)
+#define CCA_POLY_EVERY 8  // one pair in CCA_POLY_EVERY takes exp2_fma_x2 (0: none)
 #endif
 
 struct AttnMaps {
@@ -106,6 +114,13 @@ struct AttnParams {
   float scale_log2;  // softmax scale * log2(e)
   __half* o;
   unsigned* err;
+};
+
+// Per-CTA work lists: CTA c runs items[off[c] .. off[c+1]).
+struct AttnSched {
+  int use;  // 0: serpentine order instead
+  unsigned short off[MAX_CTAS + 1];
+  unsigned short items[MAX_LIST];
 };
 
 struct Item {
@@ -135,23 +150,29 @@ __device__ __forceinline__ Item get_item(const AttnParams& p, int w) {
   return it;
 }
 
-// Work item of this CTA in round r (serpentine order over the CTAs).
-__device__ __forceinline__ int item_index(int r, int cta, int grid) {
-  return r * grid + ((r & 1) ? (grid - 1 - cta) : cta);
+// Work item of this CTA in round r, or -1 when it has none left.
+__device__ __forceinline__ int item_index(const AttnSched& sc, int items, int r, int cta, int grid) {
+  if (sc.use) {
+    const int i = sc.off[cta] + r;
+    return i < sc.off[cta + 1] ? (int)sc.items[i] : -1;
+  }
+  const int w = r * grid + ((r & 1) ? (grid - 1 - cta) : cta);  // serpentine over the CTAs
+  return w < items ? w : -1;
 }
 
 __global__ void __launch_bounds__(NUM_THREADS, 1) attn_tc_kernel(const __grid_constant__ AttnMaps maps,
-                                                                 const AttnParams p) {
+                                                                 const AttnParams p,
+                                                                 const __grid_constant__ AttnSched sched) {
   extern __shared__ uint8_t smem_raw[];
   uint8_t* smem = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
   uint64_t* bars = reinterpret_cast<uint64_t*>(smem + OFF_BAR);
   uint64_t* q_full = bars + 0;
   uint64_t* q_empty = bars + 1;
-  uint64_t* k_full = bars + 2;             // [KV_STAGES]
-  uint64_t* k_empty = k_full + KV_STAGES;  // [KV_STAGES]
-  uint64_t* v_full = k_empty + KV_STAGES;  // [KV_STAGES]
-  uint64_t* v_empty = v_full + KV_STAGES;  // [KV_STAGES]
-  uint64_t* s_full = v_empty + KV_STAGES;  // [2]
+  uint64_t* k_full = bars + 2;             // [K_STAGES]
+  uint64_t* k_empty = k_full + K_STAGES;   // [K_STAGES]
+  uint64_t* v_full = k_empty + K_STAGES;   // [V_STAGES]
+  uint64_t* v_empty = v_full + V_STAGES;   // [V_STAGES]
+  uint64_t* s_full = v_empty + V_STAGES;   // [2]
   uint64_t* p_full = s_full + 2;           // [2]
   uint64_t* o_full = p_full + 2;           // [2]
   uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(o_full + 2);
@@ -161,9 +182,11 @@ __global__ void __launch_bounds__(NUM_THREADS, 1) attn_tc_kernel(const __grid_co
   if (threadIdx.x == 0) {
     mbar_init(smem_u32(q_full), 1);
     mbar_init(smem_u32(q_empty), 1);
-    for (int s = 0; s < KV_STAGES; ++s) {
+    for (int s = 0; s < K_STAGES; ++s) {
       mbar_init(smem_u32(&k_full[s]), 1);
       mbar_init(smem_u32(&k_empty[s]), 1);
+    }
+    for (int s = 0; s < V_STAGES; ++s) {
       mbar_init(smem_u32(&v_full[s]), 1);
       mbar_init(smem_u32(&v_empty[s]), 1);
     }
@@ -193,11 +216,11 @@ __global__ void __launch_bounds__(NUM_THREADS, 1) attn_tc_kernel(const __grid_co
   if (warp == 0) {
     if (lane == 0) {
       // ------------------------------------------------------------ TMA --
-      int stage = 0;
-      uint32_t phase = 0;
+      int kst = 0, vst = 0;
+      uint32_t kph = 0, vph = 0;
       for (int r = 0;; ++r) {
-        const int w = item_index(r, cta, grid);
-        if (w >= p.items) break;
+        const int w = item_index(sched, p.items, r, cta, grid);
+        if (w < 0) break;
         const Item it = get_item(p, w);
         if (!mbar_wait_bounded(smem_u32(q_empty), (r & 1) ^ 1, p.err, abort_flag, wait_site(kSiteAttn, 1, 1))) goto done;
         mbar_arrive_expect_tx(smem_u32(q_full), 2 * TILE_BYTES);
@@ -207,22 +230,34 @@ __global__ void __launch_bounds__(NUM_THREADS, 1) attn_tc_kernel(const __grid_co
           for (int hf = 0; hf < 2; ++hf)
             tma_load_3d(smem_u32(smem + OFF_Q + j * TILE_BYTES + hf * HALF_BYTES), &maps.q, smem_u32(q_full),
                         it.h[j] * D + hf * 64, it.qt[j] * TQ, it.b);
+        // K runs one tile ahead of V: the MMA thread needs K_{jj+1} right after its PVs on V_jj,
+        // and a wait for a free V slot must not hold back the next K load
+        auto load_k = [&](int jj) -> bool {
+          if (!mbar_wait_bounded(smem_u32(&k_empty[kst]), kph ^ 1, p.err, abort_flag, wait_site(kSiteAttn, 1, 2)))
+            return false;
+          mbar_arrive_expect_tx(smem_u32(&k_full[kst]), TILE_BYTES);
+#pragma unroll
+          for (int hf = 0; hf < 2; ++hf)
+            tma_load_3d(smem_u32(smem + OFF_K + kst * TILE_BYTES + hf * HALF_BYTES), &maps.k, smem_u32(&k_full[kst]),
+                        it.g * D + hf * 64, jj * TK, it.b);
+          if (++kst == K_STAGES) {
+            kst = 0;
+            kph ^= 1;
+          }
+          return true;
+        };
+        if (!load_k(0)) goto done;
         for (int jj = 0; jj < it.nkv_tiles; ++jj) {
-          if (!mbar_wait_bounded(smem_u32(&k_empty[stage]), phase ^ 1, p.err, abort_flag, wait_site(kSiteAttn, 1, 2))) goto done;
-          mbar_arrive_expect_tx(smem_u32(&k_full[stage]), TILE_BYTES);
+          if (jj + 1 < it.nkv_tiles && !load_k(jj + 1)) goto done;
+          if (!mbar_wait_bounded(smem_u32(&v_empty[vst]), vph ^ 1, p.err, abort_flag, wait_site(kSiteAttn, 1, 3))) goto done;
+          mbar_arrive_expect_tx(smem_u32(&v_full[vst]), TILE_BYTES);
 #pragma unroll
           for (int hf = 0; hf < 2; ++hf)
-            tma_load_3d(smem_u32(smem + OFF_K + stage * TILE_BYTES + hf * HALF_BYTES), &maps.k,
-                        smem_u32(&k_full[stage]), it.g * D + hf * 64, jj * TK, it.b);
-          if (!mbar_wait_bounded(smem_u32(&v_empty[stage]), phase ^ 1, p.err, abort_flag, wait_site(kSiteAttn, 1, 3))) goto done;
-          mbar_arrive_expect_tx(smem_u32(&v_full[stage]), TILE_BYTES);
-#pragma unroll
-          for (int hf = 0; hf < 2; ++hf)
-            tma_load_3d(smem_u32(smem + OFF_V + stage * TILE_BYTES + hf * HALF_BYTES), &maps.v,
-                        smem_u32(&v_full[stage]), it.g * D + hf * 64, jj * TK, it.b);
-          if (++stage == KV_STAGES) {
-            stage = 0;
-            phase ^= 1;
+            tma_load_3d(smem_u32(smem + OFF_V + vst * TILE_BYTES + hf * HALF_BYTES), &maps.v, smem_u32(&v_full[vst]),
+                        it.g * D + hf * 64, jj * TK, it.b);
+          if (++vst == V_STAGES) {
+            vst = 0;
+            vph ^= 1;
           }
         }
       }
@@ -232,41 +267,52 @@ __global__ void __launch_bounds__(NUM_THREADS, 1) attn_tc_kernel(const __grid_co
       // ------------------------------------------------------------ MMA --
       const uint32_t idesc_qk = idesc_f32acc(TQ, TK, 0, 0, kFmtF16);  // Q, K both K-major (d contiguous)
       const uint32_t idesc_pv = idesc_f32acc(TQ, D, 0, 1, kFmtF16);   // P from TMEM, V MN-major (d contiguous)
-      int stage = 0;
-      uint32_t phase = 0;
+      int kst = 0, vst = 0;
+      uint32_t kph = 0, vph = 0;
       uint32_t pcount[2] = {0, 0};
+      // K-major tiles (Q, K): LBO unused, SBO = 1024 B between 8-row groups; V (MN-major): LBO =
+      // HALF_BYTES between the two 64-column halves of d, SBO = 1024 B between 8-key groups.
+      // The start-address field counts 16-byte units, so stepping a tile by TILE_BYTES adds TILE_BYTES / 16.
+      const uint32_t sw_hi = desc_hi(smem_desc_sw128(smem_u32(smem), 16, 1024));
+      const uint32_t v_hi = desc_hi(smem_desc_sw128(smem_u32(smem), HALF_BYTES, 1024));
+      const uint32_t q_lo0 = desc_lo(smem_desc_sw128(smem_u32(smem + OFF_Q), 16, 1024));
+      const uint32_t k_lo0 = desc_lo(smem_desc_sw128(smem_u32(smem + OFF_K), 16, 1024));
+      const uint32_t v_lo0 = desc_lo(smem_desc_sw128(smem_u32(smem + OFF_V), HALF_BYTES, 1024));
+      constexpr uint32_t kTileStep = TILE_BYTES >> 4;
       for (int r = 0;; ++r) {
-        const int w = item_index(r, cta, grid);
-        if (w >= p.items) break;
+        const int w = item_index(sched, p.items, r, cta, grid);
+        if (w < 0) break;
         const Item it = get_item(p, w);
         if (!mbar_wait_bounded(smem_u32(q_full), r & 1, p.err, abort_flag, wait_site(kSiteAttn, 2, 4))) goto done;
         // O_j of the previous pair needs no guard: the first PV of this pair waits for p_full[j],
         // which the softmax group raises only after its epilogue has read O_j back.
         tc_fence_after();
-        const uint32_t q_base[2] = {smem_u32(smem + OFF_Q), smem_u32(smem + OFF_Q + TILE_BYTES)};
+        // S_j = Q_j K_st^T: descriptors built once, the K = 16 steps advance the start address
+        // (16-byte units) by 2 within a 128-byte row and by HALF_BYTES / 16 per d half
         auto issue_qk = [&](int j, int st) {
-          const uint32_t kb = smem_u32(smem + OFF_K + st * TILE_BYTES);
+          const uint32_t alo = q_lo0 + j * kTileStep, blo = k_lo0 + st * kTileStep;
 #pragma unroll
           for (int kk = 0; kk < D / 16; ++kk) {
-            const uint32_t off = (kk >> 2) * HALF_BYTES + (kk & 3) * 32;
-            umma_ss(tmem + COL_S0 + j * TK, smem_desc_sw128(q_base[j] + off, 16, 1024),
-                    smem_desc_sw128(kb + off, 16, 1024), idesc_qk, kk > 0);
+            const uint32_t off = ((kk >> 2) * HALF_BYTES + (kk & 3) * 32) >> 4;
+            umma_ss_lohi(tmem + COL_S0 + j * TK, alo + off, sw_hi, blo + off, sw_hi, idesc_qk, kk > 0);
           }
           umma_commit(smem_u32(&s_full[j]));
         };
         // first key tile: S_j = Q_j K_0^T for both tiles
-        if (!mbar_wait_bounded(smem_u32(&k_full[stage]), phase, p.err, abort_flag, wait_site(kSiteAttn, 2, 6))) goto done;
+        if (!mbar_wait_bounded(smem_u32(&k_full[kst]), kph, p.err, abort_flag, wait_site(kSiteAttn, 2, 6))) goto done;
         tc_fence_after();
         for (int j = 0; j < 2; ++j)
-          if (it.active[j]) issue_qk(j, stage);
-        umma_commit(smem_u32(&k_empty[stage]));
+          if (it.active[j]) issue_qk(j, kst);
+        umma_commit(smem_u32(&k_empty[kst]));
+        if (++kst == K_STAGES) {
+          kst = 0;
+          kph ^= 1;
+        }
         for (int jj = 0; jj < it.nkv_tiles; ++jj) {
-          const int nst = (stage + 1 == KV_STAGES) ? 0 : stage + 1;
-          const uint32_t nph = (stage + 1 == KV_STAGES) ? phase ^ 1 : phase;
           bool next_k_ready = false;
-          if (!mbar_wait_bounded(smem_u32(&v_full[stage]), phase, p.err, abort_flag, wait_site(kSiteAttn, 2, 7))) goto done;
+          if (!mbar_wait_bounded(smem_u32(&v_full[vst]), vph, p.err, abort_flag, wait_site(kSiteAttn, 2, 7))) goto done;
           tc_fence_after();
-          const uint32_t vb = smem_u32(smem + OFF_V + stage * TILE_BYTES);
+          const uint32_t vlo = v_lo0 + vst * kTileStep;
           for (int j = 0; j < 2; ++j) {
             if (!it.active[j] || jj > it.qt[j]) continue;
             if (!mbar_wait_bounded(smem_u32(&p_full[j]), pcount[j] & 1, p.err, abort_flag, wait_site(kSiteAttn, 2, 8))) goto done;
@@ -275,23 +321,31 @@ __global__ void __launch_bounds__(NUM_THREADS, 1) attn_tc_kernel(const __grid_co
             // O_j += P_j V_jj
 #pragma unroll
             for (int kk = 0; kk < TK / 16; ++kk)
-              umma_ts(tmem + COL_O0 + j * D, tmem + COL_S0 + j * TK + kk * 8,
-                      smem_desc_sw128(vb + kk * 16 * 128, HALF_BYTES, 1024), idesc_pv, (jj > 0 || kk > 0));
+              umma_ts_lohi(tmem + COL_O0 + j * D, tmem + COL_S0 + j * TK + kk * 8, vlo + ((kk * 16 * 128) >> 4),
+                           v_hi, idesc_pv, (jj > 0 || kk > 0));
             if (jj + 1 <= it.qt[j]) {
               if (!next_k_ready) {
-                if (!mbar_wait_bounded(smem_u32(&k_full[nst]), nph, p.err, abort_flag, wait_site(kSiteAttn, 2, 9))) goto done;
+                if (!mbar_wait_bounded(smem_u32(&k_full[kst]), kph, p.err, abort_flag, wait_site(kSiteAttn, 2, 9))) goto done;
                 tc_fence_after();
                 next_k_ready = true;
               }
-              issue_qk(j, nst);  // S_j = Q_j K_{jj+1}^T, overwrites P_j after the PV above
+              issue_qk(j, kst);  // S_j = Q_j K_{jj+1}^T, overwrites P_j after the PV above
             } else {
               umma_commit(smem_u32(&o_full[j]));
             }
           }
-          umma_commit(smem_u32(&v_empty[stage]));
-          if (next_k_ready) umma_commit(smem_u32(&k_empty[nst]));
-          stage = nst;
-          phase = nph;
+          umma_commit(smem_u32(&v_empty[vst]));
+          if (++vst == V_STAGES) {
+            vst = 0;
+            vph ^= 1;
+          }
+          if (next_k_ready) {
+            umma_commit(smem_u32(&k_empty[kst]));
+            if (++kst == K_STAGES) {
+              kst = 0;
+              kph ^= 1;
+            }
+          }
         }
         umma_commit(smem_u32(q_empty));
       }
@@ -306,8 +360,8 @@ __global__ void __launch_bounds__(NUM_THREADS, 1) attn_tc_kernel(const __grid_co
     const uint32_t o_col = tmem + lane_off + COL_O0 + j * D;
     uint32_t scount = 0, ocount = 0;
     for (int r = 0;; ++r) {
-      const int w = item_index(r, cta, grid);
-      if (w >= p.items) break;
+      const int w = item_index(sched, p.items, r, cta, grid);
+      if (w < 0) break;
       const Item it = get_item(p, w);
       if (it.active[j]) {
         const int qt = it.qt[j];
@@ -466,10 +520,36 @@ cudaError_t launch_attention_tc(const BlockDims& dm, const void* q, const void* 
   p.scale_log2 = dm.scale * 1.4426950408889634f;
   p.o = static_cast<__half*>(o);
   p.err = dev_err;
-  const int grid = p.items < num_sms() ? p.items : num_sms();
+  int grid = p.items < num_sms() ? p.items : num_sms();
+  if (grid > MAX_CTAS) grid = MAX_CTAS;
+  // Longest-processing-time assignment: pairs come in non-increasing order of key tiles
+  // (item index order), each goes to the CTA with the least work so far.
+  static thread_local AttnSched plan;
+  plan.use = p.items <= MAX_LIST;
+  if (plan.use) {
+    std::vector<std::vector<unsigned short>> lists(grid);
+    std::priority_queue<std::pair<long long, int>, std::vector<std::pair<long long, int>>, std::greater<>> heap;
+    for (int c = 0; c < grid; ++c) heap.push({0, c});
+    const int bgc = p.B * p.nkv, U = p.num_qt * p.G;
+    for (int w = 0; w < p.items; ++w) {
+      const int pr = p.pairs - 1 - w / bgc;
+      const int qt_last = (2 * pr + 1 < U ? 2 * pr + 1 : 2 * pr) / p.G;
+      const long long cost = 2 * (qt_last + 1) + 1;  // key tiles of both tiles, plus the pair's setup
+      auto top = heap.top();
+      heap.pop();
+      lists[top.second].push_back((unsigned short)w);
+      heap.push({top.first + cost, top.second});
+    }
+    int off = 0;
+    for (int c = 0; c < grid; ++c) {
+      plan.off[c] = (unsigned short)off;
+      for (unsigned short w : lists[c]) plan.items[off++] = w;
+    }
+    plan.off[grid] = (unsigned short)off;
+  }
   cudaError_t e = cudaFuncSetAttribute(attn_tc_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)SMEM_BYTES);
   if (e != cudaSuccess) return e;
-  attn_tc_kernel<<<grid, NUM_THREADS, SMEM_BYTES, stream>>>(maps, p);
+  attn_tc_kernel<<<grid, NUM_THREADS, SMEM_BYTES, stream>>>(maps, p, plan);
   return cudaGetLastError();
 }
 

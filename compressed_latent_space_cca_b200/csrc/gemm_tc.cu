@@ -154,6 +154,9 @@ __global__ void __launch_bounds__(NUM_THREADS, 1) gemm_tc_kernel(const __grid_co
     if (lane == 0) {
       // ------------------------------------------------------ MMA issuer --
       const uint32_t idesc = idesc_f32acc(BM, BN, 0, 0, p.in_fmt);
+      // descriptors built once; a stage step adds STAGE_BYTES / 16 to the start address, a K = 16 step 2
+      const uint32_t d_hi = desc_hi(smem_desc_sw128(smem_u32(smem), 16, 1024));
+      const uint32_t a_lo0 = desc_lo(smem_desc_sw128(smem_u32(smem), 16, 1024));
       int stage = 0;
       uint32_t phase = 0;
       int i = 0;
@@ -166,14 +169,10 @@ __global__ void __launch_bounds__(NUM_THREADS, 1) gemm_tc_kernel(const __grid_co
         for (int kb = 0; kb < kblocks; ++kb) {
           if (!mbar_wait_bounded(smem_u32(&full[stage]), phase, p.err, abort_flag, wait_site(kSiteGemm, 2, 3))) goto mma_done;
           tc_fence_after();
-          const uint32_t a_base = smem_u32(smem + stage * STAGE_BYTES);
-          const uint32_t b_base = a_base + A_BYTES;
+          const uint32_t a_lo = a_lo0 + stage * (STAGE_BYTES >> 4);
+          const uint32_t b_lo = a_lo + (A_BYTES >> 4);
 #pragma unroll
-          for (int k = 0; k < BK / 16; ++k) {
-            const uint64_t ad = smem_desc_sw128(a_base + k * 32, 16, 1024);
-            const uint64_t bd = smem_desc_sw128(b_base + k * 32, 16, 1024);
-            umma_ss(d_tmem, ad, bd, idesc, (kb | k) != 0);
-          }
+          for (int k = 0; k < BK / 16; ++k) umma_ss_lohi(d_tmem, a_lo + 2 * k, d_hi, b_lo + 2 * k, d_hi, idesc, (kb | k) != 0);
           umma_commit(smem_u32(&empty[stage]));
           if (++stage == STAGES) {
             stage = 0;
