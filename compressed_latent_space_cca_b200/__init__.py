@@ -193,6 +193,35 @@ def prefill(cfg: CcaConfig, inputs: Dict[str, torch.Tensor], *, out: Optional[Di
     return res
 
 
+def prefill_noalloc(cfg: CcaConfig, inputs: Dict[str, torch.Tensor], *,
+                    out: Optional[Dict[str, torch.Tensor]] = None, conv_state: bool = False,
+                    stream: Optional[torch.cuda.Stream] = None) -> Dict[str, torch.Tensor]:
+    """cca_prefill_noalloc: the block with its intermediates in the library's own
+    fixed device array (no workspace argument), for callers that must not allocate
+    device memory while they run. Blocks needing more than
+    CCA_NOALLOC_WORKSPACE_BYTES of workspace are rejected; calls that overlap on
+    the GPU share that array and must be ordered by the caller."""
+    x = inputs["x"]
+    device = x.device
+    if device.type != "cuda":
+        raise ValueError("inputs must be CUDA tensors")
+    sh = _shapes(cfg)
+    dt = _DT[cfg.dtype]
+    ptrs = [_check(inputs[n], n, sh[n], dt, device) for n in INPUT_NAMES]
+    if out is None:
+        out = alloc_outputs(cfg, device, conv_state)
+    y = _check(out["y"], "y", sh["y"], _DT[cfg.out_dtype], device)
+    kc = _check(out["k_cache"], "k_cache", sh["k_cache"], dt, device)
+    vc = _check(out["v_cache"], "v_cache", sh["v_cache"], dt, device)
+    cs = _check(out["conv_state"], "conv_state", sh["conv_state"], dt, device) if "conv_state" in out else None
+    if stream is None:
+        stream = torch.cuda.current_stream(device)
+    st = library().cca_prefill_noalloc(ctypes.byref(cfg), *ptrs, y, kc, vc, cs, ctypes.c_void_p(stream.cuda_stream))
+    if st != CCA_OK:
+        raise CcaError(st, "cca_prefill_noalloc")
+    return dict(out)
+
+
 def prefill_host(cfg: CcaConfig, x_host: torch.Tensor, weights: Dict[str, torch.Tensor], x_dev: torch.Tensor,
                  y_dev: torch.Tensor, y_host: torch.Tensor, k_cache: torch.Tensor, v_cache: torch.Tensor,
                  workspace: torch.Tensor, stream: Optional[torch.cuda.Stream] = None) -> None:

@@ -19,6 +19,8 @@ CCA_F32 = 0
 CCA_BF16 = 1
 CCA_F16 = 2
 
+CCA_NOALLOC_WORKSPACE_BYTES = 64 << 20
+
 CCA_PATH_AUTO = 0
 CCA_PATH_SIMT = 1
 CCA_PATH_TENSOR = 2
@@ -84,6 +86,7 @@ SIGNATURES = {
     "cca_plan": (c_int, [POINTER(CcaConfig), c_int, POINTER(CcaPlan)]),
     "cca_prefill": (c_int, _PREFILL_ARGS),
     "cca_prefill_ex": (c_int, _PREFILL_ARGS + [POINTER(CcaPrefillOpts)]),
+    "cca_prefill_noalloc": (c_int, [POINTER(CcaConfig)] + [c_void_p] * 9 + [c_void_p] * 4 + [c_void_p]),
     "cca_prefill_host": (c_int, [POINTER(CcaConfig), c_void_p, c_void_p] + [c_void_p] * 8
                          + [c_void_p, c_void_p, c_void_p, c_void_p, c_void_p, c_void_p, c_size_t, c_void_p]),
     "cca_poll_device_status": (c_int, [c_void_p]),

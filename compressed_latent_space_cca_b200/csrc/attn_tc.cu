@@ -26,10 +26,6 @@
 // masked per element. Pairs are assigned to the persistent CTAs by a host-side
 // longest-processing-time schedule (largest pair to the least-loaded CTA),
 // passed in the kernel parameters. Every mbarrier wait is bounded.
-#include <queue>
-#include <utility>
-#include <vector>
-
 #include "cca_common.cuh"
 #include "launch.h"
 
@@ -523,29 +519,48 @@ cudaError_t launch_attention_tc(const BlockDims& dm, const void* q, const void* 
   int grid = p.items < num_sms() ? p.items : num_sms();
   if (grid > MAX_CTAS) grid = MAX_CTAS;
   // Longest-processing-time assignment: pairs come in non-increasing order of key tiles
-  // (item index order), each goes to the CTA with the least work so far.
+  // (item index order), each goes to the CTA with the least work so far (a binary min-heap of
+  // CTA loads). Fixed-size arrays only: launching allocates no memory.
   static thread_local AttnSched plan;
   plan.use = p.items <= MAX_LIST;
   if (plan.use) {
-    std::vector<std::vector<unsigned short>> lists(grid);
-    std::priority_queue<std::pair<long long, int>, std::vector<std::pair<long long, int>>, std::greater<>> heap;
-    for (int c = 0; c < grid; ++c) heap.push({0, c});
+    long long load[MAX_CTAS];
+    int heap_cta[MAX_CTAS], count[MAX_CTAS];
+    static thread_local unsigned short owner[MAX_LIST];
+    for (int c = 0; c < grid; ++c) {
+      load[c] = 0;
+      heap_cta[c] = c;
+      count[c] = 0;
+    }
+    auto less = [&](int a, int b) { return load[a] < load[b] || (load[a] == load[b] && a < b); };
     const int bgc = p.B * p.nkv, U = p.num_qt * p.G;
     for (int w = 0; w < p.items; ++w) {
       const int pr = p.pairs - 1 - w / bgc;
       const int qt_last = (2 * pr + 1 < U ? 2 * pr + 1 : 2 * pr) / p.G;
-      const long long cost = 2 * (qt_last + 1) + 1;  // key tiles of both tiles, plus the pair's setup
-      auto top = heap.top();
-      heap.pop();
-      lists[top.second].push_back((unsigned short)w);
-      heap.push({top.first + cost, top.second});
+      const int c = heap_cta[0];
+      owner[w] = (unsigned short)c;
+      ++count[c];
+      load[c] += 2 * (qt_last + 1) + 1;  // key tiles of both tiles, plus the pair's setup
+      for (int i = 0;;) {                // sift the root down
+        const int l = 2 * i + 1, r = l + 1;
+        int m = i;
+        if (l < grid && less(heap_cta[l], heap_cta[m])) m = l;
+        if (r < grid && less(heap_cta[r], heap_cta[m])) m = r;
+        if (m == i) break;
+        const int t = heap_cta[i];
+        heap_cta[i] = heap_cta[m];
+        heap_cta[m] = t;
+        i = m;
+      }
     }
     int off = 0;
     for (int c = 0; c < grid; ++c) {
       plan.off[c] = (unsigned short)off;
-      for (unsigned short w : lists[c]) plan.items[off++] = w;
+      off += count[c];
+      count[c] = plan.off[c];  // fill cursor
     }
     plan.off[grid] = (unsigned short)off;
+    for (int w = 0; w < p.items; ++w) plan.items[count[owner[w]]++] = (unsigned short)w;
   }
   cudaError_t e = cudaFuncSetAttribute(attn_tc_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)SMEM_BYTES);
   if (e != cudaSuccess) return e;

@@ -316,6 +316,11 @@ cca_status_t prepare(const cca_config_t* cfg, int path, const void* const* ins, 
 
 }  // namespace
 
+int set_last_error(int status, const char* msg) {
+  t_last_error = msg;
+  return status;
+}
+
 int num_sms() {
   DeviceInfo* di = nullptr;
   if (device_info(&di) != CCA_OK) return 148;

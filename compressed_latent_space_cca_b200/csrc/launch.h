@@ -94,4 +94,8 @@ EncodeTiledFn get_encode_tiled();
 
 int num_sms();
 
+// Records msg as the calling thread's cca_last_error_message and returns status (an int
+// holding a cca_status_t, so this header needs no C-ABI types).
+int set_last_error(int status, const char* msg);
+
 }  // namespace cca

@@ -214,6 +214,36 @@ cca_status_t cca_prefill_host(const cca_config_t* cfg,
                               void* k_cache, void* v_cache, void* conv_state,
                               void* workspace, size_t workspace_bytes, void* stream);
 
+/*
+ * cca_prefill without a caller-provided workspace. The paper has no
+ * counterpart; this exists for callers that must not allocate device memory
+ * while they run: cudaMalloc can synchronize the device and stall every
+ * stream of the process, runtimes that own the whole device memory pool (and
+ * the plugins they host) forbid it, and a caller that already holds all of its
+ * memory has nowhere to get cca_workspace_size() bytes from.
+ *
+ * The intermediates go to a fixed 256-byte-aligned device array inside the
+ * library of CCA_NOALLOC_WORKSPACE_BYTES; every GPU on which this is called
+ * keeps that memory until the process exits. Blocks whose
+ * cca_workspace_size() exceeds it are rejected with CCA_ERR_WORKSPACE (e.g.
+ * B=1, S=8192, E=2048, 4 query / 2 KV heads of 128 needs 44 MB and fits;
+ * S=16384 does not). The first call on a device looks up the array's device
+ * address (cudaGetSymbolAddress); make that first call before capturing a
+ * stream. All calls share the array: calls whose work may overlap on the GPU
+ * (other streams, other host threads on the device) race on it, so order them.
+ * Nothing in it needs to start at zero. Arguments, outputs and errors are
+ * those of cca_prefill; the library allocates nothing.
+ */
+#define CCA_NOALLOC_WORKSPACE_BYTES 67108864
+cca_status_t cca_prefill_noalloc(const cca_config_t* cfg,
+                                 const void* x,
+                                 const void* W_q, const void* W_k, const void* W_v,
+                                 const void* convq_seq, const void* convq_chan,
+                                 const void* convk_seq, const void* convk_chan,
+                                 const void* W_o,
+                                 void* y, void* k_cache, void* v_cache, void* conv_state,
+                                 void* stream);
+
 /* Synchronizes `stream`, then reports and clears the device error word:
  * CCA_ERR_DEVICE_TIMEOUT if a bounded wait in a kernel gave up since the last
  * poll, CCA_ERR_NUMERIC_RANGE if a finite fp16 intermediate overflowed (its
