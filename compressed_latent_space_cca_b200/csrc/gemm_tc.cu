@@ -21,13 +21,26 @@
 namespace cca {
 namespace {
 
-constexpr int BM = 128, BN = 256, BK = 64, STAGES = 4;
-constexpr int A_BYTES = BM * BK * 2;  // 16 KB
-constexpr int B_BYTES = BN * BK * 2;  // 32 KB
-constexpr int STAGE_BYTES = A_BYTES + B_BYTES;
-constexpr int NUM_THREADS = 192;
-constexpr int TMEM_COLS = 512;  // two 128 x 256 fp32 accumulators
-constexpr size_t SMEM_BYTES = (size_t)STAGES * STAGE_BYTES + 1024 /*align slack*/ + 256 /*barriers*/;
+constexpr int BN = 256, BK = 64;
+constexpr int A_HALF_BYTES = 128 * BK * 2;  // 128 rows of A, 16 KB
+constexpr int B_BYTES = BN * BK * 2;        // 32 KB
+constexpr int TMEM_COLS = 512;
+
+// Two tile shapes. MH = 1: 128 x 256 tiles, 4 stages of 48 KB, two 256-column accumulators so the
+// epilogue of one tile overlaps the main loop of the next. MH = 2: 256 x 256 tiles (two 128-row
+// MMAs per K step share the B tile, so the operands cross from L2 a third less often per flop),
+// 3 stages of 64 KB, one accumulator pair filling all 512 columns, eight epilogue warps.
+template <int MH>
+struct Shape {
+  static constexpr int BM = 128 * MH;
+  static constexpr int STAGES = MH == 1 ? 4 : 3;
+  static constexpr int A_BYTES = A_HALF_BYTES * MH;
+  static constexpr int STAGE_BYTES = A_BYTES + B_BYTES;
+  static constexpr int ACC_BUFS = MH == 1 ? 2 : 1;
+  static constexpr int EPI_WARPS = 4 * MH;
+  static constexpr int NUM_THREADS = 64 + 32 * EPI_WARPS;
+  static constexpr size_t SMEM_BYTES = (size_t)STAGES * STAGE_BYTES + 1024 /*align slack*/ + 256 /*barriers*/;
+};
 
 struct GemmMaps {
   CUtensorMap a;
@@ -78,15 +91,19 @@ __device__ __forceinline__ bool store_row_chunk(const GemmParams& p, long long r
   return bad;
 }
 
-__global__ void __launch_bounds__(NUM_THREADS, 1) gemm_tc_kernel(const __grid_constant__ GemmMaps maps,
-                                                                 const GemmParams p) {
+template <int MH>
+__global__ void __launch_bounds__(Shape<MH>::NUM_THREADS, 1) gemm_tc_kernel(const __grid_constant__ GemmMaps maps,
+                                                                           const GemmParams p) {
+  using T = Shape<MH>;
+  constexpr int BM = T::BM, STAGES = T::STAGES, STAGE_BYTES = T::STAGE_BYTES, A_BYTES = T::A_BYTES;
+  constexpr int ACC_BUFS = T::ACC_BUFS;
   extern __shared__ uint8_t smem_raw[];
   uint8_t* smem = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
   uint64_t* bars = reinterpret_cast<uint64_t*>(smem + STAGES * STAGE_BYTES);
   uint64_t* full = bars;                 // [STAGES] TMA -> MMA
   uint64_t* empty = bars + STAGES;       // [STAGES] MMA -> TMA
-  uint64_t* tfull = bars + 2 * STAGES;   // [2] MMA -> epilogue
-  uint64_t* tempty = bars + 2 * STAGES + 2;  // [2] epilogue -> MMA
+  uint64_t* tfull = bars + 2 * STAGES;   // [ACC_BUFS] MMA -> epilogue
+  uint64_t* tempty = bars + 2 * STAGES + 2;  // [ACC_BUFS] epilogue -> MMA
   uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(bars + 2 * STAGES + 4);
   volatile int* abort_flag = reinterpret_cast<volatile int*>(tmem_slot + 1);
 
@@ -96,9 +113,9 @@ __global__ void __launch_bounds__(NUM_THREADS, 1) gemm_tc_kernel(const __grid_co
       mbar_init(smem_u32(&full[s]), 1);
       mbar_init(smem_u32(&empty[s]), 1);
     }
-    for (int a = 0; a < 2; ++a) {
+    for (int a = 0; a < ACC_BUFS; ++a) {
       mbar_init(smem_u32(&tfull[a]), 1);
-      mbar_init(smem_u32(&tempty[a]), 4);
+      mbar_init(smem_u32(&tempty[a]), T::EPI_WARPS);
     }
     *abort_flag = 0;
     fence_mbar_init();
@@ -130,7 +147,8 @@ __global__ void __launch_bounds__(NUM_THREADS, 1) gemm_tc_kernel(const __grid_co
           const uint32_t fb = smem_u32(&full[stage]);
           mbar_arrive_expect_tx(fb, STAGE_BYTES);
           uint8_t* sa = smem + stage * STAGE_BYTES;
-          tma_load_2d(smem_u32(sa), &maps.a, fb, kb * BK, m0);
+#pragma unroll
+          for (int h = 0; h < MH; ++h) tma_load_2d(smem_u32(sa + h * A_HALF_BYTES), &maps.a, fb, kb * BK, m0 + h * 128);
 #pragma unroll
           for (int h = 0; h < 2; ++h) {
             const int row = n0 + h * 128;
@@ -153,7 +171,7 @@ __global__ void __launch_bounds__(NUM_THREADS, 1) gemm_tc_kernel(const __grid_co
   } else if (warp == 1) {
     if (lane == 0) {
       // ------------------------------------------------------ MMA issuer --
-      const uint32_t idesc = idesc_f32acc(BM, BN, 0, 0, p.in_fmt);
+      const uint32_t idesc = idesc_f32acc(128, BN, 0, 0, p.in_fmt);
       // descriptors built once; a stage step adds STAGE_BYTES / 16 to the start address, a K = 16 step 2
       const uint32_t d_hi = desc_hi(smem_desc_sw128(smem_u32(smem), 16, 1024));
       const uint32_t a_lo0 = desc_lo(smem_desc_sw128(smem_u32(smem), 16, 1024));
@@ -161,8 +179,8 @@ __global__ void __launch_bounds__(NUM_THREADS, 1) gemm_tc_kernel(const __grid_co
       uint32_t phase = 0;
       int i = 0;
       for (int t = blockIdx.x; t < p.num_tiles; t += gridDim.x, ++i) {
-        const int acc = i & 1;
-        const uint32_t tph = (i >> 1) & 1;
+        const int acc = i % ACC_BUFS;
+        const uint32_t tph = (i / ACC_BUFS) & 1;
         if (!mbar_wait_bounded(smem_u32(&tempty[acc]), tph ^ 1, p.err, abort_flag, wait_site(kSiteGemm, 2, 2))) goto mma_done;
         tc_fence_after();
         const uint32_t d_tmem = tmem_base + acc * BN;
@@ -172,7 +190,11 @@ __global__ void __launch_bounds__(NUM_THREADS, 1) gemm_tc_kernel(const __grid_co
           const uint32_t a_lo = a_lo0 + stage * (STAGE_BYTES >> 4);
           const uint32_t b_lo = a_lo + (A_BYTES >> 4);
 #pragma unroll
-          for (int k = 0; k < BK / 16; ++k) umma_ss_lohi(d_tmem, a_lo + 2 * k, d_hi, b_lo + 2 * k, d_hi, idesc, (kb | k) != 0);
+          for (int k = 0; k < BK / 16; ++k)
+#pragma unroll
+            for (int h = 0; h < MH; ++h)  // rows h*128.. of the tile -> accumulator columns h*256..
+              umma_ss_lohi(d_tmem + h * BN, a_lo + h * (A_HALF_BYTES >> 4) + 2 * k, d_hi, b_lo + 2 * k, d_hi, idesc,
+                           (kb | k) != 0);
           umma_commit(smem_u32(&empty[stage]));
           if (++stage == STAGES) {
             stage = 0;
@@ -185,24 +207,26 @@ __global__ void __launch_bounds__(NUM_THREADS, 1) gemm_tc_kernel(const __grid_co
     }
   } else {
     // --------------------------------------------------------- epilogue --
-    const int quad = warp & 3;  // this warp may touch TMEM lanes [32*quad, 32*quad+32)
+    const int quad = warp & 3;        // this warp may touch TMEM lanes [32*quad, 32*quad+32)
+    const int half = (warp - 2) / 4;  // MH = 2: which 128-row half of the tile (accumulator columns half*256..)
     bool bad = false;
     int i = 0;
     for (int t = blockIdx.x; t < p.num_tiles; t += gridDim.x, ++i) {
-      const int acc = i & 1;
-      const uint32_t tph = (i >> 1) & 1;
+      const int acc = i % ACC_BUFS;
+      const uint32_t tph = (i / ACC_BUFS) & 1;
       if (!mbar_wait_bounded(smem_u32(&tfull[acc]), tph, p.err, abort_flag, wait_site(kSiteGemm, 3, 4))) break;
       tc_fence_after();
       const long long m0 = (long long)(t / p.n_tiles_n) * BM;
       const int n0 = (t % p.n_tiles_n) * BN;
-      const long long row = m0 + quad * 32 + lane;
+      const long long row = m0 + half * 128 + quad * 32 + lane;
+      const uint32_t col0 = tmem_base + ((uint32_t)(quad * 32) << 16) + (acc + half) * BN;
 #pragma unroll 1
       for (int c = 0; c < BN / 32; ++c) {
         uint32_t r[32];
-        tmem_ld_32x32b_x32(tmem_base + ((uint32_t)(quad * 32) << 16) + acc * BN + c * 32, r);
+        tmem_ld_32x32b_x32(col0 + c * 32, r);
         tmem_ld_wait();
-        const int col0 = n0 + c * 32;
-        if (row < p.M && col0 < p.N) bad |= store_row_chunk(p, row, col0, r);
+        const int col = n0 + c * 32;
+        if (row < p.M && col < p.N) bad |= store_row_chunk(p, row, col, r);
       }
       tc_fence_before();
       __syncwarp();
@@ -248,7 +272,7 @@ cudaError_t launch_gemm_tc(const GemmTcArgs& a, cudaStream_t stream) {
       a.in == DType::F16 ? CU_TENSOR_MAP_DATA_TYPE_FLOAT16 : CU_TENSOR_MAP_DATA_TYPE_BFLOAT16;
   GemmMaps maps;
   GemmParams p{};
-  if (!encode_2d(&maps.a, a.A, dt, (uint64_t)a.K, (uint64_t)a.M, BK, BM)) return cudaErrorInvalidValue;
+  if (!encode_2d(&maps.a, a.A, dt, (uint64_t)a.K, (uint64_t)a.M, BK, 128)) return cudaErrorInvalidValue;
   int start = 0;
   for (int i = 0; i < 3; ++i) {
     const int src = i < a.nb ? i : 0;
@@ -268,12 +292,24 @@ cudaError_t launch_gemm_tc(const GemmTcArgs& a, cudaStream_t stream) {
   p.in_fmt = a.in == DType::F16 ? kFmtF16 : kFmtBF16;
   p.err = a.dev_err;
   p.n_tiles_n = (N + BN - 1) / BN;
+  // 256-row tiles when the main loop is long enough to carry the epilogue it cannot overlap
+  const bool big = a.K >= 1024 && a.M >= 256;
+  const int BM = big ? 256 : 128;
   const long long m_tiles = (a.M + BM - 1) / BM;
   p.num_tiles = (int)(m_tiles * p.n_tiles_n);
   const int grid = p.num_tiles < num_sms() ? p.num_tiles : num_sms();
-  cudaError_t e = cudaFuncSetAttribute(gemm_tc_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)SMEM_BYTES);
-  if (e != cudaSuccess) return e;
-  gemm_tc_kernel<<<grid, NUM_THREADS, SMEM_BYTES, stream>>>(maps, p);
+  cudaError_t e;
+  if (big) {
+    if ((e = cudaFuncSetAttribute(gemm_tc_kernel<2>, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                                  (int)Shape<2>::SMEM_BYTES)) != cudaSuccess)
+      return e;
+    gemm_tc_kernel<2><<<grid, Shape<2>::NUM_THREADS, Shape<2>::SMEM_BYTES, stream>>>(maps, p);
+  } else {
+    if ((e = cudaFuncSetAttribute(gemm_tc_kernel<1>, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                                  (int)Shape<1>::SMEM_BYTES)) != cudaSuccess)
+      return e;
+    gemm_tc_kernel<1><<<grid, Shape<1>::NUM_THREADS, Shape<1>::SMEM_BYTES, stream>>>(maps, p);
+  }
   return cudaGetLastError();
 }
 
