@@ -81,21 +81,25 @@ __device__ __forceinline__ void mma_bf16_16816(float* c, uint32_t a0, uint32_t a
       : "r"(a0), "r"(a1), "r"(a2), "r"(a3), "r"(b0), "r"(b1));
 }
 
-// Causal depthwise seq conv of one staged head into the bf16 hi / lo tiles.
+// Causal depthwise seq conv of one staged head into the bf16 hi / lo tiles. KC: the number of
+// taps when known at compile time (0: p.K taps, at most KMAX).
+template <int KC>
 __device__ __forceinline__ void seq_conv(const PreParams& p, const __half* zbuf, __nv_bfloat16* shi,
                                          __nv_bfloat16* slo, const __nv_bfloat16* wseq) {
+  constexpr int KN = KC > 0 ? KC : KMAX;
+  const int K = KC > 0 ? KC : p.K;
   const int cp = threadIdx.x % (D / 2);  // column pair
-  float w0[KMAX], w1[KMAX];
+  float w0[KN], w1[KN];
 #pragma unroll
-  for (int j = 0; j < KMAX; ++j) {
-    w0[j] = j < p.K ? __bfloat162float(wseq[(2 * cp) * p.K + j]) : 0.f;
-    w1[j] = j < p.K ? __bfloat162float(wseq[(2 * cp + 1) * p.K + j]) : 0.f;
+  for (int j = 0; j < KN; ++j) {
+    w0[j] = j < K ? __bfloat162float(wseq[(2 * cp) * K + j]) : 0.f;
+    w1[j] = j < K ? __bfloat162float(wseq[(2 * cp + 1) * K + j]) : 0.f;
   }
   for (int t = threadIdx.x / (D / 2); t < TT; t += NT / (D / 2)) {
     float a0 = 0.f, a1 = 0.f;
 #pragma unroll
-    for (int j = 0; j < KMAX; ++j) {
-      if (j < p.K) {
+    for (int j = 0; j < KN; ++j) {
+      if (j < K) {
         const float2 z = __half22float2(*reinterpret_cast<const __half2*>(zbuf + (t + j) * ROWH + 2 * cp));
         a0 = fmaf(w0[j], z.x, a0);
         a1 = fmaf(w1[j], z.y, a1);
@@ -149,12 +153,14 @@ __device__ __forceinline__ void load_weights_async(const __nv_bfloat16* W, __nv_
   }
 }
 
+template <int KC>
 __global__ void __launch_bounds__(NT, 2) preproc_tc_kernel(const __grid_constant__ PreParams p,
                                                           const __grid_constant__ Theta th) {
   extern __shared__ __align__(16) uint8_t smem_raw[];
   const int G = p.nq / p.nkv;
   const int H1 = G + 1;
-  const int ZR = TT + p.K - 1;  // staged rows per head
+  const int KK = KC > 0 ? KC : p.K;  // seq-conv taps
+  const int ZR = TT + KK - 1;        // staged rows per head
   __nv_bfloat16* wbuf = reinterpret_cast<__nv_bfloat16*>(smem_raw);  // [D][ROWH] channel weights
   __nv_bfloat16* shi = wbuf + D * ROWH;                               // [TT][ROWH] s, bf16 high part
   __nv_bfloat16* slo = shi + TT * ROWH;                               // [TT][ROWH] s, bf16 low part
@@ -171,13 +177,13 @@ __global__ void __launch_bounds__(NT, 2) preproc_tc_kernel(const __grid_constant
   const int ncol[4] = {cg * 16, cg * 16 + 8, 64 + cg * 16, 64 + cg * 16 + 8};
   const int r0 = rb + (lane >> 2), r1 = r0 + 8;
   const int cq = (lane & 3) * 2;
-  const int zr0 = r0 + p.K - 1, zr1 = r1 + p.K - 1;  // current-token rows in the latent tiles
+  const int zr0 = r0 + KK - 1, zr1 = r1 + KK - 1;  // current-token rows in the latent tiles
   bool bad = false;
 
   // ---- all latents of the group (query heads 0..G-1, then the K head) and the K head's weights
   for (int e = threadIdx.x; e < H1 * ZR * (D / 8); e += NT) {
     const int hh = e / (ZR * (D / 8)), rem = e % (ZR * (D / 8)), r = rem / (D / 8), v = rem % (D / 8);
-    const int t = t0 - (p.K - 1) + r;
+    const int t = t0 - (KK - 1) + r;
     const int col = (hh < G) ? (g * G + hh) * D : Lq + g * D;
     const bool ok = t >= 0 && t < p.S;
     cp_async16(smem_u32(zall + (hh * ZR + r) * ROWH + v * 8), p.lat + (rowbase + (ok ? t : 0)) * Nlat + col + v * 8,
@@ -215,14 +221,15 @@ __global__ void __launch_bounds__(NT, 2) preproc_tc_kernel(const __grid_constant
         v[nt + 2][e] = x2 * rc[nt][e] + x1 * rs[nt][e];
       }
   };
-  auto zval = [&](int hh, int nt, int e) -> float {
-    return __half2float(zall[(hh * ZR + ((e < 2) ? zr0 : zr1)) * ROWH + ncol[nt] + cq + (e & 1)]);
+  // latents of head hh at this thread's two adjacent columns of n-tile nt, row r0 (rs = 0) or r1
+  auto zpair = [&](int hh, int nt, int rs) -> float2 {
+    return __half22float2(*reinterpret_cast<const __half2*>(zall + (hh * ZR + (rs ? zr1 : zr0)) * ROWH + ncol[nt] + cq));
   };
 
   // ---- the K head: conv + channel mix, c_k kept in registers
   cp_async_wait_all();
   __syncthreads();
-  seq_conv(p, zall + G * ZR * ROWH, shi, slo, p.ck_seq + (long long)g * D * p.K);
+  seq_conv<KC>(p, zall + G * ZR * ROWH, shi, slo, p.ck_seq + (long long)g * D * KK);
   __syncthreads();
   float ck[4][4];
   channel_mix(shi, slo, wbuf, rb, ncol, ck);
@@ -237,7 +244,7 @@ __global__ void __launch_bounds__(NT, 2) preproc_tc_kernel(const __grid_constant
     const int h = g * G + hh;
     __syncthreads();  // wbuf, shi, slo are free
     load_weights_async(p.cq_chan + (long long)h * D * D, wbuf);
-    seq_conv(p, zall + hh * ZR * ROWH, shi, slo, p.cq_seq + (long long)h * D * p.K);
+    seq_conv<KC>(p, zall + hh * ZR * ROWH, shi, slo, p.cq_seq + (long long)h * D * KK);
     cp_async_wait_all();
     __syncthreads();
     float acc[4][4];
@@ -245,12 +252,20 @@ __global__ void __launch_bounds__(NT, 2) preproc_tc_kernel(const __grid_constant
 #pragma unroll
     for (int nt = 0; nt < 4; ++nt)
 #pragma unroll
-      for (int e = 0; e < 4; ++e) {
-        float v = acc[nt][e];
-        if (p.mode & 1) v += 0.5f * (zval(hh, nt, e) + zval(G, nt, e));
-        if (p.mode & 2) v += 0.5f * (acc[nt][e] + ck[nt][e]);
-        csum[nt][e] += acc[nt][e];
-        acc[nt][e] = v;
+      for (int rs = 0; rs < 2; ++rs) {
+        float2 pre = make_float2(0.f, 0.f);
+        if (p.mode & 1) {
+          const float2 zq = zpair(hh, nt, rs), zk = zpair(G, nt, rs);
+          pre = make_float2(0.5f * (zq.x + zk.x), 0.5f * (zq.y + zk.y));
+        }
+#pragma unroll
+        for (int e1 = 0; e1 < 2; ++e1) {
+          const int e = 2 * rs + e1;
+          float v = acc[nt][e] + (e1 ? pre.y : pre.x);
+          if (p.mode & 2) v += 0.5f * (acc[nt][e] + ck[nt][e]);
+          csum[nt][e] += acc[nt][e];
+          acc[nt][e] = v;
+        }
       }
     if (p.use_rope) rope(acc);
     __syncthreads();  // shi becomes the q stage
@@ -278,15 +293,25 @@ __global__ void __launch_bounds__(NT, 2) preproc_tc_kernel(const __grid_constant
 #pragma unroll
     for (int nt = 0; nt < 4; ++nt)
 #pragma unroll
-      for (int e = 0; e < 4; ++e) {
-        float v = ck[nt][e];
+      for (int rs = 0; rs < 2; ++rs) {
+        float2 pre = make_float2(0.f, 0.f);
         if (p.mode & 1) {
-          float mq = 0.f;
-          for (int hh = 0; hh < G; ++hh) mq += zval(hh, nt, e);
-          v += 0.5f * (mq * invG + zval(G, nt, e));
+          float2 mq = make_float2(0.f, 0.f);
+          for (int hh = 0; hh < G; ++hh) {
+            const float2 z = zpair(hh, nt, rs);
+            mq.x += z.x;
+            mq.y += z.y;
+          }
+          const float2 zk = zpair(G, nt, rs);
+          pre = make_float2(0.5f * (mq.x * invG + zk.x), 0.5f * (mq.y * invG + zk.y));
         }
-        if (p.mode & 2) v += 0.5f * (csum[nt][e] * invG + ck[nt][e]);
-        val[nt][e] = v;
+#pragma unroll
+        for (int e1 = 0; e1 < 2; ++e1) {
+          const int e = 2 * rs + e1;
+          float v = ck[nt][e] + (e1 ? pre.y : pre.x);
+          if (p.mode & 2) v += 0.5f * (csum[nt][e] * invG + ck[nt][e]);
+          val[nt][e] = v;
+        }
       }
     if (p.use_rope) rope(val);
     __syncthreads();  // wbuf becomes the k stage
@@ -395,10 +420,11 @@ cudaError_t launch_preproc_tc(const BlockDims& dm, const BlockPtrs& p, cudaStrea
   Theta th;
   for (int i = 0; i < D / 2; ++i) th.v[i] = pow((double)dm.rope_base, -2.0 * (double)i / (double)D);
   const size_t smem = smem_bytes(dm.G, dm.K);
-  cudaError_t e = cudaFuncSetAttribute(preproc_tc_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
-  if (e != cudaSuccess) return e;
   dim3 grid((dm.S + TT - 1) / TT, dm.nkv, dm.B);
-  preproc_tc_kernel<<<grid, NT, smem, stream>>>(q, th);
+  auto kern = dm.K == 4 ? preproc_tc_kernel<4> : preproc_tc_kernel<0>;
+  cudaError_t e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
+  if (e != cudaSuccess) return e;
+  kern<<<grid, NT, smem, stream>>>(q, th);
   return cudaGetLastError();
 }
 
