@@ -11,9 +11,11 @@
 //
 // One CTA = 32 tokens of one sequence x one KV group (its G query heads and
 // its K/V head). The fp16 latents of all G+1 heads (32 tokens plus a K-1
-// token halo) arrive in shared memory by cp.async. Per head, the head's bf16
-// channel-mix weights stream in by cp.async, the causal seq conv runs on CUDA
-// cores in fp32, and its output s is split into bf16 s_hi + s_lo so that the
+// token halo) arrive in shared memory by cp.async, with the seq-conv taps of
+// all G+1 heads. The heads' bf16 channel-mix weights stream in by cp.async
+// through two buffers, so the next head's weights load while the current head
+// is mixed. Per head the causal seq conv runs on CUDA cores in fp32, and its
+// output s is split into bf16 s_hi + s_lo so that the
 // 32x128x128 channel mix runs on the tensor cores (mma.sync m16n8k16 bf16,
 // fp32 accumulate, two products per step) on the exact bf16 weights with a
 // relative error near 2^-18. Each thread owns the same accumulator positions
@@ -21,9 +23,10 @@
 // columns come in pairs (c, c+64), so RoPE is applied in registers. Output
 // tiles are staged in shared memory and written with 16-byte coalesced
 // stores: q (fp16), the bf16 K cache and the fp16 attention copy of k; then
-// the value shift copies v (bf16 cache and fp16 attention copy). Every
-// shared-memory row is padded to 272 bytes, which keeps ldmatrix, the
-// per-thread reads and the staging stores free of bank conflicts.
+// the value shift copies v (bf16 cache and fp16 attention copy). Latent and s
+// rows are padded to 272 bytes and weight rows are XOR-swizzled in 16-byte
+// chunks, which keeps ldmatrix, the per-thread reads and the staging stores
+// free of bank conflicts while two CTAs still fit on one SM.
 #include <math.h>
 
 #include "cca_common.cuh"
@@ -38,6 +41,7 @@ constexpr int NT = 256;         // threads
 constexpr int KMAX = 8;         // largest seq-conv kernel of this path
 constexpr int GMAX = 8;         // largest group (query heads per KV head) of this path
 constexpr int ROWH = D + 8;     // padded row, in 16-bit elements (272 bytes)
+constexpr int WTILE = D * D;    // one head's channel weights, unpadded (swizzled) rows
 constexpr int ZROWS = TT + KMAX - 1;
 constexpr int KSTR = D + 4;     // padded fp32 row of the k stage
 
@@ -56,14 +60,18 @@ struct PreParams {
   long long wo_n;
   unsigned* err;
   int S, nq, nkv, K, mode, vshift, use_rope;
+  int nbuf;  // weight buffers in shared memory: 2 (next head's weights prefetched) or 1
 };
 
 __device__ __forceinline__ void cp_async16(uint32_t dst, const void* src, bool valid) {
   const int n = valid ? 16 : 0;  // 0 source bytes: the 16 destination bytes are zero-filled
   asm volatile("cp.async.cg.shared.global [%0], [%1], 16, %2;" ::"r"(dst), "l"(src), "r"(n) : "memory");
 }
-__device__ __forceinline__ void cp_async_wait_all() {
-  asm volatile("cp.async.commit_group;\ncp.async.wait_group 0;" ::: "memory");
+__device__ __forceinline__ void cp_async_commit() { asm volatile("cp.async.commit_group;" ::: "memory"); }
+// wait until at most N of this thread's committed cp.async groups are pending
+template <int N>
+__device__ __forceinline__ void cp_async_wait() {
+  asm volatile("cp.async.wait_group %0;" ::"n"(N) : "memory");
 }
 
 __device__ __forceinline__ void ldsm_x4(uint32_t addr, uint32_t& r0, uint32_t& r1, uint32_t& r2, uint32_t& r3) {
@@ -85,7 +93,7 @@ __device__ __forceinline__ void mma_bf16_16816(float* c, uint32_t a0, uint32_t a
 // taps when known at compile time (0: p.K taps, at most KMAX).
 template <int KC>
 __device__ __forceinline__ void seq_conv(const PreParams& p, const __half* zbuf, __nv_bfloat16* shi,
-                                         __nv_bfloat16* slo, const __nv_bfloat16* wseq) {
+                                         __nv_bfloat16* slo, const __nv_bfloat16* wseq /* shared [D][K] */) {
   constexpr int KN = KC > 0 ? KC : KMAX;
   const int K = KC > 0 ? KC : p.K;
   const int cp = threadIdx.x % (D / 2);  // column pair
@@ -124,16 +132,23 @@ __device__ __forceinline__ void channel_mix(const __nv_bfloat16* shi, const __nv
     for (int e = 0; e < 4; ++e) acc[nt][e] = 0.f;
   const int arow = (rb + (lane & 15)) * ROWH + (lane >> 4) * 8;
   const uint32_t ahi = smem_u32(shi + arow), alo = smem_u32(slo + arow);
-  const int m = lane >> 3, rr = lane & 7;
-  const uint32_t b0base = smem_u32(wbuf + (ncol[0] + (m >> 1) * 8 + rr) * ROWH + (m & 1) * 8);
-  const uint32_t b1base = smem_u32(wbuf + (ncol[2] + (m >> 1) * 8 + rr) * ROWH + (m & 1) * 8);
+  // B matrix m = lane / 8: rows ncol[0] + (m / 2) * 8 + (lane % 8), k chunk 2 ks + (m % 2), which
+  // sits at chunk (2 ks) ^ y of the swizzled row, y = (m % 2) ^ (row % 8)
+  const int brow = ncol[0] + ((lane >> 4) << 3) + (lane & 7);
+  const int y = ((lane >> 3) & 1) ^ (lane & 7);
+  const uint32_t brow0 = smem_u32(wbuf + brow * D);
+  uint32_t bq[4];
+#pragma unroll
+  for (int j = 0; j < 4; ++j) bq[j] = brow0 + (((2 * j) ^ y) << 4);
+  constexpr uint32_t kB1 = 64 * D * 2;  // rows ncol[2] = ncol[0] + 64
 #pragma unroll
   for (int ks = 0; ks < D / 16; ++ks) {
     uint32_t h0, h1, h2, h3, l0, l1, l2, l3, b0, b1, b2, b3, c0, c1, c2, c3;
+    const uint32_t bk = bq[ks & 3] + (ks >> 2) * 128;
     ldsm_x4(ahi + ks * 32, h0, h1, h2, h3);
     ldsm_x4(alo + ks * 32, l0, l1, l2, l3);
-    ldsm_x4(b0base + ks * 32, b0, b1, b2, b3);
-    ldsm_x4(b1base + ks * 32, c0, c1, c2, c3);
+    ldsm_x4(bk, b0, b1, b2, b3);
+    ldsm_x4(bk + kB1, c0, c1, c2, c3);
     mma_bf16_16816(acc[0], h0, h1, h2, h3, b0, b1);
     mma_bf16_16816(acc[1], h0, h1, h2, h3, b2, b3);
     mma_bf16_16816(acc[2], h0, h1, h2, h3, c0, c1);
@@ -145,11 +160,12 @@ __device__ __forceinline__ void channel_mix(const __nv_bfloat16* shi, const __nv
   }
 }
 
-// Stream one head's channel-mix weights [out i][in j] (bf16) into wbuf rows of ROWH.
+// Stream one head's channel-mix weights [out i][in j] (bf16) into wbuf: row i holds 16 chunks of
+// 8 inputs, chunk c stored at position c ^ (i % 8).
 __device__ __forceinline__ void load_weights_async(const __nv_bfloat16* W, __nv_bfloat16* wbuf) {
   for (int e = threadIdx.x; e < D * (D / 8); e += NT) {
     const int r = e / (D / 8), v = e % (D / 8);
-    cp_async16(smem_u32(wbuf + r * ROWH + v * 8), W + (long long)r * D + v * 8, true);
+    cp_async16(smem_u32(wbuf + r * D + ((v ^ (r & 7)) << 3)), W + (long long)r * D + v * 8, true);
   }
 }
 
@@ -161,12 +177,15 @@ __global__ void __launch_bounds__(NT, 2) preproc_tc_kernel(const __grid_constant
   const int H1 = G + 1;
   const int KK = KC > 0 ? KC : p.K;  // seq-conv taps
   const int ZR = TT + KK - 1;        // staged rows per head
-  __nv_bfloat16* wbuf = reinterpret_cast<__nv_bfloat16*>(smem_raw);  // [D][ROWH] channel weights
-  __nv_bfloat16* shi = wbuf + D * ROWH;                               // [TT][ROWH] s, bf16 high part
+  __nv_bfloat16* wbuf = reinterpret_cast<__nv_bfloat16*>(smem_raw);  // nbuf x [D][D] channel weights
+  __nv_bfloat16* shi = wbuf + p.nbuf * WTILE;                         // [TT][ROWH] s, bf16 high part
   __nv_bfloat16* slo = shi + TT * ROWH;                               // [TT][ROWH] s, bf16 low part
   __half* zall = reinterpret_cast<__half*>(slo + TT * ROWH);          // [H1][ZR][ROWH] latents; head G = k
+  __nv_bfloat16* wsq = reinterpret_cast<__nv_bfloat16*>(zall + H1 * ZR * ROWH);  // [H1][D][K] seq taps
   __half* stage = reinterpret_cast<__half*>(shi);                     // [TT][ROWH] q output stage
   float* kst = reinterpret_cast<float*>(wbuf);                        // [TT][KSTR] k stage (fp32)
+  // weights of the i-th head in processing order (0: the K head, then query heads 0..G-1)
+  auto wslot = [&](int i) { return wbuf + (p.nbuf == 2 ? (i & 1) : 0) * WTILE; };
 
   const int Lq = p.nq * D, Lkv = p.nkv * D, Nlat = Lq + 2 * Lkv;
   const int t0 = blockIdx.x * TT, g = blockIdx.y, b = blockIdx.z;
@@ -189,7 +208,36 @@ __global__ void __launch_bounds__(NT, 2) preproc_tc_kernel(const __grid_constant
     cp_async16(smem_u32(zall + (hh * ZR + r) * ROWH + v * 8), p.lat + (rowbase + (ok ? t : 0)) * Nlat + col + v * 8,
                ok);
   }
-  load_weights_async(p.ck_chan + (long long)g * D * D, wbuf);
+  load_weights_async(p.ck_chan + (long long)g * D * D, wslot(0));
+  cp_async_commit();
+  if (p.nbuf == 2) load_weights_async(p.cq_chan + (long long)g * G * D * D, wslot(1));
+  cp_async_commit();  // (an empty group when nbuf == 1)
+  // seq-conv taps of the group's heads, [H1][D][K]: query heads g*G .. g*G+G-1, then the K head
+  for (int e = threadIdx.x; e < H1 * D * KK; e += NT) {
+    const int hh = e / (D * KK), rem = e % (D * KK);
+    wsq[e] = hh < G ? p.cq_seq[(long long)(g * G + hh) * D * KK + rem] : p.ck_seq[(long long)g * D * KK + rem];
+  }
+
+  // ---- side job, issued while the copies are in flight: this CTA's slice of W_o as fp16 (8-element vectors)
+  {
+    const long long nvec = p.wo_n / 8;
+    const long long nct = (long long)gridDim.x * gridDim.y * gridDim.z;
+    const long long cid = ((long long)blockIdx.z * gridDim.y + blockIdx.y) * gridDim.x + blockIdx.x;
+    const long long chunk = (nvec + nct - 1) / nct;
+    const long long lo = cid * chunk, hi = lo + chunk < nvec ? lo + chunk : nvec;
+    for (long long e = lo + threadIdx.x; e < hi; e += NT) {
+      const uint4 raw = *reinterpret_cast<const uint4*>(p.wo + e * 8);
+      const __nv_bfloat162* b2 = reinterpret_cast<const __nv_bfloat162*>(&raw);
+      uint32_t h[4];
+#pragma unroll
+      for (int k = 0; k < 4; ++k) {
+        const float2 f = __bfloat1622float2(b2[k]);
+        bad |= f16_overflow(f.x) || f16_overflow(f.y);
+        h[k] = pack_f16x2(f.x, f.y);
+      }
+      *reinterpret_cast<uint4*>(p.wo_lat + e * 8) = make_uint4(h[0], h[1], h[2], h[3]);
+    }
+  }
 
   // RoPE factors of this thread's (row, column < 64) positions: [nt<2][e]
   float rc[2][4], rs[2][4];
@@ -227,12 +275,12 @@ __global__ void __launch_bounds__(NT, 2) preproc_tc_kernel(const __grid_constant
   };
 
   // ---- the K head: conv + channel mix, c_k kept in registers
-  cp_async_wait_all();
+  cp_async_wait<1>();  // latents and the K head's weights
   __syncthreads();
-  seq_conv<KC>(p, zall + G * ZR * ROWH, shi, slo, p.ck_seq + (long long)g * D * KK);
+  seq_conv<KC>(p, zall + G * ZR * ROWH, shi, slo, wsq + G * D * KK);
   __syncthreads();
   float ck[4][4];
-  channel_mix(shi, slo, wbuf, rb, ncol, ck);
+  channel_mix(shi, slo, wslot(0), rb, ncol, ck);
   float csum[4][4];
 #pragma unroll
   for (int nt = 0; nt < 4; ++nt)
@@ -242,13 +290,18 @@ __global__ void __launch_bounds__(NT, 2) preproc_tc_kernel(const __grid_constant
   // ---- the G query heads
   for (int hh = 0; hh < G; ++hh) {
     const int h = g * G + hh;
-    __syncthreads();  // wbuf, shi, slo are free
-    load_weights_async(p.cq_chan + (long long)h * D * D, wbuf);
-    seq_conv<KC>(p, zall + hh * ZR * ROWH, shi, slo, p.cq_seq + (long long)h * D * KK);
-    cp_async_wait_all();
+    __syncthreads();  // shi, slo and the previous head's weight buffer are free
+    // weights of query head hh + 1 (double buffering) or hh (single buffer)
+    const int next = p.nbuf == 2 ? hh + 1 : hh;
+    const bool issue = next < G;
+    if (issue) load_weights_async(p.cq_chan + (long long)(g * G + next) * D * D, wslot(next + 1));
+    cp_async_commit();
+    seq_conv<KC>(p, zall + hh * ZR * ROWH, shi, slo, wsq + hh * D * KK);
+    if (p.nbuf == 2) cp_async_wait<1>();  // all but the group just committed: head hh's weights
+    else cp_async_wait<0>();
     __syncthreads();
     float acc[4][4];
-    channel_mix(shi, slo, wbuf, rb, ncol, acc);
+    channel_mix(shi, slo, wslot(hh + 1), rb, ncol, acc);
 #pragma unroll
     for (int nt = 0; nt < 4; ++nt)
 #pragma unroll
@@ -284,6 +337,19 @@ __global__ void __launch_bounds__(NT, 2) preproc_tc_kernel(const __grid_constant
         *reinterpret_cast<uint4*>(p.q + (rowbase + t0 + r) * Lq + (long long)h * D + v * 8) =
             *reinterpret_cast<const uint4*>(stage + r * ROWH + v * 8);
     }
+  }
+
+  // value-shift sources, loaded now so that the latency overlaps the k combine: channels
+  // [Lkv/2, Lkv) come from the previous token (8-channel vectors never straddle the boundary)
+  static_assert(TT * (D / 8) == 2 * NT, "two value vectors per thread");
+  uint4 vsrc[2];
+#pragma unroll
+  for (int i = 0; i < 2; ++i) {
+    const int e = threadIdx.x + i * NT, r = e / (D / 8), v = e % (D / 8);
+    const int t = t0 + r, gc = g * D + v * 8;
+    const int src = (p.vshift && gc >= Lkv / 2) ? t - 1 : t;
+    vsrc[i] = make_uint4(0, 0, 0, 0);
+    if (t < p.S && src >= 0) vsrc[i] = *reinterpret_cast<const uint4*>(p.lat + (rowbase + src) * Nlat + Lq + Lkv + gc);
   }
 
   // ---- k = c_k + means, RoPE; staged in fp32, written as the bf16 cache and the fp16 copy
@@ -337,15 +403,13 @@ __global__ void __launch_bounds__(NT, 2) preproc_tc_kernel(const __grid_constant
         make_uint4(pack_f16x2(lo.x, lo.y), pack_f16x2(lo.z, lo.w), pack_f16x2(hi.x, hi.y), pack_f16x2(hi.z, hi.w));
   }
 
-  // ---- value shift: channels [Lkv/2, Lkv) from the previous token (8-channel vectors never straddle)
-  for (int e = threadIdx.x; e < TT * (D / 8); e += NT) {
-    const int r = e / (D / 8), v = e % (D / 8);
-    const int t = t0 + r;
+  // ---- value shift: the bf16 cache and the fp16 attention copy of the shifted v
+#pragma unroll
+  for (int i = 0; i < 2; ++i) {
+    const int e = threadIdx.x + i * NT, r = e / (D / 8), v = e % (D / 8);
+    const int t = t0 + r, gc = g * D + v * 8;
     if (t >= p.S) continue;
-    const int gc = g * D + v * 8;
-    const int src = (p.vshift && gc >= Lkv / 2) ? t - 1 : t;
-    uint4 hv = make_uint4(0, 0, 0, 0);
-    if (src >= 0) hv = *reinterpret_cast<const uint4*>(p.lat + (rowbase + src) * Nlat + Lq + Lkv + gc);
+    const uint4 hv = vsrc[i];
     const __half2* h2 = reinterpret_cast<const __half2*>(&hv);
     uint32_t hb[4];
 #pragma unroll
@@ -358,33 +422,17 @@ __global__ void __launch_bounds__(NT, 2) preproc_tc_kernel(const __grid_constant
     *reinterpret_cast<uint4*>(p.v_att + off) = hv;
   }
 
-  // ---- side job: this CTA's slice of W_o as fp16 (8-element vectors)
-  {
-    const long long nvec = p.wo_n / 8;
-    const long long nct = (long long)gridDim.x * gridDim.y * gridDim.z;
-    const long long cid = ((long long)blockIdx.z * gridDim.y + blockIdx.y) * gridDim.x + blockIdx.x;
-    const long long chunk = (nvec + nct - 1) / nct;
-    const long long lo = cid * chunk, hi = lo + chunk < nvec ? lo + chunk : nvec;
-    for (long long e = lo + threadIdx.x; e < hi; e += NT) {
-      const uint4 raw = *reinterpret_cast<const uint4*>(p.wo + e * 8);
-      const __nv_bfloat162* b2 = reinterpret_cast<const __nv_bfloat162*>(&raw);
-      uint32_t h[4];
-#pragma unroll
-      for (int k = 0; k < 4; ++k) {
-        const float2 f = __bfloat1622float2(b2[k]);
-        bad |= f16_overflow(f.x) || f16_overflow(f.y);
-        h[k] = pack_f16x2(f.x, f.y);
-      }
-      *reinterpret_cast<uint4*>(p.wo_lat + e * 8) = make_uint4(h[0], h[1], h[2], h[3]);
-    }
-  }
   report_range(bad, p.err);
 }
 
-size_t smem_bytes(int G, int K) {
-  return sizeof(__nv_bfloat16) * ((size_t)D * ROWH + 2 * (size_t)TT * ROWH) +
-         sizeof(__half) * (size_t)(G + 1) * (TT + K - 1) * ROWH;
+size_t smem_bytes(int G, int K, int nbuf) {
+  return sizeof(__nv_bfloat16) * ((size_t)nbuf * WTILE + 2 * (size_t)TT * ROWH) +
+         sizeof(__half) * (size_t)(G + 1) * (TT + K - 1) * ROWH + sizeof(__nv_bfloat16) * (size_t)(G + 1) * D * K;
 }
+
+// Two weight buffers when two CTAs still fit on one SM (228 KB of shared memory, 1 KB reserved per
+// CTA), else one.
+int weight_buffers(int G, int K) { return smem_bytes(G, K, 2) + 1024 <= 114 * 1024 ? 2 : 1; }
 
 }  // namespace
 
@@ -419,7 +467,8 @@ cudaError_t launch_preproc_tc(const BlockDims& dm, const BlockPtrs& p, cudaStrea
   q.use_rope = dm.use_rope;
   Theta th;
   for (int i = 0; i < D / 2; ++i) th.v[i] = pow((double)dm.rope_base, -2.0 * (double)i / (double)D);
-  const size_t smem = smem_bytes(dm.G, dm.K);
+  q.nbuf = weight_buffers(dm.G, dm.K);
+  const size_t smem = smem_bytes(dm.G, dm.K, q.nbuf);
   dim3 grid((dm.S + TT - 1) / TT, dm.nkv, dm.B);
   auto kern = dm.K == 4 ? preproc_tc_kernel<4> : preproc_tc_kernel<0>;
   cudaError_t e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
