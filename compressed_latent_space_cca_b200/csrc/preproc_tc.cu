@@ -90,33 +90,59 @@ __device__ __forceinline__ void mma_bf16_16816(float* c, uint32_t a0, uint32_t a
 }
 
 // Causal depthwise seq conv of one staged head into the bf16 hi / lo tiles. KC: the number of
-// taps when known at compile time (0: p.K taps, at most KMAX).
+// taps when known at compile time (0: p.K taps, at most KMAX). Row t of the output uses staged
+// rows t .. t+K-1 (tap K-1 on the current token).
 template <int KC>
 __device__ __forceinline__ void seq_conv(const PreParams& p, const __half* zbuf, __nv_bfloat16* shi,
                                          __nv_bfloat16* slo, const __nv_bfloat16* wseq /* shared [D][K] */) {
-  constexpr int KN = KC > 0 ? KC : KMAX;
-  const int K = KC > 0 ? KC : p.K;
   const int cp = threadIdx.x % (D / 2);  // column pair
-  float w0[KN], w1[KN];
-#pragma unroll
-  for (int j = 0; j < KN; ++j) {
-    w0[j] = j < K ? __bfloat162float(wseq[(2 * cp) * K + j]) : 0.f;
-    w1[j] = j < K ? __bfloat162float(wseq[(2 * cp + 1) * K + j]) : 0.f;
-  }
-  for (int t = threadIdx.x / (D / 2); t < TT; t += NT / (D / 2)) {
-    float a0 = 0.f, a1 = 0.f;
-#pragma unroll
-    for (int j = 0; j < KN; ++j) {
-      if (j < K) {
-        const float2 z = __half22float2(*reinterpret_cast<const __half2*>(zbuf + (t + j) * ROWH + 2 * cp));
-        a0 = fmaf(w0[j], z.x, a0);
-        a1 = fmaf(w1[j], z.y, a1);
-      }
-    }
+  auto emit = [&](int t, float a0, float a1) {
     const __nv_bfloat162 hi = __floats2bfloat162_rn(a0, a1);
     const float2 hf = __bfloat1622float2(hi);
     *reinterpret_cast<__nv_bfloat162*>(shi + t * ROWH + 2 * cp) = hi;
     *reinterpret_cast<__nv_bfloat162*>(slo + t * ROWH + 2 * cp) = __floats2bfloat162_rn(a0 - hf.x, a1 - hf.y);
+  };
+  auto zrow = [&](int r) { return __half22float2(*reinterpret_cast<const __half2*>(zbuf + r * ROWH + 2 * cp)); };
+  if constexpr (KC > 0) {
+    // each thread: one column pair, TPT consecutive tokens, the last KC latent rows in registers
+    constexpr int TPT = TT / (NT / (D / 2));
+    const int tb = (threadIdx.x / (D / 2)) * TPT;
+    float2 w[KC], win[KC];
+#pragma unroll
+    for (int j = 0; j < KC; ++j)
+      w[j] = make_float2(__bfloat162float(wseq[(2 * cp) * KC + j]), __bfloat162float(wseq[(2 * cp + 1) * KC + j]));
+#pragma unroll
+    for (int j = 0; j + 1 < KC; ++j) win[j] = zrow(tb + j);
+#pragma unroll
+    for (int i = 0; i < TPT; ++i) {
+      win[KC - 1] = zrow(tb + i + KC - 1);
+      float a0 = 0.f, a1 = 0.f;
+#pragma unroll
+      for (int j = 0; j < KC; ++j) fma2(a0, a1, w[j].x, w[j].y, win[j].x, win[j].y, a0, a1);
+      emit(tb + i, a0, a1);
+#pragma unroll
+      for (int j = 0; j + 1 < KC; ++j) win[j] = win[j + 1];
+    }
+  } else {
+    const int K = p.K;
+    float w0[KMAX], w1[KMAX];
+#pragma unroll
+    for (int j = 0; j < KMAX; ++j) {
+      w0[j] = j < K ? __bfloat162float(wseq[(2 * cp) * K + j]) : 0.f;
+      w1[j] = j < K ? __bfloat162float(wseq[(2 * cp + 1) * K + j]) : 0.f;
+    }
+    for (int t = threadIdx.x / (D / 2); t < TT; t += NT / (D / 2)) {
+      float a0 = 0.f, a1 = 0.f;
+#pragma unroll
+      for (int j = 0; j < KMAX; ++j) {
+        if (j < K) {
+          const float2 z = zrow(t + j);
+          a0 = fmaf(w0[j], z.x, a0);
+          a1 = fmaf(w1[j], z.y, a1);
+        }
+      }
+      emit(t, a0, a1);
+    }
   }
 }
 
@@ -163,10 +189,20 @@ __device__ __forceinline__ void channel_mix(const __nv_bfloat16* shi, const __nv
 // Stream one head's channel-mix weights [out i][in j] (bf16) into wbuf: row i holds 16 chunks of
 // 8 inputs, chunk c stored at position c ^ (i % 8).
 __device__ __forceinline__ void load_weights_async(const __nv_bfloat16* W, __nv_bfloat16* wbuf) {
-  for (int e = threadIdx.x; e < D * (D / 8); e += NT) {
-    const int r = e / (D / 8), v = e % (D / 8);
-    cp_async16(smem_u32(wbuf + r * D + ((v ^ (r & 7)) << 3)), W + (long long)r * D + v * 8, true);
-  }
+  // thread: chunk v of rows r, r + 16, ... (r % 8 and so the swizzle stay fixed)
+  const int v = threadIdx.x % (D / 8), r = threadIdx.x / (D / 8);
+  const uint32_t dst = smem_u32(wbuf + r * D + ((v ^ (r & 7)) << 3));
+  const __nv_bfloat16* src = W + r * D + v * 8;
+  constexpr int kRows = NT / (D / 8);
+#pragma unroll
+  for (int k = 0; k < D / kRows; ++k) cp_async16(dst + k * kRows * D * 2, src + k * kRows * D, true);
+}
+
+// Byte offset of the RoPE tables: after the weight buffers, the s tiles, the latents and the seq taps.
+__host__ __device__ __forceinline__ size_t rope_table_offset(int H1, int K, int nbuf) {
+  const size_t end = 2 * ((size_t)nbuf * WTILE + 2 * (size_t)TT * ROWH + (size_t)H1 * (TT + K - 1) * ROWH +
+                          (size_t)H1 * D * K);
+  return (end + 15) & ~(size_t)15;
 }
 
 template <int KC>
@@ -182,6 +218,7 @@ __global__ void __launch_bounds__(NT, 2) preproc_tc_kernel(const __grid_constant
   __nv_bfloat16* slo = shi + TT * ROWH;                               // [TT][ROWH] s, bf16 low part
   __half* zall = reinterpret_cast<__half*>(slo + TT * ROWH);          // [H1][ZR][ROWH] latents; head G = k
   __nv_bfloat16* wsq = reinterpret_cast<__nv_bfloat16*>(zall + H1 * ZR * ROWH);  // [H1][D][K] seq taps
+  float2* rtab = reinterpret_cast<float2*>(smem_raw + rope_table_offset(H1, KK, p.nbuf));  // [2][D/2] RoPE
   __half* stage = reinterpret_cast<__half*>(shi);                     // [TT][ROWH] q output stage
   float* kst = reinterpret_cast<float*>(wbuf);                        // [TT][KSTR] k stage (fp32)
   // weights of the i-th head in processing order (0: the K head, then query heads 0..G-1)
@@ -200,8 +237,8 @@ __global__ void __launch_bounds__(NT, 2) preproc_tc_kernel(const __grid_constant
   bool bad = false;
 
   // ---- all latents of the group (query heads 0..G-1, then the K head) and the K head's weights
-  for (int e = threadIdx.x; e < H1 * ZR * (D / 8); e += NT) {
-    const int hh = e / (ZR * (D / 8)), rem = e % (ZR * (D / 8)), r = rem / (D / 8), v = rem % (D / 8);
+  for (int R = threadIdx.x / (D / 8); R < H1 * ZR; R += NT / (D / 8)) {
+    const int v = threadIdx.x % (D / 8), hh = R / ZR, r = R - hh * ZR;
     const int t = t0 - (KK - 1) + r;
     const int col = (hh < G) ? (g * G + hh) * D : Lq + g * D;
     const bool ok = t >= 0 && t < p.S;
@@ -239,26 +276,23 @@ __global__ void __launch_bounds__(NT, 2) preproc_tc_kernel(const __grid_constant
     }
   }
 
-  // RoPE factors of this thread's (row, column < 64) positions: [nt<2][e]
-  float rc[2][4], rs[2][4];
-#pragma unroll
-  for (int nt = 0; nt < 2; ++nt)
-#pragma unroll
-    for (int e = 0; e < 4; ++e) {
-      const int i = ncol[nt] + cq + (e & 1);
-      const int pos = t0 + ((e < 2) ? r0 : r1);
-      float c = 1.f, s = 0.f;
-      if (p.use_rope) {
-        const double a = (double)pos * th.v[i];
-        // reduce a modulo 2 pi with 2 pi split into a high and a low double
-        const double k = rint(a * 0.15915494309189535);
-        double r = fma(-k, 6.283185307179586, a);
-        r = fma(-k, 2.4492935982947064e-16, r);
-        sincosf((float)r, &s, &c);
-      }
-      rc[nt][e] = c;
-      rs[nt][e] = s;
+  // RoPE tables: rtab[i] = (cos, sin) of t0 * theta_i, rtab[D/2 + i] = (cos, sin) of 8 * theta_i
+  if (p.use_rope && threadIdx.x < D) {
+    const int i = threadIdx.x % (D / 2);
+    float c, sn;
+    if (threadIdx.x < D / 2) {
+      const double a = (double)t0 * th.v[i];
+      // reduce a modulo 2 pi with 2 pi split into a high and a low double
+      const double k = rint(a * 0.15915494309189535);
+      double r = fma(-k, 6.283185307179586, a);
+      r = fma(-k, 2.4492935982947064e-16, r);
+      sincosf((float)r, &sn, &c);
+    } else {
+      sincosf((float)(8.0 * th.v[i]), &sn, &c);  // at most 8 radians
     }
+    rtab[threadIdx.x] = make_float2(c, sn);
+  }
+  float rc[2][4], rs[2][4];  // RoPE factors, filled once the tables are in shared memory
   auto rope = [&](float (&v)[4][4]) {
 #pragma unroll
     for (int nt = 0; nt < 2; ++nt)
@@ -277,6 +311,33 @@ __global__ void __launch_bounds__(NT, 2) preproc_tc_kernel(const __grid_constant
   // ---- the K head: conv + channel mix, c_k kept in registers
   cp_async_wait<1>();  // latents and the K head's weights
   __syncthreads();
+
+  // RoPE factors of this thread's (row, column < 64) positions, [nt<2][e]: the angle of row r0 is
+  // t0 theta + r0 theta (r0 theta < 24 radians, reduced in fp32), row r1 = r0 + 8 adds 8 theta
+#pragma unroll
+  for (int nt = 0; nt < 2; ++nt)
+#pragma unroll
+    for (int e1 = 0; e1 < 2; ++e1) {
+      const int i = ncol[nt] + cq + e1;
+      float c0 = 1.f, s0 = 0.f, c1 = 1.f, s1 = 0.f;
+      if (p.use_rope) {
+        const float a = (float)((double)r0 * th.v[i]);
+        const float k = rintf(a * 0.15915494f);
+        float r = fmaf(-k, 6.28318548f, a);  // 2 pi = 6.28318548f - 1.7484555e-7f
+        r = fmaf(k, 1.7484555e-7f, r);
+        float ca, sa;
+        __sincosf(r, &sa, &ca);
+        const float2 b = rtab[i], d8 = rtab[D / 2 + i];
+        c0 = b.x * ca - b.y * sa;
+        s0 = b.y * ca + b.x * sa;
+        c1 = c0 * d8.x - s0 * d8.y;
+        s1 = s0 * d8.x + c0 * d8.y;
+      }
+      rc[nt][e1] = c0;
+      rs[nt][e1] = s0;
+      rc[nt][2 + e1] = c1;
+      rs[nt][2 + e1] = s1;
+    }
   seq_conv<KC>(p, zall + G * ZR * ROWH, shi, slo, wsq + G * D * KK);
   __syncthreads();
   float ck[4][4];
@@ -425,10 +486,7 @@ __global__ void __launch_bounds__(NT, 2) preproc_tc_kernel(const __grid_constant
   report_range(bad, p.err);
 }
 
-size_t smem_bytes(int G, int K, int nbuf) {
-  return sizeof(__nv_bfloat16) * ((size_t)nbuf * WTILE + 2 * (size_t)TT * ROWH) +
-         sizeof(__half) * (size_t)(G + 1) * (TT + K - 1) * ROWH + sizeof(__nv_bfloat16) * (size_t)(G + 1) * D * K;
-}
+size_t smem_bytes(int G, int K, int nbuf) { return rope_table_offset(G + 1, K, nbuf) + sizeof(float2) * D; }
 
 // Two weight buffers when two CTAs still fit on one SM (228 KB of shared memory, 1 KB reserved per
 // CTA), else one.
