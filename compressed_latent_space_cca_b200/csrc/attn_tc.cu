@@ -49,7 +49,10 @@ constexpr int OFF_K = 2 * TILE_BYTES;
 constexpr int OFF_V = OFF_K + K_STAGES * TILE_BYTES;
 constexpr int OFF_BAR = OFF_V + V_STAGES * TILE_BYTES;
 constexpr int MAX_CTAS = 160;
-constexpr int MAX_LIST = 4096;  // pairs a host schedule can hold in the kernel parameters
+constexpr int MAX_LIST = 4096;  // entries a host schedule can hold in the kernel parameters
+// A partial result of one 128-row tile: O as [d / 4][128 rows][4] fp32 (a warp's 16-byte accesses to
+// one column quad cover 512 contiguous bytes), then the running max [128] and sum [128].
+constexpr int PART_TILE = D * TQ + 2 * TQ;  // floats
 constexpr size_t SMEM_BYTES = OFF_BAR + 256 + 1024;
 
 __device__ __forceinline__ float max3f(float a, float b, float c) {
@@ -96,22 +99,34 @@ struct AttnParams {
   float scale_log2;  // softmax scale * log2(e)
   __half* o;
   unsigned* err;
+  // split key ranges: pairs 0 .. nsplit-1 (the longest) run as two halves on any CTAs; each half
+  // leaves its unnormalised O, max and sum in part, and the second to finish merges them
+  int nsplit;
+  int* split_cnt;  // [nsplit][2 tiles][4 lane quadrants], zero at launch
+  float* part;     // [nsplit][2 halves][2 tiles][PART_TILE]
 };
 
-// Per-CTA work lists: CTA c runs items[off[c] .. off[c+1]).
+// Per-CTA work lists: CTA c runs items[off[c] .. off[c+1]). An entry is a pair index in its low 12
+// bits and, in bits 12-13, 0 for the whole key range or 1 / 2 for its first / second half.
 struct AttnSched {
   int use;  // 0: serpentine order instead
   unsigned short off[MAX_CTAS + 1];
   unsigned short items[MAX_LIST];
 };
+constexpr int kEntryPairBits = 12;
 
 struct Item {
   int b, g, nkv_tiles;
+  int k0, k1;  // key tiles [k0, k1) of this entry
+  int half;    // 0 whole range, 1 / 2 first / second half of a split pair
+  int w;       // pair index
   int h[2], qt[2];
   bool active[2];
 };
 
-__device__ __forceinline__ Item get_item(const AttnParams& p, int w) {
+// `entry`: pair index in bits [0, 24), half (0, 1, 2) above.
+__device__ __forceinline__ Item get_item(const AttnParams& p, int entry) {
+  const int w = entry & 0xffffff;
   const int bgc = p.B * p.nkv;
   const int pr = p.pairs - 1 - w / bgc;  // longest pairs first
   const int bg = w % bgc;
@@ -129,14 +144,21 @@ __device__ __forceinline__ Item get_item(const AttnParams& p, int w) {
     it.h[j] = it.g * p.G + uu % p.G;
     if (it.active[j] && it.qt[j] + 1 > it.nkv_tiles) it.nkv_tiles = it.qt[j] + 1;
   }
+  it.w = w;
+  it.half = entry >> 24;
+  const int hsplit = it.nkv_tiles / 2;  // split pairs have at least 4 key tiles
+  it.k0 = it.half == 2 ? hsplit : 0;
+  it.k1 = it.half == 1 ? hsplit : it.nkv_tiles;
   return it;
 }
 
-// Work item of this CTA in round r, or -1 when it has none left.
+// Work item of this CTA in round r (pair index | half << 24), or -1 when it has none left.
 __device__ __forceinline__ int item_index(const AttnSched& sc, int items, int r, int cta, int grid) {
   if (sc.use) {
     const int i = sc.off[cta] + r;
-    return i < sc.off[cta + 1] ? (int)sc.items[i] : -1;
+    if (i >= sc.off[cta + 1]) return -1;
+    const int e = sc.items[i];
+    return (e & ((1 << kEntryPairBits) - 1)) | ((e >> kEntryPairBits) << 24);
   }
   const int w = r * grid + ((r & 1) ? (grid - 1 - cta) : cta);  // serpentine over the CTAs
   return w < items ? w : -1;
@@ -228,9 +250,9 @@ __global__ void __launch_bounds__(NUM_THREADS, 1) attn_tc_kernel(const __grid_co
           }
           return true;
         };
-        if (!load_k(0)) goto done;
-        for (int jj = 0; jj < it.nkv_tiles; ++jj) {
-          if (jj + 1 < it.nkv_tiles && !load_k(jj + 1)) goto done;
+        if (!load_k(it.k0)) goto done;
+        for (int jj = it.k0; jj < it.k1; ++jj) {
+          if (jj + 1 < it.k1 && !load_k(jj + 1)) goto done;
           if (!mbar_wait_bounded(smem_u32(&v_empty[vst]), vph ^ 1, p.err, abort_flag, wait_site(kSiteAttn, 1, 3))) goto done;
           mbar_arrive_expect_tx(smem_u32(&v_full[vst]), TILE_BYTES);
 #pragma unroll
@@ -290,7 +312,7 @@ __global__ void __launch_bounds__(NUM_THREADS, 1) attn_tc_kernel(const __grid_co
           kst = 0;
           kph ^= 1;
         }
-        for (int jj = 0; jj < it.nkv_tiles; ++jj) {
+        for (int jj = it.k0; jj < it.k1; ++jj) {
           bool next_k_ready = false;
           if (!mbar_wait_bounded(smem_u32(&v_full[vst]), vph, p.err, abort_flag, wait_site(kSiteAttn, 2, 7))) goto done;
           tc_fence_after();
@@ -304,8 +326,8 @@ __global__ void __launch_bounds__(NUM_THREADS, 1) attn_tc_kernel(const __grid_co
 #pragma unroll
             for (int kk = 0; kk < TK / 16; ++kk)
               umma_ts_lohi(tmem + COL_O0 + j * D, tmem + COL_S0 + j * TK + kk * 8, vlo + ((kk * 16 * 128) >> 4),
-                           v_hi, idesc_pv, (jj > 0 || kk > 0));
-            if (jj + 1 <= it.qt[j]) {
+                           v_hi, idesc_pv, (jj > it.k0 || kk > 0));
+            if (jj + 1 <= it.qt[j] && jj + 1 < it.k1) {
               if (!next_k_ready) {
                 if (!mbar_wait_bounded(smem_u32(&k_full[kst]), kph, p.err, abort_flag, wait_site(kSiteAttn, 2, 9))) goto done;
                 tc_fence_after();
@@ -349,7 +371,8 @@ __global__ void __launch_bounds__(NUM_THREADS, 1) attn_tc_kernel(const __grid_co
         const int qt = it.qt[j];
         float m = -INFINITY;  // running max of scaled scores (log2 domain)
         float l = 0.f;        // running row sum
-        for (int jj = 0; jj <= qt; ++jj) {
+        const int jlast = qt < it.k1 - 1 ? qt : it.k1 - 1;  // last key tile of this entry for the tile
+        for (int jj = it.k0; jj <= jlast; ++jj) {
           if (!mbar_wait_bounded(smem_u32(&s_full[j]), scount & 1, p.err, abort_flag, wait_site(kSiteAttn, 3, 10))) goto done;
           ++scount;
           tc_fence_after();
@@ -376,7 +399,7 @@ __global__ void __launch_bounds__(NUM_THREADS, 1) attn_tc_kernel(const __grid_co
           const bool need = tmax > m + RESCALE_THRESHOLD;
           float f = 1.f;  // factor for the O row and the sum
           bool rescale = false;
-          if (jj == 0) {
+          if (jj == it.k0) {
             m = tmax;
           } else if (__any_sync(0xffffffffu, need)) {
             const float mnew = fmaxf(m, tmax);
@@ -431,22 +454,80 @@ __global__ void __launch_bounds__(NUM_THREADS, 1) attn_tc_kernel(const __grid_co
         ++ocount;
         tc_fence_after();
         const int t = qt * TQ + row;
-        const float inv = 1.f / l;
+        // O_row = O * inv for a whole-range entry; a merged split pair gives c1 * O_first + c2 * O_second,
+        // evaluated in that order whichever half merges, so the result does not depend on timing
+        float c1 = 0.f, c2 = 0.f, inv = 1.f / l;
+        const float* other = nullptr;
+        bool store = true;
+        if (it.half != 0) {
+          // one half of a split pair: publish this half's unnormalised row with its max and sum;
+          // the second of the two halves to get here (counted per lane quadrant) merges them
+          const size_t tile = (size_t)it.w * 2 + j;
+          float* mine = p.part + ((size_t)it.w * 4 + (it.half - 1) * 2 + j) * PART_TILE;
+          other = p.part + ((size_t)it.w * 4 + (2 - it.half) * 2 + j) * PART_TILE;
+#pragma unroll 1
+          for (int c = 0; c < 4; ++c) {
+            uint32_t o[32];
+            tmem_ld_32x32b_x32(o_col + c * 32, o);
+            tmem_ld_wait();
+            float4* d4 = reinterpret_cast<float4*>(mine) + (c * 8) * TQ + row;  // column quad c*8 + v
+#pragma unroll
+            for (int v = 0; v < 8; ++v)
+              d4[v * TQ] = make_float4(u2f(o[4 * v]), u2f(o[4 * v + 1]), u2f(o[4 * v + 2]), u2f(o[4 * v + 3]));
+          }
+          mine[D * TQ + row] = m;
+          mine[D * TQ + TQ + row] = l;
+          __threadfence();
+          __syncwarp();
+          int ticket = 0;
+          if (lane == 0) ticket = atomicAdd(p.split_cnt + tile * 4 + quad, 1);
+          ticket = __shfl_sync(0xffffffffu, ticket, 0);
+          store = ticket != 0;
+          if (store) {
+            __threadfence();
+            const float mo = __ldcg(other + D * TQ + row), lo = __ldcg(other + D * TQ + TQ + row);
+            const float m1 = it.half == 1 ? m : mo, l1 = it.half == 1 ? l : lo;
+            const float m2 = it.half == 1 ? mo : m, l2 = it.half == 1 ? lo : l;
+            const float mm = fmaxf(m1, m2);
+            const float e1 = fast_exp2(m1 - mm), e2 = fast_exp2(m2 - mm);
+            const float rl = 1.f / __fmaf_rn(e1, l1, __fmul_rn(e2, l2));
+            c1 = __fmul_rn(e1, rl);
+            c2 = __fmul_rn(e2, rl);
+            inv = 1.f;  // the raw O rows are merged
+          }
+        }
         __half* dst = p.o + ((long long)it.b * p.S + t) * p.Lq + (long long)it.h[j] * D;
 #pragma unroll 1
-        for (int c = 0; c < 4; ++c) {
+        for (int c = 0; c < 4 && store; ++c) {
           uint32_t o[32];
           tmem_ld_32x32b_x32(o_col + c * 32, o);
           tmem_ld_wait();
+          float f[32];
+#pragma unroll
+          for (int e = 0; e < 32; ++e) f[e] = u2f(o[e]) * inv;
+          if (other != nullptr) {
+            const float4* s4 = reinterpret_cast<const float4*>(other) + (c * 8) * TQ + row;
+            const bool first = it.half == 1;  // this half holds O_first
+#pragma unroll
+            for (int v = 0; v < 8; ++v) {
+              const float4 x4 = __ldcg(s4 + v * TQ);
+              const float x[4] = {x4.x, x4.y, x4.z, x4.w};
+#pragma unroll
+              for (int u = 0; u < 4; ++u) {
+                const float o1 = first ? f[4 * v + u] : x[u], o2 = first ? x[u] : f[4 * v + u];
+                f[4 * v + u] = __fmaf_rn(c1, o1, __fmul_rn(c2, o2));
+              }
+            }
+          }
           if (t < p.S) {
             uint4* d4 = reinterpret_cast<uint4*>(dst + c * 32);
 #pragma unroll
             for (int v = 0; v < 4; ++v) {
               uint4 wv;
-              wv.x = pack_f16x2(u2f(o[8 * v + 0]) * inv, u2f(o[8 * v + 1]) * inv);
-              wv.y = pack_f16x2(u2f(o[8 * v + 2]) * inv, u2f(o[8 * v + 3]) * inv);
-              wv.z = pack_f16x2(u2f(o[8 * v + 4]) * inv, u2f(o[8 * v + 5]) * inv);
-              wv.w = pack_f16x2(u2f(o[8 * v + 6]) * inv, u2f(o[8 * v + 7]) * inv);
+              wv.x = pack_f16x2(f[8 * v + 0], f[8 * v + 1]);
+              wv.y = pack_f16x2(f[8 * v + 2], f[8 * v + 3]);
+              wv.z = pack_f16x2(f[8 * v + 4], f[8 * v + 5]);
+              wv.w = pack_f16x2(f[8 * v + 6], f[8 * v + 7]);
               d4[v] = wv;
             }
           }
@@ -474,15 +555,119 @@ bool encode_3d(CUtensorMap* m, const void* ptr, uint64_t width, uint64_t S, uint
              CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) == CUDA_SUCCESS;
 }
 
+// Schedule cost model of pair w: key tiles of its (up to) two query tiles plus one for the pair's
+// setup; nkv = key tiles of the pair.
+struct PairGeom {
+  int num_qt, pairs, items, bgc, U;
+  explicit PairGeom(const BlockDims& dm)
+      : num_qt((dm.S + TQ - 1) / TQ),
+        pairs((num_qt * dm.G + 1) / 2),
+        items(dm.B * dm.nkv * pairs),
+        bgc(dm.B * dm.nkv),
+        U(num_qt * dm.G) {}
+  int nkv(const BlockDims& dm, int w) const {
+    const int pr = pairs - 1 - w / bgc;
+    return (2 * pr + 1 < U ? 2 * pr + 1 : 2 * pr) / dm.G + 1;
+  }
+  int load(const BlockDims& dm, int w) const { return 2 * nkv(dm, w) + 1; }
+  long long total(const BlockDims& dm) const {
+    long long t = 0;
+    for (int w = 0; w < items; ++w) t += load(dm, w);
+    return t;
+  }
+  // Most pairs that may be split in two (the longest ones, with at least 4 key tiles so that both
+  // query tiles have keys in both halves).
+  int max_split(const BlockDims& dm) const {
+    if (items > MAX_LIST) return 0;
+    int n = 0;
+    while (n < items && n < kAttnMaxSplit && n + items < MAX_LIST && nkv(dm, n) >= 4) ++n;
+    return n;
+  }
+};
+
+// Entries for the first ns pairs split in two, in non-increasing order of cost. Returns the count.
+int build_entries(const BlockDims& dm, const PairGeom& g, int ns, unsigned short* entry, int* cost) {
+  unsigned short he[2 * kAttnMaxSplit];
+  int hc[2 * kAttnMaxSplit], nh = 0;
+  for (int w = 0; w < ns; ++w) {  // halves: setup plus publishing / merging the partial rows
+    const int nk = g.nkv(dm, w), h = nk / 2;
+    he[nh] = (unsigned short)(w | (2 << kEntryPairBits));
+    hc[nh++] = 2 * (nk - h) + 2;
+    he[nh] = (unsigned short)(w | (1 << kEntryPairBits));
+    hc[nh++] = 2 * h + 2;
+  }
+  for (int i = 1; i < nh; ++i)  // insertion sort, non-increasing (stable)
+    for (int k = i; k > 0 && hc[k - 1] < hc[k]; --k) {
+      const int c = hc[k];
+      hc[k] = hc[k - 1];
+      hc[k - 1] = c;
+      const unsigned short e = he[k];
+      he[k] = he[k - 1];
+      he[k - 1] = e;
+    }
+  int n = 0, i = 0, w = ns;  // merge with the whole pairs ns .. items-1 (already non-increasing)
+  while (i < nh || w < g.items) {
+    if (w >= g.items || (i < nh && hc[i] >= g.load(dm, w))) {
+      entry[n] = he[i];
+      cost[n++] = hc[i++];
+    } else {
+      entry[n] = (unsigned short)w;
+      cost[n++] = g.load(dm, w++);
+    }
+  }
+  return n;
+}
+
+// Longest-processing-time assignment of entries (in order) to `grid` CTAs, each to the CTA with the
+// least work so far (a binary min-heap of CTA loads). Fills owner[] and count[]; returns the largest
+// CTA load.
+long long assign_lpt(int n, const int* cost, int grid, unsigned short* owner, int* count) {
+  long long load[MAX_CTAS];
+  int heap_cta[MAX_CTAS];
+  for (int c = 0; c < grid; ++c) {
+    load[c] = 0;
+    heap_cta[c] = c;
+    count[c] = 0;
+  }
+  auto less = [&](int a, int b) { return load[a] < load[b] || (load[a] == load[b] && a < b); };
+  for (int i = 0; i < n; ++i) {
+    const int c = heap_cta[0];
+    owner[i] = (unsigned short)c;
+    ++count[c];
+    load[c] += cost[i];
+    for (int x = 0;;) {  // sift the root down
+      const int l = 2 * x + 1, r = l + 1;
+      int m = x;
+      if (l < grid && less(heap_cta[l], heap_cta[m])) m = l;
+      if (r < grid && less(heap_cta[r], heap_cta[m])) m = r;
+      if (m == x) break;
+      const int t = heap_cta[x];
+      heap_cta[x] = heap_cta[m];
+      heap_cta[m] = t;
+      x = m;
+    }
+  }
+  long long mx = 0;
+  for (int c = 0; c < grid; ++c) mx = load[c] > mx ? load[c] : mx;
+  return mx;
+}
+
+constexpr size_t kCounterBytes = (size_t)kAttnSplitCounters * sizeof(int);
+constexpr size_t kPartSlotBytes = (size_t)2 * 2 * PART_TILE * sizeof(float);
+
 }  // namespace
+
+size_t attention_tc_scratch_bytes(const BlockDims& dm) {
+  // the largest split set of any grid (at most MAX_CTAS CTAs)
+  return kCounterBytes + (size_t)PairGeom(dm).max_split(dm) * kPartSlotBytes;
+}
 
 bool attention_tc_supported(const BlockDims& dm) {
   return dm.lat == DType::F16 && dm.d == D && dm.S >= 1 && (long long)dm.Lq * dm.S * 2 < (1ll << 40);
 }
 
 cudaError_t launch_attention_tc(const BlockDims& dm, const void* q, const void* k, const void* v, void* o,
-                                void* sched, unsigned* dev_err, cudaStream_t stream) {
-  (void)sched;
+                                void* scratch, unsigned* dev_err, cudaStream_t stream) {
   if (!attention_tc_supported(dm)) return cudaErrorInvalidValue;
   AttnMaps maps;
   if (!encode_3d(&maps.q, q, (uint64_t)dm.Lq, (uint64_t)dm.S, (uint64_t)dm.B) ||
@@ -504,50 +689,55 @@ cudaError_t launch_attention_tc(const BlockDims& dm, const void* q, const void* 
   p.err = dev_err;
   int grid = p.items < num_sms() ? p.items : num_sms();
   if (grid > MAX_CTAS) grid = MAX_CTAS;
-  // Longest-processing-time assignment: pairs come in non-increasing order of key tiles
-  // (item index order), each goes to the CTA with the least work so far (a binary min-heap of
-  // CTA loads). Fixed-size arrays only: launching allocates no memory.
-  static thread_local AttnSched plan;
-  plan.use = p.items <= MAX_LIST;
-  if (plan.use) {
-    long long load[MAX_CTAS];
-    int heap_cta[MAX_CTAS], count[MAX_CTAS];
-    static thread_local unsigned short owner[MAX_LIST];
-    for (int c = 0; c < grid; ++c) {
-      load[c] = 0;
-      heap_cta[c] = c;
-      count[c] = 0;
-    }
-    auto less = [&](int a, int b) { return load[a] < load[b] || (load[a] == load[b] && a < b); };
-    const int bgc = p.B * p.nkv, U = p.num_qt * p.G;
-    for (int w = 0; w < p.items; ++w) {
-      const int pr = p.pairs - 1 - w / bgc;
-      const int qt_last = (2 * pr + 1 < U ? 2 * pr + 1 : 2 * pr) / p.G;
-      const int c = heap_cta[0];
-      owner[w] = (unsigned short)c;
-      ++count[c];
-      load[c] += 2 * (qt_last + 1) + 1;  // key tiles of both tiles, plus the pair's setup
-      for (int i = 0;;) {                // sift the root down
-        const int l = 2 * i + 1, r = l + 1;
-        int m = i;
-        if (l < grid && less(heap_cta[l], heap_cta[m])) m = l;
-        if (r < grid && less(heap_cta[r], heap_cta[m])) m = r;
-        if (m == i) break;
-        const int t = heap_cta[i];
-        heap_cta[i] = heap_cta[m];
-        heap_cta[m] = t;
-        i = m;
+  p.split_cnt = static_cast<int*>(scratch);
+  p.part = reinterpret_cast<float*>(static_cast<unsigned char*>(scratch) + kCounterBytes);
+  // Schedule: the longest pairs may run as two halves of their key range (merged by the half that
+  // ends second); of all split counts the one with the smallest simulated makespan is taken. The
+  // plan depends on the shape and the grid only and is kept for the next launch of the same shape.
+  // Fixed-size arrays only: launching allocates no memory.
+  struct PlanCache {
+    int key[6] = {-1, -1, -1, -1, -1, -1};
+    int nsplit = 0;
+    AttnSched plan;
+  };
+  static thread_local PlanCache cache;
+  const int key[6] = {dm.B, dm.S, dm.G, dm.nkv, grid, (int)PairGeom(dm).items};
+  bool hit = true;
+  for (int i = 0; i < 6; ++i) hit = hit && cache.key[i] == key[i];
+  if (!hit) {
+    const PairGeom geom(dm);
+    static thread_local unsigned short owner[MAX_LIST], entry[MAX_LIST];
+    static thread_local int cost[MAX_LIST];
+    int count[MAX_CTAS];
+    AttnSched& plan = cache.plan;
+    plan.use = p.items <= MAX_LIST;
+    cache.nsplit = 0;
+    if (plan.use) {
+      long long best = -1;
+      const int maxs = geom.max_split(dm);
+      for (int ns = 0; ns <= maxs; ++ns) {
+        const int n = build_entries(dm, geom, ns, entry, cost);
+        const long long mk = assign_lpt(n, cost, grid, owner, count);
+        if (best < 0 || mk < best) {
+          best = mk;
+          cache.nsplit = ns;
+        }
       }
+      const int n = build_entries(dm, geom, cache.nsplit, entry, cost);
+      assign_lpt(n, cost, grid, owner, count);
+      int off = 0;
+      for (int c = 0; c < grid; ++c) {
+        plan.off[c] = (unsigned short)off;
+        off += count[c];
+        count[c] = plan.off[c];  // fill cursor
+      }
+      plan.off[grid] = (unsigned short)off;
+      for (int i = 0; i < n; ++i) plan.items[count[owner[i]]++] = entry[i];
     }
-    int off = 0;
-    for (int c = 0; c < grid; ++c) {
-      plan.off[c] = (unsigned short)off;
-      off += count[c];
-      count[c] = plan.off[c];  // fill cursor
-    }
-    plan.off[grid] = (unsigned short)off;
-    for (int w = 0; w < p.items; ++w) plan.items[count[owner[w]]++] = (unsigned short)w;
+    for (int i = 0; i < 6; ++i) cache.key[i] = key[i];
   }
+  p.nsplit = cache.nsplit;
+  const AttnSched& plan = cache.plan;
   cudaError_t e = cudaFuncSetAttribute(attn_tc_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)SMEM_BYTES);
   if (e != cudaSuccess) return e;
   attn_tc_kernel<<<grid, NUM_THREADS, SMEM_BYTES, stream>>>(maps, p, plan);

@@ -135,7 +135,7 @@ cca_workspace_layout_t layout_of(const BlockDims& dm) {
   L.wo_offset = off;
   if (sep) off = align_up(off + (size_t)dm.E * dm.Lq * eb);
   L.sched_offset = off;
-  off = align_up(off + 256);
+  off = align_up(off + (attention_tc_supported(dm) ? attention_tc_scratch_bytes(dm) : 256));
   L.total_bytes = off;
   return L;
 }

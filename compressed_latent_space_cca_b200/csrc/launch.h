@@ -42,7 +42,7 @@ struct BlockPtrs {
   void* v_att;    // [T, Lkv] lat: attention values (== v_cache when lat == io)
   void* o;        // [T, Lq]  lat: attention output
   void* wo_lat;   // [E, Lq]  lat copy of W_o (== Wo when lat == io)
-  void* sched;
+  void* sched;    // scratch of the tensor-core attention (split-pair counters, partial rows)
   unsigned* dev_err;
 };
 
@@ -81,7 +81,12 @@ cudaError_t launch_gemm_tc(const GemmTcArgs& a, cudaStream_t stream);
 
 bool attention_tc_supported(const BlockDims& dm);
 cudaError_t launch_attention_tc(const BlockDims& dm, const void* q, const void* k, const void* v, void* o,
-                                void* sched, unsigned* dev_err, cudaStream_t stream);
+                                void* scratch, unsigned* dev_err, cudaStream_t stream);
+// Split-pair scratch of the tensor-core attention: kAttnSplitCounters ints that must be zero when
+// it starts (the preprocessing kernels clear them), then the partial rows.
+constexpr int kAttnMaxSplit = 64;
+constexpr int kAttnSplitCounters = kAttnMaxSplit * 2 * 4;
+size_t attention_tc_scratch_bytes(const BlockDims& dm);
 
 // ---- misc ----
 cudaError_t launch_wait_timeout_selftest(unsigned* dev_err, unsigned long long limit_ns, cudaStream_t stream);

@@ -30,7 +30,7 @@ __global__ void __launch_bounds__(PP_THREADS) preproc_simt_kernel(
     const Tc* __restrict__ ck_seq, const Tc* __restrict__ ck_chan, Tl* __restrict__ qout, Tc* __restrict__ kout,
     Tc* __restrict__ vout, Tl* __restrict__ katt, Tl* __restrict__ vatt, const Tc* __restrict__ wo,
     Tl* __restrict__ wo_lat, long long wo_n, unsigned* __restrict__ err, int S, int nq, int nkv, int d, int K,
-    int mode, int vshift, int use_rope, float rope_base) {
+    int mode, int vshift, int use_rope, float rope_base, int* __restrict__ zero_cnt) {
   extern __shared__ float sm[];
   const int G = nq / nkv;
   const int H1 = G + 1;  // G query heads + the K head of the group
@@ -186,6 +186,9 @@ __global__ void __launch_bounds__(PP_THREADS) preproc_simt_kernel(
       bad |= f16_overflow(w);
     }
   }
+  // side job: clear the attention's split-pair counters for the launch that follows
+  if (zero_cnt != nullptr && blockIdx.x == 0 && blockIdx.y == 0 && blockIdx.z == 0)
+    for (int i = tid; i < kAttnSplitCounters; i += PP_THREADS) zero_cnt[i] = 0;
   report_range(bad, err);
 }
 
@@ -232,7 +235,8 @@ cudaError_t preproc_typed(const BlockDims& dm, const BlockPtrs& p, cudaStream_t 
       (const Tl*)p.qkv_lat, (const Tc*)p.cq_seq, (const Tc*)p.cq_chan, (const Tc*)p.ck_seq, (const Tc*)p.ck_chan,
       (Tl*)p.q, (Tc*)p.k_cache, (Tc*)p.v_cache, sep ? (Tl*)p.k_att : nullptr, sep ? (Tl*)p.v_att : nullptr,
       (const Tc*)p.Wo, sep ? (Tl*)p.wo_lat : nullptr, (long long)dm.E * dm.Lq, p.dev_err, dm.S, dm.nq, dm.nkv, dm.d,
-      dm.K, dm.qk_mean_mode, dm.value_shift, dm.use_rope, dm.rope_base);
+      dm.K, dm.qk_mean_mode, dm.value_shift, dm.use_rope, dm.rope_base,
+      attention_tc_supported(dm) ? static_cast<int*>(p.sched) : nullptr);
   return cudaGetLastError();
 }
 }  // namespace

@@ -59,6 +59,7 @@ struct PreParams {
   __half* wo_lat;
   long long wo_n;
   unsigned* err;
+  int* zero_cnt;  // split-pair counters of the attention launch that follows (cleared here)
   int S, nq, nkv, K, mode, vshift, use_rope;
   int nbuf;  // weight buffers in shared memory: 2 (next head's weights prefetched) or 1
 };
@@ -274,6 +275,8 @@ __global__ void __launch_bounds__(NT, 2) preproc_tc_kernel(const __grid_constant
       }
       *reinterpret_cast<uint4*>(p.wo_lat + e * 8) = make_uint4(h[0], h[1], h[2], h[3]);
     }
+    if (p.zero_cnt != nullptr && cid == 0)
+      for (int i = threadIdx.x; i < kAttnSplitCounters; i += NT) p.zero_cnt[i] = 0;
   }
 
   // RoPE tables: rtab[i] = (cos, sin) of t0 * theta_i, rtab[D/2 + i] = (cos, sin) of 8 * theta_i
@@ -516,6 +519,7 @@ cudaError_t launch_preproc_tc(const BlockDims& dm, const BlockPtrs& p, cudaStrea
   q.wo_lat = static_cast<__half*>(p.wo_lat);
   q.wo_n = (long long)dm.E * dm.Lq;
   q.err = p.dev_err;
+  q.zero_cnt = attention_tc_supported(dm) ? static_cast<int*>(p.sched) : nullptr;
   q.S = dm.S;
   q.nq = dm.nq;
   q.nkv = dm.nkv;

@@ -134,7 +134,7 @@ typedef struct cca_workspace_layout {
   size_t v_att_offset;      /* [T, Lkv]: v as the attention reads it */
   size_t o_offset;          /* [T, Lq]: attention output, heads concatenated */
   size_t wo_offset;         /* [E, Lq]: W_o in the intermediate type */
-  size_t sched_offset;      /* small scheduling scratch of the attention kernel */
+  size_t sched_offset;      /* scratch of the attention kernel: split-pair counters and partial rows */
 } cca_workspace_layout_t;
 
 /* Checks a configuration. CCA_OK if some kernel path accepts it. */

@@ -74,6 +74,22 @@ def test_bf16_small(path, case):
     check_all(sh, run_gpu(sh, inp, path=path), run_oracle(sh, inp))
 
 
+# The tensor-core attention runs the longest (query tile pair, KV group) items as two halves of
+# their key range on different CTAs and merges the halves' partial rows. With 16 or fewer items the
+# grid has one CTA per item, so the longest items are split whatever the GPU; every row is compared.
+SPLIT_CASES = [
+    dict(seq_len=1024, n_q_heads=4, n_kv_heads=2, hidden=512),  # G=2: two heads per item
+    dict(seq_len=1000, n_q_heads=2, n_kv_heads=2, hidden=512),  # G=1: consecutive query tiles, ragged
+]
+
+
+@pytest.mark.parametrize("case", range(len(SPLIT_CASES)))
+def test_bf16_split_key_ranges(case):
+    sh = shape(**SPLIT_CASES[case])
+    inp = workloads.make_inputs(sh)
+    check_all(sh, run_gpu(sh, inp, path=TENSOR), run_oracle(sh, inp))
+
+
 @pytest.mark.parametrize("path", [SIMT, AUTO, TENSOR], ids=["simt", "auto", "tensor"])
 @pytest.mark.parametrize("mode,vshift,rope", [(0, 0, 0), (1, 0, 1), (2, 1, 0), (3, 1, 1), (0, 1, 1)])
 def test_bf16_modes(path, mode, vshift, rope):
