@@ -12,9 +12,12 @@
 // issues TMA loads of 128 x 64 A tiles and 256 x 64 B tiles (128-byte swizzle)
 // into a 4-stage shared-memory ring; one thread of warp 1 issues
 // tcgen05.mma (M=128, N=256, K=16) into one of two 256-column fp32
-// accumulators in tensor memory; warps 2-5 drain the other accumulator
-// (tcgen05.ld -> convert -> global store) so the epilogue of tile i overlaps
-// the main loop of tile i+1. Every mbarrier wait is bounded.
+// accumulators in tensor memory; warps 2-5 drain the other accumulator so the
+// epilogue of tile i overlaps the main loop of tile i+1. For 16-bit outputs
+// each epilogue warp converts 32 rows x 64 columns at a time into its own
+// staging buffer (128-byte swizzle) and one of its threads writes the chunk
+// with a TMA tensor store, so global writes leave in whole lines; fp32
+// outputs are stored directly. Every mbarrier wait is bounded.
 #include "cca_common.cuh"
 #include "launch.h"
 
@@ -39,12 +42,19 @@ struct Shape {
   static constexpr int ACC_BUFS = MH == 1 ? 2 : 1;
   static constexpr int EPI_WARPS = 4 * MH;
   static constexpr int NUM_THREADS = 64 + 32 * EPI_WARPS;
-  static constexpr size_t SMEM_BYTES = (size_t)STAGES * STAGE_BYTES + 1024 /*align slack*/ + 256 /*barriers*/;
+  // per epilogue warp, staging buffers of 32 rows x 64 columns (16-bit) for TMA stores (MH = 1)
+  static constexpr int EPI_BUFS = MH == 1 ? 2 : 0;
+  static constexpr int STG_BYTES = 32 * 64 * 2;
+  static constexpr size_t SMEM_BYTES = (size_t)STAGES * STAGE_BYTES + (size_t)EPI_WARPS * EPI_BUFS * STG_BYTES +
+                                       1024 /*align slack*/ + 256 /*barriers*/;
+  static_assert(SMEM_BYTES <= 232448, "shared memory of one CTA");
+  static constexpr int EPI_BUF_COUNT = EPI_BUFS > 0 ? EPI_BUFS : 1;  // (unused when MH = 2)
 };
 
 struct GemmMaps {
   CUtensorMap a;
   CUtensorMap b[3];
+  CUtensorMap c;  // 16-bit output, boxes of 64 columns x 32 rows (used when tma_store)
 };
 
 struct GemmParams {
@@ -60,6 +70,7 @@ struct GemmParams {
   unsigned* err;
   int num_tiles;
   int n_tiles_n;
+  int tma_store;  // 16-bit output written through shared memory and maps.c
 };
 
 // Stores 32 fp32 accumulators of one row; returns true if an fp16 output overflowed.
@@ -99,7 +110,8 @@ __global__ void __launch_bounds__(Shape<MH>::NUM_THREADS, 1) gemm_tc_kernel(cons
   constexpr int ACC_BUFS = T::ACC_BUFS;
   extern __shared__ uint8_t smem_raw[];
   uint8_t* smem = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
-  uint64_t* bars = reinterpret_cast<uint64_t*>(smem + STAGES * STAGE_BYTES);
+  uint8_t* staging = smem + STAGES * STAGE_BYTES;  // [EPI_WARPS][EPI_BUFS][32 rows][128 B]
+  uint64_t* bars = reinterpret_cast<uint64_t*>(staging + T::EPI_WARPS * T::EPI_BUFS * T::STG_BYTES);
   uint64_t* full = bars;                 // [STAGES] TMA -> MMA
   uint64_t* empty = bars + STAGES;       // [STAGES] MMA -> TMA
   uint64_t* tfull = bars + 2 * STAGES;   // [ACC_BUFS] MMA -> epilogue
@@ -209,6 +221,8 @@ __global__ void __launch_bounds__(Shape<MH>::NUM_THREADS, 1) gemm_tc_kernel(cons
     // --------------------------------------------------------- epilogue --
     const int quad = warp & 3;        // this warp may touch TMEM lanes [32*quad, 32*quad+32)
     const int half = (warp - 2) / 4;  // MH = 2: which 128-row half of the tile (accumulator columns half*256..)
+    uint8_t* stg = staging + (warp - 2) * T::EPI_BUFS * T::STG_BYTES;
+    int sbuf = 0;
     bool bad = false;
     int i = 0;
     for (int t = blockIdx.x; t < p.num_tiles; t += gridDim.x, ++i) {
@@ -218,20 +232,59 @@ __global__ void __launch_bounds__(Shape<MH>::NUM_THREADS, 1) gemm_tc_kernel(cons
       tc_fence_after();
       const long long m0 = (long long)(t / p.n_tiles_n) * BM;
       const int n0 = (t % p.n_tiles_n) * BN;
-      const long long row = m0 + half * 128 + quad * 32 + lane;
+      const long long row0 = m0 + half * 128 + quad * 32;  // this warp's 32 rows
+      const long long row = row0 + lane;
       const uint32_t col0 = tmem_base + ((uint32_t)(quad * 32) << 16) + (acc + half) * BN;
+      if (T::EPI_BUFS > 0 && p.tma_store) {
+        const bool h = p.out_type == (int)DType::F16;
 #pragma unroll 1
-      for (int c = 0; c < BN / 32; ++c) {
-        uint32_t r[32];
-        tmem_ld_32x32b_x32(col0 + c * 32, r);
-        tmem_ld_wait();
-        const int col = n0 + c * 32;
-        if (row < p.M && col < p.N) bad |= store_row_chunk(p, row, col, r);
+        for (int c = 0; c < BN / 64; ++c) {
+          uint32_t r[64];
+          tmem_ld_32x32b_x32(col0 + c * 64, r);
+          tmem_ld_32x32b_x32(col0 + c * 64 + 32, r + 32);
+          tmem_ld_wait();
+          uint32_t w[32];
+#pragma unroll
+          for (int e = 0; e < 32; ++e) {
+            const float x0 = u2f(r[2 * e]), x1 = u2f(r[2 * e + 1]);
+            if (h) {
+              w[e] = pack_f16x2(x0, x1);
+              bad |= f16_overflow(x0) || f16_overflow(x1);
+            } else {
+              w[e] = pack_bf16x2(x0, x1);
+            }
+          }
+          // the buffer's previous store has read it; row `lane`, 16-byte chunk j at j ^ (lane % 8)
+          if (lane == 0) bulk_wait_read<T::EPI_BUF_COUNT - 1>();
+          __syncwarp();
+          uint8_t* buf = stg + sbuf * T::STG_BYTES;
+#pragma unroll
+          for (int j = 0; j < 8; ++j)
+            *reinterpret_cast<uint4*>(buf + lane * 128 + ((j ^ (lane & 7)) << 4)) =
+                make_uint4(w[4 * j], w[4 * j + 1], w[4 * j + 2], w[4 * j + 3]);
+          fence_async_smem();
+          __syncwarp();
+          if (lane == 0 && row0 < p.M) {  // rows past M and columns past N are clipped by the map
+            tma_store_2d(&maps.c, smem_u32(buf), n0 + c * 64, (int)row0);
+            bulk_commit();
+          }
+          sbuf = sbuf + 1 == T::EPI_BUF_COUNT ? 0 : sbuf + 1;
+        }
+      } else {
+#pragma unroll 1
+        for (int c = 0; c < BN / 32; ++c) {
+          uint32_t r[32];
+          tmem_ld_32x32b_x32(col0 + c * 32, r);
+          tmem_ld_wait();
+          const int col = n0 + c * 32;
+          if (row < p.M && col < p.N) bad |= store_row_chunk(p, row, col, r);
+        }
       }
       tc_fence_before();
       __syncwarp();
       if (lane == 0) mbar_arrive(smem_u32(&tempty[acc]));
     }
+    if (lane == 0) bulk_wait_all();  // the staging buffers stay valid until the stores are done
     report_range(bad, p.err);
   }
   tc_fence_before();
@@ -240,12 +293,13 @@ __global__ void __launch_bounds__(Shape<MH>::NUM_THREADS, 1) gemm_tc_kernel(cons
   if (warp == 1) tmem_dealloc(tmem_base, TMEM_COLS);
 }
 
+// 2D map of a row-major 16-bit matrix, 128-byte swizzle; row_bytes = 0 for densely packed rows.
 bool encode_2d(CUtensorMap* m, const void* ptr, CUtensorMapDataType dt, uint64_t inner, uint64_t outer,
-               uint32_t box_inner, uint32_t box_outer) {
+               uint32_t box_inner, uint32_t box_outer, uint64_t row_bytes = 0) {
   EncodeTiledFn enc = get_encode_tiled();
   if (enc == nullptr) return false;
   cuuint64_t dims[2] = {inner, outer};
-  cuuint64_t strides[1] = {inner * 2};
+  cuuint64_t strides[1] = {row_bytes ? row_bytes : inner * 2};
   cuuint32_t box[2] = {box_inner, box_outer};
   cuuint32_t estr[2] = {1, 1};
   return enc(m, dt, 2, const_cast<void*>(ptr), dims, strides, box, estr,
@@ -290,10 +344,19 @@ cudaError_t launch_gemm_tc(const GemmTcArgs& a, cudaStream_t stream) {
   p.ldc = a.ldc;
   p.out_type = (int)a.out;
   p.in_fmt = a.in == DType::F16 ? kFmtF16 : kFmtBF16;
+  // 256-row tiles keep direct stores: their single accumulator leaves nothing to overlap the wait
+  // for a staging buffer with, while direct stores retire without waiting
+  const bool big = a.K >= 1024 && a.M >= 256;
+  p.tma_store = !big && (a.out == DType::BF16 || a.out == DType::F16);
+  if (p.tma_store) {
+    const CUtensorMapDataType ct =
+        a.out == DType::F16 ? CU_TENSOR_MAP_DATA_TYPE_FLOAT16 : CU_TENSOR_MAP_DATA_TYPE_BFLOAT16;
+    if (!encode_2d(&maps.c, a.C, ct, (uint64_t)N, (uint64_t)a.M, 64, 32, (uint64_t)a.ldc * 2))
+      return cudaErrorInvalidValue;
+  }
   p.err = a.dev_err;
   p.n_tiles_n = (N + BN - 1) / BN;
   // 256-row tiles when the main loop is long enough to carry the epilogue it cannot overlap
-  const bool big = a.K >= 1024 && a.M >= 256;
   const int BM = big ? 256 : 128;
   const long long m_tiles = (a.M + BM - 1) / BM;
   p.num_tiles = (int)(m_tiles * p.n_tiles_n);
