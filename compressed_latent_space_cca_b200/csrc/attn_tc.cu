@@ -555,8 +555,11 @@ bool encode_3d(CUtensorMap* m, const void* ptr, uint64_t width, uint64_t S, uint
              CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) == CUDA_SUCCESS;
 }
 
-// Schedule cost model of pair w: key tiles of its (up to) two query tiles plus one for the pair's
-// setup; nkv = key tiles of the pair.
+// Schedule cost model, in units of about half a key-tile step (one step: both query tiles of the
+// pair against one key tile): two per step plus a fixed cost per entry for its setup, pipeline
+// fill and epilogue; a half of a split pair pays more for publishing or merging its partial rows.
+// The constants follow per-entry timings of this kernel on B200 (about 2 us per step, 4 to 6 us
+// per entry, 4 us more for a split half); nkv = key tiles of the pair.
 struct PairGeom {
   int num_qt, pairs, items, bgc, U;
   explicit PairGeom(const BlockDims& dm)
@@ -569,7 +572,8 @@ struct PairGeom {
     const int pr = pairs - 1 - w / bgc;
     return (2 * pr + 1 < U ? 2 * pr + 1 : 2 * pr) / dm.G + 1;
   }
-  int load(const BlockDims& dm, int w) const { return 2 * nkv(dm, w) + 1; }
+  static constexpr int kEntryCost = 4, kSplitCost = 4;
+  int load(const BlockDims& dm, int w) const { return 2 * nkv(dm, w) + kEntryCost; }
   long long total(const BlockDims& dm) const {
     long long t = 0;
     for (int w = 0; w < items; ++w) t += load(dm, w);
@@ -589,12 +593,12 @@ struct PairGeom {
 int build_entries(const BlockDims& dm, const PairGeom& g, int ns, unsigned short* entry, int* cost) {
   unsigned short he[2 * kAttnMaxSplit];
   int hc[2 * kAttnMaxSplit], nh = 0;
-  for (int w = 0; w < ns; ++w) {  // halves: setup plus publishing / merging the partial rows
+  for (int w = 0; w < ns; ++w) {
     const int nk = g.nkv(dm, w), h = nk / 2;
     he[nh] = (unsigned short)(w | (2 << kEntryPairBits));
-    hc[nh++] = 2 * (nk - h) + 2;
+    hc[nh++] = 2 * (nk - h) + PairGeom::kEntryCost + PairGeom::kSplitCost;
     he[nh] = (unsigned short)(w | (1 << kEntryPairBits));
-    hc[nh++] = 2 * h + 2;
+    hc[nh++] = 2 * h + PairGeom::kEntryCost + PairGeom::kSplitCost;
   }
   for (int i = 1; i < nh; ++i)  // insertion sort, non-increasing (stable)
     for (int k = i; k > 0 && hc[k - 1] < hc[k]; --k) {
