@@ -67,6 +67,7 @@ class CcaWorkspaceLayout(Structure):
         ("v_att_offset", c_size_t),
         ("o_offset", c_size_t),
         ("wo_offset", c_size_t),
+        ("wc_offset", c_size_t),
         ("sched_offset", c_size_t),
     ]
 

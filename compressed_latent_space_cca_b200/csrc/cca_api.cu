@@ -134,6 +134,8 @@ cca_workspace_layout_t layout_of(const BlockDims& dm) {
   off = align_up(off + (size_t)dm.T * dm.Lq * eb);
   L.wo_offset = off;
   if (sep) off = align_up(off + (size_t)dm.E * dm.Lq * eb);
+  L.wc_offset = off;
+  if (sep) off = align_up(off + (size_t)(dm.nq + dm.nkv) * dm.d * dm.d * eb);
   L.sched_offset = off;
   off = align_up(off + (attention_tc_supported(dm) ? attention_tc_scratch_bytes(dm) : 256));
   L.total_bytes = off;
@@ -210,6 +212,15 @@ cca_status_t run_block(const Resolved& r, BlockPtrs p, cudaStream_t stream, void
     a.in = dm.io;
     a.out = dm.lat;
     a.dev_err = p.dev_err;
+    if (r.tc_pre) {  // the fp16 channel-conv weights of the preprocessing kernel, made on the side
+      const long long nc = (long long)dm.d * dm.d;
+      a.side_src[0] = p.cq_chan;
+      a.side_dst[0] = p.wc_lat;
+      a.side_n[0] = nc * dm.nq;
+      a.side_src[1] = p.ck_chan;
+      a.side_dst[1] = static_cast<char*>(p.wc_lat) + nc * dm.nq * eb;
+      a.side_n[1] = nc * dm.nkv;
+    }
     if ((e = launch_gemm_tc(a, stream)) != cudaSuccess) return cuda_fail("down-projection (tcgen05)", e);
   } else {
     char* out = static_cast<char*>(p.qkv_lat);
@@ -221,6 +232,13 @@ cca_status_t run_block(const Resolved& r, BlockPtrs p, cudaStream_t stream, void
                                 ns[i], dm.E, stream)) != cudaSuccess)
         return cuda_fail("down-projection (SIMT)", e);
       col += ns[i];
+    }
+    if (r.tc_pre) {
+      const long long nc = (long long)dm.d * dm.d;
+      if ((e = launch_convert_f16(p.cq_chan, p.wc_lat, nc * dm.nq, p.dev_err, stream)) != cudaSuccess ||
+          (e = launch_convert_f16(p.ck_chan, static_cast<char*>(p.wc_lat) + nc * dm.nq * eb, nc * dm.nkv, p.dev_err,
+                                  stream)) != cudaSuccess)
+        return cuda_fail("channel-conv weight copy", e);
     }
   }
   if ((e = mark(1)) != cudaSuccess) return cuda_fail("event", e);
@@ -309,6 +327,7 @@ cca_status_t prepare(const cca_config_t* cfg, int path, const void* const* ins, 
   p->v_att = sep ? ws + L.v_att_offset : outs[2];
   p->o = ws + L.o_offset;
   p->wo_lat = sep ? ws + L.wo_offset : const_cast<void*>(ins[8]);
+  p->wc_lat = sep ? ws + L.wc_offset : nullptr;
   p->sched = ws + L.sched_offset;
   p->dev_err = nullptr;
   return CCA_OK;
@@ -406,7 +425,9 @@ cca_status_t cca_plan(const cca_config_t* cfg, int path, cca_plan_t* out) {
   out->attention_tensor = r.tc_attn;
   out->out_proj_tensor = r.tc_out;
   out->preproc_tensor = r.tc_pre;
-  out->launches = (r.tc_down ? 1 : 3) + 1 + 1 + 1;
+  // down-projection (one tcgen05 GEMM, or three SIMT GEMMs plus the two fp16 weight copies that the
+  // tcgen05 GEMM otherwise makes on the side), preprocessing, attention, output projection
+  out->launches = (r.tc_down ? 1 : 3 + (r.tc_pre ? 2 : 0)) + 1 + 1 + 1;
   return CCA_OK;
 }
 

@@ -71,6 +71,10 @@ struct GemmParams {
   int num_tiles;
   int n_tiles_n;
   int tma_store;  // 16-bit output written through shared memory and maps.c
+  // side job (bf16 -> fp16 copies), done by the epilogue warps before their first tile
+  const __nv_bfloat16* side_src[2];
+  __half* side_dst[2];
+  long long side_n[2];
 };
 
 // Stores 32 fp32 accumulators of one row; returns true if an fp16 output overflowed.
@@ -224,6 +228,25 @@ __global__ void __launch_bounds__(Shape<MH>::NUM_THREADS, 1) gemm_tc_kernel(cons
     uint8_t* stg = staging + (warp - 2) * T::EPI_BUFS * T::STG_BYTES;
     int sbuf = 0;
     bool bad = false;
+    // side job while the first accumulator fills: this CTA's share of the fp16 copies, 8 elements
+    // per 16-byte vector (the sizes are multiples of 8)
+    for (int i = 0; i < 2; ++i) {
+      const long long nvec = p.side_n[i] / 8;
+      const long long chunk = (nvec + gridDim.x - 1) / gridDim.x;
+      const long long lo = blockIdx.x * chunk, hi = lo + chunk < nvec ? lo + chunk : nvec;
+      for (long long e = lo + (threadIdx.x - 64); e < hi; e += 32 * T::EPI_WARPS) {
+        const uint4 raw = *reinterpret_cast<const uint4*>(p.side_src[i] + e * 8);
+        const __nv_bfloat162* b2 = reinterpret_cast<const __nv_bfloat162*>(&raw);
+        uint32_t h[4];
+#pragma unroll
+        for (int k = 0; k < 4; ++k) {
+          const float2 f = __bfloat1622float2(b2[k]);
+          bad |= f16_overflow(f.x) || f16_overflow(f.y);
+          h[k] = pack_f16x2(f.x, f.y);
+        }
+        *reinterpret_cast<uint4*>(p.side_dst[i] + e * 8) = make_uint4(h[0], h[1], h[2], h[3]);
+      }
+    }
     int i = 0;
     for (int t = blockIdx.x; t < p.num_tiles; t += gridDim.x, ++i) {
       const int acc = i % ACC_BUFS;
@@ -344,6 +367,14 @@ cudaError_t launch_gemm_tc(const GemmTcArgs& a, cudaStream_t stream) {
   p.ldc = a.ldc;
   p.out_type = (int)a.out;
   p.in_fmt = a.in == DType::F16 ? kFmtF16 : kFmtBF16;
+  for (int i = 0; i < 2; ++i) {
+    if (a.side_n[i] > 0 && (a.side_n[i] % 8 != 0 || (reinterpret_cast<uintptr_t>(a.side_src[i]) & 15) != 0 ||
+                            (reinterpret_cast<uintptr_t>(a.side_dst[i]) & 15) != 0))
+      return cudaErrorInvalidValue;
+    p.side_src[i] = static_cast<const __nv_bfloat16*>(a.side_src[i]);
+    p.side_dst[i] = static_cast<__half*>(a.side_dst[i]);
+    p.side_n[i] = a.side_n[i] > 0 ? a.side_n[i] : 0;
+  }
   // 256-row tiles keep direct stores: their single accumulator leaves nothing to overlap the wait
   // for a staging buffer with, while direct stores retire without waiting
   const bool big = a.K >= 1024 && a.M >= 256;

@@ -42,6 +42,7 @@ struct BlockPtrs {
   void* v_att;    // [T, Lkv] lat: attention values (== v_cache when lat == io)
   void* o;        // [T, Lq]  lat: attention output
   void* wo_lat;   // [E, Lq]  lat copy of W_o (== Wo when lat == io)
+  void* wc_lat;   // [nq + nkv, d, d] lat copy of the channel-conv weights (null when lat == io)
   void* sched;    // scratch of the tensor-core attention (split-pair counters, partial rows)
   unsigned* dev_err;
 };
@@ -76,8 +77,15 @@ struct GemmTcArgs {
   long long ldc;
   DType in, out;
   unsigned* dev_err;
+  // optional side job of the epilogue warps before their first tile: side_dst[i][0, side_n[i]) =
+  // fp16 copy of the bf16 side_src[i] (fp16 overflow reported as a range error)
+  const void* side_src[2];
+  void* side_dst[2];
+  long long side_n[2];
 };
 cudaError_t launch_gemm_tc(const GemmTcArgs& a, cudaStream_t stream);
+// dst[0, n) = fp16 copy of the bf16 src (fp16 overflow reported as a range error)
+cudaError_t launch_convert_f16(const void* src, void* dst, long long n, unsigned* dev_err, cudaStream_t stream);
 
 bool attention_tc_supported(const BlockDims& dm);
 cudaError_t launch_attention_tc(const BlockDims& dm, const void* q, const void* k, const void* v, void* o,

@@ -12,13 +12,14 @@
 // One CTA = 32 tokens of one sequence x one KV group (its G query heads and
 // its K/V head). The fp16 latents of all G+1 heads (32 tokens plus a K-1
 // token halo) arrive in shared memory by cp.async, with the seq-conv taps of
-// all G+1 heads. The heads' bf16 channel-mix weights stream in by cp.async
+// all G+1 heads. The heads' channel-mix weights (fp16 copies made once per
+// call, exact for bf16 weights in fp16's normal range) stream in by cp.async
 // through two buffers, so the next head's weights load while the current head
-// is mixed. Per head the causal seq conv runs on CUDA cores in fp32, and its
-// output s is split into bf16 s_hi + s_lo so that the
-// 32x128x128 channel mix runs on the tensor cores (mma.sync m16n8k16 bf16,
-// fp32 accumulate, two products per step) on the exact bf16 weights with a
-// relative error near 2^-18. Each thread owns the same accumulator positions
+// is mixed. Per head the causal seq conv runs on
+// CUDA cores in fp32 and its output s is rounded to fp16, so that the
+// 32x128x128 channel mix runs on the tensor cores (mma.sync m16n8k16 fp16,
+// fp32 accumulate): the rounding of s adds an error of the size of the fp16
+// rounding that q and k get anyway. Each thread owns the same accumulator positions
 // for every head, so c_k and the sum of the c_q stay in registers, and its
 // columns come in pairs (c, c+64), so RoPE is applied in registers. Output
 // tiles are staged in shared memory and written with 16-byte coalesced
@@ -51,7 +52,8 @@ struct Theta {
 
 struct PreParams {
   const __half* lat;  // [T, Nlat] q~ | k~ | v~
-  const __nv_bfloat16 *cq_seq, *cq_chan, *ck_seq, *ck_chan;
+  const __nv_bfloat16 *cq_seq, *ck_seq;
+  const __half *cq_chan, *ck_chan;  // fp16 copies of the channel-conv weights
   __half* q;                          // [T, Lq]
   __nv_bfloat16 *k_cache, *v_cache;   // [T, Lkv]
   __half *k_att, *v_att;              // [T, Lkv]
@@ -81,10 +83,10 @@ __device__ __forceinline__ void ldsm_x4(uint32_t addr, uint32_t& r0, uint32_t& r
                : "r"(addr));
 }
 
-__device__ __forceinline__ void mma_bf16_16816(float* c, uint32_t a0, uint32_t a1, uint32_t a2, uint32_t a3,
-                                               uint32_t b0, uint32_t b1) {
+__device__ __forceinline__ void mma_f16_16816(float* c, uint32_t a0, uint32_t a1, uint32_t a2, uint32_t a3,
+                                              uint32_t b0, uint32_t b1) {
   asm volatile(
-      "mma.sync.aligned.m16n8k16.row.col.f32.bf16.bf16.f32 {%0,%1,%2,%3}, {%4,%5,%6,%7}, {%8,%9}, "
+      "mma.sync.aligned.m16n8k16.row.col.f32.f16.f16.f32 {%0,%1,%2,%3}, {%4,%5,%6,%7}, {%8,%9}, "
       "{%0,%1,%2,%3};"
       : "+f"(c[0]), "+f"(c[1]), "+f"(c[2]), "+f"(c[3])
       : "r"(a0), "r"(a1), "r"(a2), "r"(a3), "r"(b0), "r"(b1));
@@ -94,14 +96,11 @@ __device__ __forceinline__ void mma_bf16_16816(float* c, uint32_t a0, uint32_t a
 // taps when known at compile time (0: p.K taps, at most KMAX). Row t of the output uses staged
 // rows t .. t+K-1 (tap K-1 on the current token).
 template <int KC>
-__device__ __forceinline__ void seq_conv(const PreParams& p, const __half* zbuf, __nv_bfloat16* shi,
-                                         __nv_bfloat16* slo, const __nv_bfloat16* wseq /* shared [D][K] */) {
+__device__ __forceinline__ void seq_conv(const PreParams& p, const __half* zbuf, __half* sbuf,
+                                         const __nv_bfloat16* wseq /* shared [D][K] */) {
   const int cp = threadIdx.x % (D / 2);  // column pair
   auto emit = [&](int t, float a0, float a1) {
-    const __nv_bfloat162 hi = __floats2bfloat162_rn(a0, a1);
-    const float2 hf = __bfloat1622float2(hi);
-    *reinterpret_cast<__nv_bfloat162*>(shi + t * ROWH + 2 * cp) = hi;
-    *reinterpret_cast<__nv_bfloat162*>(slo + t * ROWH + 2 * cp) = __floats2bfloat162_rn(a0 - hf.x, a1 - hf.y);
+    *reinterpret_cast<__half2*>(sbuf + t * ROWH + 2 * cp) = __floats2half2_rn(a0, a1);
   };
   auto zrow = [&](int r) { return __half22float2(*reinterpret_cast<const __half2*>(zbuf + r * ROWH + 2 * cp)); };
   if constexpr (KC > 0) {
@@ -147,10 +146,9 @@ __device__ __forceinline__ void seq_conv(const PreParams& p, const __half* zbuf,
   }
 }
 
-// Channel mix of the warp's 16 rows x 4 n-tiles: acc[nt][0..3] (m16n8 layout),
-// acc = (s_hi + s_lo) W^T.
-__device__ __forceinline__ void channel_mix(const __nv_bfloat16* shi, const __nv_bfloat16* slo,
-                                            const __nv_bfloat16* wbuf, int rb, const int* ncol,
+// Channel mix of the warp's 16 rows x 4 n-tiles: acc[nt][0..3] (m16n8 layout), acc = s W^T
+// (fp16 s and W, fp32 accumulation).
+__device__ __forceinline__ void channel_mix(const __half* sbuf, const __half* wbuf, int rb, const int* ncol,
                                             float (&acc)[4][4]) {
   const int lane = threadIdx.x & 31;
 #pragma unroll
@@ -158,7 +156,7 @@ __device__ __forceinline__ void channel_mix(const __nv_bfloat16* shi, const __nv
 #pragma unroll
     for (int e = 0; e < 4; ++e) acc[nt][e] = 0.f;
   const int arow = (rb + (lane & 15)) * ROWH + (lane >> 4) * 8;
-  const uint32_t ahi = smem_u32(shi + arow), alo = smem_u32(slo + arow);
+  const uint32_t abase = smem_u32(sbuf + arow);
   // B matrix m = lane / 8: rows ncol[0] + (m / 2) * 8 + (lane % 8), k chunk 2 ks + (m % 2), which
   // sits at chunk (2 ks) ^ y of the swizzled row, y = (m % 2) ^ (row % 8)
   const int brow = ncol[0] + ((lane >> 4) << 3) + (lane & 7);
@@ -170,38 +168,33 @@ __device__ __forceinline__ void channel_mix(const __nv_bfloat16* shi, const __nv
   constexpr uint32_t kB1 = 64 * D * 2;  // rows ncol[2] = ncol[0] + 64
 #pragma unroll
   for (int ks = 0; ks < D / 16; ++ks) {
-    uint32_t h0, h1, h2, h3, l0, l1, l2, l3, b0, b1, b2, b3, c0, c1, c2, c3;
+    uint32_t a0, a1, a2, a3, b0, b1, b2, b3, c0, c1, c2, c3;
     const uint32_t bk = bq[ks & 3] + (ks >> 2) * 128;
-    ldsm_x4(ahi + ks * 32, h0, h1, h2, h3);
-    ldsm_x4(alo + ks * 32, l0, l1, l2, l3);
+    ldsm_x4(abase + ks * 32, a0, a1, a2, a3);
     ldsm_x4(bk, b0, b1, b2, b3);
     ldsm_x4(bk + kB1, c0, c1, c2, c3);
-    mma_bf16_16816(acc[0], h0, h1, h2, h3, b0, b1);
-    mma_bf16_16816(acc[1], h0, h1, h2, h3, b2, b3);
-    mma_bf16_16816(acc[2], h0, h1, h2, h3, c0, c1);
-    mma_bf16_16816(acc[3], h0, h1, h2, h3, c2, c3);
-    mma_bf16_16816(acc[0], l0, l1, l2, l3, b0, b1);
-    mma_bf16_16816(acc[1], l0, l1, l2, l3, b2, b3);
-    mma_bf16_16816(acc[2], l0, l1, l2, l3, c0, c1);
-    mma_bf16_16816(acc[3], l0, l1, l2, l3, c2, c3);
+    mma_f16_16816(acc[0], a0, a1, a2, a3, b0, b1);
+    mma_f16_16816(acc[1], a0, a1, a2, a3, b2, b3);
+    mma_f16_16816(acc[2], a0, a1, a2, a3, c0, c1);
+    mma_f16_16816(acc[3], a0, a1, a2, a3, c2, c3);
   }
 }
 
-// Stream one head's channel-mix weights [out i][in j] (bf16) into wbuf: row i holds 16 chunks of
+// Stream one head's channel-mix weights [out i][in j] (fp16) into wbuf: row i holds 16 chunks of
 // 8 inputs, chunk c stored at position c ^ (i % 8).
-__device__ __forceinline__ void load_weights_async(const __nv_bfloat16* W, __nv_bfloat16* wbuf) {
+__device__ __forceinline__ void load_weights_async(const __half* W, __half* wbuf) {
   // thread: chunk v of rows r, r + 16, ... (r % 8 and so the swizzle stay fixed)
   const int v = threadIdx.x % (D / 8), r = threadIdx.x / (D / 8);
   const uint32_t dst = smem_u32(wbuf + r * D + ((v ^ (r & 7)) << 3));
-  const __nv_bfloat16* src = W + r * D + v * 8;
+  const __half* src = W + r * D + v * 8;
   constexpr int kRows = NT / (D / 8);
 #pragma unroll
   for (int k = 0; k < D / kRows; ++k) cp_async16(dst + k * kRows * D * 2, src + k * kRows * D, true);
 }
 
-// Byte offset of the RoPE tables: after the weight buffers, the s tiles, the latents and the seq taps.
+// Byte offset of the RoPE tables: after the weight buffers, the s tile, the latents and the seq taps.
 __host__ __device__ __forceinline__ size_t rope_table_offset(int H1, int K, int nbuf) {
-  const size_t end = 2 * ((size_t)nbuf * WTILE + 2 * (size_t)TT * ROWH + (size_t)H1 * (TT + K - 1) * ROWH +
+  const size_t end = 2 * ((size_t)nbuf * WTILE + (size_t)TT * ROWH + (size_t)H1 * (TT + K - 1) * ROWH +
                           (size_t)H1 * D * K);
   return (end + 15) & ~(size_t)15;
 }
@@ -214,13 +207,12 @@ __global__ void __launch_bounds__(NT, 2) preproc_tc_kernel(const __grid_constant
   const int H1 = G + 1;
   const int KK = KC > 0 ? KC : p.K;  // seq-conv taps
   const int ZR = TT + KK - 1;        // staged rows per head
-  __nv_bfloat16* wbuf = reinterpret_cast<__nv_bfloat16*>(smem_raw);  // nbuf x [D][D] channel weights
-  __nv_bfloat16* shi = wbuf + p.nbuf * WTILE;                         // [TT][ROWH] s, bf16 high part
-  __nv_bfloat16* slo = shi + TT * ROWH;                               // [TT][ROWH] s, bf16 low part
-  __half* zall = reinterpret_cast<__half*>(slo + TT * ROWH);          // [H1][ZR][ROWH] latents; head G = k
+  __half* wbuf = reinterpret_cast<__half*>(smem_raw);  // nbuf x [D][D] channel weights (fp16)
+  __half* sbuf = wbuf + p.nbuf * WTILE;                // [TT][ROWH] seq-conv output s (fp16)
+  __half* zall = sbuf + TT * ROWH;                     // [H1][ZR][ROWH] latents; head G = k
   __nv_bfloat16* wsq = reinterpret_cast<__nv_bfloat16*>(zall + H1 * ZR * ROWH);  // [H1][D][K] seq taps
   float2* rtab = reinterpret_cast<float2*>(smem_raw + rope_table_offset(H1, KK, p.nbuf));  // [2][D/2] RoPE
-  __half* stage = reinterpret_cast<__half*>(shi);                     // [TT][ROWH] q output stage
+  __half* stage = sbuf;                                               // [TT][ROWH] q output stage
   float* kst = reinterpret_cast<float*>(wbuf);                        // [TT][KSTR] k stage (fp32)
   // weights of the i-th head in processing order (0: the K head, then query heads 0..G-1)
   auto wslot = [&](int i) { return wbuf + (p.nbuf == 2 ? (i & 1) : 0) * WTILE; };
@@ -341,10 +333,10 @@ __global__ void __launch_bounds__(NT, 2) preproc_tc_kernel(const __grid_constant
       rc[nt][2 + e1] = c1;
       rs[nt][2 + e1] = s1;
     }
-  seq_conv<KC>(p, zall + G * ZR * ROWH, shi, slo, wsq + G * D * KK);
+  seq_conv<KC>(p, zall + G * ZR * ROWH, sbuf, wsq + G * D * KK);
   __syncthreads();
   float ck[4][4];
-  channel_mix(shi, slo, wslot(0), rb, ncol, ck);
+  channel_mix(sbuf, wslot(0), rb, ncol, ck);
   float csum[4][4];
 #pragma unroll
   for (int nt = 0; nt < 4; ++nt)
@@ -354,18 +346,18 @@ __global__ void __launch_bounds__(NT, 2) preproc_tc_kernel(const __grid_constant
   // ---- the G query heads
   for (int hh = 0; hh < G; ++hh) {
     const int h = g * G + hh;
-    __syncthreads();  // shi, slo and the previous head's weight buffer are free
+    __syncthreads();  // sbuf and the previous head's weight buffer are free
     // weights of query head hh + 1 (double buffering) or hh (single buffer)
     const int next = p.nbuf == 2 ? hh + 1 : hh;
     const bool issue = next < G;
     if (issue) load_weights_async(p.cq_chan + (long long)(g * G + next) * D * D, wslot(next + 1));
     cp_async_commit();
-    seq_conv<KC>(p, zall + hh * ZR * ROWH, shi, slo, wsq + hh * D * KK);
+    seq_conv<KC>(p, zall + hh * ZR * ROWH, sbuf, wsq + hh * D * KK);
     if (p.nbuf == 2) cp_async_wait<1>();  // all but the group just committed: head hh's weights
     else cp_async_wait<0>();
     __syncthreads();
     float acc[4][4];
-    channel_mix(shi, slo, wslot(hh + 1), rb, ncol, acc);
+    channel_mix(sbuf, wslot(hh + 1), rb, ncol, acc);
 #pragma unroll
     for (int nt = 0; nt < 4; ++nt)
 #pragma unroll
@@ -385,7 +377,7 @@ __global__ void __launch_bounds__(NT, 2) preproc_tc_kernel(const __grid_constant
         }
       }
     if (p.use_rope) rope(acc);
-    __syncthreads();  // shi becomes the q stage
+    __syncthreads();  // sbuf becomes the q stage
 #pragma unroll
     for (int nt = 0; nt < 4; ++nt) {
       const int col = ncol[nt] + cq;
@@ -507,9 +499,9 @@ cudaError_t launch_preproc_tc(const BlockDims& dm, const BlockPtrs& p, cudaStrea
   PreParams q;
   q.lat = static_cast<const __half*>(p.qkv_lat);
   q.cq_seq = static_cast<const __nv_bfloat16*>(p.cq_seq);
-  q.cq_chan = static_cast<const __nv_bfloat16*>(p.cq_chan);
+  q.cq_chan = static_cast<const __half*>(p.wc_lat);
   q.ck_seq = static_cast<const __nv_bfloat16*>(p.ck_seq);
-  q.ck_chan = static_cast<const __nv_bfloat16*>(p.ck_chan);
+  q.ck_chan = static_cast<const __half*>(p.wc_lat) + (long long)dm.nq * D * D;
   q.q = static_cast<__half*>(p.q);
   q.k_cache = static_cast<__nv_bfloat16*>(p.k_cache);
   q.v_cache = static_cast<__nv_bfloat16*>(p.v_cache);

@@ -7,6 +7,8 @@
 //  * attention_simt_kernel: causal softmax attention on the compressed heads,
 //    one K/V head per group of G query heads (es 2.A and 2.C), computed with
 //    an online softmax over key tiles.
+//  * convert_f16_kernel: an fp16 copy of a bf16 array (the intermediate-type copy of the
+//    channel-conv weights when no tensor-core down-projection carries it as a side job).
 #include "cca_common.cuh"
 #include "launch.h"
 
@@ -212,6 +214,28 @@ cudaError_t launch_attention_simt(const BlockDims& dm, const void* q, const void
   } else {
     return cudaErrorInvalidValue;
   }
+  return cudaGetLastError();
+}
+
+namespace {
+__global__ void __launch_bounds__(256) convert_f16_kernel(const __nv_bfloat16* __restrict__ src, __half* __restrict__ dst,
+                                                          long long n, unsigned* err) {
+  bool bad = false;
+  for (long long i = (long long)blockIdx.x * blockDim.x + threadIdx.x; i < n; i += (long long)gridDim.x * blockDim.x) {
+    const float f = __bfloat162float(src[i]);
+    bad |= f16_overflow(f);
+    dst[i] = __float2half_rn(f);
+  }
+  report_range(bad, err);
+}
+}  // namespace
+
+cudaError_t launch_convert_f16(const void* src, void* dst, long long n, unsigned* dev_err, cudaStream_t stream) {
+  if (n <= 0) return cudaSuccess;
+  long long blocks = (n + 255) / 256;
+  if (blocks > 1184) blocks = 1184;
+  convert_f16_kernel<<<(unsigned)blocks, 256, 0, stream>>>(static_cast<const __nv_bfloat16*>(src),
+                                                             static_cast<__half*>(dst), n, dev_err);
   return cudaGetLastError();
 }
 

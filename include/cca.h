@@ -122,7 +122,8 @@ typedef struct cca_prefill_opts {
  * blocks are fp16 (same tensor-core rate as bf16, 8x finer rounding), which
  * keeps the block's chain of roundings small; inputs, the KV cache and y keep
  * cfg->dtype / cfg->out_dtype. For fp32 blocks the k_att / v_att / W_o
- * regions are empty (the attention reads the KV cache and W_o directly). */
+ * regions are empty (the attention reads the KV cache and W_o directly), and
+ * so is the W_c region. */
 typedef struct cca_workspace_layout {
   size_t total_bytes;
   size_t elem_bytes;        /* bytes per intermediate element */
@@ -134,6 +135,8 @@ typedef struct cca_workspace_layout {
   size_t v_att_offset;      /* [T, Lkv]: v as the attention reads it */
   size_t o_offset;          /* [T, Lq]: attention output, heads concatenated */
   size_t wo_offset;         /* [E, Lq]: W_o in the intermediate type */
+  size_t wc_offset;         /* [n_q + n_kv, d, d]: channel-conv weights (q heads, then K heads) in the
+                               intermediate type */
   size_t sched_offset;      /* scratch of the attention kernel: split-pair counters and partial rows */
 } cca_workspace_layout_t;
 

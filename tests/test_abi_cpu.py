@@ -30,7 +30,7 @@ def test_library_exports_every_declared_function():
 
 def test_struct_layouts():
     assert ctypes.sizeof(cca.CcaConfig) == 15 * 4
-    assert ctypes.sizeof(cca.CcaWorkspaceLayout) == 2 * 8 + 2 * 4 + 7 * 8
+    assert ctypes.sizeof(cca.CcaWorkspaceLayout) == 2 * 8 + 2 * 4 + 8 * 8
 
 
 def good(**kw):
@@ -50,10 +50,11 @@ def test_valid_configs_and_workspace():
     assert lay.v_att_offset - lay.k_att_offset >= T * Lkv * 2
     assert lay.o_offset - lay.v_att_offset >= T * Lkv * 2
     assert lay.wo_offset - lay.o_offset >= T * Lq * 2
-    assert lay.sched_offset - lay.wo_offset >= 2048 * Lq * 2
+    assert lay.wc_offset - lay.wo_offset >= 2048 * Lq * 2
+    assert lay.sched_offset - lay.wc_offset >= (4 + 2) * 128 * 128 * 2
     assert cca.workspace_size(cfg) == lay.total_bytes
     for off in (lay.qkv_lat_offset, lay.q_offset, lay.k_att_offset, lay.v_att_offset, lay.o_offset,
-                lay.wo_offset, lay.sched_offset, lay.total_bytes):
+                lay.wo_offset, lay.wc_offset, lay.sched_offset, lay.total_bytes):
         assert off % 256 == 0
     tiny = cca.make_config(batch=1, seq_len=64, hidden=128, n_q_heads=2, n_kv_heads=2, head_dim=16, dtype="f32")
     assert cca.validate(tiny) == cca.CCA_OK
