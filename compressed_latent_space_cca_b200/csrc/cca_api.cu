@@ -229,7 +229,7 @@ cca_status_t run_block(const Resolved& r, BlockPtrs p, cudaStream_t stream, void
     int col = 0;
     for (int i = 0; i < 3; ++i) {
       if ((e = launch_gemm_simt(dm.io, dm.lat, p.x, dm.E, Ws[i], dm.E, out + (size_t)col * eb, dm.Nlat, dm.T,
-                                ns[i], dm.E, stream)) != cudaSuccess)
+                                ns[i], dm.E, stream, p.dev_err)) != cudaSuccess)
         return cuda_fail("down-projection (SIMT)", e);
       col += ns[i];
     }
@@ -275,8 +275,8 @@ cca_status_t run_block(const Resolved& r, BlockPtrs p, cudaStream_t stream, void
     a.dev_err = p.dev_err;
     if ((e = launch_gemm_tc(a, stream)) != cudaSuccess) return cuda_fail("output projection (tcgen05)", e);
   } else {
-    if ((e = launch_gemm_simt(dm.lat, dm.out, p.o, dm.Lq, p.wo_lat, dm.Lq, p.y, dm.E, dm.T, dm.E, dm.Lq,
-                              stream)) != cudaSuccess)
+    if ((e = launch_gemm_simt(dm.lat, dm.out, p.o, dm.Lq, p.wo_lat, dm.Lq, p.y, dm.E, dm.T, dm.E, dm.Lq, stream,
+                              p.dev_err)) != cudaSuccess)
       return cuda_fail("output projection (SIMT)", e);
   }
   if ((e = mark(4)) != cudaSuccess) return cuda_fail("event", e);

@@ -50,7 +50,8 @@ struct BlockPtrs {
 // ---- SIMT path (any dtype, any even head_dim <= 128) ----
 // C[M, ldc] (cols [0,N)) = A[M,K] (row stride lda) * B[N,K]^T (row stride ldb)
 cudaError_t launch_gemm_simt(DType in, DType out, const void* A, long long lda, const void* Bm, long long ldb,
-                             void* C, long long ldc, long long M, int N, int K, cudaStream_t stream);
+                             void* C, long long ldc, long long M, int N, int K, cudaStream_t stream,
+                             unsigned* dev_err);  // fp16 outputs beyond fp16's range are reported here
 cudaError_t launch_attention_simt(const BlockDims& dm, const void* q, const void* k, const void* v, void* o,
                                   cudaStream_t stream);
 

@@ -228,6 +228,7 @@ __global__ void __launch_bounds__(NT, 2) preproc_tc_kernel(const __grid_constant
   const int cq = (lane & 3) * 2;
   const int zr0 = r0 + KK - 1, zr1 = r1 + KK - 1;  // current-token rows in the latent tiles
   bool bad = false;
+  float amax = 0.f;  // largest |q|, |k| of this thread
 
   // ---- all latents of the group (query heads 0..G-1, then the K head) and the K head's weights
   for (int R = threadIdx.x / (D / 8); R < H1 * ZR; R += NT / (D / 8)) {
@@ -242,10 +243,20 @@ __global__ void __launch_bounds__(NT, 2) preproc_tc_kernel(const __grid_constant
   cp_async_commit();
   if (p.nbuf == 2) load_weights_async(p.cq_chan + (long long)g * G * D * D, wslot(1));
   cp_async_commit();  // (an empty group when nbuf == 1)
-  // seq-conv taps of the group's heads, [H1][D][K]: query heads g*G .. g*G+G-1, then the K head
-  for (int e = threadIdx.x; e < H1 * D * KK; e += NT) {
-    const int hh = e / (D * KK), rem = e % (D * KK);
-    wsq[e] = hh < G ? p.cq_seq[(long long)(g * G + hh) * D * KK + rem] : p.ck_seq[(long long)g * D * KK + rem];
+  // seq-conv taps of the group's heads, [H1][D][K]: query heads g*G .. g*G+G-1 (contiguous in
+  // cq_seq), then the K head; 16-byte vectors when both sources allow them
+  {
+    const __nv_bfloat16* qs = p.cq_seq + (long long)g * G * D * KK;
+    const __nv_bfloat16* ks = p.ck_seq + (long long)g * D * KK;
+    if (((reinterpret_cast<uintptr_t>(qs) | reinterpret_cast<uintptr_t>(ks)) & 15) == 0) {
+      const int nq8 = G * D * KK / 8, n8 = H1 * D * KK / 8;  // D * KK is a multiple of 8
+      for (int v = threadIdx.x; v < n8; v += NT)
+        reinterpret_cast<uint4*>(wsq)[v] =
+            v < nq8 ? reinterpret_cast<const uint4*>(qs)[v] : reinterpret_cast<const uint4*>(ks)[v - nq8];
+    } else {
+      for (int e = threadIdx.x; e < H1 * D * KK; e += NT)
+        wsq[e] = e < G * D * KK ? qs[e] : ks[e - G * D * KK];
+    }
   }
 
   // ---- side job, issued while the copies are in flight: this CTA's slice of W_o as fp16 (8-element vectors)
@@ -384,7 +395,7 @@ __global__ void __launch_bounds__(NT, 2) preproc_tc_kernel(const __grid_constant
       *reinterpret_cast<__half2*>(stage + r0 * ROWH + col) = __floats2half2_rn(acc[nt][0], acc[nt][1]);
       *reinterpret_cast<__half2*>(stage + r1 * ROWH + col) = __floats2half2_rn(acc[nt][2], acc[nt][3]);
 #pragma unroll
-      for (int e = 0; e < 4; ++e) bad |= f16_overflow(acc[nt][e]);
+      for (int e = 0; e < 4; ++e) amax = fmaxf(amax, fabsf(acc[nt][e]));
     }
     __syncthreads();
     for (int e = threadIdx.x; e < TT * (D / 8); e += NT) {
@@ -443,7 +454,7 @@ __global__ void __launch_bounds__(NT, 2) preproc_tc_kernel(const __grid_constant
       *reinterpret_cast<float2*>(kst + r0 * KSTR + col) = make_float2(val[nt][0], val[nt][1]);
       *reinterpret_cast<float2*>(kst + r1 * KSTR + col) = make_float2(val[nt][2], val[nt][3]);
 #pragma unroll
-      for (int e = 0; e < 4; ++e) bad |= f16_overflow(val[nt][e]);
+      for (int e = 0; e < 4; ++e) amax = fmaxf(amax, fabsf(val[nt][e]));
     }
   }
   __syncthreads();
@@ -478,7 +489,8 @@ __global__ void __launch_bounds__(NT, 2) preproc_tc_kernel(const __grid_constant
     *reinterpret_cast<uint4*>(p.v_att + off) = hv;
   }
 
-  report_range(bad, p.err);
+  // q and k leave as fp16: any of this thread's values beyond fp16's range (infinities included)
+  report_range(bad || amax > 65504.0f, p.err);
 }
 
 size_t smem_bytes(int G, int K, int nbuf) { return rope_table_offset(G + 1, K, nbuf) + sizeof(float2) * D; }

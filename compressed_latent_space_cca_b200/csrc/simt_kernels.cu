@@ -9,6 +9,8 @@
 //    an online softmax over key tiles.
 //  * convert_f16_kernel: an fp16 copy of a bf16 array (the intermediate-type copy of the
 //    channel-conv weights when no tensor-core down-projection carries it as a side job).
+#include <type_traits>
+
 #include "cca_common.cuh"
 #include "launch.h"
 
@@ -21,7 +23,7 @@ template <typename Tin, typename Tout>
 __global__ void __launch_bounds__(256) gemm_simt_kernel(const Tin* __restrict__ A, long long lda,
                                                         const Tin* __restrict__ Bm, long long ldb,
                                                         Tout* __restrict__ C, long long ldc, long long M, int N,
-                                                        int K) {
+                                                        int K, unsigned* err) {
   __shared__ float As[GT_K][GT_M + 4];
   __shared__ float Bs[GT_K][GT_N + 4];
   const int tid = threadIdx.x;
@@ -54,6 +56,7 @@ __global__ void __launch_bounds__(256) gemm_simt_kernel(const Tin* __restrict__ 
     }
     __syncthreads();
   }
+  float amax = 0.f;  // largest |C| stored, for the fp16 range report
 #pragma unroll
   for (int i = 0; i < 4; ++i) {
     long long gm = m0 + tr * 4 + i;
@@ -61,9 +64,13 @@ __global__ void __launch_bounds__(256) gemm_simt_kernel(const Tin* __restrict__ 
 #pragma unroll
     for (int j = 0; j < 4; ++j) {
       int gn = n0 + tc * 4 + j;
-      if (gn < N) st_f(C + gm * ldc + gn, acc[i][j]);
+      if (gn < N) {
+        st_f(C + gm * ldc + gn, acc[i][j]);
+        amax = fmaxf(amax, fabsf(acc[i][j]));
+      }
     }
   }
+  if (std::is_same<Tout, __half>::value) report_range(amax > 65504.0f, err);
 }
 
 // Causal attention, SIMT. One CTA = 64 query rows of one query head; two
@@ -165,29 +172,32 @@ __global__ void __launch_bounds__(128) attention_simt_kernel(const T* __restrict
 namespace {
 template <typename Tin, typename Tout>
 void gemm_simt_typed(const void* A, long long lda, const void* Bm, long long ldb, void* C, long long ldc,
-                     long long M, int N, int K, dim3 grid, cudaStream_t stream) {
+                     long long M, int N, int K, unsigned* err, dim3 grid, cudaStream_t stream) {
   gemm_simt_kernel<Tin, Tout><<<grid, 256, 0, stream>>>((const Tin*)A, lda, (const Tin*)Bm, ldb, (Tout*)C, ldc, M,
-                                                         N, K);
+                                                         N, K, err);
 }
 template <typename Tin>
 void gemm_simt_out(DType out, const void* A, long long lda, const void* Bm, long long ldb, void* C, long long ldc,
-                   long long M, int N, int K, dim3 grid, cudaStream_t stream) {
+                   long long M, int N, int K, unsigned* err, dim3 grid, cudaStream_t stream) {
   switch (out) {
-    case DType::F32: gemm_simt_typed<Tin, float>(A, lda, Bm, ldb, C, ldc, M, N, K, grid, stream); break;
-    case DType::BF16: gemm_simt_typed<Tin, __nv_bfloat16>(A, lda, Bm, ldb, C, ldc, M, N, K, grid, stream); break;
-    case DType::F16: gemm_simt_typed<Tin, __half>(A, lda, Bm, ldb, C, ldc, M, N, K, grid, stream); break;
+    case DType::F32: gemm_simt_typed<Tin, float>(A, lda, Bm, ldb, C, ldc, M, N, K, err, grid, stream); break;
+    case DType::BF16: gemm_simt_typed<Tin, __nv_bfloat16>(A, lda, Bm, ldb, C, ldc, M, N, K, err, grid, stream); break;
+    case DType::F16: gemm_simt_typed<Tin, __half>(A, lda, Bm, ldb, C, ldc, M, N, K, err, grid, stream); break;
   }
 }
 }  // namespace
 
 cudaError_t launch_gemm_simt(DType in, DType out, const void* A, long long lda, const void* Bm, long long ldb,
-                             void* C, long long ldc, long long M, int N, int K, cudaStream_t stream) {
+                             void* C, long long ldc, long long M, int N, int K, cudaStream_t stream,
+                             unsigned* dev_err) {
   if (M <= 0 || N <= 0) return cudaSuccess;
   dim3 grid((N + GT_N - 1) / GT_N, (unsigned)((M + GT_M - 1) / GT_M));
   switch (in) {
-    case DType::F32: gemm_simt_out<float>(out, A, lda, Bm, ldb, C, ldc, M, N, K, grid, stream); break;
-    case DType::BF16: gemm_simt_out<__nv_bfloat16>(out, A, lda, Bm, ldb, C, ldc, M, N, K, grid, stream); break;
-    case DType::F16: gemm_simt_out<__half>(out, A, lda, Bm, ldb, C, ldc, M, N, K, grid, stream); break;
+    case DType::F32: gemm_simt_out<float>(out, A, lda, Bm, ldb, C, ldc, M, N, K, dev_err, grid, stream); break;
+    case DType::BF16:
+      gemm_simt_out<__nv_bfloat16>(out, A, lda, Bm, ldb, C, ldc, M, N, K, dev_err, grid, stream);
+      break;
+    case DType::F16: gemm_simt_out<__half>(out, A, lda, Bm, ldb, C, ldc, M, N, K, dev_err, grid, stream); break;
   }
   return cudaGetLastError();
 }

@@ -40,3 +40,25 @@ def test_invalid_calls_rejected_before_launch():
     assert ei.value.status == cca.CCA_ERR_INVALID_ARG
     torch.cuda.synchronize()
     assert torch.equal(out["y"], sentinel)  # outputs untouched
+
+
+@pytest.mark.parametrize("path", [cca.CCA_PATH_AUTO, cca.CCA_PATH_SIMT], ids=["auto", "simt"])
+@pytest.mark.parametrize("where", ["latents", "channel_mix"])
+def test_fp16_range_reported(path, where):
+    """bf16 blocks keep their intermediates in fp16. Values beyond fp16's range
+    are reported by the next status poll as a numeric-range error, not passed on
+    silently: latents that overflow in the down-projection, or q after a channel
+    mix whose weights are fine in fp16 but whose outputs are not."""
+    sh = workloads.BlockShape("range", 1, 300, 512, 4, 2, 128, 4, "bf16", 5)
+    inp = workloads.make_inputs(sh)
+    if where == "latents":
+        inp["x"] = (inp["x"].float() * 1e5).to(torch.bfloat16)
+    else:  # latents below 6 and weights below 43k, but about 4 % of q beyond 65504
+        inp["x"] = (inp["x"].float() * 3).to(torch.bfloat16)
+        inp["convq_chan"] = (inp["convq_chan"].float() * 1e5).to(torch.bfloat16)
+        assert float(inp["convq_chan"].float().abs().max()) < 65504.0
+    cfg = cca.config_from_shape(sh)
+    assert cca.poll_device_status() == cca.CCA_OK
+    cca.prefill(cfg, {k: v.cuda() for k, v in inp.items()}, path=path)
+    assert cca.poll_device_status() == cca.CCA_ERR_NUMERIC_RANGE
+    assert cca.poll_device_status() == cca.CCA_OK  # cleared by the poll
