@@ -88,6 +88,7 @@ __device__ __forceinline__ void exp2_fma_x2(float x0, float x1, float& p0, float
 
 struct AttnMaps {
   CUtensorMap q, k, v;
+  CUtensorMap o;  // attention output, boxes of 64 columns x 32 rows (one warp's rows)
 };
 
 struct AttnParams {
@@ -179,7 +180,8 @@ __global__ void __launch_bounds__(NUM_THREADS, 1) attn_tc_kernel(const __grid_co
   uint64_t* s_full = v_empty + V_STAGES;   // [2]
   uint64_t* p_full = s_full + 2;           // [2]
   uint64_t* o_full = p_full + 2;           // [2]
-  uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(o_full + 2);
+  uint64_t* q_stage_free = o_full + 2;     // [2] Q_j's buffer, used to stage O_j, may take the next Q_j
+  uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(q_stage_free + 2);
   volatile int* abort_flag = reinterpret_cast<volatile int*>(tmem_slot + 1);
 
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
@@ -198,6 +200,7 @@ __global__ void __launch_bounds__(NUM_THREADS, 1) attn_tc_kernel(const __grid_co
       mbar_init(smem_u32(&s_full[j]), 1);
       mbar_init(smem_u32(&p_full[j]), 4);
       mbar_init(smem_u32(&o_full[j]), 1);
+      mbar_init(smem_u32(&q_stage_free[j]), 4);
     }
     *abort_flag = 0;
     fence_mbar_init();
@@ -227,6 +230,11 @@ __global__ void __launch_bounds__(NUM_THREADS, 1) attn_tc_kernel(const __grid_co
         if (w < 0) break;
         const Item it = get_item(p, w);
         if (!mbar_wait_bounded(smem_u32(q_empty), (r & 1) ^ 1, p.err, abort_flag, wait_site(kSiteAttn, 1, 1))) goto done;
+        // the softmax groups stage the previous entry's O in the Q buffers and release them per tile
+        for (int j = 0; j < 2; ++j)
+          if (r > 0 && !mbar_wait_bounded(smem_u32(&q_stage_free[j]), (r - 1) & 1, p.err, abort_flag,
+                                          wait_site(kSiteAttn, 1, 13)))
+            goto done;
         mbar_arrive_expect_tx(smem_u32(q_full), 2 * TILE_BYTES);
 #pragma unroll
         for (int j = 0; j < 2; ++j)
@@ -453,7 +461,6 @@ __global__ void __launch_bounds__(NUM_THREADS, 1) attn_tc_kernel(const __grid_co
         if (!mbar_wait_bounded(smem_u32(&o_full[j]), ocount & 1, p.err, abort_flag, wait_site(kSiteAttn, 3, 11))) goto done;
         ++ocount;
         tc_fence_after();
-        const int t = qt * TQ + row;
         // O_row = O * inv for a whole-range entry; a merged split pair gives c1 * O_first + c2 * O_second,
         // evaluated in that order whichever half merges, so the result does not depend on timing
         float c1 = 0.f, c2 = 0.f, inv = 1.f / l;
@@ -496,7 +503,9 @@ __global__ void __launch_bounds__(NUM_THREADS, 1) attn_tc_kernel(const __grid_co
             inv = 1.f;  // the raw O rows are merged
           }
         }
-        __half* dst = p.o + ((long long)it.b * p.S + t) * p.Lq + (long long)it.h[j] * D;
+        // O rows leave through Q_j's buffer (its last QK has completed): [2 halves][128 rows][128 B]
+        // with the 128-byte swizzle, one TMA tensor store per 64-column half of this warp's 32 rows
+        uint8_t* stage = smem + OFF_Q + j * TILE_BYTES;
 #pragma unroll 1
         for (int c = 0; c < 4 && store; ++c) {
           uint32_t o[32];
@@ -519,36 +528,48 @@ __global__ void __launch_bounds__(NUM_THREADS, 1) attn_tc_kernel(const __grid_co
               }
             }
           }
-          if (t < p.S) {
-            uint4* d4 = reinterpret_cast<uint4*>(dst + c * 32);
 #pragma unroll
-            for (int v = 0; v < 4; ++v) {
-              uint4 wv;
-              wv.x = pack_f16x2(f[8 * v + 0], f[8 * v + 1]);
-              wv.y = pack_f16x2(f[8 * v + 2], f[8 * v + 3]);
-              wv.z = pack_f16x2(f[8 * v + 4], f[8 * v + 5]);
-              wv.w = pack_f16x2(f[8 * v + 6], f[8 * v + 7]);
-              d4[v] = wv;
-            }
+          for (int u = 0; u < 4; ++u) {  // columns c*32 + 8u .. +7: half c/2, chunk (c%2)*4 + u
+            const int chunk = (c & 1) * 4 + u;
+            *reinterpret_cast<uint4*>(stage + (c >> 1) * HALF_BYTES + row * 128 + ((chunk ^ (row & 7)) << 4)) =
+                make_uint4(pack_f16x2(f[8 * u + 0], f[8 * u + 1]), pack_f16x2(f[8 * u + 2], f[8 * u + 3]),
+                           pack_f16x2(f[8 * u + 4], f[8 * u + 5]), pack_f16x2(f[8 * u + 6], f[8 * u + 7]));
+          }
+        }
+        if (store) {
+          fence_async_smem();
+          __syncwarp();
+          if (lane == 0) {  // rows past S are clipped by the map
+#pragma unroll
+            for (int hf = 0; hf < 2; ++hf)
+              tma_store_3d(&maps.o, smem_u32(stage + hf * HALF_BYTES + quad * 32 * 128), it.h[j] * D + hf * 64,
+                           qt * TQ + quad * 32, it.b);
+            bulk_commit();
           }
         }
         tc_fence_before();
       }
+      // every entry, active tile or not: Q_j's buffer may take the next entry's Q once this warp's
+      // stores have read it
+      if (lane == 0) bulk_wait_read<0>();
+      __syncwarp();
+      if (lane == 0) mbar_arrive(smem_u32(&q_stage_free[j]));
     }
   }
 done:
+  if (warp >= 2 && lane == 0) bulk_wait_all();  // staged stores finish before the CTA's shared memory goes
   tc_fence_before();
   __syncthreads();
   tc_fence_after();
   if (warp == 1) tmem_dealloc(tmem, TMEM_COLS);
 }
 
-bool encode_3d(CUtensorMap* m, const void* ptr, uint64_t width, uint64_t S, uint64_t B) {
+bool encode_3d(CUtensorMap* m, const void* ptr, uint64_t width, uint64_t S, uint64_t B, uint32_t box_rows = 128) {
   EncodeTiledFn enc = get_encode_tiled();
   if (enc == nullptr) return false;
   cuuint64_t dims[3] = {width, S, B};
   cuuint64_t strides[2] = {width * 2, width * S * 2};
-  cuuint32_t box[3] = {64, 128, 1};
+  cuuint32_t box[3] = {64, box_rows, 1};
   cuuint32_t estr[3] = {1, 1, 1};
   return enc(m, CU_TENSOR_MAP_DATA_TYPE_FLOAT16, 3, const_cast<void*>(ptr), dims, strides, box, estr,
              CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B, CU_TENSOR_MAP_L2_PROMOTION_L2_256B,
@@ -574,11 +595,6 @@ struct PairGeom {
   }
   static constexpr int kEntryCost = 4, kSplitCost = 4;
   int load(const BlockDims& dm, int w) const { return 2 * nkv(dm, w) + kEntryCost; }
-  long long total(const BlockDims& dm) const {
-    long long t = 0;
-    for (int w = 0; w < items; ++w) t += load(dm, w);
-    return t;
-  }
   // Most pairs that may be split in two (the longest ones, with at least 4 key tiles so that both
   // query tiles have keys in both halves).
   int max_split(const BlockDims& dm) const {
@@ -676,7 +692,8 @@ cudaError_t launch_attention_tc(const BlockDims& dm, const void* q, const void* 
   AttnMaps maps;
   if (!encode_3d(&maps.q, q, (uint64_t)dm.Lq, (uint64_t)dm.S, (uint64_t)dm.B) ||
       !encode_3d(&maps.k, k, (uint64_t)dm.Lkv, (uint64_t)dm.S, (uint64_t)dm.B) ||
-      !encode_3d(&maps.v, v, (uint64_t)dm.Lkv, (uint64_t)dm.S, (uint64_t)dm.B))
+      !encode_3d(&maps.v, v, (uint64_t)dm.Lkv, (uint64_t)dm.S, (uint64_t)dm.B) ||
+      !encode_3d(&maps.o, o, (uint64_t)dm.Lq, (uint64_t)dm.S, (uint64_t)dm.B, 32))
     return cudaErrorInvalidValue;
   AttnParams p;
   p.B = dm.B;
