@@ -375,6 +375,9 @@ def run_ours(args, shape):
             "gpu_launches": launches_per_step * args.steps,
             "clocks": clocks,
         }
+        if (world == 1 and not args.no_mha and my_shape.dtype == "bf16" and my_shape.conv_kernel > 0 and
+                my_shape.hidden % 128 == 0):
+            line["mha_baseline"] = run_mha_baseline(cca, dev, my_shape, ms_per_step)
         if world == 1 and not args.no_cpu_baseline:
             line["cpu_baseline"] = cpu_baseline(my_shape, inputs_cpu)
         print(json.dumps(line, default=float), flush=True)
@@ -382,6 +385,52 @@ def run_ours(args, shape):
         dist.barrier()
         dist.destroy_process_group()
     return 0
+
+
+def mha_shape(shape: workloads.BlockShape) -> workloads.BlockShape:
+    """The uncompressed baseline of a block: plain multi-head attention (C = 1, heads of 128, no
+    convolutions, QK-mean or value shift) with the same batch, sequence length and width."""
+    base = workloads.WORKLOADS["mha_16k_bf16"]
+    nh = shape.hidden // base.head_dim
+    return base.replace(name=f"mha_b{shape.batch}_s{shape.seq_len}_e{shape.hidden}", batch=shape.batch,
+                        seq_len=shape.seq_len, hidden=shape.hidden, n_q_heads=nh, n_kv_heads=nh)
+
+
+def run_mha_baseline(cca, dev, shape, cca_ms_per_step, steps=10, warmup=3):
+    """Times the plain multi-head block of the same shape with the same method (L2 flushed between
+    steps, CUDA events around each stage) and returns its numbers and the CCA block's speedup."""
+    mshape = mha_shape(shape)
+    cfg = cca.config_from_shape(mshape)
+    inputs = {k: v.to(dev) for k, v in workloads.make_inputs(mshape).items()}
+    out = cca.alloc_outputs(cfg, dev)
+    ws = cca.alloc_workspace(cfg, dev)
+    flush = torch.empty(L2_FLUSH_BYTES, dtype=torch.uint8, device=dev)
+    for _ in range(warmup):
+        flush.zero_()
+        cca.prefill(cfg, inputs, out=out, workspace=ws)
+    evs = [[torch.cuda.Event(enable_timing=True) for _ in range(5)] for _ in range(steps)]
+    torch.cuda.synchronize()
+    for i in range(steps):
+        flush.zero_()
+        cca.prefill(cfg, inputs, out=out, workspace=ws, stage_events=evs[i])
+    torch.cuda.synchronize()
+    if cca.poll_device_status() != 0:
+        raise SystemExit("device status error in the MHA baseline")
+    stage = np.array([[evs[i][j].elapsed_time(evs[i][j + 1]) for j in range(4)] for i in range(steps)])
+    ms = float(stage.sum(axis=1).mean())
+    stage_ms = stage.mean(axis=0)
+    work = algorithmic_work(mshape)
+    del inputs, out, ws, flush
+    torch.cuda.empty_cache()
+    return {
+        "workload": mshape.name, "n_q_heads": mshape.n_q_heads, "n_kv_heads": mshape.n_kv_heads,
+        "head_dim": mshape.head_dim, "C": mshape.compression, "steps": steps, "warmup": warmup,
+        "ms_per_step": ms, "tokens_per_s": mshape.tokens / (ms / 1e3),
+        "attention_tflops": work["attention_flops"] / (stage_ms[2] / 1e3) / 1e12,
+        "kernels_ms": {"down_proj": stage_ms[0], "rope_cache": stage_ms[1], "attention": stage_ms[2],
+                       "out_proj": stage_ms[3]},
+        "cca_speedup": ms / cca_ms_per_step,
+    }
 
 
 def run_e2e(cca, cfg, args, inputs_cpu, inputs, out, ws, stream, shape, world, barrier, reduce_max):
@@ -447,6 +496,8 @@ def main(argv=None):
     ap.add_argument("--workload", default=DEFAULT_WORKLOAD, choices=sorted(workloads.WORKLOADS))
     ap.add_argument("--no-cpu-baseline", action="store_true", help="skip the oracle timing (rank 0, N=1)")
     ap.add_argument("--no-e2e", action="store_true", help="skip the host-buffer end-to-end timing")
+    ap.add_argument("--no-mha", action="store_true",
+                    help="skip timing the plain multi-head block of the same shape (the uncompressed baseline)")
     ap.add_argument("--batch", type=int, default=None, help="override the workload's batch (profiling cases)")
     ap.add_argument("--seq-len", type=int, default=None, help="override the workload's sequence length")
     args = ap.parse_args(argv)

@@ -114,6 +114,19 @@ def _shapes(cfg: CcaConfig) -> Dict[str, tuple]:
     }
 
 
+def _input_ptrs(cfg: CcaConfig, tensors: Dict[str, torch.Tensor], names, dtype, device) -> list:
+    """Device pointers of the block inputs; a plain block (conv_kernel 0) may omit the conv weights,
+    which are then passed as NULL."""
+    sh = _shapes(cfg)
+    ptrs = []
+    for n in names:
+        if cfg.conv_kernel == 0 and n.startswith("conv") and tensors.get(n) is None:
+            ptrs.append(None)
+        else:
+            ptrs.append(_check(tensors[n], n, sh[n], dtype, device))
+    return ptrs
+
+
 def _check(t: torch.Tensor, name: str, shape: tuple, dtype: torch.dtype, device) -> int:
     if not isinstance(t, torch.Tensor):
         raise TypeError(f"{name} must be a torch.Tensor")
@@ -163,7 +176,7 @@ def prefill(cfg: CcaConfig, inputs: Dict[str, torch.Tensor], *, out: Optional[Di
         raise ValueError("inputs must be CUDA tensors")
     sh = _shapes(cfg)
     dt = _DT[cfg.dtype]
-    ptrs = [_check(inputs[n], n, sh[n], dt, device) for n in INPUT_NAMES]
+    ptrs = _input_ptrs(cfg, inputs, INPUT_NAMES, dt, device)
     if out is None:
         out = alloc_outputs(cfg, device, conv_state)
     y = _check(out["y"], "y", sh["y"], _DT[cfg.out_dtype], device)
@@ -207,7 +220,7 @@ def prefill_noalloc(cfg: CcaConfig, inputs: Dict[str, torch.Tensor], *,
         raise ValueError("inputs must be CUDA tensors")
     sh = _shapes(cfg)
     dt = _DT[cfg.dtype]
-    ptrs = [_check(inputs[n], n, sh[n], dt, device) for n in INPUT_NAMES]
+    ptrs = _input_ptrs(cfg, inputs, INPUT_NAMES, dt, device)
     if out is None:
         out = alloc_outputs(cfg, device, conv_state)
     y = _check(out["y"], "y", sh["y"], _DT[cfg.out_dtype], device)
@@ -235,7 +248,7 @@ def prefill_host(cfg: CcaConfig, x_host: torch.Tensor, weights: Dict[str, torch.
         raise ValueError("x_host shape/dtype mismatch")
     if tuple(y_host.shape) != sh["y"] or y_host.dtype != _DT[cfg.out_dtype] or not y_host.is_contiguous():
         raise ValueError("y_host shape/dtype mismatch")
-    wp = [_check(weights[n], n, sh[n], dt, device) for n in INPUT_NAMES[1:]]
+    wp = _input_ptrs(cfg, weights, INPUT_NAMES[1:], dt, device)
     xd = _check(x_dev, "x_dev", sh["x"], dt, device)
     yd = _check(y_dev, "y_dev", sh["y"], _DT[cfg.out_dtype], device)
     kc = _check(k_cache, "k_cache", sh["k_cache"], dt, device)

@@ -76,7 +76,9 @@ cca_status_t check_config(const cca_config_t* c, BlockDims* dm) {
   if (c->C < 1) return fail(CCA_ERR_INVALID_ARG, "C must be >= 1");
   if ((long long)c->C * c->n_q_heads * c->head_dim != c->hidden)
     return fail(CCA_ERR_INVALID_ARG, "hidden must equal C * n_q_heads * head_dim");
-  if (c->conv_kernel < 1 || c->conv_kernel > 64) return fail(CCA_ERR_INVALID_ARG, "conv_kernel must be in [1, 64]");
+  if (c->conv_kernel < 0 || c->conv_kernel > 64) return fail(CCA_ERR_INVALID_ARG, "conv_kernel must be in [0, 64]");
+  if (c->conv_kernel == 0 && (c->qk_mean_mode != 0 || c->value_shift != 0))
+    return fail(CCA_ERR_INVALID_ARG, "a plain block (conv_kernel 0) takes qk_mean_mode 0 and value_shift 0");
   if (c->qk_mean_mode < 0 || c->qk_mean_mode > 3) return fail(CCA_ERR_INVALID_ARG, "qk_mean_mode must be in [0, 3]");
   if (c->value_shift != 0 && c->value_shift != 1) return fail(CCA_ERR_INVALID_ARG, "value_shift must be 0 or 1");
   if (c->use_rope != 0 && c->use_rope != 1) return fail(CCA_ERR_INVALID_ARG, "use_rope must be 0 or 1");
@@ -135,7 +137,7 @@ cca_workspace_layout_t layout_of(const BlockDims& dm) {
   L.wo_offset = off;
   if (sep) off = align_up(off + (size_t)dm.E * dm.Lq * eb);
   L.wc_offset = off;
-  if (sep) off = align_up(off + (size_t)(dm.nq + dm.nkv) * dm.d * dm.d * eb);
+  if (sep && dm.K > 0) off = align_up(off + (size_t)(dm.nq + dm.nkv) * dm.d * dm.d * eb);
   L.sched_offset = off;
   off = align_up(off + (attention_tc_supported(dm) ? attention_tc_scratch_bytes(dm) : 256));
   L.total_bytes = off;
@@ -166,7 +168,7 @@ cca_status_t resolve(const cca_config_t* cfg, int path, Resolved* r) {
   const bool attn = sm100 && b16 && dm.d == 128 && attention_tc_supported(dm);
   const bool out = sm100 && b16 && gemm_tc_supported(dm.T, dm.E, dm.Lq);
   const bool pre = preproc_tc_supported(dm);
-  if (path == CCA_PATH_TENSOR && !(down && attn && out && pre))
+  if (path == CCA_PATH_TENSOR && !(down && attn && out && (pre || dm.K == 0)))
     return fail(CCA_ERR_UNSUPPORTED, "tensor-core path needs sm_100, bf16, head_dim 128 and 128-aligned widths");
   if (masked && (((path & 1) && !down) || ((path & 2) && !attn) || ((path & 4) && !out) || ((path & 8) && !pre)))
     return fail(CCA_ERR_UNSUPPORTED, "a stage asked for the tensor-core kernel cannot use it");
@@ -243,7 +245,9 @@ cca_status_t run_block(const Resolved& r, BlockPtrs p, cudaStream_t stream, void
   }
   if ((e = mark(1)) != cudaSuccess) return cuda_fail("event", e);
   // 2. seq conv, channel conv, QK-mean, RoPE, value shift; KV cache written here
-  if (r.tc_pre) {
+  if (dm.K == 0) {
+    if ((e = launch_plain_preproc(dm, p, stream)) != cudaSuccess) return cuda_fail("RoPE and KV cache (plain)", e);
+  } else if (r.tc_pre) {
     if ((e = launch_preproc_tc(dm, p, stream)) != cudaSuccess) return cuda_fail("preprocessing (mma)", e);
   } else {
     if ((e = launch_preproc_simt(dm, p, stream)) != cudaSuccess) return cuda_fail("preprocessing (SIMT)", e);
@@ -289,7 +293,9 @@ cca_status_t prepare(const cca_config_t* cfg, int path, const void* const* ins, 
   if (st != CCA_OK) return st;
   static const char* in_names[9] = {"x", "W_q", "W_k", "W_v", "convq_seq", "convq_chan", "convk_seq", "convk_chan",
                                     "W_o"};
+  const bool plain = r->dm.K == 0;  // no convolutions: their weights may be NULL
   for (int i = 0; i < 9; ++i) {
+    if (plain && i >= 4 && i <= 7 && ins[i] == nullptr) continue;
     if (ins[i] == nullptr) return fail(CCA_ERR_INVALID_ARG, std::string(in_names[i]) + " is NULL");
     if (!aligned16(ins[i])) return fail(CCA_ERR_INVALID_ARG, std::string(in_names[i]) + " is not 16-byte aligned");
   }
@@ -300,6 +306,7 @@ cca_status_t prepare(const cca_config_t* cfg, int path, const void* const* ins, 
   }
   if (conv_state != nullptr && !aligned16(conv_state))
     return fail(CCA_ERR_INVALID_ARG, "conv_state is not 16-byte aligned");
+  if (conv_state != nullptr && plain) return fail(CCA_ERR_INVALID_ARG, "a plain block (conv_kernel 0) has no conv state");
   const cca_workspace_layout_t L = layout_of(r->dm);
   if (workspace == nullptr) return fail(CCA_ERR_WORKSPACE, "workspace is NULL");
   if ((reinterpret_cast<uintptr_t>(workspace) & (kAlign - 1)) != 0)

@@ -58,6 +58,9 @@ cudaError_t launch_attention_simt(const BlockDims& dm, const void* q, const void
 // ---- preprocessing (seq conv, channel conv, QK-mean, RoPE, value shift) ----
 cudaError_t launch_preproc_simt(const BlockDims& dm, const BlockPtrs& p, cudaStream_t stream);
 cudaError_t launch_conv_state(const BlockDims& dm, const BlockPtrs& p, cudaStream_t stream);
+// plain blocks (K == 0, no convolutions, QK-mean or value shift): RoPE on q and k, the KV cache
+// and the attention copies, the W_o copy and the attention's split counters
+cudaError_t launch_plain_preproc(const BlockDims& dm, const BlockPtrs& p, cudaStream_t stream);
 // bf16 blocks with head_dim 128: channel mix on the tensor cores (mma.sync), coalesced I/O
 bool preproc_tc_supported(const BlockDims& dm);
 cudaError_t launch_preproc_tc(const BlockDims& dm, const BlockPtrs& p, cudaStream_t stream);

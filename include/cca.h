@@ -74,7 +74,10 @@ typedef struct cca_config {
   int n_q_heads;     /* query heads in the latent */
   int n_kv_heads;    /* K/V heads; n_q_heads % n_kv_heads == 0 (CCGQA when <) */
   int head_dim;      /* d, even */
-  int conv_kernel;   /* K >= 1 taps of the causal sequence conv */
+  int conv_kernel;   /* K >= 1 taps of the causal sequence conv; 0: a plain attention block
+                        (no convolutions, the uncompressed baseline when C = 1): qk_mean_mode and
+                        value_shift must be 0, the four conv weight pointers may be NULL and
+                        conv_state must be NULL */
   int qk_mean_mode;  /* OR of CCA_QK_MEAN_*; 3 is the method as described */
   int value_shift;   /* 1 = shift the upper half of v's channels by one token */
   int use_rope;      /* 1 = rotate-half RoPE on q and k */

@@ -108,3 +108,17 @@ def test_prefill_without_device_fails_cleanly():
     assert st in (cca.CCA_ERR_CUDA, cca.CCA_ERR_UNSUPPORTED)
     st = lib.cca_prefill(ctypes.byref(cfg), *null, *outs, None, None, 0, None)
     assert st != cca.CCA_OK
+
+
+def test_plain_block_configs():
+    """conv_kernel 0 is a plain attention block: no convolutions, so QK-mean and the value shift
+    must be off; its workspace has no channel-conv weight region."""
+    plain = good(conv_kernel=0, qk_mean_mode=0, value_shift=0)
+    assert cca.validate(plain) == cca.CCA_OK
+    for kw in (dict(qk_mean_mode=3), dict(qk_mean_mode=1), dict(value_shift=1)):
+        bad = good(conv_kernel=0, **{**dict(qk_mean_mode=0, value_shift=0), **kw})
+        assert cca.validate(bad) == cca.CCA_ERR_INVALID_ARG
+        assert "plain block" in cca.library().cca_last_error_message().decode()
+    lay = cca.workspace_layout(plain)
+    assert lay.sched_offset == lay.wc_offset
+    assert cca.validate(good(conv_kernel=-1)) == cca.CCA_ERR_INVALID_ARG

@@ -90,6 +90,34 @@ def test_bf16_split_key_ranges(case):
     check_all(sh, run_gpu(sh, inp, path=TENSOR), run_oracle(sh, inp))
 
 
+# Plain attention blocks (conv_kernel 0): the uncompressed baseline the method is compared
+# against. The oracle computes each as the CCA block it equals, with one seq-conv tap of 1 and
+# identity channel mixes (QK-mean and value shift off in both).
+PLAIN_CASES = [
+    dict(seq_len=300, n_q_heads=4, n_kv_heads=4, hidden=512),               # MHA, C = 1, ragged tail
+    dict(seq_len=520, n_q_heads=4, n_kv_heads=2, hidden=512, batch=2),      # GQA, C = 1
+    dict(seq_len=200, n_q_heads=2, n_kv_heads=2, hidden=1024, use_rope=0),  # C = 4, no RoPE
+]
+
+
+@pytest.mark.parametrize("path", [SIMT, AUTO], ids=["simt", "auto"])
+@pytest.mark.parametrize("case", range(len(PLAIN_CASES)))
+def test_plain_blocks(path, case):
+    sh = shape(conv_kernel=0, qk_mean_mode=0, value_shift=0, **PLAIN_CASES[case])
+    inp = workloads.make_inputs(sh)
+    assert not any(n.startswith("conv") for n in inp)  # passed to the library as NULL
+    one, oi = workloads.plain_as_identity(sh, inp)
+    check_all(sh, run_gpu(sh, inp, path=path), run_oracle(one, oi))
+
+
+def test_plain_block_fp32():
+    sh = shape(dtype="f32", conv_kernel=0, qk_mean_mode=0, value_shift=0, seq_len=97, n_q_heads=4,
+               n_kv_heads=2, head_dim=32, hidden=128, batch=2)
+    inp = workloads.make_inputs(sh)
+    one, oi = workloads.plain_as_identity(sh, inp)
+    check_all(sh, run_gpu(sh, inp), run_oracle(one, oi))
+
+
 @pytest.mark.parametrize("path", [SIMT, AUTO, TENSOR], ids=["simt", "auto", "tensor"])
 @pytest.mark.parametrize("mode,vshift,rope", [(0, 0, 0), (1, 0, 1), (2, 1, 0), (3, 1, 1), (0, 1, 1)])
 def test_bf16_modes(path, mode, vshift, rope):

@@ -62,13 +62,17 @@ class BlockShape:
 
 # The five workloads: a tiny fp32 CCA block, dense CCA, and three CCGQA shapes
 # (long prefill, 8x KV-cache compression with less-compressed queries, and a
-# 64k context).
+# 64k context); and the MHA baseline of the long prefill.
 WORKLOADS: Dict[str, BlockShape] = {
     "tiny_cca_fp32": BlockShape("tiny_cca_fp32", 1, 64, 128, 2, 2, 16, 4, "f32", 0),
     "cca_dense_bf16": BlockShape("cca_dense_bf16", 4, 4096, 2048, 4, 4, 128, 4, "bf16", 1),
     "ccgqa_16k_bf16": BlockShape("ccgqa_16k_bf16", 1, 16384, 2048, 4, 2, 128, 4, "bf16", 2),
     "ccgqa_8x_bf16": BlockShape("ccgqa_8x_bf16", 2, 8192, 2048, 8, 2, 128, 4, "bf16", 3),
     "ccgqa_64k_bf16": BlockShape("ccgqa_64k_bf16", 1, 65536, 4096, 8, 2, 128, 4, "bf16", 4),
+    # the uncompressed baseline of the long prefill: plain multi-head attention (C = 1, 16 heads
+    # of 128, no convolutions, QK-mean or value shift) at the same S and E
+    "mha_16k_bf16": BlockShape("mha_16k_bf16", 1, 16384, 2048, 16, 16, 128, 0, "bf16", 6, qk_mean_mode=0,
+                               value_shift=0),
 }
 
 # Order in which tensors are drawn from one generator; changing it changes
@@ -118,6 +122,8 @@ def make_inputs(shape: BlockShape, seed: int | None = None) -> Dict[str, torch.T
     dt = torch_dtype(shape.dtype)
     out = {}
     for name in DRAW_ORDER:
+        if shape.conv_kernel == 0 and name.startswith("conv"):
+            continue  # a plain block has no convolutions
         t = torch.randn(shapes[name], generator=g, dtype=torch.float32)
         t.mul_(_std(name))
         out[name] = t.to(dt).contiguous()
@@ -127,6 +133,14 @@ def make_inputs(shape: BlockShape, seed: int | None = None) -> Dict[str, torch.T
 def as_float64(inputs: Dict[str, torch.Tensor]):
     """The same values as numpy float64 arrays (exact up-cast)."""
     return {k: v.to(torch.float64).numpy() for k, v in inputs.items()}
+
+
+def plain_as_identity(shape: BlockShape, inputs: Dict[str, torch.Tensor]):
+    """A plain block (conv_kernel 0) as the CCA block it equals: one seq-conv tap of 1, identity
+    channel mixes (QK-mean and value shift are off in both)."""
+    assert shape.conv_kernel == 0 and shape.qk_mean_mode == 0 and shape.value_shift == 0
+    one = shape.replace(conv_kernel=1)
+    return one, identity_convs(one, inputs)
 
 
 def identity_convs(shape: BlockShape, inputs: Dict[str, torch.Tensor]) -> Dict[str, torch.Tensor]:
