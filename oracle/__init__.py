@@ -11,6 +11,7 @@ from .cca_oracle import (  # noqa: F401
     causal_attention,
     cca_block,
     channel_conv,
+    decode_step,
     default_scale,
     down_project,
     qk_mean,

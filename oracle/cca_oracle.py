@@ -293,6 +293,59 @@ def cca_block(inp: Dict[str, np.ndarray], n_q: int, n_kv: int, d: int, *,
     return out
 
 
+# ---------------------------------------------------------------------------
+# 10. One decode step: the same steps as cca_block for one more token of one
+# sequence, from the state a prefill of the earlier tokens leaves (the KV cache
+# and the last K-1 pre-conv latents of q and k plus the last v latent; es 1
+# item 2: the compressed cache is what decoding reads).
+# ---------------------------------------------------------------------------
+def decode_step(inp: Dict[str, np.ndarray], x_t: np.ndarray, k_cache: np.ndarray, v_cache: np.ndarray,
+                conv_state: np.ndarray, t: int, n_q: int, n_kv: int, d: int, *, qk_mean_mode: int = 3,
+                use_value_shift: bool = True, use_rope: bool = True, rope_base: float = 10000.0,
+                softmax_scale: float = 0.0) -> Dict[str, np.ndarray]:
+    """Token t of one sequence. x_t [E]; k_cache, v_cache [>= t, n_kv, d] (rows 0..t-1 are read);
+    conv_state [(K-1)*(Lq+Lkv) + Lkv]: the last K-1 rows of q~, then of k~, then the last row of v~
+    (zero rows before the sequence start). Returns y [E], q [Lq], k [n_kv, d], v [n_kv, d] (the new
+    cache rows) and the conv state advanced by this token."""
+    Lq, Lkv = n_q * d, n_kv * d
+    K = inp["convq_seq"].shape[1]
+    q_lat = down_project(x_t[None, :], inp["W_q"])
+    k_lat = down_project(x_t[None, :], inp["W_k"])
+    v_lat = down_project(x_t[None, :], inp["W_v"])
+    q_rows = conv_state[:(K - 1) * Lq].reshape(K - 1, Lq)
+    k_rows = conv_state[(K - 1) * Lq:(K - 1) * (Lq + Lkv)].reshape(K - 1, Lkv)
+    v_prev = conv_state[(K - 1) * (Lq + Lkv):]
+    # the seq conv over the window of the K-1 earlier latents and this one, at its last row
+    cq = channel_conv(seq_conv_causal(np.vstack([q_rows, q_lat]), inp["convq_seq"])[-1:], inp["convq_chan"], n_q, d)
+    ck = channel_conv(seq_conv_causal(np.vstack([k_rows, k_lat]), inp["convk_seq"])[-1:], inp["convk_chan"], n_kv, d)
+    mq_pre, mk_pre = qk_mean(q_lat, k_lat, n_q, n_kv, d)
+    mq_post, mk_post = qk_mean(cq, ck, n_q, n_kv, d)
+    q = cq.copy()
+    k = ck.copy()
+    if qk_mean_mode & QK_MEAN_PRE:
+        q += mq_pre
+        k += mk_pre
+    if qk_mean_mode & QK_MEAN_POST:
+        q += mq_post
+        k += mk_post
+    if use_rope:
+        pos = np.array([t])
+        q = rope(q, n_q, d, rope_base, positions=pos)
+        k = rope(k, n_kv, d, rope_base, positions=pos)
+    v = v_lat.copy()
+    if use_value_shift:  # channels [Lkv/2, Lkv) from the previous token
+        v[0, Lkv // 2:] = v_prev[Lkv // 2:]
+    keys = np.vstack([k_cache[:t].reshape(t, Lkv), k])
+    values = np.vstack([v_cache[:t].reshape(t, Lkv), v])
+    q_all = np.zeros((t + 1, Lq))
+    q_all[t] = q[0]
+    o = causal_attention(q_all, keys, values, n_q, n_kv, d, default_scale(d, softmax_scale), rows=[t])
+    y = o[0] @ inp["W_o"].T
+    state = np.concatenate([np.vstack([q_rows, q_lat])[1:].reshape(-1), np.vstack([k_rows, k_lat])[1:].reshape(-1),
+                            v_lat[0]])
+    return {"y": y, "q": q[0], "k": k.reshape(n_kv, d), "v": v.reshape(n_kv, d), "conv_state": state}
+
+
 def attention_flops(batch: int, seq_len: int, n_q: int, d: int) -> float:
     """Causal attention FLOPs, masked half excluded: 2 GEMMs x 2 flop/MAC x S^2/2."""
     return 2.0 * batch * n_q * seq_len * seq_len * d

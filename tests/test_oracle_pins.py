@@ -354,3 +354,56 @@ def test_conv_state_is_tail_of_latents():
     np.testing.assert_array_equal(cs[:, 0], 0.0)
     np.testing.assert_array_equal(cs[:, 1:], res["q_lat"])
     np.testing.assert_array_equal(res["conv_state_v"][:, 0], res["v_lat"][:, -1])
+
+
+# --------------------------------------------------------------- decode step --
+@pytest.mark.parametrize("mode,vshift,rope_on,G", [(3, 1, 1, 2), (0, 0, 1, 2), (1, 1, 0, 1), (2, 0, 1, 4)])
+def test_decode_step_continues_the_prefill(mode, vshift, rope_on, G):
+    """A prefill of S tokens equals a prefill of S-1 tokens followed by one decode step from its
+    state (KV cache and conv state): y, q, the new cache rows and the advanced conv state, at fp64."""
+    nkv, d, S = 2, 8, 23
+    sh = workloads.BlockShape("dec", 2, S, G * nkv * d * 2, G * nkv, nkv, d, 3, "f32", 7,
+                              qk_mean_mode=mode, value_shift=vshift, use_rope=rope_on)
+    inp = workloads.as_float64(workloads.make_inputs(sh))
+    kw = dict(qk_mean_mode=mode, use_value_shift=bool(vshift), use_rope=bool(rope_on))
+    full = oracle.cca_block(inp, G * nkv, nkv, d, **kw)
+    head = dict(inp, x=inp["x"][:, :S - 1])
+    pre = oracle.cca_block(head, G * nkv, nkv, d, **kw)
+    K, Lq, Lkv = 3, G * nkv * d, nkv * d
+    for b in range(2):
+        state = np.concatenate([pre["conv_state_q"][b].reshape(-1), pre["conv_state_k"][b].reshape(-1),
+                                pre["conv_state_v"][b].reshape(-1)])
+        assert state.size == (K - 1) * (Lq + Lkv) + Lkv
+        out = oracle.decode_step(inp, inp["x"][b, S - 1], pre["k_cache"][b], pre["v_cache"][b], state, S - 1,
+                                 G * nkv, nkv, d, **kw)
+        np.testing.assert_allclose(out["y"], full["y"][b, S - 1], rtol=1e-11, atol=1e-12)
+        np.testing.assert_allclose(out["q"], full["q"][b, S - 1], rtol=1e-11, atol=1e-12)
+        np.testing.assert_allclose(out["k"], full["k_cache"][b, S - 1], rtol=1e-11, atol=1e-12)
+        np.testing.assert_allclose(out["v"], full["v_cache"][b, S - 1], rtol=1e-11, atol=1e-12)
+        full_state = np.concatenate([full["conv_state_q"][b].reshape(-1), full["conv_state_k"][b].reshape(-1),
+                                     full["conv_state_v"][b].reshape(-1)])
+        np.testing.assert_allclose(out["conv_state"], full_state, rtol=1e-14, atol=1e-15)  # same latents, to rounding
+
+
+def test_decode_steps_chain_and_first_token():
+    """Three decode steps after a prefill of S-3 tokens reproduce the last three rows of a prefill
+    of S; one step from an empty cache and a zero conv state is a prefill of one token."""
+    G, nkv, d, S = 2, 2, 8, 19
+    sh = workloads.BlockShape("dec", 1, S, G * nkv * d * 2, G * nkv, nkv, d, 4, "f32", 8)
+    inp = workloads.as_float64(workloads.make_inputs(sh))
+    full = oracle.cca_block(inp, G * nkv, nkv, d)
+    pre = oracle.cca_block(dict(inp, x=inp["x"][:, :S - 3]), G * nkv, nkv, d)
+    kc = np.zeros((S, nkv, d))
+    vc = np.zeros((S, nkv, d))
+    kc[:S - 3] = pre["k_cache"][0]
+    vc[:S - 3] = pre["v_cache"][0]
+    state = np.concatenate([pre["conv_state_q"][0].reshape(-1), pre["conv_state_k"][0].reshape(-1),
+                            pre["conv_state_v"][0].reshape(-1)])
+    for t in range(S - 3, S):
+        out = oracle.decode_step(inp, inp["x"][0, t], kc, vc, state, t, G * nkv, nkv, d)
+        kc[t], vc[t], state = out["k"], out["v"], out["conv_state"]
+        np.testing.assert_allclose(out["y"], full["y"][0, t], rtol=1e-11, atol=1e-12)
+    one = oracle.cca_block(dict(inp, x=inp["x"][:, :1]), G * nkv, nkv, d)
+    K, Lq, Lkv = 4, G * nkv * d, nkv * d
+    out = oracle.decode_step(inp, inp["x"][0, 0], kc, vc, np.zeros((K - 1) * (Lq + Lkv) + Lkv), 0, G * nkv, nkv, d)
+    np.testing.assert_allclose(out["y"], one["y"][0, 0], rtol=1e-11, atol=1e-12)
