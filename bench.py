@@ -378,6 +378,8 @@ def run_ours(args, shape):
         if (world == 1 and not args.no_mha and my_shape.dtype == "bf16" and my_shape.conv_kernel > 0 and
                 my_shape.hidden % 128 == 0):
             line["mha_baseline"] = run_mha_baseline(cca, dev, my_shape, ms_per_step)
+        if world == 1 and not args.no_decode and cca.decode_workspace_size(cfg) > 0:
+            line["decode"] = run_decode(cca, dev, my_shape, inputs, out, peaks)
         if world == 1 and not args.no_cpu_baseline:
             line["cpu_baseline"] = cpu_baseline(my_shape, inputs_cpu)
         print(json.dumps(line, default=float), flush=True)
@@ -430,6 +432,87 @@ def run_mha_baseline(cca, dev, shape, cca_ms_per_step, steps=10, warmup=3):
         "kernels_ms": {"down_proj": stage_ms[0], "rope_cache": stage_ms[1], "attention": stage_ms[2],
                        "out_proj": stage_ms[3]},
         "cca_speedup": ms / cca_ms_per_step,
+    }
+
+
+def decode_bytes(shape: workloads.BlockShape, t: int) -> float:
+    """Bytes one decode step must move at position t: every weight once, the cache rows 0..t-1
+    read and row t written, the conv state read and written, x_t read and y_t written."""
+    B, E, d, K = shape.batch, shape.hidden, shape.head_dim, shape.conv_kernel
+    Lq, Lkv = shape.latent_q, shape.latent_kv
+    eb = 2 if shape.dtype == "bf16" else 4
+    w = (Lq + 2 * Lkv) * E + E * Lq + (Lq + Lkv) * K + (shape.n_q_heads + shape.n_kv_heads) * d * d * (K > 0)
+    state = (K - 1) * (Lq + Lkv) + Lkv if K > 0 else 0
+    per_seq = 2 * (t + 1) * Lkv + 2 * state + 2 * E
+    return float((w + B * per_seq) * eb)
+
+
+def run_decode(cca, dev, shape, inputs, out, peaks, steps=50, warmup=5):
+    """One decode step (cca_decode) at the last position of the workload, t = S - 1, reading the
+    cache the timed prefill wrote. The step is captured once in a CUDA graph, as a serving loop
+    runs it, and each replay is timed with CUDA events, L2 flushed before each. The host cost of
+    one direct call (argument checks, four launches) is reported on its own."""
+    t = shape.seq_len - 1
+    cfg = cca.config_from_shape(shape)  # seq_len = t + 1
+    B = shape.batch
+    weights = {k: v for k, v in inputs.items() if k != "x"}
+    x_t = inputs["x"][:, t].contiguous()
+    K = shape.conv_kernel
+    cs = None
+    if K > 0:
+        n = (K - 1) * (shape.latent_q + shape.latent_kv) + shape.latent_kv
+        cs = torch.zeros((B, n), dtype=out["k_cache"].dtype, device=dev)
+    y = torch.empty((B, shape.hidden), dtype=out["y"].dtype, device=dev)
+    ws = torch.empty(cca.decode_workspace_size(cfg), dtype=torch.uint8, device=dev)
+    flush = torch.empty(L2_FLUSH_BYTES, dtype=torch.uint8, device=dev)
+
+    def step(stream=None):
+        cca.decode(cfg, x_t, weights, out["k_cache"], out["v_cache"], cs, y=y, workspace=ws, stream=stream)
+
+    side = torch.cuda.Stream(device=dev)
+    side.wait_stream(torch.cuda.current_stream(dev))
+    with torch.cuda.stream(side):
+        for _ in range(warmup):
+            step()
+    torch.cuda.current_stream(dev).wait_stream(side)
+    torch.cuda.synchronize()
+    # host cost of a direct call: wall clock over calls queued behind one long flush
+    flush.zero_()
+    h0 = time.perf_counter()
+    for _ in range(20):
+        step()
+    host_us = (time.perf_counter() - h0) / 20 * 1e6
+    torch.cuda.synchronize()
+    graph = torch.cuda.CUDAGraph()
+    with torch.cuda.graph(graph):
+        step()
+    stream = torch.cuda.current_stream(dev)
+    for _ in range(warmup):
+        flush.zero_()
+        graph.replay()
+    evs = [(torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)) for _ in range(steps)]
+    torch.cuda.synchronize()
+    for i in range(steps):
+        flush.zero_()
+        evs[i][0].record(stream)
+        graph.replay()
+        evs[i][1].record(stream)
+    torch.cuda.synchronize()
+    if cca.poll_device_status() != 0:
+        raise SystemExit("device status error in the decode timing")
+    del graph
+    us = np.array([a.elapsed_time(b) * 1e3 for a, b in evs])
+    nbytes = decode_bytes(shape, t)
+    hbm = float(peaks.get("hbm_gbs", FALLBACK_PEAKS["hbm_gbs"]))
+    mean_us = float(us.mean())
+    gemv_launches = 2 * ((B + 7) // 8)
+    return {
+        "position": t, "batch": B, "steps": steps, "warmup": warmup, "us_per_step": mean_us,
+        "us_median": float(np.median(us)), "tokens_per_s": B / (mean_us / 1e6),
+        "bytes_per_step": nbytes, "gbs": nbytes / (mean_us / 1e6) / 1e9,
+        "frac_hbm": nbytes / (mean_us / 1e6) / 1e9 / hbm, "timing": "CUDA graph replay",
+        "host_us_per_call": host_us, "launches_per_step": gemv_launches + 1 + (K > 0),
+        "l2": "flushed before each step (256 MiB write)",
     }
 
 
@@ -498,6 +581,7 @@ def main(argv=None):
     ap.add_argument("--no-e2e", action="store_true", help="skip the host-buffer end-to-end timing")
     ap.add_argument("--no-mha", action="store_true",
                     help="skip timing the plain multi-head block of the same shape (the uncompressed baseline)")
+    ap.add_argument("--no-decode", action="store_true", help="skip timing one decode step at position S - 1")
     ap.add_argument("--batch", type=int, default=None, help="override the workload's batch (profiling cases)")
     ap.add_argument("--seq-len", type=int, default=None, help="override the workload's sequence length")
     args = ap.parse_args(argv)

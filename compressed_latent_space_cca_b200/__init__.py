@@ -262,6 +262,53 @@ def prefill_host(cfg: CcaConfig, x_host: torch.Tensor, weights: Dict[str, torch.
         raise CcaError(st, "cca_prefill_host")
 
 
+def decode_workspace_size(cfg: CcaConfig) -> int:
+    """Bytes of workspace cca_decode needs (0 if the shape is not supported); independent of seq_len."""
+    return library().cca_decode_workspace_size(ctypes.byref(cfg))
+
+
+def decode(cfg: CcaConfig, x_t: torch.Tensor, weights: Dict[str, torch.Tensor], k_cache: torch.Tensor,
+           v_cache: torch.Tensor, conv_state: Optional[torch.Tensor] = None, *, y: Optional[torch.Tensor] = None,
+           workspace: Optional[torch.Tensor] = None,
+           stream: Optional[torch.cuda.Stream] = None) -> torch.Tensor:
+    """cca_decode: one decode step, the token at position cfg.seq_len - 1 of every sequence.
+
+    x_t [B, E]; weights: the eight weight tensors of INPUT_NAMES[1:]; k_cache, v_cache
+    [B, rows, n_kv, d] with rows >= seq_len (rows 0..t-1 read, row t written); conv_state
+    [B, (K-1)*(Lq+Lkv) + Lkv] advanced in place (None for conv_kernel 0). Returns y_t [B, E].
+    """
+    device = x_t.device
+    if device.type != "cuda":
+        raise ValueError("inputs must be CUDA tensors")
+    sh = _shapes(cfg)
+    dt = _DT[cfg.dtype]
+    B, E = cfg.batch, cfg.hidden
+    xp = _check(x_t, "x_t", (B, E), dt, device)
+    wp = _input_ptrs(cfg, weights, INPUT_NAMES[1:], dt, device)
+    if k_cache.dim() != 4:
+        raise ValueError("k_cache must be [B, rows, n_kv, d]")
+    rows = k_cache.shape[1]
+    cshape = (B, rows, cfg.n_kv_heads, cfg.head_dim)
+    kc = _check(k_cache, "k_cache", cshape, dt, device)
+    vc = _check(v_cache, "v_cache", cshape, dt, device)
+    cs = None if conv_state is None else _check(conv_state, "conv_state", sh["conv_state"], dt, device)
+    if y is None:
+        y = torch.empty((B, E), dtype=_DT[cfg.out_dtype], device=device)
+    yp = _check(y, "y_t", (B, E), _DT[cfg.out_dtype], device)
+    if workspace is None:
+        n = decode_workspace_size(cfg)
+        if n == 0:
+            raise CcaError(CCA_ERR_UNSUPPORTED, "cca_decode_workspace_size")
+        workspace = torch.empty(n, dtype=torch.uint8, device=device)
+    if stream is None:
+        stream = torch.cuda.current_stream(device)
+    st = library().cca_decode(ctypes.byref(cfg), rows, xp, *wp, yp, kc, vc, cs, workspace.data_ptr(),
+                              workspace.numel(), ctypes.c_void_p(stream.cuda_stream))
+    if st != CCA_OK:
+        raise CcaError(st, "cca_decode")
+    return y
+
+
 def poll_device_status(stream: Optional[torch.cuda.Stream] = None) -> int:
     """Synchronize and return the device status (CCA_OK or CCA_ERR_DEVICE_TIMEOUT ...)."""
     s = stream.cuda_stream if stream is not None else torch.cuda.current_stream().cuda_stream

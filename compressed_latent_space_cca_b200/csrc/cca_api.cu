@@ -493,6 +493,52 @@ cca_status_t cca_prefill_host(const cca_config_t* cfg, const void* x_host, void*
   return CCA_OK;
 }
 
+size_t cca_decode_workspace_size(const cca_config_t* cfg) {
+  BlockDims dm;
+  if (check_config(cfg, &dm) != CCA_OK || !decode_supported(dm)) return 0;
+  return decode_workspace_bytes(dm);
+}
+
+cca_status_t cca_decode(const cca_config_t* cfg, int cache_rows, const void* x_t, const void* W_q, const void* W_k,
+                        const void* W_v, const void* convq_seq, const void* convq_chan, const void* convk_seq,
+                        const void* convk_chan, const void* W_o, void* y_t, void* k_cache, void* v_cache,
+                        void* conv_state, void* workspace, size_t workspace_bytes, void* stream) {
+  BlockDims dm;
+  cca_status_t st = check_config(cfg, &dm);
+  if (st != CCA_OK) return st;
+  if (!decode_supported(dm))
+    return fail(CCA_ERR_UNSUPPORTED,
+                "decode needs head_dim 32, 64 or 128, n_q_heads / n_kv_heads <= 8, hidden and n_q_heads * "
+                "head_dim multiples of 8");
+  if (cache_rows < dm.S) return fail(CCA_ERR_INVALID_ARG, "cache_rows must be >= seq_len");
+  if ((long long)dm.B * cache_rows > (1ll << 30)) return fail(CCA_ERR_UNSUPPORTED, "cache extent too large");
+  static const char* names[10] = {"x_t", "W_q", "W_k", "W_v", "convq_seq", "convq_chan", "convk_seq", "convk_chan",
+                                  "W_o", "y_t"};
+  const void* ptrs[10] = {x_t, W_q, W_k, W_v, convq_seq, convq_chan, convk_seq, convk_chan, W_o, y_t};
+  const bool plain = dm.K == 0;
+  for (int i = 0; i < 10; ++i) {
+    if (plain && i >= 4 && i <= 7 && ptrs[i] == nullptr) continue;
+    if (ptrs[i] == nullptr) return fail(CCA_ERR_INVALID_ARG, std::string(names[i]) + " is NULL");
+    if (!aligned16(ptrs[i])) return fail(CCA_ERR_INVALID_ARG, std::string(names[i]) + " is not 16-byte aligned");
+  }
+  if (k_cache == nullptr || v_cache == nullptr) return fail(CCA_ERR_INVALID_ARG, "k_cache / v_cache is NULL");
+  if (!aligned16(k_cache) || !aligned16(v_cache))
+    return fail(CCA_ERR_INVALID_ARG, "k_cache / v_cache is not 16-byte aligned");
+  if (plain && conv_state != nullptr)
+    return fail(CCA_ERR_INVALID_ARG, "a plain block (conv_kernel 0) has no conv state");
+  if (!plain && conv_state == nullptr) return fail(CCA_ERR_INVALID_ARG, "conv_state is NULL");
+  if (workspace == nullptr) return fail(CCA_ERR_WORKSPACE, "workspace is NULL");
+  if ((reinterpret_cast<uintptr_t>(workspace) & (kAlign - 1)) != 0)
+    return fail(CCA_ERR_WORKSPACE, "workspace is not 256-byte aligned");
+  if (workspace_bytes < decode_workspace_bytes(dm))
+    return fail(CCA_ERR_WORKSPACE, "workspace smaller than cca_decode_workspace_size()");
+  DecodePtrs p{x_t, W_q, W_k, W_v, convq_seq, convq_chan, convk_seq, convk_chan, W_o,
+               y_t, k_cache, v_cache, conv_state, workspace};
+  const cudaError_t e = launch_decode(dm, p, cache_rows, static_cast<cudaStream_t>(stream));
+  if (e != cudaSuccess) return cuda_fail("decode", e);
+  return CCA_OK;
+}
+
 cca_status_t cca_poll_device_status(void* stream) {
   DeviceInfo* di = nullptr;
   cca_status_t st = device_info(&di);

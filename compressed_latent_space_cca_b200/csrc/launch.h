@@ -100,6 +100,19 @@ constexpr int kAttnMaxSplit = 64;
 constexpr int kAttnSplitCounters = kAttnMaxSplit * 2 * 4;
 size_t attention_tc_scratch_bytes(const BlockDims& dm);
 
+// ---- one decode step (token t = S - 1 of every sequence), fp32 arithmetic ----
+struct DecodePtrs {
+  const void *x, *Wq, *Wk, *Wv, *cq_seq, *cq_chan, *ck_seq, *ck_chan, *Wo;  // x: [B, E]
+  void *y;                  // [B, E] out
+  void *k_cache, *v_cache;  // [B, cache_rows, nkv, d]: rows 0..t-1 read, row t written
+  void* conv_state;         // [B, (K-1)*(Lq+Lkv) + Lkv], advanced in place (NULL when K == 0)
+  void* workspace;          // decode_workspace_bytes(dm), 256-byte aligned
+};
+// head_dim 32, 64 or 128; G <= 8; E and Lq multiples of 8
+bool decode_supported(const BlockDims& dm);
+size_t decode_workspace_bytes(const BlockDims& dm);  // independent of S
+cudaError_t launch_decode(const BlockDims& dm, const DecodePtrs& p, int cache_rows, cudaStream_t stream);
+
 // ---- misc ----
 cudaError_t launch_wait_timeout_selftest(unsigned* dev_err, unsigned long long limit_ns, cudaStream_t stream);
 

@@ -250,6 +250,45 @@ cca_status_t cca_prefill_noalloc(const cca_config_t* cfg,
                                  void* y, void* k_cache, void* v_cache, void* conv_state,
                                  void* stream);
 
+/*
+ * One decode step of the block ("Compressed Convolutional Attention",
+ * gist.science/es/paper/2510.04476, section 1 item 2: decoding reads the
+ * compressed KV cache, C times smaller than a multi-head one; the steps are
+ * those of the prefill, section 2, for one more token): the token at position
+ * t = cfg->seq_len - 1 of each of the cfg->batch sequences, given the state a
+ * cca_prefill of tokens 0..t-1 (or earlier decode steps) left. All sequences
+ * are at the same position. Arithmetic is fp32; inputs, weights, the cache
+ * and the conv state are cfg->dtype.
+ *
+ *   cache_rows  rows allocated per sequence in k_cache / v_cache, >= seq_len
+ *   x_t         [B, E]                 hidden state of the new token
+ *   W_q ... W_o as in cca_prefill (the conv weights may be NULL when K == 0)
+ *   y_t         [B, E] out             cfg->out_dtype
+ *   k_cache, v_cache [B, cache_rows, n_kv, d] in/out: rows 0..t-1 are read,
+ *               row t is written. A prefill writes [B, S, n_kv, d]; with
+ *               B > 1 its rows must be copied into the wider cache first.
+ *   conv_state  [B, (K-1)*(Lq+Lkv) + Lkv] in/out, as cca_prefill writes it;
+ *               advanced by one token in place. Required when K >= 1, NULL
+ *               when K == 0.
+ *   workspace   >= cca_decode_workspace_size(cfg) bytes, 256-byte aligned,
+ *               need not start at zero. The size does not depend on seq_len,
+ *               so one buffer serves every step.
+ * Supported: head_dim 32, 64 or 128; n_q_heads / n_kv_heads <= 8; hidden and
+ * n_q_heads * head_dim multiples of 8; all pointers 16-byte aligned.
+ * Launches 4 kernels (3 when K == 0) for B <= 8, and two more per further 8
+ * sequences. Errors: INVALID_ARG / UNSUPPORTED / WORKSPACE before any launch,
+ * CUDA if a launch fails. No kernel of this step waits on another.
+ */
+size_t cca_decode_workspace_size(const cca_config_t* cfg);
+cca_status_t cca_decode(const cca_config_t* cfg, int cache_rows,
+                        const void* x_t,
+                        const void* W_q, const void* W_k, const void* W_v,
+                        const void* convq_seq, const void* convq_chan,
+                        const void* convk_seq, const void* convk_chan,
+                        const void* W_o,
+                        void* y_t, void* k_cache, void* v_cache, void* conv_state,
+                        void* workspace, size_t workspace_bytes, void* stream);
+
 /* Synchronizes `stream`, then reports and clears the device error word:
  * CCA_ERR_DEVICE_TIMEOUT if a bounded wait in a kernel gave up since the last
  * poll, CCA_ERR_NUMERIC_RANGE if a finite fp16 intermediate overflowed (its

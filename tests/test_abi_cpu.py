@@ -122,3 +122,39 @@ def test_plain_block_configs():
     lay = cca.workspace_layout(plain)
     assert lay.sched_offset == lay.wc_offset
     assert cca.validate(good(conv_kernel=-1)) == cca.CCA_ERR_INVALID_ARG
+
+
+def test_decode_workspace_and_shapes():
+    """The decode workspace depends on the batch and head layout, not on the position; shapes the
+    decode kernels do not take report 0."""
+    sizes = {cca.decode_workspace_size(good(seq_len=s)) for s in (1, 100, 16384, 100000)}
+    assert len(sizes) == 1 and sizes.pop() > 0
+    assert cca.decode_workspace_size(good(batch=8)) > cca.decode_workspace_size(good(batch=1))
+    assert cca.decode_workspace_size(good(n_q_heads=32, n_kv_heads=2, hidden=32 * 128)) == 0  # G = 16
+    assert cca.decode_workspace_size(good(head_dim=16, hidden=4 * 16)) == 0
+    assert cca.decode_workspace_size(good(head_dim=64, hidden=4 * 64)) > 0
+    assert cca.decode_workspace_size(good(batch=0)) == 0
+
+
+def test_decode_argument_checks():
+    """Every argument error is reported before any launch (no GPU here)."""
+    lib = cca.library()
+    cfg = good(seq_len=10)
+    p = ctypes.c_void_p(256)
+    ws, nws = ctypes.c_void_p(1 << 20), cca.decode_workspace_size(cfg)
+
+    def call(rows=16, ptrs=None, state=p, w=ws, n=nws, c=cfg):
+        args = ptrs if ptrs is not None else [p] * 10
+        return lib.cca_decode(ctypes.byref(c), rows, *args[:9], args[9], p, p, state, w, n, None)
+    assert call(rows=9) == cca.CCA_ERR_INVALID_ARG
+    assert "cache_rows" in lib.cca_last_error_message().decode()
+    assert call(ptrs=[None] + [p] * 9) == cca.CCA_ERR_INVALID_ARG
+    assert call(ptrs=[ctypes.c_void_p(258)] + [p] * 9) == cca.CCA_ERR_INVALID_ARG
+    assert call(state=None) == cca.CCA_ERR_INVALID_ARG
+    assert call(w=None) == cca.CCA_ERR_WORKSPACE
+    assert call(w=ctypes.c_void_p(256 + 16)) == cca.CCA_ERR_WORKSPACE
+    assert call(n=nws - 1) == cca.CCA_ERR_WORKSPACE
+    plain = good(seq_len=10, conv_kernel=0, qk_mean_mode=0, value_shift=0)
+    assert call(c=plain) == cca.CCA_ERR_INVALID_ARG  # a plain block has no conv state
+    assert "plain block" in lib.cca_last_error_message().decode()
+    assert call(c=good(seq_len=10, head_dim=16, hidden=64)) == cca.CCA_ERR_UNSUPPORTED
