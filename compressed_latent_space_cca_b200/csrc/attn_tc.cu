@@ -12,13 +12,17 @@
 // of one head), so every K/V tile it loads serves both. Roles:
 //   warp 0      TMA: Q tiles once per pair, then K tiles (3-stage ring) and V
 //               tiles (2-stage ring)
-//   warp 1      one thread issues tcgen05.mma: S_j = Q_j K^T (SS form) into
-//               TMEM, then O_j += P_j V (TS form, P read from TMEM)
-//   warps 2-5   softmax of tile 0, warps 6-9 softmax of tile 1: each thread
-//               owns one query row, reads its S row from TMEM, keeps the
-//               running max / sum, writes P (fp16) back over S in TMEM,
-//               rescales its O row in TMEM when the max grows by more than
-//               2^8, and finally normalises O and stores it.
+//   warp 1      the MMA loop, run by the whole warp so that its control flow
+//               and descriptor arithmetic stay warp-uniform; an elected lane
+//               issues tcgen05.mma: S_j = Q_j K^T (SS form) into TMEM, then
+//               O_j += P_j V (TS form, P read from TMEM)
+//   warps 2-17  softmax, eight warps per tile, two on each SMSP: each warp owns
+//               16 query rows (half a TMEM lane quadrant) and reads its S rows
+//               with the 16-lane TMEM shapes, so each thread holds 32 keys of two
+//               rows and a quad of threads shares a row; they keep the
+//               running max / sum, write P (fp16) back over S in TMEM, rescale
+//               their O rows in TMEM when the max grows by more than 2^8, and
+//               finally normalise O and store it.
 // TMEM (512 columns): S0 | S1 | O0 | O1, 128 fp32 columns each; P_j overlays
 // the first 64 columns of S_j. The two tiles ping-pong: while one softmax
 // group works, the tensor core runs the other tile's MMAs. Key tiles above
@@ -38,7 +42,8 @@ constexpr int TK = 128;          // keys per tile
 constexpr int K_STAGES = 3, V_STAGES = 2;
 constexpr int HALF_BYTES = 128 * 64 * 2;  // 128 rows x 64 fp16 (one 128-byte swizzle span)
 constexpr int TILE_BYTES = 2 * HALF_BYTES;  // 128 x 128 fp16
-constexpr int NUM_THREADS = 320;
+constexpr int NUM_SOFTMAX_WARPS = 16;  // eight per query tile
+constexpr int NUM_THREADS = 64 + 32 * NUM_SOFTMAX_WARPS;
 constexpr int TMEM_COLS = 512;
 constexpr uint32_t COL_S0 = 0, COL_O0 = 256;
 constexpr float RESCALE_THRESHOLD = 8.0f;  // log2 units: rescale O only if the max grows by > 2^8
@@ -50,8 +55,8 @@ constexpr int OFF_V = OFF_K + K_STAGES * TILE_BYTES;
 constexpr int OFF_BAR = OFF_V + V_STAGES * TILE_BYTES;
 constexpr int MAX_CTAS = 160;
 constexpr int MAX_LIST = 4096;  // entries a host schedule can hold in the kernel parameters
-// A partial result of one 128-row tile: O as [d / 4][128 rows][4] fp32 (a warp's 16-byte accesses to
-// one column quad cover 512 contiguous bytes), then the running max [128] and sum [128].
+// A partial result of one 128-row tile: O as [16 chunks of 8 columns][128 rows][8] fp32 (a warp's
+// accesses to one chunk cover 256 contiguous bytes per 8 rows), then the running max [128] and sum [128].
 constexpr int PART_TILE = D * TQ + 2 * TQ;  // floats
 constexpr size_t SMEM_BYTES = OFF_BAR + 256 + 1024;
 
@@ -88,7 +93,7 @@ __device__ __forceinline__ void exp2_fma_x2(float x0, float x1, float& p0, float
 
 struct AttnMaps {
   CUtensorMap q, k, v;
-  CUtensorMap o;  // attention output, boxes of 64 columns x 32 rows (one warp's rows)
+  CUtensorMap o;  // attention output, boxes of 64 columns x 16 rows (one softmax warp's rows)
 };
 
 struct AttnParams {
@@ -103,7 +108,7 @@ struct AttnParams {
   // split key ranges: pairs 0 .. nsplit-1 (the longest) run as two halves on any CTAs; each half
   // leaves its unnormalised O, max and sum in part, and the second to finish merges them
   int nsplit;
-  int* split_cnt;  // [nsplit][2 tiles][4 lane quadrants], zero at launch
+  int* split_cnt;  // [nsplit][2 tiles][8 softmax warps], zero at launch
   float* part;     // [nsplit][2 halves][2 tiles][PART_TILE]
 };
 
@@ -198,9 +203,9 @@ __global__ void __launch_bounds__(NUM_THREADS, 1) attn_tc_kernel(const __grid_co
     }
     for (int j = 0; j < 2; ++j) {
       mbar_init(smem_u32(&s_full[j]), 1);
-      mbar_init(smem_u32(&p_full[j]), 4);
+      mbar_init(smem_u32(&p_full[j]), 8);
       mbar_init(smem_u32(&o_full[j]), 1);
-      mbar_init(smem_u32(&q_stage_free[j]), 4);
+      mbar_init(smem_u32(&q_stage_free[j]), 8);
     }
     *abort_flag = 0;
     fence_mbar_init();
@@ -275,8 +280,10 @@ __global__ void __launch_bounds__(NUM_THREADS, 1) attn_tc_kernel(const __grid_co
       }
     }
   } else if (warp == 1) {
-    if (lane == 0) {
+    {
       // ------------------------------------------------------------ MMA --
+      // Every lane runs this loop and its bounded waits; elect_one_sync picks the lane that issues
+      // each tcgen05 instruction (issuing from a lane-divergent branch costs more per MMA).
       const uint32_t idesc_qk = idesc_f32acc(TQ, TK, 0, 0, kFmtF16);  // Q, K both K-major (d contiguous)
       const uint32_t idesc_pv = idesc_f32acc(TQ, D, 0, 1, kFmtF16);   // P from TMEM, V MN-major (d contiguous)
       int kst = 0, vst = 0;
@@ -306,16 +313,16 @@ __global__ void __launch_bounds__(NUM_THREADS, 1) attn_tc_kernel(const __grid_co
 #pragma unroll
           for (int kk = 0; kk < D / 16; ++kk) {
             const uint32_t off = ((kk >> 2) * HALF_BYTES + (kk & 3) * 32) >> 4;
-            umma_ss_lohi(tmem + COL_S0 + j * TK, alo + off, sw_hi, blo + off, sw_hi, idesc_qk, kk > 0);
+            if (elect_one_sync()) umma_ss_lohi(tmem + COL_S0 + j * TK, alo + off, sw_hi, blo + off, sw_hi, idesc_qk, kk > 0);
           }
-          umma_commit(smem_u32(&s_full[j]));
+          if (elect_one_sync()) umma_commit(smem_u32(&s_full[j]));
         };
         // first key tile: S_j = Q_j K_0^T for both tiles
         if (!mbar_wait_bounded(smem_u32(&k_full[kst]), kph, p.err, abort_flag, wait_site(kSiteAttn, 2, 6))) goto done;
         tc_fence_after();
         for (int j = 0; j < 2; ++j)
           if (it.active[j]) issue_qk(j, kst);
-        umma_commit(smem_u32(&k_empty[kst]));
+        if (elect_one_sync()) umma_commit(smem_u32(&k_empty[kst]));
         if (++kst == K_STAGES) {
           kst = 0;
           kph ^= 1;
@@ -333,7 +340,7 @@ __global__ void __launch_bounds__(NUM_THREADS, 1) attn_tc_kernel(const __grid_co
             // O_j += P_j V_jj
 #pragma unroll
             for (int kk = 0; kk < TK / 16; ++kk)
-              umma_ts_lohi(tmem + COL_O0 + j * D, tmem + COL_S0 + j * TK + kk * 8, vlo + ((kk * 16 * 128) >> 4),
+              if (elect_one_sync()) umma_ts_lohi(tmem + COL_O0 + j * D, tmem + COL_S0 + j * TK + kk * 8, vlo + ((kk * 16 * 128) >> 4),
                            v_hi, idesc_pv, (jj > it.k0 || kk > 0));
             if (jj + 1 <= it.qt[j] && jj + 1 < it.k1) {
               if (!next_k_ready) {
@@ -343,31 +350,40 @@ __global__ void __launch_bounds__(NUM_THREADS, 1) attn_tc_kernel(const __grid_co
               }
               issue_qk(j, kst);  // S_j = Q_j K_{jj+1}^T, overwrites P_j after the PV above
             } else {
-              umma_commit(smem_u32(&o_full[j]));
+              if (elect_one_sync()) umma_commit(smem_u32(&o_full[j]));
             }
           }
-          umma_commit(smem_u32(&v_empty[vst]));
+          if (elect_one_sync()) umma_commit(smem_u32(&v_empty[vst]));
           if (++vst == V_STAGES) {
             vst = 0;
             vph ^= 1;
           }
           if (next_k_ready) {
-            umma_commit(smem_u32(&k_empty[kst]));
+            if (elect_one_sync()) umma_commit(smem_u32(&k_empty[kst]));
             if (++kst == K_STAGES) {
               kst = 0;
               kph ^= 1;
             }
           }
         }
-        umma_commit(smem_u32(q_empty));
+        if (elect_one_sync()) umma_commit(smem_u32(q_empty));
       }
     }
   } else {
     // -------------------------------------------------------- softmax --
-    const int j = (warp - 2) >> 2;  // tile of this warpgroup
-    const int quad = warp & 3;      // TMEM lanes [32*quad, 32*quad + 32)
-    const int row = quad * 32 + lane;
-    const uint32_t lane_off = (uint32_t)(quad * 32) << 16;
+    // Eight warps per tile, two on each SMSP: warp (quad, hf) owns the 16 rows 32 quad + 16 hf .. +15
+    // of its TMEM lane quadrant. With the 16-lane TMEM shapes thread t holds rows ra = base + t/4 and
+    // rb = ra + 8, and of every 8-key chunk c the keys 8c + 2(t%4) + {0, 1}: a row is spread over
+    // the four threads of a quad, which combine its max with two shuffles; the row sums stay
+    // per thread until the epilogue.
+    const int sw = warp - 2;                // 0 .. 15
+    const int j = sw >> 3;                  // tile of this warp
+    const int wt = sw & 7;                  // warp within the tile
+    const int quad = warp & 3;              // TMEM lanes [32*quad, 32*quad + 32)
+    const int rbase = quad * 32 + ((wt >> 2) << 4);  // first of this warp's 16 rows
+    const int qd = lane & 3;                // key pair within each 8-key chunk
+    const int ra = rbase + (lane >> 2), rb = ra + 8;
+    const uint32_t lane_off = (uint32_t)rbase << 16;
     const uint32_t s_col = tmem + lane_off + COL_S0 + j * TK;
     const uint32_t o_col = tmem + lane_off + COL_O0 + j * D;
     uint32_t scount = 0, ocount = 0;
@@ -377,163 +393,209 @@ __global__ void __launch_bounds__(NUM_THREADS, 1) attn_tc_kernel(const __grid_co
       const Item it = get_item(p, w);
       if (it.active[j]) {
         const int qt = it.qt[j];
-        float m = -INFINITY;  // running max of scaled scores (log2 domain)
-        float l = 0.f;        // running row sum
+        float ma = -INFINITY, mb = -INFINITY;  // running max of scaled scores (log2 domain), rows ra / rb
+        float la = 0.f, lb = 0.f;              // this thread's share of the running row sums
         const int jlast = qt < it.k1 - 1 ? qt : it.k1 - 1;  // last key tile of this entry for the tile
         for (int jj = it.k0; jj <= jlast; ++jj) {
           if (!mbar_wait_bounded(smem_u32(&s_full[j]), scount & 1, p.err, abort_flag, wait_site(kSiteAttn, 3, 10))) goto done;
           ++scount;
           tc_fence_after();
-          uint32_t s[128];
-#pragma unroll
-          for (int c = 0; c < 4; ++c) tmem_ld_32x32b_x32(s_col + c * 32, s + c * 32);
+          uint32_t s[64];  // s[4c + e]: row ra, key 8c + 2qd + e; s[4c + 2 + e]: row rb (c = 0 .. 15)
+          tmem_ld_16x256b_x8(s_col, s);
+          tmem_ld_16x256b_x8(s_col + 64, s + 32);
           tmem_ld_wait();
           if (jj == qt) {  // diagonal tile: key c is visible to query row iff c <= row
 #pragma unroll
-            for (int c = 0; c < 128; ++c)
-              if (c > row) s[c] = __float_as_uint(-INFINITY);
-          }
-          // row max of the raw scores (the scale is positive), four independent chains
-          float mx0 = -INFINITY, mx1 = -INFINITY, mx2 = -INFINITY, mx3 = -INFINITY;
+            for (int c = 0; c < 16; ++c)
 #pragma unroll
-          for (int c = 0; c < 128; c += 8) {
-            mx0 = max3f(mx0, u2f(s[c + 0]), u2f(s[c + 1]));
-            mx1 = max3f(mx1, u2f(s[c + 2]), u2f(s[c + 3]));
-            mx2 = max3f(mx2, u2f(s[c + 4]), u2f(s[c + 5]));
-            mx3 = max3f(mx3, u2f(s[c + 6]), u2f(s[c + 7]));
+              for (int e = 0; e < 2; ++e) {
+                const int key = 8 * c + 2 * qd + e;
+                if (key > ra) s[4 * c + e] = __float_as_uint(-INFINITY);
+                if (key > rb) s[4 * c + 2 + e] = __float_as_uint(-INFINITY);
+              }
           }
-          const float tmax = fmaxf(fmaxf(mx0, mx1), fmaxf(mx2, mx3)) * p.scale_log2;
+          // row max of the raw scores (the scale is positive): two chains per row, then the quad
+          float xa0 = -INFINITY, xa1 = -INFINITY, xb0 = -INFINITY, xb1 = -INFINITY;
+#pragma unroll
+          for (int c = 0; c < 16; c += 2) {
+            xa0 = max3f(xa0, u2f(s[4 * c + 0]), u2f(s[4 * c + 1]));
+            xb0 = max3f(xb0, u2f(s[4 * c + 2]), u2f(s[4 * c + 3]));
+            xa1 = max3f(xa1, u2f(s[4 * c + 4]), u2f(s[4 * c + 5]));
+            xb1 = max3f(xb1, u2f(s[4 * c + 6]), u2f(s[4 * c + 7]));
+          }
+          float ta = fmaxf(xa0, xa1), tb = fmaxf(xb0, xb1);
+          ta = fmaxf(ta, __shfl_xor_sync(0xffffffffu, ta, 1));
+          tb = fmaxf(tb, __shfl_xor_sync(0xffffffffu, tb, 1));
+          ta = fmaxf(ta, __shfl_xor_sync(0xffffffffu, ta, 2)) * p.scale_log2;
+          tb = fmaxf(tb, __shfl_xor_sync(0xffffffffu, tb, 2)) * p.scale_log2;
           // lazy rescale: keep the stale max unless it grew by more than 2^8
-          const bool need = tmax > m + RESCALE_THRESHOLD;
-          float f = 1.f;  // factor for the O row and the sum
-          bool rescale = false;
+          float fa = 1.f, fb = 1.f;  // factors for the O rows and the sums
           if (jj == it.k0) {
-            m = tmax;
-          } else if (__any_sync(0xffffffffu, need)) {
-            const float mnew = fmaxf(m, tmax);
-            f = fast_exp2(m - mnew);
-            m = mnew;
-            rescale = true;
+            ma = ta;
+            mb = tb;
+          } else if (__any_sync(0xffffffffu, ta > ma + RESCALE_THRESHOLD || tb > mb + RESCALE_THRESHOLD)) {
+            const float na = fmaxf(ma, ta), nb = fmaxf(mb, tb);
+            fa = fast_exp2(ma - na);
+            fb = fast_exp2(mb - nb);
+            ma = na;
+            mb = nb;
+            // O_j is stable: the commit behind s_full covered the previous PV, and this warp raises
+            // p_full (which lets the next PV in) only after these stores have completed
+#pragma unroll 1
+            for (int g = 0; g < 4; ++g) {
+              uint32_t o[16];
+              tmem_ld_16x256b_x4(o_col + g * 32, o);
+              tmem_ld_wait();
+#pragma unroll
+              for (int c = 0; c < 4; ++c) {
+                o[4 * c + 0] = __float_as_uint(u2f(o[4 * c + 0]) * fa);
+                o[4 * c + 1] = __float_as_uint(u2f(o[4 * c + 1]) * fa);
+                o[4 * c + 2] = __float_as_uint(u2f(o[4 * c + 2]) * fb);
+                o[4 * c + 3] = __float_as_uint(u2f(o[4 * c + 3]) * fb);
+              }
+              tmem_st_16x256b_x4(o_col + g * 32, o);
+            }
           }
-          const float sc = p.scale_log2, nm = -m;
+          const float sc = p.scale_log2, nma = -ma, nmb = -mb;
           float sa0 = 0.f, sa1 = 0.f, sb0 = 0.f, sb1 = 0.f;  // packed partial row sums
 #pragma unroll
-          for (int c2 = 0; c2 < 2; ++c2) {
-            uint32_t pk[32];
+          for (int h2 = 0; h2 < 2; ++h2) {
+            // P columns 32 h2 .. 32 h2 + 31 (keys 64 h2 .. 64 h2 + 63) over the first half of S_j:
+            // pk[2cc] = row ra, pk[2cc + 1] = row rb, column 32 h2 + 4 cc + qd (keys 8c + 2qd, +1)
+            uint32_t pk[16];
 #pragma unroll
-            for (int e = 0; e < 32; ++e) {
-              float x0, x1, p0, p1;
-              fma2(x0, x1, u2f(s[c2 * 64 + 2 * e]), u2f(s[c2 * 64 + 2 * e + 1]), sc, sc, nm, nm);
-              if (CCA_POLY_EVERY > 0 && (e % (CCA_POLY_EVERY > 0 ? CCA_POLY_EVERY : 1)) == CCA_POLY_EVERY - 1) {
+            for (int cc = 0; cc < 8; ++cc) {
+              const int c = 8 * h2 + cc;
+              float x0, x1, x2, x3, p0, p1, p2, p3;
+              fma2(x0, x1, u2f(s[4 * c + 0]), u2f(s[4 * c + 1]), sc, sc, nma, nma);
+              fma2(x2, x3, u2f(s[4 * c + 2]), u2f(s[4 * c + 3]), sc, sc, nmb, nmb);
+              if (CCA_POLY_EVERY > 0 && (cc % (CCA_POLY_EVERY > 0 ? CCA_POLY_EVERY : 1)) == CCA_POLY_EVERY - 1) {
                 exp2_fma_x2(x0, x1, p0, p1);
+                exp2_fma_x2(x2, x3, p2, p3);
               } else {
                 p0 = fast_exp2(x0);
                 p1 = fast_exp2(x1);
+                p2 = fast_exp2(x2);
+                p3 = fast_exp2(x3);
               }
-              if (e & 1)
-                add2(sb0, sb1, sb0, sb1, p0, p1);
-              else
-                add2(sa0, sa1, sa0, sa1, p0, p1);
-              pk[e] = pack_f16x2(p0, p1);
+              add2(sa0, sa1, sa0, sa1, p0, p1);
+              add2(sb0, sb1, sb0, sb1, p2, p3);
+              pk[2 * cc] = pack_f16x2(p0, p1);
+              pk[2 * cc + 1] = pack_f16x2(p2, p3);
             }
-            tmem_st_32x32b_x32(s_col + c2 * 32, pk);
+            tmem_st_16x128b_x8(s_col + h2 * 32, pk);
           }
-          const float sum = (sa0 + sa1) + (sb0 + sb1);
-          l = l * f + sum;
-          if (rescale) {
-            // O_j is stable: the commit behind s_full covered the previous PV
-#pragma unroll 1
-            for (int c = 0; c < 4; ++c) {
-              uint32_t o[32];
-              tmem_ld_32x32b_x32(o_col + c * 32, o);
-              tmem_ld_wait();
-#pragma unroll
-              for (int e = 0; e < 32; ++e) o[e] = __float_as_uint(u2f(o[e]) * f);
-              tmem_st_32x32b_x32(o_col + c * 32, o);
-            }
-          }
+          la = la * fa + (sa0 + sa1);
+          lb = lb * fb + (sb0 + sb1);
           tmem_st_wait();
           tc_fence_before();
           __syncwarp();
           if (lane == 0) mbar_arrive(smem_u32(&p_full[j]));
         }
         // epilogue: O / l -> fp16 -> global
+        la += __shfl_xor_sync(0xffffffffu, la, 1);
+        lb += __shfl_xor_sync(0xffffffffu, lb, 1);
+        la += __shfl_xor_sync(0xffffffffu, la, 2);
+        lb += __shfl_xor_sync(0xffffffffu, lb, 2);
         if (!mbar_wait_bounded(smem_u32(&o_full[j]), ocount & 1, p.err, abort_flag, wait_site(kSiteAttn, 3, 11))) goto done;
         ++ocount;
         tc_fence_after();
         // O_row = O * inv for a whole-range entry; a merged split pair gives c1 * O_first + c2 * O_second,
         // evaluated in that order whichever half merges, so the result does not depend on timing
-        float c1 = 0.f, c2 = 0.f, inv = 1.f / l;
+        float c1a = 0.f, c2a = 0.f, c1b = 0.f, c2b = 0.f, inva = 1.f / la, invb = 1.f / lb;
         const float* other = nullptr;
         bool store = true;
         if (it.half != 0) {
-          // one half of a split pair: publish this half's unnormalised row with its max and sum;
-          // the second of the two halves to get here (counted per lane quadrant) merges them
+          // one half of a split pair: publish this half's unnormalised rows with their max and sum
+          // ([16 chunks of 8 columns][128 rows][8] fp32, then max [128] and sum [128]); the second of
+          // the two halves to get here (counted per warp) merges them
           const size_t tile = (size_t)it.w * 2 + j;
           float* mine = p.part + ((size_t)it.w * 4 + (it.half - 1) * 2 + j) * PART_TILE;
           other = p.part + ((size_t)it.w * 4 + (2 - it.half) * 2 + j) * PART_TILE;
 #pragma unroll 1
-          for (int c = 0; c < 4; ++c) {
-            uint32_t o[32];
-            tmem_ld_32x32b_x32(o_col + c * 32, o);
+          for (int g = 0; g < 4; ++g) {
+            uint32_t o[16];
+            tmem_ld_16x256b_x4(o_col + g * 32, o);
             tmem_ld_wait();
-            float4* d4 = reinterpret_cast<float4*>(mine) + (c * 8) * TQ + row;  // column quad c*8 + v
 #pragma unroll
-            for (int v = 0; v < 8; ++v)
-              d4[v * TQ] = make_float4(u2f(o[4 * v]), u2f(o[4 * v + 1]), u2f(o[4 * v + 2]), u2f(o[4 * v + 3]));
+            for (int c = 0; c < 4; ++c) {
+              const int ch = 4 * g + c;
+              *reinterpret_cast<float2*>(mine + ((size_t)ch * TQ + ra) * 8 + 2 * qd) =
+                  make_float2(u2f(o[4 * c + 0]), u2f(o[4 * c + 1]));
+              *reinterpret_cast<float2*>(mine + ((size_t)ch * TQ + rb) * 8 + 2 * qd) =
+                  make_float2(u2f(o[4 * c + 2]), u2f(o[4 * c + 3]));
+            }
           }
-          mine[D * TQ + row] = m;
-          mine[D * TQ + TQ + row] = l;
+          if (qd == 0) {
+            mine[D * TQ + ra] = ma;
+            mine[D * TQ + rb] = mb;
+            mine[D * TQ + TQ + ra] = la;
+            mine[D * TQ + TQ + rb] = lb;
+          }
           __threadfence();
           __syncwarp();
           int ticket = 0;
-          if (lane == 0) ticket = atomicAdd(p.split_cnt + tile * 4 + quad, 1);
+          if (lane == 0) ticket = atomicAdd(p.split_cnt + tile * 8 + wt, 1);
           ticket = __shfl_sync(0xffffffffu, ticket, 0);
           store = ticket != 0;
           if (store) {
             __threadfence();
-            const float mo = __ldcg(other + D * TQ + row), lo = __ldcg(other + D * TQ + TQ + row);
-            const float m1 = it.half == 1 ? m : mo, l1 = it.half == 1 ? l : lo;
-            const float m2 = it.half == 1 ? mo : m, l2 = it.half == 1 ? lo : l;
-            const float mm = fmaxf(m1, m2);
-            const float e1 = fast_exp2(m1 - mm), e2 = fast_exp2(m2 - mm);
-            const float rl = 1.f / __fmaf_rn(e1, l1, __fmul_rn(e2, l2));
-            c1 = __fmul_rn(e1, rl);
-            c2 = __fmul_rn(e2, rl);
-            inv = 1.f;  // the raw O rows are merged
+            const bool first = it.half == 1;  // this half holds O_first
+            auto coeffs = [&](int row, float m, float l, float& c1, float& c2) {
+              const float mo = __ldcg(other + D * TQ + row), lo = __ldcg(other + D * TQ + TQ + row);
+              const float m1 = first ? m : mo, l1 = first ? l : lo;
+              const float m2 = first ? mo : m, l2 = first ? lo : l;
+              const float mm = fmaxf(m1, m2);
+              const float e1 = fast_exp2(m1 - mm), e2 = fast_exp2(m2 - mm);
+              const float rl = 1.f / __fmaf_rn(e1, l1, __fmul_rn(e2, l2));
+              c1 = __fmul_rn(e1, rl);
+              c2 = __fmul_rn(e2, rl);
+            };
+            coeffs(ra, ma, la, c1a, c2a);
+            coeffs(rb, mb, lb, c1b, c2b);
+            inva = invb = 1.f;  // the raw O rows are merged
           }
         }
         // O rows leave through Q_j's buffer (its last QK has completed): [2 halves][128 rows][128 B]
-        // with the 128-byte swizzle, one TMA tensor store per 64-column half of this warp's 32 rows
+        // with the 128-byte swizzle, one TMA tensor store per 64-column half of this warp's 16 rows
         uint8_t* stage = smem + OFF_Q + j * TILE_BYTES;
 #pragma unroll 1
-        for (int c = 0; c < 4 && store; ++c) {
-          uint32_t o[32];
-          tmem_ld_32x32b_x32(o_col + c * 32, o);
+        for (int g = 0; g < 4 && store; ++g) {
+          uint32_t o[16];
+          tmem_ld_16x256b_x4(o_col + g * 32, o);
           tmem_ld_wait();
-          float f[32];
+          float f[16];
 #pragma unroll
-          for (int e = 0; e < 32; ++e) f[e] = u2f(o[e]) * inv;
+          for (int c = 0; c < 4; ++c) {
+            f[4 * c + 0] = u2f(o[4 * c + 0]) * inva;
+            f[4 * c + 1] = u2f(o[4 * c + 1]) * inva;
+            f[4 * c + 2] = u2f(o[4 * c + 2]) * invb;
+            f[4 * c + 3] = u2f(o[4 * c + 3]) * invb;
+          }
           if (other != nullptr) {
-            const float4* s4 = reinterpret_cast<const float4*>(other) + (c * 8) * TQ + row;
-            const bool first = it.half == 1;  // this half holds O_first
+            const bool first = it.half == 1;
 #pragma unroll
-            for (int v = 0; v < 8; ++v) {
-              const float4 x4 = __ldcg(s4 + v * TQ);
-              const float x[4] = {x4.x, x4.y, x4.z, x4.w};
+            for (int c = 0; c < 4; ++c) {
+              const int ch = 4 * g + c;
+              const float2 xa = __ldcg(reinterpret_cast<const float2*>(other + ((size_t)ch * TQ + ra) * 8 + 2 * qd));
+              const float2 xb = __ldcg(reinterpret_cast<const float2*>(other + ((size_t)ch * TQ + rb) * 8 + 2 * qd));
+              const float x[4] = {xa.x, xa.y, xb.x, xb.y};
 #pragma unroll
               for (int u = 0; u < 4; ++u) {
-                const float o1 = first ? f[4 * v + u] : x[u], o2 = first ? x[u] : f[4 * v + u];
-                f[4 * v + u] = __fmaf_rn(c1, o1, __fmul_rn(c2, o2));
+                const float k1 = u < 2 ? c1a : c1b, k2 = u < 2 ? c2a : c2b;
+                const float o1 = first ? f[4 * c + u] : x[u], o2 = first ? x[u] : f[4 * c + u];
+                f[4 * c + u] = __fmaf_rn(k1, o1, __fmul_rn(k2, o2));
               }
             }
           }
 #pragma unroll
-          for (int u = 0; u < 4; ++u) {  // columns c*32 + 8u .. +7: half c/2, chunk (c%2)*4 + u
-            const int chunk = (c & 1) * 4 + u;
-            *reinterpret_cast<uint4*>(stage + (c >> 1) * HALF_BYTES + row * 128 + ((chunk ^ (row & 7)) << 4)) =
-                make_uint4(pack_f16x2(f[8 * u + 0], f[8 * u + 1]), pack_f16x2(f[8 * u + 2], f[8 * u + 3]),
-                           pack_f16x2(f[8 * u + 4], f[8 * u + 5]), pack_f16x2(f[8 * u + 6], f[8 * u + 7]));
+          for (int c = 0; c < 4; ++c) {  // columns 8 ch + 2 qd, +1 of 16-byte chunk ch: half ch / 8, chunk ch % 8
+            const int ch = 4 * g + c;
+            uint8_t* base = stage + (ch >> 3) * HALF_BYTES + 4 * qd;
+            *reinterpret_cast<uint32_t*>(base + ra * 128 + (((ch & 7) ^ (ra & 7)) << 4)) =
+                pack_f16x2(f[4 * c + 0], f[4 * c + 1]);
+            *reinterpret_cast<uint32_t*>(base + rb * 128 + (((ch & 7) ^ (rb & 7)) << 4)) =
+                pack_f16x2(f[4 * c + 2], f[4 * c + 3]);
           }
         }
         if (store) {
@@ -542,8 +604,8 @@ __global__ void __launch_bounds__(NUM_THREADS, 1) attn_tc_kernel(const __grid_co
           if (lane == 0) {  // rows past S are clipped by the map
 #pragma unroll
             for (int hf = 0; hf < 2; ++hf)
-              tma_store_3d(&maps.o, smem_u32(stage + hf * HALF_BYTES + quad * 32 * 128), it.h[j] * D + hf * 64,
-                           qt * TQ + quad * 32, it.b);
+              tma_store_3d(&maps.o, smem_u32(stage + hf * HALF_BYTES + rbase * 128), it.h[j] * D + hf * 64,
+                           qt * TQ + rbase, it.b);
             bulk_commit();
           }
         }
@@ -693,7 +755,7 @@ cudaError_t launch_attention_tc(const BlockDims& dm, const void* q, const void* 
   if (!encode_3d(&maps.q, q, (uint64_t)dm.Lq, (uint64_t)dm.S, (uint64_t)dm.B) ||
       !encode_3d(&maps.k, k, (uint64_t)dm.Lkv, (uint64_t)dm.S, (uint64_t)dm.B) ||
       !encode_3d(&maps.v, v, (uint64_t)dm.Lkv, (uint64_t)dm.S, (uint64_t)dm.B) ||
-      !encode_3d(&maps.o, o, (uint64_t)dm.Lq, (uint64_t)dm.S, (uint64_t)dm.B, 32))
+      !encode_3d(&maps.o, o, (uint64_t)dm.Lq, (uint64_t)dm.S, (uint64_t)dm.B, 16))
     return cudaErrorInvalidValue;
   AttnParams p;
   p.B = dm.B;

@@ -10,8 +10,8 @@
 //
 // Design: persistent CTAs (one per SM) walk 128 x 256 output tiles. Warp 0
 // issues TMA loads of 128 x 64 A tiles and 256 x 64 B tiles (128-byte swizzle)
-// into a 4-stage shared-memory ring; one thread of warp 1 issues
-// tcgen05.mma (M=128, N=256, K=16) into one of two 256-column fp32
+// into a 4-stage shared-memory ring; warp 1 runs the MMA loop and an elected
+// lane issues tcgen05.mma (M=128, N=256, K=16) into one of two 256-column fp32
 // accumulators in tensor memory; warps 2-5 drain the other accumulator so the
 // epilogue of tile i overlaps the main loop of tile i+1. For 16-bit outputs
 // each epilogue warp converts 32 rows x 64 columns at a time into its own
@@ -185,8 +185,10 @@ __global__ void __launch_bounds__(Shape<MH>::NUM_THREADS, 1) gemm_tc_kernel(cons
     producer_done:;
     }
   } else if (warp == 1) {
-    if (lane == 0) {
+    {
       // ------------------------------------------------------ MMA issuer --
+      // Every lane runs this loop and its bounded waits; elect_one_sync picks the lane that issues
+      // each tcgen05 instruction (issuing from a lane-divergent branch costs more per MMA).
       const uint32_t idesc = idesc_f32acc(128, BN, 0, 0, p.in_fmt);
       // descriptors built once; a stage step adds STAGE_BYTES / 16 to the start address, a K = 16 step 2
       const uint32_t d_hi = desc_hi(smem_desc_sw128(smem_u32(smem), 16, 1024));
@@ -209,15 +211,15 @@ __global__ void __launch_bounds__(Shape<MH>::NUM_THREADS, 1) gemm_tc_kernel(cons
           for (int k = 0; k < BK / 16; ++k)
 #pragma unroll
             for (int h = 0; h < MH; ++h)  // rows h*128.. of the tile -> accumulator columns h*256..
-              umma_ss_lohi(d_tmem + h * BN, a_lo + h * (A_HALF_BYTES >> 4) + 2 * k, d_hi, b_lo + 2 * k, d_hi, idesc,
+              if (elect_one_sync()) umma_ss_lohi(d_tmem + h * BN, a_lo + h * (A_HALF_BYTES >> 4) + 2 * k, d_hi, b_lo + 2 * k, d_hi, idesc,
                            (kb | k) != 0);
-          umma_commit(smem_u32(&empty[stage]));
+          if (elect_one_sync()) umma_commit(smem_u32(&empty[stage]));
           if (++stage == STAGES) {
             stage = 0;
             phase ^= 1;
           }
         }
-        umma_commit(smem_u32(&tfull[acc]));
+        if (elect_one_sync()) umma_commit(smem_u32(&tfull[acc]));
       }
     mma_done:;
     }

@@ -97,7 +97,7 @@ cudaError_t launch_attention_tc(const BlockDims& dm, const void* q, const void* 
 // Split-pair scratch of the tensor-core attention: kAttnSplitCounters ints that must be zero when
 // it starts (the preprocessing kernels clear them), then the partial rows.
 constexpr int kAttnMaxSplit = 64;
-constexpr int kAttnSplitCounters = kAttnMaxSplit * 2 * 4;
+constexpr int kAttnSplitCounters = kAttnMaxSplit * 2 * 8;
 size_t attention_tc_scratch_bytes(const BlockDims& dm);
 
 // ---- one decode step (token t = S - 1 of every sequence), fp32 arithmetic ----
