@@ -10,8 +10,9 @@
 // One CTA owns a pair of 128-query tiles of one KV group (for G >= 2 two
 // query heads at the same positions, for G = 1 two consecutive query tiles
 // of one head), so every K/V tile it loads serves both. Roles:
-//   warp 0      TMA: Q tiles once per pair, then K tiles (3-stage ring) and V
-//               tiles (2-stage ring)
+//   warp 0      TMA, run by the whole warp with an elected lane issuing: Q
+//               tiles once per pair, then K tiles (3-stage ring) and V tiles
+//               (2-stage ring)
 //   warp 1      the MMA loop, run by the whole warp so that its control flow
 //               and descriptor arithmetic stay warp-uniform; an elected lane
 //               issues tcgen05.mma: S_j = Q_j K^T (SS form) into TMEM, then
@@ -88,7 +89,7 @@ __device__ __forceinline__ void exp2_fma_x2(float x0, float x1, float& p0, float
   p1 = __int_as_float(__float_as_int(q1) + (__float_as_int(t1) << 23));
 }
 #ifndef CCA_POLY_EVERY
-#define CCA_POLY_EVERY 8  // one pair in CCA_POLY_EVERY takes exp2_fma_x2 (0: none)
+#define CCA_POLY_EVERY 4  // one pair in CCA_POLY_EVERY takes exp2_fma_x2 (0: none)
 #endif
 
 struct AttnMaps {
@@ -226,8 +227,9 @@ __global__ void __launch_bounds__(NUM_THREADS, 1) attn_tc_kernel(const __grid_co
   const int cta = blockIdx.x, grid = gridDim.x;
 
   if (warp == 0) {
-    if (lane == 0) {
+    {
       // ------------------------------------------------------------ TMA --
+      // Every lane runs this loop and its bounded waits; an elected lane issues each copy.
       int kst = 0, vst = 0;
       uint32_t kph = 0, vph = 0;
       for (int r = 0;; ++r) {
@@ -240,22 +242,22 @@ __global__ void __launch_bounds__(NUM_THREADS, 1) attn_tc_kernel(const __grid_co
           if (r > 0 && !mbar_wait_bounded(smem_u32(&q_stage_free[j]), (r - 1) & 1, p.err, abort_flag,
                                           wait_site(kSiteAttn, 1, 13)))
             goto done;
-        mbar_arrive_expect_tx(smem_u32(q_full), 2 * TILE_BYTES);
+        if (elect_one_sync()) mbar_arrive_expect_tx(smem_u32(q_full), 2 * TILE_BYTES);
 #pragma unroll
         for (int j = 0; j < 2; ++j)
 #pragma unroll
           for (int hf = 0; hf < 2; ++hf)
-            tma_load_3d(smem_u32(smem + OFF_Q + j * TILE_BYTES + hf * HALF_BYTES), &maps.q, smem_u32(q_full),
+            if (elect_one_sync()) tma_load_3d(smem_u32(smem + OFF_Q + j * TILE_BYTES + hf * HALF_BYTES), &maps.q, smem_u32(q_full),
                         it.h[j] * D + hf * 64, it.qt[j] * TQ, it.b);
         // K runs one tile ahead of V: the MMA thread needs K_{jj+1} right after its PVs on V_jj,
         // and a wait for a free V slot must not hold back the next K load
         auto load_k = [&](int jj) -> bool {
           if (!mbar_wait_bounded(smem_u32(&k_empty[kst]), kph ^ 1, p.err, abort_flag, wait_site(kSiteAttn, 1, 2)))
             return false;
-          mbar_arrive_expect_tx(smem_u32(&k_full[kst]), TILE_BYTES);
+          if (elect_one_sync()) mbar_arrive_expect_tx(smem_u32(&k_full[kst]), TILE_BYTES);
 #pragma unroll
           for (int hf = 0; hf < 2; ++hf)
-            tma_load_3d(smem_u32(smem + OFF_K + kst * TILE_BYTES + hf * HALF_BYTES), &maps.k, smem_u32(&k_full[kst]),
+            if (elect_one_sync()) tma_load_3d(smem_u32(smem + OFF_K + kst * TILE_BYTES + hf * HALF_BYTES), &maps.k, smem_u32(&k_full[kst]),
                         it.g * D + hf * 64, jj * TK, it.b);
           if (++kst == K_STAGES) {
             kst = 0;
@@ -267,10 +269,10 @@ __global__ void __launch_bounds__(NUM_THREADS, 1) attn_tc_kernel(const __grid_co
         for (int jj = it.k0; jj < it.k1; ++jj) {
           if (jj + 1 < it.k1 && !load_k(jj + 1)) goto done;
           if (!mbar_wait_bounded(smem_u32(&v_empty[vst]), vph ^ 1, p.err, abort_flag, wait_site(kSiteAttn, 1, 3))) goto done;
-          mbar_arrive_expect_tx(smem_u32(&v_full[vst]), TILE_BYTES);
+          if (elect_one_sync()) mbar_arrive_expect_tx(smem_u32(&v_full[vst]), TILE_BYTES);
 #pragma unroll
           for (int hf = 0; hf < 2; ++hf)
-            tma_load_3d(smem_u32(smem + OFF_V + vst * TILE_BYTES + hf * HALF_BYTES), &maps.v, smem_u32(&v_full[vst]),
+            if (elect_one_sync()) tma_load_3d(smem_u32(smem + OFF_V + vst * TILE_BYTES + hf * HALF_BYTES), &maps.v, smem_u32(&v_full[vst]),
                         it.g * D + hf * 64, jj * TK, it.b);
           if (++vst == V_STAGES) {
             vst = 0;
