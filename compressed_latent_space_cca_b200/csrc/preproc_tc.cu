@@ -199,8 +199,9 @@ __host__ __device__ __forceinline__ size_t rope_table_offset(int H1, int K, int 
   return (end + 15) & ~(size_t)15;
 }
 
-template <int KC>
-__global__ void __launch_bounds__(NT, 2) preproc_tc_kernel(const __grid_constant__ PreParams p,
+// MINB: CTAs per SM the launch is built for (2, or 3 with one weight buffer and 80 registers)
+template <int KC, int MINB>
+__global__ void __launch_bounds__(NT, MINB) preproc_tc_kernel(const __grid_constant__ PreParams p,
                                                           const __grid_constant__ Theta th) {
   extern __shared__ __align__(16) uint8_t smem_raw[];
   const int G = p.nq / p.nkv;
@@ -495,9 +496,14 @@ __global__ void __launch_bounds__(NT, 2) preproc_tc_kernel(const __grid_constant
 
 size_t smem_bytes(int G, int K, int nbuf) { return rope_table_offset(G + 1, K, nbuf) + sizeof(float2) * D; }
 
-// Two weight buffers when two CTAs still fit on one SM (228 KB of shared memory, 1 KB reserved per
-// CTA), else one.
-int weight_buffers(int G, int K) { return smem_bytes(G, K, 2) + 1024 <= 114 * 1024 ? 2 : 1; }
+// Occupancy of a shape (228 KB of shared memory per SM, 1 KB reserved per CTA): three CTAs per SM
+// with one weight buffer when they fit (the warps of the other CTAs hide the unprefetched weights;
+// 80 registers, a few spilled: measured 52.3 -> 50.1 us at S=16384, G=2), else two CTAs with two
+// weight buffers (the next head's weights prefetched), else two or one with one buffer.
+int ctas_per_sm(int G, int K) { return smem_bytes(G, K, 1) + 1024 <= 76 * 1024 ? 3 : 2; }
+int weight_buffers(int G, int K) {
+  return ctas_per_sm(G, K) == 3 || smem_bytes(G, K, 2) + 1024 > 114 * 1024 ? 1 : 2;
+}
 
 }  // namespace
 
@@ -536,7 +542,9 @@ cudaError_t launch_preproc_tc(const BlockDims& dm, const BlockPtrs& p, cudaStrea
   q.nbuf = weight_buffers(dm.G, dm.K);
   const size_t smem = smem_bytes(dm.G, dm.K, q.nbuf);
   dim3 grid((dm.S + TT - 1) / TT, dm.nkv, dm.B);
-  auto kern = dm.K == 4 ? preproc_tc_kernel<4> : preproc_tc_kernel<0>;
+  const bool three = ctas_per_sm(dm.G, dm.K) == 3;
+  auto kern = dm.K == 4 ? (three ? preproc_tc_kernel<4, 3> : preproc_tc_kernel<4, 2>)
+                        : (three ? preproc_tc_kernel<0, 3> : preproc_tc_kernel<0, 2>);
   cudaError_t e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
   if (e != cudaSuccess) return e;
   kern<<<grid, NT, smem, stream>>>(q, th);
