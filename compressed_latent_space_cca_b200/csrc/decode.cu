@@ -21,7 +21,8 @@
 //                       cache row t). Body: lanes split each key's head_dim, hold q in registers
 //                       and keep an online softmax per head; the CTA's lane groups merge in shared
 //                       memory, and the last chunk of a (group, sequence) to finish (an atomic
-//                       count, no waiting) merges the chunks
+//                       count, no waiting) merges the chunks in two rounds of loads (every chunk's
+//                       max and sum, then every chunk's output columns, a batch at a time)
 //   decode_out_kernel   y_t = o W_o^T, a warp per output channel
 // No kernel waits on a later one, so the chain always completes.
 #include <math.h>
@@ -36,7 +37,6 @@ constexpr int DNT = 256;           // threads of the GEMV and conv kernels
 constexpr int ANT = 256;           // attention threads
 constexpr int kGemvBatch = 8;      // sequences per GEMV launch
 constexpr int kMaxChunks = 256;    // key chunks per (KV group, sequence)
-constexpr int kRingStages = 4;     // attention: 32 KB stages of key and value rows in flight
 constexpr float kLog2e = 1.4426950408889634f;
 
 struct DecodeArgs {
@@ -628,75 +628,78 @@ __global__ void __launch_bounds__(ANT) decode_attn_kernel(const __grid_constant_
   if (*flag != a.nch - 1) return;
 
   // the last chunk to finish merges the chunks of this (group, sequence): o = sum_c 2^(m_c - M) o_c /
-  // sum_c 2^(m_c - M) l_c. Thread (piece, sb) takes float4 piece `piece` of the chunks c = sb mod
-  // nsub, loading a batch of them at once and keeping a running max; the nsub results then merge.
-  const float* po_all = a.part_o + bg * a.nch * G * D;
-  const float* pml_all = a.part_ml + bg * a.nch * G * 2;
-  const int n4 = G * D / 4;  // float4 pieces of the group's output (<= ANT)
-  const int nsub = ANT / n4;
-  const int piece = threadIdx.x % n4, sb = threadIdx.x / n4;
-  if (sb < nsub) {
-    constexpr int MB = 16;
-    const int h = piece * 4 / D;
-    float M = -INFINITY, Ls = 0.f;
-    float4 acc = make_float4(0.f, 0.f, 0.f, 0.f);
-    for (int c0 = sb; c0 < a.nch; c0 += MB * nsub) {
-      float4 ov[MB];
-      float2 ml[MB];
+  // sum_c 2^(m_c - M) l_c, in two rounds of loads: first every chunk's (max, sum) (thread c) and
+  // from them the maxima M and the sums L per head; then thread (head, columns) reads its columns
+  // of every chunk, a batch of independent loads at a time.
+  {
+    constexpr int NW = ANT / 32;
+    constexpr int OPT = GM * D / ANT > 0 ? GM * D / ANT : 1;  // output columns per thread
+    static_assert(OPT == 1 || OPT == 2 || OPT == 4, "output columns per thread");
+    static_assert((size_t)kMaxChunks * GM * sizeof(float) <= C::RING, "merge weights fit the ring");
+    static_assert(2 * GM * NW * sizeof(float) <= 24 * ANT, "merge sums fit the scratch");
+    const float* po_all = a.part_o + bg * a.nch * G * D;
+    const float* pml_all = a.part_ml + bg * a.nch * G * 2;
+    float* wgt = reinterpret_cast<float*>(sma);                 // [nch][GM] weights, over the ring
+    float* mred = reinterpret_cast<float*>(sma + C::OFF_SUB);  // [2][GM][NW] per-warp max and sum
+    const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+    const int c = threadIdx.x;  // nch <= kMaxChunks = ANT
+    float cm[GM], cl[GM];
 #pragma unroll
-      for (int k = 0; k < MB; ++k) {
-        const int c = c0 + k * nsub;
-        if (c < a.nch) {
-          ov[k] = __ldcg(reinterpret_cast<const float4*>(po_all + (long long)c * G * D) + piece);
-          ml[k] = __ldcg(reinterpret_cast<const float2*>(pml_all + (c * G + h) * 2));
-        } else {
-          ov[k] = make_float4(0.f, 0.f, 0.f, 0.f);
-          ml[k] = make_float2(-INFINITY, 0.f);
-        }
-      }
+    for (int h = 0; h < GM; ++h) {
+      const float2 ml = (c < a.nch && h < G) ? __ldcg(reinterpret_cast<const float2*>(pml_all + (c * G + h) * 2))
+                                             : make_float2(-INFINITY, 0.f);
+      cm[h] = ml.x;
+      cl[h] = ml.y;
+      const float wm = warp_max(cm[h]);
+      if (lane == 0) mred[h * NW + warp] = wm;
+    }
+    __syncthreads();
 #pragma unroll
-      for (int k = 0; k < MB; ++k) {
-        if (ml[k].x == -INFINITY) continue;
-        if (ml[k].x > M) {
-          const float sc = exp2f(M - ml[k].x);  // 0 when M is still -inf
-          acc.x *= sc, acc.y *= sc, acc.z *= sc, acc.w *= sc;
-          Ls *= sc;
-          M = ml[k].x;
+    for (int h = 0; h < GM; ++h) {
+      float M = -INFINITY;
+#pragma unroll
+      for (int w = 0; w < NW; ++w) M = fmaxf(M, mred[h * NW + w]);
+      const float wc = cm[h] == -INFINITY ? 0.f : exp2f(cm[h] - M);
+      if (c < a.nch) wgt[c * GM + h] = wc;
+      const float ws = warp_sum(wc * cl[h]);
+      if (lane == 0) mred[GM * NW + h * NW + warp] = ws;
+    }
+    __syncthreads();
+    const int oh = threadIdx.x * OPT / D, oc = threadIdx.x * OPT % D;
+    if (oh < G) {
+      float L = 0.f;
+#pragma unroll
+      for (int w = 0; w < NW; ++w) L += mred[GM * NW + oh * NW + w];
+      float r[OPT];
+#pragma unroll
+      for (int e = 0; e < OPT; ++e) r[e] = 0.f;
+      constexpr int MB = 32;  // chunk values in flight per thread
+      for (int c0 = 0; c0 < a.nch; c0 += MB) {
+        float x[MB][OPT];
+#pragma unroll
+        for (int k = 0; k < MB; ++k) {
+          const float* src = po_all + (long long)(c0 + k) * G * D + oh * D + oc;
+#pragma unroll
+          for (int e = 0; e < OPT; ++e) x[k][e] = c0 + k < a.nch ? __ldcg(src + e) : 0.f;
         }
-        const float w = exp2f(ml[k].x - M);
-        acc.x = fmaf(w, ov[k].x, acc.x);
-        acc.y = fmaf(w, ov[k].y, acc.y);
-        acc.z = fmaf(w, ov[k].z, acc.z);
-        acc.w = fmaf(w, ov[k].w, acc.w);
-        Ls = fmaf(w, ml[k].y, Ls);
+        float ru[4][OPT];
+#pragma unroll
+        for (int u = 0; u < 4; ++u)
+#pragma unroll
+          for (int e = 0; e < OPT; ++e) ru[u][e] = 0.f;
+#pragma unroll
+        for (int k = 0; k < MB; ++k) {
+          const float w = c0 + k < a.nch ? wgt[(c0 + k) * GM + oh] : 0.f;
+#pragma unroll
+          for (int e = 0; e < OPT; ++e) ru[k & 3][e] = fmaf(w, x[k][e], ru[k & 3][e]);
+        }
+#pragma unroll
+        for (int e = 0; e < OPT; ++e) r[e] += (ru[0][e] + ru[1][e]) + (ru[2][e] + ru[3][e]);
       }
+      const float li = 1.f / L;
+#pragma unroll
+      for (int e = 0; e < OPT; ++e) a.o[(long long)b * a.Lq + (long long)(g * G + oh) * D + oc + e] = r[e] * li;
     }
-    sub[threadIdx.x] = acc;
-    sub_ml[threadIdx.x] = make_float2(M, Ls);
-  }
-  __syncthreads();
-  if (threadIdx.x < n4) {
-    float M = -INFINITY;
-    for (int k = 0; k < nsub; ++k) M = fmaxf(M, sub_ml[k * n4 + threadIdx.x].x);
-    float4 r = make_float4(0.f, 0.f, 0.f, 0.f);
-    float Ls = 0.f;
-    for (int k = 0; k < nsub; ++k) {
-      const float2 ml = sub_ml[k * n4 + threadIdx.x];
-      if (ml.x == -INFINITY) continue;
-      const float w = exp2f(ml.x - M);
-      const float4 u = sub[k * n4 + threadIdx.x];
-      r.x = fmaf(w, u.x, r.x);
-      r.y = fmaf(w, u.y, r.y);
-      r.z = fmaf(w, u.z, r.z);
-      r.w = fmaf(w, u.w, r.w);
-      Ls = fmaf(w, ml.y, Ls);
-    }
-    const float li = 1.f / Ls;
-    r.x *= li;
-    r.y *= li;
-    r.z *= li;
-    r.w *= li;
-    *reinterpret_cast<float4*>(a.o + (long long)b * a.Lq + (long long)g * G * D + threadIdx.x * 4) = r;
   }
 }
 
