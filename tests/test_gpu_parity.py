@@ -63,6 +63,7 @@ BF16_CASES = [
     dict(seq_len=129, n_q_heads=8, n_kv_heads=2, hidden=1024, batch=3),   # G=4
     dict(seq_len=200, n_q_heads=2, n_kv_heads=1, hidden=512),             # n_kv=1: shift within the head
     dict(seq_len=383, n_q_heads=2, n_kv_heads=2, hidden=256),             # C=1
+    dict(seq_len=300, n_q_heads=3, n_kv_heads=1, hidden=384),             # G=3; GEMM widths 640 and 384 end mid-tile
 ]
 
 
