@@ -171,6 +171,21 @@ def test_deterministic_and_causal(path):
         assert not np.array_equal(c[k][1, t0], a[k][1, t0]), k
 
 
+@pytest.mark.parametrize("path", [AUTO, TENSOR], ids=["auto", "tensor"])
+def test_bf16_long_ragged(path):
+    """S = 4097: 33 query tiles whose last holds one row, two sequences, the split
+    schedule of a long sequence; caches in full, y and O on sampled rows."""
+    sh = shape(seq_len=4097, batch=2)
+    inp = workloads.make_inputs(sh)
+    rows = sample_rows(sh.seq_len, 40, seed=5)
+    gpu = run_gpu(sh, inp, path=path, rows=rows, stages=False)
+    ref = run_oracle(sh, inp, rows=rows)
+    assert_close("k_cache", gpu["k_cache"], ref["k_cache"], "bf16")
+    assert_close("v_cache", gpu["v_cache"], ref["v_cache"], "bf16")
+    assert_close("o", gpu["o"], ref["o"], "bf16")
+    assert_close("y", gpu["y"], ref["y"], "bf16")
+
+
 # ------------------------------------------------- the five named workloads --
 @pytest.mark.parametrize("name", ["cca_dense_bf16", "ccgqa_16k_bf16", "ccgqa_8x_bf16", "ccgqa_64k_bf16"])
 def test_named_workload_full_size(name):
