@@ -366,6 +366,13 @@ __global__ void __launch_bounds__(Shape<MH, PAIR>::NUM_THREADS, 1)
   }
   tc_fence_before();
   __syncthreads();
+  // after a wait of this CTA timed out, copies and MMAs it issued may still be landing in its shared
+  // and tensor memory: give them a bounded 20 us before that memory is released
+  if (*abort_flag) {
+    const unsigned long long t0 = globaltimer_ns();
+    while (globaltimer_ns() - t0 < 20000ull) {
+    }
+  }
   // a pair leaves together: no remote arrival or MMA of one CTA is still pending on the other
   if constexpr (PAIR) cluster_sync_all();
   tc_fence_after();
