@@ -22,6 +22,7 @@ import json
 import os
 import statistics
 import subprocess
+import tempfile
 import sys
 import time
 
@@ -114,7 +115,9 @@ class ClockSampler:
     def __init__(self, index: int):
         self.index = index
         self.proc = None
-        self.path = os.path.join(ROOT, "gpurun_out", f"clocks_rank{index}.csv")
+        # the raw samples: $CCA_BENCH_CLOCKS_DIR if set, else the system temporary directory
+        d = os.environ.get("CCA_BENCH_CLOCKS_DIR") or tempfile.gettempdir()
+        self.path = os.path.join(d, f"cca_bench_clocks_rank{index}.csv")
 
     def start(self):
         try:
