@@ -180,10 +180,31 @@ __global__ void __launch_bounds__(NT, 1) preproc_umma_kernel(const __grid_consta
     issue_loads(0);
   }
 
-  // seq-conv taps of the group's heads, [H1][D][K] in processing order (K head first)
-  for (int e = threadIdx.x; e < H1 * D * KK; e += NT) {
-    const int i = e / (D * KK), r = e - i * D * KK;
-    taps[e] = i == 0 ? p.ck_seq[(long long)g * D * KK + r] : p.cq_seq[(long long)(g * G + i - 1) * D * KK + r];
+  // seq-conv taps of the group's heads, [H1][D][K] in processing order (K head first): the K
+  // head's D*K taps, then the G query heads' (contiguous in cq_seq); 16-byte vectors when both
+  // sources allow them (D*K is a multiple of 8), every load issued before the stores
+  {
+    const __nv_bfloat16* qs = p.cq_seq + (long long)g * G * D * KK;
+    const __nv_bfloat16* ks = p.ck_seq + (long long)g * D * KK;
+    const int nk8 = D * KK / 8, n8 = H1 * D * KK / 8;
+    if (((reinterpret_cast<uintptr_t>(qs) | reinterpret_cast<uintptr_t>(ks)) & 15) == 0) {
+      constexpr int PER = ((GMAX + 1) * D * KMAX / 8 + NT - 1) / NT;
+      uint4 v[PER];
+#pragma unroll
+      for (int k = 0; k < PER; ++k) {
+        const int e = threadIdx.x + k * NT;
+        if (e < n8)
+          v[k] = e < nk8 ? reinterpret_cast<const uint4*>(ks)[e] : reinterpret_cast<const uint4*>(qs)[e - nk8];
+      }
+#pragma unroll
+      for (int k = 0; k < PER; ++k) {
+        const int e = threadIdx.x + k * NT;
+        if (e < n8) reinterpret_cast<uint4*>(taps)[e] = v[k];
+      }
+    } else {
+      for (int e = threadIdx.x; e < H1 * D * KK; e += NT)
+        taps[e] = e < D * KK ? ks[e] : qs[e - D * KK];
+    }
   }
   // RoPE table: (cos, sin) of t0 * theta_i, the angle reduced modulo 2 pi in fp64
   if (p.use_rope && threadIdx.x < D / 2) {
@@ -204,17 +225,24 @@ __global__ void __launch_bounds__(NT, 1) preproc_umma_kernel(const __grid_consta
     const long long cid = ((long long)blockIdx.z * gridDim.y + blockIdx.y) * gridDim.x + blockIdx.x;
     const long long chunk = (nvec + nct - 1) / nct;
     const long long lo = cid * chunk, hi = lo + chunk < nvec ? lo + chunk : nvec;
-    for (long long e = lo + threadIdx.x; e < hi; e += NT) {
-      const uint4 raw = *reinterpret_cast<const uint4*>(p.wo + e * 8);
-      const __nv_bfloat162* b2 = reinterpret_cast<const __nv_bfloat162*>(&raw);
-      uint32_t h[4];
+    for (long long e0 = lo + threadIdx.x; e0 < hi; e0 += 4 * NT) {  // four independent loads in flight
+      uint4 raw[4];
+#pragma unroll
+      for (int k = 0; k < 4; ++k)
+        if (e0 + k * NT < hi) raw[k] = *reinterpret_cast<const uint4*>(p.wo + (e0 + k * NT) * 8);
 #pragma unroll
       for (int k = 0; k < 4; ++k) {
-        const float2 f = __bfloat1622float2(b2[k]);
-        bad |= f16_overflow(f.x) || f16_overflow(f.y);
-        h[k] = pack_f16x2(f.x, f.y);
+        if (e0 + k * NT >= hi) continue;
+        const __nv_bfloat162* b2 = reinterpret_cast<const __nv_bfloat162*>(&raw[k]);
+        uint32_t h[4];
+#pragma unroll
+        for (int q = 0; q < 4; ++q) {
+          const float2 f = __bfloat1622float2(b2[q]);
+          bad |= f16_overflow(f.x) || f16_overflow(f.y);
+          h[q] = pack_f16x2(f.x, f.y);
+        }
+        *reinterpret_cast<uint4*>(p.wo_lat + (e0 + k * NT) * 8) = make_uint4(h[0], h[1], h[2], h[3]);
       }
-      *reinterpret_cast<uint4*>(p.wo_lat + e * 8) = make_uint4(h[0], h[1], h[2], h[3]);
     }
     if (p.zero_cnt != nullptr && cid == 0)
       for (int i = threadIdx.x; i < kAttnSplitCounters; i += NT) p.zero_cnt[i] = 0;
@@ -412,6 +440,21 @@ __global__ void __launch_bounds__(NT, 1) preproc_umma_kernel(const __grid_consta
     }
   }
 
+  {  // (a block of its own: the waits above leave to `done` past its declarations)
+  // value-shift sources, loaded now so that their latency overlaps the K head's combine: channels
+  // [Lkv/2, Lkv) come from the previous token (0 at a sequence start); 8-channel vectors never
+  // straddle that boundary
+  constexpr int VPER = TT * (D / 8) / NT;
+  uint4 vsrc[VPER];
+#pragma unroll
+  for (int k = 0; k < VPER; ++k) {
+    const int e = threadIdx.x + k * NT, rr = e / (D / 8), vv = e % (D / 8);
+    const int t = t0 + rr, gc = g * D + vv * 8;
+    const int src = (p.vshift && gc >= Lkv / 2) ? t - 1 : t;
+    vsrc[k] = make_uint4(0, 0, 0, 0);
+    if (t < p.S && src >= 0) vsrc[k] = *reinterpret_cast<const uint4*>(p.lat + (rowbase + src) * Nlat + Lq + Lkv + gc);
+  }
+
   // ---- the K head: k = c_k + PRE (mean q~ + k~)/2 + POST (mean c_q + c_k)/2, RoPE; staged as the
   // bf16 cache in s and the fp16 attention copy in weight buffer 0 (every MMA has completed)
   {
@@ -480,15 +523,13 @@ __global__ void __launch_bounds__(NT, 1) preproc_umma_kernel(const __grid_consta
     }
   }
 
-  // ---- value shift: channels [Lkv/2, Lkv) come from the previous token (0 at a sequence start);
-  // 8-channel vectors never straddle that boundary
-  for (int e = threadIdx.x; e < TT * (D / 8); e += NT) {
-    const int rr = e / (D / 8), vv = e % (D / 8);
+  // ---- value shift: the bf16 cache and the fp16 attention copy of the shifted v
+#pragma unroll
+  for (int k = 0; k < VPER; ++k) {
+    const int e = threadIdx.x + k * NT, rr = e / (D / 8), vv = e % (D / 8);
     const int t = t0 + rr, gc = g * D + vv * 8;
     if (t >= p.S) continue;
-    const int src = (p.vshift && gc >= Lkv / 2) ? t - 1 : t;
-    uint4 hv = make_uint4(0, 0, 0, 0);
-    if (src >= 0) hv = *reinterpret_cast<const uint4*>(p.lat + (rowbase + src) * Nlat + Lq + Lkv + gc);
+    const uint4 hv = vsrc[k];
     const __half2* h2 = reinterpret_cast<const __half2*>(&hv);
     uint32_t hb[4];
 #pragma unroll
@@ -499,6 +540,7 @@ __global__ void __launch_bounds__(NT, 1) preproc_umma_kernel(const __grid_consta
     const long long off = (rowbase + t) * Lkv + gc;
     *reinterpret_cast<uint4*>(p.v_cache + off) = make_uint4(hb[0], hb[1], hb[2], hb[3]);
     *reinterpret_cast<uint4*>(p.v_att + off) = hv;
+  }
   }
 
 done:
