@@ -56,7 +56,8 @@ constexpr int OFF_WB = OFF_SB + TILE;
 constexpr int OFF_TAPS = OFF_WB + 2 * TILE;
 constexpr int TAPS_BYTES = (GMAX + 1) * D * KMAX * 2;
 constexpr int OFF_RTAB = OFF_TAPS + TAPS_BYTES;
-constexpr int OFF_BAR = OFF_RTAB + (D / 2) * 8;
+constexpr int OFF_THF = OFF_RTAB + (D / 2) * 8;
+constexpr int OFF_BAR = OFF_THF + (D / 2) * 4;
 constexpr int SMEM_BYTES = OFF_BAR + 128 + 1024;  // barriers, TMEM slot, abort flag; alignment slack
 static_assert(SMEM_BYTES <= 232448, "shared memory of one CTA");
 static_assert(ZRMAX * 128 <= ZHALF, "latent half");
@@ -126,6 +127,7 @@ __global__ void __launch_bounds__(NT, 1) preproc_umma_kernel(const __grid_consta
   const uint32_t sbase = smem_u32(smem);
   __nv_bfloat16* taps = reinterpret_cast<__nv_bfloat16*>(smem + OFF_TAPS);  // [H1][D][K]
   float2* rtab = reinterpret_cast<float2*>(smem + OFF_RTAB);                 // (cos, sin) of t0 theta_i
+  float* thf = reinterpret_cast<float*>(smem + OFF_THF);                      // theta_i in fp32
   uint64_t* bars = reinterpret_cast<uint64_t*>(smem + OFF_BAR);
   uint64_t* lat_bar = bars;      // [3]: K head latents, query-head buffers 0 and 1
   uint64_t* w_bar = bars + 3;    // [2]: weight buffers
@@ -216,6 +218,7 @@ __global__ void __launch_bounds__(NT, 1) preproc_umma_kernel(const __grid_consta
     float c, sn;
     sincosf((float)r, &sn, &c);
     rtab[i] = make_float2(c, sn);
+    thf[i] = (float)th.v[i];
   }
   // side jobs while the first copies are in flight: this CTA's slice of the W_o fp16 copy, and the
   // attention's split counters
@@ -259,7 +262,7 @@ __global__ void __launch_bounds__(NT, 1) preproc_umma_kernel(const __grid_consta
     c = 1.f;
     s = 0.f;
     if (!p.use_rope) return;
-    const float a = (float)((double)r * th.v[i]);
+    const float a = (float)r * thf[i];  // r < 128: fp32 keeps the angle to a few ulp
     const float k = rintf(a * 0.15915494f);
     float x = fmaf(-k, 6.28318548f, a);  // 2 pi = 6.28318548f - 1.7484555e-7f
     x = fmaf(k, 1.7484555e-7f, x);
