@@ -150,7 +150,7 @@ __global__ void __launch_bounds__(NT, 1) preproc_umma_kernel(const __grid_consta
   auto wc_row = [&](int i) { return i == 0 ? (p.nq + g) * D : (g * G + i - 1) * D; };
   auto lat_buf = [&](int i) { return i == 0 ? OFF_LK : OFF_LQ + ((i - 1) & 1) * ZHEAD; };
   auto lat_barrier = [&](int i) { return smem_u32(&lat_bar[i == 0 ? 0 : 1 + ((i - 1) & 1)]); };
-  // one elected lane of warp 0 issues the copies of head i: latents and channel weights
+  // thread 0 issues the copies of head i: latents and channel weights
   auto issue_loads = [&](int i) {
     const uint32_t lb = lat_barrier(i), wb = smem_u32(&w_bar[i & 1]);
     mbar_arrive_expect_tx(lb, lat_bytes);
@@ -176,7 +176,7 @@ __global__ void __launch_bounds__(NT, 1) preproc_umma_kernel(const __grid_consta
   __syncthreads();
   tc_fence_after();
   const uint32_t tmem = *tmem_slot;
-  if (warp == 0 && elect_one_sync()) {
+  if (threadIdx.x == 0) {
     prefetch_tmap(&maps.lat);
     prefetch_tmap(&maps.wc);
     issue_loads(0);
@@ -290,7 +290,12 @@ __global__ void __launch_bounds__(NT, 1) preproc_umma_kernel(const __grid_consta
 
   for (int i = 0; i < H1; ++i) {
     // the next head's copies go into the buffers head i - 1 used, which it has finished with
-    if (i + 1 < H1 && warp == 0 && elect_one_sync()) issue_loads(i + 1);
+    // (thread 0, which also issues the q stores and so owns their bulk groups: the buffer the next
+    // weights go into may still be read by the store of head i - 2's q, staged there)
+    if (i + 1 < H1 && threadIdx.x == 0) {
+      bulk_wait_read<0>();
+      issue_loads(i + 1);
+    }
     const int lb = lat_buf(i);
     const uint32_t lpar = i == 0 ? 0u : (uint32_t)(((i - 1) >> 1) & 1);
     if (!mbar_wait_bounded(lat_barrier(i), lpar, p.err, abort_flag, wait_site(kSitePreUmma, 1, 1))) goto done;
@@ -371,9 +376,11 @@ __global__ void __launch_bounds__(NT, 1) preproc_umma_kernel(const __grid_consta
     tc_fence_after();
 
     if (i > 0) {
-      // ---- query head i - 1: q = c_q + PRE (q~ + k~)/2 + POST (c_q + c_k)/2, RoPE, staged in s
-      // (the MMAs that read s have completed)
+      // ---- query head i - 1: q = c_q + PRE (q~ + k~)/2 + POST (c_q + c_k)/2, RoPE, staged in the
+      // weight buffer this head's MMAs have finished reading (free until the loads of head i + 2),
+      // so the next head's conv need not wait for the store
       const int qb = lb;
+      const int qstage = OFF_WB + (i & 1) * TILE;
 #pragma unroll 1
       for (int sub = 0; sub < 2; ++sub) {
         const int i0 = cg * 32 + sub * 16;  // pairs i0 .. i0 + 15: columns i and i + 64
@@ -426,7 +433,7 @@ __global__ void __launch_bounds__(NT, 1) preproc_umma_kernel(const __grid_consta
             uint32_t w4[4];
 #pragma unroll
             for (int e = 0; e < 4; ++e) w4[e] = pack_f16x2(v[h][8 * c8 + 2 * e], v[h][8 * c8 + 2 * e + 1]);
-            *reinterpret_cast<uint4*>(smem + OFF_SB + sw128(r, i0 + 64 * h + 8 * c8, HALF)) =
+            *reinterpret_cast<uint4*>(smem + qstage + sw128(r, i0 + 64 * h + 8 * c8, HALF)) =
                 make_uint4(w4[0], w4[1], w4[2], w4[3]);
           }
       }
@@ -435,14 +442,16 @@ __global__ void __launch_bounds__(NT, 1) preproc_umma_kernel(const __grid_consta
       __syncthreads();
       if (threadIdx.x == 0) {
         const int h = g * G + i - 1;
-        for (int hf = 0; hf < 2; ++hf) tma_store_3d(&maps.q, sbase + OFF_SB + hf * HALF, h * D + 64 * hf, t0, b);
+        for (int hf = 0; hf < 2; ++hf) tma_store_3d(&maps.q, sbase + qstage + hf * HALF, h * D + 64 * hf, t0, b);
         bulk_commit();
-        bulk_wait_read<0>();  // s is rewritten by the next head's conv
       }
       __syncthreads();
     }
   }
 
+  // the K head stages in s and weight buffer 0: the last q store must have read its buffer
+  if (threadIdx.x == 0) bulk_wait_read<0>();
+  __syncthreads();
   {  // (a block of its own: the waits above leave to `done` past its declarations)
   // value-shift sources, loaded now so that their latency overlaps the K head's combine: channels
   // [Lkv/2, Lkv) come from the previous token (0 at a sequence start); 8-channel vectors never
