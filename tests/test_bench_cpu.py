@@ -39,3 +39,13 @@ def test_warmup_floor():
     r = subprocess.run([sys.executable, "bench.py", "--warmup", "2"], cwd=ROOT, capture_output=True, text=True,
                        timeout=120)
     assert r.returncode != 0
+
+
+def test_clock_samples_directory(monkeypatch, tmp_path):
+    """The raw nvidia-smi samples go to $CCA_BENCH_CLOCKS_DIR when set, else the temp directory."""
+    import tempfile
+    import bench
+    monkeypatch.setenv("CCA_BENCH_CLOCKS_DIR", str(tmp_path))
+    assert bench.ClockSampler(1).path == str(tmp_path / "cca_bench_clocks_rank1.csv")
+    monkeypatch.delenv("CCA_BENCH_CLOCKS_DIR")
+    assert bench.ClockSampler(0).path.startswith(tempfile.gettempdir())
