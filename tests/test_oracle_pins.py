@@ -407,3 +407,107 @@ def test_decode_steps_chain_and_first_token():
     K, Lq, Lkv = 4, G * nkv * d, nkv * d
     out = oracle.decode_step(inp, inp["x"][0, 0], kc, vc, np.zeros((K - 1) * (Lq + Lkv) + Lkv), 0, G * nkv, nkv, d)
     np.testing.assert_allclose(out["y"], one["y"][0, 0], rtol=1e-11, atol=1e-12)
+
+
+# ------------------------------------------------------ step composition --
+# The pins above check each step alone; these fix how the block composes them
+# (es 2.B item 1: the sequence conv, then the channel mix within the head;
+# item 2: the QK-mean terms are taken on the latents before the convs and on
+# the channel-mix output after them; es section 3 item 2 and 2.C: the cache
+# holds k after RoPE). One sequence of 3 tokens, E = 2, one head of d = 2,
+# K = 2, W_q = W_v = W_o = I, W_k = 2 I, so q~ = v~ = x and k~ = 2 x. The seq
+# taps differ per channel (channel 0 reads only the previous token, channel 1
+# only the current one) and the channel mixes are a shear and a swap, so that
+# taking the two convs in the other order, or the mean on the seq-conv output,
+# changes the result. Every expected value below is worked out by hand.
+_COMP_X = [[1.0, 2.0], [3.0, 5.0], [7.0, 11.0]]
+# hand-worked, seq conv first: s_q = (x[t-1,0], x[t,1]) = (0,2) (1,5) (3,11);
+#   c_q = [[1,2],[0,1]] s_q = (s0 + 2 s1, s1)
+_COMP_CQ = [[4.0, 2.0], [11.0, 5.0], [25.0, 11.0]]
+# s_k = (2x[t-1,0], 2x[t,1]) = (0,4) (2,10) (6,22); c_k = swap(s_k)
+_COMP_CK = [[4.0, 0.0], [10.0, 2.0], [22.0, 6.0]]
+
+
+def _composition_inputs(S=3):
+    eye = np.eye(2)
+    return {
+        "x": np.array([_COMP_X[:S]]),
+        "W_q": eye.copy(), "W_k": 2.0 * eye, "W_v": eye.copy(), "W_o": eye.copy(),
+        "convq_seq": np.array([[1.0, 0.0], [0.0, 1.0]]),      # [channel, tap]; tap 1 = current token
+        "convk_seq": np.array([[1.0, 0.0], [0.0, 1.0]]),
+        "convq_chan": np.array([[[1.0, 2.0], [0.0, 1.0]]]),   # out_i = sum_j W[i][j] in_j
+        "convk_chan": np.array([[[0.0, 1.0], [1.0, 0.0]]]),
+    }
+
+
+def test_block_seq_conv_before_channel_mix():
+    """No QK-mean, RoPE or shift: q and the cached k are c_q and c_k of the hand-worked
+    sequence conv followed by the channel mix (the other order gives (5,2) (13,5) (29,11))."""
+    res = oracle.cca_block(_composition_inputs(), 1, 1, 2, qk_mean_mode=0, use_value_shift=False,
+                           use_rope=False)
+    np.testing.assert_array_equal(res["q"][0], _COMP_CQ)
+    np.testing.assert_array_equal(res["k_cache"][0].reshape(3, 2), _COMP_CK)
+
+
+def test_block_post_mean_on_channel_mix_output():
+    """POST only: q = c_q + (c_q + c_k)/2 and k = c_k + (c_q + c_k)/2, the mean taken on the
+    channel-mix outputs. With the seq-conv outputs instead, q[0] would be (4, 5)."""
+    res = oracle.cca_block(_composition_inputs(), 1, 1, 2, qk_mean_mode=2, use_value_shift=False,
+                           use_rope=False)
+    # c_q + c_k = (8,2) (21,7) (47,17)
+    np.testing.assert_array_equal(res["q"][0], [[8.0, 3.0], [21.5, 8.5], [48.5, 19.5]])
+    np.testing.assert_array_equal(res["k_cache"][0].reshape(3, 2), [[8.0, 1.0], [20.5, 5.5], [45.5, 14.5]])
+
+
+def test_block_pre_and_post_mean_together():
+    """PRE|POST: q = c_q + (q~ + k~)/2 + (c_q + c_k)/2 with q~ + k~ = 3x, the PRE term taken on
+    the latents before any conv."""
+    res = oracle.cca_block(_composition_inputs(), 1, 1, 2, qk_mean_mode=3, use_value_shift=False,
+                           use_rope=False)
+    # 1.5 x = (1.5,3) (4.5,7.5) (10.5,16.5)
+    np.testing.assert_array_equal(res["q"][0], [[9.5, 6.0], [26.0, 16.0], [59.0, 36.0]])
+    np.testing.assert_array_equal(res["k_cache"][0].reshape(3, 2), [[9.5, 4.0], [25.0, 13.0], [56.0, 31.0]])
+
+
+def test_block_cache_holds_k_after_rope_and_shifted_v():
+    """With RoPE (d = 2: theta_0 = 1, so token t turns by t radians) the cache holds the rotated
+    c_k; v keeps channel 0 of token t and takes channel 1 from token t-1 (zero at t = 0); y at
+    t = 0 is v[0] and at t = 1 a two-way softmax of the rotated q and k."""
+    res = oracle.cca_block(_composition_inputs(), 1, 1, 2, qk_mean_mode=0, use_value_shift=True,
+                           use_rope=True)
+
+    def rot(a, b, t):
+        return [a * math.cos(t) - b * math.sin(t), b * math.cos(t) + a * math.sin(t)]
+
+    kc = res["k_cache"][0].reshape(3, 2)
+    for t in range(3):
+        np.testing.assert_allclose(kc[t], rot(*_COMP_CK[t], t), rtol=0, atol=1e-13)
+    np.testing.assert_array_equal(res["v_cache"][0].reshape(3, 2), [[1.0, 0.0], [3.0, 2.0], [7.0, 5.0]])
+    y = res["y"][0]
+    np.testing.assert_allclose(y[0], [1.0, 0.0], atol=1e-15)
+    q1 = rot(*_COMP_CQ[1], 1)
+    k0, k1 = rot(*_COMP_CK[0], 0), rot(*_COMP_CK[1], 1)
+    s0 = (q1[0] * k0[0] + q1[1] * k0[1]) / math.sqrt(2.0)
+    s1 = (q1[0] * k1[0] + q1[1] * k1[1]) / math.sqrt(2.0)
+    p1 = 1.0 / (1.0 + math.exp(s0 - s1))
+    np.testing.assert_allclose(y[1], [(1 - p1) * 1.0 + p1 * 3.0, (1 - p1) * 0.0 + p1 * 2.0], rtol=1e-12)
+
+
+@pytest.mark.parametrize("mode,expect_q,expect_k", [
+    (0, [25.0, 11.0], [22.0, 6.0]),
+    (2, [48.5, 19.5], [45.5, 14.5]),
+    (3, [59.0, 36.0], [56.0, 31.0]),
+])
+def test_decode_step_composition_by_hand(mode, expect_q, expect_k):
+    """The decode step of token 2 from the state of tokens 0..1 (conv state: q~[1] = (3,5),
+    k~[1] = (6,10), v~[1] = (3,5)) gives the hand-worked row 2 above, without any prefill."""
+    inp = _composition_inputs()
+    state = np.array([3.0, 5.0, 6.0, 10.0, 3.0, 5.0])
+    kc = np.array([[[4.0, 0.0]], [[10.0, 2.0]]])   # any cache rows: only y depends on them
+    vc = np.array([[[1.0, 0.0]], [[3.0, 2.0]]])
+    out = oracle.decode_step(inp, np.array(_COMP_X[2]), kc, vc, state, 2, 1, 1, 2, qk_mean_mode=mode,
+                             use_value_shift=True, use_rope=False)
+    np.testing.assert_array_equal(out["q"], expect_q)
+    np.testing.assert_array_equal(out["k"].reshape(2), expect_k)
+    np.testing.assert_array_equal(out["v"].reshape(2), [7.0, 5.0])
+    np.testing.assert_array_equal(out["conv_state"], [7.0, 11.0, 14.0, 22.0, 7.0, 11.0])
