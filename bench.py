@@ -112,8 +112,11 @@ class ClockSampler:
               "clocks_event_reasons.hw_slowdown", "clocks_event_reasons.hw_thermal_slowdown",
               "clocks_event_reasons.sw_thermal_slowdown", "clocks_event_reasons.sw_power_cap"]
 
-    def __init__(self, index: int):
+    def __init__(self, index: int, device_id: str = None):
         self.index = index
+        # nvidia-smi numbers GPUs without regard to CUDA_VISIBLE_DEVICES, so the sampled GPU is named
+        # by the UUID of the CUDA device when it is known
+        self.device_id = device_id or str(index)
         self.proc = None
         # the raw samples: $CCA_BENCH_CLOCKS_DIR if set, else the system temporary directory
         d = os.environ.get("CCA_BENCH_CLOCKS_DIR") or tempfile.gettempdir()
@@ -124,7 +127,7 @@ class ClockSampler:
             os.makedirs(os.path.dirname(self.path), exist_ok=True)
             self.fh = open(self.path, "w")
             self.proc = subprocess.Popen(
-                ["nvidia-smi", f"--id={self.index}", "--query-gpu=" + ",".join(self.FIELDS),
+                ["nvidia-smi", f"--id={self.device_id}", "--query-gpu=" + ",".join(self.FIELDS),
                  "--format=csv,noheader,nounits", "-lms", "100"], stdout=self.fh, stderr=subprocess.DEVNULL)
         except Exception:
             self.proc = None
@@ -156,7 +159,18 @@ class ClockSampler:
         if not sm:
             return None
         return {"sm_mhz": statistics.median(sm), "sm_max_mhz": mx, "reasons": sorted(reasons),
-                "samples": len(sm)}
+                "samples": len(sm), "gpu": self.device_id}
+
+
+def cuda_device_uuid(dev) -> str:
+    """nvidia-smi's name for the CUDA device ("GPU-<uuid>"), or None if torch does not report it."""
+    try:
+        u = str(torch.cuda.get_device_properties(dev).uuid)
+    except Exception:
+        return None
+    if not u:
+        return None
+    return u if u.startswith("GPU-") else "GPU-" + u
 
 
 # ---------------------------------------------------------- oracle timing --
@@ -223,47 +237,62 @@ def cpu_baseline(shape, inputs, repeats=2):
             "sample_seconds": round(repeats * sum(t for _, t in pts), 2)}
 
 
+REF_MAX_ROWS = 16384  # query rows of one reference step; at S <= 16384 a step is the whole block
+
+
 def run_reference(args, shape):
+    """The oracle as the reference arm: every step (warm-up and timed) is one oracle call on the
+    same inputs. At S <= 16384 the call is the whole block, so `ms_per_step` is the block's time.
+    Longer sequences run every per-token stage over all S tokens and attention and the output
+    projection for 16384 evenly spaced query rows; the whole-block time is then extrapolated
+    linearly in rows from one more call of 2048 rows (made after the timed steps) and labelled."""
     rank = int(os.environ.get("RANK", "0"))
     if rank != 0:
         return 0
     inputs = workloads.make_inputs(shape)
     inp64 = workloads.as_float64(inputs)
-    samples = {r: [] for r in ROW_SAMPLES}
+    rows = spaced_rows(shape.seq_len, min(shape.seq_len, REF_MAX_ROWS))
+    full = len(rows) == shape.seq_len
+    times = []
     for i in range(args.warmup + args.steps):
-        r = ROW_SAMPLES[i % 2]
-        rows = spaced_rows(shape.seq_len, r)
-        t = oracle_call(shape, inp64, rows)
+        t = oracle_call(shape, inp64, None if full else rows)
         if i >= args.warmup:
-            samples[r].append(t)
-    if not samples[ROW_SAMPLES[1]]:  # a single timed step: take the other point from warm-up
-        rows = spaced_rows(shape.seq_len, ROW_SAMPLES[1])
-        samples[ROW_SAMPLES[1]].append(oracle_call(shape, inp64, rows))
-    if not samples[ROW_SAMPLES[0]]:
-        rows = spaced_rows(shape.seq_len, ROW_SAMPLES[0])
-        samples[ROW_SAMPLES[0]].append(oracle_call(shape, inp64, rows))
-    pts = [(len(spaced_rows(shape.seq_len, r)), statistics.mean(samples[r])) for r in ROW_SAMPLES]
-    t_full = oracle_extrapolate(pts, shape.seq_len)
+            times.append(t)
+    t_step = statistics.mean(times)
+    if full:
+        t_full = t_step
+        sample = (f"oracle (numpy float64) on the {shape.name} inputs: the whole block, all "
+                  f"{shape.tokens} tokens, every step")
+    else:
+        small = spaced_rows(shape.seq_len, ROW_SAMPLES[0])
+        t_small = oracle_call(shape, inp64, small)
+        t_full = oracle_extrapolate([(len(small), t_small), (len(rows), t_step)], shape.seq_len)
+        sample = (f"oracle (numpy float64) on the {shape.name} inputs: every per-token stage over all "
+                  f"{shape.tokens} tokens, attention and output projection for {len(rows)} evenly spaced query "
+                  f"rows per step; the whole-block time extrapolated linearly in rows (one more call of "
+                  f"{len(small)} rows)")
     value = shape.tokens / t_full
     cores = oracle_threads()
     line = {
         "impl": "reference", "metric": METRIC, "value": value, "unit": "tokens/s", "n_gpus": args.gpus,
-        "steps": args.steps, "warmup": args.warmup, "ms_per_step": t_full * 1e3, "higher_is_better": True,
+        "steps": args.steps, "warmup": args.warmup, "ms_per_step": t_step * 1e3, "higher_is_better": True,
         "scaling": "weak", "vs_baseline": None, "dtype": "f64", "data": "synthetic",
-        "config": config_dict(shape, "oracle"),
+        "config": config_dict(shape), "path": "oracle",
+        "full_block_ms": t_full * 1e3, "full_block_extrapolated": not full,
         "cpu_baseline": {"value": value, "unit": "tokens/s", "cores": cores, "kind": "oracle",
-                         "sample": oracle_sample_text(shape), "extrapolated": oracle_extrapolated(shape)},
+                         "sample": sample, "extrapolated": not full},
         "e2e": {"value": value, "unit": "tokens/s", "h2d_bytes_per_step": 0, "d2h_bytes_per_step": 0},
     }
     print(json.dumps(line), flush=True)
     return 0
 
 
-def config_dict(shape, path):
+def config_dict(shape):
+    """The workload, identical in both arms (the kernels that ran are the line's `path`)."""
     return {"workload": shape.name, "batch": shape.batch, "seq_len": shape.seq_len, "hidden": shape.hidden,
             "C": shape.compression, "n_q_heads": shape.n_q_heads, "n_kv_heads": shape.n_kv_heads,
             "head_dim": shape.head_dim, "conv_kernel": shape.conv_kernel, "qk_mean_mode": shape.qk_mean_mode,
-            "value_shift": shape.value_shift, "rope_base": shape.rope_base, "path": path,
+            "value_shift": shape.value_shift, "rope_base": shape.rope_base,
             "l2": "flushed between timed steps (256 MiB write)"}
 
 
@@ -303,27 +332,40 @@ def run_ours(args, shape):
         return float(t.item())
 
     # which kernels run (tcgen05 or SIMT per stage) and how many launches a step makes
-    plan = cca.plan(cfg)
+    path = PREPROC_PATHS[args.preproc]
+    plan = cca.plan(cfg, path)
+    if args.decode_only:
+        # one prefill writes the cache, then only the decode step is timed (profiling runs)
+        cca.prefill(cfg, inputs, out=out, workspace=ws, path=path)
+        torch.cuda.synchronize()
+        if rank == 0:
+            res = run_decode(cca, dev, my_shape, inputs, out, load_peaks()[0], steps=args.steps,
+                             warmup=args.warmup)
+            print(json.dumps({"mode": "decode-only", "workload": my_shape.name, "decode": res}, default=float),
+                  flush=True)
+        if world > 1:
+            dist.destroy_process_group()
+        return 0
     path_tensor = plan["attention_tensor"]
     launches_per_step = plan["launches"]
 
     for _ in range(args.warmup):
         flush.zero_()
-        cca.prefill(cfg, inputs, out=out, workspace=ws)
+        cca.prefill(cfg, inputs, out=out, workspace=ws, path=path)
     torch.cuda.synchronize()
     st = cca.poll_device_status()
     if st != 0:
         raise SystemExit(f"device status {st} after warm-up")
 
     evs = [[torch.cuda.Event(enable_timing=True) for _ in range(5)] for _ in range(args.steps)]
-    sampler = ClockSampler(local)
+    sampler = ClockSampler(local, cuda_device_uuid(dev))
     sampler.start()
     time.sleep(0.3)
     barrier()
     torch.cuda.synchronize()
     for i in range(args.steps):
         flush.zero_()
-        cca.prefill(cfg, inputs, out=out, workspace=ws, stage_events=evs[i])
+        cca.prefill(cfg, inputs, out=out, workspace=ws, stage_events=evs[i], path=path)
     torch.cuda.synchronize()
     barrier()
     clocks = sampler.stop()
@@ -371,7 +413,7 @@ def run_ours(args, shape):
             "metric": METRIC, "value": value, "unit": "tokens/s", "n_gpus": world, "steps": args.steps,
             "warmup": args.warmup, "ms_per_step": ms_per_step, "higher_is_better": True, "scaling": "weak",
             "vs_baseline": None, "dtype": "bf16", "data": "synthetic",
-            "config": config_dict(shape, plan_name(plan)),
+            "config": config_dict(shape), "path": plan_name(plan),
             "attention_tflops": attn_tflops,
             "roofline": roofline,
             "kernels": kernels,
@@ -574,8 +616,13 @@ def run_e2e(cca, cfg, args, inputs_cpu, inputs, out, ws, stream, shape, world, b
 def plan_name(plan):
     k = lambda b: "tcgen05" if b else "simt"  # noqa: E731
     return (f"down_proj={k(plan['down_proj_tensor'])},"
-            f"preproc={'mma' if plan['preproc_tensor'] else 'simt'},attention={k(plan['attention_tensor'])},"
+            f"preproc={plan['preproc_kind']},attention={k(plan['attention_tensor'])},"
             f"out_proj={k(plan['out_proj_tensor'])}")
+
+
+# --preproc: which preprocessing kernel the timed block runs (the other stages on their tensor-core
+# kernels where the shape allows them)
+PREPROC_PATHS = {"auto": 0, "mma": 0x100 | 1 | 2 | 4 | 8, "tcgen05": 0x100 | 1 | 2 | 4 | 16}
 
 
 def main(argv=None):
@@ -590,6 +637,10 @@ def main(argv=None):
     ap.add_argument("--no-mha", action="store_true",
                     help="skip timing the plain multi-head block of the same shape (the uncompressed baseline)")
     ap.add_argument("--no-decode", action="store_true", help="skip timing one decode step at position S - 1")
+    ap.add_argument("--decode-only", action="store_true",
+                    help="time only the decode step at position S - 1 after one prefill (profiling runs)")
+    ap.add_argument("--preproc", choices=sorted(PREPROC_PATHS), default="auto",
+                    help="preprocessing kernel of the timed block (auto: the library's choice)")
     ap.add_argument("--batch", type=int, default=None, help="override the workload's batch (profiling cases)")
     ap.add_argument("--seq-len", type=int, default=None, help="override the workload's sequence length")
     args = ap.parse_args(argv)

@@ -27,8 +27,9 @@ CCA_PATH_TENSOR = 2
 
 
 def CCA_PATH_TENSOR_MASK(bits: int) -> int:
-    """bit0 down-projection, bit1 attention, bit2 output projection, bit3 preprocessing."""
-    return 0x100 | (bits & 15)
+    """bit0 down-projection, bit1 attention, bit2 output projection, bit3 preprocessing (mma.sync),
+    bit4 preprocessing (tcgen05)."""
+    return 0x100 | (bits & 31)
 
 
 class CcaConfig(Structure):

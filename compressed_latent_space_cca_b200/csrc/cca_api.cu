@@ -149,7 +149,8 @@ bool aligned16(const void* p) { return (reinterpret_cast<uintptr_t>(p) & 15u) ==
 struct Resolved {
   BlockDims dm;
   bool tc_down, tc_attn, tc_out;  // tcgen05 kernels per stage
-  bool tc_pre;                    // tensor-core preprocessing kernel
+  bool tc_pre;                    // tensor-core preprocessing kernel (mma.sync form)
+  bool pre_umma;                  // tensor-core preprocessing kernel (tcgen05 form)
 };
 
 cca_status_t resolve(const cca_config_t* cfg, int path, Resolved* r) {
@@ -158,7 +159,7 @@ cca_status_t resolve(const cca_config_t* cfg, int path, Resolved* r) {
   DeviceInfo* di = nullptr;
   if ((st = device_info(&di)) != CCA_OK) return st;
   const BlockDims& dm = r->dm;
-  const bool masked = (path & ~15) == CCA_PATH_TENSOR_MASK(0);
+  const bool masked = (path & ~31) == CCA_PATH_TENSOR_MASK(0);
   if (path != CCA_PATH_AUTO && path != CCA_PATH_SIMT && path != CCA_PATH_TENSOR && !masked)
     return fail(CCA_ERR_INVALID_ARG, "unknown path");
   const bool sm100 = di->major == 10;
@@ -168,15 +169,20 @@ cca_status_t resolve(const cca_config_t* cfg, int path, Resolved* r) {
   const bool attn = sm100 && b16 && dm.d == 128 && attention_tc_supported(dm);
   const bool out = sm100 && b16 && gemm_tc_supported(dm.T, dm.E, dm.Lq);
   const bool pre = preproc_tc_supported(dm);
+  const bool umma = sm100 && preproc_umma_supported(dm);
   if (path == CCA_PATH_TENSOR && !(down && attn && out && (pre || dm.K == 0)))
     return fail(CCA_ERR_UNSUPPORTED, "tensor-core path needs sm_100, bf16, head_dim 128 and 128-aligned widths");
-  if (masked && (((path & 1) && !down) || ((path & 2) && !attn) || ((path & 4) && !out) || ((path & 8) && !pre)))
+  if (masked && (((path & 1) && !down) || ((path & 2) && !attn) || ((path & 4) && !out) || ((path & 8) && !pre) ||
+                 ((path & 16) && !umma)))
     return fail(CCA_ERR_UNSUPPORTED, "a stage asked for the tensor-core kernel cannot use it");
+  if (masked && (path & 8) && (path & 16))
+    return fail(CCA_ERR_INVALID_ARG, "path bits 3 and 4 both choose the preprocessing kernel");
   const bool use = path != CCA_PATH_SIMT;
   r->tc_down = masked ? (path & 1) != 0 : use && down;
   r->tc_attn = masked ? (path & 2) != 0 : use && attn;
   r->tc_out = masked ? (path & 4) != 0 : use && out;
   r->tc_pre = masked ? (path & 8) != 0 : use && pre;
+  r->pre_umma = masked && (path & 16) != 0;
   return CCA_OK;
 }
 
@@ -214,7 +220,7 @@ cca_status_t run_block(const Resolved& r, BlockPtrs p, cudaStream_t stream, void
     a.in = dm.io;
     a.out = dm.lat;
     a.dev_err = p.dev_err;
-    if (r.tc_pre) {  // the fp16 channel-conv weights of the preprocessing kernel, made on the side
+    if (r.tc_pre || r.pre_umma) {  // the fp16 channel-conv weights of the preprocessing kernel, made on the side
       const long long nc = (long long)dm.d * dm.d;
       a.side_src[0] = p.cq_chan;
       a.side_dst[0] = p.wc_lat;
@@ -235,7 +241,7 @@ cca_status_t run_block(const Resolved& r, BlockPtrs p, cudaStream_t stream, void
         return cuda_fail("down-projection (SIMT)", e);
       col += ns[i];
     }
-    if (r.tc_pre) {
+    if (r.tc_pre || r.pre_umma) {
       const long long nc = (long long)dm.d * dm.d;
       if ((e = launch_convert_f16(p.cq_chan, p.wc_lat, nc * dm.nq, p.dev_err, stream)) != cudaSuccess ||
           (e = launch_convert_f16(p.ck_chan, static_cast<char*>(p.wc_lat) + nc * dm.nq * eb, nc * dm.nkv, p.dev_err,
@@ -247,6 +253,8 @@ cca_status_t run_block(const Resolved& r, BlockPtrs p, cudaStream_t stream, void
   // 2. seq conv, channel conv, QK-mean, RoPE, value shift; KV cache written here
   if (dm.K == 0) {
     if ((e = launch_plain_preproc(dm, p, stream)) != cudaSuccess) return cuda_fail("RoPE and KV cache (plain)", e);
+  } else if (r.pre_umma) {
+    if ((e = launch_preproc_umma(dm, p, stream)) != cudaSuccess) return cuda_fail("preprocessing (tcgen05)", e);
   } else if (r.tc_pre) {
     if ((e = launch_preproc_tc(dm, p, stream)) != cudaSuccess) return cuda_fail("preprocessing (mma)", e);
   } else {
@@ -431,10 +439,10 @@ cca_status_t cca_plan(const cca_config_t* cfg, int path, cca_plan_t* out) {
   out->down_proj_tensor = r.tc_down;
   out->attention_tensor = r.tc_attn;
   out->out_proj_tensor = r.tc_out;
-  out->preproc_tensor = r.tc_pre;
+  out->preproc_tensor = r.pre_umma ? 2 : (r.tc_pre ? 1 : 0);
   // down-projection (one tcgen05 GEMM, or three SIMT GEMMs plus the two fp16 weight copies that the
   // tcgen05 GEMM otherwise makes on the side), preprocessing, attention, output projection
-  out->launches = (r.tc_down ? 1 : 3 + (r.tc_pre ? 2 : 0)) + 1 + 1 + 1;
+  out->launches = (r.tc_down ? 1 : 3 + (r.tc_pre || r.pre_umma ? 2 : 0)) + 1 + 1 + 1;
   return CCA_OK;
 }
 

@@ -64,7 +64,7 @@ cudaError_t launch_plain_preproc(const BlockDims& dm, const BlockPtrs& p, cudaSt
 // bf16 blocks with head_dim 128: channel mix on the tensor cores (mma.sync), coalesced I/O
 bool preproc_tc_supported(const BlockDims& dm);
 // The same steps with the channel mix on tcgen05 (128-token tiles, operands in tensor memory);
-// needs the fp16 W_c copy (wc_lat). Built and compiled; not yet selected by cca_prefill.
+// needs the fp16 W_c copy (wc_lat). Selected by bit 4 of the path mask.
 bool preproc_umma_supported(const BlockDims& dm);
 cudaError_t launch_preproc_umma(const BlockDims& dm, const BlockPtrs& p, cudaStream_t stream);
 cudaError_t launch_preproc_tc(const BlockDims& dm, const BlockPtrs& p, cudaStream_t stream);

@@ -12,7 +12,10 @@
 //
 // Limits and sharing: the array holds CCA_NOALLOC_WORKSPACE_BYTES (64 MiB);
 // every GPU on which this entry point runs keeps that much memory until the
-// process exits. Larger blocks are rejected with CCA_ERR_WORKSPACE. All calls
+// process exits. That holds under lazy module loading (CUDA_MODULE_LOADING=LAZY,
+// the default of recent CUDA runtimes); with CUDA_MODULE_LOADING=EAGER every
+// device on which the library is loaded reserves the 64 MiB, used or not.
+// Larger blocks are rejected with CCA_ERR_WORKSPACE. All calls
 // share the one array: two calls whose work overlaps on the GPU (different
 // streams, or different host threads on the same device) race on it, so they
 // must be ordered by the caller. No part of the workspace has to start at

@@ -98,16 +98,18 @@ typedef enum cca_path {
   CCA_PATH_TENSOR = 2   /* CCA_ERR_UNSUPPORTED if the shape does not allow it */
 } cca_path_t;
 /* Per-stage choice: bit0 down-projection, bit1 attention, bit2 output
- * projection, bit3 preprocessing on the tensor-core kernel, the other stages
- * on SIMT. */
-#define CCA_PATH_TENSOR_MASK(bits) (0x100 | ((bits) & 15))
+ * projection, bit3 preprocessing on the tensor-core kernel (channel mix on
+ * mma.sync), bit4 preprocessing on the tcgen05 kernel (channel mix as
+ * tcgen05 MMAs into tensor memory; bits 3 and 4 exclude each other); the other
+ * stages on SIMT. */
+#define CCA_PATH_TENSOR_MASK(bits) (0x100 | ((bits) & 31))
 
 /* Which kernels a call would launch (cca_plan). */
 typedef struct cca_plan {
   int down_proj_tensor;   /* 1: tcgen05 GEMM, 0: SIMT GEMM (three launches) */
   int attention_tensor;   /* 1: tcgen05 flash attention, 0: SIMT attention */
   int out_proj_tensor;    /* 1: tcgen05 GEMM, 0: SIMT GEMM */
-  int preproc_tensor;     /* 1: preprocessing with the channel mix on tensor cores (mma.sync) */
+  int preproc_tensor;     /* 1: preprocessing with the channel mix on mma.sync, 2: on tcgen05 */
   int launches;           /* kernel launches of one cca_prefill without conv_state */
 } cca_plan_t;
 
@@ -230,7 +232,9 @@ cca_status_t cca_prefill_host(const cca_config_t* cfg,
  *
  * The intermediates go to a fixed 256-byte-aligned device array inside the
  * library of CCA_NOALLOC_WORKSPACE_BYTES; every GPU on which this is called
- * keeps that memory until the process exits. Blocks whose
+ * keeps that memory until the process exits (under lazy module loading, the
+ * default of recent CUDA runtimes; with CUDA_MODULE_LOADING=EAGER every GPU on
+ * which the library is loaded reserves it, whether or not this is called). Blocks whose
  * cca_workspace_size() exceeds it are rejected with CCA_ERR_WORKSPACE (e.g.
  * B=1, S=8192, E=2048, 4 query / 2 KV heads of 128 needs 44 MB and fits;
  * S=16384 does not). The first call on a device looks up the array's device

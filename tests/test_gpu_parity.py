@@ -11,6 +11,10 @@ from parity import assert_close, run_gpu, run_oracle, sample_rows
 pytestmark = pytest.mark.gpu
 
 SIMT, AUTO, TENSOR = cca.CCA_PATH_SIMT, cca.CCA_PATH_AUTO, cca.CCA_PATH_TENSOR
+# every stage on its tensor-core kernel, the preprocessing on the tcgen05 form
+UMMA = cca.CCA_PATH_TENSOR_MASK(1 | 2 | 4 | 16)
+PATHS = [SIMT, AUTO, TENSOR, UMMA]
+PATH_IDS = ["simt", "auto", "tensor", "umma"]
 
 
 def shape(**kw):
@@ -67,7 +71,7 @@ BF16_CASES = [
 ]
 
 
-@pytest.mark.parametrize("path", [SIMT, AUTO, TENSOR], ids=["simt", "auto", "tensor"])
+@pytest.mark.parametrize("path", PATHS, ids=PATH_IDS)
 @pytest.mark.parametrize("case", range(len(BF16_CASES)))
 def test_bf16_small(path, case):
     sh = shape(**BF16_CASES[case])
@@ -119,7 +123,7 @@ def test_plain_block_fp32():
     check_all(sh, run_gpu(sh, inp), run_oracle(one, oi))
 
 
-@pytest.mark.parametrize("path", [SIMT, AUTO, TENSOR], ids=["simt", "auto", "tensor"])
+@pytest.mark.parametrize("path", PATHS, ids=PATH_IDS)
 @pytest.mark.parametrize("mode,vshift,rope", [(0, 0, 0), (1, 0, 1), (2, 1, 0), (3, 1, 1), (0, 1, 1)])
 def test_bf16_modes(path, mode, vshift, rope):
     sh = shape(seq_len=257, qk_mean_mode=mode, value_shift=vshift, use_rope=rope, batch=2)
@@ -127,7 +131,7 @@ def test_bf16_modes(path, mode, vshift, rope):
     check_all(sh, run_gpu(sh, inp, path=path), run_oracle(sh, inp))
 
 
-@pytest.mark.parametrize("path", [SIMT, AUTO, TENSOR], ids=["simt", "auto", "tensor"])
+@pytest.mark.parametrize("path", PATHS, ids=PATH_IDS)
 def test_fp32_output_and_conv_state(path):
     sh = shape(seq_len=190, batch=2)
     inp = workloads.make_inputs(sh)
@@ -148,7 +152,7 @@ def test_fp32_output_and_conv_state(path):
     np.testing.assert_array_equal(cs[:, :nq_part].reshape(2, K - 1, lq), lat)
 
 
-@pytest.mark.parametrize("path", [SIMT, AUTO, TENSOR], ids=["simt", "auto", "tensor"])
+@pytest.mark.parametrize("path", PATHS, ids=PATH_IDS)
 def test_deterministic_and_causal(path):
     """Three runs are bit-identical; perturbing x[t0] leaves every output row
     before t0 bit-identical (nothing reads the future)."""
@@ -171,7 +175,7 @@ def test_deterministic_and_causal(path):
         assert not np.array_equal(c[k][1, t0], a[k][1, t0]), k
 
 
-@pytest.mark.parametrize("path", [AUTO, TENSOR], ids=["auto", "tensor"])
+@pytest.mark.parametrize("path", [AUTO, TENSOR, UMMA], ids=["auto", "tensor", "umma"])
 def test_bf16_long_ragged(path):
     """S = 4097: 33 query tiles whose last holds one row, two sequences, the split
     schedule of a long sequence; caches in full, y and O on sampled rows."""
@@ -187,15 +191,16 @@ def test_bf16_long_ragged(path):
 
 
 # ------------------------------------------------- the five named workloads --
+@pytest.mark.parametrize("path", [AUTO, UMMA], ids=["auto", "umma"])
 @pytest.mark.parametrize("name", ["cca_dense_bf16", "ccgqa_16k_bf16", "ccgqa_8x_bf16", "ccgqa_64k_bf16"])
-def test_named_workload_full_size(name):
-    """Full-size run in the bench's launch configuration (auto path); the
-    KV cache is compared in full, y and the attention output on sampled rows
+def test_named_workload_full_size(name, path):
+    """Full-size run in the bench's launch configuration (auto path) and with the tcgen05
+    preprocessing; the KV cache is compared in full, y and the attention output on sampled rows
     the oracle computes one by one."""
     sh = workloads.WORKLOADS[name]
     inp = workloads.make_inputs(sh)
     rows = sample_rows(sh.seq_len, 40, seed=sh.seed)
-    gpu = run_gpu(sh, inp, rows=rows, stages=False)
+    gpu = run_gpu(sh, inp, rows=rows, stages=False, path=path)
     ref = run_oracle(sh, inp, rows=rows)
     assert_close("k_cache", gpu["k_cache"], ref["k_cache"], "bf16")
     assert_close("v_cache", gpu["v_cache"], ref["v_cache"], "bf16")
