@@ -150,7 +150,7 @@ struct Resolved {
   BlockDims dm;
   bool tc_down, tc_attn, tc_out;  // tcgen05 kernels per stage
   bool tc_pre;                    // tensor-core preprocessing kernel (mma.sync form)
-  bool pre_umma;                  // tensor-core preprocessing kernel (tcgen05 form)
+  bool pre_ws;                    // tensor-core preprocessing kernel (warp-specialised tcgen05 form)
 };
 
 cca_status_t resolve(const cca_config_t* cfg, int path, Resolved* r) {
@@ -169,11 +169,11 @@ cca_status_t resolve(const cca_config_t* cfg, int path, Resolved* r) {
   const bool attn = sm100 && b16 && dm.d == 128 && attention_tc_supported(dm);
   const bool out = sm100 && b16 && gemm_tc_supported(dm.T, dm.E, dm.Lq);
   const bool pre = preproc_tc_supported(dm);
-  const bool umma = sm100 && preproc_umma_supported(dm);
+  const bool ws = sm100 && preproc_ws_supported(dm);
   if (path == CCA_PATH_TENSOR && !(down && attn && out && (pre || dm.K == 0)))
     return fail(CCA_ERR_UNSUPPORTED, "tensor-core path needs sm_100, bf16, head_dim 128 and 128-aligned widths");
   if (masked && (((path & 1) && !down) || ((path & 2) && !attn) || ((path & 4) && !out) || ((path & 8) && !pre) ||
-                 ((path & 16) && !umma)))
+                 ((path & 16) && !ws)))
     return fail(CCA_ERR_UNSUPPORTED, "a stage asked for the tensor-core kernel cannot use it");
   if (masked && (path & 8) && (path & 16))
     return fail(CCA_ERR_INVALID_ARG, "path bits 3 and 4 both choose the preprocessing kernel");
@@ -181,8 +181,10 @@ cca_status_t resolve(const cca_config_t* cfg, int path, Resolved* r) {
   r->tc_down = masked ? (path & 1) != 0 : use && down;
   r->tc_attn = masked ? (path & 2) != 0 : use && attn;
   r->tc_out = masked ? (path & 4) != 0 : use && out;
-  r->tc_pre = masked ? (path & 8) != 0 : use && pre;
-  r->pre_umma = masked && (path & 16) != 0;
+  // AUTO takes the warp-specialised tcgen05 preprocessing where it applies (the QK-mean includes the
+  // after-conv term), else the mma.sync kernel; TENSOR keeps the mma.sync kernel
+  r->pre_ws = masked ? (path & 16) != 0 : (path == CCA_PATH_AUTO && ws);
+  r->tc_pre = masked ? (path & 8) != 0 : use && pre && !r->pre_ws;
   return CCA_OK;
 }
 
@@ -220,8 +222,9 @@ cca_status_t run_block(const Resolved& r, BlockPtrs p, cudaStream_t stream, void
     a.in = dm.io;
     a.out = dm.lat;
     a.dev_err = p.dev_err;
-    if (r.tc_pre || r.pre_umma) {  // the fp16 channel-conv weights of the preprocessing kernel, made on the side
+    if (r.tc_pre || r.pre_ws) {  // the fp16 channel-conv weights of the preprocessing kernel, made on the side
       const long long nc = (long long)dm.d * dm.d;
+      a.side_scale = r.pre_ws ? kWsWeightScale : 1.0f;
       a.side_src[0] = p.cq_chan;
       a.side_dst[0] = p.wc_lat;
       a.side_n[0] = nc * dm.nq;
@@ -241,11 +244,12 @@ cca_status_t run_block(const Resolved& r, BlockPtrs p, cudaStream_t stream, void
         return cuda_fail("down-projection (SIMT)", e);
       col += ns[i];
     }
-    if (r.tc_pre || r.pre_umma) {
+    if (r.tc_pre || r.pre_ws) {
       const long long nc = (long long)dm.d * dm.d;
-      if ((e = launch_convert_f16(p.cq_chan, p.wc_lat, nc * dm.nq, p.dev_err, stream)) != cudaSuccess ||
+      const float sc = r.pre_ws ? kWsWeightScale : 1.0f;
+      if ((e = launch_convert_f16(p.cq_chan, p.wc_lat, nc * dm.nq, p.dev_err, stream, sc)) != cudaSuccess ||
           (e = launch_convert_f16(p.ck_chan, static_cast<char*>(p.wc_lat) + nc * dm.nq * eb, nc * dm.nkv, p.dev_err,
-                                  stream)) != cudaSuccess)
+                                  stream, sc)) != cudaSuccess)
         return cuda_fail("channel-conv weight copy", e);
     }
   }
@@ -253,8 +257,8 @@ cca_status_t run_block(const Resolved& r, BlockPtrs p, cudaStream_t stream, void
   // 2. seq conv, channel conv, QK-mean, RoPE, value shift; KV cache written here
   if (dm.K == 0) {
     if ((e = launch_plain_preproc(dm, p, stream)) != cudaSuccess) return cuda_fail("RoPE and KV cache (plain)", e);
-  } else if (r.pre_umma) {
-    if ((e = launch_preproc_umma(dm, p, stream)) != cudaSuccess) return cuda_fail("preprocessing (tcgen05)", e);
+  } else if (r.pre_ws) {
+    if ((e = launch_preproc_ws(dm, p, stream)) != cudaSuccess) return cuda_fail("preprocessing (tcgen05)", e);
   } else if (r.tc_pre) {
     if ((e = launch_preproc_tc(dm, p, stream)) != cudaSuccess) return cuda_fail("preprocessing (mma)", e);
   } else {
@@ -439,10 +443,10 @@ cca_status_t cca_plan(const cca_config_t* cfg, int path, cca_plan_t* out) {
   out->down_proj_tensor = r.tc_down;
   out->attention_tensor = r.tc_attn;
   out->out_proj_tensor = r.tc_out;
-  out->preproc_tensor = r.pre_umma ? 2 : (r.tc_pre ? 1 : 0);
+  out->preproc_tensor = r.pre_ws ? 2 : (r.tc_pre ? 1 : 0);
   // down-projection (one tcgen05 GEMM, or three SIMT GEMMs plus the two fp16 weight copies that the
   // tcgen05 GEMM otherwise makes on the side), preprocessing, attention, output projection
-  out->launches = (r.tc_down ? 1 : 3 + (r.tc_pre || r.pre_umma ? 2 : 0)) + 1 + 1 + 1;
+  out->launches = (r.tc_down ? 1 : 3 + (r.tc_pre || r.pre_ws ? 2 : 0)) + 1 + 1 + 1;
   return CCA_OK;
 }
 
@@ -563,10 +567,10 @@ cca_status_t cca_poll_device_status(void* stream) {
       return cuda_fail("clear device error word", e);
     if ((h & 0xffu) == kDevErrRange)
       return fail(CCA_ERR_NUMERIC_RANGE, "an intermediate exceeded the fp16 range (|value| > 65504)");
-    static const char* kernels[4] = {"?", "gemm", "attention", "self-test"};
+    static const char* kernels[6] = {"?", "gemm", "attention", "self-test", "?", "preprocessing (tcgen05)"};
     char msg[160];
     snprintf(msg, sizeof(msg), "a bounded device-side wait gave up (kernel %s, role %u, barrier %u)",
-             kernels[((h >> 8) & 0xffu) < 4 ? ((h >> 8) & 0xffu) : 0], (h >> 16) & 0xffu, (h >> 24) & 0xffu);
+             kernels[((h >> 8) & 0xffu) < 6 ? ((h >> 8) & 0xffu) : 0], (h >> 16) & 0xffu, (h >> 24) & 0xffu);
     return fail(CCA_ERR_DEVICE_TIMEOUT, msg);
   }
   return CCA_OK;

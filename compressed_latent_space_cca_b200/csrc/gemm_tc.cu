@@ -90,6 +90,7 @@ struct GemmParams {
   const __nv_bfloat16* side_src[2];
   __half* side_dst[2];
   long long side_n[2];
+  float side_scale;
 };
 
 // Stores 32 fp32 accumulators of one row; returns true if an fp16 output overflowed.
@@ -292,8 +293,9 @@ __global__ void __launch_bounds__(Shape<MH, PAIR>::NUM_THREADS, 1)
 #pragma unroll
         for (int k = 0; k < 4; ++k) {
           const float2 f = __bfloat1622float2(b2[k]);
-          bad |= f16_overflow(f.x) || f16_overflow(f.y);
-          h[k] = pack_f16x2(f.x, f.y);
+          const float fx = f.x * p.side_scale, fy = f.y * p.side_scale;
+          bad |= f16_overflow(fx) || f16_overflow(fy);
+          h[k] = pack_f16x2(fx, fy);
         }
         *reinterpret_cast<uint4*>(p.side_dst[i] + e * 8) = make_uint4(h[0], h[1], h[2], h[3]);
       }
@@ -479,6 +481,7 @@ cudaError_t launch_gemm_tc(const GemmTcArgs& a, cudaStream_t stream) {
     p.side_dst[i] = static_cast<__half*>(a.side_dst[i]);
     p.side_n[i] = a.side_n[i] > 0 ? a.side_n[i] : 0;
   }
+  p.side_scale = a.side_scale != 0.f ? a.side_scale : 1.f;
   // 256-row tiles keep direct stores: their single accumulator leaves nothing to overlap the wait
   // for a staging buffer with, while direct stores retire without waiting
   // Pairs whenever a 256-row tile has rows to fill (on this workload's projections: 37.0 -> 34.9 us

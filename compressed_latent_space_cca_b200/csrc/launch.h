@@ -63,10 +63,12 @@ cudaError_t launch_conv_state(const BlockDims& dm, const BlockPtrs& p, cudaStrea
 cudaError_t launch_plain_preproc(const BlockDims& dm, const BlockPtrs& p, cudaStream_t stream);
 // bf16 blocks with head_dim 128: channel mix on the tensor cores (mma.sync), coalesced I/O
 bool preproc_tc_supported(const BlockDims& dm);
-// The same steps with the channel mix on tcgen05 (128-token tiles, operands in tensor memory);
-// needs the fp16 W_c copy (wc_lat). Selected by bit 4 of the path mask.
-bool preproc_umma_supported(const BlockDims& dm);
-cudaError_t launch_preproc_umma(const BlockDims& dm, const BlockPtrs& p, cudaStream_t stream);
+// The same steps as a persistent warp-specialised tcgen05 kernel (128-token tiles, every QK-mean and
+// channel-mix term accumulated in tensor memory); needs the after-conv QK-mean and the fp16 W_c copy
+// (wc_lat) scaled by kWsWeightScale.
+constexpr float kWsWeightScale = 1.5f;
+bool preproc_ws_supported(const BlockDims& dm);
+cudaError_t launch_preproc_ws(const BlockDims& dm, const BlockPtrs& p, cudaStream_t stream);
 cudaError_t launch_preproc_tc(const BlockDims& dm, const BlockPtrs& p, cudaStream_t stream);
 
 // ---- tensor-core path (16-bit operands, sm_100a) ----
@@ -86,14 +88,17 @@ struct GemmTcArgs {
   DType in, out;
   unsigned* dev_err;
   // optional side job of the epilogue warps before their first tile: side_dst[i][0, side_n[i]) =
-  // fp16 copy of the bf16 side_src[i] (fp16 overflow reported as a range error)
+  // fp16 copy of the bf16 side_src[i] times side_scale (0 means 1; fp16 overflow reported as a range
+  // error)
   const void* side_src[2];
   void* side_dst[2];
   long long side_n[2];
+  float side_scale;
 };
 cudaError_t launch_gemm_tc(const GemmTcArgs& a, cudaStream_t stream);
-// dst[0, n) = fp16 copy of the bf16 src (fp16 overflow reported as a range error)
-cudaError_t launch_convert_f16(const void* src, void* dst, long long n, unsigned* dev_err, cudaStream_t stream);
+// dst[0, n) = fp16 copy of the bf16 src times scale (fp16 overflow reported as a range error)
+cudaError_t launch_convert_f16(const void* src, void* dst, long long n, unsigned* dev_err, cudaStream_t stream,
+                               float scale = 1.0f);
 
 bool attention_tc_supported(const BlockDims& dm);
 cudaError_t launch_attention_tc(const BlockDims& dm, const void* q, const void* k, const void* v, void* o,

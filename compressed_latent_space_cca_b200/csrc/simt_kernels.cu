@@ -229,10 +229,10 @@ cudaError_t launch_attention_simt(const BlockDims& dm, const void* q, const void
 
 namespace {
 __global__ void __launch_bounds__(256) convert_f16_kernel(const __nv_bfloat16* __restrict__ src, __half* __restrict__ dst,
-                                                          long long n, unsigned* err) {
+                                                          long long n, unsigned* err, float scale) {
   bool bad = false;
   for (long long i = (long long)blockIdx.x * blockDim.x + threadIdx.x; i < n; i += (long long)gridDim.x * blockDim.x) {
-    const float f = __bfloat162float(src[i]);
+    const float f = __bfloat162float(src[i]) * scale;
     bad |= f16_overflow(f);
     dst[i] = __float2half_rn(f);
   }
@@ -240,12 +240,13 @@ __global__ void __launch_bounds__(256) convert_f16_kernel(const __nv_bfloat16* _
 }
 }  // namespace
 
-cudaError_t launch_convert_f16(const void* src, void* dst, long long n, unsigned* dev_err, cudaStream_t stream) {
+cudaError_t launch_convert_f16(const void* src, void* dst, long long n, unsigned* dev_err, cudaStream_t stream,
+                               float scale) {
   if (n <= 0) return cudaSuccess;
   long long blocks = (n + 255) / 256;
   if (blocks > 1184) blocks = 1184;
   convert_f16_kernel<<<(unsigned)blocks, 256, 0, stream>>>(static_cast<const __nv_bfloat16*>(src),
-                                                             static_cast<__half*>(dst), n, dev_err);
+                                                             static_cast<__half*>(dst), n, dev_err, scale);
   return cudaGetLastError();
 }
 

@@ -90,8 +90,10 @@ typedef struct cca_config {
 /* Kernel path selection (cca_prefill_ex). AUTO runs each stage on its
  * tensor-core kernel (tcgen05/TMEM fed by TMA, sm_100 only) when that kernel
  * takes the shape (bf16; head_dim 128 for attention and preprocessing) and on
- * its SIMT kernel otherwise. SIMT forces every stage onto the SIMT kernels;
- * TENSOR requires the tensor-core kernels for every stage. */
+ * its SIMT kernel otherwise; its preprocessing is the tcgen05 kernel when the
+ * QK-mean includes the after-conv term (CCA_QK_MEAN_POST) and the mma.sync
+ * kernel otherwise. SIMT forces every stage onto the SIMT kernels; TENSOR
+ * requires the tensor-core kernels for every stage (preprocessing: mma.sync). */
 typedef enum cca_path {
   CCA_PATH_AUTO = 0,
   CCA_PATH_SIMT = 1,

@@ -11,10 +11,10 @@ from parity import assert_close, run_gpu, run_oracle, sample_rows
 pytestmark = pytest.mark.gpu
 
 SIMT, AUTO, TENSOR = cca.CCA_PATH_SIMT, cca.CCA_PATH_AUTO, cca.CCA_PATH_TENSOR
-# every stage on its tensor-core kernel, the preprocessing on the tcgen05 form
-UMMA = cca.CCA_PATH_TENSOR_MASK(1 | 2 | 4 | 16)
-PATHS = [SIMT, AUTO, TENSOR, UMMA]
-PATH_IDS = ["simt", "auto", "tensor", "umma"]
+# every stage on its tensor-core kernel, the preprocessing on the warp-specialised tcgen05 kernel
+WS = cca.CCA_PATH_TENSOR_MASK(1 | 2 | 4 | 16)
+PATHS = [SIMT, AUTO, TENSOR, WS]
+PATH_IDS = ["simt", "auto", "tensor", "tcgen05pre"]
 
 
 def shape(**kw):
@@ -128,6 +128,12 @@ def test_plain_block_fp32():
 def test_bf16_modes(path, mode, vshift, rope):
     sh = shape(seq_len=257, qk_mean_mode=mode, value_shift=vshift, use_rope=rope, batch=2)
     inp = workloads.make_inputs(sh)
+    if path == WS and not mode & 2:
+        # the tcgen05 preprocessing folds the after-conv mean into its MMAs: without it, it declines
+        with pytest.raises(cca.CcaError) as ei:
+            run_gpu(sh, inp, path=path)
+        assert ei.value.status == cca.CCA_ERR_UNSUPPORTED
+        return
     check_all(sh, run_gpu(sh, inp, path=path), run_oracle(sh, inp))
 
 
@@ -175,7 +181,7 @@ def test_deterministic_and_causal(path):
         assert not np.array_equal(c[k][1, t0], a[k][1, t0]), k
 
 
-@pytest.mark.parametrize("path", [AUTO, TENSOR, UMMA], ids=["auto", "tensor", "umma"])
+@pytest.mark.parametrize("path", [AUTO, TENSOR, WS], ids=["auto", "tensor", "tcgen05pre"])
 def test_bf16_long_ragged(path):
     """S = 4097: 33 query tiles whose last holds one row, two sequences, the split
     schedule of a long sequence; caches in full, y and O on sampled rows."""
@@ -191,7 +197,7 @@ def test_bf16_long_ragged(path):
 
 
 # ------------------------------------------------- the five named workloads --
-@pytest.mark.parametrize("path", [AUTO, UMMA], ids=["auto", "umma"])
+@pytest.mark.parametrize("path", [AUTO, WS], ids=["auto", "tcgen05pre"])
 @pytest.mark.parametrize("name", ["cca_dense_bf16", "ccgqa_16k_bf16", "ccgqa_8x_bf16", "ccgqa_64k_bf16"])
 def test_named_workload_full_size(name, path):
     """Full-size run in the bench's launch configuration (auto path) and with the tcgen05
