@@ -617,12 +617,14 @@ def plan_name(plan):
     k = lambda b: "tcgen05" if b else "simt"  # noqa: E731
     return (f"down_proj={k(plan['down_proj_tensor'])},"
             f"preproc={plan['preproc_kind']},attention={k(plan['attention_tensor'])},"
-            f"out_proj={k(plan['out_proj_tensor'])}")
+            f"out_proj={k(plan['out_proj_tensor'])}" + (",value_shift=down_proj_epilogue" if plan.get("value_shift_fused")
+                                                          else ""))
 
 
 # --preproc: which preprocessing kernel the timed block runs (the other stages on their tensor-core
 # kernels where the shape allows them)
-PREPROC_PATHS = {"auto": 0, "mma": 0x100 | 1 | 2 | 4 | 8, "tcgen05": 0x100 | 1 | 2 | 4 | 16}
+PREPROC_PATHS = {"auto": 0, "mma": 0x100 | 1 | 2 | 4 | 8, "tcgen05": 0x100 | 1 | 2 | 4 | 16,
+                 "tcgen05+vshift": 0x100 | 1 | 2 | 4 | 16 | 32}
 
 
 def main(argv=None):

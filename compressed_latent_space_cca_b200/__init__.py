@@ -98,7 +98,8 @@ def plan(cfg: CcaConfig, path: int = CCA_PATH_AUTO) -> dict:
         raise CcaError(st, "cca_plan")
     return {"down_proj_tensor": bool(out.down_proj_tensor), "attention_tensor": bool(out.attention_tensor),
             "out_proj_tensor": bool(out.out_proj_tensor), "preproc_tensor": bool(out.preproc_tensor),
-            "preproc_kind": {0: "simt", 1: "mma", 2: "tcgen05"}[out.preproc_tensor], "launches": out.launches}
+            "preproc_kind": {0: "simt", 1: "mma", 2: "tcgen05"}[out.preproc_tensor], "launches": out.launches,
+            "value_shift_fused": bool(out.value_shift_fused)}
 
 
 def _shapes(cfg: CcaConfig) -> Dict[str, tuple]:

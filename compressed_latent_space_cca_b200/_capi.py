@@ -28,8 +28,8 @@ CCA_PATH_TENSOR = 2
 
 def CCA_PATH_TENSOR_MASK(bits: int) -> int:
     """bit0 down-projection, bit1 attention, bit2 output projection, bit3 preprocessing (mma.sync),
-    bit4 preprocessing (tcgen05)."""
-    return 0x100 | (bits & 31)
+    bit4 preprocessing (tcgen05), bit5 value shift in the down-projection (with bits 0 and 4)."""
+    return 0x100 | (bits & 63)
 
 
 class CcaConfig(Structure):
@@ -75,7 +75,7 @@ class CcaWorkspaceLayout(Structure):
 
 class CcaPlan(Structure):
     _fields_ = [("down_proj_tensor", c_int), ("attention_tensor", c_int), ("out_proj_tensor", c_int),
-                ("preproc_tensor", c_int), ("launches", c_int)]
+                ("preproc_tensor", c_int), ("launches", c_int), ("value_shift_fused", c_int)]
 
 
 _PREFILL_ARGS = [POINTER(CcaConfig)] + [c_void_p] * 9 + [c_void_p] * 4 + [c_void_p, c_size_t, c_void_p]

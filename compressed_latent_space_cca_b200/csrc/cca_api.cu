@@ -151,6 +151,7 @@ struct Resolved {
   bool tc_down, tc_attn, tc_out;  // tcgen05 kernels per stage
   bool tc_pre;                    // tensor-core preprocessing kernel (mma.sync form)
   bool pre_ws;                    // tensor-core preprocessing kernel (warp-specialised tcgen05 form)
+  bool v_fuse;                    // value shift in the down-projection's epilogue (with pre_ws)
 };
 
 cca_status_t resolve(const cca_config_t* cfg, int path, Resolved* r) {
@@ -159,7 +160,7 @@ cca_status_t resolve(const cca_config_t* cfg, int path, Resolved* r) {
   DeviceInfo* di = nullptr;
   if ((st = device_info(&di)) != CCA_OK) return st;
   const BlockDims& dm = r->dm;
-  const bool masked = (path & ~31) == CCA_PATH_TENSOR_MASK(0);
+  const bool masked = (path & ~63) == CCA_PATH_TENSOR_MASK(0);
   if (path != CCA_PATH_AUTO && path != CCA_PATH_SIMT && path != CCA_PATH_TENSOR && !masked)
     return fail(CCA_ERR_INVALID_ARG, "unknown path");
   const bool sm100 = di->major == 10;
@@ -177,6 +178,8 @@ cca_status_t resolve(const cca_config_t* cfg, int path, Resolved* r) {
     return fail(CCA_ERR_UNSUPPORTED, "a stage asked for the tensor-core kernel cannot use it");
   if (masked && (path & 8) && (path & 16))
     return fail(CCA_ERR_INVALID_ARG, "path bits 3 and 4 both choose the preprocessing kernel");
+  if (masked && (path & 32) && !((path & 1) && (path & 16)))
+    return fail(CCA_ERR_INVALID_ARG, "path bit 5 (value shift in the down-projection) needs bits 0 and 4");
   const bool use = path != CCA_PATH_SIMT;
   r->tc_down = masked ? (path & 1) != 0 : use && down;
   r->tc_attn = masked ? (path & 2) != 0 : use && attn;
@@ -185,6 +188,7 @@ cca_status_t resolve(const cca_config_t* cfg, int path, Resolved* r) {
   // after-conv term), else the mma.sync kernel; TENSOR keeps the mma.sync kernel
   r->pre_ws = masked ? (path & 16) != 0 : (path == CCA_PATH_AUTO && ws);
   r->tc_pre = masked ? (path & 8) != 0 : use && pre && !r->pre_ws;
+  r->v_fuse = masked && (path & 32) != 0;
   return CCA_OK;
 }
 
@@ -225,6 +229,14 @@ cca_status_t run_block(const Resolved& r, BlockPtrs p, cudaStream_t stream, void
     if (r.tc_pre || r.pre_ws) {  // the fp16 channel-conv weights of the preprocessing kernel, made on the side
       const long long nc = (long long)dm.d * dm.d;
       a.side_scale = r.pre_ws ? kWsWeightScale : 1.0f;
+      if (p.v_fused) {  // v~ leaves the epilogue as the value-shifted V cache and its attention copy
+        a.v_cache = p.v_cache;
+        a.v_att = p.v_att;
+        a.v_col0 = dm.Lq + dm.Lkv;
+        a.Lkv = dm.Lkv;
+        a.S = dm.S;
+        a.vshift = dm.value_shift;
+      }
       a.side_src[0] = p.cq_chan;
       a.side_dst[0] = p.wc_lat;
       a.side_n[0] = nc * dm.nq;
@@ -349,6 +361,8 @@ cca_status_t prepare(const cca_config_t* cfg, int path, const void* const* ins, 
   p->wc_lat = sep ? ws + L.wc_offset : nullptr;
   p->sched = ws + L.sched_offset;
   p->dev_err = nullptr;
+  // the conv state keeps the last v~ row, which the fused value shift does not write
+  p->v_fused = r->v_fuse && conv_state == nullptr;
   return CCA_OK;
 }
 
@@ -444,6 +458,7 @@ cca_status_t cca_plan(const cca_config_t* cfg, int path, cca_plan_t* out) {
   out->attention_tensor = r.tc_attn;
   out->out_proj_tensor = r.tc_out;
   out->preproc_tensor = r.pre_ws ? 2 : (r.tc_pre ? 1 : 0);
+  out->value_shift_fused = r.v_fuse;
   // down-projection (one tcgen05 GEMM, or three SIMT GEMMs plus the two fp16 weight copies that the
   // tcgen05 GEMM otherwise makes on the side), preprocessing, attention, output projection
   out->launches = (r.tc_down ? 1 : 3 + (r.tc_pre || r.pre_ws ? 2 : 0)) + 1 + 1 + 1;

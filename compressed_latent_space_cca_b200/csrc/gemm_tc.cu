@@ -91,7 +91,49 @@ struct GemmParams {
   __half* side_dst[2];
   long long side_n[2];
   float side_scale;
+  // value shift in the epilogue (v_cache non-null): see GemmTcArgs
+  __nv_bfloat16* v_cache;
+  __half* v_att;
+  int v_col0, Lkv, S, vshift;
 };
+
+// The value shift of 64 accumulators of one row of v~ (columns vc .. vc + 63 of the V latent): the bf16
+// cache and the fp16 attention copy, one row down within the sequence for the shifted channels
+// (nothing past the sequence end; zeros at its start). Returns true if an fp16 value overflowed.
+__device__ __forceinline__ bool store_value_shift(const GemmParams& p, long long row, int vc, const uint32_t* r) {
+  const bool shifted = p.vshift && vc >= p.Lkv / 2;
+  const long long s = row % p.S;
+  bool bad = false;
+  if (!shifted || s + 1 < p.S) {
+    const long long off = (shifted ? row + 1 : row) * p.Lkv + vc;
+    uint4* dh = reinterpret_cast<uint4*>(p.v_att + off);
+    uint4* db = reinterpret_cast<uint4*>(p.v_cache + off);
+#pragma unroll
+    for (int v = 0; v < 8; ++v) {
+      uint32_t h[4], b[4];
+#pragma unroll
+      for (int e = 0; e < 4; ++e) {
+        const float x0 = u2f(r[8 * v + 2 * e]), x1 = u2f(r[8 * v + 2 * e + 1]);
+        bad |= f16_overflow(x0) || f16_overflow(x1);
+        h[e] = pack_f16x2(x0, x1);
+        b[e] = pack_bf16x2(x0, x1);
+      }
+      dh[v] = make_uint4(h[0], h[1], h[2], h[3]);
+      db[v] = make_uint4(b[0], b[1], b[2], b[3]);
+    }
+  }
+  if (shifted && s == 0) {
+    const long long off = row * p.Lkv + vc;
+    uint4* dh = reinterpret_cast<uint4*>(p.v_att + off);
+    uint4* db = reinterpret_cast<uint4*>(p.v_cache + off);
+#pragma unroll
+    for (int v = 0; v < 8; ++v) {
+      dh[v] = make_uint4(0, 0, 0, 0);
+      db[v] = make_uint4(0, 0, 0, 0);
+    }
+  }
+  return bad;
+}
 
 // Stores 32 fp32 accumulators of one row; returns true if an fp16 output overflowed.
 __device__ __forceinline__ bool store_row_chunk(const GemmParams& p, long long row, int col0, const uint32_t* r) {
@@ -319,6 +361,10 @@ __global__ void __launch_bounds__(Shape<MH, PAIR>::NUM_THREADS, 1)
           tmem_ld_32x32b_x32(col0 + c * 64, r);
           tmem_ld_32x32b_x32(col0 + c * 64 + 32, r + 32);
           tmem_ld_wait();
+          if (p.v_cache != nullptr && n0 + c * 64 >= p.v_col0) {  // v~: the value shift, stored directly
+            if (row < p.M && n0 + c * 64 < p.N) bad |= store_value_shift(p, row, n0 + c * 64 - p.v_col0, r);
+            continue;
+          }
           uint32_t w[32];
 #pragma unroll
           for (int e = 0; e < 32; ++e) {
@@ -353,6 +399,20 @@ __global__ void __launch_bounds__(Shape<MH, PAIR>::NUM_THREADS, 1)
           tmem_ld_32x32b_x32(col0 + c * 32, r);
           tmem_ld_wait();
           const int col = n0 + c * 32;
+          if (p.v_cache != nullptr && col >= p.v_col0) {  // v~: the value shift, 64 columns at a time
+            uint32_t r2[32];
+            tmem_ld_32x32b_x32(col0 + c * 32 + 32, r2);
+            tmem_ld_wait();
+            uint32_t rr[64];
+#pragma unroll
+            for (int e = 0; e < 32; ++e) {
+              rr[e] = r[e];
+              rr[32 + e] = r2[e];
+            }
+            if (row < p.M && col < p.N) bad |= store_value_shift(p, row, col - p.v_col0, rr);
+            ++c;
+            continue;
+          }
           if (row < p.M && col < p.N) bad |= store_row_chunk(p, row, col, r);
         }
       }
@@ -482,6 +542,18 @@ cudaError_t launch_gemm_tc(const GemmTcArgs& a, cudaStream_t stream) {
     p.side_n[i] = a.side_n[i] > 0 ? a.side_n[i] : 0;
   }
   p.side_scale = a.side_scale != 0.f ? a.side_scale : 1.f;
+  if (a.v_cache != nullptr) {
+    // 64-column groups of v~ start on a 64-column boundary and never straddle the shifted half
+    if (a.v_col0 % 64 != 0 || a.Lkv % 128 != 0 || a.S < 1 || a.v_col0 + a.Lkv != N || a.out != DType::F16 ||
+        ((reinterpret_cast<uintptr_t>(a.v_cache) | reinterpret_cast<uintptr_t>(a.v_att)) & 15) != 0)
+      return cudaErrorInvalidValue;
+    p.v_cache = static_cast<__nv_bfloat16*>(a.v_cache);
+    p.v_att = static_cast<__half*>(a.v_att);
+    p.v_col0 = a.v_col0;
+    p.Lkv = a.Lkv;
+    p.S = a.S;
+    p.vshift = a.vshift;
+  }
   // 256-row tiles keep direct stores: their single accumulator leaves nothing to overlap the wait
   // for a staging buffer with, while direct stores retire without waiting
   // Pairs whenever a 256-row tile has rows to fill (on this workload's projections: 37.0 -> 34.9 us

@@ -45,6 +45,7 @@ struct BlockPtrs {
   void* wc_lat;   // [nq + nkv, d, d] lat copy of the channel-conv weights (null when lat == io)
   void* sched;    // scratch of the tensor-core attention (split-pair counters, partial rows)
   unsigned* dev_err;
+  bool v_fused;   // the down-projection has written the V cache and v_att (value shift in its epilogue)
 };
 
 // ---- SIMT path (any dtype, any even head_dim <= 128) ----
@@ -94,6 +95,13 @@ struct GemmTcArgs {
   void* side_dst[2];
   long long side_n[2];
   float side_scale;
+  // optional value shift in the epilogue (non-null v_cache): output columns [v_col0, v_col0 + Lkv)
+  // are v~ and go, shifted, to v_cache (bf16) and v_att (fp16) [T, Lkv] instead of C: channels
+  // [Lkv/2, Lkv) move one row down within their sequence of S rows (zero at a sequence start) when
+  // vshift is set
+  void* v_cache;
+  void* v_att;
+  int v_col0, Lkv, S, vshift;
 };
 cudaError_t launch_gemm_tc(const GemmTcArgs& a, cudaStream_t stream);
 // dst[0, n) = fp16 copy of the bf16 src times scale (fp16 overflow reported as a range error)

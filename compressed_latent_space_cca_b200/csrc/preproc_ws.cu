@@ -133,6 +133,7 @@ struct WsParams {
   unsigned* err;
   int* zero_cnt;  // split-pair counters of the attention launch that follows (cleared here)
   int B, S, nq, nkv, K, pre, vshift, use_rope;
+  int v_done;  // the down-projection's epilogue has written the V cache and its attention copy
   int ntiles, nT;
 };
 
@@ -607,6 +608,7 @@ __global__ void __launch_bounds__(NT, 1) preproc_ws_kernel(const __grid_constant
       }
       if (!ok) break;
       mbar_arrive(bar(B_TAPS_FREE + tb));
+      if (p.v_done) continue;
       // value shift of the group's V head: channels [Lkv/2, Lkv) of the latent come from the
       // previous token (zero at a sequence start); 8-channel vectors never straddle that boundary
       constexpr int VPER = TT * (D / 8) / 128;
@@ -883,6 +885,7 @@ cudaError_t launch_preproc_ws(const BlockDims& dm, const BlockPtrs& p, cudaStrea
   q.pre = dm.qk_mean_mode & 1;
   q.vshift = dm.value_shift;
   q.use_rope = dm.use_rope;
+  q.v_done = p.v_fused ? 1 : 0;
   q.nT = (dm.S + TT - 1) / TT;
   q.ntiles = dm.B * q.nT * dm.nkv;
   Theta th;

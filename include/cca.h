@@ -102,9 +102,14 @@ typedef enum cca_path {
 /* Per-stage choice: bit0 down-projection, bit1 attention, bit2 output
  * projection, bit3 preprocessing on the tensor-core kernel (channel mix on
  * mma.sync), bit4 preprocessing on the tcgen05 kernel (channel mix as
- * tcgen05 MMAs into tensor memory; bits 3 and 4 exclude each other); the other
- * stages on SIMT. */
-#define CCA_PATH_TENSOR_MASK(bits) (0x100 | ((bits) & 31))
+ * tcgen05 MMAs into tensor memory; bits 3 and 4 exclude each other), bit5
+ * (with bits 0 and 4) the value shift fused into the down-projection: its
+ * epilogue writes the V cache and the attention copy of v directly, so the
+ * V latent never makes the round trip through memory (the v~ region of the
+ * workspace is then not written; with a conv_state the shift stays in the
+ * preprocessing kernel, which needs the last v~ row); the other stages on
+ * SIMT. */
+#define CCA_PATH_TENSOR_MASK(bits) (0x100 | ((bits) & 63))
 
 /* Which kernels a call would launch (cca_plan). */
 typedef struct cca_plan {
@@ -113,6 +118,7 @@ typedef struct cca_plan {
   int out_proj_tensor;    /* 1: tcgen05 GEMM, 0: SIMT GEMM */
   int preproc_tensor;     /* 1: preprocessing with the channel mix on mma.sync, 2: on tcgen05 */
   int launches;           /* kernel launches of one cca_prefill without conv_state */
+  int value_shift_fused;  /* 1: the value shift runs in the down-projection's epilogue (path bit 5) */
 } cca_plan_t;
 
 typedef struct cca_prefill_opts {

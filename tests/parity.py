@@ -72,6 +72,7 @@ def run_gpu(shape, inputs, path=cca.CCA_PATH_AUTO, conv_state=False, out_dtype=N
         out[k] = v.double().cpu().numpy()
     if keep_device:
         out["_device"] = res
+    out["_v_fused"] = cca.plan(cfg, path)["value_shift_fused"] and not conv_state
     return out
 
 

@@ -13,8 +13,10 @@ pytestmark = pytest.mark.gpu
 SIMT, AUTO, TENSOR = cca.CCA_PATH_SIMT, cca.CCA_PATH_AUTO, cca.CCA_PATH_TENSOR
 # every stage on its tensor-core kernel, the preprocessing on the warp-specialised tcgen05 kernel
 WS = cca.CCA_PATH_TENSOR_MASK(1 | 2 | 4 | 16)
-PATHS = [SIMT, AUTO, TENSOR, WS]
-PATH_IDS = ["simt", "auto", "tensor", "tcgen05pre"]
+# the same with the value shift fused into the down-projection's epilogue (no v~ in the workspace)
+WSV = cca.CCA_PATH_TENSOR_MASK(1 | 2 | 4 | 16 | 32)
+PATHS = [SIMT, AUTO, TENSOR, WS, WSV]
+PATH_IDS = ["simt", "auto", "tensor", "tcgen05pre", "vfused"]
 
 
 def shape(**kw):
@@ -34,7 +36,8 @@ def check_all(sh, gpu, ref, stages=True):
         lat = gpu["qkv_lat"]
         assert_close("q_lat", lat[..., :lq], ref["q_lat"], dt)
         assert_close("k_lat", lat[..., lq:lq + lkv], ref["k_lat"], dt)
-        assert_close("v_lat", lat[..., lq + lkv:], ref["v_lat"], dt)
+        if not gpu.get("_v_fused"):  # the fused value shift leaves no v~ in the workspace
+            assert_close("v_lat", lat[..., lq + lkv:], ref["v_lat"], dt)
         assert_close("q", gpu["q"], ref["q"], dt)
         if "k_att" in gpu:
             assert_close("k_att", gpu["k_att"], ref["k_cache"].reshape(gpu["k_att"].shape), dt)
@@ -128,7 +131,7 @@ def test_plain_block_fp32():
 def test_bf16_modes(path, mode, vshift, rope):
     sh = shape(seq_len=257, qk_mean_mode=mode, value_shift=vshift, use_rope=rope, batch=2)
     inp = workloads.make_inputs(sh)
-    if path == WS and not mode & 2:
+    if path in (WS, WSV) and not mode & 2:
         # the tcgen05 preprocessing folds the after-conv mean into its MMAs: without it, it declines
         with pytest.raises(cca.CcaError) as ei:
             run_gpu(sh, inp, path=path)
@@ -181,7 +184,7 @@ def test_deterministic_and_causal(path):
         assert not np.array_equal(c[k][1, t0], a[k][1, t0]), k
 
 
-@pytest.mark.parametrize("path", [AUTO, TENSOR, WS], ids=["auto", "tensor", "tcgen05pre"])
+@pytest.mark.parametrize("path", [AUTO, TENSOR, WS, WSV], ids=["auto", "tensor", "tcgen05pre", "vfused"])
 def test_bf16_long_ragged(path):
     """S = 4097: 33 query tiles whose last holds one row, two sequences, the split
     schedule of a long sequence; caches in full, y and O on sampled rows."""
@@ -197,7 +200,7 @@ def test_bf16_long_ragged(path):
 
 
 # ------------------------------------------------- the five named workloads --
-@pytest.mark.parametrize("path", [AUTO, WS], ids=["auto", "tcgen05pre"])
+@pytest.mark.parametrize("path", [AUTO, TENSOR, WSV], ids=["auto", "tensor", "vfused"])
 @pytest.mark.parametrize("name", ["cca_dense_bf16", "ccgqa_16k_bf16", "ccgqa_8x_bf16", "ccgqa_64k_bf16"])
 def test_named_workload_full_size(name, path):
     """Full-size run in the bench's launch configuration (auto path) and with the tcgen05
