@@ -617,10 +617,13 @@ __global__ void __launch_bounds__(ANT) decode_attn_kernel(const __grid_constant_
       pml[2 * h + 1] = Ls;
     }
   }
-  // publish: the CTA's writes are ordered before thread 0's fenced count; the last chunk merges
+  // publish: every thread fences its own partial-row stores at device scope before the barrier, so
+  // all of the CTA's stores are visible before thread 0's count can be seen (a fence by thread 0
+  // alone orders only thread 0's stores: the last chunk could read other threads' rows before they
+  // landed); the last chunk merges
+  __threadfence();
   __syncthreads();
   if (threadIdx.x == 0) {
-    __threadfence();
     *flag = atomicAdd(a.cnt + bg, 1);
     __threadfence();
   }
@@ -728,18 +731,22 @@ cudaError_t launch_k(void (*kernel)(KArgs...), dim3 grid, size_t smem, cudaStrea
   return cudaLaunchKernelEx(&cfg, kernel, args...);
 }
 
-// The attention kernel is launched without programmatic dependent launch (it starts once the conv
-// kernel has completed): with it, a two-step decode test produced a non-finite output in about one
-// run in twenty, consistent with its early copies of cache rows reading a row the previous step
-// wrote; launched plainly, none in 160 runs.
+// Every kernel of the step is launched plainly: each starts once the one before it has completed.
+// With programmatic dependent launch on the attention kernel, the two-step decode of two sequences
+// produced a non-finite row in about one run in twenty; reading the chain did not show how, so no
+// kernel of the step relies on early launch (the griddepcontrol instructions in the kernels are
+// no-ops for a plain launch).
+constexpr bool kDecodePdl = false;
+
 template <typename Tc, int D>
 cudaError_t launch_attn_g(const DecodeArgs& a, cudaStream_t stream) {
   static_assert(ANT == DNT, "one block size");
   const dim3 grid(a.nch, a.nkv, a.B);
-  if (a.G <= 1) return launch_k(decode_attn_kernel<Tc, D, 1>, grid, AttnCfg<Tc, D, 1>::SMEM, stream, false, a);
-  if (a.G <= 2) return launch_k(decode_attn_kernel<Tc, D, 2>, grid, AttnCfg<Tc, D, 2>::SMEM, stream, false, a);
-  if (a.G <= 4) return launch_k(decode_attn_kernel<Tc, D, 4>, grid, AttnCfg<Tc, D, 4>::SMEM, stream, false, a);
-  return launch_k(decode_attn_kernel<Tc, D, 8>, grid, AttnCfg<Tc, D, 8>::SMEM, stream, false, a);
+  const bool pdl = kDecodePdl && a.K > 0;
+  if (a.G <= 1) return launch_k(decode_attn_kernel<Tc, D, 1>, grid, AttnCfg<Tc, D, 1>::SMEM, stream, pdl, a);
+  if (a.G <= 2) return launch_k(decode_attn_kernel<Tc, D, 2>, grid, AttnCfg<Tc, D, 2>::SMEM, stream, pdl, a);
+  if (a.G <= 4) return launch_k(decode_attn_kernel<Tc, D, 4>, grid, AttnCfg<Tc, D, 4>::SMEM, stream, pdl, a);
+  return launch_k(decode_attn_kernel<Tc, D, 8>, grid, AttnCfg<Tc, D, 8>::SMEM, stream, pdl, a);
 }
 
 template <typename Tc, typename To>
@@ -755,7 +762,7 @@ cudaError_t launch_typed(const DecodeArgs& a, cudaStream_t stream) {
   }
   // 2. seq conv, channel mix, value shift, conv state
   if (a.K > 0 && (e = launch_k(decode_conv_kernel<Tc>, dim3(a.G + 1, a.nkv, a.B), ConvSmem<Tc>::bytes(a.d, a.K),
-                               stream, true, a)) != cudaSuccess)
+                               stream, kDecodePdl, a)) != cudaSuccess)
     return e;
   // 3. attention
   switch (a.d) {
@@ -768,7 +775,7 @@ cudaError_t launch_typed(const DecodeArgs& a, cudaStream_t stream) {
   for (int b0 = 0; b0 < a.B; b0 += kGemvBatch) {
     const int nb = a.B - b0 < kGemvBatch ? a.B - b0 : kGemvBatch;
     if ((e = launch_k(decode_out_kernel<Tc, To>, dim3((a.E + DNT / 32 - 1) / (DNT / 32)),
-                      sizeof(float) * (size_t)nb * a.Lq, stream, true, a, b0, nb)) != cudaSuccess)
+                      sizeof(float) * (size_t)nb * a.Lq, stream, kDecodePdl, a, b0, nb)) != cudaSuccess)
       return e;
   }
   return cudaSuccess;
