@@ -55,14 +55,46 @@ def library() -> ctypes.CDLL:
 def make_config(*, batch: int, seq_len: int, hidden: int, n_q_heads: int, n_kv_heads: int, head_dim: int,
                 conv_kernel: int = 4, dtype="bf16", out_dtype=None, qk_mean_mode: int = 3,
                 value_shift: int = 1, use_rope: int = 1, rope_base: float = 10000.0,
-                softmax_scale: float = 0.0, C: Optional[int] = None) -> CcaConfig:
+                softmax_scale: float = 0.0, C: Optional[int] = None, kv_channel_offset: int = 0,
+                kv_total_channels: int = 0) -> CcaConfig:
     """Build a cca_config_t. C defaults to hidden / (n_q_heads * head_dim)."""
     dt = _DT_CODE[dtype]
     odt = dt if out_dtype is None else _DT_CODE[out_dtype]
     if C is None:
         C = hidden // max(1, n_q_heads * head_dim)
     return CcaConfig(batch, seq_len, hidden, C, n_q_heads, n_kv_heads, head_dim, conv_kernel, qk_mean_mode,
-                     value_shift, use_rope, rope_base, softmax_scale, dt, odt)
+                     value_shift, use_rope, rope_base, softmax_scale, dt, odt, kv_channel_offset, kv_total_channels)
+
+
+def kv_group_shard(cfg: CcaConfig, inputs: Dict[str, torch.Tensor], rank: int, world: int):
+    """The block made of one share of the KV groups, for splitting one sequence's heads over `world`
+    GPUs: share `rank` holds KV groups [rank * n, (rank + 1) * n) (n = n_kv_heads / world) and their
+    query heads. Returns (cfg, inputs) of that block: the rows of W_q, W_k, W_v and the conv weights
+    of its heads, the columns of W_o of its query heads, x unchanged, and the V-channel offset and
+    width of the whole block so that the value shift splits the whole block's V channels. The
+    block's y summed over the shares is the whole block's y; its KV cache is the whole cache's slice
+    of its heads."""
+    nkv, nq, d = cfg.n_kv_heads, cfg.n_q_heads, cfg.head_dim
+    if world < 1 or nkv % world != 0 or not 0 <= rank < world:
+        raise ValueError("n_kv_heads must be a multiple of world, 0 <= rank < world")
+    G = nq // nkv
+    gk = nkv // world
+    k0, k1 = rank * gk * d, (rank + 1) * gk * d                # V / K channels of the share
+    q0, q1 = rank * gk * G * d, (rank + 1) * gk * G * d        # Q channels of the share
+    out = {"x": inputs["x"], "W_q": inputs["W_q"][q0:q1].contiguous(), "W_k": inputs["W_k"][k0:k1].contiguous(),
+           "W_v": inputs["W_v"][k0:k1].contiguous(),
+           "W_o": inputs["W_o"][:, q0:q1].contiguous()}
+    if cfg.conv_kernel > 0:
+        out["convq_seq"] = inputs["convq_seq"][q0:q1].contiguous()
+        out["convk_seq"] = inputs["convk_seq"][k0:k1].contiguous()
+        out["convq_chan"] = inputs["convq_chan"][rank * gk * G:(rank + 1) * gk * G].contiguous()
+        out["convk_chan"] = inputs["convk_chan"][rank * gk:(rank + 1) * gk].contiguous()
+    sh = CcaConfig.from_buffer_copy(cfg)
+    sh.n_q_heads, sh.n_kv_heads = gk * G, gk
+    sh.C = cfg.hidden // (gk * G * d)
+    sh.kv_channel_offset = cfg.kv_channel_offset + k0
+    sh.kv_total_channels = cfg.kv_total_channels or nkv * d
+    return sh, out
 
 
 def config_from_shape(shape, out_dtype=None) -> CcaConfig:
@@ -71,7 +103,9 @@ def config_from_shape(shape, out_dtype=None) -> CcaConfig:
                        n_q_heads=shape.n_q_heads, n_kv_heads=shape.n_kv_heads, head_dim=shape.head_dim,
                        conv_kernel=shape.conv_kernel, dtype=shape.dtype, out_dtype=out_dtype,
                        qk_mean_mode=shape.qk_mean_mode, value_shift=shape.value_shift,
-                       use_rope=shape.use_rope, rope_base=shape.rope_base, softmax_scale=shape.softmax_scale)
+                       use_rope=shape.use_rope, rope_base=shape.rope_base, softmax_scale=shape.softmax_scale,
+                       kv_channel_offset=getattr(shape, "kv_channel_offset", 0),
+                       kv_total_channels=getattr(shape, "kv_total_channels", 0))
 
 
 def validate(cfg: CcaConfig) -> int:

@@ -49,6 +49,8 @@ class CcaConfig(Structure):
         ("softmax_scale", c_float),
         ("dtype", c_int),
         ("out_dtype", c_int),
+        ("kv_channel_offset", c_int),
+        ("kv_total_channels", c_int),
     ]
 
 

@@ -87,6 +87,16 @@ cca_status_t check_config(const cca_config_t* c, BlockDims* dm) {
   if (!(c->softmax_scale >= 0.0f) || !isfinite(c->softmax_scale))
     return fail(CCA_ERR_INVALID_ARG, "softmax_scale must be finite and >= 0");
   if (!is_dtype(c->dtype) || !is_dtype(c->out_dtype)) return fail(CCA_ERR_INVALID_ARG, "unknown dtype");
+  {
+    const long long lkv = (long long)c->n_kv_heads * c->head_dim;
+    if (c->kv_channel_offset < 0 || c->kv_total_channels < 0 || c->kv_channel_offset % 8 != 0 ||
+        c->kv_total_channels % 16 != 0 ||
+        (c->kv_total_channels > 0 && c->kv_total_channels < c->kv_channel_offset + lkv) ||
+        (c->kv_total_channels == 0 && c->kv_channel_offset != 0))
+      return fail(CCA_ERR_INVALID_ARG,
+                  "kv_channel_offset must be a multiple of 8 and kv_total_channels a multiple of 16 that holds "
+                  "this block's V channels past the offset (both 0 for a whole block)");
+  }
   if (c->head_dim > 128) return fail(CCA_ERR_UNSUPPORTED, "head_dim > 128 is not supported");
   const long long T = (long long)c->batch * c->seq_len;
   const long long Nlat = (long long)(c->n_q_heads + 2 * c->n_kv_heads) * c->head_dim;
@@ -107,6 +117,12 @@ cca_status_t check_config(const cca_config_t* c, BlockDims* dm) {
     dm->T = T;
     dm->qk_mean_mode = c->qk_mean_mode;
     dm->value_shift = c->value_shift;
+    {
+      const long long total = c->kv_total_channels > 0 ? c->kv_total_channels : (long long)dm->Lkv;
+      long long from = total / 2 - c->kv_channel_offset;
+      from = from < 0 ? 0 : (from > dm->Lkv ? dm->Lkv : from);
+      dm->vshift_from = (int)from;
+    }
     dm->use_rope = c->use_rope;
     dm->rope_base = c->rope_base;
     dm->scale = c->softmax_scale > 0.f ? c->softmax_scale : 1.0f / sqrtf((float)c->head_dim);
@@ -236,6 +252,7 @@ cca_status_t run_block(const Resolved& r, BlockPtrs p, cudaStream_t stream, void
         a.Lkv = dm.Lkv;
         a.S = dm.S;
         a.vshift = dm.value_shift;
+        a.vfrom = dm.vshift_from;
       }
       a.side_src[0] = p.cq_chan;
       a.side_dst[0] = p.wc_lat;
@@ -361,8 +378,9 @@ cca_status_t prepare(const cca_config_t* cfg, int path, const void* const* ins, 
   p->wc_lat = sep ? ws + L.wc_offset : nullptr;
   p->sched = ws + L.sched_offset;
   p->dev_err = nullptr;
-  // the conv state keeps the last v~ row, which the fused value shift does not write
-  p->v_fused = r->v_fuse && conv_state == nullptr;
+  // the conv state keeps the last v~ row, which the fused value shift does not write; the fused
+  // epilogue shifts whole 64-channel groups
+  p->v_fused = r->v_fuse && conv_state == nullptr && r->dm.vshift_from % 64 == 0;
   return CCA_OK;
 }
 

@@ -48,7 +48,7 @@ struct DecodeArgs {
   // finished-chunk counter per (sequence, KV group)
   float *z, *c, *vt, *o, *part_o, *part_ml;
   int* cnt;
-  int B, E, nkv, d, K, G, Lq, Lkv, Nlat, t, rows, mode, vshift, use_rope;
+  int B, E, nkv, d, K, G, Lq, Lkv, Nlat, t, rows, mode, vshift, vfrom, use_rope;
   int chunk_len, nch;  // keys per chunk, chunks per (KV group, sequence)
   float qscale;        // softmax scale * log2(e): scores in base-2 units
   float2 rot[64];      // (cos, sin) of t * base^(-2i/d), computed in double on the host
@@ -318,7 +318,7 @@ __global__ void __launch_bounds__(DNT) decode_conv_kernel(const __grid_constant_
   }
   if (!isq && threadIdx.x < d) {
     const int i = threadIdx.x;
-    a.vt[(long long)b * a.Lkv + g * d + i] = (a.vshift && g * d + i >= a.Lkv / 2) ? ld_f(vprev_s + i) : zvi;
+    a.vt[(long long)b * a.Lkv + g * d + i] = (a.vshift && g * d + i >= a.vfrom) ? ld_f(vprev_s + i) : zvi;
     st_f(vrow + i, zvi);
   }
   __syncthreads();
@@ -867,6 +867,7 @@ cudaError_t launch_decode(const BlockDims& dm, const DecodePtrs& p, int cache_ro
   a.rows = cache_rows;
   a.mode = dm.qk_mean_mode;
   a.vshift = dm.value_shift;
+  a.vfrom = dm.vshift_from;
   a.use_rope = dm.use_rope;
   a.qscale = dm.scale * kLog2e;
   for (int i = 0; i < dm.d / 2; ++i) {

@@ -94,14 +94,14 @@ struct GemmParams {
   // value shift in the epilogue (v_cache non-null): see GemmTcArgs
   __nv_bfloat16* v_cache;
   __half* v_att;
-  int v_col0, Lkv, S, vshift;
+  int v_col0, Lkv, S, vshift, vfrom;
 };
 
 // The value shift of 64 accumulators of one row of v~ (columns vc .. vc + 63 of the V latent): the bf16
 // cache and the fp16 attention copy, one row down within the sequence for the shifted channels
 // (nothing past the sequence end; zeros at its start). Returns true if an fp16 value overflowed.
 __device__ __forceinline__ bool store_value_shift(const GemmParams& p, long long row, int vc, const uint32_t* r) {
-  const bool shifted = p.vshift && vc >= p.Lkv / 2;
+  const bool shifted = p.vshift && vc >= p.vfrom;
   const long long s = row % p.S;
   bool bad = false;
   if (!shifted || s + 1 < p.S) {
@@ -544,7 +544,8 @@ cudaError_t launch_gemm_tc(const GemmTcArgs& a, cudaStream_t stream) {
   p.side_scale = a.side_scale != 0.f ? a.side_scale : 1.f;
   if (a.v_cache != nullptr) {
     // 64-column groups of v~ start on a 64-column boundary and never straddle the shifted half
-    if (a.v_col0 % 64 != 0 || a.Lkv % 128 != 0 || a.S < 1 || a.v_col0 + a.Lkv != N || a.out != DType::F16 ||
+    if (a.v_col0 % 64 != 0 || a.Lkv % 128 != 0 || a.vfrom % 64 != 0 || a.S < 1 || a.v_col0 + a.Lkv != N ||
+        a.out != DType::F16 ||
         ((reinterpret_cast<uintptr_t>(a.v_cache) | reinterpret_cast<uintptr_t>(a.v_att)) & 15) != 0)
       return cudaErrorInvalidValue;
     p.v_cache = static_cast<__nv_bfloat16*>(a.v_cache);
@@ -553,6 +554,7 @@ cudaError_t launch_gemm_tc(const GemmTcArgs& a, cudaStream_t stream) {
     p.Lkv = a.Lkv;
     p.S = a.S;
     p.vshift = a.vshift;
+    p.vfrom = a.vfrom;
   }
   // 256-row tiles keep direct stores: their single accumulator leaves nothing to overlap the wait
   // for a staging buffer with, while direct stores retire without waiting

@@ -27,6 +27,7 @@ struct BlockDims {
   int Nlat;     // Lq + 2*Lkv: width of the down-projection output
   long long T;  // B*S
   int qk_mean_mode, value_shift, use_rope;
+  int vshift_from;  // V channels [vshift_from, Lkv) take the previous token (with value_shift)
   float rope_base, scale;
   DType io, lat, out;
 };
@@ -97,11 +98,11 @@ struct GemmTcArgs {
   float side_scale;
   // optional value shift in the epilogue (non-null v_cache): output columns [v_col0, v_col0 + Lkv)
   // are v~ and go, shifted, to v_cache (bf16) and v_att (fp16) [T, Lkv] instead of C: channels
-  // [Lkv/2, Lkv) move one row down within their sequence of S rows (zero at a sequence start) when
+  // [vfrom, Lkv) move one row down within their sequence of S rows (zero at a sequence start) when
   // vshift is set
   void* v_cache;
   void* v_att;
-  int v_col0, Lkv, S, vshift;
+  int v_col0, Lkv, S, vshift, vfrom;
 };
 cudaError_t launch_gemm_tc(const GemmTcArgs& a, cudaStream_t stream);
 // dst[0, n) = fp16 copy of the bf16 src times scale (fp16 overflow reported as a range error)

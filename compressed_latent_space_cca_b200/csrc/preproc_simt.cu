@@ -30,7 +30,7 @@ __global__ void __launch_bounds__(PP_THREADS) preproc_simt_kernel(
     const Tc* __restrict__ ck_seq, const Tc* __restrict__ ck_chan, Tl* __restrict__ qout, Tc* __restrict__ kout,
     Tc* __restrict__ vout, Tl* __restrict__ katt, Tl* __restrict__ vatt, const Tc* __restrict__ wo,
     Tl* __restrict__ wo_lat, long long wo_n, unsigned* __restrict__ err, int S, int nq, int nkv, int d, int K,
-    int mode, int vshift, int use_rope, float rope_base, int* __restrict__ zero_cnt) {
+    int mode, int vfrom, int use_rope, float rope_base, int* __restrict__ zero_cnt) {
   extern __shared__ float sm[];
   const int G = nq / nkv;
   const int H1 = G + 1;  // G query heads + the K head of the group
@@ -162,13 +162,13 @@ __global__ void __launch_bounds__(PP_THREADS) preproc_simt_kernel(
     }
   }
 
-  // value shift: channels [Lkv/2, Lkv) come from the previous token
+  // value shift: channels [vfrom, Lkv) come from the previous token (vfrom = Lkv: no shift)
   for (int e = tid; e < PP_TT * d; e += PP_THREADS) {
     int tt = e / d, i = e % d;
     int t = t0 + tt;
     if (t >= S) continue;
     int gc = g * d + i;
-    int src = (vshift && gc >= Lkv / 2) ? t - 1 : t;
+    int src = gc >= vfrom ? t - 1 : t;
     const float val = (src >= 0) ? ld_f(qkv + (rowbase + src) * Nlat + Lq + Lkv + gc) : 0.f;
     st_f(vout + (rowbase + t) * Lkv + gc, val);
     if (vatt != nullptr) st_f(vatt + (rowbase + t) * Lkv + gc, val);
@@ -235,7 +235,7 @@ cudaError_t preproc_typed(const BlockDims& dm, const BlockPtrs& p, cudaStream_t 
       (const Tl*)p.qkv_lat, (const Tc*)p.cq_seq, (const Tc*)p.cq_chan, (const Tc*)p.ck_seq, (const Tc*)p.ck_chan,
       (Tl*)p.q, (Tc*)p.k_cache, (Tc*)p.v_cache, sep ? (Tl*)p.k_att : nullptr, sep ? (Tl*)p.v_att : nullptr,
       (const Tc*)p.Wo, sep ? (Tl*)p.wo_lat : nullptr, (long long)dm.E * dm.Lq, p.dev_err, dm.S, dm.nq, dm.nkv, dm.d,
-      dm.K, dm.qk_mean_mode, dm.value_shift, dm.use_rope, dm.rope_base,
+      dm.K, dm.qk_mean_mode, dm.value_shift ? dm.vshift_from : dm.Lkv, dm.use_rope, dm.rope_base,
       attention_tc_supported(dm) ? static_cast<int*>(p.sched) : nullptr);
   return cudaGetLastError();
 }

@@ -62,7 +62,7 @@ struct PreParams {
   long long wo_n;
   unsigned* err;
   int* zero_cnt;  // split-pair counters of the attention launch that follows (cleared here)
-  int S, nq, nkv, K, mode, vshift, use_rope;
+  int S, nq, nkv, K, mode, vshift, vfrom, use_rope;
   int nbuf;  // weight buffers in shared memory: 2 (next head's weights prefetched) or 1
 };
 
@@ -408,14 +408,14 @@ __global__ void __launch_bounds__(NT, MINB) preproc_tc_kernel(const __grid_const
   }
 
   // value-shift sources, loaded now so that the latency overlaps the k combine: channels
-  // [Lkv/2, Lkv) come from the previous token (8-channel vectors never straddle the boundary)
+  // [vfrom, Lkv) come from the previous token (8-channel vectors never straddle the boundary)
   static_assert(TT * (D / 8) == 2 * NT, "two value vectors per thread");
   uint4 vsrc[2];
 #pragma unroll
   for (int i = 0; i < 2; ++i) {
     const int e = threadIdx.x + i * NT, r = e / (D / 8), v = e % (D / 8);
     const int t = t0 + r, gc = g * D + v * 8;
-    const int src = (p.vshift && gc >= Lkv / 2) ? t - 1 : t;
+    const int src = (p.vshift && gc >= p.vfrom) ? t - 1 : t;
     vsrc[i] = make_uint4(0, 0, 0, 0);
     if (t < p.S && src >= 0) vsrc[i] = *reinterpret_cast<const uint4*>(p.lat + (rowbase + src) * Nlat + Lq + Lkv + gc);
   }
@@ -536,6 +536,7 @@ cudaError_t launch_preproc_tc(const BlockDims& dm, const BlockPtrs& p, cudaStrea
   q.K = dm.K;
   q.mode = dm.qk_mean_mode;
   q.vshift = dm.value_shift;
+  q.vfrom = dm.vshift_from;
   q.use_rope = dm.use_rope;
   Theta th;
   for (int i = 0; i < D / 2; ++i) th.v[i] = pow((double)dm.rope_base, -2.0 * (double)i / (double)D);

@@ -132,7 +132,7 @@ struct WsParams {
   long long wo_n;
   unsigned* err;
   int* zero_cnt;  // split-pair counters of the attention launch that follows (cleared here)
-  int B, S, nq, nkv, K, pre, vshift, use_rope;
+  int B, S, nq, nkv, K, pre, vshift, vfrom, use_rope;
   int v_done;  // the down-projection's epilogue has written the V cache and its attention copy
   int ntiles, nT;
 };
@@ -609,7 +609,7 @@ __global__ void __launch_bounds__(NT, 1) preproc_ws_kernel(const __grid_constant
       if (!ok) break;
       mbar_arrive(bar(B_TAPS_FREE + tb));
       if (p.v_done) continue;
-      // value shift of the group's V head: channels [Lkv/2, Lkv) of the latent come from the
+      // value shift of the group's V head: channels [vfrom, Lkv) of the latent come from the
       // previous token (zero at a sequence start); 8-channel vectors never straddle that boundary
       constexpr int VPER = TT * (D / 8) / 128;
       const long long rowbase = (long long)tl.b * p.S;
@@ -618,7 +618,7 @@ __global__ void __launch_bounds__(NT, 1) preproc_ws_kernel(const __grid_constant
       for (int k = 0; k < VPER; ++k) {
         const int e = tc + k * 128, rr = e >> 4, vv = e & 15;
         const int t = tl.t0 + rr, gc = tl.g * D + vv * 8;
-        const int src = (p.vshift && gc >= Lkv / 2) ? t - 1 : t;
+        const int src = (p.vshift && gc >= p.vfrom) ? t - 1 : t;
         vsrc[k] = make_uint4(0, 0, 0, 0);
         if (t < p.S && src >= 0)
           vsrc[k] = *reinterpret_cast<const uint4*>(p.lat + (rowbase + src) * Nlat + Lq + Lkv + gc);
@@ -884,6 +884,7 @@ cudaError_t launch_preproc_ws(const BlockDims& dm, const BlockPtrs& p, cudaStrea
   q.K = dm.K;
   q.pre = dm.qk_mean_mode & 1;
   q.vshift = dm.value_shift;
+  q.vfrom = dm.vshift_from;
   q.use_rope = dm.use_rope;
   q.v_done = p.v_fused ? 1 : 0;
   q.nT = (dm.S + TT - 1) / TT;

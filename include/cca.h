@@ -85,6 +85,18 @@ typedef struct cca_config {
   float softmax_scale; /* 0 => 1/sqrt(head_dim) */
   int dtype;         /* cca_dtype_t of every input, the KV cache and the conv state */
   int out_dtype;     /* cca_dtype_t of y (CCA_F32 allowed for bf16 inputs) */
+  /* A block that holds some of the KV groups of a wider block (heads split over GPUs: the QK-mean
+   * couples a query head only with its own group, so each share of groups is a block of its own,
+   * and y is the sum of the shares' outputs). The value shift divides the WHOLE block's V channels
+   * in halves (es 2.B item 3), so a share needs to know where its channels sit:
+   *   kv_channel_offset  the wider block's V channel index of this block's V channel 0 (a multiple
+   *                      of 8; 0 for a whole block)
+   *   kv_total_channels  the wider block's V width n_kv_total * head_dim (a multiple of 16, at
+   *                      least kv_channel_offset + n_kv_heads * head_dim; 0 for a whole block)
+   * This block's V channel c takes the previous token when value_shift is set and
+   * kv_channel_offset + c >= kv_total_channels / 2. */
+  int kv_channel_offset;
+  int kv_total_channels;
 } cca_config_t;
 
 /* Kernel path selection (cca_prefill_ex). AUTO runs each stage on its

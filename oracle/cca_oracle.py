@@ -151,10 +151,11 @@ def rope(z: np.ndarray, n_heads: int, d: int, base: float,
 # 7. Value shift (es 2.B item 3: one kind of value from the current input and
 # one from the previous input; half the heads cannot see the present token).
 # ---------------------------------------------------------------------------
-def value_shift(v: np.ndarray) -> np.ndarray:
-    """Channels [0, L/2) keep token t; channels [L/2, L) take token t-1 (0 at t=0)."""
+def value_shift(v: np.ndarray, boundary: Optional[int] = None) -> np.ndarray:
+    """Channels [0, b) keep token t; channels [b, L) take token t-1 (0 at t=0), b = L/2 unless
+    given (a block holding some of a wider block's KV groups shifts from the wider block's half)."""
     S, L = v.shape
-    half = L // 2
+    half = L // 2 if boundary is None else min(max(int(boundary), 0), L)
     out = v.copy()
     out[:, half:] = 0.0
     if S > 1:
@@ -213,7 +214,7 @@ def cca_block(inp: Dict[str, np.ndarray], n_q: int, n_kv: int, d: int, *,
               qk_mean_mode: int = 3, use_value_shift: bool = True,
               use_rope: bool = True, rope_base: float = 10000.0,
               softmax_scale: float = 0.0, rows: Optional[Sequence[int]] = None,
-              return_probs: bool = False) -> Dict[str, np.ndarray]:
+              return_probs: bool = False, value_shift_from: Optional[int] = None) -> Dict[str, np.ndarray]:
     """Prefill forward of one block, per sequence, in float64.
 
     inp holds float64 arrays: x [B,S,E], W_q [Lq,E], W_k/W_v [Lkv,E],
@@ -255,7 +256,7 @@ def cca_block(inp: Dict[str, np.ndarray], n_q: int, n_kv: int, d: int, *,
         if use_rope:
             q = rope(q, n_q, d, rope_base)
             k = rope(k, n_kv, d, rope_base)
-        v = value_shift(v_lat) if use_value_shift else v_lat.copy()
+        v = value_shift(v_lat, value_shift_from) if use_value_shift else v_lat.copy()
 
         att = causal_attention(q, k, v, n_q, n_kv, d, scale, rows=rows,
                                return_probs=return_probs)

@@ -29,7 +29,7 @@ def test_library_exports_every_declared_function():
 
 
 def test_struct_layouts():
-    assert ctypes.sizeof(cca.CcaConfig) == 15 * 4
+    assert ctypes.sizeof(cca.CcaConfig) == 17 * 4
     assert ctypes.sizeof(cca.CcaWorkspaceLayout) == 2 * 8 + 2 * 4 + 8 * 8
 
 

@@ -217,3 +217,51 @@ def test_named_workload_full_size(name, path):
     assert_close("y", gpu["y"], ref["y"], "bf16")
     del gpu
     torch.cuda.empty_cache()
+
+
+# ----------------------------------------------- KV groups split over GPUs, on one GPU --
+# One sequence's heads split in two shares of KV groups (es 2.C, 2.B item 2): each share is a block
+# of its own, given the whole block's V-channel offset and width so that its value shift splits the
+# whole block's V channels (es 2.B item 3); the shares' outputs summed are the whole block's y, and
+# each share's KV cache is the whole cache's slice of its heads. Both shares run here, one after the
+# other, through the C ABI (on several GPUs, one per GPU and one all-reduce of y).
+SPLIT_PATHS = [AUTO, TENSOR, SIMT, WSV]
+
+
+@pytest.mark.parametrize("path", SPLIT_PATHS, ids=["auto", "tensor", "simt", "vfused"])
+@pytest.mark.parametrize("nq,nkv", [(4, 2), (8, 4)])
+def test_kv_group_split_shares_sum_to_the_block(path, nq, nkv):
+    sh = shape(seq_len=300, batch=2, n_q_heads=nq, n_kv_heads=nkv, hidden=nq * 128 * 2)
+    inp = workloads.make_inputs(sh)
+    cfg = cca.config_from_shape(sh, "f32")
+    dev = {k: v.cuda() for k, v in inp.items()}
+    ref = run_oracle(sh, inp)
+    y = None
+    for rank in range(2):
+        cfg_r, inp_r = cca.kv_group_shard(cfg, dev, rank, 2)
+        res = cca.prefill(cfg_r, inp_r, path=path)
+        assert cca.poll_device_status() == cca.CCA_OK
+        y = res["y"].double() if y is None else y + res["y"].double()
+        gk = nkv // 2
+        assert_close(f"k_cache[{rank}]", res["k_cache"].double().cpu().numpy(),
+                     ref["k_cache"][:, :, rank * gk:(rank + 1) * gk], "bf16")
+        assert_close(f"v_cache[{rank}]", res["v_cache"].double().cpu().numpy(),
+                     ref["v_cache"][:, :, rank * gk:(rank + 1) * gk], "bf16")
+    assert_close("y", y.cpu().numpy(), ref["y"], "bf16")
+
+
+def test_kv_group_split_fp32():
+    sh = shape(dtype="f32", seq_len=70, batch=2, n_q_heads=4, n_kv_heads=4, head_dim=16, hidden=128)
+    inp = workloads.make_inputs(sh)
+    cfg = cca.config_from_shape(sh)
+    dev = {k: v.cuda() for k, v in inp.items()}
+    ref = run_oracle(sh, inp)
+    y = 0
+    for rank in range(2):
+        cfg_r, inp_r = cca.kv_group_shard(cfg, dev, rank, 2)
+        res = cca.prefill(cfg_r, inp_r)
+        assert cca.poll_device_status() == cca.CCA_OK
+        y = y + res["y"].double()
+        assert_close(f"v_cache[{rank}]", res["v_cache"].double().cpu().numpy(),
+                     ref["v_cache"][:, :, rank * 2:(rank + 1) * 2], "f32")
+    assert_close("y", y.cpu().numpy(), ref["y"], "f32")

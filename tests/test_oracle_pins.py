@@ -157,6 +157,14 @@ def test_value_shift_closed_form():
     np.testing.assert_array_equal(out[0, 4:], 0.0)
     np.testing.assert_array_equal(out[1:, 4:], v[:-1, 4:])
     assert oracle.value_shift(v[:1]).shape == (1, L)
+    # a share of a wider block's V channels shifts from the wider block's half: boundary 0 shifts all,
+    # L none, 3 the channels [3, L)
+    np.testing.assert_array_equal(oracle.value_shift(v, 0)[1:], v[:-1])
+    np.testing.assert_array_equal(oracle.value_shift(v, 0)[0], 0.0)
+    np.testing.assert_array_equal(oracle.value_shift(v, L), v)
+    b3 = oracle.value_shift(v, 3)
+    np.testing.assert_array_equal(b3[:, :3], v[:, :3])
+    np.testing.assert_array_equal(b3[1:, 3:], v[:-1, 3:])
 
 
 # --------------------------------------------------------------- attention --
