@@ -10,13 +10,18 @@ from .cca_oracle import (  # noqa: F401
     block_flops,
     causal_attention,
     cca_block,
+    cca_block_backward,
     channel_conv,
     decode_step,
     default_scale,
     down_project,
     qk_mean,
+    qk_mean_adjoint,
     rope,
     rope_angles,
+    rope_backward,
+    seq_conv_backward,
     seq_conv_causal,
     value_shift,
+    value_shift_backward,
 )

@@ -22,6 +22,10 @@ exact form of each step is the plainest reading of their prose:
      groups of query heads                               (es 2.A, 2.C)
   9. output projection back to width E (implied: the block's output is
      E wide and no up-projection happens before attention, es 2.A)
+ 10. one decode step (the same steps for one more token, es 1 item 2)
+ 11. the backward pass: the gradients of every input, the chain rule through
+     steps 1-9 in reverse (es 4 reports the backward's speed; its form
+     follows from the forward)
 
 Readings where the pages are silent (each restated in the project notes):
   * no biases anywhere; no q/k normalisation or temperature;
@@ -362,3 +366,141 @@ def block_flops(batch: int, seq_len: int, hidden: int, n_q: int, n_kv: int, d: i
         "attention": attention_flops(batch, seq_len, n_q, d),
         "out_proj": 2.0 * T * Lq * hidden,
     }
+
+
+# ---------------------------------------------------------------------------
+# 11. The backward pass of the block (the gradients a training step needs; es section 4 reports a
+# faster backward for CCGQA): given dL/dy, the gradients of L with respect to x and every weight, by
+# the chain rule through the steps of cca_block taken in reverse. Attention uses the full probability
+# matrix of each head (small cases only).
+# ---------------------------------------------------------------------------
+def qk_mean_adjoint(dmq: np.ndarray, dmk: np.ndarray, n_q: int, n_kv: int, d: int):
+    """The transpose of (a, b) -> qk_mean(a, b): given the gradients of the two mean terms, the
+    gradients of the query-side input a [S, n_q*d] and the key-side input b [S, n_kv*d]."""
+    S = dmq.shape[0]
+    G = n_q // n_kv
+    dq = dmq.reshape(S, n_q, d)
+    dk = dmk.reshape(S, n_kv, d)
+    da = np.empty_like(dq)
+    db = np.empty_like(dk)
+    for h in range(n_q):
+        da[:, h, :] = 0.5 * dq[:, h, :] + (0.5 / G) * dk[:, h // G, :]
+    for g in range(n_kv):
+        db[:, g, :] = 0.5 * dq[:, g * G:(g + 1) * G, :].sum(axis=1) + 0.5 * dk[:, g, :]
+    return da.reshape(S, n_q * d), db.reshape(S, n_kv * d)
+
+
+def seq_conv_backward(z: np.ndarray, w: np.ndarray, ds: np.ndarray):
+    """Gradients of the causal depthwise conv s = seq_conv_causal(z, w) for the output gradient ds:
+    (dz [S, L], dw [L, K])."""
+    S, L = z.shape
+    K = w.shape[1]
+    dz = np.zeros_like(z)
+    dw = np.zeros_like(w)
+    for j in range(K):
+        lag = K - 1 - j
+        if lag == 0:
+            dz += w[:, j] * ds
+            dw[:, j] += (ds * z).sum(axis=0)
+        elif lag < S:
+            dz[:-lag] += w[:, j] * ds[lag:]
+            dw[:, j] += (ds[lag:] * z[:-lag]).sum(axis=0)
+    return dz, dw
+
+
+def rope_backward(dz: np.ndarray, n_heads: int, d: int, base: float) -> np.ndarray:
+    """The transpose of RoPE: each pair turns back by its angle."""
+    S = dz.shape[0]
+    return rope(dz, n_heads, d, base, positions=-np.arange(S))
+
+
+def value_shift_backward(dv: np.ndarray, boundary: Optional[int] = None) -> np.ndarray:
+    """The transpose of value_shift: the shifted channels' gradient moves one token back."""
+    S, L = dv.shape
+    half = L // 2 if boundary is None else min(max(int(boundary), 0), L)
+    out = dv.copy()
+    out[:, half:] = 0.0
+    if S > 1:
+        out[:-1, half:] = dv[1:, half:]
+    return out
+
+
+def cca_block_backward(inp: Dict[str, np.ndarray], dy: np.ndarray, n_q: int, n_kv: int, d: int, *,
+                       qk_mean_mode: int = 3, use_value_shift: bool = True, use_rope: bool = True,
+                       rope_base: float = 10000.0, softmax_scale: float = 0.0,
+                       value_shift_from: Optional[int] = None) -> Dict[str, np.ndarray]:
+    """dL/d(input) for L with dL/dy = dy [B, S, E], for every input of cca_block (same names and
+    shapes), in float64."""
+    x = inp["x"]
+    B, S, E = x.shape
+    G = n_q // n_kv
+    scale = default_scale(d, softmax_scale)
+    R = 1.0 if qk_mean_mode & QK_MEAN_PRE else 0.0
+    P = 1.0 if qk_mean_mode & QK_MEAN_POST else 0.0
+    grads = {k: np.zeros_like(v) for k, v in inp.items()}
+    for b in range(B):
+        xb = x[b]
+        # forward, keeping what the backward needs
+        q_lat = down_project(xb, inp["W_q"])
+        k_lat = down_project(xb, inp["W_k"])
+        v_lat = down_project(xb, inp["W_v"])
+        s_q = seq_conv_causal(q_lat, inp["convq_seq"])
+        s_k = seq_conv_causal(k_lat, inp["convk_seq"])
+        c_q = channel_conv(s_q, inp["convq_chan"], n_q, d)
+        c_k = channel_conv(s_k, inp["convk_chan"], n_kv, d)
+        mq_pre, mk_pre = qk_mean(q_lat, k_lat, n_q, n_kv, d)
+        mq_post, mk_post = qk_mean(c_q, c_k, n_q, n_kv, d)
+        qa = c_q + R * mq_pre + P * mq_post
+        ka = c_k + R * mk_pre + P * mk_post
+        q = rope(qa, n_q, d, rope_base) if use_rope else qa
+        k = rope(ka, n_kv, d, rope_base) if use_rope else ka
+        v = value_shift(v_lat, value_shift_from) if use_value_shift else v_lat
+        o, probs = causal_attention(q, k, v, n_q, n_kv, d, scale, return_probs=True)
+        # output projection
+        grads["W_o"] += dy[b].T @ o
+        do = dy[b] @ inp["W_o"]
+        # attention
+        dq = np.zeros_like(q)
+        dk = np.zeros_like(k)
+        dv = np.zeros_like(v)
+        for h in range(n_q):
+            g = h // G
+            p = probs[h]                        # [S, S], zero above the diagonal
+            qh = q[:, h * d:(h + 1) * d]
+            kh = k[:, g * d:(g + 1) * d]
+            vh = v[:, g * d:(g + 1) * d]
+            doh = do[:, h * d:(h + 1) * d]
+            dv[:, g * d:(g + 1) * d] += p.T @ doh
+            dp = doh @ vh.T
+            dsc = p * (dp - (dp * p).sum(axis=1, keepdims=True))
+            dq[:, h * d:(h + 1) * d] = scale * (dsc @ kh)
+            dk[:, g * d:(g + 1) * d] += scale * (dsc.T @ qh)
+        # value shift, RoPE
+        dv_lat = value_shift_backward(dv, value_shift_from) if use_value_shift else dv
+        dqa = rope_backward(dq, n_q, d, rope_base) if use_rope else dq
+        dka = rope_backward(dk, n_kv, d, rope_base) if use_rope else dk
+        # QK-mean terms: qa, ka depend on (q~, k~) through the PRE mean, on (c_q, c_k) directly and
+        # through the POST mean
+        da, db = qk_mean_adjoint(dqa, dka, n_q, n_kv, d)
+        dc_q = dqa + P * da
+        dc_k = dka + P * db
+        dq_lat = R * da
+        dk_lat = R * db
+        # channel conv: c[t,h,i] = sum_j W[h,i,j] s[t,h,j]
+        for name, dc, s, nh in (("convq_chan", dc_q, s_q, n_q), ("convk_chan", dc_k, s_k, n_kv)):
+            grads[name] += np.einsum("thi,thj->hij", dc.reshape(S, nh, d), s.reshape(S, nh, d))
+        ds_q = np.einsum("thi,hij->thj", dc_q.reshape(S, n_q, d), inp["convq_chan"]).reshape(S, n_q * d)
+        ds_k = np.einsum("thi,hij->thj", dc_k.reshape(S, n_kv, d), inp["convk_chan"]).reshape(S, n_kv * d)
+        # sequence conv
+        dz_q, dwq = seq_conv_backward(q_lat, inp["convq_seq"], ds_q)
+        dz_k, dwk = seq_conv_backward(k_lat, inp["convk_seq"], ds_k)
+        grads["convq_seq"] += dwq
+        grads["convk_seq"] += dwk
+        dq_lat = dq_lat + dz_q
+        dk_lat = dk_lat + dz_k
+        # down-projection
+        grads["W_q"] += dq_lat.T @ xb
+        grads["W_k"] += dk_lat.T @ xb
+        grads["W_v"] += dv_lat.T @ xb
+        grads["x"][b] = dq_lat @ inp["W_q"] + dk_lat @ inp["W_k"] + dv_lat @ inp["W_v"]
+    return grads
