@@ -344,6 +344,46 @@ def decode(cfg: CcaConfig, x_t: torch.Tensor, weights: Dict[str, torch.Tensor], 
     return y
 
 
+GRAD_NAMES = ("x", "W_q", "W_k", "W_v", "convq_seq", "convq_chan", "convk_seq", "convk_chan", "W_o")
+
+
+def backward_workspace_size(cfg: CcaConfig) -> int:
+    """Bytes of workspace cca_backward needs (0 if the configuration is not supported)."""
+    return library().cca_backward_workspace_size(ctypes.byref(cfg))
+
+
+def backward(cfg: CcaConfig, inputs: Dict[str, torch.Tensor], dy: torch.Tensor, *,
+             grads: Optional[Dict[str, torch.Tensor]] = None, workspace: Optional[torch.Tensor] = None,
+             stream: Optional[torch.cuda.Stream] = None) -> Dict[str, torch.Tensor]:
+    """cca_backward: the gradients of x and of the eight weights for dL/dy = dy.
+
+    inputs: the nine tensors of INPUT_NAMES (dtype cfg.dtype); dy [B, S, E] in cfg.out_dtype.
+    Returns fp32 tensors named as the inputs, in their shapes (overwritten, not accumulated).
+    """
+    x = inputs["x"]
+    device = x.device
+    if device.type != "cuda":
+        raise ValueError("inputs must be CUDA tensors")
+    sh = _shapes(cfg)
+    ptrs = _input_ptrs(cfg, inputs, INPUT_NAMES, _DT[cfg.dtype], device)
+    dyp = _check(dy, "dy", sh["y"], _DT[cfg.out_dtype], device)
+    if grads is None:
+        grads = {n: torch.empty(sh[n], dtype=torch.float32, device=device) for n in GRAD_NAMES}
+    gp = [_check(grads[n], "d" + n, sh[n], torch.float32, device) for n in GRAD_NAMES]
+    if workspace is None:
+        n = backward_workspace_size(cfg)
+        if n == 0:
+            raise CcaError(CCA_ERR_UNSUPPORTED, "cca_backward_workspace_size")
+        workspace = torch.empty(n, dtype=torch.uint8, device=device)
+    if stream is None:
+        stream = torch.cuda.current_stream(device)
+    st = library().cca_backward(ctypes.byref(cfg), *ptrs, dyp, *gp, workspace.data_ptr(), workspace.numel(),
+                                ctypes.c_void_p(stream.cuda_stream))
+    if st != CCA_OK:
+        raise CcaError(st, "cca_backward")
+    return grads
+
+
 def poll_device_status(stream: Optional[torch.cuda.Stream] = None) -> int:
     """Synchronize and return the device status (CCA_OK or CCA_ERR_DEVICE_TIMEOUT ...)."""
     s = stream.cuda_stream if stream is not None else torch.cuda.current_stream().cuda_stream

@@ -96,6 +96,9 @@ SIGNATURES = {
     "cca_decode_workspace_size": (c_size_t, [POINTER(CcaConfig)]),
     "cca_decode": (c_int, [POINTER(CcaConfig), c_int] + [c_void_p] * 9 + [c_void_p] * 4
                    + [c_void_p, c_size_t, c_void_p]),
+    "cca_backward_workspace_size": (c_size_t, [POINTER(CcaConfig)]),
+    "cca_backward": (c_int, [POINTER(CcaConfig)] + [c_void_p] * 10 + [c_void_p] * 9
+                     + [c_void_p, c_size_t, c_void_p]),
     "cca_poll_device_status": (c_int, [c_void_p]),
     "cca_selftest_wait_timeout": (c_int, [c_uint, c_void_p]),
     "cca_status_string": (c_char_p, [c_int]),

@@ -1,0 +1,748 @@
+// The backward pass of one CCA / CCGQA block: given dL/dy, the gradients of x and of every weight
+// ("Compressed Convolutional Attention", gist.science/es/paper/2510.04476, section 4 reports the
+// backward of CCGQA; its form is the chain rule through the forward of section 2 in reverse).
+//
+// The forward's activations are recomputed by the forward kernels into the backward's workspace;
+// then, in fp32:
+//   dO = dy W_o;  dW_o = dy^T O                                  (strided GEMMs)
+//   per (row, head): LSE of the softmax and delta = rowsum(dO o O)
+//   attention backward (FlashAttention-2 form): a CTA per 64-key block of one KV group walks the
+//     query blocks at or after it for each query head of the group, recomputes P from q, k and the
+//     LSE, accumulates dV and dK in registers and adds dQ atomically
+//   per token: RoPE turned back, the QK-mean terms' transpose (which feeds dc and the latents
+//     directly), the value shift's transpose
+//   channel mix: ds = W_c^T dc, dW_c = sum_t dc^T s (s recomputed from the latents)
+//   seq conv: dz[t] = sum_j w_j ds[t + K-1-j], dw_j = sum_t ds[t] z[t-K+1+j]
+//   down-projection: dx = dlat [W_q; W_k; W_v], dW = dlat^T x       (strided GEMMs)
+// Every product here runs on the CUDA cores in fp32 (a first form of this pass: correct, not fast).
+#include <math.h>
+
+#include "cca_common.cuh"
+#include "launch.h"
+
+namespace cca {
+namespace {
+
+// ------------------------------------------------------------------ strided GEMM --
+// C[z][m][n] (+)= sum_k A[z][m*sam + k*sak] * B[z][n*sbn + k*sbk] in fp32, for a batch of z problems
+// whose operands start zsa, zsb and zsc elements apart. 64 x 64 tiles, 16-deep K steps, 256 threads
+// with 4 x 4 outputs each. With ksplit > 1 the K range is cut into ksplit slices (grid z = batch x
+// ksplit) whose partial sums are added atomically into C.
+constexpr int SG_M = 64, SG_N = 64, SG_K = 16;
+
+template <typename TA, typename TB>
+__global__ void __launch_bounds__(256) gemm_strided_kernel(const TA* __restrict__ A, long long sam, long long sak,
+                                                           long long zsa, const TB* __restrict__ B, long long sbn,
+                                                           long long sbk, long long zsb, float* __restrict__ C,
+                                                           long long ldc, long long zsc, int M, int N, long long K,
+                                                           int accumulate, int ksplit) {
+  __shared__ float As[SG_K][SG_M + 4];
+  __shared__ float Bs[SG_K][SG_N + 4];
+  const int tid = threadIdx.x;
+  const long long z = blockIdx.z / ksplit;
+  const int slice = blockIdx.z % ksplit;
+  A += z * zsa;
+  B += z * zsb;
+  C += z * zsc;
+  const int m0 = blockIdx.y * SG_M, n0 = blockIdx.x * SG_N;
+  const int tr = tid / 16, tc = tid % 16;
+  const long long kchunk = ((K + ksplit - 1) / ksplit + SG_K - 1) / SG_K * SG_K;
+  const long long kbeg = slice * kchunk, kend = kbeg + kchunk < K ? kbeg + kchunk : K;
+  float acc[4][4] = {};
+  for (long long k0 = kbeg; k0 < kend; k0 += SG_K) {
+    // each thread loads 4 elements of each tile; the fastest-moving index follows the operand's
+    // unit stride where it has one
+    for (int e = tid; e < SG_K * SG_M; e += 256) {
+      int kk, mm;
+      if (sam == 1) {
+        mm = e % SG_M;
+        kk = e / SG_M;
+      } else {
+        kk = e % SG_K;
+        mm = e / SG_K;
+      }
+      const long long k = k0 + kk;
+      const int m = m0 + mm;
+      As[kk][mm] = (m < M && k < kend) ? ld_f(A + m * sam + k * sak) : 0.f;
+    }
+    for (int e = tid; e < SG_K * SG_N; e += 256) {
+      int kk, nn;
+      if (sbn == 1) {
+        nn = e % SG_N;
+        kk = e / SG_N;
+      } else {
+        kk = e % SG_K;
+        nn = e / SG_K;
+      }
+      const long long k = k0 + kk;
+      const int n = n0 + nn;
+      Bs[kk][nn] = (n < N && k < kend) ? ld_f(B + n * sbn + k * sbk) : 0.f;
+    }
+    __syncthreads();
+#pragma unroll
+    for (int kk = 0; kk < SG_K; ++kk) {
+      float a[4], b[4];
+#pragma unroll
+      for (int i = 0; i < 4; ++i) a[i] = As[kk][tr * 4 + i];
+#pragma unroll
+      for (int j = 0; j < 4; ++j) b[j] = Bs[kk][tc * 4 + j];
+#pragma unroll
+      for (int i = 0; i < 4; ++i)
+#pragma unroll
+        for (int j = 0; j < 4; ++j) acc[i][j] = fmaf(a[i], b[j], acc[i][j]);
+    }
+    __syncthreads();
+  }
+#pragma unroll
+  for (int i = 0; i < 4; ++i) {
+    const int m = m0 + tr * 4 + i;
+    if (m >= M) continue;
+#pragma unroll
+    for (int j = 0; j < 4; ++j) {
+      const int n = n0 + tc * 4 + j;
+      if (n >= N) continue;
+      float* c = C + (long long)m * ldc + n;
+      if (ksplit > 1) atomicAdd(c, acc[i][j]);
+      else *c = accumulate ? *c + acc[i][j] : acc[i][j];
+    }
+  }
+}
+
+struct Mat {
+  const void* p;
+  DType t;
+};
+
+template <typename TA>
+cudaError_t gemm_b(Mat a, long long sam, long long sak, long long zsa, Mat b, long long sbn, long long sbk,
+                   long long zsb, float* C, long long ldc, long long zsc, int M, int N, long long K, int batch,
+                   bool accumulate, int ksplit, cudaStream_t s) {
+  const dim3 grid((N + SG_N - 1) / SG_N, (M + SG_M - 1) / SG_M, batch * ksplit);
+  const TA* A = static_cast<const TA*>(a.p);
+  switch (b.t) {
+    case DType::F32:
+      gemm_strided_kernel<TA, float><<<grid, 256, 0, s>>>(A, sam, sak, zsa, static_cast<const float*>(b.p), sbn, sbk,
+                                                          zsb, C, ldc, zsc, M, N, K, accumulate, ksplit);
+      break;
+    case DType::BF16:
+      gemm_strided_kernel<TA, __nv_bfloat16><<<grid, 256, 0, s>>>(A, sam, sak, zsa,
+                                                                  static_cast<const __nv_bfloat16*>(b.p), sbn, sbk,
+                                                                  zsb, C, ldc, zsc, M, N, K, accumulate, ksplit);
+      break;
+    case DType::F16:
+      gemm_strided_kernel<TA, __half><<<grid, 256, 0, s>>>(A, sam, sak, zsa, static_cast<const __half*>(b.p), sbn,
+                                                           sbk, zsb, C, ldc, zsc, M, N, K, accumulate, ksplit);
+      break;
+  }
+  return cudaGetLastError();
+}
+
+// A long K (the token dimension of a weight gradient) with few output tiles is split so that the
+// grid covers the SMs about twice; C (a contiguous [batch][M][ldc] block) is cleared first unless
+// it accumulates.
+cudaError_t gemm(Mat a, long long sam, long long sak, long long zsa, Mat b, long long sbn, long long sbk, long long zsb,
+                 float* C, long long ldc, long long zsc, int M, int N, long long K, int batch, bool accumulate,
+                 cudaStream_t s) {
+  const long long tiles = (long long)((N + SG_N - 1) / SG_N) * ((M + SG_M - 1) / SG_M) * batch;
+  const long long want = (2LL * num_sms() + tiles - 1) / tiles;
+  long long ksplit = want < K / 512 ? want : K / 512;
+  if (ksplit < 1) ksplit = 1;
+  if (ksplit > 1 && !accumulate) {
+    const long long n = (long long)(batch - 1) * zsc + (long long)(M - 1) * ldc + N;
+    const cudaError_t e = cudaMemsetAsync(C, 0, sizeof(float) * n, s);
+    if (e != cudaSuccess) return e;
+  }
+  const int ks = (int)ksplit;
+  switch (a.t) {
+    case DType::F32: return gemm_b<float>(a, sam, sak, zsa, b, sbn, sbk, zsb, C, ldc, zsc, M, N, K, batch, accumulate, ks, s);
+    case DType::BF16:
+      return gemm_b<__nv_bfloat16>(a, sam, sak, zsa, b, sbn, sbk, zsb, C, ldc, zsc, M, N, K, batch, accumulate, ks, s);
+    case DType::F16:
+      return gemm_b<__half>(a, sam, sak, zsa, b, sbn, sbk, zsb, C, ldc, zsc, M, N, K, batch, accumulate, ks, s);
+  }
+  return cudaErrorInvalidValue;
+}
+
+// ------------------------------------------------------------------ row statistics --
+// Per (row t, query head h): lse = m + log(l) of the causal softmax of scale * q k^T (base e), and
+// delta = sum_i dO[t,h,i] O[t,h,i]. A CTA per (64-row block, head, sequence) walks the key blocks
+// at or before it: each thread holds a 4 x 4 patch of the score tile, rows are reduced over the 16
+// threads that share them, and every thread keeps the running (m, l) of its 4 rows.
+constexpr int RB = 64;
+
+template <typename Tl>
+__global__ void __launch_bounds__(256, 2) row_stats_kernel(const Tl* __restrict__ q, const Tl* __restrict__ k,
+                                                        const Tl* __restrict__ o, const float* __restrict__ dO,
+                                                        float* __restrict__ lse, float* __restrict__ delta, int S,
+                                                        int nq, int nkv, int d, float scale) {
+  extern __shared__ float rsm[];
+  const int DP = d + 1;  // padded rows: the 16 rows a warp reads fall in different banks
+  float* qs = rsm;           // [RB][DP]
+  float* ks = qs + RB * DP;  // [RB][DP]
+  const int qb = blockIdx.x, h = blockIdx.y, b = blockIdx.z;
+  const int G = nq / nkv, g = h / G, Lq = nq * d, Lkv = nkv * d;
+  const long long rb = (long long)b * S;
+  const int q0 = qb * RB, tid = threadIdx.x;
+  const int qr = tid / 16, kc = tid % 16;
+  for (int e = tid; e < RB * d; e += 256) {
+    const int r = e / d, c = e % d;
+    qs[r * DP + c] = q0 + r < S ? ld_f(q + (rb + q0 + r) * Lq + h * d + c) : 0.f;
+  }
+  float m[4], l[4];
+#pragma unroll
+  for (int i = 0; i < 4; ++i) {
+    m[i] = -INFINITY;
+    l[i] = 0.f;
+  }
+  for (int k0 = 0; k0 <= q0; k0 += RB) {
+    __syncthreads();
+    for (int e = tid; e < RB * d; e += 256) {
+      const int r = e / d, c = e % d;
+      ks[r * DP + c] = k0 + r < S ? ld_f(k + (rb + k0 + r) * Lkv + g * d + c) : 0.f;
+    }
+    __syncthreads();
+    float sacc[4][4] = {};
+    for (int c = 0; c < d; ++c) {
+      float qa[4], kb[4];
+#pragma unroll
+      for (int i = 0; i < 4; ++i) {
+        qa[i] = qs[(qr * 4 + i) * DP + c];
+        kb[i] = ks[(kc * 4 + i) * DP + c];
+      }
+#pragma unroll
+      for (int a = 0; a < 4; ++a)
+#pragma unroll
+        for (int bb = 0; bb < 4; ++bb) sacc[a][bb] = fmaf(qa[a], kb[bb], sacc[a][bb]);
+    }
+#pragma unroll
+    for (int a = 0; a < 4; ++a) {
+      const int t = q0 + qr * 4 + a;
+      float mx = -INFINITY;
+#pragma unroll
+      for (int bb = 0; bb < 4; ++bb) {
+        const int key = k0 + kc * 4 + bb;
+        sacc[a][bb] = (key <= t && key < S) ? sacc[a][bb] * scale : -INFINITY;
+        mx = fmaxf(mx, sacc[a][bb]);
+      }
+#pragma unroll
+      for (int off = 8; off > 0; off >>= 1) mx = fmaxf(mx, __shfl_xor_sync(0xffffffffu, mx, off));
+      const float mn = fmaxf(m[a], mx);
+      float sum = 0.f;
+      if (mn != -INFINITY) {
+#pragma unroll
+        for (int bb = 0; bb < 4; ++bb) sum += sacc[a][bb] == -INFINITY ? 0.f : expf(sacc[a][bb] - mn);
+      }
+#pragma unroll
+      for (int off = 8; off > 0; off >>= 1) sum += __shfl_xor_sync(0xffffffffu, sum, off);
+      l[a] = (m[a] == -INFINITY ? 0.f : l[a] * expf(m[a] - mn)) + sum;
+      m[a] = mn;
+    }
+  }
+  if (kc == 0) {
+#pragma unroll
+    for (int a = 0; a < 4; ++a) {
+      const int t = q0 + qr * 4 + a;
+      if (t < S) lse[(rb + t) * nq + h] = m[a] + logf(l[a]);
+    }
+  }
+  // delta: 4 threads per row, each over a quarter of the columns
+  {
+    const int r = tid / 4, part = tid % 4;
+    float dl = 0.f;
+    if (q0 + r < S) {
+      const Tl* orow = o + (rb + q0 + r) * Lq + h * d;
+      const float* drow = dO + (rb + q0 + r) * Lq + h * d;
+      for (int c = part; c < d; c += 4) dl = fmaf(ld_f(orow + c), drow[c], dl);
+    }
+    dl += __shfl_xor_sync(0xffffffffu, dl, 1);
+    dl += __shfl_xor_sync(0xffffffffu, dl, 2);
+    if (part == 0 && q0 + r < S) delta[(rb + q0 + r) * nq + h] = dl;
+  }
+}
+
+// ------------------------------------------------------------------ attention backward --
+// A CTA per (64-key block j, KV group g, sequence b). For each query head h of the group and each
+// 64-query block i >= j: S = scale q_i k_j^T, P = exp(S - lse) (causal), dV_j += P^T dO_i,
+// dP = dO_i v_j^T, dS = P o (dP - delta), dK_j += scale dS^T q_i, dQ_i += scale dS k_j (atomic).
+constexpr int AB = 64;  // keys and queries per block
+
+template <typename Tl>
+__global__ void __launch_bounds__(256) attn_bwd_kernel(const Tl* __restrict__ q, const Tl* __restrict__ k,
+                                                       const Tl* __restrict__ v, const float* __restrict__ dO,
+                                                       const float* __restrict__ lse, const float* __restrict__ delta,
+                                                       float* __restrict__ dq, float* __restrict__ dk,
+                                                       float* __restrict__ dv, int S, int nq, int nkv, int d,
+                                                       float scale) {
+  extern __shared__ float sb[];
+  const int D = d, DP = d + 1;  // padded rows: the rows a warp reads at one column fall in different banks
+  float* ks = sb;                // [AB][DP]
+  float* vs = ks + AB * DP;      // [AB][DP]
+  float* qs = vs + AB * DP;      // [AB][DP]
+  float* dos = qs + AB * DP;     // [AB][DP]
+  float* ps = dos + AB * DP;     // [AB][AB + 1] P
+  float* dps = ps + AB * (AB + 1);  // [AB][AB + 1] dP
+  float* ls = dps + AB * (AB + 1);  // [AB] lse
+  float* ds_ = ls + AB;             // [AB] delta
+  const int j = blockIdx.x, g = blockIdx.y, b = blockIdx.z;
+  const int G = nq / nkv, Lq = nq * d, Lkv = nkv * d;
+  const long long rb = (long long)b * S;
+  const int k0 = j * AB;
+  if (k0 >= S) return;
+  const int tid = threadIdx.x;
+  for (int e = tid; e < AB * D; e += 256) {
+    const int r = e / D, c = e % D;
+    const bool ok = k0 + r < S;
+    ks[r * DP + c] = ok ? ld_f(k + (rb + k0 + r) * Lkv + g * d + c) : 0.f;
+    vs[r * DP + c] = ok ? ld_f(v + (rb + k0 + r) * Lkv + g * d + c) : 0.f;
+  }
+  // dK_j and dV_j: thread owns (row r = tid / 4, columns c = (tid % 4) + 4 u) for u < D / 4
+  const int orow = tid >> 2, ocol = tid & 3;
+  float dka[32], dva[32];
+#pragma unroll
+  for (int u = 0; u < 32; ++u) dka[u] = dva[u] = 0.f;
+  __syncthreads();
+  for (int hh = 0; hh < G; ++hh) {
+    const int h = g * G + hh;
+    for (int q0 = k0; q0 < S; q0 += AB) {
+      for (int e = tid; e < AB * D; e += 256) {
+        const int r = e / D, c = e % D;
+        const bool ok = q0 + r < S;
+        qs[r * DP + c] = ok ? ld_f(q + (rb + q0 + r) * Lq + h * d + c) : 0.f;
+        dos[r * DP + c] = ok ? dO[(rb + q0 + r) * Lq + h * d + c] : 0.f;
+      }
+      for (int r = tid; r < AB; r += 256) {
+        const bool ok = q0 + r < S;
+        ls[r] = ok ? lse[(rb + q0 + r) * nq + h] : 0.f;
+        ds_[r] = ok ? delta[(rb + q0 + r) * nq + h] : 0.f;
+      }
+      __syncthreads();
+      // P and dP: thread computes a 4 x 4 patch (query rows qr*4.., key cols kc*4..)
+      {
+        const int qr = tid / 16, kc = tid % 16;
+        float sacc[4][4] = {}, pacc[4][4] = {};
+        for (int c = 0; c < D; ++c) {
+          float qa[4], da[4], kb[4], vb[4];
+#pragma unroll
+          for (int i = 0; i < 4; ++i) {
+            qa[i] = qs[(qr * 4 + i) * DP + c];
+            da[i] = dos[(qr * 4 + i) * DP + c];
+          }
+#pragma unroll
+          for (int i = 0; i < 4; ++i) {
+            kb[i] = ks[(kc * 4 + i) * DP + c];
+            vb[i] = vs[(kc * 4 + i) * DP + c];
+          }
+#pragma unroll
+          for (int a = 0; a < 4; ++a)
+#pragma unroll
+            for (int bb = 0; bb < 4; ++bb) {
+              sacc[a][bb] = fmaf(qa[a], kb[bb], sacc[a][bb]);
+              pacc[a][bb] = fmaf(da[a], vb[bb], pacc[a][bb]);
+            }
+        }
+#pragma unroll
+        for (int a = 0; a < 4; ++a)
+#pragma unroll
+          for (int bb = 0; bb < 4; ++bb) {
+            const int qi = qr * 4 + a, kj = kc * 4 + bb;
+            const bool vis = q0 + qi < S && k0 + kj < S && k0 + kj <= q0 + qi;
+            const float p = vis ? expf(sacc[a][bb] * scale - ls[qi]) : 0.f;
+            ps[qi * (AB + 1) + kj] = p;
+            dps[qi * (AB + 1) + kj] = p * (pacc[a][bb] - ds_[qi]);  // dS (before the scale)
+          }
+      }
+      __syncthreads();
+      // dV_j += P^T dO_i, dK_j += scale dS^T q_i
+      for (int qi = 0; qi < AB; ++qi) {
+        const float p = ps[qi * (AB + 1) + orow], dsv = dps[qi * (AB + 1) + orow];
+#pragma unroll
+        for (int u = 0; u < 32; ++u) {
+          const int c = ocol + 4 * u;
+          if (c < D) {
+            dva[u] = fmaf(p, dos[qi * DP + c], dva[u]);
+            dka[u] = fmaf(dsv * scale, qs[qi * DP + c], dka[u]);
+          }
+        }
+      }
+      // dQ_i += scale dS k_j: thread (row qi = tid / 4, columns ocol + 4u)
+      {
+        const int qi = orow;
+        if (q0 + qi < S) {
+          float acc[32];
+#pragma unroll
+          for (int u = 0; u < 32; ++u) acc[u] = 0.f;
+          for (int kj = 0; kj < AB; ++kj) {
+            const float dsv = dps[qi * (AB + 1) + kj] * scale;
+#pragma unroll
+            for (int u = 0; u < 32; ++u) {
+              const int c = ocol + 4 * u;
+              if (c < D) acc[u] = fmaf(dsv, ks[kj * DP + c], acc[u]);
+            }
+          }
+          float* dqr = dq + (rb + q0 + qi) * Lq + h * d;
+#pragma unroll
+          for (int u = 0; u < 32; ++u) {
+            const int c = ocol + 4 * u;
+            if (c < D) atomicAdd(dqr + c, acc[u]);
+          }
+        }
+      }
+      __syncthreads();
+    }
+  }
+  if (k0 + orow < S) {
+#pragma unroll
+    for (int u = 0; u < 32; ++u) {
+      const int c = ocol + 4 * u;
+      if (c < D) {
+        dk[(rb + k0 + orow) * Lkv + g * d + c] = dka[u];
+        dv[(rb + k0 + orow) * Lkv + g * d + c] = dva[u];
+      }
+    }
+  }
+}
+
+// ------------------------------------------------------------------ per-token backward --
+// Row t of one sequence: dq, dk turned back by RoPE; the QK-mean transpose gives dc (the
+// channel-mix outputs' gradient) and the latents' direct gradient dpre; dv goes through the value
+// shift's transpose (channels [vfrom, Lkv) take the next token's gradient). Thread = one pair
+// (i, i + d/2) of one head (q heads, then K heads), or one V channel.
+struct Theta64 {
+  double v[64];  // base^(-2i/d)
+};
+
+__global__ void __launch_bounds__(256) token_bwd_kernel(const float* __restrict__ dq, const float* __restrict__ dk,
+                                                        const float* __restrict__ dv, float* __restrict__ dc,
+                                                        float* __restrict__ dpre, float* __restrict__ dlat, int S,
+                                                        int nq, int nkv, int d, int mode, int vshift, int vfrom,
+                                                        int use_rope, const __grid_constant__ Theta64 theta) {
+  const long long row = blockIdx.x;  // b * S + t
+  const int t = (int)(row % S);
+  const int G = nq / nkv, Lq = nq * d, Lkv = nkv * d, half = d / 2, Nlat = Lq + 2 * Lkv;
+  const float R = (mode & 1) ? 1.f : 0.f, P = (mode & 2) ? 1.f : 0.f;
+  extern __shared__ float ta[];  // dqa [Lq], dka [Lkv]
+  float* dqa = ta;
+  float* dka = ta + Lq;
+  for (int e = threadIdx.x; e < (nq + nkv) * half; e += blockDim.x) {
+    const int hh = e / half, i = e % half;
+    const bool isq = hh < nq;
+    const float* src = isq ? dq + row * Lq + hh * d : dk + row * Lkv + (hh - nq) * d;
+    float x1 = src[i], x2 = src[i + half];
+    if (use_rope) {  // turn back by t theta_i (angle reduced in fp64)
+      const double a = (double)t * theta.v[i];
+      const double kk = rint(a * 0.15915494309189535);
+      double r = fma(-kk, 6.283185307179586, a);
+      r = fma(-kk, 2.4492935982947064e-16, r);
+      float sn, cs;
+      sincosf((float)r, &sn, &cs);
+      const float y1 = x1 * cs + x2 * sn, y2 = x2 * cs - x1 * sn;
+      x1 = y1;
+      x2 = y2;
+    }
+    float* dst = isq ? dqa + hh * d : dka + (hh - nq) * d;
+    dst[i] = x1;
+    dst[i + half] = x2;
+  }
+  __syncthreads();
+  // QK-mean transpose: da_h = dqa_h / 2 + dka_g / (2G), db_g = sum_{h in g} dqa_h / 2 + dka_g / 2
+  for (int e = threadIdx.x; e < Lq + Lkv; e += blockDim.x) {
+    float a, bsum;
+    float direct;
+    if (e < Lq) {
+      const int h = e / d, i = e % d, g = h / G;
+      direct = dqa[e];
+      a = 0.5f * dqa[e] + (0.5f / (float)G) * dka[g * d + i];
+      bsum = a;
+    } else {
+      const int c = e - Lq, g = c / d, i = c % d;
+      direct = dka[c];
+      float s = 0.f;
+      for (int hh = 0; hh < G; ++hh) s += dqa[(g * G + hh) * d + i];
+      a = 0.5f * s + 0.5f * dka[c];
+      bsum = a;
+    }
+    dc[row * (Lq + Lkv) + e] = direct + P * bsum;
+    dpre[row * (Lq + Lkv) + e] = R * a;
+  }
+  // value shift transpose
+  for (int c = threadIdx.x; c < Lkv; c += blockDim.x) {
+    float val;
+    if (vshift && c >= vfrom) val = (t + 1 < S) ? dv[(row + 1) * Lkv + c] : 0.f;
+    else val = dv[row * Lkv + c];
+    dlat[row * Nlat + Lq + Lkv + c] = val;
+  }
+}
+
+// Channel mix transpose and the recomputed seq-conv output: per row t, per head (q heads then K
+// heads) ds[t] = W_c^T dc[t] and s[t] = seq_conv(z)[t]. Block = one row; thread = one channel.
+template <typename Tl, typename Tc>
+__global__ void __launch_bounds__(256) chan_bwd_kernel(const float* __restrict__ dc, const Tl* __restrict__ lat,
+                                                       const Tc* __restrict__ cq_chan, const Tc* __restrict__ ck_chan,
+                                                       const Tc* __restrict__ cq_seq, const Tc* __restrict__ ck_seq,
+                                                       float* __restrict__ ds, float* __restrict__ s_out, int S,
+                                                       int nq, int nkv, int d, int K) {
+  const long long row = blockIdx.x;
+  const int t = (int)(row % S);
+  const int Lq = nq * d, Lkv = nkv * d, Nlat = Lq + 2 * Lkv, W = Lq + Lkv;
+  for (int e = threadIdx.x; e < W; e += blockDim.x) {
+    const bool isq = e < Lq;
+    const int c = isq ? e : e - Lq;
+    const int h = c / d, jj = c % d;
+    const Tc* Wc = (isq ? cq_chan : ck_chan) + (long long)h * d * d;
+    const float* dcr = dc + row * W + (isq ? 0 : Lq) + h * d;
+    float acc = 0.f;
+    for (int i = 0; i < d; ++i) acc = fmaf(ld_f(Wc + (long long)i * d + jj), dcr[i], acc);
+    ds[row * W + e] = acc;
+    const Tc* w = (isq ? cq_seq : ck_seq) + (long long)c * K;
+    const int col = isq ? c : Lq + c;
+    float sv = 0.f;
+    for (int j = 0; j < K; ++j) {
+      const int src = t - (K - 1) + j;
+      if (src >= 0) sv = fmaf(ld_f(w + j), ld_f(lat + (row - t + src) * Nlat + col), sv);
+    }
+    s_out[row * W + e] = sv;
+  }
+}
+
+// Seq-conv transpose: dlat[t, c] = dpre[t, c] + sum_j w[c][j] ds[t + K-1-j, c] (within the sequence).
+template <typename Tc>
+__global__ void __launch_bounds__(256) seq_bwd_kernel(const float* __restrict__ ds, const float* __restrict__ dpre,
+                                                      const Tc* __restrict__ cq_seq, const Tc* __restrict__ ck_seq,
+                                                      float* __restrict__ dlat, int S, int nq, int nkv, int d, int K) {
+  const long long row = blockIdx.x;
+  const int t = (int)(row % S);
+  const int Lq = nq * d, Lkv = nkv * d, Nlat = Lq + 2 * Lkv, W = Lq + Lkv;
+  for (int e = threadIdx.x; e < W; e += blockDim.x) {
+    const bool isq = e < Lq;
+    const int c = isq ? e : e - Lq;
+    const Tc* w = (isq ? cq_seq : ck_seq) + (long long)c * K;
+    float acc = dpre[row * W + e];
+    for (int j = 0; j < K; ++j) {
+      const int tt = t + K - 1 - j;
+      if (tt < S) acc = fmaf(ld_f(w + j), ds[(row - t + tt) * W + e], acc);
+    }
+    dlat[row * Nlat + e] = acc;
+  }
+}
+
+// Seq-conv tap gradients: dw[c][j] = sum over rows t of ds[t, c] z[t - K+1 + j, c] (within each
+// sequence). Block = 32 channels x 8 row slices; the slices reduce in shared memory, then atomically
+// across blocks of rows.
+template <typename Tl>
+__global__ void __launch_bounds__(256) tap_grad_kernel(const float* __restrict__ ds, const Tl* __restrict__ lat,
+                                                       float* __restrict__ dwq, float* __restrict__ dwk, int B, int S,
+                                                       int nq, int nkv, int d, int K, int rows_per_block) {
+  __shared__ float red[8][32][8];
+  const int Lq = nq * d, Lkv = nkv * d, Nlat = Lq + 2 * Lkv, W = Lq + Lkv;
+  const int e = blockIdx.x * 32 + (threadIdx.x & 31);
+  const int slice = threadIdx.x >> 5;
+  const long long T = (long long)B * S;
+  const long long r0 = (long long)blockIdx.y * rows_per_block;
+  float acc[8] = {};
+  if (e < W) {
+    const int col = e < Lq ? e : Lq + (e - Lq);
+    for (long long row = r0 + slice; row < r0 + rows_per_block && row < T; row += 8) {
+      const int t = (int)(row % S);
+      const float g = ds[row * W + e];
+      for (int j = 0; j < K && j < 8; ++j) {
+        const int src = t - (K - 1) + j;
+        if (src >= 0) acc[j] = fmaf(g, ld_f(lat + (row - t + src) * Nlat + col), acc[j]);
+      }
+    }
+  }
+#pragma unroll
+  for (int j = 0; j < 8; ++j) red[slice][threadIdx.x & 31][j] = acc[j];
+  __syncthreads();
+  if (slice == 0 && e < W) {
+    for (int j = 0; j < K && j < 8; ++j) {
+      float s = 0.f;
+      for (int sl = 0; sl < 8; ++sl) s += red[sl][threadIdx.x & 31][j];
+      float* dst = e < Lq ? dwq + (long long)e * K + j : dwk + (long long)(e - Lq) * K + j;
+      atomicAdd(dst, s);
+    }
+  }
+}
+
+size_t up256(size_t v) { return (v + 255) / 256 * 256; }
+
+}  // namespace
+
+bool backward_supported(const BlockDims& dm) {
+  // the per-token kernel keeps one row's q and K gradients in shared memory
+  return dm.K >= 1 && dm.K <= 8 && dm.d <= 128 && dm.d % 2 == 0 && dm.Lq + dm.Lkv <= 12288 &&
+         ((dm.io == DType::BF16 && dm.lat == DType::F16) || (dm.io == DType::F32 && dm.lat == DType::F32));
+}
+
+// Workspace of the backward pass after the forward's own layout: the forward's outputs y, k_cache,
+// v_cache (recomputed), then the fp32 buffers below.
+BackwardLayout backward_layout(const BlockDims& dm, size_t forward_bytes) {
+  BackwardLayout L;
+  const size_t f = sizeof(float), T = (size_t)dm.T, W = (size_t)dm.Lq + dm.Lkv;
+  size_t off = up256(forward_bytes);
+  L.y = off;
+  off = up256(off + T * dm.E * dtype_bytes(dm.out));
+  L.k_cache = off;
+  off = up256(off + T * dm.Lkv * dtype_bytes(dm.io));
+  L.v_cache = off;
+  off = up256(off + T * dm.Lkv * dtype_bytes(dm.io));
+  L.dO = off;
+  off = up256(off + f * T * dm.Lq);
+  L.lse = off;
+  off = up256(off + f * T * dm.nq);
+  L.delta = off;
+  off = up256(off + f * T * dm.nq);
+  L.dq = off;
+  off = up256(off + f * T * dm.Lq);
+  L.dk = off;
+  off = up256(off + f * T * dm.Lkv);
+  L.dv = off;
+  off = up256(off + f * T * dm.Lkv);
+  L.dc = off;
+  off = up256(off + f * T * W);
+  L.dpre = off;
+  off = up256(off + f * T * W);
+  L.ds = off;
+  off = up256(off + f * T * W);
+  L.s = off;
+  off = up256(off + f * T * W);
+  L.dlat = off;
+  off = up256(off + f * T * dm.Nlat);
+  L.total = off;
+  return L;
+}
+
+cudaError_t launch_backward(const BlockDims& dm, const BlockPtrs& p, const BackwardPtrs& g, const BackwardLayout& L,
+                            char* ws, cudaStream_t stream) {
+  cudaError_t e;
+  const long long T = dm.T;
+  const int Lq = dm.Lq, Lkv = dm.Lkv, Nlat = dm.Nlat, E = dm.E, W = Lq + Lkv, d = dm.d;
+  float* dO = reinterpret_cast<float*>(ws + L.dO);
+  float* lse = reinterpret_cast<float*>(ws + L.lse);
+  float* delta = reinterpret_cast<float*>(ws + L.delta);
+  float* dq = reinterpret_cast<float*>(ws + L.dq);
+  float* dk = reinterpret_cast<float*>(ws + L.dk);
+  float* dv = reinterpret_cast<float*>(ws + L.dv);
+  float* dc = reinterpret_cast<float*>(ws + L.dc);
+  float* dpre = reinterpret_cast<float*>(ws + L.dpre);
+  float* ds = reinterpret_cast<float*>(ws + L.ds);
+  float* s = reinterpret_cast<float*>(ws + L.s);
+  float* dlat = reinterpret_cast<float*>(ws + L.dlat);
+  const DType lt = dm.lat, it = dm.io, ot = dm.out;
+  // 1. dO = dy W_o  [T, Lq];  dW_o = dy^T O  [E, Lq]
+  if ((e = gemm({g.dy, ot}, E, 1, 0, {p.Wo, it}, 1, Lq, 0, dO, Lq, 0, (int)T, Lq, E, 1, false, stream)) != cudaSuccess)
+    return e;
+  if ((e = gemm({g.dy, ot}, 1, E, 0, {p.o, lt}, 1, Lq, 0, g.dWo, Lq, 0, E, Lq, T, 1, false, stream)) != cudaSuccess)
+    return e;
+  // 2. softmax statistics
+  {
+    const size_t smem = sizeof(float) * 2 * RB * (d + 1);
+    const dim3 grid((dm.S + RB - 1) / RB, dm.nq, dm.B);
+    if ((e = cudaFuncSetAttribute(row_stats_kernel<__half>, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem)) !=
+            cudaSuccess ||
+        (e = cudaFuncSetAttribute(row_stats_kernel<float>, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem)) !=
+            cudaSuccess)
+      return e;
+    if (lt == DType::F16)
+      row_stats_kernel<__half><<<grid, 256, smem, stream>>>(static_cast<const __half*>(p.q),
+                                                            static_cast<const __half*>(p.k_att),
+                                                            static_cast<const __half*>(p.o), dO, lse, delta, dm.S,
+                                                            dm.nq, dm.nkv, d, dm.scale);
+    else
+      row_stats_kernel<float><<<grid, 256, smem, stream>>>(static_cast<const float*>(p.q),
+                                                           static_cast<const float*>(p.k_att),
+                                                           static_cast<const float*>(p.o), dO, lse, delta, dm.S,
+                                                           dm.nq, dm.nkv, d, dm.scale);
+    if ((e = cudaGetLastError()) != cudaSuccess) return e;
+  }
+  // 3. attention backward
+  if ((e = cudaMemsetAsync(dq, 0, sizeof(float) * T * Lq, stream)) != cudaSuccess) return e;
+  {
+    const size_t smem = sizeof(float) * ((size_t)4 * AB * (d + 1) + 2 * AB * (AB + 1) + 2 * AB);
+    const dim3 grid((dm.S + AB - 1) / AB, dm.nkv, dm.B);
+    if (lt == DType::F16) {
+      auto k = attn_bwd_kernel<__half>;
+      if ((e = cudaFuncSetAttribute(k, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem)) != cudaSuccess)
+        return e;
+      k<<<grid, 256, smem, stream>>>(static_cast<const __half*>(p.q), static_cast<const __half*>(p.k_att),
+                                     static_cast<const __half*>(p.v_att), dO, lse, delta, dq, dk, dv, dm.S, dm.nq,
+                                     dm.nkv, d, dm.scale);
+    } else {
+      auto k = attn_bwd_kernel<float>;
+      if ((e = cudaFuncSetAttribute(k, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem)) != cudaSuccess)
+        return e;
+      k<<<grid, 256, smem, stream>>>(static_cast<const float*>(p.q), static_cast<const float*>(p.k_att),
+                                     static_cast<const float*>(p.v_att), dO, lse, delta, dq, dk, dv, dm.S, dm.nq,
+                                     dm.nkv, d, dm.scale);
+    }
+    if ((e = cudaGetLastError()) != cudaSuccess) return e;
+  }
+  // 4. per-token: RoPE back, QK-mean transpose, value-shift transpose
+  {
+    Theta64 th{};
+    for (int i = 0; i < d / 2; ++i) th.v[i] = pow((double)dm.rope_base, -2.0 * (double)i / (double)d);
+    token_bwd_kernel<<<(unsigned)T, 256, sizeof(float) * W, stream>>>(
+        dq, dk, dv, dc, dpre, dlat, dm.S, dm.nq, dm.nkv, d, dm.qk_mean_mode, dm.value_shift, dm.vshift_from,
+        dm.use_rope, th);
+    if ((e = cudaGetLastError()) != cudaSuccess) return e;
+  }
+  // 5. channel mix: ds = W_c^T dc (and s recomputed); dW_c[h] = sum_t dc[t,h]^T s[t,h]
+  if (lt == DType::F16 && it == DType::BF16)
+    chan_bwd_kernel<__half, __nv_bfloat16><<<(unsigned)T, 256, 0, stream>>>(
+        dc, static_cast<const __half*>(p.qkv_lat), static_cast<const __nv_bfloat16*>(p.cq_chan),
+        static_cast<const __nv_bfloat16*>(p.ck_chan), static_cast<const __nv_bfloat16*>(p.cq_seq),
+        static_cast<const __nv_bfloat16*>(p.ck_seq), ds, s, dm.S, dm.nq, dm.nkv, d, dm.K);
+  else
+    chan_bwd_kernel<float, float><<<(unsigned)T, 256, 0, stream>>>(
+        dc, static_cast<const float*>(p.qkv_lat), static_cast<const float*>(p.cq_chan),
+        static_cast<const float*>(p.ck_chan), static_cast<const float*>(p.cq_seq), static_cast<const float*>(p.ck_seq),
+        ds, s, dm.S, dm.nq, dm.nkv, d, dm.K);
+  if ((e = cudaGetLastError()) != cudaSuccess) return e;
+  // dW_c (q heads, then K heads): batch over heads; A[i][t] = dc[t][h d + i], B[j][t] = s[t][h d + j]
+  if ((e = gemm({dc, DType::F32}, 1, W, d, {s, DType::F32}, 1, W, d, g.dconvq_chan, d, (long long)d * d, d, d, T,
+                dm.nq, false, stream)) != cudaSuccess)
+    return e;
+  if ((e = gemm({dc + Lq, DType::F32}, 1, W, d, {s + Lq, DType::F32}, 1, W, d, g.dconvk_chan, d, (long long)d * d, d,
+                d, T, dm.nkv, false, stream)) != cudaSuccess)
+    return e;
+  // 6. seq conv: dlat (q and k channels) and the tap gradients
+  if (it == DType::BF16)
+    seq_bwd_kernel<__nv_bfloat16><<<(unsigned)T, 256, 0, stream>>>(
+        ds, dpre, static_cast<const __nv_bfloat16*>(p.cq_seq), static_cast<const __nv_bfloat16*>(p.ck_seq), dlat,
+        dm.S, dm.nq, dm.nkv, d, dm.K);
+  else
+    seq_bwd_kernel<float><<<(unsigned)T, 256, 0, stream>>>(ds, dpre, static_cast<const float*>(p.cq_seq),
+                                                            static_cast<const float*>(p.ck_seq), dlat, dm.S, dm.nq,
+                                                            dm.nkv, d, dm.K);
+  if ((e = cudaGetLastError()) != cudaSuccess) return e;
+  if ((e = cudaMemsetAsync(g.dconvq_seq, 0, sizeof(float) * Lq * dm.K, stream)) != cudaSuccess ||
+      (e = cudaMemsetAsync(g.dconvk_seq, 0, sizeof(float) * Lkv * dm.K, stream)) != cudaSuccess)
+    return e;
+  {
+    const int rpb = 512;
+    const dim3 grid((W + 31) / 32, (unsigned)((T + rpb - 1) / rpb));
+    if (lt == DType::F16)
+      tap_grad_kernel<__half><<<grid, 256, 0, stream>>>(ds, static_cast<const __half*>(p.qkv_lat), g.dconvq_seq,
+                                                        g.dconvk_seq, dm.B, dm.S, dm.nq, dm.nkv, d, dm.K, rpb);
+    else
+      tap_grad_kernel<float><<<grid, 256, 0, stream>>>(ds, static_cast<const float*>(p.qkv_lat), g.dconvq_seq,
+                                                       g.dconvk_seq, dm.B, dm.S, dm.nq, dm.nkv, d, dm.K, rpb);
+    if ((e = cudaGetLastError()) != cudaSuccess) return e;
+  }
+  // 7. down-projection: dx = dlat [W_q; W_k; W_v];  dW_* = dlat^T x
+  const void* Ws[3] = {p.Wq, p.Wk, p.Wv};
+  float* dWs[3] = {g.dWq, g.dWk, g.dWv};
+  const int col0[3] = {0, Lq, Lq + Lkv}, rows[3] = {Lq, Lkv, Lkv};
+  for (int i = 0; i < 3; ++i) {
+    // dx[t][e] (+)= sum_c dlat[t][col0 + c] W[c][e]
+    if ((e = gemm({dlat + col0[i], DType::F32}, Nlat, 1, 0, {Ws[i], it}, 1, E, 0, g.dx, E, 0, (int)T, E, rows[i], 1,
+                  i > 0, stream)) != cudaSuccess)
+      return e;
+    // dW[c][e] = sum_t dlat[t][col0 + c] x[t][e]
+    if ((e = gemm({dlat + col0[i], DType::F32}, 1, Nlat, 0, {p.x, it}, 1, E, 0, dWs[i], E, 0, rows[i], E, T, 1, false,
+                  stream)) != cudaSuccess)
+      return e;
+  }
+  return cudaSuccess;
+}
+
+}  // namespace cca

@@ -584,6 +584,57 @@ cca_status_t cca_decode(const cca_config_t* cfg, int cache_rows, const void* x_t
   return CCA_OK;
 }
 
+size_t cca_backward_workspace_size(const cca_config_t* cfg) {
+  BlockDims dm;
+  if (check_config(cfg, &dm) != CCA_OK || !backward_supported(dm)) return 0;
+  return backward_layout(dm, layout_of(dm).total_bytes).total;
+}
+
+cca_status_t cca_backward(const cca_config_t* cfg, const void* x, const void* W_q, const void* W_k, const void* W_v,
+                          const void* convq_seq, const void* convq_chan, const void* convk_seq,
+                          const void* convk_chan, const void* W_o, const void* dy, float* dx, float* dW_q,
+                          float* dW_k, float* dW_v, float* dconvq_seq, float* dconvq_chan, float* dconvk_seq,
+                          float* dconvk_chan, float* dW_o, void* workspace, size_t workspace_bytes, void* stream) {
+  BlockDims dm;
+  cca_status_t st = check_config(cfg, &dm);
+  if (st != CCA_OK) return st;
+  if (!backward_supported(dm))
+    return fail(CCA_ERR_UNSUPPORTED,
+                "backward needs conv_kernel 1..8, an even head_dim <= 128, n_q_heads + n_kv_heads times head_dim "
+                "<= 12288 and bf16 or fp32");
+  static const char* g_names[10] = {"dy",         "dx",          "dW_q",       "dW_k",        "dW_v",
+                                    "dconvq_seq", "dconvq_chan", "dconvk_seq", "dconvk_chan", "dW_o"};
+  const void* gp[10] = {dy, dx, dW_q, dW_k, dW_v, dconvq_seq, dconvq_chan, dconvk_seq, dconvk_chan, dW_o};
+  for (int i = 0; i < 10; ++i) {
+    if (gp[i] == nullptr) return fail(CCA_ERR_INVALID_ARG, std::string(g_names[i]) + " is NULL");
+    if (!aligned16(gp[i])) return fail(CCA_ERR_INVALID_ARG, std::string(g_names[i]) + " is not 16-byte aligned");
+  }
+  const void* ins[9] = {x, W_q, W_k, W_v, convq_seq, convq_chan, convk_seq, convk_chan, W_o};
+  static const char* in_names[9] = {"x", "W_q", "W_k", "W_v", "convq_seq", "convq_chan", "convk_seq", "convk_chan",
+                                    "W_o"};
+  for (int i = 0; i < 9; ++i) {
+    if (ins[i] == nullptr) return fail(CCA_ERR_INVALID_ARG, std::string(in_names[i]) + " is NULL");
+    if (!aligned16(ins[i])) return fail(CCA_ERR_INVALID_ARG, std::string(in_names[i]) + " is not 16-byte aligned");
+  }
+  if (workspace == nullptr) return fail(CCA_ERR_WORKSPACE, "workspace is NULL");
+  if ((reinterpret_cast<uintptr_t>(workspace) & (kAlign - 1)) != 0)
+    return fail(CCA_ERR_WORKSPACE, "workspace is not 256-byte aligned");
+  const size_t fwd = layout_of(dm).total_bytes;
+  const BackwardLayout BL = backward_layout(dm, fwd);
+  if (workspace_bytes < BL.total) return fail(CCA_ERR_WORKSPACE, "workspace smaller than cca_backward_workspace_size()");
+  char* ws = static_cast<char*>(workspace);
+  void* outs[3] = {ws + BL.y, ws + BL.k_cache, ws + BL.v_cache};
+  Resolved r;
+  BlockPtrs p;
+  if ((st = prepare(cfg, CCA_PATH_AUTO, ins, outs, nullptr, workspace, fwd, &r, &p)) != CCA_OK) return st;
+  cudaStream_t s = static_cast<cudaStream_t>(stream);
+  if ((st = run_block(r, p, s, nullptr)) != CCA_OK) return st;
+  const BackwardPtrs g{dy, dx, dW_q, dW_k, dW_v, dconvq_seq, dconvq_chan, dconvk_seq, dconvk_chan, dW_o};
+  const cudaError_t e = launch_backward(r.dm, p, g, BL, ws, s);
+  if (e != cudaSuccess) return cuda_fail("backward", e);
+  return CCA_OK;
+}
+
 cca_status_t cca_poll_device_status(void* stream) {
   DeviceInfo* di = nullptr;
   cca_status_t st = device_info(&di);

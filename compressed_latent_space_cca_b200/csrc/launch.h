@@ -131,6 +131,26 @@ bool decode_supported(const BlockDims& dm);
 size_t decode_workspace_bytes(const BlockDims& dm);  // independent of S
 cudaError_t launch_decode(const BlockDims& dm, const DecodePtrs& p, int cache_rows, cudaStream_t stream);
 
+// ---- backward of the block (fp32 arithmetic) ----
+// dL/d(input) for the gradient dy of y, from the forward's activations (BlockPtrs, recomputed by
+// the forward kernels). Every gradient is fp32 in its input's layout; dy is in `out`.
+struct BackwardPtrs {
+  const void* dy;  // [T, E]
+  float *dx, *dWq, *dWk, *dWv, *dconvq_seq, *dconvq_chan, *dconvk_seq, *dconvk_chan, *dWo;
+};
+// Byte offsets (from the workspace start) of the backward's own buffers after the forward's
+// `forward_bytes`: the forward's y, k_cache, v_cache, then fp32 dO, lse, delta, dq, dk, dv, dc
+// (channel-mix output gradient), dpre (latents' direct QK-mean gradient), ds (seq-conv output
+// gradient), s (recomputed seq-conv output) and dlat (latents' gradient).
+struct BackwardLayout {
+  size_t y, k_cache, v_cache, dO, lse, delta, dq, dk, dv, dc, dpre, ds, s, dlat, total;
+};
+// conv_kernel 1..8, head_dim <= 128 (even), io bf16 or fp32
+bool backward_supported(const BlockDims& dm);
+BackwardLayout backward_layout(const BlockDims& dm, size_t forward_bytes);
+cudaError_t launch_backward(const BlockDims& dm, const BlockPtrs& p, const BackwardPtrs& g, const BackwardLayout& L,
+                            char* ws, cudaStream_t stream);
+
 // ---- misc ----
 cudaError_t launch_wait_timeout_selftest(unsigned* dev_err, unsigned long long limit_ns, cudaStream_t stream);
 

@@ -313,6 +313,47 @@ cca_status_t cca_decode(const cca_config_t* cfg, int cache_rows,
                         void* y_t, void* k_cache, void* v_cache, void* conv_state,
                         void* workspace, size_t workspace_bytes, void* stream);
 
+/*
+ * The backward pass of one block ("Compressed Convolutional Attention",
+ * gist.science/es/paper/2510.04476: section 4 times the backward of CCGQA;
+ * what it computes is the chain rule through the forward of section 2 taken
+ * in reverse): given dy = dL/dy, the gradient of L with respect to x and to
+ * every weight, for the same inputs as cca_prefill.
+ *
+ * The forward's activations are recomputed first, by the forward's own
+ * kernels (the path AUTO picks), into the workspace; the backward's kernels
+ * then run in fp32 on the CUDA cores, reading the forward's 16-bit
+ * intermediates where cfg->dtype is bf16.
+ *
+ *   x ... W_o   as in cca_prefill, cfg->dtype
+ *   dy          [B, S, E]              cfg->out_dtype
+ *   dx          [B, S, E] out          fp32
+ *   dW_q        [Lq, E] out, dW_k and dW_v [Lkv, E] out     fp32
+ *   dconvq_seq  [Lq, K], dconvq_chan [n_q, d, d] out        fp32
+ *   dconvk_seq  [Lkv, K], dconvk_chan [n_kv, d, d] out      fp32
+ *   dW_o        [E, Lq] out            fp32
+ *   workspace   >= cca_backward_workspace_size(cfg) bytes, 256-byte aligned,
+ *               need not start at zero
+ * Every output is overwritten (not accumulated). Supported: conv_kernel 1..8,
+ * even head_dim <= 128, dtype bf16 or fp32, and what cca_prefill supports for
+ * cfg; all pointers 16-byte aligned, no output aliasing another buffer.
+ * cca_backward_workspace_size returns 0 for an unsupported or invalid cfg.
+ * Errors: INVALID_ARG / UNSUPPORTED / WORKSPACE before any launch, CUDA if a
+ * launch fails; device-side conditions (an fp16 intermediate of the forward
+ * out of range, a bounded wait that gave up) through cca_poll_device_status.
+ */
+size_t cca_backward_workspace_size(const cca_config_t* cfg);
+cca_status_t cca_backward(const cca_config_t* cfg,
+                          const void* x,
+                          const void* W_q, const void* W_k, const void* W_v,
+                          const void* convq_seq, const void* convq_chan,
+                          const void* convk_seq, const void* convk_chan,
+                          const void* W_o, const void* dy,
+                          float* dx, float* dW_q, float* dW_k, float* dW_v,
+                          float* dconvq_seq, float* dconvq_chan,
+                          float* dconvk_seq, float* dconvk_chan, float* dW_o,
+                          void* workspace, size_t workspace_bytes, void* stream);
+
 /* Synchronizes `stream`, then reports and clears the device error word:
  * CCA_ERR_DEVICE_TIMEOUT if a bounded wait in a kernel gave up since the last
  * poll, CCA_ERR_NUMERIC_RANGE if a finite fp16 intermediate overflowed (its

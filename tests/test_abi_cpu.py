@@ -158,3 +158,31 @@ def test_decode_argument_checks():
     assert call(c=plain) == cca.CCA_ERR_INVALID_ARG  # a plain block has no conv state
     assert "plain block" in lib.cca_last_error_message().decode()
     assert call(c=good(seq_len=10, head_dim=16, hidden=64)) == cca.CCA_ERR_UNSUPPORTED
+
+
+def test_backward_workspace_and_argument_checks():
+    """The backward's workspace holds the forward's and its own fp32 buffers; shapes it does not take
+    report 0; every argument error is reported before any launch (no GPU here)."""
+    cfg = good(seq_len=100)
+    n = cca.backward_workspace_size(cfg)
+    assert n > cca.workspace_size(cfg)
+    assert cca.backward_workspace_size(good(seq_len=200)) > n
+    assert cca.backward_workspace_size(good(conv_kernel=0, qk_mean_mode=0, value_shift=0)) == 0
+    assert cca.backward_workspace_size(good(conv_kernel=9)) == 0
+    assert cca.backward_workspace_size(good(batch=0)) == 0
+    lib = cca.library()
+    p = ctypes.c_void_p(256)
+
+    def call(ins=None, grads=None, w=ctypes.c_void_p(1 << 20), nw=n, c=cfg):
+        ins = ins if ins is not None else [p] * 9
+        grads = grads if grads is not None else [p] * 10
+        return lib.cca_backward(ctypes.byref(c), *ins, *grads, w, nw, None)
+    assert call(ins=[None] + [p] * 8) == cca.CCA_ERR_INVALID_ARG
+    assert call(ins=[p] * 8 + [ctypes.c_void_p(264)]) == cca.CCA_ERR_INVALID_ARG
+    assert call(grads=[None] + [p] * 9) == cca.CCA_ERR_INVALID_ARG          # dy
+    assert "dy" in lib.cca_last_error_message().decode()
+    assert call(grads=[p] * 9 + [None]) == cca.CCA_ERR_INVALID_ARG          # dW_o
+    assert call(w=None) == cca.CCA_ERR_WORKSPACE
+    assert call(w=ctypes.c_void_p(256 + 16)) == cca.CCA_ERR_WORKSPACE
+    assert call(nw=n - 1) == cca.CCA_ERR_WORKSPACE
+    assert call(c=good(conv_kernel=0, qk_mean_mode=0, value_shift=0)) == cca.CCA_ERR_UNSUPPORTED

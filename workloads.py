@@ -130,6 +130,14 @@ def make_inputs(shape: BlockShape, seed: int | None = None) -> Dict[str, torch.T
     return out
 
 
+def make_dy(shape: BlockShape, seed: int = 1) -> torch.Tensor:
+    """A seeded gradient of the block output y [B, S, E] ~ N(0, 1) in the workload dtype (the
+    upstream gradient a backward pass starts from)."""
+    g = torch.Generator().manual_seed(1_000_003 * (shape.seed + 1) + seed)
+    t = torch.randn((shape.batch, shape.seq_len, shape.hidden), generator=g, dtype=torch.float32)
+    return t.to(torch_dtype(shape.dtype)).contiguous()
+
+
 def as_float64(inputs: Dict[str, torch.Tensor]):
     """The same values as numpy float64 arrays (exact up-cast)."""
     return {k: v.to(torch.float64).numpy() for k, v in inputs.items()}
