@@ -424,6 +424,8 @@ def run_ours(args, shape):
         if (world == 1 and not args.no_mha and my_shape.dtype == "bf16" and my_shape.conv_kernel > 0 and
                 my_shape.hidden % 128 == 0):
             line["mha_baseline"] = run_mha_baseline(cca, dev, my_shape, ms_per_step)
+        if world == 1 and not args.no_backward and cca.backward_workspace_size(cfg) > 0:
+            line["backward"] = run_backward(cca, dev, my_shape, inputs, peaks)
         if world == 1 and not args.no_decode and cca.decode_workspace_size(cfg) > 0:
             line["decode"] = run_decode(cca, dev, my_shape, inputs, out, peaks)
         if world == 1 and not args.no_cpu_baseline:
@@ -479,6 +481,51 @@ def run_mha_baseline(cca, dev, shape, cca_ms_per_step, steps=10, warmup=3):
                        "out_proj": stage_ms[3]},
         "cca_speedup": ms / cca_ms_per_step,
     }
+
+
+def backward_flops(shape: workloads.BlockShape):
+    """Algorithmic FLOPs of cca_backward: the forward it recomputes, then per projection two GEMMs of
+    the forward's size (the input and the weight gradients) and, for the causal attention, five
+    products of the forward's QK^T size (S and dP recomputed, dV, dK, dQ)."""
+    w = algorithmic_work(shape)
+    fwd = w["down_proj_flops"] + w["attention_flops"] + w["out_proj_flops"]
+    attn_bwd = 2.5 * w["attention_flops"]
+    gemm_bwd = 2.0 * (w["down_proj_flops"] + w["out_proj_flops"])
+    return {"forward": fwd, "attention_backward": attn_bwd, "projections_backward": gemm_bwd,
+            "total": fwd + attn_bwd + gemm_bwd}
+
+
+def run_backward(cca, dev, shape, inputs, peaks, steps=5, warmup=3):
+    """cca_backward (the forward recomputed, then every gradient) at the workload, dL/dy seeded,
+    timed with CUDA events around each call with L2 flushed before it."""
+    cfg = cca.config_from_shape(shape)
+    dy = workloads.make_dy(shape).to(dev)
+    ws = torch.empty(cca.backward_workspace_size(cfg), dtype=torch.uint8, device=dev)
+    grads = {n: torch.empty(tuple(inputs[n].shape), dtype=torch.float32, device=dev) for n in cca.GRAD_NAMES}
+    flush = torch.empty(L2_FLUSH_BYTES, dtype=torch.uint8, device=dev)
+    for _ in range(warmup):
+        flush.zero_()
+        cca.backward(cfg, inputs, dy, grads=grads, workspace=ws)
+    evs = [(torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)) for _ in range(steps)]
+    torch.cuda.synchronize()
+    stream = torch.cuda.current_stream(dev)
+    for i in range(steps):
+        flush.zero_()
+        evs[i][0].record(stream)
+        cca.backward(cfg, inputs, dy, grads=grads, workspace=ws)
+        evs[i][1].record(stream)
+    torch.cuda.synchronize()
+    if cca.poll_device_status() != 0:
+        raise SystemExit("device status error in the backward timing")
+    ms = float(np.mean([a.elapsed_time(b) for a, b in evs]))
+    fl = backward_flops(shape)
+    peak = float(peaks.get("bf16_tflops", FALLBACK_PEAKS["bf16_tflops"]))
+    tflops = fl["total"] / (ms / 1e3) / 1e12
+    del ws, grads, flush, dy
+    torch.cuda.empty_cache()
+    return {"ms_per_step": ms, "tokens_per_s": shape.tokens / (ms / 1e3), "steps": steps, "warmup": warmup,
+            "includes": "forward recompute + all gradients", "flops": fl, "tflops": tflops,
+            "frac_of_bf16_peak": tflops / peak, "timing": "CUDA events, L2 flushed before each call"}
 
 
 def decode_bytes(shape: workloads.BlockShape, t: int) -> float:
@@ -639,6 +686,7 @@ def main(argv=None):
     ap.add_argument("--no-mha", action="store_true",
                     help="skip timing the plain multi-head block of the same shape (the uncompressed baseline)")
     ap.add_argument("--no-decode", action="store_true", help="skip timing one decode step at position S - 1")
+    ap.add_argument("--no-backward", action="store_true", help="skip timing the backward pass (cca_backward)")
     ap.add_argument("--decode-only", action="store_true",
                     help="time only the decode step at position S - 1 after one prefill (profiling runs)")
     ap.add_argument("--preproc", choices=sorted(PREPROC_PATHS), default="auto",

@@ -111,6 +111,9 @@ struct AttnParams {
   int nsplit;
   int* split_cnt;  // [nsplit][2 tiles][8 softmax warps], zero at launch
   float* part;     // [nsplit][2 halves][2 tiles][PART_TILE]
+  // optional: base-2 log-sum-exp of every row's scaled scores, lse2[(b * nq + h) * lse_stride + t]
+  float* lse2;
+  int lse_stride;
 };
 
 // Per-CTA work lists: CTA c runs items[off[c] .. off[c+1]). An entry is a pair index in its low 12
@@ -499,6 +502,14 @@ __global__ void __launch_bounds__(NUM_THREADS, 1) attn_tc_kernel(const __grid_co
         lb += __shfl_xor_sync(0xffffffffu, lb, 1);
         la += __shfl_xor_sync(0xffffffffu, la, 2);
         lb += __shfl_xor_sync(0xffffffffu, lb, 2);
+        // the rows' log-sum-exp (a half of a split pair leaves it to the merge below): the sums are
+        // relative to the running max, so lse2 = max + log2(sum)
+        float* lse_row = p.lse2 != nullptr ? p.lse2 + ((size_t)it.b * p.nq + it.h[j]) * p.lse_stride : nullptr;
+        const int ta = qt * TQ + ra, tb = qt * TQ + rb;
+        if (lse_row != nullptr && it.half == 0 && qd == 0) {
+          if (ta < p.S) lse_row[ta] = ma + log2f(la);
+          if (tb < p.S) lse_row[tb] = mb + log2f(lb);
+        }
         if (!mbar_wait_bounded(smem_u32(&o_full[j]), ocount & 1, p.err, abort_flag, wait_site(kSiteAttn, 3, 11))) goto done;
         ++ocount;
         tc_fence_after();
@@ -543,18 +554,25 @@ __global__ void __launch_bounds__(NUM_THREADS, 1) attn_tc_kernel(const __grid_co
           if (store) {
             __threadfence();
             const bool first = it.half == 1;  // this half holds O_first
-            auto coeffs = [&](int row, float m, float l, float& c1, float& c2) {
+            auto coeffs = [&](int row, float m, float l, float& c1, float& c2, float& lse) {
               const float mo = __ldcg(other + D * TQ + row), lo = __ldcg(other + D * TQ + TQ + row);
               const float m1 = first ? m : mo, l1 = first ? l : lo;
               const float m2 = first ? mo : m, l2 = first ? lo : l;
               const float mm = fmaxf(m1, m2);
               const float e1 = fast_exp2(m1 - mm), e2 = fast_exp2(m2 - mm);
-              const float rl = 1.f / __fmaf_rn(e1, l1, __fmul_rn(e2, l2));
+              const float lsum = __fmaf_rn(e1, l1, __fmul_rn(e2, l2));
+              const float rl = 1.f / lsum;
               c1 = __fmul_rn(e1, rl);
               c2 = __fmul_rn(e2, rl);
+              lse = mm + log2f(lsum);
             };
-            coeffs(ra, ma, la, c1a, c2a);
-            coeffs(rb, mb, lb, c1b, c2b);
+            float lsea, lseb;
+            coeffs(ra, ma, la, c1a, c2a, lsea);
+            coeffs(rb, mb, lb, c1b, c2b, lseb);
+            if (lse_row != nullptr && qd == 0) {
+              if (ta < p.S) lse_row[ta] = lsea;
+              if (tb < p.S) lse_row[tb] = lseb;
+            }
             inva = invb = 1.f;  // the raw O rows are merged
           }
         }
@@ -751,7 +769,7 @@ bool attention_tc_supported(const BlockDims& dm) {
 }
 
 cudaError_t launch_attention_tc(const BlockDims& dm, const void* q, const void* k, const void* v, void* o,
-                                void* scratch, unsigned* dev_err, cudaStream_t stream) {
+                                void* scratch, unsigned* dev_err, cudaStream_t stream, float* lse2, int lse_stride) {
   if (!attention_tc_supported(dm)) return cudaErrorInvalidValue;
   AttnMaps maps;
   if (!encode_3d(&maps.q, q, (uint64_t)dm.Lq, (uint64_t)dm.S, (uint64_t)dm.B) ||
@@ -772,6 +790,8 @@ cudaError_t launch_attention_tc(const BlockDims& dm, const void* q, const void* 
   p.scale_log2 = dm.scale * 1.4426950408889634f;
   p.o = static_cast<__half*>(o);
   p.err = dev_err;
+  p.lse2 = lse2;
+  p.lse_stride = lse_stride;
   int grid = p.items < num_sms() ? p.items : num_sms();
   if (grid > MAX_CTAS) grid = MAX_CTAS;
   p.split_cnt = static_cast<int*>(scratch);

@@ -260,6 +260,30 @@ __global__ void __launch_bounds__(256, 2) row_stats_kernel(const Tl* __restrict_
   }
 }
 
+// dO in fp16 for the tensor-core attention backward, and delta_t = sum_i dO[t,h,i] O[t,h,i] in the
+// [B][nq][stride] layout it reads. A warp per (row, head) of head_dim 128: four columns a lane.
+__global__ void __launch_bounds__(256) do_prep_kernel(const float* __restrict__ dO, const __half* __restrict__ o,
+                                                      __half* __restrict__ dO16, float* __restrict__ delta, long long T,
+                                                      int S, int nq, int stride) {
+  const long long wid = (long long)blockIdx.x * 8 + (threadIdx.x >> 5);
+  const int lane = threadIdx.x & 31;
+  if (wid >= T * nq) return;
+  const long long row = wid / nq;
+  const int h = (int)(wid % nq);
+  const long long off = row * nq * 128 + h * 128 + lane * 4;
+  const float4 g = *reinterpret_cast<const float4*>(dO + off);
+  const uint2 ov = *reinterpret_cast<const uint2*>(o + off);
+  const __half2 o01 = *reinterpret_cast<const __half2*>(&ov.x), o23 = *reinterpret_cast<const __half2*>(&ov.y);
+  float dl = g.x * __low2float(o01) + g.y * __high2float(o01) + g.z * __low2float(o23) + g.w * __high2float(o23);
+  *reinterpret_cast<uint2*>(dO16 + off) = make_uint2(pack_f16x2(g.x, g.y), pack_f16x2(g.z, g.w));
+#pragma unroll
+  for (int m = 16; m > 0; m >>= 1) dl += __shfl_xor_sync(0xffffffffu, dl, m);
+  if (lane == 0) {
+    const long long b = row / S, t = row % S;
+    delta[(b * nq + h) * stride + t] = dl;
+  }
+}
+
 // ------------------------------------------------------------------ attention backward --
 // A CTA per (64-key block j, KV group g, sequence b). For each query head h of the group and each
 // 64-query block i >= j: S = scale q_i k_j^T, P = exp(S - lse) (causal), dV_j += P^T dO_i,
@@ -563,6 +587,106 @@ __global__ void __launch_bounds__(256) tap_grad_kernel(const float* __restrict__
   }
 }
 
+// Operands of the tensor-core GEMMs are bf16. A value v that bf16 does not hold exactly is carried as
+// the pair hi = bf16(v), lo = bf16(v - hi) (about 16 significant bits, bf16's exponent range), laid
+// side by side along the contraction so that one GEMM with a K two or three times longer sums
+// hi*b + lo*b; the other operand repeats its bf16 values over the same segments ("Leveraging the
+// bfloat16 artificial intelligence datatype for higher-precision computations", Henry et al., 2019).
+enum SegKind : int { kSegNone = 0, kSegHi = 1, kSegLo = 2 };
+struct Segs {
+  int kind[3];
+  long long off[3];  // element offset of each segment along the contraction
+};
+constexpr Segs kOneHi = {{kSegHi, kSegNone, kSegNone}, {0, 0, 0}};
+__host__ __device__ constexpr Segs segs2(int k0, int k1, long long off1) { return {{k0, k1, kSegNone}, {0, off1, 0}}; }
+__host__ __device__ constexpr Segs segs3(int k0, int k1, int k2, long long off) {
+  return {{k0, k1, k2}, {0, off, 2 * off}};
+}
+
+__device__ __forceinline__ __nv_bfloat16 seg_value(float v, int kind) {
+  const __nv_bfloat16 hi = __float2bfloat16_rn(v);
+  return kind == kSegLo ? __float2bfloat16_rn(v - __bfloat162float(hi)) : hi;
+}
+
+// Transposed: out[c * ldo + seg.off + r] = segment of in[r * ldi + c] for r < R, zero for R <= r < Rp
+// (the padding of a contraction dimension). Row-major (rm non-null): rm[r * ldrm + rseg.off + c]. 32 x 32
+// tiles through shared memory; rows of `in` run along grid x.
+template <typename Ti>
+__global__ void __launch_bounds__(256) transpose_bf16_kernel(const Ti* __restrict__ in, long long ldi, int R, int C,
+                                                             int Rp, __nv_bfloat16* __restrict__ out, long long ldo,
+                                                             Segs seg, __nv_bfloat16* __restrict__ rm, long long ldrm,
+                                                             Segs rseg) {
+  __shared__ float tile[32][33];
+  const long long r0 = (long long)blockIdx.x * 32;
+  const int c0 = blockIdx.y * 32;
+  const int tx = threadIdx.x & 31, ty = threadIdx.x >> 5;
+  for (int i = ty; i < 32; i += 8) {
+    const long long r = r0 + i;
+    const int c = c0 + tx;
+    float v = 0.f;
+    if (r < R && c < C) {
+      v = ld_f(in + r * ldi + c);
+      if (rm != nullptr) {
+#pragma unroll
+        for (int k = 0; k < 3; ++k)
+          if (rseg.kind[k] != kSegNone) rm[r * ldrm + rseg.off[k] + c] = seg_value(v, rseg.kind[k]);
+      }
+    }
+    tile[i][tx] = v;
+  }
+  __syncthreads();
+  if (out == nullptr) return;
+  for (int i = ty; i < 32; i += 8) {
+    const int c = c0 + i;
+    const long long r = r0 + tx;
+    if (c < C && r < Rp) {
+      const float v = tile[tx][i];
+#pragma unroll
+      for (int k = 0; k < 3; ++k)
+        if (seg.kind[k] != kSegNone) out[(long long)c * ldo + seg.off[k] + r] = seg_value(v, seg.kind[k]);
+    }
+  }
+}
+
+cudaError_t transpose_bf16(Mat in, long long ldi, int R, int C, int Rp, __nv_bfloat16* out, long long ldo, Segs seg,
+                           __nv_bfloat16* rm = nullptr, long long ldrm = 0, Segs rseg = kOneHi,
+                           cudaStream_t s = 0) {
+  const dim3 grid((unsigned)((Rp + 31) / 32), (unsigned)((C + 31) / 32));
+  switch (in.t) {
+    case DType::F32:
+      transpose_bf16_kernel<float><<<grid, 256, 0, s>>>(static_cast<const float*>(in.p), ldi, R, C, Rp, out, ldo, seg,
+                                                        rm, ldrm, rseg);
+      break;
+    case DType::BF16:
+      transpose_bf16_kernel<__nv_bfloat16><<<grid, 256, 0, s>>>(static_cast<const __nv_bfloat16*>(in.p), ldi, R, C, Rp,
+                                                                 out, ldo, seg, rm, ldrm, rseg);
+      break;
+    case DType::F16:
+      transpose_bf16_kernel<__half><<<grid, 256, 0, s>>>(static_cast<const __half*>(in.p), ldi, R, C, Rp, out, ldo,
+                                                         seg, rm, ldrm, rseg);
+      break;
+  }
+  return cudaGetLastError();
+}
+
+// C[M, N] (fp32, row stride ldc) = A[M, K] B[N, K]^T on the tensor cores, bf16 operands
+cudaError_t gemm_tc_bf16(const void* A, long long M, const void* B, int N, int K, float* C, long long ldc,
+                         unsigned* err, cudaStream_t s) {
+  GemmTcArgs a{};
+  a.A = A;
+  a.M = M;
+  a.K = K;
+  a.B[0] = B;
+  a.nrows[0] = N;
+  a.nb = 1;
+  a.C = C;
+  a.ldc = ldc;
+  a.in = DType::BF16;
+  a.out = DType::F32;
+  a.dev_err = err;
+  return launch_gemm_tc(a, s);
+}
+
 size_t up256(size_t v) { return (v + 255) / 256 * 256; }
 
 }  // namespace
@@ -585,12 +709,16 @@ BackwardLayout backward_layout(const BlockDims& dm, size_t forward_bytes) {
   off = up256(off + T * dm.Lkv * dtype_bytes(dm.io));
   L.v_cache = off;
   off = up256(off + T * dm.Lkv * dtype_bytes(dm.io));
+  L.stat_stride = (dm.S + 127) / 128 * 128;
+  const size_t stats = (size_t)dm.B * dm.nq * L.stat_stride;  // >= T * nq, the SIMT path's layout
   L.dO = off;
   off = up256(off + f * T * dm.Lq);
+  L.dO16 = off;
+  off = up256(off + 2 * T * dm.Lq);
   L.lse = off;
-  off = up256(off + f * T * dm.nq);
+  off = up256(off + f * stats);
   L.delta = off;
-  off = up256(off + f * T * dm.nq);
+  off = up256(off + f * stats);
   L.dq = off;
   off = up256(off + f * T * dm.Lq);
   L.dk = off;
@@ -607,12 +735,33 @@ BackwardLayout backward_layout(const BlockDims& dm, size_t forward_bytes) {
   off = up256(off + f * T * W);
   L.dlat = off;
   off = up256(off + f * T * dm.Nlat);
+  // bf16 operands of the tensor-core GEMMs: transposed copies padded to Tp tokens (a multiple of the
+  // GEMM's 64-deep K step), row-major copies, transposed weights
+  L.Tp = (T + 63) / 64 * 64;
+  const size_t h = 2, Tp = (size_t)L.Tp;
+  // (up to three segments along the contraction, see Segs)
+  L.dy16 = off;
+  off = up256(off + h * T * dm.E * 2);
+  L.dy_t = off;
+  off = up256(off + h * dm.E * Tp * 3);
+  L.x_t = off;
+  off = up256(off + h * dm.E * Tp * 2);
+  L.o_t = off;
+  off = up256(off + h * dm.Lq * Tp * 3);
+  L.dlat16 = off;
+  off = up256(off + h * T * dm.Nlat * 2);
+  L.dlat_t = off;
+  off = up256(off + h * dm.Nlat * Tp * 2);
+  L.wo_t = off;
+  off = up256(off + h * dm.Lq * dm.E * 2);
+  L.w_t = off;
+  off = up256(off + h * dm.E * dm.Nlat * 2);
   L.total = off;
   return L;
 }
 
 cudaError_t launch_backward(const BlockDims& dm, const BlockPtrs& p, const BackwardPtrs& g, const BackwardLayout& L,
-                            char* ws, cudaStream_t stream) {
+                            char* ws, cudaStream_t stream, bool tc_attention, bool tc_gemm) {
   cudaError_t e;
   const long long T = dm.T;
   const int Lq = dm.Lq, Lkv = dm.Lkv, Nlat = dm.Nlat, E = dm.E, W = Lq + Lkv, d = dm.d;
@@ -628,53 +777,109 @@ cudaError_t launch_backward(const BlockDims& dm, const BlockPtrs& p, const Backw
   float* s = reinterpret_cast<float*>(ws + L.s);
   float* dlat = reinterpret_cast<float*>(ws + L.dlat);
   const DType lt = dm.lat, it = dm.io, ot = dm.out;
+  const int Tp = L.Tp;
+  __nv_bfloat16* dy16 = reinterpret_cast<__nv_bfloat16*>(ws + L.dy16);
+  __nv_bfloat16* dy_t = reinterpret_cast<__nv_bfloat16*>(ws + L.dy_t);
+  __nv_bfloat16* x_t = reinterpret_cast<__nv_bfloat16*>(ws + L.x_t);
+  __nv_bfloat16* o_t = reinterpret_cast<__nv_bfloat16*>(ws + L.o_t);
+  __nv_bfloat16* dlat16 = reinterpret_cast<__nv_bfloat16*>(ws + L.dlat16);
+  __nv_bfloat16* dlat_t = reinterpret_cast<__nv_bfloat16*>(ws + L.dlat_t);
+  __nv_bfloat16* wo_t = reinterpret_cast<__nv_bfloat16*>(ws + L.wo_t);
+  __nv_bfloat16* w_t = reinterpret_cast<__nv_bfloat16*>(ws + L.w_t);
   // 1. dO = dy W_o  [T, Lq];  dW_o = dy^T O  [E, Lq]
-  if ((e = gemm({g.dy, ot}, E, 1, 0, {p.Wo, it}, 1, Lq, 0, dO, Lq, 0, (int)T, Lq, E, 1, false, stream)) != cudaSuccess)
-    return e;
-  if ((e = gemm({g.dy, ot}, 1, E, 0, {p.o, lt}, 1, Lq, 0, g.dWo, Lq, 0, E, Lq, T, 1, false, stream)) != cudaSuccess)
-    return e;
-  // 2. softmax statistics
-  {
-    const size_t smem = sizeof(float) * 2 * RB * (d + 1);
-    const dim3 grid((dm.S + RB - 1) / RB, dm.nq, dm.B);
-    if ((e = cudaFuncSetAttribute(row_stats_kernel<__half>, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem)) !=
-            cudaSuccess ||
-        (e = cudaFuncSetAttribute(row_stats_kernel<float>, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem)) !=
-            cudaSuccess)
-      return e;
-    if (lt == DType::F16)
-      row_stats_kernel<__half><<<grid, 256, smem, stream>>>(static_cast<const __half*>(p.q),
-                                                            static_cast<const __half*>(p.k_att),
-                                                            static_cast<const __half*>(p.o), dO, lse, delta, dm.S,
-                                                            dm.nq, dm.nkv, d, dm.scale);
-    else
-      row_stats_kernel<float><<<grid, 256, smem, stream>>>(static_cast<const float*>(p.q),
-                                                           static_cast<const float*>(p.k_att),
-                                                           static_cast<const float*>(p.o), dO, lse, delta, dm.S,
-                                                           dm.nq, dm.nkv, d, dm.scale);
-    if ((e = cudaGetLastError()) != cudaSuccess) return e;
-  }
-  // 3. attention backward
-  if ((e = cudaMemsetAsync(dq, 0, sizeof(float) * T * Lq, stream)) != cudaSuccess) return e;
-  {
-    const size_t smem = sizeof(float) * ((size_t)4 * AB * (d + 1) + 2 * AB * (AB + 1) + 2 * AB);
-    const dim3 grid((dm.S + AB - 1) / AB, dm.nkv, dm.B);
-    if (lt == DType::F16) {
-      auto k = attn_bwd_kernel<__half>;
-      if ((e = cudaFuncSetAttribute(k, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem)) != cudaSuccess)
+  if (tc_gemm) {
+    // dO = dy W_o: exact bf16 products when dy is bf16; an fp32 dy is split in two segments
+    // dW_o = dy^T O: O (fp16) is split; so is an fp32 dy, with the segments [hi, hi, lo] x [hi, lo, hi]
+    const bool dy_bf16 = ot == DType::BF16;
+    const long long TpL = Tp;
+    if (dy_bf16) {
+      if ((e = transpose_bf16({g.dy, ot}, E, (int)T, E, Tp, dy_t, 2 * TpL, segs2(kSegHi, kSegHi, TpL), nullptr, 0,
+                              kOneHi, stream)) != cudaSuccess ||
+          (e = transpose_bf16({p.Wo, it}, Lq, E, Lq, E, wo_t, E, kOneHi, nullptr, 0, kOneHi, stream)) != cudaSuccess ||
+          (e = transpose_bf16({p.o, lt}, Lq, (int)T, Lq, Tp, o_t, 2 * TpL, segs2(kSegHi, kSegLo, TpL), nullptr, 0,
+                              kOneHi, stream)) != cudaSuccess)
         return e;
-      k<<<grid, 256, smem, stream>>>(static_cast<const __half*>(p.q), static_cast<const __half*>(p.k_att),
-                                     static_cast<const __half*>(p.v_att), dO, lse, delta, dq, dk, dv, dm.S, dm.nq,
-                                     dm.nkv, d, dm.scale);
+      if ((e = gemm_tc_bf16(g.dy, T, wo_t, Lq, E, dO, Lq, p.dev_err, stream)) != cudaSuccess ||
+          (e = gemm_tc_bf16(dy_t, E, o_t, Lq, 2 * Tp, g.dWo, Lq, p.dev_err, stream)) != cudaSuccess)
+        return e;
     } else {
-      auto k = attn_bwd_kernel<float>;
-      if ((e = cudaFuncSetAttribute(k, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem)) != cudaSuccess)
+      if ((e = transpose_bf16({g.dy, ot}, E, (int)T, E, Tp, dy_t, 3 * TpL, segs3(kSegHi, kSegHi, kSegLo, TpL), dy16,
+                              2LL * E, segs2(kSegHi, kSegLo, E), stream)) != cudaSuccess ||
+          (e = transpose_bf16({p.Wo, it}, Lq, E, Lq, E, wo_t, 2LL * E, segs2(kSegHi, kSegHi, E), nullptr, 0, kOneHi,
+                              stream)) != cudaSuccess ||
+          (e = transpose_bf16({p.o, lt}, Lq, (int)T, Lq, Tp, o_t, 3 * TpL, segs3(kSegHi, kSegLo, kSegHi, TpL), nullptr,
+                              0, kOneHi, stream)) != cudaSuccess)
         return e;
-      k<<<grid, 256, smem, stream>>>(static_cast<const float*>(p.q), static_cast<const float*>(p.k_att),
-                                     static_cast<const float*>(p.v_att), dO, lse, delta, dq, dk, dv, dm.S, dm.nq,
-                                     dm.nkv, d, dm.scale);
+      if ((e = gemm_tc_bf16(dy16, T, wo_t, Lq, 2 * E, dO, Lq, p.dev_err, stream)) != cudaSuccess ||
+          (e = gemm_tc_bf16(dy_t, E, o_t, Lq, 3 * Tp, g.dWo, Lq, p.dev_err, stream)) != cudaSuccess)
+        return e;
     }
-    if ((e = cudaGetLastError()) != cudaSuccess) return e;
+  } else {
+    if ((e = gemm({g.dy, ot}, E, 1, 0, {p.Wo, it}, 1, Lq, 0, dO, Lq, 0, (int)T, Lq, E, 1, false, stream)) !=
+        cudaSuccess)
+      return e;
+    if ((e = gemm({g.dy, ot}, 1, E, 0, {p.o, lt}, 1, Lq, 0, g.dWo, Lq, 0, E, Lq, T, 1, false, stream)) != cudaSuccess)
+      return e;
+  }
+  if (tc_attention) {
+    // 2. dO in fp16 and delta; the forward's tensor-core attention left lse2 (base 2)
+    {
+      const long long warps = T * dm.nq;
+      do_prep_kernel<<<(unsigned)((warps + 7) / 8), 256, 0, stream>>>(
+          dO, static_cast<const __half*>(p.o), reinterpret_cast<__half*>(ws + L.dO16), delta, T, dm.S, dm.nq,
+          L.stat_stride);
+      if ((e = cudaGetLastError()) != cudaSuccess) return e;
+    }
+    // 3. attention backward on the tensor cores (dk, dv are sums over the CTAs of a key tile)
+    if ((e = cudaMemsetAsync(dk, 0, sizeof(float) * T * Lkv, stream)) != cudaSuccess ||
+        (e = cudaMemsetAsync(dv, 0, sizeof(float) * T * Lkv, stream)) != cudaSuccess)
+      return e;
+    AttnBwdPtrs a{p.q, p.k_att, p.v_att, ws + L.dO16, lse, delta, L.stat_stride, dq, dk, dv};
+    if ((e = launch_attention_bwd_tc(dm, a, p.dev_err, stream)) != cudaSuccess) return e;
+  } else {
+    // 2. softmax statistics
+    {
+      const size_t smem = sizeof(float) * 2 * RB * (d + 1);
+      const dim3 grid((dm.S + RB - 1) / RB, dm.nq, dm.B);
+      if ((e = cudaFuncSetAttribute(row_stats_kernel<__half>, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem)) !=
+              cudaSuccess ||
+          (e = cudaFuncSetAttribute(row_stats_kernel<float>, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem)) !=
+              cudaSuccess)
+        return e;
+      if (lt == DType::F16)
+        row_stats_kernel<__half><<<grid, 256, smem, stream>>>(static_cast<const __half*>(p.q),
+                                                              static_cast<const __half*>(p.k_att),
+                                                              static_cast<const __half*>(p.o), dO, lse, delta, dm.S,
+                                                              dm.nq, dm.nkv, d, dm.scale);
+      else
+        row_stats_kernel<float><<<grid, 256, smem, stream>>>(static_cast<const float*>(p.q),
+                                                             static_cast<const float*>(p.k_att),
+                                                             static_cast<const float*>(p.o), dO, lse, delta, dm.S,
+                                                             dm.nq, dm.nkv, d, dm.scale);
+      if ((e = cudaGetLastError()) != cudaSuccess) return e;
+    }
+    // 3. attention backward
+    if ((e = cudaMemsetAsync(dq, 0, sizeof(float) * T * Lq, stream)) != cudaSuccess) return e;
+    {
+      const size_t smem = sizeof(float) * ((size_t)4 * AB * (d + 1) + 2 * AB * (AB + 1) + 2 * AB);
+      const dim3 grid((dm.S + AB - 1) / AB, dm.nkv, dm.B);
+      if (lt == DType::F16) {
+        auto k = attn_bwd_kernel<__half>;
+        if ((e = cudaFuncSetAttribute(k, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem)) != cudaSuccess)
+          return e;
+        k<<<grid, 256, smem, stream>>>(static_cast<const __half*>(p.q), static_cast<const __half*>(p.k_att),
+                                       static_cast<const __half*>(p.v_att), dO, lse, delta, dq, dk, dv, dm.S, dm.nq,
+                                       dm.nkv, d, dm.scale);
+      } else {
+        auto k = attn_bwd_kernel<float>;
+        if ((e = cudaFuncSetAttribute(k, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem)) != cudaSuccess)
+          return e;
+        k<<<grid, 256, smem, stream>>>(static_cast<const float*>(p.q), static_cast<const float*>(p.k_att),
+                                       static_cast<const float*>(p.v_att), dO, lse, delta, dq, dk, dv, dm.S, dm.nq,
+                                       dm.nkv, d, dm.scale);
+      }
+      if ((e = cudaGetLastError()) != cudaSuccess) return e;
+    }
   }
   // 4. per-token: RoPE back, QK-mean transpose, value-shift transpose
   {
@@ -732,6 +937,26 @@ cudaError_t launch_backward(const BlockDims& dm, const BlockPtrs& p, const Backw
   const void* Ws[3] = {p.Wq, p.Wk, p.Wv};
   float* dWs[3] = {g.dWq, g.dWk, g.dWv};
   const int col0[3] = {0, Lq, Lq + Lkv}, rows[3] = {Lq, Lkv, Lkv};
+  if (tc_gemm) {
+    // dlat (fp32) split in two segments, row-major for dx and transposed for dW; x and the weights
+    // are exact in bf16 and repeat over both segments
+    const long long TpL = Tp;
+    if ((e = transpose_bf16({dlat, DType::F32}, Nlat, (int)T, Nlat, Tp, dlat_t, 2 * TpL, segs2(kSegHi, kSegLo, TpL),
+                            dlat16, 2LL * Nlat, segs2(kSegHi, kSegLo, Nlat), stream)) != cudaSuccess ||
+        (e = transpose_bf16({p.x, it}, E, (int)T, E, Tp, x_t, 2 * TpL, segs2(kSegHi, kSegHi, TpL), nullptr, 0, kOneHi,
+                            stream)) != cudaSuccess)
+      return e;
+    for (int i = 0; i < 3; ++i)
+      if ((e = transpose_bf16({Ws[i], it}, E, rows[i], E, rows[i], w_t + col0[i], 2LL * Nlat,
+                              segs2(kSegHi, kSegHi, Nlat), nullptr, 0, kOneHi, stream)) != cudaSuccess)
+        return e;
+    if ((e = gemm_tc_bf16(dlat16, T, w_t, E, 2 * Nlat, g.dx, E, p.dev_err, stream)) != cudaSuccess) return e;
+    for (int i = 0; i < 3; ++i)
+      if ((e = gemm_tc_bf16(dlat_t + (size_t)col0[i] * 2 * Tp, rows[i], x_t, E, 2 * Tp, dWs[i], E, p.dev_err,
+                            stream)) != cudaSuccess)
+        return e;
+    return cudaSuccess;
+  }
   for (int i = 0; i < 3; ++i) {
     // dx[t][e] (+)= sum_c dlat[t][col0 + c] W[c][e]
     if ((e = gemm({dlat + col0[i], DType::F32}, Nlat, 1, 0, {Ws[i], it}, 1, E, 0, g.dx, E, 0, (int)T, E, rows[i], 1,

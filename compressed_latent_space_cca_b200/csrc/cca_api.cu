@@ -297,7 +297,8 @@ cca_status_t run_block(const Resolved& r, BlockPtrs p, cudaStream_t stream, void
   if ((e = mark(2)) != cudaSuccess) return cuda_fail("event", e);
   // 3. causal attention on the compressed heads
   if (r.tc_attn) {
-    if ((e = launch_attention_tc(dm, p.q, p.k_att, p.v_att, p.o, p.sched, p.dev_err, stream)) != cudaSuccess)
+    if ((e = launch_attention_tc(dm, p.q, p.k_att, p.v_att, p.o, p.sched, p.dev_err, stream, p.lse2,
+                                 p.lse_stride)) != cudaSuccess)
       return cuda_fail("attention (tcgen05)", e);
   } else {
     if ((e = launch_attention_simt(dm, p.q, p.k_att, p.v_att, p.o, stream)) != cudaSuccess)
@@ -378,6 +379,8 @@ cca_status_t prepare(const cca_config_t* cfg, int path, const void* const* ins, 
   p->wc_lat = sep ? ws + L.wc_offset : nullptr;
   p->sched = ws + L.sched_offset;
   p->dev_err = nullptr;
+  p->lse2 = nullptr;
+  p->lse_stride = 0;
   // the conv state keeps the last v~ row, which the fused value shift does not write; the fused
   // epilogue shifts whole 64-channel groups
   p->v_fused = r->v_fuse && conv_state == nullptr && r->dm.vshift_from % 64 == 0;
@@ -628,9 +631,18 @@ cca_status_t cca_backward(const cca_config_t* cfg, const void* x, const void* W_
   BlockPtrs p;
   if ((st = prepare(cfg, CCA_PATH_AUTO, ins, outs, nullptr, workspace, fwd, &r, &p)) != CCA_OK) return st;
   cudaStream_t s = static_cast<cudaStream_t>(stream);
+  // the tensor-core attention backward reads the log-sum-exp rows the forward's attention leaves
+  const bool tc_bwd = r.tc_attn && attention_bwd_tc_supported(r.dm);
+  if (tc_bwd) {
+    p.lse2 = reinterpret_cast<float*>(ws + BL.lse);
+    p.lse_stride = BL.stat_stride;
+  }
   if ((st = run_block(r, p, s, nullptr)) != CCA_OK) return st;
+  DeviceInfo* di = nullptr;
+  if ((st = device_info(&di)) != CCA_OK) return st;
+  p.dev_err = di->err_ptr;  // the backward kernels' bounded waits and range checks report here
   const BackwardPtrs g{dy, dx, dW_q, dW_k, dW_v, dconvq_seq, dconvq_chan, dconvk_seq, dconvk_chan, dW_o};
-  const cudaError_t e = launch_backward(r.dm, p, g, BL, ws, s);
+  const cudaError_t e = launch_backward(r.dm, p, g, BL, ws, s, tc_bwd, r.tc_down && r.tc_out);
   if (e != cudaSuccess) return cuda_fail("backward", e);
   return CCA_OK;
 }
@@ -651,10 +663,11 @@ cca_status_t cca_poll_device_status(void* stream) {
       return cuda_fail("clear device error word", e);
     if ((h & 0xffu) == kDevErrRange)
       return fail(CCA_ERR_NUMERIC_RANGE, "an intermediate exceeded the fp16 range (|value| > 65504)");
-    static const char* kernels[6] = {"?", "gemm", "attention", "self-test", "?", "preprocessing (tcgen05)"};
+    static const char* kernels[7] = {"?",         "gemm", "attention", "self-test", "?", "preprocessing (tcgen05)",
+                                     "attention backward"};
     char msg[160];
     snprintf(msg, sizeof(msg), "a bounded device-side wait gave up (kernel %s, role %u, barrier %u)",
-             kernels[((h >> 8) & 0xffu) < 6 ? ((h >> 8) & 0xffu) : 0], (h >> 16) & 0xffu, (h >> 24) & 0xffu);
+             kernels[((h >> 8) & 0xffu) < 7 ? ((h >> 8) & 0xffu) : 0], (h >> 16) & 0xffu, (h >> 24) & 0xffu);
     return fail(CCA_ERR_DEVICE_TIMEOUT, msg);
   }
   return CCA_OK;

@@ -116,7 +116,14 @@ __device__ __forceinline__ bool mbar_try_wait(uint32_t bar, uint32_t parity) {
 __host__ __device__ constexpr unsigned wait_site(unsigned kernel, unsigned role, unsigned barrier) {
   return (kernel << 8) | (role << 16) | (barrier << 24);
 }
-enum WaitKernel : unsigned { kSiteGemm = 1, kSiteAttn = 2, kSiteSelftest = 3, kSitePreUmma = 4, kSitePreWs = 5 };
+enum WaitKernel : unsigned {
+  kSiteGemm = 1,
+  kSiteAttn = 2,
+  kSiteSelftest = 3,
+  kSitePreUmma = 4,
+  kSitePreWs = 5,
+  kSiteAttnBwd = 6
+};
 
 // Waits for phase `parity` of the mbarrier to complete. Gives up after
 // kWaitTimeoutNs (or as soon as *abort is set by another warp of the CTA),

@@ -47,6 +47,10 @@ struct BlockPtrs {
   void* sched;    // scratch of the tensor-core attention (split-pair counters, partial rows)
   unsigned* dev_err;
   bool v_fused;   // the down-projection has written the V cache and v_att (value shift in its epilogue)
+  // optional (non-null): the tensor-core attention also leaves the base-2 log-sum-exp of each row,
+  // lse2[(b * nq + h) * lse_stride + t] = log2 sum_s 2^(scale log2(e) q_t . k_s)
+  float* lse2;
+  int lse_stride;
 };
 
 // ---- SIMT path (any dtype, any even head_dim <= 128) ----
@@ -111,7 +115,20 @@ cudaError_t launch_convert_f16(const void* src, void* dst, long long n, unsigned
 
 bool attention_tc_supported(const BlockDims& dm);
 cudaError_t launch_attention_tc(const BlockDims& dm, const void* q, const void* k, const void* v, void* o,
-                                void* scratch, unsigned* dev_err, cudaStream_t stream);
+                                void* scratch, unsigned* dev_err, cudaStream_t stream, float* lse2 = nullptr,
+                                int lse_stride = 0);
+// Attention backward on the tensor cores (head_dim 128, fp16 operands): dq written, dk and dv added
+// to (fp32, [B, S, width], scale applied); lse2 and delta [B][nq][stat_stride] (stat_stride a
+// multiple of 64, >= S).
+struct AttnBwdPtrs {
+  const void *q, *k, *v, *dO;  // fp16, the forward's attention inputs and dL/dO
+  const float *lse2, *delta;
+  int stat_stride;
+  float *dq, *dk, *dv;
+};
+bool attention_bwd_tc_supported(const BlockDims& dm);
+cudaError_t launch_attention_bwd_tc(const BlockDims& dm, const AttnBwdPtrs& a, unsigned* dev_err,
+                                    cudaStream_t stream);
 // Split-pair scratch of the tensor-core attention: kAttnSplitCounters ints that must be zero when
 // it starts (the preprocessing kernels clear them), then the partial rows.
 constexpr int kAttnMaxSplit = 64;
@@ -139,17 +156,24 @@ struct BackwardPtrs {
   float *dx, *dWq, *dWk, *dWv, *dconvq_seq, *dconvq_chan, *dconvk_seq, *dconvk_chan, *dWo;
 };
 // Byte offsets (from the workspace start) of the backward's own buffers after the forward's
-// `forward_bytes`: the forward's y, k_cache, v_cache, then fp32 dO, lse, delta, dq, dk, dv, dc
-// (channel-mix output gradient), dpre (latents' direct QK-mean gradient), ds (seq-conv output
-// gradient), s (recomputed seq-conv output) and dlat (latents' gradient).
+// `forward_bytes`: the forward's y, k_cache, v_cache, then fp32 dO, its fp16 copy dO16, lse, delta,
+// dq, dk, dv, dc (channel-mix output gradient), dpre (latents' direct QK-mean gradient), ds
+// (seq-conv output gradient), s (recomputed seq-conv output) and dlat (latents' gradient).
 struct BackwardLayout {
-  size_t y, k_cache, v_cache, dO, lse, delta, dq, dk, dv, dc, dpre, ds, s, dlat, total;
+  size_t y, k_cache, v_cache, dO, dO16, lse, delta, dq, dk, dv, dc, dpre, ds, s, dlat;
+  // bf16 operands of the tensor-core GEMMs (token dimension padded to Tp in the transposed copies)
+  size_t dy16, dy_t, x_t, o_t, dlat16, dlat_t, wo_t, w_t;
+  size_t total;
+  int stat_stride;  // lse / delta rows of the tensor-core path: [B][nq][stat_stride]
+  int Tp;           // tokens rounded up to a multiple of 64
 };
 // conv_kernel 1..8, head_dim <= 128 (even), io bf16 or fp32
 bool backward_supported(const BlockDims& dm);
 BackwardLayout backward_layout(const BlockDims& dm, size_t forward_bytes);
+// tc_attention: the forward ran the tensor-core attention with p.lse2 set (BackwardLayout::lse);
+// tc_gemm: the projections' shapes suit the tensor-core GEMM (bf16 blocks on sm_100)
 cudaError_t launch_backward(const BlockDims& dm, const BlockPtrs& p, const BackwardPtrs& g, const BackwardLayout& L,
-                            char* ws, cudaStream_t stream);
+                            char* ws, cudaStream_t stream, bool tc_attention, bool tc_gemm);
 
 // ---- misc ----
 cudaError_t launch_wait_timeout_selftest(unsigned* dev_err, unsigned long long limit_ns, cudaStream_t stream);

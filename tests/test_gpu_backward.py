@@ -31,10 +31,12 @@ def _err(gpu, ref):
     return float(e.max()), float(e.mean())
 
 
-def _run(shape, kv_split=None):
+def _run(shape, kv_split=None, out_dtype=None):
     inp = workloads.make_inputs(shape)
     dy = workloads.make_dy(shape)
-    cfg = cca.config_from_shape(shape)
+    if out_dtype == "f32":
+        dy = dy.float()
+    cfg = cca.config_from_shape(shape, out_dtype)
     vfrom = None
     if kv_split is not None:  # one rank's share of a block twice as wide in KV groups
         rank, world = kv_split
@@ -90,12 +92,21 @@ BF16_CASES = [
     S_("bf16_pre_mean", 2, 96, 256, 2, 2, 128, 4, "bf16", qk_mean_mode=1),  # mma.sync preprocessing
     S_("bf16_simt_d64", 1, 130, 128, 2, 1, 64, 3, "bf16"),     # SIMT forward
     S_("bf16_1k", 1, 1024, 1024, 4, 2, 128, 4, "bf16"),
+    S_("bf16_g4_split", 1, 1600, 1024, 8, 2, 128, 4, "bf16"),   # key tiles split over CTAs, ragged
+    S_("bf16_b2_mha", 2, 333, 512, 4, 4, 128, 3, "bf16"),       # G = 1, two sequences, ragged
 ]
 
 
 @pytest.mark.parametrize("shape", BF16_CASES, ids=[s.name for s in BF16_CASES])
 def test_backward_bf16_matches_oracle(shape):
     got, ref = _run(shape)
+    _check(shape, got, ref)
+
+
+def test_backward_bf16_block_fp32_output():
+    """A bf16 block whose y (so dy) is fp32: the GEMM operands are converted to bf16 first."""
+    shape = BF16_CASES[0]
+    got, ref = _run(shape, out_dtype="f32")
     _check(shape, got, ref)
 
 
