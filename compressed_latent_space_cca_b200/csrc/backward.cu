@@ -497,8 +497,129 @@ __global__ void __launch_bounds__(256) token_bwd_kernel(const float* __restrict_
   }
 }
 
-// Channel mix transpose and the recomputed seq-conv output: per row t, per head (q heads then K
-// heads) ds[t] = W_c^T dc[t] and s[t] = seq_conv(z)[t]. Block = one row; thread = one channel.
+// Channel-mix backward of one head over a block of rows: ds[t] = W_c^T dc[t] and the block's share
+// of dW_c = sum_t dc[t]^T s[t], s being the seq-conv output recomputed from the latents. A CTA per
+// (CM_ROWS-row block, head; q heads then K heads), head_dim 128: W_c in shared memory, then 32-row
+// sub-blocks of dc (row-major and transposed) and s; each thread owns 4 x 4 outputs of ds and an
+// 8 x 8 patch of dW_c, added to the fp32 sum with vector atomics at the end.
+constexpr int CM_ROWS = 256, CM_SUB = 32, CM_D = 128, CM_KMAX = 8;
+constexpr size_t CM_SMEM = sizeof(float) * ((size_t)CM_D * CM_D + 2 * CM_SUB * CM_D + CM_D * (CM_SUB + 4) +
+                                            (size_t)(CM_SUB + CM_KMAX - 1) * CM_D + CM_D * CM_KMAX);
+
+template <typename Tl, typename Tc>
+__global__ void __launch_bounds__(256) chanmix_bwd_kernel(const float* __restrict__ dc, const Tl* __restrict__ lat,
+                                                          const Tc* __restrict__ cq_chan, const Tc* __restrict__ ck_chan,
+                                                          const Tc* __restrict__ cq_seq, const Tc* __restrict__ ck_seq,
+                                                          float* __restrict__ ds, float* __restrict__ dwq,
+                                                          float* __restrict__ dwk, long long T, int S, int nq, int nkv,
+                                                          int K) {
+  extern __shared__ float cm[];
+  float* Wc = cm;                         // [i][j]
+  float* dcR = Wc + CM_D * CM_D;          // [t][i]
+  float* sR = dcR + CM_SUB * CM_D;        // [t][j]
+  float* dcT = sR + CM_SUB * CM_D;        // [i][t] (row stride CM_SUB + 4)
+  constexpr int LT = CM_SUB + 4;
+  float* latS = dcT + CM_D * LT;          // [K - 1 + CM_SUB rows][CM_D]: latents of the sub-block and its halo
+  float* wS = latS + (CM_SUB + CM_KMAX - 1) * CM_D;  // [c][k] seq-conv taps of the head
+  const int h = blockIdx.y, tid = threadIdx.x;
+  const bool isq = h < nq;
+  const int hh = isq ? h : h - nq;
+  const int Lq = nq * CM_D, W = Lq + nkv * CM_D, Nlat = Lq + 2 * nkv * CM_D;
+  const int ccol = isq ? hh * CM_D : Lq + hh * CM_D;  // this head's first column in dc / ds / lat
+  const Tc* wsrc = (isq ? cq_chan : ck_chan) + (size_t)hh * CM_D * CM_D;
+  const Tc* wseq = (isq ? cq_seq : ck_seq) + (size_t)hh * CM_D * K;
+  for (int e = tid; e < CM_D * CM_D; e += 256) Wc[e] = ld_f(wsrc + e);
+  for (int e = tid; e < CM_D * K; e += 256) wS[e] = ld_f(wseq + e);
+  const int rq = tid >> 5, cq = tid & 31;  // ds: rows 4 rq .. +3, columns 4 cq .. +3
+  const int pi = tid >> 4, pj = tid & 15;  // dW: rows 8 pi .. +7, columns 8 pj .. +7
+  float acc[8][8];
+#pragma unroll
+  for (int a = 0; a < 8; ++a)
+#pragma unroll
+    for (int b = 0; b < 8; ++b) acc[a][b] = 0.f;
+  const long long r_begin = (long long)blockIdx.x * CM_ROWS;
+  const long long r_end = r_begin + CM_ROWS < T ? r_begin + CM_ROWS : T;
+  for (long long r0 = r_begin; r0 < r_end; r0 += CM_SUB) {
+    __syncthreads();  // the previous sub-block's tiles are consumed (and Wc, wS are in place)
+    // dc rows (four columns a thread) and the latent rows r0 - (K-1) .. r0 + CM_SUB - 1
+    for (int e = tid; e < CM_SUB * (CM_D / 4); e += 256) {
+      const int t = e / (CM_D / 4), c = 4 * (e % (CM_D / 4));
+      const long long row = r0 + t;
+      float4 v = make_float4(0.f, 0.f, 0.f, 0.f);
+      if (row < r_end) v = *reinterpret_cast<const float4*>(dc + row * W + ccol + c);
+      *reinterpret_cast<float4*>(dcR + t * CM_D + c) = v;
+      dcT[(c + 0) * LT + t] = v.x;
+      dcT[(c + 1) * LT + t] = v.y;
+      dcT[(c + 2) * LT + t] = v.z;
+      dcT[(c + 3) * LT + t] = v.w;
+    }
+    for (int e = tid; e < (CM_SUB + K - 1) * CM_D; e += 256) {
+      const int i = e / CM_D, c = e % CM_D;
+      const long long row = r0 - (K - 1) + i;
+      latS[i * CM_D + c] = (row >= 0 && row < r_end) ? ld_f(lat + row * Nlat + ccol + c) : 0.f;
+    }
+    __syncthreads();
+    // s = the seq conv of the latents within each sequence (taps before a sequence start read nothing)
+    for (int e = tid; e < CM_SUB * CM_D; e += 256) {
+      const int t = e / CM_D, c = e % CM_D;
+      const long long row = r0 + t;
+      const int ts = (int)(row % S);
+      float sv = 0.f;
+      for (int k = 0; k < K; ++k)
+        if (ts - (K - 1) + k >= 0) sv = fmaf(wS[c * K + k], latS[(t + k) * CM_D + c], sv);
+      sR[t * CM_D + c] = sv;
+    }
+    __syncthreads();
+    // ds = dc W_c: ds[t][j] = sum_i dc[t][i] W[i][j]
+    {
+      float o[4][4] = {};
+#pragma unroll 4
+      for (int i = 0; i < CM_D; ++i) {
+        const float4 av = *reinterpret_cast<const float4*>(dcT + i * LT + 4 * rq);
+        const float4 bv = *reinterpret_cast<const float4*>(Wc + i * CM_D + 4 * cq);
+        const float a4[4] = {av.x, av.y, av.z, av.w}, b4[4] = {bv.x, bv.y, bv.z, bv.w};
+#pragma unroll
+        for (int a = 0; a < 4; ++a)
+#pragma unroll
+          for (int b = 0; b < 4; ++b) o[a][b] = fmaf(a4[a], b4[b], o[a][b]);
+      }
+#pragma unroll
+      for (int a = 0; a < 4; ++a) {
+        const long long row = r0 + 4 * rq + a;
+        if (row < r_end)
+          *reinterpret_cast<float4*>(ds + row * W + ccol + 4 * cq) = make_float4(o[a][0], o[a][1], o[a][2], o[a][3]);
+      }
+    }
+    // dW[i][j] += sum_t dc[t][i] s[t][j]
+#pragma unroll 2
+    for (int t = 0; t < CM_SUB; ++t) {
+      const float4 a0 = *reinterpret_cast<const float4*>(dcR + t * CM_D + 8 * pi);
+      const float4 a1 = *reinterpret_cast<const float4*>(dcR + t * CM_D + 8 * pi + 4);
+      const float4 b0 = *reinterpret_cast<const float4*>(sR + t * CM_D + 8 * pj);
+      const float4 b1 = *reinterpret_cast<const float4*>(sR + t * CM_D + 8 * pj + 4);
+      const float av[8] = {a0.x, a0.y, a0.z, a0.w, a1.x, a1.y, a1.z, a1.w};
+      const float bv[8] = {b0.x, b0.y, b0.z, b0.w, b1.x, b1.y, b1.z, b1.w};
+#pragma unroll
+      for (int a = 0; a < 8; ++a)
+#pragma unroll
+        for (int b = 0; b < 8; ++b) acc[a][b] = fmaf(av[a], bv[b], acc[a][b]);
+    }
+  }
+  float* dw = (isq ? dwq : dwk) + (size_t)hh * CM_D * CM_D;
+#pragma unroll
+  for (int a = 0; a < 8; ++a) {
+    float* rowp = dw + (size_t)(8 * pi + a) * CM_D + 8 * pj;
+    asm volatile("red.global.add.v4.f32 [%0], {%1, %2, %3, %4};" ::"l"(rowp), "f"(acc[a][0]), "f"(acc[a][1]),
+                 "f"(acc[a][2]), "f"(acc[a][3])
+                 : "memory");
+    asm volatile("red.global.add.v4.f32 [%0], {%1, %2, %3, %4};" ::"l"(rowp + 4), "f"(acc[a][4]), "f"(acc[a][5]),
+                 "f"(acc[a][6]), "f"(acc[a][7])
+                 : "memory");
+  }
+}
+
+// The same for any even head_dim: per row t, per head, ds[t] = W_c^T dc[t] and s[t] recomputed
+// (block = one row; thread = one channel); dW_c then comes from a strided GEMM over the rows.
 template <typename Tl, typename Tc>
 __global__ void __launch_bounds__(256) chan_bwd_kernel(const float* __restrict__ dc, const Tl* __restrict__ lat,
                                                        const Tc* __restrict__ cq_chan, const Tc* __restrict__ ck_chan,
@@ -669,10 +790,16 @@ cudaError_t transpose_bf16(Mat in, long long ldi, int R, int C, int Rp, __nv_bfl
   return cudaGetLastError();
 }
 
-// C[M, N] (fp32, row stride ldc) = A[M, K] B[N, K]^T on the tensor cores, bf16 operands
+// C[M, N] (fp32, row stride ldc, contiguous rows) = A[M, K] B[N, K]^T on the tensor cores, bf16
+// operands; a long K over few output tiles is split (C cleared, slices added)
 cudaError_t gemm_tc_bf16(const void* A, long long M, const void* B, int N, int K, float* C, long long ldc,
                          unsigned* err, cudaStream_t s) {
   GemmTcArgs a{};
+  a.ksplit = gemm_tc_ksplit(M, N, K);
+  if (a.ksplit > 1) {
+    const cudaError_t e = cudaMemsetAsync(C, 0, sizeof(float) * ((size_t)(M - 1) * ldc + N), s);
+    if (e != cudaSuccess) return e;
+  }
   a.A = A;
   a.M = M;
   a.K = K;
@@ -890,25 +1017,52 @@ cudaError_t launch_backward(const BlockDims& dm, const BlockPtrs& p, const Backw
         dm.use_rope, th);
     if ((e = cudaGetLastError()) != cudaSuccess) return e;
   }
-  // 5. channel mix: ds = W_c^T dc (and s recomputed); dW_c[h] = sum_t dc[t,h]^T s[t,h]
-  if (lt == DType::F16 && it == DType::BF16)
-    chan_bwd_kernel<__half, __nv_bfloat16><<<(unsigned)T, 256, 0, stream>>>(
-        dc, static_cast<const __half*>(p.qkv_lat), static_cast<const __nv_bfloat16*>(p.cq_chan),
-        static_cast<const __nv_bfloat16*>(p.ck_chan), static_cast<const __nv_bfloat16*>(p.cq_seq),
-        static_cast<const __nv_bfloat16*>(p.ck_seq), ds, s, dm.S, dm.nq, dm.nkv, d, dm.K);
-  else
-    chan_bwd_kernel<float, float><<<(unsigned)T, 256, 0, stream>>>(
-        dc, static_cast<const float*>(p.qkv_lat), static_cast<const float*>(p.cq_chan),
-        static_cast<const float*>(p.ck_chan), static_cast<const float*>(p.cq_seq), static_cast<const float*>(p.ck_seq),
-        ds, s, dm.S, dm.nq, dm.nkv, d, dm.K);
-  if ((e = cudaGetLastError()) != cudaSuccess) return e;
-  // dW_c (q heads, then K heads): batch over heads; A[i][t] = dc[t][h d + i], B[j][t] = s[t][h d + j]
-  if ((e = gemm({dc, DType::F32}, 1, W, d, {s, DType::F32}, 1, W, d, g.dconvq_chan, d, (long long)d * d, d, d, T,
-                dm.nq, false, stream)) != cudaSuccess)
-    return e;
-  if ((e = gemm({dc + Lq, DType::F32}, 1, W, d, {s + Lq, DType::F32}, 1, W, d, g.dconvk_chan, d, (long long)d * d, d,
-                d, T, dm.nkv, false, stream)) != cudaSuccess)
-    return e;
+  // 5. channel mix: ds = W_c^T dc; dW_c[h] = sum_t dc[t,h]^T s[t,h] (s recomputed from the latents)
+  if (d == CM_D) {
+    if ((e = cudaMemsetAsync(g.dconvq_chan, 0, sizeof(float) * dm.nq * d * d, stream)) != cudaSuccess ||
+        (e = cudaMemsetAsync(g.dconvk_chan, 0, sizeof(float) * dm.nkv * d * d, stream)) != cudaSuccess)
+      return e;
+    const dim3 grid((unsigned)((T + CM_ROWS - 1) / CM_ROWS), dm.nq + dm.nkv);
+    if (lt == DType::F16 && it == DType::BF16) {
+      auto k = chanmix_bwd_kernel<__half, __nv_bfloat16>;
+      if ((e = cudaFuncSetAttribute(k, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)CM_SMEM)) != cudaSuccess)
+        return e;
+      k<<<grid, 256, CM_SMEM, stream>>>(dc, static_cast<const __half*>(p.qkv_lat),
+                                        static_cast<const __nv_bfloat16*>(p.cq_chan),
+                                        static_cast<const __nv_bfloat16*>(p.ck_chan),
+                                        static_cast<const __nv_bfloat16*>(p.cq_seq),
+                                        static_cast<const __nv_bfloat16*>(p.ck_seq), ds, g.dconvq_chan, g.dconvk_chan, T,
+                                        dm.S, dm.nq, dm.nkv, dm.K);
+    } else {
+      auto k = chanmix_bwd_kernel<float, float>;
+      if ((e = cudaFuncSetAttribute(k, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)CM_SMEM)) != cudaSuccess)
+        return e;
+      k<<<grid, 256, CM_SMEM, stream>>>(dc, static_cast<const float*>(p.qkv_lat), static_cast<const float*>(p.cq_chan),
+                                        static_cast<const float*>(p.ck_chan), static_cast<const float*>(p.cq_seq),
+                                        static_cast<const float*>(p.ck_seq), ds, g.dconvq_chan, g.dconvk_chan, T, dm.S,
+                                        dm.nq, dm.nkv, dm.K);
+    }
+    if ((e = cudaGetLastError()) != cudaSuccess) return e;
+  } else {
+    if (lt == DType::F16 && it == DType::BF16)
+      chan_bwd_kernel<__half, __nv_bfloat16><<<(unsigned)T, 256, 0, stream>>>(
+          dc, static_cast<const __half*>(p.qkv_lat), static_cast<const __nv_bfloat16*>(p.cq_chan),
+          static_cast<const __nv_bfloat16*>(p.ck_chan), static_cast<const __nv_bfloat16*>(p.cq_seq),
+          static_cast<const __nv_bfloat16*>(p.ck_seq), ds, s, dm.S, dm.nq, dm.nkv, d, dm.K);
+    else
+      chan_bwd_kernel<float, float><<<(unsigned)T, 256, 0, stream>>>(
+          dc, static_cast<const float*>(p.qkv_lat), static_cast<const float*>(p.cq_chan),
+          static_cast<const float*>(p.ck_chan), static_cast<const float*>(p.cq_seq), static_cast<const float*>(p.ck_seq),
+          ds, s, dm.S, dm.nq, dm.nkv, d, dm.K);
+    if ((e = cudaGetLastError()) != cudaSuccess) return e;
+    // dW_c (q heads, then K heads): batch over heads; A[i][t] = dc[t][h d + i], B[j][t] = s[t][h d + j]
+    if ((e = gemm({dc, DType::F32}, 1, W, d, {s, DType::F32}, 1, W, d, g.dconvq_chan, d, (long long)d * d, d, d, T,
+                  dm.nq, false, stream)) != cudaSuccess)
+      return e;
+    if ((e = gemm({dc + Lq, DType::F32}, 1, W, d, {s + Lq, DType::F32}, 1, W, d, g.dconvk_chan, d, (long long)d * d,
+                  d, d, T, dm.nkv, false, stream)) != cudaSuccess)
+      return e;
+  }
   // 6. seq conv: dlat (q and k channels) and the tap gradients
   if (it == DType::BF16)
     seq_bwd_kernel<__nv_bfloat16><<<(unsigned)T, 256, 0, stream>>>(

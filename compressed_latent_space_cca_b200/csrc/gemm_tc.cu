@@ -83,8 +83,11 @@ struct GemmParams {
   int out_type;  // DType of C
   int in_fmt;    // kFmtBF16 or kFmtF16
   unsigned* err;
-  int num_tiles;
+  int num_tiles;  // work items: output tiles x K slices
   int n_tiles_n;
+  int tiles;      // output tiles
+  int ksplit;     // K slices per tile (fp32 output added with reductions when > 1)
+  int kb_slice;   // 64-deep K blocks per slice
   int tma_store;  // 16-bit output written through shared memory and maps.c
   // side job (bf16 -> fp16 copies), done by the epilogue warps before their first tile
   const __nv_bfloat16* side_src[2];
@@ -156,6 +159,13 @@ __device__ __forceinline__ bool store_row_chunk(const GemmParams& p, long long r
       }
       dst[v] = make_uint4(w[0], w[1], w[2], w[3]);
     }
+  } else if (p.ksplit > 1) {  // a K slice's share, added to the sum of all slices
+    float* dst = static_cast<float*>(p.C) + row * p.ldc + col0;
+#pragma unroll
+    for (int v = 0; v < 8; ++v)
+      asm volatile("red.global.add.v4.f32 [%0], {%1, %2, %3, %4};" ::"l"(dst + 4 * v), "f"(u2f(r[4 * v])),
+                   "f"(u2f(r[4 * v + 1])), "f"(u2f(r[4 * v + 2])), "f"(u2f(r[4 * v + 3]))
+                   : "memory");
   } else {
     uint4* dst = reinterpret_cast<uint4*>(static_cast<float*>(p.C) + row * p.ldc + col0);
 #pragma unroll
@@ -224,9 +234,11 @@ __global__ void __launch_bounds__(Shape<MH, PAIR>::NUM_THREADS, 1)
       int stage = 0;
       uint32_t phase = 0;
       for (int t = unit; t < p.num_tiles; t += n_units) {
-        const int m0 = (t / p.n_tiles_n) * TM + (int)rank * 128;  // this CTA's first row
-        const int n0 = (t % p.n_tiles_n) * BN;
-        for (int kb = 0; kb < kblocks; ++kb) {
+        const int tile = t % p.tiles, kb0 = (t / p.tiles) * p.kb_slice;
+        const int kb1 = kb0 + p.kb_slice < kblocks ? kb0 + p.kb_slice : kblocks;
+        const int m0 = (tile / p.n_tiles_n) * TM + (int)rank * 128;  // this CTA's first row
+        const int n0 = (tile % p.n_tiles_n) * BN;
+        for (int kb = kb0; kb < kb1; ++kb) {
           if (!mbar_wait_bounded(smem_u32(&empty[stage]), phase ^ 1, p.err, abort_flag, wait_site(kSiteGemm, 1, 1))) goto producer_done;
           uint32_t fb = smem_u32(&full[stage]);
           if constexpr (PAIR) {
@@ -280,7 +292,9 @@ __global__ void __launch_bounds__(Shape<MH, PAIR>::NUM_THREADS, 1)
         if (!mbar_wait_bounded(smem_u32(&tempty[acc]), tph ^ 1, p.err, abort_flag, wait_site(kSiteGemm, 2, 2))) goto mma_done;
         tc_fence_after();
         const uint32_t d_tmem = tmem_base + acc * BN;
-        for (int kb = 0; kb < kblocks; ++kb) {
+        const int kb0 = (t / p.tiles) * p.kb_slice;
+        const int kb1 = kb0 + p.kb_slice < kblocks ? kb0 + p.kb_slice : kblocks;
+        for (int kb = kb0; kb < kb1; ++kb) {
           if (!mbar_wait_bounded(smem_u32(&full[stage]), phase, p.err, abort_flag, wait_site(kSiteGemm, 2, 3))) goto mma_done;
           tc_fence_after();
           const uint32_t a_lo = a_lo0 + stage * (STAGE_BYTES >> 4);
@@ -291,10 +305,10 @@ __global__ void __launch_bounds__(Shape<MH, PAIR>::NUM_THREADS, 1)
             for (int h = 0; h < MH; ++h) {  // rows h*128.. of the tile -> accumulator columns h*256..
               if constexpr (PAIR) {
                 if (elect_one_sync()) umma_ss_pair_lohi(d_tmem + h * BN, a_lo + h * (A_HALF_BYTES >> 4) + 2 * k, d_hi, b_lo + 2 * k,
-                                                        d_hi, idesc, (kb | k) != 0);
+                                                        d_hi, idesc, (kb != kb0 || k != 0));
               } else {
                 if (elect_one_sync()) umma_ss_lohi(d_tmem + h * BN, a_lo + h * (A_HALF_BYTES >> 4) + 2 * k, d_hi, b_lo + 2 * k, d_hi, idesc,
-                             (kb | k) != 0);
+                             (kb != kb0 || k != 0));
               }
             }
           if constexpr (PAIR) {
@@ -348,8 +362,9 @@ __global__ void __launch_bounds__(Shape<MH, PAIR>::NUM_THREADS, 1)
       const uint32_t tph = (i / ACC_BUFS) & 1;
       if (!mbar_wait_bounded(smem_u32(&tfull[acc]), tph, p.err, abort_flag, wait_site(kSiteGemm, 3, 4))) break;
       tc_fence_after();
-      const long long m0 = (long long)(t / p.n_tiles_n) * TM + rank * 128;
-      const int n0 = (t % p.n_tiles_n) * BN;
+      const int tile = t % p.tiles;
+      const long long m0 = (long long)(tile / p.n_tiles_n) * TM + rank * 128;
+      const int n0 = (tile % p.n_tiles_n) * BN;
       const long long row0 = m0 + half * T::HS + quad * 32;  // this warp's 32 rows
       const long long row = row0 + lane;
       const uint32_t col0 = tmem_base + ((uint32_t)(quad * 32) << 16) + (acc + half) * BN;
@@ -459,6 +474,16 @@ bool encode_2d(CUtensorMap* m, const void* ptr, CUtensorMapDataType dt, uint64_t
 }
 
 }  // namespace
+
+int gemm_tc_ksplit(long long M, int N, int K) {
+  const long long tiles = ((M + 255) / 256) * ((N + 255) / 256);
+  const long long units = num_sms() / 2;
+  if (tiles >= units) return 1;  // a full round of tiles already: slices would only add reductions
+  long long ks = (2 * units + tiles - 1) / tiles;
+  const long long kmax = K / 256;
+  if (ks > kmax) ks = kmax;
+  return ks < 1 ? 1 : (int)ks;
+}
 
 bool gemm_tc_supported(long long M, int N, int K) {
   return M >= 1 && M < (1ll << 31) && K >= BK && K % BK == 0 && N >= 128 && N % 128 == 0;
@@ -574,7 +599,15 @@ cudaError_t launch_gemm_tc(const GemmTcArgs& a, cudaStream_t stream) {
   // 256-row tiles (one CTA, or a pair) when the main loop is long enough to carry the epilogue
   const int TM = big || pair ? 256 : 128;
   const long long m_tiles = (a.M + TM - 1) / TM;
-  p.num_tiles = (int)(m_tiles * p.n_tiles_n);
+  p.tiles = (int)(m_tiles * p.n_tiles_n);
+  const int kblocks = a.K / BK;
+  int ks = a.ksplit > 1 ? a.ksplit : 1;
+  if (ks > kblocks) ks = kblocks;
+  if (ks > 1 && (a.out != DType::F32 || a.v_cache != nullptr || a.side_n[0] > 0 || a.side_n[1] > 0))
+    return cudaErrorInvalidValue;
+  p.kb_slice = (kblocks + ks - 1) / ks;
+  p.ksplit = (kblocks + p.kb_slice - 1) / p.kb_slice;  // no empty slice
+  p.num_tiles = p.tiles * p.ksplit;
   cudaError_t e;
   if (pair) {
     const int clusters = p.num_tiles < pair_clusters<1>() ? p.num_tiles : pair_clusters<1>();

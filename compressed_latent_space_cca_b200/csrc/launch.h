@@ -107,8 +107,14 @@ struct GemmTcArgs {
   void* v_cache;
   void* v_att;
   int v_col0, Lkv, S, vshift, vfrom;
+  // optional split of K into ksplit slices (fp32 C only): each slice's product is added to C, which
+  // the caller clears first
+  int ksplit;
 };
 cudaError_t launch_gemm_tc(const GemmTcArgs& a, cudaStream_t stream);
+// K slices that give a GEMM with fewer 256 x 256 output tiles than the device has CTA pairs about
+// two rounds of work (1 otherwise), with slices of at least 256 along K
+int gemm_tc_ksplit(long long M, int N, int K);
 // dst[0, n) = fp16 copy of the bf16 src times scale (fp16 overflow reported as a range error)
 cudaError_t launch_convert_f16(const void* src, void* dst, long long n, unsigned* dev_err, cudaStream_t stream,
                                float scale = 1.0f);
