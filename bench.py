@@ -421,11 +421,11 @@ def run_ours(args, shape):
             "gpu_launches": launches_per_step * args.steps,
             "clocks": clocks,
         }
-        if (world == 1 and not args.no_mha and my_shape.dtype == "bf16" and my_shape.conv_kernel > 0 and
-                my_shape.hidden % 128 == 0):
-            line["mha_baseline"] = run_mha_baseline(cca, dev, my_shape, ms_per_step)
         if world == 1 and not args.no_backward and cca.backward_workspace_size(cfg) > 0:
             line["backward"] = run_backward(cca, dev, my_shape, inputs, peaks)
+        if (world == 1 and not args.no_mha and my_shape.dtype == "bf16" and my_shape.conv_kernel > 0 and
+                my_shape.hidden % 128 == 0):
+            line["mha_baseline"] = run_mha_baseline(cca, dev, my_shape, ms_per_step, line.get("backward"), peaks)
         if world == 1 and not args.no_decode and cca.decode_workspace_size(cfg) > 0:
             line["decode"] = run_decode(cca, dev, my_shape, inputs, out, peaks)
         if world == 1 and not args.no_cpu_baseline:
@@ -446,9 +446,10 @@ def mha_shape(shape: workloads.BlockShape) -> workloads.BlockShape:
                         seq_len=shape.seq_len, hidden=shape.hidden, n_q_heads=nh, n_kv_heads=nh)
 
 
-def run_mha_baseline(cca, dev, shape, cca_ms_per_step, steps=10, warmup=3):
+def run_mha_baseline(cca, dev, shape, cca_ms_per_step, cca_backward=None, peaks=None, steps=10, warmup=3):
     """Times the plain multi-head block of the same shape with the same method (L2 flushed between
-    steps, CUDA events around each stage) and returns its numbers and the CCA block's speedup."""
+    steps, CUDA events around each stage) and returns its numbers and the CCA block's speedup; with
+    the CCA block's backward timing given, the MHA block's backward too."""
     mshape = mha_shape(shape)
     cfg = cca.config_from_shape(mshape)
     inputs = {k: v.to(dev) for k, v in workloads.make_inputs(mshape).items()}
@@ -470,7 +471,13 @@ def run_mha_baseline(cca, dev, shape, cca_ms_per_step, steps=10, warmup=3):
     ms = float(stage.sum(axis=1).mean())
     stage_ms = stage.mean(axis=0)
     work = algorithmic_work(mshape)
-    del inputs, out, ws, flush
+    del out, ws, flush
+    torch.cuda.empty_cache()
+    bwd = None
+    if cca_backward is not None and cca.backward_workspace_size(cfg) > 0:
+        bwd = run_backward(cca, dev, mshape, inputs, peaks if peaks is not None else load_peaks()[0])
+        bwd["cca_backward_speedup"] = bwd["ms_per_step"] / cca_backward["ms_per_step"]
+    del inputs
     torch.cuda.empty_cache()
     return {
         "workload": mshape.name, "n_q_heads": mshape.n_q_heads, "n_kv_heads": mshape.n_kv_heads,
@@ -480,6 +487,7 @@ def run_mha_baseline(cca, dev, shape, cca_ms_per_step, steps=10, warmup=3):
         "kernels_ms": {"down_proj": stage_ms[0], "rope_cache": stage_ms[1], "attention": stage_ms[2],
                        "out_proj": stage_ms[3]},
         "cca_speedup": ms / cca_ms_per_step,
+        "backward": bwd,
     }
 
 
@@ -501,7 +509,8 @@ def run_backward(cca, dev, shape, inputs, peaks, steps=5, warmup=3):
     cfg = cca.config_from_shape(shape)
     dy = workloads.make_dy(shape).to(dev)
     ws = torch.empty(cca.backward_workspace_size(cfg), dtype=torch.uint8, device=dev)
-    grads = {n: torch.empty(tuple(inputs[n].shape), dtype=torch.float32, device=dev) for n in cca.GRAD_NAMES}
+    grads = {n: torch.empty(tuple(inputs[n].shape), dtype=torch.float32, device=dev)
+             for n in cca.GRAD_NAMES if n in inputs}  # a plain block has no conv weights
     flush = torch.empty(L2_FLUSH_BYTES, dtype=torch.uint8, device=dev)
     for _ in range(warmup):
         flush.zero_()

@@ -358,7 +358,8 @@ def backward(cfg: CcaConfig, inputs: Dict[str, torch.Tensor], dy: torch.Tensor, 
     """cca_backward: the gradients of x and of the eight weights for dL/dy = dy.
 
     inputs: the nine tensors of INPUT_NAMES (dtype cfg.dtype); dy [B, S, E] in cfg.out_dtype.
-    Returns fp32 tensors named as the inputs, in their shapes (overwritten, not accumulated).
+    Returns fp32 tensors named as the inputs, in their shapes (overwritten, not accumulated); a plain
+    block (conv_kernel 0) has no conv weights and returns no gradients for them.
     """
     x = inputs["x"]
     device = x.device
@@ -367,9 +368,10 @@ def backward(cfg: CcaConfig, inputs: Dict[str, torch.Tensor], dy: torch.Tensor, 
     sh = _shapes(cfg)
     ptrs = _input_ptrs(cfg, inputs, INPUT_NAMES, _DT[cfg.dtype], device)
     dyp = _check(dy, "dy", sh["y"], _DT[cfg.out_dtype], device)
+    names = [n for n in GRAD_NAMES if not (cfg.conv_kernel == 0 and n.startswith("conv"))]
     if grads is None:
-        grads = {n: torch.empty(sh[n], dtype=torch.float32, device=device) for n in GRAD_NAMES}
-    gp = [_check(grads[n], "d" + n, sh[n], torch.float32, device) for n in GRAD_NAMES]
+        grads = {n: torch.empty(sh[n], dtype=torch.float32, device=device) for n in names}
+    gp = [_check(grads[n], "d" + n, sh[n], torch.float32, device) if n in names else None for n in GRAD_NAMES]
     if workspace is None:
         n = backward_workspace_size(cfg)
         if n == 0:

@@ -21,8 +21,9 @@
 //   where they are the K-major A operands of dV += P^T dO_i and dK += dS^T Q_i (Q_i and dO_i read
 //   MN-major); the epilogue adds the chunk's dK (scaled) and dV to fp32 sums with vector atomics,
 //   so that the long key tiles near the start of a sequence can be split over several CTAs.
-// Both: warp 0 issues the TMA loads, warp 1 the MMAs (an elected lane each), warps 2-5 own the TMEM
-// lane quadrants 2, 3, 0, 1 (one row per thread). Two TMEM / shared-memory slots let the softmax of
+// Both: warp 0 issues the TMA loads, warp 1 the MMAs (an elected lane each); warps 2-9 do the softmax
+// and the epilogue, two per TMEM lane quadrant (warp w reads lanes 32 (w % 4) ..), one row per thread,
+// each of the two taking half of the row's columns. Two TMEM / shared-memory slots let the softmax of
 // one unit overlap the MMAs of its neighbours. Every mbarrier wait is bounded.
 #include "cca_common.cuh"
 #include "launch.h"
@@ -31,7 +32,8 @@ namespace cca {
 namespace {
 
 constexpr int D = 128;
-constexpr int NUM_THREADS = 192;  // loader, MMA, 4 softmax / epilogue warps
+constexpr int NUM_SM_WARPS = 8;  // softmax / epilogue warps
+constexpr int NUM_THREADS = 64 + 32 * NUM_SM_WARPS;
 constexpr int TMEM_COLS = 512;
 constexpr int SW = 128;  // bytes of one swizzled row (64 fp16)
 
@@ -94,6 +96,16 @@ __device__ __forceinline__ void bulk_load(uint32_t dst, const void* src, uint32_
       : "memory");
 }
 
+// 32 lanes x 16 columns of 32-bit: thread i stores r[0..15] to lane (base + i), columns [col, col + 16)
+__device__ __forceinline__ void tmem_st_32x32b_x16(uint32_t taddr, const uint32_t* r) {
+  asm volatile(
+      "tcgen05.st.sync.aligned.32x32b.x16.b32"
+      " [%0], {%1,%2,%3,%4,%5,%6,%7,%8,%9,%10,%11,%12,%13,%14,%15,%16};" ::"r"(taddr),
+      "r"(r[0]), "r"(r[1]), "r"(r[2]), "r"(r[3]), "r"(r[4]), "r"(r[5]), "r"(r[6]), "r"(r[7]), "r"(r[8]),
+      "r"(r[9]), "r"(r[10]), "r"(r[11]), "r"(r[12]), "r"(r[13]), "r"(r[14]), "r"(r[15])
+      : "memory");
+}
+
 __device__ __forceinline__ void red_add_v4(float* p, float a, float b, float c, float d) {
   asm volatile("red.global.add.v4.f32 [%0], {%1, %2, %3, %4};" ::"l"(p), "f"(a), "f"(b), "f"(c), "f"(d)
                : "memory");
@@ -115,7 +127,7 @@ __global__ void __launch_bounds__(NUM_THREADS, 1) attn_bwd_dq_kernel(const __gri
   uint64_t* kv_full = bars + 1;                   // [3]
   uint64_t* kv_empty = kv_full + DQ_KV_STAGES;    // [3]
   uint64_t* st_full = kv_empty + DQ_KV_STAGES;    // [2] S and dP of a block in TMEM
-  uint64_t* ds_full = st_full + 2;                // [2] dS written over S (4 warps)
+  uint64_t* ds_full = st_full + 2;                // [2] dS written over S (every softmax warp)
   uint64_t* dq_full = ds_full + 2;                // dQ complete
   uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(dq_full + 1);
   volatile int* abort_flag = reinterpret_cast<volatile int*>(tmem_slot + 1);
@@ -137,7 +149,7 @@ __global__ void __launch_bounds__(NUM_THREADS, 1) attn_bwd_dq_kernel(const __gri
     }
     for (int s = 0; s < 2; ++s) {
       mbar_init(smem_u32(&st_full[s]), 1);
-      mbar_init(smem_u32(&ds_full[s]), 4);
+      mbar_init(smem_u32(&ds_full[s]), NUM_SM_WARPS);
     }
     mbar_init(smem_u32(dq_full), 1);
     *abort_flag = 0;
@@ -241,6 +253,7 @@ __global__ void __launch_bounds__(NUM_THREADS, 1) attn_bwd_dq_kernel(const __gri
   } else {
     // ------------------------------------------------------------ softmax --
     const int quad = warp & 3;
+    const int half = (warp - 2) >> 2;  // this warp's 32 of the block's 64 keys
     const int r = quad * 32 + lane;
     const int t = qt * DQ_QT + r;
     const bool row_ok = t < p.S;
@@ -255,16 +268,14 @@ __global__ void __launch_bounds__(NUM_THREADS, 1) attn_bwd_dq_kernel(const __gri
       if (!mbar_wait_bounded(smem_u32(&st_full[s]), (j >> 1) & 1, p.err, abort_flag, wait_site(kSiteAttnBwd, 3, 5)))
         goto done;
       tc_fence_after();
-      uint32_t sv[64], dp[64];
-      tmem_ld_32x32b_x32(tmem + lane_off + DQ_COL_S + 64 * s, sv);
-      tmem_ld_32x32b_x32(tmem + lane_off + DQ_COL_S + 64 * s + 32, sv + 32);
-      tmem_ld_32x32b_x32(tmem + lane_off + DQ_COL_DP + 64 * s, dp);
-      tmem_ld_32x32b_x32(tmem + lane_off + DQ_COL_DP + 64 * s + 32, dp + 32);
+      uint32_t sv[32], dp[32];
+      tmem_ld_32x32b_x32(tmem + lane_off + DQ_COL_S + 64 * s + 32 * half, sv);
+      tmem_ld_32x32b_x32(tmem + lane_off + DQ_COL_DP + 64 * s + 32 * half, dp);
       tmem_ld_wait();
-      const int key0 = j * DQ_KB;
-      uint32_t pk[32];
+      const int key0 = j * DQ_KB + 32 * half;
+      uint32_t pk[16];
 #pragma unroll
-      for (int c = 0; c < 64; c += 2) {
+      for (int c = 0; c < 32; c += 2) {
         float ds[2];
 #pragma unroll
         for (int e = 0; e < 2; ++e) {
@@ -275,7 +286,8 @@ __global__ void __launch_bounds__(NUM_THREADS, 1) attn_bwd_dq_kernel(const __gri
         }
         pk[c >> 1] = pack_f16x2(ds[0], ds[1]);
       }
-      tmem_st_32x32b_x32(tmem + lane_off + DQ_COL_S + 64 * s, pk);
+      // keys 2c, 2c + 1 of the block go to packed column c: this half's 16 columns
+      tmem_st_32x32b_x16(tmem + lane_off + DQ_COL_S + 64 * s + 16 * half, pk);
       tmem_st_wait();
       tc_fence_before();
       __syncwarp();
@@ -286,7 +298,7 @@ __global__ void __launch_bounds__(NUM_THREADS, 1) attn_bwd_dq_kernel(const __gri
     tc_fence_after();
     float* out = p.dq + ((size_t)b * p.S + t) * p.Lq + h * D;
 #pragma unroll 1
-    for (int c4 = 0; c4 < 4; ++c4) {
+    for (int c4 = 2 * half; c4 < 2 * half + 2; ++c4) {
       uint32_t v[32];
       tmem_ld_32x32b_x32(tmem + lane_off + DQ_COL_DQ + 32 * c4, v);
       tmem_ld_wait();
@@ -343,7 +355,7 @@ __global__ void __launch_bounds__(NUM_THREADS, 1) attn_bwd_dkv_kernel(const __gr
   uint64_t* qd_full = bars + 1;        // [2] Q_i, dO_i, lse2, delta of a unit
   uint64_t* qd_empty = qd_full + 2;    // [2]
   uint64_t* st_full = qd_empty + 2;    // [2] S^T, dP^T in TMEM
-  uint64_t* p_full = st_full + 2;      // [2] P^T, dS^T in shared memory (4 warps)
+  uint64_t* p_full = st_full + 2;      // [2] P^T, dS^T in shared memory (every softmax warp)
   uint64_t* pt_free = p_full + 2;      // [2] P^T, dS^T read by their MMAs
   uint64_t* acc_full = pt_free + 2;    // dK, dV complete
   uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(acc_full + 1);
@@ -359,7 +371,7 @@ __global__ void __launch_bounds__(NUM_THREADS, 1) attn_bwd_dkv_kernel(const __gr
       mbar_init(smem_u32(&qd_full[s]), 1);
       mbar_init(smem_u32(&qd_empty[s]), 1);
       mbar_init(smem_u32(&st_full[s]), 1);
-      mbar_init(smem_u32(&p_full[s]), 4);
+      mbar_init(smem_u32(&p_full[s]), NUM_SM_WARPS);
       mbar_init(smem_u32(&pt_free[s]), 1);
     }
     mbar_init(smem_u32(acc_full), 1);
@@ -478,6 +490,7 @@ __global__ void __launch_bounds__(NUM_THREADS, 1) attn_bwd_dkv_kernel(const __gr
   } else {
     // ------------------------------------------------------------ softmax --
     const int quad = warp & 3;
+    const int half = (warp - 2) >> 2;  // this warp's 32 of a unit's 64 queries
     const int r = quad * 32 + lane;
     const int key = it.kt * KV_KT + r;
     const uint32_t lane_off = (uint32_t)(quad * 32) << 16;
@@ -489,11 +502,9 @@ __global__ void __launch_bounds__(NUM_THREADS, 1) attn_bwd_dkv_kernel(const __gr
       if (!mbar_wait_bounded(smem_u32(&st_full[s]), (n >> 1) & 1, p.err, abort_flag, wait_site(kSiteAttnBwd, 6, 5)))
         goto done;
       tc_fence_after();
-      uint32_t sv[64], dp[64];
-      tmem_ld_32x32b_x32(tmem + lane_off + KV_COL_ST + 64 * s, sv);
-      tmem_ld_32x32b_x32(tmem + lane_off + KV_COL_ST + 64 * s + 32, sv + 32);
-      tmem_ld_32x32b_x32(tmem + lane_off + KV_COL_DPT + 64 * s, dp);
-      tmem_ld_32x32b_x32(tmem + lane_off + KV_COL_DPT + 64 * s + 32, dp + 32);
+      uint32_t sv[32], dp[32];
+      tmem_ld_32x32b_x32(tmem + lane_off + KV_COL_ST + 64 * s + 32 * half, sv);
+      tmem_ld_32x32b_x32(tmem + lane_off + KV_COL_DPT + 64 * s + 32 * half, dp);
       tmem_ld_wait();
       // the MMAs of unit n - 2 have finished reading this slot's P^T and dS^T
       if (n >= 2 && !mbar_wait_bounded(smem_u32(&pt_free[s]), ((n >> 1) & 1) ^ 1, p.err, abort_flag,
@@ -508,19 +519,21 @@ __global__ void __launch_bounds__(NUM_THREADS, 1) attn_bwd_dkv_kernel(const __gr
       uint8_t* prow = smem + KV_OFF_PT + s * KV_KT * SW + r * SW;
       uint8_t* drow = smem + KV_OFF_DST + s * KV_KT * SW + r * SW;
 #pragma unroll
-      for (int ch = 0; ch < 8; ++ch) {  // 8 queries per 16-byte chunk
+      for (int cc = 0; cc < 4; ++cc) {  // 8 queries per 16-byte chunk: chunks 4 half .. 4 half + 3
+        const int ch = 4 * half + cc;
         uint32_t pp[4], dd[4];
 #pragma unroll
         for (int e = 0; e < 4; ++e) {
           float pv[2], dv[2];
 #pragma unroll
           for (int f = 0; f < 2; ++f) {
-            const int c = 8 * ch + 2 * e + f;
+            const int cl = 8 * cc + 2 * e + f;  // column within this warp's half
+            const int c = 32 * half + cl;
             const int t = q0 + c;
             const bool vis = key <= t && t < p.S;
-            const float pr = vis ? fast_exp2(fmaf(u2f(sv[c]), c2, -lse_s[c])) : 0.f;
+            const float pr = vis ? fast_exp2(fmaf(u2f(sv[cl]), c2, -lse_s[c])) : 0.f;
             pv[f] = pr;
-            dv[f] = vis ? pr * (u2f(dp[c]) - del_s[c]) : 0.f;
+            dv[f] = vis ? pr * (u2f(dp[cl]) - del_s[c]) : 0.f;
             bad |= f16_overflow(dv[f]);
           }
           pp[e] = pack_f16x2(pv[0], pv[1]);
@@ -541,7 +554,7 @@ __global__ void __launch_bounds__(NUM_THREADS, 1) attn_bwd_dkv_kernel(const __gr
     const bool key_ok = key < p.S;
     const size_t orow = ((size_t)it.b * p.S + key) * p.Lkv + it.g * D;
 #pragma unroll 1
-    for (int c4 = 0; c4 < 4; ++c4) {
+    for (int c4 = 2 * half; c4 < 2 * half + 2; ++c4) {
       uint32_t v[32], k[32];
       tmem_ld_32x32b_x32(tmem + lane_off + KV_COL_DV + 32 * c4, v);
       tmem_ld_32x32b_x32(tmem + lane_off + KV_COL_DK + 32 * c4, k);

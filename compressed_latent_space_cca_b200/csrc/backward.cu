@@ -439,7 +439,8 @@ __global__ void __launch_bounds__(256) token_bwd_kernel(const float* __restrict_
                                                         const float* __restrict__ dv, float* __restrict__ dc,
                                                         float* __restrict__ dpre, float* __restrict__ dlat, int S,
                                                         int nq, int nkv, int d, int mode, int vshift, int vfrom,
-                                                        int use_rope, const __grid_constant__ Theta64 theta) {
+                                                        int use_rope, const __grid_constant__ Theta64 theta,
+                                                        int plain) {
   const long long row = blockIdx.x;  // b * S + t
   const int t = (int)(row % S);
   const int G = nq / nkv, Lq = nq * d, Lkv = nkv * d, half = d / 2, Nlat = Lq + 2 * Lkv;
@@ -485,8 +486,12 @@ __global__ void __launch_bounds__(256) token_bwd_kernel(const float* __restrict_
       a = 0.5f * s + 0.5f * dka[c];
       bsum = a;
     }
-    dc[row * (Lq + Lkv) + e] = direct + P * bsum;
-    dpre[row * (Lq + Lkv) + e] = R * a;
+    if (plain) {  // no convolutions: the attention inputs are the latents
+      dlat[row * Nlat + e] = direct;
+    } else {
+      dc[row * (Lq + Lkv) + e] = direct + P * bsum;
+      dpre[row * (Lq + Lkv) + e] = R * a;
+    }
   }
   // value shift transpose
   for (int c = threadIdx.x; c < Lkv; c += blockDim.x) {
@@ -504,7 +509,7 @@ __global__ void __launch_bounds__(256) token_bwd_kernel(const float* __restrict_
 // 8 x 8 patch of dW_c, added to the fp32 sum with vector atomics at the end.
 constexpr int CM_ROWS = 256, CM_SUB = 32, CM_D = 128, CM_KMAX = 8;
 constexpr size_t CM_SMEM = sizeof(float) * ((size_t)CM_D * CM_D + 2 * CM_SUB * CM_D + CM_D * (CM_SUB + 4) +
-                                            (size_t)(CM_SUB + CM_KMAX - 1) * CM_D + CM_D * CM_KMAX);
+                                            (size_t)(CM_SUB + CM_KMAX - 1) * CM_D + CM_D * CM_KMAX + CM_SUB);
 
 template <typename Tl, typename Tc>
 __global__ void __launch_bounds__(256) chanmix_bwd_kernel(const float* __restrict__ dc, const Tl* __restrict__ lat,
@@ -521,6 +526,7 @@ __global__ void __launch_bounds__(256) chanmix_bwd_kernel(const float* __restric
   constexpr int LT = CM_SUB + 4;
   float* latS = dcT + CM_D * LT;          // [K - 1 + CM_SUB rows][CM_D]: latents of the sub-block and its halo
   float* wS = latS + (CM_SUB + CM_KMAX - 1) * CM_D;  // [c][k] seq-conv taps of the head
+  int* tsS = reinterpret_cast<int*>(wS + CM_D * CM_KMAX);  // [t] position of each row in its sequence
   const int h = blockIdx.y, tid = threadIdx.x;
   const bool isq = h < nq;
   const int hh = isq ? h : h - nq;
@@ -548,22 +554,20 @@ __global__ void __launch_bounds__(256) chanmix_bwd_kernel(const float* __restric
       float4 v = make_float4(0.f, 0.f, 0.f, 0.f);
       if (row < r_end) v = *reinterpret_cast<const float4*>(dc + row * W + ccol + c);
       *reinterpret_cast<float4*>(dcR + t * CM_D + c) = v;
-      dcT[(c + 0) * LT + t] = v.x;
-      dcT[(c + 1) * LT + t] = v.y;
-      dcT[(c + 2) * LT + t] = v.z;
-      dcT[(c + 3) * LT + t] = v.w;
     }
+    if (tid < CM_SUB) tsS[tid] = (int)((r0 + tid) % S);
     for (int e = tid; e < (CM_SUB + K - 1) * CM_D; e += 256) {
       const int i = e / CM_D, c = e % CM_D;
       const long long row = r0 - (K - 1) + i;
       latS[i * CM_D + c] = (row >= 0 && row < r_end) ? ld_f(lat + row * Nlat + ccol + c) : 0.f;
     }
     __syncthreads();
-    // s = the seq conv of the latents within each sequence (taps before a sequence start read nothing)
+    // s = the seq conv of the latents within each sequence (taps before a sequence start read
+    // nothing), and dc transposed (a warp's stores spread over eight banks)
     for (int e = tid; e < CM_SUB * CM_D; e += 256) {
       const int t = e / CM_D, c = e % CM_D;
-      const long long row = r0 + t;
-      const int ts = (int)(row % S);
+      dcT[c * LT + t] = dcR[t * CM_D + c];
+      const int ts = tsS[t];
       float sv = 0.f;
       for (int k = 0; k < K; ++k)
         if (ts - (K - 1) + k >= 0) sv = fmaf(wS[c * K + k], latS[(t + k) * CM_D + c], sv);
@@ -820,7 +824,7 @@ size_t up256(size_t v) { return (v + 255) / 256 * 256; }
 
 bool backward_supported(const BlockDims& dm) {
   // the per-token kernel keeps one row's q and K gradients in shared memory
-  return dm.K >= 1 && dm.K <= 8 && dm.d <= 128 && dm.d % 2 == 0 && dm.Lq + dm.Lkv <= 12288 &&
+  return dm.K >= 0 && dm.K <= 8 && dm.d <= 128 && dm.d % 2 == 0 && dm.Lq + dm.Lkv <= 12288 &&
          ((dm.io == DType::BF16 && dm.lat == DType::F16) || (dm.io == DType::F32 && dm.lat == DType::F32));
 }
 
@@ -1014,9 +1018,10 @@ cudaError_t launch_backward(const BlockDims& dm, const BlockPtrs& p, const Backw
     for (int i = 0; i < d / 2; ++i) th.v[i] = pow((double)dm.rope_base, -2.0 * (double)i / (double)d);
     token_bwd_kernel<<<(unsigned)T, 256, sizeof(float) * W, stream>>>(
         dq, dk, dv, dc, dpre, dlat, dm.S, dm.nq, dm.nkv, d, dm.qk_mean_mode, dm.value_shift, dm.vshift_from,
-        dm.use_rope, th);
+        dm.use_rope, th, dm.K == 0);
     if ((e = cudaGetLastError()) != cudaSuccess) return e;
   }
+  if (dm.K > 0) {
   // 5. channel mix: ds = W_c^T dc; dW_c[h] = sum_t dc[t,h]^T s[t,h] (s recomputed from the latents)
   if (d == CM_D) {
     if ((e = cudaMemsetAsync(g.dconvq_chan, 0, sizeof(float) * dm.nq * d * d, stream)) != cudaSuccess ||
@@ -1087,6 +1092,7 @@ cudaError_t launch_backward(const BlockDims& dm, const BlockPtrs& p, const Backw
                                                        g.dconvk_seq, dm.B, dm.S, dm.nq, dm.nkv, d, dm.K, rpb);
     if ((e = cudaGetLastError()) != cudaSuccess) return e;
   }
+  }  // convolutions
   // 7. down-projection: dx = dlat [W_q; W_k; W_v];  dW_* = dlat^T x
   const void* Ws[3] = {p.Wq, p.Wk, p.Wv};
   float* dWs[3] = {g.dWq, g.dWk, g.dWv};

@@ -603,12 +603,14 @@ cca_status_t cca_backward(const cca_config_t* cfg, const void* x, const void* W_
   if (st != CCA_OK) return st;
   if (!backward_supported(dm))
     return fail(CCA_ERR_UNSUPPORTED,
-                "backward needs conv_kernel 1..8, an even head_dim <= 128, n_q_heads + n_kv_heads times head_dim "
+                "backward needs conv_kernel 0..8, an even head_dim <= 128, n_q_heads + n_kv_heads times head_dim "
                 "<= 12288 and bf16 or fp32");
+  const bool plain = dm.K == 0;  // no convolutions: their weights and gradients may be NULL
   static const char* g_names[10] = {"dy",         "dx",          "dW_q",       "dW_k",        "dW_v",
                                     "dconvq_seq", "dconvq_chan", "dconvk_seq", "dconvk_chan", "dW_o"};
   const void* gp[10] = {dy, dx, dW_q, dW_k, dW_v, dconvq_seq, dconvq_chan, dconvk_seq, dconvk_chan, dW_o};
   for (int i = 0; i < 10; ++i) {
+    if (plain && i >= 5 && i <= 8 && gp[i] == nullptr) continue;
     if (gp[i] == nullptr) return fail(CCA_ERR_INVALID_ARG, std::string(g_names[i]) + " is NULL");
     if (!aligned16(gp[i])) return fail(CCA_ERR_INVALID_ARG, std::string(g_names[i]) + " is not 16-byte aligned");
   }
@@ -616,6 +618,7 @@ cca_status_t cca_backward(const cca_config_t* cfg, const void* x, const void* W_
   static const char* in_names[9] = {"x", "W_q", "W_k", "W_v", "convq_seq", "convq_chan", "convk_seq", "convk_chan",
                                     "W_o"};
   for (int i = 0; i < 9; ++i) {
+    if (plain && i >= 4 && i <= 7 && ins[i] == nullptr) continue;
     if (ins[i] == nullptr) return fail(CCA_ERR_INVALID_ARG, std::string(in_names[i]) + " is NULL");
     if (!aligned16(ins[i])) return fail(CCA_ERR_INVALID_ARG, std::string(in_names[i]) + " is not 16-byte aligned");
   }

@@ -334,9 +334,11 @@ cca_status_t cca_decode(const cca_config_t* cfg, int cache_rows,
  *   dW_o        [E, Lq] out            fp32
  *   workspace   >= cca_backward_workspace_size(cfg) bytes, 256-byte aligned,
  *               need not start at zero
- * Every output is overwritten (not accumulated). Supported: conv_kernel 1..8,
- * even head_dim <= 128, dtype bf16 or fp32, and what cca_prefill supports for
- * cfg; all pointers 16-byte aligned, no output aliasing another buffer.
+ * Every output is overwritten (not accumulated). Supported: conv_kernel 0..8
+ * (a plain block, conv_kernel 0, takes NULL for the four conv weights and
+ * their gradients), even head_dim <= 128, (n_q_heads + n_kv_heads) * head_dim
+ * <= 12288, dtype bf16 or fp32, and what cca_prefill supports for cfg; all
+ * pointers 16-byte aligned, no output aliasing another buffer.
  * cca_backward_workspace_size returns 0 for an unsupported or invalid cfg.
  * Errors: INVALID_ARG / UNSUPPORTED / WORKSPACE before any launch, CUDA if a
  * launch fails; device-side conditions (an fp16 intermediate of the forward

@@ -118,6 +118,37 @@ def test_backward_kv_group_share(rank):
     _check(shape, got, ref)
 
 
+PLAIN_CASES = [
+    S_("plain_mha_bf16", 1, 300, 512, 4, 4, 128, 0, "bf16", qk_mean_mode=0, value_shift=0),
+    S_("plain_gqa_fp32", 2, 90, 128, 4, 2, 32, 0, qk_mean_mode=0, value_shift=0),
+]
+
+
+@pytest.mark.parametrize("shape", PLAIN_CASES, ids=[s.name for s in PLAIN_CASES])
+def test_backward_plain_block(shape):
+    """A plain block (no convolutions, QK-mean or value shift: multi-head or grouped attention on the
+    projections) against the oracle's backward of the same block written with one seq-conv tap of 1
+    and identity channel mixes; the gradients of x and the projections must agree."""
+    import numpy as np
+    inp = workloads.make_inputs(shape)
+    dy = workloads.make_dy(shape)
+    cfg = cca.config_from_shape(shape)
+    g = cca.backward(cfg, {k: v.cuda() for k, v in inp.items()}, dy.cuda())
+    assert cca.poll_device_status() == cca.CCA_OK
+    assert set(g) == {"x", "W_q", "W_k", "W_v", "W_o"}
+    nq, nkv, d = shape.n_q_heads, shape.n_kv_heads, shape.head_dim
+    ref_in = workloads.as_float64(inp)
+    ref_in.update(convq_seq=np.ones((nq * d, 1)), convk_seq=np.ones((nkv * d, 1)),
+                  convq_chan=np.broadcast_to(np.eye(d), (nq, d, d)).copy(),
+                  convk_chan=np.broadcast_to(np.eye(d), (nkv, d, d)).copy())
+    ref = oracle.cca_block_backward(ref_in, dy.double().numpy(), nq, nkv, d, qk_mean_mode=0,
+                                    use_value_shift=False, use_rope=bool(shape.use_rope))
+    mx_lim, mean_lim = TOL[shape.dtype]
+    for name in g:
+        mx, mean = _err(g[name].cpu().numpy(), ref[name])
+        assert mx <= mx_lim and (mean_lim is None or mean <= mean_lim), (name, mx, mean)
+
+
 def test_backward_overwrites_outputs():
     """Every gradient is written in full: outputs that start as NaN come back finite and equal to a
     second call's."""
@@ -152,6 +183,6 @@ def test_backward_rejects_bad_arguments():
     assert st == cca.CCA_ERR_INVALID_ARG
     st = lib.cca_backward(ctypes.byref(cfg), *ptrs, dy.data_ptr(), *g, ws.data_ptr(), n - 256, s)
     assert st == cca.CCA_ERR_WORKSPACE
-    plain = cca.config_from_shape(shape.replace(conv_kernel=0, qk_mean_mode=0, value_shift=0))
-    assert cca.backward_workspace_size(plain) == 0
+    too_long = cca.config_from_shape(shape.replace(conv_kernel=9))
+    assert cca.backward_workspace_size(too_long) == 0
     torch.cuda.synchronize()
