@@ -346,6 +346,15 @@ def run_ours(args, shape):
         if world > 1:
             dist.destroy_process_group()
         return 0
+    if args.backward_only:
+        # only the backward pass (cca_backward) is timed (profiling runs)
+        if rank == 0:
+            res = run_backward(cca, dev, my_shape, inputs, load_peaks()[0], steps=args.steps, warmup=args.warmup)
+            print(json.dumps({"mode": "backward-only", "workload": my_shape.name, "backward": res}, default=float),
+                  flush=True)
+        if world > 1:
+            dist.destroy_process_group()
+        return 0
     path_tensor = plan["attention_tensor"]
     launches_per_step = plan["launches"]
 
@@ -696,6 +705,8 @@ def main(argv=None):
                     help="skip timing the plain multi-head block of the same shape (the uncompressed baseline)")
     ap.add_argument("--no-decode", action="store_true", help="skip timing one decode step at position S - 1")
     ap.add_argument("--no-backward", action="store_true", help="skip timing the backward pass (cca_backward)")
+    ap.add_argument("--backward-only", action="store_true",
+                    help="time only cca_backward at the workload (for profiling)")
     ap.add_argument("--decode-only", action="store_true",
                     help="time only the decode step at position S - 1 after one prefill (profiling runs)")
     ap.add_argument("--preproc", choices=sorted(PREPROC_PATHS), default="auto",

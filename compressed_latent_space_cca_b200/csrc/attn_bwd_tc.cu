@@ -17,14 +17,15 @@
 //   (A from TMEM, K_j read MN-major) accumulates in TMEM; the epilogue scales and stores dQ.
 //  dkv kernel (key-stationary): a CTA per (sequence, KV group, 128-key tile, chunk of up to
 //   kUnitsPerChunk (64-query block, head) units) holds K and V and walks its units. S^T = K Q_i^T
-//   and dP^T = V dO_i^T go to TMEM; the softmax warps write P^T and dS^T (fp16) to shared memory,
-//   where they are the K-major A operands of dV += P^T dO_i and dK += dS^T Q_i (Q_i and dO_i read
+//   and dP^T = V dO_i^T go to TMEM; the softmax warps write P^T and dS^T (fp16) over them in TMEM,
+//   where they are the A operands of dV += P^T dO_i and dK += dS^T Q_i (Q_i and dO_i read
 //   MN-major); the epilogue adds the chunk's dK (scaled) and dV to fp32 sums with vector atomics,
 //   so that the long key tiles near the start of a sequence can be split over several CTAs.
-// Both: warp 0 issues the TMA loads, warp 1 the MMAs (an elected lane each); warps 2-9 do the softmax
-// and the epilogue, two per TMEM lane quadrant (warp w reads lanes 32 (w % 4) ..), one row per thread,
-// each of the two taking half of the row's columns. Two TMEM / shared-memory slots let the softmax of
-// one unit overlap the MMAs of its neighbours. Every mbarrier wait is bounded.
+// Both: warp 0 issues the TMA loads, warp 1 the MMAs (an elected lane each); the other warps do the
+// softmax and the epilogue, two (dq) or four (dkv) per TMEM lane quadrant (warp w reads lanes
+// 32 (w % 4) ..), one row per thread, each taking its share of the row's columns. Two TMEM slots let
+// the softmax of one unit overlap the MMAs of its neighbours, and the load rings (three K/V stages,
+// four Q/dO slots) keep the next units' operands in flight. Every mbarrier wait is bounded.
 #include "cca_common.cuh"
 #include "launch.h"
 
@@ -32,8 +33,11 @@ namespace cca {
 namespace {
 
 constexpr int D = 128;
-constexpr int NUM_SM_WARPS = 8;  // softmax / epilogue warps
-constexpr int NUM_THREADS = 64 + 32 * NUM_SM_WARPS;
+// softmax / epilogue warps of each kernel and the columns of a 64-column block each one takes
+// (measured at S = 16384: the dq kernel is fastest with 8, the dkv kernel with 16)
+constexpr int DQ_SM_WARPS = 8, KV_SM_WARPS = 16;
+constexpr int DQ_THREADS = 64 + 32 * DQ_SM_WARPS, KV_THREADS = 64 + 32 * KV_SM_WARPS;
+constexpr int DQ_COLS = 64 / (DQ_SM_WARPS / 4), KV_COLS = 64 / (KV_SM_WARPS / 4);
 constexpr int TMEM_COLS = 512;
 constexpr int SW = 128;  // bytes of one swizzled row (64 fp16)
 
@@ -58,15 +62,15 @@ constexpr int KV_TILE_HALF = KV_KT * SW;          // 16 KB
 constexpr int KV_Q_HALF = KV_QB * SW;             // 8 KB
 constexpr int KV_OFF_K = 0;
 constexpr int KV_OFF_V = KV_OFF_K + 2 * KV_TILE_HALF;
-constexpr int KV_OFF_Q = KV_OFF_V + 2 * KV_TILE_HALF;      // [2 slots][2 halves]
-constexpr int KV_OFF_DO = KV_OFF_Q + 4 * KV_Q_HALF;        // [2 slots][2 halves]
-constexpr int KV_OFF_PT = KV_OFF_DO + 4 * KV_Q_HALF;       // [2 slots] 128 keys x 64 queries
-constexpr int KV_OFF_DST = KV_OFF_PT + 2 * KV_KT * SW;     // [2 slots]
-constexpr int KV_OFF_LSE = KV_OFF_DST + 2 * KV_KT * SW;    // [2 slots][64] fp32
-constexpr int KV_OFF_DELTA = KV_OFF_LSE + 2 * KV_QB * 4;   // [2 slots][64] fp32
-constexpr int KV_OFF_BAR = KV_OFF_DELTA + 2 * KV_QB * 4;
+constexpr int KV_QSLOTS = 4;                               // load ring depth
+constexpr int KV_OFF_Q = KV_OFF_V + 2 * KV_TILE_HALF;      // [slots][2 halves]
+constexpr int KV_OFF_DO = KV_OFF_Q + KV_QSLOTS * 2 * KV_Q_HALF;
+constexpr int KV_OFF_LSE = KV_OFF_DO + KV_QSLOTS * 2 * KV_Q_HALF;  // [slots][64] fp32
+constexpr int KV_OFF_DELTA = KV_OFF_LSE + KV_QSLOTS * KV_QB * 4;   // [slots][64] fp32
+constexpr int KV_OFF_BAR = KV_OFF_DELTA + KV_QSLOTS * KV_QB * 4;
 constexpr size_t KV_SMEM = KV_OFF_BAR + 256 + 1024;
-constexpr uint32_t KV_COL_ST = 0, KV_COL_DPT = 128, KV_COL_DV = 256, KV_COL_DK = 384;  // St, dPt at +64 s
+// St[s], dPt[s] at +64 s; P^T and dS^T (fp16 pairs) overlay the first 32 columns of St[s] and dPt[s]
+constexpr uint32_t KV_COL_ST = 0, KV_COL_DPT = 128, KV_COL_DV = 256, KV_COL_DK = 384;
 constexpr int kUnitsPerChunk = 48;
 static_assert(DQ_SMEM <= 232448 && KV_SMEM <= 232448, "shared memory of one CTA");
 
@@ -106,6 +110,20 @@ __device__ __forceinline__ void tmem_st_32x32b_x16(uint32_t taddr, const uint32_
       : "memory");
 }
 
+__device__ __forceinline__ void tmem_st_32x32b_x8(uint32_t taddr, const uint32_t* r) {
+  asm volatile("tcgen05.st.sync.aligned.32x32b.x8.b32 [%0], {%1,%2,%3,%4,%5,%6,%7,%8};" ::"r"(taddr), "r"(r[0]),
+               "r"(r[1]), "r"(r[2]), "r"(r[3]), "r"(r[4]), "r"(r[5]), "r"(r[6]), "r"(r[7])
+               : "memory");
+}
+__device__ __forceinline__ void tmem_ld_32x32b_x16(uint32_t taddr, uint32_t* r) {
+  asm volatile(
+      "tcgen05.ld.sync.aligned.32x32b.x16.b32"
+      " {%0,%1,%2,%3,%4,%5,%6,%7,%8,%9,%10,%11,%12,%13,%14,%15}, [%16];"
+      : "=r"(r[0]), "=r"(r[1]), "=r"(r[2]), "=r"(r[3]), "=r"(r[4]), "=r"(r[5]), "=r"(r[6]), "=r"(r[7]),
+        "=r"(r[8]), "=r"(r[9]), "=r"(r[10]), "=r"(r[11]), "=r"(r[12]), "=r"(r[13]), "=r"(r[14]), "=r"(r[15])
+      : "r"(taddr));
+}
+
 __device__ __forceinline__ void red_add_v4(float* p, float a, float b, float c, float d) {
   asm volatile("red.global.add.v4.f32 [%0], {%1, %2, %3, %4};" ::"l"(p), "f"(a), "f"(b), "f"(c), "f"(d)
                : "memory");
@@ -118,7 +136,7 @@ __device__ __forceinline__ uint32_t kmaj_step(int kk, int half) {
 }
 
 // ============================================================ dq kernel ==
-__global__ void __launch_bounds__(NUM_THREADS, 1) attn_bwd_dq_kernel(const __grid_constant__ BwdMaps maps,
+__global__ void __launch_bounds__(DQ_THREADS, 1) attn_bwd_dq_kernel(const __grid_constant__ BwdMaps maps,
                                                                      const BwdParams p) {
   extern __shared__ uint8_t smem_raw[];
   uint8_t* smem = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
@@ -149,7 +167,7 @@ __global__ void __launch_bounds__(NUM_THREADS, 1) attn_bwd_dq_kernel(const __gri
     }
     for (int s = 0; s < 2; ++s) {
       mbar_init(smem_u32(&st_full[s]), 1);
-      mbar_init(smem_u32(&ds_full[s]), NUM_SM_WARPS);
+      mbar_init(smem_u32(&ds_full[s]), DQ_SM_WARPS);
     }
     mbar_init(smem_u32(dq_full), 1);
     *abort_flag = 0;
@@ -253,7 +271,7 @@ __global__ void __launch_bounds__(NUM_THREADS, 1) attn_bwd_dq_kernel(const __gri
   } else {
     // ------------------------------------------------------------ softmax --
     const int quad = warp & 3;
-    const int half = (warp - 2) >> 2;  // this warp's 32 of the block's 64 keys
+    const int part = (warp - 2) >> 2;  // this warp's DQ_COLS of the block's 64 keys
     const int r = quad * 32 + lane;
     const int t = qt * DQ_QT + r;
     const bool row_ok = t < p.S;
@@ -268,14 +286,15 @@ __global__ void __launch_bounds__(NUM_THREADS, 1) attn_bwd_dq_kernel(const __gri
       if (!mbar_wait_bounded(smem_u32(&st_full[s]), (j >> 1) & 1, p.err, abort_flag, wait_site(kSiteAttnBwd, 3, 5)))
         goto done;
       tc_fence_after();
-      uint32_t sv[32], dp[32];
-      tmem_ld_32x32b_x32(tmem + lane_off + DQ_COL_S + 64 * s + 32 * half, sv);
-      tmem_ld_32x32b_x32(tmem + lane_off + DQ_COL_DP + 64 * s + 32 * half, dp);
+      static_assert(DQ_COLS == 32, "the dq softmax reads 32 columns a warp");
+      uint32_t sv[DQ_COLS], dp[DQ_COLS];
+      tmem_ld_32x32b_x32(tmem + lane_off + DQ_COL_S + 64 * s + DQ_COLS * part, sv);
+      tmem_ld_32x32b_x32(tmem + lane_off + DQ_COL_DP + 64 * s + DQ_COLS * part, dp);
       tmem_ld_wait();
-      const int key0 = j * DQ_KB + 32 * half;
-      uint32_t pk[16];
+      const int key0 = j * DQ_KB + DQ_COLS * part;
+      uint32_t pk[DQ_COLS / 2];
 #pragma unroll
-      for (int c = 0; c < 32; c += 2) {
+      for (int c = 0; c < DQ_COLS; c += 2) {
         float ds[2];
 #pragma unroll
         for (int e = 0; e < 2; ++e) {
@@ -286,8 +305,8 @@ __global__ void __launch_bounds__(NUM_THREADS, 1) attn_bwd_dq_kernel(const __gri
         }
         pk[c >> 1] = pack_f16x2(ds[0], ds[1]);
       }
-      // keys 2c, 2c + 1 of the block go to packed column c: this half's 16 columns
-      tmem_st_32x32b_x16(tmem + lane_off + DQ_COL_S + 64 * s + 16 * half, pk);
+      // keys 2c, 2c + 1 of the block go to packed column c: this warp's DQ_COLS / 2 columns
+      tmem_st_32x32b_x16(tmem + lane_off + DQ_COL_S + 64 * s + (DQ_COLS / 2) * part, pk);
       tmem_st_wait();
       tc_fence_before();
       __syncwarp();
@@ -298,7 +317,7 @@ __global__ void __launch_bounds__(NUM_THREADS, 1) attn_bwd_dq_kernel(const __gri
     tc_fence_after();
     float* out = p.dq + ((size_t)b * p.S + t) * p.Lq + h * D;
 #pragma unroll 1
-    for (int c4 = 2 * half; c4 < 2 * half + 2; ++c4) {
+    for (int c4 = 2 * part; c4 < 2 * part + 2; ++c4) {  // 64 of the 128 columns per warp
       uint32_t v[32];
       tmem_ld_32x32b_x32(tmem + lane_off + DQ_COL_DQ + 32 * c4, v);
       tmem_ld_wait();
@@ -346,18 +365,17 @@ __device__ __forceinline__ KvItem kv_item(const BwdParams& p, int w) {
   return it;
 }
 
-__global__ void __launch_bounds__(NUM_THREADS, 1) attn_bwd_dkv_kernel(const __grid_constant__ BwdMaps maps,
+__global__ void __launch_bounds__(KV_THREADS, 1) attn_bwd_dkv_kernel(const __grid_constant__ BwdMaps maps,
                                                                       const BwdParams p) {
   extern __shared__ uint8_t smem_raw[];
   uint8_t* smem = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
   uint64_t* bars = reinterpret_cast<uint64_t*>(smem + KV_OFF_BAR);
   uint64_t* kv_full = bars;            // K and V of the tile
-  uint64_t* qd_full = bars + 1;        // [2] Q_i, dO_i, lse2, delta of a unit
-  uint64_t* qd_empty = qd_full + 2;    // [2]
-  uint64_t* st_full = qd_empty + 2;    // [2] S^T, dP^T in TMEM
-  uint64_t* p_full = st_full + 2;      // [2] P^T, dS^T in shared memory (every softmax warp)
-  uint64_t* pt_free = p_full + 2;      // [2] P^T, dS^T read by their MMAs
-  uint64_t* acc_full = pt_free + 2;    // dK, dV complete
+  uint64_t* qd_full = bars + 1;                // [KV_QSLOTS] Q_i, dO_i, lse2, delta of a unit
+  uint64_t* qd_empty = qd_full + KV_QSLOTS;    // [KV_QSLOTS]
+  uint64_t* st_full = qd_empty + KV_QSLOTS;    // [2] S^T, dP^T in TMEM
+  uint64_t* p_full = st_full + 2;      // [2] P^T, dS^T written over them (every softmax warp)
+  uint64_t* acc_full = p_full + 2;     // dK, dV complete
   uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(acc_full + 1);
   volatile int* abort_flag = reinterpret_cast<volatile int*>(tmem_slot + 1);
 
@@ -367,12 +385,13 @@ __global__ void __launch_bounds__(NUM_THREADS, 1) attn_bwd_dkv_kernel(const __gr
 
   if (threadIdx.x == 0) {
     mbar_init(smem_u32(kv_full), 1);
-    for (int s = 0; s < 2; ++s) {
+    for (int s = 0; s < KV_QSLOTS; ++s) {
       mbar_init(smem_u32(&qd_full[s]), 1);
       mbar_init(smem_u32(&qd_empty[s]), 1);
+    }
+    for (int s = 0; s < 2; ++s) {
       mbar_init(smem_u32(&st_full[s]), 1);
-      mbar_init(smem_u32(&p_full[s]), NUM_SM_WARPS);
-      mbar_init(smem_u32(&pt_free[s]), 1);
+      mbar_init(smem_u32(&p_full[s]), KV_SM_WARPS);
     }
     mbar_init(smem_u32(acc_full), 1);
     *abort_flag = 0;
@@ -406,9 +425,9 @@ __global__ void __launch_bounds__(NUM_THREADS, 1) attn_bwd_dkv_kernel(const __gr
                     it.kt * KV_KT, it.b);
     }
     for (int n = 0; n < n_units; ++n) {
-      const int u = it.u0 + n, s = n & 1;
+      const int u = it.u0 + n, s = n % KV_QSLOTS;
       const int qb = it.nqb0 + u / p.G, h = it.g * p.G + u % p.G;
-      if (!mbar_wait_bounded(smem_u32(&qd_empty[s]), ((n >> 1) & 1) ^ 1, p.err, abort_flag,
+      if (!mbar_wait_bounded(smem_u32(&qd_empty[s]), ((n / KV_QSLOTS) & 1) ^ 1, p.err, abort_flag,
                              wait_site(kSiteAttnBwd, 4, 1)))
         break;
       if (elect_one_sync()) mbar_arrive_expect_tx(smem_u32(&qd_full[s]), 4 * KV_Q_HALF + 2 * KV_QB * 4);
@@ -431,7 +450,7 @@ __global__ void __launch_bounds__(NUM_THREADS, 1) attn_bwd_dkv_kernel(const __gr
   } else if (warp == 1) {
     // ---------------------------------------------------------------- MMA --
     const uint32_t idesc_st = idesc_f32acc(KV_KT, KV_QB, 0, 0, kFmtF16);  // K (V) and Q (dO) K-major
-    const uint32_t idesc_acc = idesc_f32acc(KV_KT, D, 0, 1, kFmtF16);     // P^T (dS^T) K-major, dO (Q) MN-major
+    const uint32_t idesc_acc = idesc_f32acc(KV_KT, D, 0, 1, kFmtF16);     // P^T (dS^T) from TMEM, dO (Q) MN-major
     const uint32_t sw_hi = desc_hi(smem_desc_sw128(smem_u32(smem), 16, 1024));
     const uint32_t mn_hi = desc_hi(smem_desc_sw128(smem_u32(smem), KV_Q_HALF, 1024));
     const uint32_t k_lo = desc_lo(smem_desc_sw128(smem_u32(smem + KV_OFF_K), 16, 1024));
@@ -440,110 +459,101 @@ __global__ void __launch_bounds__(NUM_THREADS, 1) attn_bwd_dkv_kernel(const __gr
     const uint32_t do_lo = desc_lo(smem_desc_sw128(smem_u32(smem + KV_OFF_DO), 16, 1024));
     const uint32_t qmn_lo = desc_lo(smem_desc_sw128(smem_u32(smem + KV_OFF_Q), KV_Q_HALF, 1024));
     const uint32_t domn_lo = desc_lo(smem_desc_sw128(smem_u32(smem + KV_OFF_DO), KV_Q_HALF, 1024));
-    const uint32_t pt_lo = desc_lo(smem_desc_sw128(smem_u32(smem + KV_OFF_PT), 16, 1024));
-    const uint32_t dst_lo = desc_lo(smem_desc_sw128(smem_u32(smem + KV_OFF_DST), 16, 1024));
-    constexpr uint32_t kQSlot = (2 * KV_Q_HALF) >> 4, kPSlot = (KV_KT * SW) >> 4;
+    constexpr uint32_t kQSlot = (2 * KV_Q_HALF) >> 4;
     if (!mbar_wait_bounded(smem_u32(kv_full), 0, p.err, abort_flag, wait_site(kSiteAttnBwd, 5, 2))) goto done;
     tc_fence_after();
     for (int n = 0; n <= n_units; ++n) {
       if (n < n_units) {
-        const int s = n & 1;
-        if (!mbar_wait_bounded(smem_u32(&qd_full[s]), (n >> 1) & 1, p.err, abort_flag, wait_site(kSiteAttnBwd, 5, 3)))
+        const int s = n & 1, q = n % KV_QSLOTS;  // TMEM slot, load slot
+        if (!mbar_wait_bounded(smem_u32(&qd_full[q]), (n / KV_QSLOTS) & 1, p.err, abort_flag,
+                               wait_site(kSiteAttnBwd, 5, 3)))
           goto done;
         tc_fence_after();
         // S^T[s] = K Q_i^T, dP^T[s] = V dO_i^T; slot s was last read by the softmax of unit n - 2,
-        // whose p_full this loop waited for at n - 1
+        // whose p_full this loop waited for at n - 1, and by the dV / dK MMAs of unit n - 2 issued
+        // before (tcgen05 MMAs of one thread run in order)
 #pragma unroll
         for (int kk = 0; kk < D / 16; ++kk)
           if (elect_one_sync())
             umma_ss_lohi(tmem + KV_COL_ST + 64 * s, k_lo + kmaj_step(kk, KV_TILE_HALF), sw_hi,
-                         q_lo + s * kQSlot + kmaj_step(kk, KV_Q_HALF), sw_hi, idesc_st, kk > 0);
+                         q_lo + q * kQSlot + kmaj_step(kk, KV_Q_HALF), sw_hi, idesc_st, kk > 0);
 #pragma unroll
         for (int kk = 0; kk < D / 16; ++kk)
           if (elect_one_sync())
             umma_ss_lohi(tmem + KV_COL_DPT + 64 * s, v_lo + kmaj_step(kk, KV_TILE_HALF), sw_hi,
-                         do_lo + s * kQSlot + kmaj_step(kk, KV_Q_HALF), sw_hi, idesc_st, kk > 0);
+                         do_lo + q * kQSlot + kmaj_step(kk, KV_Q_HALF), sw_hi, idesc_st, kk > 0);
         if (elect_one_sync()) umma_commit(smem_u32(&st_full[s]));
       }
       if (n >= 1) {
-        const int np = n - 1, sp = np & 1;
+        const int np = n - 1, sp = np & 1, qp = np % KV_QSLOTS;
         if (!mbar_wait_bounded(smem_u32(&p_full[sp]), (np >> 1) & 1, p.err, abort_flag, wait_site(kSiteAttnBwd, 5, 4)))
           goto done;
         tc_fence_after();
-        // dV += P^T dO_i and dK += dS^T Q_i: A = [128 keys x 64 queries] K-major (one 128-byte row per
-        // key), B = dO_i / Q_i read as [d x queries] MN-major; 16 queries per MMA
+        // dV += P^T dO_i and dK += dS^T Q_i: A = [128 keys x 64 queries] from TMEM (fp16 pairs, 8
+        // columns per 16 queries), B = dO_i / Q_i read as [d x queries] MN-major; 16 queries per MMA
 #pragma unroll
         for (int kk = 0; kk < KV_QB / 16; ++kk) {
           const uint32_t bstep = (uint32_t)((kk * 16 * SW) >> 4);
           if (elect_one_sync())
-            umma_ss_lohi(tmem + KV_COL_DV, pt_lo + sp * kPSlot + 2 * kk, sw_hi, domn_lo + sp * kQSlot + bstep, mn_hi,
+            umma_ts_lohi(tmem + KV_COL_DV, tmem + KV_COL_ST + 64 * sp + kk * 8, domn_lo + qp * kQSlot + bstep, mn_hi,
                          idesc_acc, np > 0 || kk > 0);
           if (elect_one_sync())
-            umma_ss_lohi(tmem + KV_COL_DK, dst_lo + sp * kPSlot + 2 * kk, sw_hi, qmn_lo + sp * kQSlot + bstep, mn_hi,
+            umma_ts_lohi(tmem + KV_COL_DK, tmem + KV_COL_DPT + 64 * sp + kk * 8, qmn_lo + qp * kQSlot + bstep, mn_hi,
                          idesc_acc, np > 0 || kk > 0);
         }
-        if (elect_one_sync()) umma_commit(smem_u32(&qd_empty[sp]));
-        if (elect_one_sync()) umma_commit(smem_u32(&pt_free[sp]));
+        if (elect_one_sync()) umma_commit(smem_u32(&qd_empty[qp]));
       }
     }
     if (elect_one_sync()) umma_commit(smem_u32(acc_full));
   } else {
     // ------------------------------------------------------------ softmax --
     const int quad = warp & 3;
-    const int half = (warp - 2) >> 2;  // this warp's 32 of a unit's 64 queries
+    const int part = (warp - 2) >> 2;  // this warp's KV_COLS of a unit's 64 queries
     const int r = quad * 32 + lane;
     const int key = it.kt * KV_KT + r;
     const uint32_t lane_off = (uint32_t)(quad * 32) << 16;
     const float c2 = p.c2;
     bool bad = false;
     for (int n = 0; n < n_units; ++n) {
-      const int u = it.u0 + n, s = n & 1;
+      const int u = it.u0 + n, s = n & 1, q = n % KV_QSLOTS;
       const int q0 = (it.nqb0 + u / p.G) * KV_QB;
       if (!mbar_wait_bounded(smem_u32(&st_full[s]), (n >> 1) & 1, p.err, abort_flag, wait_site(kSiteAttnBwd, 6, 5)))
         goto done;
       tc_fence_after();
-      uint32_t sv[32], dp[32];
-      tmem_ld_32x32b_x32(tmem + lane_off + KV_COL_ST + 64 * s + 32 * half, sv);
-      tmem_ld_32x32b_x32(tmem + lane_off + KV_COL_DPT + 64 * s + 32 * half, dp);
+      static_assert(KV_COLS == 16, "the dkv softmax reads 16 columns a warp");
+      uint32_t sv[KV_COLS], dp[KV_COLS];
+      tmem_ld_32x32b_x16(tmem + lane_off + KV_COL_ST + 64 * s + KV_COLS * part, sv);
+      tmem_ld_32x32b_x16(tmem + lane_off + KV_COL_DPT + 64 * s + KV_COLS * part, dp);
       tmem_ld_wait();
-      // the MMAs of unit n - 2 have finished reading this slot's P^T and dS^T
-      if (n >= 2 && !mbar_wait_bounded(smem_u32(&pt_free[s]), ((n >> 1) & 1) ^ 1, p.err, abort_flag,
-                                       wait_site(kSiteAttnBwd, 6, 6)))
-        goto done;
       // lse2 and delta of this unit came by bulk copy: observe its completion here too (the slot
       // cannot be refilled before this warp's p_full, so this is the unit's own phase)
-      if (!mbar_wait_bounded(smem_u32(&qd_full[s]), (n >> 1) & 1, p.err, abort_flag, wait_site(kSiteAttnBwd, 6, 8)))
+      if (!mbar_wait_bounded(smem_u32(&qd_full[q]), (n / KV_QSLOTS) & 1, p.err, abort_flag,
+                             wait_site(kSiteAttnBwd, 6, 8)))
         goto done;
-      const float* lse_s = reinterpret_cast<const float*>(smem + KV_OFF_LSE + s * KV_QB * 4);
-      const float* del_s = reinterpret_cast<const float*>(smem + KV_OFF_DELTA + s * KV_QB * 4);
-      uint8_t* prow = smem + KV_OFF_PT + s * KV_KT * SW + r * SW;
-      uint8_t* drow = smem + KV_OFF_DST + s * KV_KT * SW + r * SW;
+      const float* lse_s = reinterpret_cast<const float*>(smem + KV_OFF_LSE + q * KV_QB * 4);
+      const float* del_s = reinterpret_cast<const float*>(smem + KV_OFF_DELTA + q * KV_QB * 4);
+      uint32_t pp[KV_COLS / 2], dd[KV_COLS / 2];  // this warp's queries 2c, 2c + 1 -> packed column c
 #pragma unroll
-      for (int cc = 0; cc < 4; ++cc) {  // 8 queries per 16-byte chunk: chunks 4 half .. 4 half + 3
-        const int ch = 4 * half + cc;
-        uint32_t pp[4], dd[4];
+      for (int c2i = 0; c2i < KV_COLS / 2; ++c2i) {
+        float pv[2], dv[2];
 #pragma unroll
-        for (int e = 0; e < 4; ++e) {
-          float pv[2], dv[2];
-#pragma unroll
-          for (int f = 0; f < 2; ++f) {
-            const int cl = 8 * cc + 2 * e + f;  // column within this warp's half
-            const int c = 32 * half + cl;
-            const int t = q0 + c;
-            const bool vis = key <= t && t < p.S;
-            const float pr = vis ? fast_exp2(fmaf(u2f(sv[cl]), c2, -lse_s[c])) : 0.f;
-            pv[f] = pr;
-            dv[f] = vis ? pr * (u2f(dp[cl]) - del_s[c]) : 0.f;
-            bad |= f16_overflow(dv[f]);
-          }
-          pp[e] = pack_f16x2(pv[0], pv[1]);
-          dd[e] = pack_f16x2(dv[0], dv[1]);
+        for (int f = 0; f < 2; ++f) {
+          const int cl = 2 * c2i + f;  // column within this warp's share
+          const int c = KV_COLS * part + cl;
+          const int t = q0 + c;
+          const bool vis = key <= t && t < p.S;
+          const float pr = vis ? fast_exp2(fmaf(u2f(sv[cl]), c2, -lse_s[c])) : 0.f;
+          pv[f] = pr;
+          dv[f] = vis ? pr * (u2f(dp[cl]) - del_s[c]) : 0.f;
+          bad |= f16_overflow(dv[f]);
         }
-        const int off = ((ch ^ (r & 7)) << 4);
-        *reinterpret_cast<uint4*>(prow + off) = make_uint4(pp[0], pp[1], pp[2], pp[3]);
-        *reinterpret_cast<uint4*>(drow + off) = make_uint4(dd[0], dd[1], dd[2], dd[3]);
+        pp[c2i] = pack_f16x2(pv[0], pv[1]);
+        dd[c2i] = pack_f16x2(dv[0], dv[1]);
       }
-      fence_async_smem();  // the generic-proxy stores above are read by the tensor core
+      // P^T over S^T[s] and dS^T over dP^T[s] (both already read above)
+      tmem_st_32x32b_x8(tmem + lane_off + KV_COL_ST + 64 * s + (KV_COLS / 2) * part, pp);
+      tmem_st_32x32b_x8(tmem + lane_off + KV_COL_DPT + 64 * s + (KV_COLS / 2) * part, dd);
+      tmem_st_wait();
       tc_fence_before();
       __syncwarp();
       if (lane == 0) mbar_arrive(smem_u32(&p_full[s]));
@@ -554,7 +564,7 @@ __global__ void __launch_bounds__(NUM_THREADS, 1) attn_bwd_dkv_kernel(const __gr
     const bool key_ok = key < p.S;
     const size_t orow = ((size_t)it.b * p.S + key) * p.Lkv + it.g * D;
 #pragma unroll 1
-    for (int c4 = 2 * half; c4 < 2 * half + 2; ++c4) {
+    for (int c4 = part; c4 < part + 1; ++c4) {  // 32 of the 128 columns per warp
       uint32_t v[32], k[32];
       tmem_ld_32x32b_x32(tmem + lane_off + KV_COL_DV + 32 * c4, v);
       tmem_ld_32x32b_x32(tmem + lane_off + KV_COL_DK + 32 * c4, k);
@@ -632,7 +642,7 @@ cudaError_t launch_attention_bwd_tc(const BlockDims& dm, const AttnBwdPtrs& a, u
         cudaSuccess)
       return e;
     const unsigned grid = (unsigned)(dm.B * dm.nq * ((dm.S + DQ_QT - 1) / DQ_QT));
-    attn_bwd_dq_kernel<<<grid, NUM_THREADS, DQ_SMEM, stream>>>(m, p);
+    attn_bwd_dq_kernel<<<grid, DQ_THREADS, DQ_SMEM, stream>>>(m, p);
     if ((e = cudaGetLastError()) != cudaSuccess) return e;
   }
   {
@@ -644,7 +654,7 @@ cudaError_t launch_attention_bwd_tc(const BlockDims& dm, const AttnBwdPtrs& a, u
         cudaSuccess)
       return e;
     const unsigned grid = (unsigned)(dm.B * dm.nkv * p.chunks);
-    attn_bwd_dkv_kernel<<<grid, NUM_THREADS, KV_SMEM, stream>>>(m, p);
+    attn_bwd_dkv_kernel<<<grid, KV_THREADS, KV_SMEM, stream>>>(m, p);
     if ((e = cudaGetLastError()) != cudaSuccess) return e;
   }
   return cudaSuccess;
