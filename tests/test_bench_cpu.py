@@ -30,9 +30,19 @@ def test_algorithmic_work_of_the_headline_workload():
     assert w["attention_flops"] == 2.0 * 4 * 16384 ** 2 * 128          # 274.9 GFLOP, causal half
     assert w["down_proj_flops"] == 2.0 * 16384 * 2048 * 1024           # 68.7 GFLOP
     assert w["out_proj_flops"] == 2.0 * 16384 * 512 * 2048             # 34.4 GFLOP
-    # 67.1 MB of latents in and q / K / V cache out, plus fp16 attention copies of k and v (16.8 MB)
-    # and the fp16 copy of W_o (4.2 MB)
-    assert w["preproc_bytes"] == 16384 * (1024 + 512 + 512) * 2.0 + 2 * 16384 * 256 * 2 + 2 * 2048 * 512 * 2
+    # the roofline's bytes: 67.1 MB of latents in and q / K / V cache out
+    assert w["preproc_bytes"] == 16384 * (1024 + 512 + 512) * 2.0
+    # moved by this design: plus fp16 attention copies of k and v (16.8 MB) and the fp16 W_o (4.2 MB)
+    assert w["preproc_bytes_moved"] == w["preproc_bytes"] + 2 * 16384 * 256 * 2 + 2 * 2048 * 512 * 2
+
+
+def test_backward_flops_of_the_headline_workload():
+    w = bench.algorithmic_work(workloads.WORKLOADS["ccgqa_16k_bf16"])
+    f = bench.backward_flops(workloads.WORKLOADS["ccgqa_16k_bf16"])
+    # five products of the forward attention's QK^T size (2.5 x its two), two GEMMs per projection
+    assert f["attention_backward"] == 2.5 * w["attention_flops"]
+    assert f["projections_backward"] == 2 * (w["down_proj_flops"] + w["out_proj_flops"])
+    assert f["total"] == f["forward"] + f["attention_backward"] + f["projections_backward"]
 
 
 def test_warmup_floor():
