@@ -1023,7 +1023,13 @@ cudaError_t launch_backward(const BlockDims& dm, const BlockPtrs& p, const Backw
   }
   if (dm.K > 0) {
   // 5. channel mix: ds = W_c^T dc; dW_c[h] = sum_t dc[t,h]^T s[t,h] (s recomputed from the latents)
-  if (d == CM_D) {
+  if (tc_gemm && it == DType::BF16 && chanmix_bwd_tc_supported(dm)) {  // tensor cores (bf16 W_c is exact)
+    if ((e = cudaMemsetAsync(g.dconvq_chan, 0, sizeof(float) * dm.nq * d * d, stream)) != cudaSuccess ||
+        (e = cudaMemsetAsync(g.dconvk_chan, 0, sizeof(float) * dm.nkv * d * d, stream)) != cudaSuccess ||
+        (e = launch_chanmix_bwd_tc(dm, dc, p.qkv_lat, p.cq_chan, p.ck_chan, p.cq_seq, p.ck_seq, ds, g.dconvq_chan,
+                                   g.dconvk_chan, p.dev_err, stream)) != cudaSuccess)
+      return e;
+  } else if (d == CM_D) {
     if ((e = cudaMemsetAsync(g.dconvq_chan, 0, sizeof(float) * dm.nq * d * d, stream)) != cudaSuccess ||
         (e = cudaMemsetAsync(g.dconvk_chan, 0, sizeof(float) * dm.nkv * d * d, stream)) != cudaSuccess)
       return e;

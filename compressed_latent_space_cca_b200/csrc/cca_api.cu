@@ -666,11 +666,11 @@ cca_status_t cca_poll_device_status(void* stream) {
       return cuda_fail("clear device error word", e);
     if ((h & 0xffu) == kDevErrRange)
       return fail(CCA_ERR_NUMERIC_RANGE, "an intermediate exceeded the fp16 range (|value| > 65504)");
-    static const char* kernels[7] = {"?",         "gemm", "attention", "self-test", "?", "preprocessing (tcgen05)",
-                                     "attention backward"};
+    static const char* kernels[8] = {"?",         "gemm", "attention", "self-test", "?", "preprocessing (tcgen05)",
+                                     "attention backward", "channel-mix backward"};
     char msg[160];
     snprintf(msg, sizeof(msg), "a bounded device-side wait gave up (kernel %s, role %u, barrier %u)",
-             kernels[((h >> 8) & 0xffu) < 7 ? ((h >> 8) & 0xffu) : 0], (h >> 16) & 0xffu, (h >> 24) & 0xffu);
+             kernels[((h >> 8) & 0xffu) < 8 ? ((h >> 8) & 0xffu) : 0], (h >> 16) & 0xffu, (h >> 24) & 0xffu);
     return fail(CCA_ERR_DEVICE_TIMEOUT, msg);
   }
   return CCA_OK;

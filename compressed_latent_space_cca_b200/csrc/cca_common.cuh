@@ -122,7 +122,8 @@ enum WaitKernel : unsigned {
   kSiteSelftest = 3,
   kSitePreUmma = 4,
   kSitePreWs = 5,
-  kSiteAttnBwd = 6
+  kSiteAttnBwd = 6,
+  kSiteChanmix = 7
 };
 
 // Waits for phase `parity` of the mbarrier to complete. Gives up after

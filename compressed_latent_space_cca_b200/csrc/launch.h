@@ -173,7 +173,13 @@ struct BackwardLayout {
   int stat_stride;  // lse / delta rows of the tensor-core path: [B][nq][stat_stride]
   int Tp;           // tokens rounded up to a multiple of 64
 };
-// conv_kernel 1..8, head_dim <= 128 (even), io bf16 or fp32
+// The channel-mix backward on the tensor cores (head_dim 128, K <= 8): ds written, dW_c added to
+// (fp32; cleared by the caller)
+bool chanmix_bwd_tc_supported(const BlockDims& dm);
+cudaError_t launch_chanmix_bwd_tc(const BlockDims& dm, const float* dc, const void* lat, const void* cq_chan,
+                                  const void* ck_chan, const void* cq_seq, const void* ck_seq, float* ds, float* dwq,
+                                  float* dwk, unsigned* err, cudaStream_t stream);
+// conv_kernel 0..8, head_dim <= 128 (even), io bf16 or fp32
 bool backward_supported(const BlockDims& dm);
 BackwardLayout backward_layout(const BlockDims& dm, size_t forward_bytes);
 // tc_attention: the forward ran the tensor-core attention with p.lse2 set (BackwardLayout::lse);
