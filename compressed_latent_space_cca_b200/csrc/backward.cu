@@ -264,7 +264,8 @@ __global__ void __launch_bounds__(256, 2) row_stats_kernel(const Tl* __restrict_
 // [B][nq][stride] layout it reads. A warp per (row, head) of head_dim 128: four columns a lane.
 __global__ void __launch_bounds__(256) do_prep_kernel(const float* __restrict__ dO, const __half* __restrict__ o,
                                                       __half* __restrict__ dO16, float* __restrict__ delta, long long T,
-                                                      int S, int nq, int stride) {
+                                                      int S, int nq, int stride, __nv_bfloat16* __restrict__ o_planes,
+                                                      long long Tp) {
   const long long wid = (long long)blockIdx.x * 8 + (threadIdx.x >> 5);
   const int lane = threadIdx.x & 31;
   if (wid >= T * nq) return;
@@ -276,6 +277,19 @@ __global__ void __launch_bounds__(256) do_prep_kernel(const float* __restrict__ 
   const __half2 o01 = *reinterpret_cast<const __half2*>(&ov.x), o23 = *reinterpret_cast<const __half2*>(&ov.y);
   float dl = g.x * __low2float(o01) + g.y * __high2float(o01) + g.z * __low2float(o23) + g.w * __high2float(o23);
   *reinterpret_cast<uint2*>(dO16 + off) = make_uint2(pack_f16x2(g.x, g.y), pack_f16x2(g.z, g.w));
+  if (o_planes != nullptr) {  // O as bf16 hi / lo planes [2][Tp][Lq] (the dW_o GEMM's operand)
+    const float of[4] = {__low2float(o01), __high2float(o01), __low2float(o23), __high2float(o23)};
+    float hf[4], lf[4];
+#pragma unroll
+    for (int u = 0; u < 4; ++u) {
+      const __nv_bfloat16 hb = __float2bfloat16_rn(of[u]);
+      hf[u] = __bfloat162float(hb);
+      lf[u] = of[u] - hf[u];
+    }
+    *reinterpret_cast<uint2*>(o_planes + off) = make_uint2(pack_bf16x2(hf[0], hf[1]), pack_bf16x2(hf[2], hf[3]));
+    *reinterpret_cast<uint2*>(o_planes + Tp * nq * 128 + off) =
+        make_uint2(pack_bf16x2(lf[0], lf[1]), pack_bf16x2(lf[2], lf[3]));
+  }
 #pragma unroll
   for (int m = 16; m > 0; m >>= 1) dl += __shfl_xor_sync(0xffffffffu, dl, m);
   if (lane == 0) {
@@ -426,6 +440,29 @@ __global__ void __launch_bounds__(256) attn_bwd_kernel(const Tl* __restrict__ q,
   }
 }
 
+// Where the latents' gradient goes: fp32 [T, Nlat] (f32), or for the tensor-core GEMMs its bf16 pair
+// hi = bf16(v), lo = bf16(v - hi) twice: row-major [T][hi Nlat | lo Nlat] (rm, the dx GEMM's K-major
+// operand) and as two planes [2][Tp][Nlat] (planes, the weight-gradient GEMMs' MN-major operand).
+struct DlatOut {
+  float* f32;
+  __nv_bfloat16* rm;
+  __nv_bfloat16* planes;
+  int Nlat;
+  long long Tp;
+};
+
+__device__ __forceinline__ void store_dlat(const DlatOut& o, long long row, int col, float v) {
+  if (o.f32 != nullptr) {
+    o.f32[row * o.Nlat + col] = v;
+  } else {
+    const __nv_bfloat16 hi = __float2bfloat16_rn(v), lo = __float2bfloat16_rn(v - __bfloat162float(hi));
+    o.rm[row * 2 * o.Nlat + col] = hi;
+    o.rm[row * 2 * o.Nlat + o.Nlat + col] = lo;
+    o.planes[row * o.Nlat + col] = hi;
+    o.planes[(o.Tp + row) * o.Nlat + col] = lo;
+  }
+}
+
 // ------------------------------------------------------------------ per-token backward --
 // Row t of one sequence: dq, dk turned back by RoPE; the QK-mean transpose gives dc (the
 // channel-mix outputs' gradient) and the latents' direct gradient dpre; dv goes through the value
@@ -437,7 +474,7 @@ struct Theta64 {
 
 __global__ void __launch_bounds__(256) token_bwd_kernel(const float* __restrict__ dq, const float* __restrict__ dk,
                                                         const float* __restrict__ dv, float* __restrict__ dc,
-                                                        float* __restrict__ dpre, float* __restrict__ dlat, int S,
+                                                        float* __restrict__ dpre, const DlatOut dlat, int S,
                                                         int nq, int nkv, int d, int mode, int vshift, int vfrom,
                                                         int use_rope, const __grid_constant__ Theta64 theta,
                                                         int plain) {
@@ -487,7 +524,7 @@ __global__ void __launch_bounds__(256) token_bwd_kernel(const float* __restrict_
       bsum = a;
     }
     if (plain) {  // no convolutions: the attention inputs are the latents
-      dlat[row * Nlat + e] = direct;
+      store_dlat(dlat, row, e, direct);
     } else {
       dc[row * (Lq + Lkv) + e] = direct + P * bsum;
       dpre[row * (Lq + Lkv) + e] = R * a;
@@ -498,7 +535,7 @@ __global__ void __launch_bounds__(256) token_bwd_kernel(const float* __restrict_
     float val;
     if (vshift && c >= vfrom) val = (t + 1 < S) ? dv[(row + 1) * Lkv + c] : 0.f;
     else val = dv[row * Lkv + c];
-    dlat[row * Nlat + Lq + Lkv + c] = val;
+    store_dlat(dlat, row, Lq + Lkv + c, val);
   }
 }
 
@@ -657,10 +694,10 @@ __global__ void __launch_bounds__(256) chan_bwd_kernel(const float* __restrict__
 template <typename Tc>
 __global__ void __launch_bounds__(256) seq_bwd_kernel(const float* __restrict__ ds, const float* __restrict__ dpre,
                                                       const Tc* __restrict__ cq_seq, const Tc* __restrict__ ck_seq,
-                                                      float* __restrict__ dlat, int S, int nq, int nkv, int d, int K) {
+                                                      const DlatOut dlat, int S, int nq, int nkv, int d, int K) {
   const long long row = blockIdx.x;
   const int t = (int)(row % S);
-  const int Lq = nq * d, Lkv = nkv * d, Nlat = Lq + 2 * Lkv, W = Lq + Lkv;
+  const int Lq = nq * d, Lkv = nkv * d, W = Lq + Lkv;
   for (int e = threadIdx.x; e < W; e += blockDim.x) {
     const bool isq = e < Lq;
     const int c = isq ? e : e - Lq;
@@ -670,7 +707,7 @@ __global__ void __launch_bounds__(256) seq_bwd_kernel(const float* __restrict__ 
       const int tt = t + K - 1 - j;
       if (tt < S) acc = fmaf(ld_f(w + j), ds[(row - t + tt) * W + e], acc);
     }
-    dlat[row * Nlat + e] = acc;
+    store_dlat(dlat, row, e, acc);
   }
 }
 
@@ -715,7 +752,7 @@ __global__ void __launch_bounds__(256) tap_grad_kernel(const float* __restrict__
 // Operands of the tensor-core GEMMs are bf16. A value v that bf16 does not hold exactly is carried as
 // the pair hi = bf16(v), lo = bf16(v - hi) (about 16 significant bits, bf16's exponent range), laid
 // side by side along the contraction so that one GEMM with a K two or three times longer sums
-// hi*b + lo*b; the other operand repeats its bf16 values over the same segments ("Leveraging the
+// hi*b + lo*b; the other operand, stored once, repeats along K (the GEMM's K wrap) ("Leveraging the
 // bfloat16 artificial intelligence datatype for higher-precision computations", Henry et al., 2019).
 enum SegKind : int { kSegNone = 0, kSegHi = 1, kSegLo = 2 };
 struct Segs {
@@ -794,11 +831,31 @@ cudaError_t transpose_bf16(Mat in, long long ldi, int R, int C, int Rp, __nv_bfl
   return cudaGetLastError();
 }
 
+// How the tcgen05 GEMM reads an operand: K wrap period and the K it holds (0: K), MN-major layout
+// ([K][M or N]) and its row stride (0: dense)
+struct Opnd {
+  int kwrap = 0, kext = 0, mn = 0;
+  long long ld = 0;
+};
+Opnd wrap(int period) {
+  Opnd o;
+  o.kwrap = period;
+  return o;
+}
+
 // C[M, N] (fp32, row stride ldc, contiguous rows) = A[M, K] B[N, K]^T on the tensor cores, bf16
 // operands; a long K over few output tiles is split (C cleared, slices added)
 cudaError_t gemm_tc_bf16(const void* A, long long M, const void* B, int N, int K, float* C, long long ldc,
-                         unsigned* err, cudaStream_t s) {
+                         unsigned* err, cudaStream_t s, Opnd ao = Opnd(), Opnd bo = Opnd()) {
   GemmTcArgs a{};
+  a.a_kwrap = ao.kwrap;
+  a.a_kext = ao.kext;
+  a.a_mn = ao.mn;
+  a.lda = ao.ld;
+  a.b_kwrap = bo.kwrap;
+  a.b_kext = bo.kext;
+  a.b_mn = bo.mn;
+  a.ldb = bo.ld;
   a.ksplit = gemm_tc_ksplit(M, N, K);
   if (a.ksplit > 1) {
     const cudaError_t e = cudaMemsetAsync(C, 0, sizeof(float) * ((size_t)(M - 1) * ldc + N), s);
@@ -870,13 +927,13 @@ BackwardLayout backward_layout(const BlockDims& dm, size_t forward_bytes) {
   // GEMM's 64-deep K step), row-major copies, transposed weights
   L.Tp = (T + 63) / 64 * 64;
   const size_t h = 2, Tp = (size_t)L.Tp;
-  // (up to three segments along the contraction, see Segs)
+  // (segments along the contraction, see Segs)
   L.dy16 = off;
   off = up256(off + h * T * dm.E * 2);
   L.dy_t = off;
-  off = up256(off + h * dm.E * Tp * 3);
-  L.x_t = off;
   off = up256(off + h * dm.E * Tp * 2);
+  L.x_t = off;
+  off = up256(off + h * dm.E * Tp);
   L.o_t = off;
   off = up256(off + h * dm.Lq * Tp * 3);
   L.dlat16 = off;
@@ -884,9 +941,11 @@ BackwardLayout backward_layout(const BlockDims& dm, size_t forward_bytes) {
   L.dlat_t = off;
   off = up256(off + h * dm.Nlat * Tp * 2);
   L.wo_t = off;
-  off = up256(off + h * dm.Lq * dm.E * 2);
+  off = up256(off + h * dm.Lq * dm.E);
   L.w_t = off;
-  off = up256(off + h * dm.E * dm.Nlat * 2);
+  off = up256(off + h * dm.E * dm.Nlat);
+  L.dw_all = off;  // fp32 [Nlat, E]: the three weight gradients of the down-projection from one GEMM
+  off = up256(off + f * dm.Nlat * dm.E);
   L.total = off;
   return L;
 }
@@ -917,32 +976,42 @@ cudaError_t launch_backward(const BlockDims& dm, const BlockPtrs& p, const Backw
   __nv_bfloat16* dlat_t = reinterpret_cast<__nv_bfloat16*>(ws + L.dlat_t);
   __nv_bfloat16* wo_t = reinterpret_cast<__nv_bfloat16*>(ws + L.wo_t);
   __nv_bfloat16* w_t = reinterpret_cast<__nv_bfloat16*>(ws + L.w_t);
-  // 1. dO = dy W_o  [T, Lq];  dW_o = dy^T O  [E, Lq]
-  if (tc_gemm) {
+  // The tensor-core GEMMs read dy, x and W_o in place (MN-major where they are the transposed operand);
+  // the latents' gradient and O come as bf16 hi / lo forms written by the kernels that make them.
+  // An fp32 dy, or a block whose attention ran on the CUDA cores, takes bf16 copies made by transposes.
+  const bool direct = tc_gemm && tc_attention && ot == DType::BF16;
+  const long long TpLL = Tp;
+  // 1. dO = dy W_o  [T, Lq];  dW_o = dy^T O  [E, Lq] (after step 2 on the direct path)
+  if (direct) {
+    Opnd wo;  // W_o [E][Lq] is [K][N]
+    wo.mn = 1;
+    wo.ld = Lq;
+    if ((e = gemm_tc_bf16(g.dy, T, p.Wo, Lq, E, dO, Lq, p.dev_err, stream, Opnd(), wo)) != cudaSuccess) return e;
+  } else if (tc_gemm) {
     // dO = dy W_o: exact bf16 products when dy is bf16; an fp32 dy is split in two segments
-    // dW_o = dy^T O: O (fp16) is split; so is an fp32 dy, with the segments [hi, hi, lo] x [hi, lo, hi]
+    // dW_o = dy^T O: O (fp16) is split, dy repeats over both segments; an fp32 dy is split too, with
+    // the segments [hi, lo, hi] (dy repeating after two) x [hi, hi, lo] (three products)
     const bool dy_bf16 = ot == DType::BF16;
     const long long TpL = Tp;
+    if ((e = transpose_bf16({p.Wo, it}, Lq, E, Lq, E, wo_t, E, kOneHi, nullptr, 0, kOneHi, stream)) != cudaSuccess)
+      return e;
     if (dy_bf16) {
-      if ((e = transpose_bf16({g.dy, ot}, E, (int)T, E, Tp, dy_t, 2 * TpL, segs2(kSegHi, kSegHi, TpL), nullptr, 0,
-                              kOneHi, stream)) != cudaSuccess ||
-          (e = transpose_bf16({p.Wo, it}, Lq, E, Lq, E, wo_t, E, kOneHi, nullptr, 0, kOneHi, stream)) != cudaSuccess ||
+      if ((e = transpose_bf16({g.dy, ot}, E, (int)T, E, Tp, dy_t, TpL, kOneHi, nullptr, 0, kOneHi, stream)) !=
+              cudaSuccess ||
           (e = transpose_bf16({p.o, lt}, Lq, (int)T, Lq, Tp, o_t, 2 * TpL, segs2(kSegHi, kSegLo, TpL), nullptr, 0,
                               kOneHi, stream)) != cudaSuccess)
         return e;
       if ((e = gemm_tc_bf16(g.dy, T, wo_t, Lq, E, dO, Lq, p.dev_err, stream)) != cudaSuccess ||
-          (e = gemm_tc_bf16(dy_t, E, o_t, Lq, 2 * Tp, g.dWo, Lq, p.dev_err, stream)) != cudaSuccess)
+          (e = gemm_tc_bf16(dy_t, E, o_t, Lq, 2 * Tp, g.dWo, Lq, p.dev_err, stream, wrap(Tp))) != cudaSuccess)
         return e;
     } else {
-      if ((e = transpose_bf16({g.dy, ot}, E, (int)T, E, Tp, dy_t, 3 * TpL, segs3(kSegHi, kSegHi, kSegLo, TpL), dy16,
-                              2LL * E, segs2(kSegHi, kSegLo, E), stream)) != cudaSuccess ||
-          (e = transpose_bf16({p.Wo, it}, Lq, E, Lq, E, wo_t, 2LL * E, segs2(kSegHi, kSegHi, E), nullptr, 0, kOneHi,
-                              stream)) != cudaSuccess ||
-          (e = transpose_bf16({p.o, lt}, Lq, (int)T, Lq, Tp, o_t, 3 * TpL, segs3(kSegHi, kSegLo, kSegHi, TpL), nullptr,
+      if ((e = transpose_bf16({g.dy, ot}, E, (int)T, E, Tp, dy_t, 2 * TpL, segs2(kSegHi, kSegLo, TpL), dy16, 2LL * E,
+                              segs2(kSegHi, kSegLo, E), stream)) != cudaSuccess ||
+          (e = transpose_bf16({p.o, lt}, Lq, (int)T, Lq, Tp, o_t, 3 * TpL, segs3(kSegHi, kSegHi, kSegLo, TpL), nullptr,
                               0, kOneHi, stream)) != cudaSuccess)
         return e;
-      if ((e = gemm_tc_bf16(dy16, T, wo_t, Lq, 2 * E, dO, Lq, p.dev_err, stream)) != cudaSuccess ||
-          (e = gemm_tc_bf16(dy_t, E, o_t, Lq, 3 * Tp, g.dWo, Lq, p.dev_err, stream)) != cudaSuccess)
+      if ((e = gemm_tc_bf16(dy16, T, wo_t, Lq, 2 * E, dO, Lq, p.dev_err, stream, Opnd(), wrap(E))) != cudaSuccess ||
+          (e = gemm_tc_bf16(dy_t, E, o_t, Lq, 3 * Tp, g.dWo, Lq, p.dev_err, stream, wrap(2 * Tp))) != cudaSuccess)
         return e;
     }
   } else {
@@ -958,8 +1027,24 @@ cudaError_t launch_backward(const BlockDims& dm, const BlockPtrs& p, const Backw
       const long long warps = T * dm.nq;
       do_prep_kernel<<<(unsigned)((warps + 7) / 8), 256, 0, stream>>>(
           dO, static_cast<const __half*>(p.o), reinterpret_cast<__half*>(ws + L.dO16), delta, T, dm.S, dm.nq,
-          L.stat_stride);
+          L.stat_stride, direct ? o_t : nullptr, TpLL);
       if ((e = cudaGetLastError()) != cudaSuccess) return e;
+    }
+    if (direct) {
+      // dW_o = dy^T [O_hi; O_lo]: dy read [T][E] as the MN-major A, repeating after Tp rows (T of them
+      // held); O's two planes [2][Tp][Lq] as the MN-major B, their padding rows cleared
+      for (int pl = 0; pl < 2 && Tp > T; ++pl)
+        if ((e = cudaMemsetAsync(o_t + ((size_t)pl * Tp + T) * Lq, 0, sizeof(__nv_bfloat16) * (Tp - T) * Lq,
+                                 stream)) != cudaSuccess)
+          return e;
+      Opnd dya, ob;
+      dya.kwrap = Tp;
+      dya.kext = (int)T;
+      dya.mn = 1;
+      dya.ld = E;
+      ob.mn = 1;
+      ob.ld = Lq;
+      if ((e = gemm_tc_bf16(g.dy, E, o_t, Lq, 2 * Tp, g.dWo, Lq, p.dev_err, stream, dya, ob)) != cudaSuccess) return e;
     }
     // 3. attention backward on the tensor cores (dk, dv are sums over the CTAs of a key tile)
     if ((e = cudaMemsetAsync(dk, 0, sizeof(float) * T * Lkv, stream)) != cudaSuccess ||
@@ -1012,12 +1097,19 @@ cudaError_t launch_backward(const BlockDims& dm, const BlockPtrs& p, const Backw
       if ((e = cudaGetLastError()) != cudaSuccess) return e;
     }
   }
+  // the latents' gradient: fp32, or (direct) its bf16 hi / lo forms with the planes' padding rows cleared
+  DlatOut dlat_out{direct ? nullptr : dlat, dlat16, dlat_t, Nlat, TpLL};
+  if (direct)
+    for (int pl = 0; pl < 2 && Tp > T; ++pl)
+      if ((e = cudaMemsetAsync(dlat_t + ((size_t)pl * Tp + T) * Nlat, 0, sizeof(__nv_bfloat16) * (Tp - T) * Nlat,
+                               stream)) != cudaSuccess)
+        return e;
   // 4. per-token: RoPE back, QK-mean transpose, value-shift transpose
   {
     Theta64 th{};
     for (int i = 0; i < d / 2; ++i) th.v[i] = pow((double)dm.rope_base, -2.0 * (double)i / (double)d);
     token_bwd_kernel<<<(unsigned)T, 256, sizeof(float) * W, stream>>>(
-        dq, dk, dv, dc, dpre, dlat, dm.S, dm.nq, dm.nkv, d, dm.qk_mean_mode, dm.value_shift, dm.vshift_from,
+        dq, dk, dv, dc, dpre, dlat_out, dm.S, dm.nq, dm.nkv, d, dm.qk_mean_mode, dm.value_shift, dm.vshift_from,
         dm.use_rope, th, dm.K == 0);
     if ((e = cudaGetLastError()) != cudaSuccess) return e;
   }
@@ -1077,11 +1169,11 @@ cudaError_t launch_backward(const BlockDims& dm, const BlockPtrs& p, const Backw
   // 6. seq conv: dlat (q and k channels) and the tap gradients
   if (it == DType::BF16)
     seq_bwd_kernel<__nv_bfloat16><<<(unsigned)T, 256, 0, stream>>>(
-        ds, dpre, static_cast<const __nv_bfloat16*>(p.cq_seq), static_cast<const __nv_bfloat16*>(p.ck_seq), dlat,
+        ds, dpre, static_cast<const __nv_bfloat16*>(p.cq_seq), static_cast<const __nv_bfloat16*>(p.ck_seq), dlat_out,
         dm.S, dm.nq, dm.nkv, d, dm.K);
   else
     seq_bwd_kernel<float><<<(unsigned)T, 256, 0, stream>>>(ds, dpre, static_cast<const float*>(p.cq_seq),
-                                                            static_cast<const float*>(p.ck_seq), dlat, dm.S, dm.nq,
+                                                            static_cast<const float*>(p.ck_seq), dlat_out, dm.S, dm.nq,
                                                             dm.nkv, d, dm.K);
   if ((e = cudaGetLastError()) != cudaSuccess) return e;
   if ((e = cudaMemsetAsync(g.dconvq_seq, 0, sizeof(float) * Lq * dm.K, stream)) != cudaSuccess ||
@@ -1103,23 +1195,50 @@ cudaError_t launch_backward(const BlockDims& dm, const BlockPtrs& p, const Backw
   const void* Ws[3] = {p.Wq, p.Wk, p.Wv};
   float* dWs[3] = {g.dWq, g.dWk, g.dWv};
   const int col0[3] = {0, Lq, Lq + Lkv}, rows[3] = {Lq, Lkv, Lkv};
+  if (direct) {
+    // dx = [dlat_hi | dlat_lo] [W; W]: W^T (small) repeats over both segments; dW_* = [dlat_hi; dlat_lo]^T x:
+    // the planes' columns of the weight as the MN-major A, x [T][E] as the MN-major B repeating after Tp
+    for (int i = 0; i < 3; ++i)
+      if ((e = transpose_bf16({Ws[i], it}, E, rows[i], E, rows[i], w_t + col0[i], Nlat, kOneHi, nullptr, 0, kOneHi,
+                              stream)) != cudaSuccess)
+        return e;
+    if ((e = gemm_tc_bf16(dlat16, T, w_t, E, 2 * Nlat, g.dx, E, p.dev_err, stream, Opnd(), wrap(Nlat))) != cudaSuccess)
+      return e;
+    // one GEMM over all Nlat latent channels (four times the output tiles of the W_k or W_v share
+    // alone) into fp32 scratch, then each weight's rows to its output
+    Opnd la, xb;
+    la.mn = 1;
+    la.ld = Nlat;
+    xb.kwrap = Tp;
+    xb.kext = (int)T;
+    xb.mn = 1;
+    xb.ld = E;
+    float* dW_all = reinterpret_cast<float*>(ws + L.dw_all);  // [Nlat, E]
+    if ((e = gemm_tc_bf16(dlat_t, Nlat, p.x, E, 2 * Tp, dW_all, E, p.dev_err, stream, la, xb)) != cudaSuccess) return e;
+    for (int i = 0; i < 3; ++i)
+      if ((e = cudaMemcpyAsync(dWs[i], dW_all + (size_t)col0[i] * E, sizeof(float) * rows[i] * E,
+                               cudaMemcpyDeviceToDevice, stream)) != cudaSuccess)
+        return e;
+    return cudaSuccess;
+  }
   if (tc_gemm) {
     // dlat (fp32) split in two segments, row-major for dx and transposed for dW; x and the weights
-    // are exact in bf16 and repeat over both segments
+    // are exact in bf16, stored once and repeated over both segments
     const long long TpL = Tp;
     if ((e = transpose_bf16({dlat, DType::F32}, Nlat, (int)T, Nlat, Tp, dlat_t, 2 * TpL, segs2(kSegHi, kSegLo, TpL),
                             dlat16, 2LL * Nlat, segs2(kSegHi, kSegLo, Nlat), stream)) != cudaSuccess ||
-        (e = transpose_bf16({p.x, it}, E, (int)T, E, Tp, x_t, 2 * TpL, segs2(kSegHi, kSegHi, TpL), nullptr, 0, kOneHi,
-                            stream)) != cudaSuccess)
+        (e = transpose_bf16({p.x, it}, E, (int)T, E, Tp, x_t, TpL, kOneHi, nullptr, 0, kOneHi, stream)) != cudaSuccess)
       return e;
     for (int i = 0; i < 3; ++i)
-      if ((e = transpose_bf16({Ws[i], it}, E, rows[i], E, rows[i], w_t + col0[i], 2LL * Nlat,
-                              segs2(kSegHi, kSegHi, Nlat), nullptr, 0, kOneHi, stream)) != cudaSuccess)
+      if ((e = transpose_bf16({Ws[i], it}, E, rows[i], E, rows[i], w_t + col0[i], Nlat, kOneHi, nullptr, 0, kOneHi,
+                              stream)) != cudaSuccess)
         return e;
-    if ((e = gemm_tc_bf16(dlat16, T, w_t, E, 2 * Nlat, g.dx, E, p.dev_err, stream)) != cudaSuccess) return e;
+    if ((e = gemm_tc_bf16(dlat16, T, w_t, E, 2 * Nlat, g.dx, E, p.dev_err, stream, Opnd(), wrap(Nlat))) !=
+        cudaSuccess)
+      return e;
     for (int i = 0; i < 3; ++i)
-      if ((e = gemm_tc_bf16(dlat_t + (size_t)col0[i] * 2 * Tp, rows[i], x_t, E, 2 * Tp, dWs[i], E, p.dev_err,
-                            stream)) != cudaSuccess)
+      if ((e = gemm_tc_bf16(dlat_t + (size_t)col0[i] * 2 * Tp, rows[i], x_t, E, 2 * Tp, dWs[i], E, p.dev_err, stream,
+                            Opnd(), wrap(Tp))) != cudaSuccess)
         return e;
     return cudaSuccess;
   }

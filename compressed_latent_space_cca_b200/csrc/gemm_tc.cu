@@ -35,6 +35,7 @@ namespace {
 
 constexpr int BN = 256, BK = 64;
 constexpr int A_HALF_BYTES = 128 * BK * 2;  // 128 rows of A, 16 KB
+constexpr int MN_CHUNK_BYTES = 64 * BK * 2;  // an MN-major operand's [64 K][64 M or N] chunk, 8 KB
 constexpr int TMEM_COLS = 512;
 
 // Two tile shapes. MH = 1: 128 x 256 tiles, 4 stages of 48 KB, two 256-column accumulators so the
@@ -88,6 +89,8 @@ struct GemmParams {
   int tiles;      // output tiles
   int ksplit;     // K slices per tile (fp32 output added with reductions when > 1)
   int kb_slice;   // 64-deep K blocks per slice
+  int a_kwrap, b_kwrap;  // the operand's own K extent when it repeats along K (0: K)
+  int a_mn, b_mn;        // operand stored [K][M] ([K][N]): loaded as 64 x 64 boxes, read MN-major
   int tma_store;  // 16-bit output written through shared memory and maps.c
   // side job (bf16 -> fp16 copies), done by the epilogue warps before their first tile
   const __nv_bfloat16* side_src[2];
@@ -249,10 +252,21 @@ __global__ void __launch_bounds__(Shape<MH, PAIR>::NUM_THREADS, 1)
             mbar_arrive_expect_tx(fb, STAGE_BYTES);
           }
           uint8_t* sa = smem + stage * STAGE_BYTES;
+          const int ka = p.a_kwrap ? (kb * BK) % p.a_kwrap : kb * BK;
+          const int kbx = p.b_kwrap ? (kb * BK) % p.b_kwrap : kb * BK;
 #pragma unroll
           for (int h = 0; h < MH; ++h) {
-            if constexpr (PAIR) tma_load_2d_pair(smem_u32(sa + h * A_HALF_BYTES), &maps.a, fb, kb * BK, m0 + h * T::HS);
-            else tma_load_2d(smem_u32(sa + h * A_HALF_BYTES), &maps.a, fb, kb * BK, m0 + h * T::HS);
+            if (p.a_mn) {  // two 64-row chunks of M, each [64 K][64 M]
+#pragma unroll
+              for (int c = 0; c < 2; ++c) {
+                const uint32_t dst = smem_u32(sa + h * A_HALF_BYTES + c * MN_CHUNK_BYTES);
+                if constexpr (PAIR) tma_load_2d_pair(dst, &maps.a, fb, m0 + h * T::HS + c * 64, ka);
+                else tma_load_2d(dst, &maps.a, fb, m0 + h * T::HS + c * 64, ka);
+              }
+            } else {
+              if constexpr (PAIR) tma_load_2d_pair(smem_u32(sa + h * A_HALF_BYTES), &maps.a, fb, ka, m0 + h * T::HS);
+              else tma_load_2d(smem_u32(sa + h * A_HALF_BYTES), &maps.a, fb, ka, m0 + h * T::HS);
+            }
           }
 #pragma unroll
           for (int h = 0; h < T::B_ROWS / 128; ++h) {
@@ -263,8 +277,17 @@ __global__ void __launch_bounds__(Shape<MH, PAIR>::NUM_THREADS, 1)
               while (mi + 1 < p.nb && row >= p.row_start[mi + 1]) ++mi;
               r = row - p.row_start[mi];
             }
-            if constexpr (PAIR) tma_load_2d_pair(smem_u32(sa + A_BYTES + h * (128 * BK * 2)), &maps.b[mi], fb, kb * BK, r);
-            else tma_load_2d(smem_u32(sa + A_BYTES + h * (128 * BK * 2)), &maps.b[mi], fb, kb * BK, r);
+            if (p.b_mn) {  // one B matrix stored [K][N]: two 64-column chunks of N, each [64 K][64 N]
+#pragma unroll
+              for (int c = 0; c < 2; ++c) {
+                const uint32_t dst = smem_u32(sa + A_BYTES + h * (128 * BK * 2) + c * MN_CHUNK_BYTES);
+                if constexpr (PAIR) tma_load_2d_pair(dst, &maps.b[0], fb, row + c * 64, kbx);
+                else tma_load_2d(dst, &maps.b[0], fb, row + c * 64, kbx);
+              }
+            } else {
+              if constexpr (PAIR) tma_load_2d_pair(smem_u32(sa + A_BYTES + h * (128 * BK * 2)), &maps.b[mi], fb, kbx, r);
+              else tma_load_2d(smem_u32(sa + A_BYTES + h * (128 * BK * 2)), &maps.b[mi], fb, kbx, r);
+            }
           }
           if (++stage == STAGES) {
             stage = 0;
@@ -279,10 +302,14 @@ __global__ void __launch_bounds__(Shape<MH, PAIR>::NUM_THREADS, 1)
       // ------------------------------------------------------ MMA issuer --
       // Every lane runs this loop and its bounded waits; elect_one_sync picks the lane that issues
       // each tcgen05 instruction (issuing from a lane-divergent branch costs more per MMA).
-      const uint32_t idesc = idesc_f32acc(PAIR ? 256 : 128, BN, 0, 0, p.in_fmt);
+      const uint32_t idesc = idesc_f32acc(PAIR ? 256 : 128, BN, p.a_mn, p.b_mn, p.in_fmt);
       // descriptors built once; a stage step adds STAGE_BYTES / 16 to the start address, a K = 16 step 2
+      // (K-major: 32 bytes along the row) or 128 (MN-major: 16 rows of 128 bytes); MN-major operands
+      // carry LBO = the 64-wide chunk's bytes (it lives in the low word), SBO = 8 rows either way
       const uint32_t d_hi = desc_hi(smem_desc_sw128(smem_u32(smem), 16, 1024));
-      const uint32_t a_lo0 = desc_lo(smem_desc_sw128(smem_u32(smem), 16, 1024));
+      const uint32_t a_lo0 = desc_lo(smem_desc_sw128(smem_u32(smem), p.a_mn ? MN_CHUNK_BYTES : 16, 1024));
+      const uint32_t b_lo0 = desc_lo(smem_desc_sw128(smem_u32(smem + A_BYTES), p.b_mn ? MN_CHUNK_BYTES : 16, 1024));
+      const uint32_t a_kstep = p.a_mn ? 128 : 2, b_kstep = p.b_mn ? 128 : 2;
       int stage = 0;
       uint32_t phase = 0;
       int i = 0;
@@ -298,17 +325,17 @@ __global__ void __launch_bounds__(Shape<MH, PAIR>::NUM_THREADS, 1)
           if (!mbar_wait_bounded(smem_u32(&full[stage]), phase, p.err, abort_flag, wait_site(kSiteGemm, 2, 3))) goto mma_done;
           tc_fence_after();
           const uint32_t a_lo = a_lo0 + stage * (STAGE_BYTES >> 4);
-          const uint32_t b_lo = a_lo + (A_BYTES >> 4);
+          const uint32_t b_lo = b_lo0 + stage * (STAGE_BYTES >> 4);
 #pragma unroll
           for (int k = 0; k < BK / 16; ++k)
 #pragma unroll
             for (int h = 0; h < MH; ++h) {  // rows h*128.. of the tile -> accumulator columns h*256..
               if constexpr (PAIR) {
-                if (elect_one_sync()) umma_ss_pair_lohi(d_tmem + h * BN, a_lo + h * (A_HALF_BYTES >> 4) + 2 * k, d_hi, b_lo + 2 * k,
-                                                        d_hi, idesc, (kb != kb0 || k != 0));
+                if (elect_one_sync()) umma_ss_pair_lohi(d_tmem + h * BN, a_lo + h * (A_HALF_BYTES >> 4) + a_kstep * k, d_hi,
+                                                        b_lo + b_kstep * k, d_hi, idesc, (kb != kb0 || k != 0));
               } else {
-                if (elect_one_sync()) umma_ss_lohi(d_tmem + h * BN, a_lo + h * (A_HALF_BYTES >> 4) + 2 * k, d_hi, b_lo + 2 * k, d_hi, idesc,
-                             (kb != kb0 || k != 0));
+                if (elect_one_sync()) umma_ss_lohi(d_tmem + h * BN, a_lo + h * (A_HALF_BYTES >> 4) + a_kstep * k, d_hi,
+                                                   b_lo + b_kstep * k, d_hi, idesc, (kb != kb0 || k != 0));
               }
             }
           if constexpr (PAIR) {
@@ -540,11 +567,32 @@ cudaError_t launch_gemm_tc(const GemmTcArgs& a, cudaStream_t stream) {
       a.in == DType::F16 ? CU_TENSOR_MAP_DATA_TYPE_FLOAT16 : CU_TENSOR_MAP_DATA_TYPE_BFLOAT16;
   GemmMaps maps;
   GemmParams p{};
-  if (!encode_2d(&maps.a, a.A, dt, (uint64_t)a.K, (uint64_t)a.M, BK, 128)) return cudaErrorInvalidValue;
+  // an operand that repeats along K (its own extent whole 64-deep blocks, at most K)
+  for (const int w : {a.a_kwrap, a.b_kwrap})
+    if (w < 0 || (w > 0 && (w % BK != 0 || w > a.K))) return cudaErrorInvalidValue;
+  p.a_kwrap = a.a_kwrap;
+  p.b_kwrap = a.b_kwrap;
+  p.a_mn = a.a_mn ? 1 : 0;
+  p.b_mn = a.b_mn ? 1 : 0;
+  if (p.b_mn && a.nb != 1) return cudaErrorInvalidValue;
+  if ((a.lda != 0 && (a.lda * 2) % 16 != 0) || (a.ldb != 0 && (a.ldb * 2) % 16 != 0)) return cudaErrorInvalidValue;
+  // the maps' K extents: what the operand holds (kext), else its wrap period, else K; columns of a
+  // period past the operand's extent read zeros
+  const int ka = a.a_kext ? a.a_kext : (a.a_kwrap ? a.a_kwrap : a.K);
+  const int kb_ext = a.b_kext ? a.b_kext : (a.b_kwrap ? a.b_kwrap : a.K);
+  if (a.a_kext < 0 || a.b_kext < 0 || (a.a_kext > 0 && a.a_kext > (a.a_kwrap ? a.a_kwrap : a.K)) ||
+      (a.b_kext > 0 && a.b_kext > (a.b_kwrap ? a.b_kwrap : a.K)))
+    return cudaErrorInvalidValue;
+  // K-major: [M][K] rows of K; MN-major: [K][M] rows of M, 64 x 64 boxes (row strides lda / ldb)
+  if (p.a_mn ? !encode_2d(&maps.a, a.A, dt, (uint64_t)a.M, (uint64_t)ka, 64, BK, (uint64_t)a.lda * 2)
+             : !encode_2d(&maps.a, a.A, dt, (uint64_t)ka, (uint64_t)a.M, BK, 128, (uint64_t)a.lda * 2))
+    return cudaErrorInvalidValue;
   int start = 0;
   for (int i = 0; i < 3; ++i) {
     const int src = i < a.nb ? i : 0;
-    if (!encode_2d(&maps.b[i], a.B[src], dt, (uint64_t)a.K, (uint64_t)a.nrows[src], BK, 128))
+    if (p.b_mn ? !encode_2d(&maps.b[i], a.B[src], dt, (uint64_t)a.nrows[src], (uint64_t)kb_ext, 64, BK,
+                            (uint64_t)a.ldb * 2)
+               : !encode_2d(&maps.b[i], a.B[src], dt, (uint64_t)kb_ext, (uint64_t)a.nrows[src], BK, 128))
       return cudaErrorInvalidValue;
     p.row_start[i] = i < a.nb ? start : N;
     p.nrows[i] = a.nrows[src];

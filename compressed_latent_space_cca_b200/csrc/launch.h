@@ -110,6 +110,16 @@ struct GemmTcArgs {
   // optional split of K into ksplit slices (fp32 C only): each slice's product is added to C, which
   // the caller clears first
   int ksplit;
+  // optional: A (B) holds only a_kwrap (b_kwrap) columns of K and repeats along it, column k of the
+  // product reading its column k % a_kwrap (a multiple of 64, at most K; 0: A holds all K)
+  int a_kwrap, b_kwrap;
+  // optional: A stored [K][M] (row stride lda elements, 0: M) instead of [M][K]; B stored [K][N]
+  // (row stride ldb, 0: N; one B matrix) instead of [N][K]. lda also sets a K-major A's row stride.
+  int a_mn, b_mn;
+  long long lda, ldb;
+  // optional: the K columns A (B) actually holds when fewer than its wrap period (or K); the rest of
+  // each period reads as zeros
+  int a_kext, b_kext;
 };
 cudaError_t launch_gemm_tc(const GemmTcArgs& a, cudaStream_t stream);
 // K slices that give a GEMM with fewer 256 x 256 output tiles than the device has CTA pairs about
@@ -169,6 +179,7 @@ struct BackwardLayout {
   size_t y, k_cache, v_cache, dO, dO16, lse, delta, dq, dk, dv, dc, dpre, ds, s, dlat;
   // bf16 operands of the tensor-core GEMMs (token dimension padded to Tp in the transposed copies)
   size_t dy16, dy_t, x_t, o_t, dlat16, dlat_t, wo_t, w_t;
+  size_t dw_all;  // fp32 [Nlat, E] scratch for the down-projection's weight gradients
   size_t total;
   int stat_stride;  // lse / delta rows of the tensor-core path: [B][nq][stat_stride]
   int Tp;           // tokens rounded up to a multiple of 64
