@@ -11,10 +11,12 @@
 // c = scale log2(e).
 //
 // Two kernels, so that no dQ sums cross CTAs:
-//  dq kernel (query-stationary): a CTA per (sequence, query head, 128-query tile) walks the 64-key
-//   blocks at or before the diagonal. S = Q K_j^T and dP = dO V_j^T (both operands K-major) go to
-//   TMEM; four softmax warps turn each pair into dS (fp16), written over S in TMEM; dQ += dS K_j
-//   (A from TMEM, K_j read MN-major) accumulates in TMEM; the epilogue scales and stores dQ.
+//  dq kernel (query-stationary): a CTA per (sequence, query head, 128-query tile) walks the 128-key
+//   blocks at or before the diagonal. S = Q K_j^T (two TMEM slots) and dP = dO V_j^T (one slot, freed
+//   as soon as the softmax warps have read it) go to TMEM; the softmax warps turn each pair into dS
+//   (fp16), written over S; dQ += dS K_j (A from TMEM, K_j read MN-major) accumulates in TMEM; the
+//   epilogue scales and stores dQ. 128-key blocks keep every MMA at N = 128 or K = 128: the MMAs
+//   are issued by one lane at a rate that N = 64 products would not keep up with.
 //  dkv kernel (key-stationary): a CTA per (sequence, KV group, 128-key tile, chunk of up to
 //   kUnitsPerChunk (64-query block, head) units) holds K and V and walks its units. S^T = K Q_i^T
 //   and dP^T = V dO_i^T go to TMEM; the softmax warps write P^T and dS^T (fp16) over them in TMEM,
@@ -34,26 +36,26 @@ namespace {
 
 constexpr int D = 128;
 // softmax / epilogue warps of each kernel and the columns of a 64-column block each one takes
-// (measured at S = 16384: the dq kernel is fastest with 8, the dkv kernel with 16)
-constexpr int DQ_SM_WARPS = 8, KV_SM_WARPS = 16;
+// (the dq kernel's 128-key blocks, the dkv kernel's 64-query units)
+constexpr int DQ_SM_WARPS = 16, KV_SM_WARPS = 16;
 constexpr int DQ_THREADS = 64 + 32 * DQ_SM_WARPS, KV_THREADS = 64 + 32 * KV_SM_WARPS;
-constexpr int DQ_COLS = 64 / (DQ_SM_WARPS / 4), KV_COLS = 64 / (KV_SM_WARPS / 4);
+constexpr int DQ_COLS = 128 / (DQ_SM_WARPS / 4), KV_COLS = 64 / (KV_SM_WARPS / 4);
 constexpr int TMEM_COLS = 512;
 constexpr int SW = 128;  // bytes of one swizzled row (64 fp16)
 
 // ---- dq kernel geometry ----
 constexpr int DQ_QT = 128;                        // queries per tile
-constexpr int DQ_KB = 64;                         // keys per block
-constexpr int DQ_KV_STAGES = 3;
+constexpr int DQ_KB = 128;                        // keys per block
+constexpr int DQ_K_STAGES = 3, DQ_V_STAGES = 2;  // V is released when dP has read it, K after dQ
 constexpr int DQ_TILE_HALF = DQ_QT * SW;          // 16 KB: 128 rows x 64 columns
-constexpr int DQ_KV_HALF = DQ_KB * SW;            // 8 KB: 64 rows x 64 columns
+constexpr int DQ_KV_HALF = DQ_KB * SW;            // 16 KB: 128 rows x 64 columns
 constexpr int DQ_OFF_Q = 0;
 constexpr int DQ_OFF_DO = DQ_OFF_Q + 2 * DQ_TILE_HALF;
 constexpr int DQ_OFF_K = DQ_OFF_DO + 2 * DQ_TILE_HALF;
-constexpr int DQ_OFF_V = DQ_OFF_K + DQ_KV_STAGES * 2 * DQ_KV_HALF;
-constexpr int DQ_OFF_BAR = DQ_OFF_V + DQ_KV_STAGES * 2 * DQ_KV_HALF;
+constexpr int DQ_OFF_V = DQ_OFF_K + DQ_K_STAGES * 2 * DQ_KV_HALF;
+constexpr int DQ_OFF_BAR = DQ_OFF_V + DQ_V_STAGES * 2 * DQ_KV_HALF;
 constexpr size_t DQ_SMEM = DQ_OFF_BAR + 256 + 1024;
-constexpr uint32_t DQ_COL_S = 0, DQ_COL_DP = 128, DQ_COL_DQ = 256;  // S[s], dP[s] at +64 s
+constexpr uint32_t DQ_COL_S = 0, DQ_COL_DP = 256, DQ_COL_DQ = 384;  // S[s] at +128 s, one dP
 
 // ---- dkv kernel geometry ----
 constexpr int KV_KT = 128;                        // keys per tile
@@ -142,11 +144,14 @@ __global__ void __launch_bounds__(DQ_THREADS, 1) attn_bwd_dq_kernel(const __grid
   uint8_t* smem = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
   uint64_t* bars = reinterpret_cast<uint64_t*>(smem + DQ_OFF_BAR);
   uint64_t* q_full = bars;                        // Q and dO of the tile
-  uint64_t* kv_full = bars + 1;                   // [3]
-  uint64_t* kv_empty = kv_full + DQ_KV_STAGES;    // [3]
-  uint64_t* st_full = kv_empty + DQ_KV_STAGES;    // [2] S and dP of a block in TMEM
+  uint64_t* k_full = bars + 1;                    // [DQ_K_STAGES]
+  uint64_t* k_empty = k_full + DQ_K_STAGES;       // [DQ_K_STAGES]
+  uint64_t* v_full = k_empty + DQ_K_STAGES;       // [DQ_V_STAGES]
+  uint64_t* v_empty = v_full + DQ_V_STAGES;       // [DQ_V_STAGES]
+  uint64_t* st_full = v_empty + DQ_V_STAGES;      // [2] S and dP of a block in TMEM
   uint64_t* ds_full = st_full + 2;                // [2] dS written over S (every softmax warp)
-  uint64_t* dq_full = ds_full + 2;                // dQ complete
+  uint64_t* dp_free = ds_full + 2;                // dP read by every softmax warp
+  uint64_t* dq_full = dp_free + 1;                // dQ complete
   uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(dq_full + 1);
   volatile int* abort_flag = reinterpret_cast<volatile int*>(tmem_slot + 1);
 
@@ -161,14 +166,19 @@ __global__ void __launch_bounds__(DQ_THREADS, 1) attn_bwd_dq_kernel(const __grid
 
   if (threadIdx.x == 0) {
     mbar_init(smem_u32(q_full), 1);
-    for (int s = 0; s < DQ_KV_STAGES; ++s) {
-      mbar_init(smem_u32(&kv_full[s]), 1);
-      mbar_init(smem_u32(&kv_empty[s]), 1);
+    for (int s = 0; s < DQ_K_STAGES; ++s) {
+      mbar_init(smem_u32(&k_full[s]), 1);
+      mbar_init(smem_u32(&k_empty[s]), 1);
+    }
+    for (int s = 0; s < DQ_V_STAGES; ++s) {
+      mbar_init(smem_u32(&v_full[s]), 1);
+      mbar_init(smem_u32(&v_empty[s]), 1);
     }
     for (int s = 0; s < 2; ++s) {
       mbar_init(smem_u32(&st_full[s]), 1);
       mbar_init(smem_u32(&ds_full[s]), DQ_SM_WARPS);
     }
+    mbar_init(smem_u32(dp_free), DQ_SM_WARPS);
     mbar_init(smem_u32(dq_full), 1);
     *abort_flag = 0;
     fence_mbar_init();
@@ -201,20 +211,25 @@ __global__ void __launch_bounds__(DQ_THREADS, 1) attn_bwd_dq_kernel(const __grid
                     qt * DQ_QT, b);
     }
     for (int j = 0; j < nkb; ++j) {
-      const int st = j % DQ_KV_STAGES;
-      if (!mbar_wait_bounded(smem_u32(&kv_empty[st]), ((j / DQ_KV_STAGES) & 1) ^ 1, p.err, abort_flag,
+      const int sk = j % DQ_K_STAGES, sv = j % DQ_V_STAGES;
+      if (!mbar_wait_bounded(smem_u32(&k_empty[sk]), ((j / DQ_K_STAGES) & 1) ^ 1, p.err, abort_flag,
                              wait_site(kSiteAttnBwd, 1, 1)))
         break;
-      if (elect_one_sync()) mbar_arrive_expect_tx(smem_u32(&kv_full[st]), 4 * DQ_KV_HALF);
+      if (elect_one_sync()) mbar_arrive_expect_tx(smem_u32(&k_full[sk]), 2 * DQ_KV_HALF);
 #pragma unroll
-      for (int hf = 0; hf < 2; ++hf) {
+      for (int hf = 0; hf < 2; ++hf)
         if (elect_one_sync())
-          tma_load_3d(smem_u32(smem + DQ_OFF_K + (st * 2 + hf) * DQ_KV_HALF), &maps.k, smem_u32(&kv_full[st]),
+          tma_load_3d(smem_u32(smem + DQ_OFF_K + (sk * 2 + hf) * DQ_KV_HALF), &maps.k, smem_u32(&k_full[sk]),
                       g * D + hf * 64, j * DQ_KB, b);
+      if (!mbar_wait_bounded(smem_u32(&v_empty[sv]), ((j / DQ_V_STAGES) & 1) ^ 1, p.err, abort_flag,
+                             wait_site(kSiteAttnBwd, 1, 7)))
+        break;
+      if (elect_one_sync()) mbar_arrive_expect_tx(smem_u32(&v_full[sv]), 2 * DQ_KV_HALF);
+#pragma unroll
+      for (int hf = 0; hf < 2; ++hf)
         if (elect_one_sync())
-          tma_load_3d(smem_u32(smem + DQ_OFF_V + (st * 2 + hf) * DQ_KV_HALF), &maps.v, smem_u32(&kv_full[st]),
+          tma_load_3d(smem_u32(smem + DQ_OFF_V + (sv * 2 + hf) * DQ_KV_HALF), &maps.v, smem_u32(&v_full[sv]),
                       g * D + hf * 64, j * DQ_KB, b);
-      }
     }
   } else if (warp == 1) {
     // ---------------------------------------------------------------- MMA --
@@ -232,46 +247,55 @@ __global__ void __launch_bounds__(DQ_THREADS, 1) attn_bwd_dq_kernel(const __grid
     tc_fence_after();
     for (int j = 0; j <= nkb; ++j) {
       if (j < nkb) {
-        const int st = j % DQ_KV_STAGES, s = j & 1;
-        if (!mbar_wait_bounded(smem_u32(&kv_full[st]), (j / DQ_KV_STAGES) & 1, p.err, abort_flag,
+        const int sk = j % DQ_K_STAGES, sv = j % DQ_V_STAGES, s = j & 1;
+        if (!mbar_wait_bounded(smem_u32(&k_full[sk]), (j / DQ_K_STAGES) & 1, p.err, abort_flag,
                                wait_site(kSiteAttnBwd, 2, 3)))
           goto done;
         tc_fence_after();
-        // S[s] = Q K_j^T and dP[s] = dO V_j^T; slot s was last read by the softmax of block j - 2,
-        // whose ds_full this loop waited for at j - 1, and by the dQ MMA of block j - 2 issued before
+        // S[s] = Q K_j^T: slot s was last read by the softmax of block j - 2, whose ds_full this loop
+        // waited for at j - 1, and by the dQ MMA of block j - 2 issued before
 #pragma unroll
         for (int kk = 0; kk < D / 16; ++kk)
           if (elect_one_sync())
-            umma_ss_lohi(tmem + DQ_COL_S + 64 * s, q_lo + kmaj_step(kk, DQ_TILE_HALF), sw_hi,
-                         k_lo + st * kStageStep + kmaj_step(kk, DQ_KV_HALF), sw_hi, idesc_s, kk > 0);
+            umma_ss_lohi(tmem + DQ_COL_S + 128 * s, q_lo + kmaj_step(kk, DQ_TILE_HALF), sw_hi,
+                         k_lo + sk * kStageStep + kmaj_step(kk, DQ_KV_HALF), sw_hi, idesc_s, kk > 0);
+        // dP = dO V_j^T into the one dP slot, once the softmax warps have read block j - 1's
+        if (j >= 1 && !mbar_wait_bounded(smem_u32(dp_free), (j - 1) & 1, p.err, abort_flag,
+                                         wait_site(kSiteAttnBwd, 2, 5)))
+          goto done;
+        if (!mbar_wait_bounded(smem_u32(&v_full[sv]), (j / DQ_V_STAGES) & 1, p.err, abort_flag,
+                               wait_site(kSiteAttnBwd, 2, 6)))
+          goto done;
+        tc_fence_after();
 #pragma unroll
         for (int kk = 0; kk < D / 16; ++kk)
           if (elect_one_sync())
-            umma_ss_lohi(tmem + DQ_COL_DP + 64 * s, do_lo + kmaj_step(kk, DQ_TILE_HALF), sw_hi,
-                         v_lo + st * kStageStep + kmaj_step(kk, DQ_KV_HALF), sw_hi, idesc_s, kk > 0);
+            umma_ss_lohi(tmem + DQ_COL_DP, do_lo + kmaj_step(kk, DQ_TILE_HALF), sw_hi,
+                         v_lo + sv * kStageStep + kmaj_step(kk, DQ_KV_HALF), sw_hi, idesc_s, kk > 0);
         if (elect_one_sync()) umma_commit(smem_u32(&st_full[s]));
+        if (elect_one_sync()) umma_commit(smem_u32(&v_empty[sv]));  // V_j is read by dP alone
       }
       if (j >= 1) {
-        const int jp = j - 1, sp = jp & 1, stp = jp % DQ_KV_STAGES;
+        const int jp = j - 1, sp = jp & 1, skp = jp % DQ_K_STAGES;
         if (!mbar_wait_bounded(smem_u32(&ds_full[sp]), (jp >> 1) & 1, p.err, abort_flag,
                                wait_site(kSiteAttnBwd, 2, 4)))
           goto done;
         tc_fence_after();
-        // dQ += dS K_jp: A = dS (fp16 pairs over the first 32 columns of S[sp]), B = K_jp read as
+        // dQ += dS K_jp: A = dS (fp16 pairs over the first 64 columns of S[sp]), B = K_jp read as
         // [d x keys] MN-major (LBO = the 64-column half, SBO = 8 keys), 16 keys per MMA
 #pragma unroll
         for (int kk = 0; kk < DQ_KB / 16; ++kk)
           if (elect_one_sync())
-            umma_ts_lohi(tmem + DQ_COL_DQ, tmem + DQ_COL_S + 64 * sp + kk * 8,
-                         kmn_lo + stp * kStageStep + ((kk * 16 * SW) >> 4), mn_hi, idesc_dq, jp > 0 || kk > 0);
-        if (elect_one_sync()) umma_commit(smem_u32(&kv_empty[stp]));
+            umma_ts_lohi(tmem + DQ_COL_DQ, tmem + DQ_COL_S + 128 * sp + kk * 8,
+                         kmn_lo + skp * kStageStep + ((kk * 16 * SW) >> 4), mn_hi, idesc_dq, jp > 0 || kk > 0);
+        if (elect_one_sync()) umma_commit(smem_u32(&k_empty[skp]));
       }
     }
     if (elect_one_sync()) umma_commit(smem_u32(dq_full));
   } else {
     // ------------------------------------------------------------ softmax --
     const int quad = warp & 3;
-    const int part = (warp - 2) >> 2;  // this warp's DQ_COLS of the block's 64 keys
+    const int part = (warp - 2) >> 2;  // this warp's DQ_COLS of the block's 128 keys
     const int r = quad * 32 + lane;
     const int t = qt * DQ_QT + r;
     const bool row_ok = t < p.S;
@@ -288,25 +312,42 @@ __global__ void __launch_bounds__(DQ_THREADS, 1) attn_bwd_dq_kernel(const __grid
       tc_fence_after();
       static_assert(DQ_COLS == 32, "the dq softmax reads 32 columns a warp");
       uint32_t sv[DQ_COLS], dp[DQ_COLS];
-      tmem_ld_32x32b_x32(tmem + lane_off + DQ_COL_S + 64 * s + DQ_COLS * part, sv);
-      tmem_ld_32x32b_x32(tmem + lane_off + DQ_COL_DP + 64 * s + DQ_COLS * part, dp);
+      tmem_ld_32x32b_x32(tmem + lane_off + DQ_COL_S + 128 * s + DQ_COLS * part, sv);
+      tmem_ld_32x32b_x32(tmem + lane_off + DQ_COL_DP + DQ_COLS * part, dp);
       tmem_ld_wait();
+      tc_fence_before();  // dP may take the next block's product
+      __syncwarp();
+      if (lane == 0) mbar_arrive(smem_u32(dp_free));
       const int key0 = j * DQ_KB + DQ_COLS * part;
       uint32_t pk[DQ_COLS / 2];
+      float dmax = 0.f;  // largest |dS| of the block, checked against the fp16 range once
+      // every key of the warp's share visible to every row of the warp: the choice is warp-uniform, so
+      // the warp stays converged for the tcgen05.st that follows
+      if (__all_sync(0xffffffffu, row_ok && key0 + DQ_COLS - 1 <= t)) {
 #pragma unroll
-      for (int c = 0; c < DQ_COLS; c += 2) {
-        float ds[2];
-#pragma unroll
-        for (int e = 0; e < 2; ++e) {
-          const bool vis = row_ok && key0 + c + e <= t;
-          const float pr = vis ? fast_exp2(fmaf(u2f(sv[c + e]), c2, -lse2)) : 0.f;
-          ds[e] = vis ? pr * (u2f(dp[c + e]) - dl) : 0.f;
-          bad |= f16_overflow(ds[e]);
+        for (int c = 0; c < DQ_COLS; c += 2) {
+          const float d0 = fast_exp2(fmaf(u2f(sv[c]), c2, -lse2)) * (u2f(dp[c]) - dl);
+          const float d1 = fast_exp2(fmaf(u2f(sv[c + 1]), c2, -lse2)) * (u2f(dp[c + 1]) - dl);
+          dmax = fmaxf(dmax, fmaxf(fabsf(d0), fabsf(d1)));
+          pk[c >> 1] = pack_f16x2(d0, d1);
         }
-        pk[c >> 1] = pack_f16x2(ds[0], ds[1]);
+      } else {
+#pragma unroll
+        for (int c = 0; c < DQ_COLS; c += 2) {
+          float ds[2];
+#pragma unroll
+          for (int e = 0; e < 2; ++e) {
+            const bool vis = row_ok && key0 + c + e <= t;
+            const float pr = vis ? fast_exp2(fmaf(u2f(sv[c + e]), c2, -lse2)) : 0.f;
+            ds[e] = vis ? pr * (u2f(dp[c + e]) - dl) : 0.f;
+            dmax = fmaxf(dmax, fabsf(ds[e]));
+          }
+          pk[c >> 1] = pack_f16x2(ds[0], ds[1]);
+        }
       }
+      bad |= f16_overflow(dmax);
       // keys 2c, 2c + 1 of the block go to packed column c: this warp's DQ_COLS / 2 columns
-      tmem_st_32x32b_x16(tmem + lane_off + DQ_COL_S + 64 * s + (DQ_COLS / 2) * part, pk);
+      tmem_st_32x32b_x16(tmem + lane_off + DQ_COL_S + 128 * s + (DQ_COLS / 2) * part, pk);
       tmem_st_wait();
       tc_fence_before();
       __syncwarp();
@@ -317,7 +358,7 @@ __global__ void __launch_bounds__(DQ_THREADS, 1) attn_bwd_dq_kernel(const __grid
     tc_fence_after();
     float* out = p.dq + ((size_t)b * p.S + t) * p.Lq + h * D;
 #pragma unroll 1
-    for (int c4 = 2 * part; c4 < 2 * part + 2; ++c4) {  // 64 of the 128 columns per warp
+    for (int c4 = part; c4 < part + 1; ++c4) {  // 32 of the 128 columns per warp
       uint32_t v[32];
       tmem_ld_32x32b_x32(tmem + lane_off + DQ_COL_DQ + 32 * c4, v);
       tmem_ld_wait();
@@ -533,23 +574,49 @@ __global__ void __launch_bounds__(KV_THREADS, 1) attn_bwd_dkv_kernel(const __gri
       const float* lse_s = reinterpret_cast<const float*>(smem + KV_OFF_LSE + q * KV_QB * 4);
       const float* del_s = reinterpret_cast<const float*>(smem + KV_OFF_DELTA + q * KV_QB * 4);
       uint32_t pp[KV_COLS / 2], dd[KV_COLS / 2];  // this warp's queries 2c, 2c + 1 -> packed column c
+      // this warp's statistics, four at a time (every lane reads the same addresses)
+      float ls[KV_COLS], de[KV_COLS];
 #pragma unroll
-      for (int c2i = 0; c2i < KV_COLS / 2; ++c2i) {
-        float pv[2], dv[2];
-#pragma unroll
-        for (int f = 0; f < 2; ++f) {
-          const int cl = 2 * c2i + f;  // column within this warp's share
-          const int c = KV_COLS * part + cl;
-          const int t = q0 + c;
-          const bool vis = key <= t && t < p.S;
-          const float pr = vis ? fast_exp2(fmaf(u2f(sv[cl]), c2, -lse_s[c])) : 0.f;
-          pv[f] = pr;
-          dv[f] = vis ? pr * (u2f(dp[cl]) - del_s[c]) : 0.f;
-          bad |= f16_overflow(dv[f]);
-        }
-        pp[c2i] = pack_f16x2(pv[0], pv[1]);
-        dd[c2i] = pack_f16x2(dv[0], dv[1]);
+      for (int v4 = 0; v4 < KV_COLS / 4; ++v4) {
+        const float4 a = *reinterpret_cast<const float4*>(lse_s + KV_COLS * part + 4 * v4);
+        const float4 b = *reinterpret_cast<const float4*>(del_s + KV_COLS * part + 4 * v4);
+        ls[4 * v4] = a.x, ls[4 * v4 + 1] = a.y, ls[4 * v4 + 2] = a.z, ls[4 * v4 + 3] = a.w;
+        de[4 * v4] = b.x, de[4 * v4 + 1] = b.y, de[4 * v4 + 2] = b.z, de[4 * v4 + 3] = b.w;
       }
+      const int qa = q0 + KV_COLS * part;  // this warp's first query
+      float dmax = 0.f;  // largest |dS|, checked against the fp16 range once
+      // every query of the share sees every key row of the warp: the choice is warp-uniform, so the warp
+      // stays converged for the tcgen05.st that follows
+      if (__all_sync(0xffffffffu, key <= qa && qa + KV_COLS - 1 < p.S)) {
+#pragma unroll
+        for (int c2i = 0; c2i < KV_COLS / 2; ++c2i) {
+          const int c = 2 * c2i;
+          const float p0 = fast_exp2(fmaf(u2f(sv[c]), c2, -ls[c]));
+          const float p1 = fast_exp2(fmaf(u2f(sv[c + 1]), c2, -ls[c + 1]));
+          const float d0 = p0 * (u2f(dp[c]) - de[c]), d1 = p1 * (u2f(dp[c + 1]) - de[c + 1]);
+          dmax = fmaxf(dmax, fmaxf(fabsf(d0), fabsf(d1)));
+          pp[c2i] = pack_f16x2(p0, p1);
+          dd[c2i] = pack_f16x2(d0, d1);
+        }
+      } else {
+#pragma unroll
+        for (int c2i = 0; c2i < KV_COLS / 2; ++c2i) {
+          float pv[2], dv[2];
+#pragma unroll
+          for (int f = 0; f < 2; ++f) {
+            const int cl = 2 * c2i + f;  // column within this warp's share
+            const int t = qa + cl;
+            const bool vis = key <= t && t < p.S;
+            const float pr = vis ? fast_exp2(fmaf(u2f(sv[cl]), c2, -ls[cl])) : 0.f;
+            pv[f] = pr;
+            dv[f] = vis ? pr * (u2f(dp[cl]) - de[cl]) : 0.f;
+            dmax = fmaxf(dmax, fabsf(dv[f]));
+          }
+          pp[c2i] = pack_f16x2(pv[0], pv[1]);
+          dd[c2i] = pack_f16x2(dv[0], dv[1]);
+        }
+      }
+      bad |= f16_overflow(dmax);
       // P^T over S^T[s] and dS^T over dP^T[s] (both already read above)
       tmem_st_32x32b_x8(tmem + lane_off + KV_COL_ST + 64 * s + (KV_COLS / 2) * part, pp);
       tmem_st_32x32b_x8(tmem + lane_off + KV_COL_DPT + 64 * s + (KV_COLS / 2) * part, dd);
