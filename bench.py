@@ -491,6 +491,9 @@ def run_mha_baseline(cca, dev, shape, cca_ms_per_step, cca_backward=None, peaks=
     if cca_backward is not None and cca.backward_workspace_size(cfg) > 0:
         bwd = run_backward(cca, dev, mshape, inputs, peaks if peaks is not None else load_peaks()[0])
         bwd["cca_backward_speedup"] = bwd["ms_per_step"] / cca_backward["ms_per_step"]
+        if bwd.get("saved_forward") and cca_backward.get("saved_forward"):
+            bwd["saved_forward"]["cca_backward_speedup"] = (bwd["saved_forward"]["ms_per_step"] /
+                                                            cca_backward["saved_forward"]["ms_per_step"])
     del inputs
     torch.cuda.empty_cache()
     return {
@@ -544,11 +547,36 @@ def run_backward(cca, dev, shape, inputs, peaks, steps=5, warmup=3):
     fl = backward_flops(shape)
     peak = float(peaks.get("bf16_tflops", FALLBACK_PEAKS["bf16_tflops"]))
     tflops = fl["total"] / (ms / 1e3) / 1e12
+    # the backward of a training step whose forward (prefill_train) kept its activations: no recompute
+    saved = None
+    try:
+        cca.prefill_train(cfg, inputs, workspace=ws)
+    except cca.CcaError:
+        pass  # a block the saved forward does not take (fp32, CUDA-core attention)
+    else:
+        for _ in range(warmup):
+            flush.zero_()
+            cca.backward(cfg, inputs, dy, grads=grads, workspace=ws, saved=True)
+        torch.cuda.synchronize()
+        for i in range(steps):
+            flush.zero_()
+            evs[i][0].record(stream)
+            cca.backward(cfg, inputs, dy, grads=grads, workspace=ws, saved=True)
+            evs[i][1].record(stream)
+        torch.cuda.synchronize()
+        if cca.poll_device_status() != 0:
+            raise SystemExit("device status error in the saved-forward backward timing")
+        sms = float(np.mean([a.elapsed_time(b) for a, b in evs]))
+        sfl = fl["attention_backward"] + fl["projections_backward"]
+        saved = {"ms_per_step": sms, "includes": "all gradients from prefill_train's saved activations",
+                 "flops": sfl, "tflops": sfl / (sms / 1e3) / 1e12,
+                 "frac_of_bf16_peak": sfl / (sms / 1e3) / 1e12 / peak}
     del ws, grads, flush, dy
     torch.cuda.empty_cache()
     return {"ms_per_step": ms, "tokens_per_s": shape.tokens / (ms / 1e3), "steps": steps, "warmup": warmup,
             "includes": "forward recompute + all gradients", "flops": fl, "tflops": tflops,
-            "frac_of_bf16_peak": tflops / peak, "timing": "CUDA events, L2 flushed before each call"}
+            "frac_of_bf16_peak": tflops / peak, "timing": "CUDA events, L2 flushed before each call",
+            "saved_forward": saved}
 
 
 def decode_bytes(shape: workloads.BlockShape, t: int) -> float:

@@ -352,14 +352,49 @@ def backward_workspace_size(cfg: CcaConfig) -> int:
     return library().cca_backward_workspace_size(ctypes.byref(cfg))
 
 
+def prefill_train(cfg: CcaConfig, inputs: Dict[str, torch.Tensor], *,
+                  out: Optional[Dict[str, torch.Tensor]] = None, workspace: Optional[torch.Tensor] = None,
+                  stream: Optional[torch.cuda.Stream] = None) -> Dict[str, torch.Tensor]:
+    """cca_prefill_train: the forward of a training step. Returns {"y", "k_cache", "v_cache",
+    "workspace"}; pass the same inputs and that workspace to backward(..., saved=True)."""
+    x = inputs["x"]
+    device = x.device
+    if device.type != "cuda":
+        raise ValueError("inputs must be CUDA tensors")
+    sh = _shapes(cfg)
+    dt = _DT[cfg.dtype]
+    ptrs = _input_ptrs(cfg, inputs, INPUT_NAMES, dt, device)
+    if out is None:
+        out = alloc_outputs(cfg, device)
+    y = _check(out["y"], "y", sh["y"], _DT[cfg.out_dtype], device)
+    kc = _check(out["k_cache"], "k_cache", sh["k_cache"], dt, device)
+    vc = _check(out["v_cache"], "v_cache", sh["v_cache"], dt, device)
+    if workspace is None:
+        n = backward_workspace_size(cfg)
+        if n == 0:
+            raise CcaError(CCA_ERR_UNSUPPORTED, "cca_backward_workspace_size")
+        workspace = torch.empty(n, dtype=torch.uint8, device=device)
+    if stream is None:
+        stream = torch.cuda.current_stream(device)
+    st = library().cca_prefill_train(ctypes.byref(cfg), *ptrs, y, kc, vc, workspace.data_ptr(), workspace.numel(),
+                                     ctypes.c_void_p(stream.cuda_stream))
+    if st != CCA_OK:
+        raise CcaError(st, "cca_prefill_train")
+    res = dict(out)
+    res["workspace"] = workspace
+    return res
+
+
 def backward(cfg: CcaConfig, inputs: Dict[str, torch.Tensor], dy: torch.Tensor, *,
              grads: Optional[Dict[str, torch.Tensor]] = None, workspace: Optional[torch.Tensor] = None,
-             stream: Optional[torch.cuda.Stream] = None) -> Dict[str, torch.Tensor]:
+             saved: bool = False, stream: Optional[torch.cuda.Stream] = None) -> Dict[str, torch.Tensor]:
     """cca_backward: the gradients of x and of the eight weights for dL/dy = dy.
 
     inputs: the nine tensors of INPUT_NAMES (dtype cfg.dtype); dy [B, S, E] in cfg.out_dtype.
     Returns fp32 tensors named as the inputs, in their shapes (overwritten, not accumulated); a plain
-    block (conv_kernel 0) has no conv weights and returns no gradients for them.
+    block (conv_kernel 0) has no conv weights and returns no gradients for them. With saved=True the
+    workspace is the one prefill_train filled for the same inputs (cca_backward_saved: no forward
+    recomputation).
     """
     x = inputs["x"]
     device = x.device
@@ -373,16 +408,19 @@ def backward(cfg: CcaConfig, inputs: Dict[str, torch.Tensor], dy: torch.Tensor, 
         grads = {n: torch.empty(sh[n], dtype=torch.float32, device=device) for n in names}
     gp = [_check(grads[n], "d" + n, sh[n], torch.float32, device) if n in names else None for n in GRAD_NAMES]
     if workspace is None:
+        if saved:
+            raise ValueError("saved=True needs the workspace prefill_train filled")
         n = backward_workspace_size(cfg)
         if n == 0:
             raise CcaError(CCA_ERR_UNSUPPORTED, "cca_backward_workspace_size")
         workspace = torch.empty(n, dtype=torch.uint8, device=device)
     if stream is None:
         stream = torch.cuda.current_stream(device)
-    st = library().cca_backward(ctypes.byref(cfg), *ptrs, dyp, *gp, workspace.data_ptr(), workspace.numel(),
-                                ctypes.c_void_p(stream.cuda_stream))
+    fn = library().cca_backward_saved if saved else library().cca_backward
+    st = fn(ctypes.byref(cfg), *ptrs, dyp, *gp, workspace.data_ptr(), workspace.numel(),
+            ctypes.c_void_p(stream.cuda_stream))
     if st != CCA_OK:
-        raise CcaError(st, "cca_backward")
+        raise CcaError(st, "cca_backward_saved" if saved else "cca_backward")
     return grads
 
 

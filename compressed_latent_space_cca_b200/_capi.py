@@ -99,6 +99,10 @@ SIGNATURES = {
     "cca_backward_workspace_size": (c_size_t, [POINTER(CcaConfig)]),
     "cca_backward": (c_int, [POINTER(CcaConfig)] + [c_void_p] * 10 + [c_void_p] * 9
                      + [c_void_p, c_size_t, c_void_p]),
+    "cca_prefill_train": (c_int, [POINTER(CcaConfig)] + [c_void_p] * 9 + [c_void_p] * 3
+                          + [c_void_p, c_size_t, c_void_p]),
+    "cca_backward_saved": (c_int, [POINTER(CcaConfig)] + [c_void_p] * 10 + [c_void_p] * 9
+                           + [c_void_p, c_size_t, c_void_p]),
     "cca_poll_device_status": (c_int, [c_void_p]),
     "cca_selftest_wait_timeout": (c_int, [c_uint, c_void_p]),
     "cca_status_string": (c_char_p, [c_int]),

@@ -71,7 +71,8 @@ constexpr int KV_OFF_LSE = KV_OFF_DO + KV_QSLOTS * 2 * KV_Q_HALF;  // [slots][64
 constexpr int KV_OFF_DELTA = KV_OFF_LSE + KV_QSLOTS * KV_QB * 4;   // [slots][64] fp32
 constexpr int KV_OFF_BAR = KV_OFF_DELTA + KV_QSLOTS * KV_QB * 4;
 constexpr size_t KV_SMEM = KV_OFF_BAR + 256 + 1024;
-// St[s], dPt[s] at +64 s; P^T and dS^T (fp16 pairs) overlay the first 32 columns of St[s] and dPt[s]
+// St[s], dPt[s] at +64 s; P^T and dS^T (fp16 pairs) overlay them, each softmax warp's 16 queries in
+// the first 8 of its own 16 columns
 constexpr uint32_t KV_COL_ST = 0, KV_COL_DPT = 128, KV_COL_DV = 256, KV_COL_DK = 384;
 constexpr int kUnitsPerChunk = 48;
 static_assert(DQ_SMEM <= 232448 && KV_SMEM <= 232448, "shared memory of one CTA");
@@ -281,12 +282,14 @@ __global__ void __launch_bounds__(DQ_THREADS, 1) attn_bwd_dq_kernel(const __grid
                                wait_site(kSiteAttnBwd, 2, 4)))
           goto done;
         tc_fence_after();
-        // dQ += dS K_jp: A = dS (fp16 pairs over the first 64 columns of S[sp]), B = K_jp read as
-        // [d x keys] MN-major (LBO = the 64-column half, SBO = 8 keys), 16 keys per MMA
+        // dQ += dS K_jp: A = dS (fp16 pairs: keys 16 kk .. 16 kk + 15 in the 8 columns from
+        // DQ_COLS (kk / 2) + 8 (kk % 2) of S[sp], each softmax warp's packed share at the start of its
+        // own columns), B = K_jp read as [d x keys] MN-major (LBO = the 64-column half, SBO = 8 keys)
+        static_assert(DQ_COLS == 32, "two 16-key MMA steps per softmax warp's share");
 #pragma unroll
         for (int kk = 0; kk < DQ_KB / 16; ++kk)
           if (elect_one_sync())
-            umma_ts_lohi(tmem + DQ_COL_DQ, tmem + DQ_COL_S + 128 * sp + kk * 8,
+            umma_ts_lohi(tmem + DQ_COL_DQ, tmem + DQ_COL_S + 128 * sp + DQ_COLS * (kk >> 1) + 8 * (kk & 1),
                          kmn_lo + skp * kStageStep + ((kk * 16 * SW) >> 4), mn_hi, idesc_dq, jp > 0 || kk > 0);
         if (elect_one_sync()) umma_commit(smem_u32(&k_empty[skp]));
       }
@@ -346,8 +349,9 @@ __global__ void __launch_bounds__(DQ_THREADS, 1) attn_bwd_dq_kernel(const __grid
         }
       }
       bad |= f16_overflow(dmax);
-      // keys 2c, 2c + 1 of the block go to packed column c: this warp's DQ_COLS / 2 columns
-      tmem_st_32x32b_x16(tmem + lane_off + DQ_COL_S + 128 * s + (DQ_COLS / 2) * part, pk);
+      // the warp's keys 2c, 2c + 1 go to packed column c of its own share of S[s] (the first half of
+      // the columns this warp has just read): another warp's unread scores are never overwritten
+      tmem_st_32x32b_x16(tmem + lane_off + DQ_COL_S + 128 * s + DQ_COLS * part, pk);
       tmem_st_wait();
       tc_fence_before();
       __syncwarp();
@@ -530,17 +534,19 @@ __global__ void __launch_bounds__(KV_THREADS, 1) attn_bwd_dkv_kernel(const __gri
         if (!mbar_wait_bounded(smem_u32(&p_full[sp]), (np >> 1) & 1, p.err, abort_flag, wait_site(kSiteAttnBwd, 5, 4)))
           goto done;
         tc_fence_after();
-        // dV += P^T dO_i and dK += dS^T Q_i: A = [128 keys x 64 queries] from TMEM (fp16 pairs, 8
-        // columns per 16 queries), B = dO_i / Q_i read as [d x queries] MN-major; 16 queries per MMA
+        // dV += P^T dO_i and dK += dS^T Q_i: A = [128 keys x 64 queries] from TMEM (fp16 pairs:
+        // queries 16 kk .. 16 kk + 15 in the 8 columns from 16 kk, softmax warp kk's packed share), B =
+        // dO_i / Q_i read as [d x queries] MN-major; 16 queries per MMA
+        static_assert(KV_COLS == 16, "one 16-query MMA step per softmax warp's share");
 #pragma unroll
         for (int kk = 0; kk < KV_QB / 16; ++kk) {
           const uint32_t bstep = (uint32_t)((kk * 16 * SW) >> 4);
           if (elect_one_sync())
-            umma_ts_lohi(tmem + KV_COL_DV, tmem + KV_COL_ST + 64 * sp + kk * 8, domn_lo + qp * kQSlot + bstep, mn_hi,
-                         idesc_acc, np > 0 || kk > 0);
+            umma_ts_lohi(tmem + KV_COL_DV, tmem + KV_COL_ST + 64 * sp + KV_COLS * kk, domn_lo + qp * kQSlot + bstep,
+                         mn_hi, idesc_acc, np > 0 || kk > 0);
           if (elect_one_sync())
-            umma_ts_lohi(tmem + KV_COL_DK, tmem + KV_COL_DPT + 64 * sp + kk * 8, qmn_lo + qp * kQSlot + bstep, mn_hi,
-                         idesc_acc, np > 0 || kk > 0);
+            umma_ts_lohi(tmem + KV_COL_DK, tmem + KV_COL_DPT + 64 * sp + KV_COLS * kk, qmn_lo + qp * kQSlot + bstep,
+                         mn_hi, idesc_acc, np > 0 || kk > 0);
         }
         if (elect_one_sync()) umma_commit(smem_u32(&qd_empty[qp]));
       }
@@ -617,9 +623,10 @@ __global__ void __launch_bounds__(KV_THREADS, 1) attn_bwd_dkv_kernel(const __gri
         }
       }
       bad |= f16_overflow(dmax);
-      // P^T over S^T[s] and dS^T over dP^T[s] (both already read above)
-      tmem_st_32x32b_x8(tmem + lane_off + KV_COL_ST + 64 * s + (KV_COLS / 2) * part, pp);
-      tmem_st_32x32b_x8(tmem + lane_off + KV_COL_DPT + 64 * s + (KV_COLS / 2) * part, dd);
+      // P^T over S^T[s] and dS^T over dP^T[s], each at the start of this warp's own share of the
+      // columns (read above): another warp's unread values are never overwritten
+      tmem_st_32x32b_x8(tmem + lane_off + KV_COL_ST + 64 * s + KV_COLS * part, pp);
+      tmem_st_32x32b_x8(tmem + lane_off + KV_COL_DPT + 64 * s + KV_COLS * part, dd);
       tmem_st_wait();
       tc_fence_before();
       __syncwarp();

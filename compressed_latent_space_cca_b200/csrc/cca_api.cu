@@ -593,11 +593,17 @@ size_t cca_backward_workspace_size(const cca_config_t* cfg) {
   return backward_layout(dm, layout_of(dm).total_bytes).total;
 }
 
-cca_status_t cca_backward(const cca_config_t* cfg, const void* x, const void* W_q, const void* W_k, const void* W_v,
-                          const void* convq_seq, const void* convq_chan, const void* convk_seq,
-                          const void* convk_chan, const void* W_o, const void* dy, float* dx, float* dW_q,
-                          float* dW_k, float* dW_v, float* dconvq_seq, float* dconvq_chan, float* dconvk_seq,
-                          float* dconvk_chan, float* dW_o, void* workspace, size_t workspace_bytes, void* stream) {
+}  // extern "C"
+
+namespace {
+// The three ways a backward call or its forward run: the backward with the forward recomputed into
+// its workspace (RECOMPUTE), a forward that keeps what a later backward reads (KEEP: y, the KV
+// cache and, in the workspace, the intermediates and the rows' log-sum-exp), and the backward from
+// such a workspace (SAVED).
+enum class BwdMode { RECOMPUTE, KEEP, SAVED };
+
+cca_status_t backward_call(BwdMode mode, const cca_config_t* cfg, const void* const* ins, const void* dy, float* const* gp9,
+                           void* const* outs3, void* workspace, size_t workspace_bytes, void* stream) {
   BlockDims dm;
   cca_status_t st = check_config(cfg, &dm);
   if (st != CCA_OK) return st;
@@ -606,15 +612,16 @@ cca_status_t cca_backward(const cca_config_t* cfg, const void* x, const void* W_
                 "backward needs conv_kernel 0..8, an even head_dim <= 128, n_q_heads + n_kv_heads times head_dim "
                 "<= 12288 and bf16 or fp32");
   const bool plain = dm.K == 0;  // no convolutions: their weights and gradients may be NULL
-  static const char* g_names[10] = {"dy",         "dx",          "dW_q",       "dW_k",        "dW_v",
-                                    "dconvq_seq", "dconvq_chan", "dconvk_seq", "dconvk_chan", "dW_o"};
-  const void* gp[10] = {dy, dx, dW_q, dW_k, dW_v, dconvq_seq, dconvq_chan, dconvk_seq, dconvk_chan, dW_o};
-  for (int i = 0; i < 10; ++i) {
-    if (plain && i >= 5 && i <= 8 && gp[i] == nullptr) continue;
-    if (gp[i] == nullptr) return fail(CCA_ERR_INVALID_ARG, std::string(g_names[i]) + " is NULL");
-    if (!aligned16(gp[i])) return fail(CCA_ERR_INVALID_ARG, std::string(g_names[i]) + " is not 16-byte aligned");
+  if (mode != BwdMode::KEEP) {
+    static const char* g_names[10] = {"dy",         "dx",          "dW_q",       "dW_k",        "dW_v",
+                                      "dconvq_seq", "dconvq_chan", "dconvk_seq", "dconvk_chan", "dW_o"};
+    const void* gp[10] = {dy, gp9[0], gp9[1], gp9[2], gp9[3], gp9[4], gp9[5], gp9[6], gp9[7], gp9[8]};
+    for (int i = 0; i < 10; ++i) {
+      if (plain && i >= 5 && i <= 8 && gp[i] == nullptr) continue;
+      if (gp[i] == nullptr) return fail(CCA_ERR_INVALID_ARG, std::string(g_names[i]) + " is NULL");
+      if (!aligned16(gp[i])) return fail(CCA_ERR_INVALID_ARG, std::string(g_names[i]) + " is not 16-byte aligned");
+    }
   }
-  const void* ins[9] = {x, W_q, W_k, W_v, convq_seq, convq_chan, convk_seq, convk_chan, W_o};
   static const char* in_names[9] = {"x", "W_q", "W_k", "W_v", "convq_seq", "convq_chan", "convk_seq", "convk_chan",
                                     "W_o"};
   for (int i = 0; i < 9; ++i) {
@@ -629,25 +636,66 @@ cca_status_t cca_backward(const cca_config_t* cfg, const void* x, const void* W_
   const BackwardLayout BL = backward_layout(dm, fwd);
   if (workspace_bytes < BL.total) return fail(CCA_ERR_WORKSPACE, "workspace smaller than cca_backward_workspace_size()");
   char* ws = static_cast<char*>(workspace);
-  void* outs[3] = {ws + BL.y, ws + BL.k_cache, ws + BL.v_cache};
+  void* inner[3] = {ws + BL.y, ws + BL.k_cache, ws + BL.v_cache};
   Resolved r;
   BlockPtrs p;
-  if ((st = prepare(cfg, CCA_PATH_AUTO, ins, outs, nullptr, workspace, fwd, &r, &p)) != CCA_OK) return st;
+  if ((st = prepare(cfg, CCA_PATH_AUTO, ins, mode == BwdMode::KEEP ? outs3 : inner, nullptr, workspace, fwd, &r, &p)) !=
+      CCA_OK)
+    return st;
   cudaStream_t s = static_cast<cudaStream_t>(stream);
   // the tensor-core attention backward reads the log-sum-exp rows the forward's attention leaves
   const bool tc_bwd = r.tc_attn && attention_bwd_tc_supported(r.dm);
+  // a saved forward lives in the workspace only where its attention operands are the workspace's own
+  // copies and the log-sum-exp rows exist: bf16 blocks on the tensor-core attention
+  if (mode != BwdMode::RECOMPUTE && !(tc_bwd && r.dm.lat != r.dm.io))
+    return fail(CCA_ERR_UNSUPPORTED,
+                "a saved forward needs a bf16 block on the tensor-core attention (use cca_backward otherwise)");
   if (tc_bwd) {
     p.lse2 = reinterpret_cast<float*>(ws + BL.lse);
     p.lse_stride = BL.stat_stride;
   }
-  if ((st = run_block(r, p, s, nullptr)) != CCA_OK) return st;
+  if (mode != BwdMode::SAVED && (st = run_block(r, p, s, nullptr)) != CCA_OK) return st;
+  if (mode == BwdMode::KEEP) return CCA_OK;
   DeviceInfo* di = nullptr;
   if ((st = device_info(&di)) != CCA_OK) return st;
   p.dev_err = di->err_ptr;  // the backward kernels' bounded waits and range checks report here
-  const BackwardPtrs g{dy, dx, dW_q, dW_k, dW_v, dconvq_seq, dconvq_chan, dconvk_seq, dconvk_chan, dW_o};
+  const BackwardPtrs g{dy, gp9[0], gp9[1], gp9[2], gp9[3], gp9[4], gp9[5], gp9[6], gp9[7], gp9[8]};
   const cudaError_t e = launch_backward(r.dm, p, g, BL, ws, s, tc_bwd, r.tc_down && r.tc_out);
   if (e != cudaSuccess) return cuda_fail("backward", e);
   return CCA_OK;
+}
+}  // namespace
+
+extern "C" {
+
+cca_status_t cca_backward(const cca_config_t* cfg, const void* x, const void* W_q, const void* W_k, const void* W_v,
+                          const void* convq_seq, const void* convq_chan, const void* convk_seq,
+                          const void* convk_chan, const void* W_o, const void* dy, float* dx, float* dW_q,
+                          float* dW_k, float* dW_v, float* dconvq_seq, float* dconvq_chan, float* dconvk_seq,
+                          float* dconvk_chan, float* dW_o, void* workspace, size_t workspace_bytes, void* stream) {
+  const void* ins[9] = {x, W_q, W_k, W_v, convq_seq, convq_chan, convk_seq, convk_chan, W_o};
+  float* g[9] = {dx, dW_q, dW_k, dW_v, dconvq_seq, dconvq_chan, dconvk_seq, dconvk_chan, dW_o};
+  return backward_call(BwdMode::RECOMPUTE, cfg, ins, dy, g, nullptr, workspace, workspace_bytes, stream);
+}
+
+cca_status_t cca_prefill_train(const cca_config_t* cfg, const void* x, const void* W_q, const void* W_k,
+                               const void* W_v, const void* convq_seq, const void* convq_chan, const void* convk_seq,
+                               const void* convk_chan, const void* W_o, void* y, void* k_cache, void* v_cache,
+                               void* workspace, size_t workspace_bytes, void* stream) {
+  const void* ins[9] = {x, W_q, W_k, W_v, convq_seq, convq_chan, convk_seq, convk_chan, W_o};
+  void* outs[3] = {y, k_cache, v_cache};
+  return backward_call(BwdMode::KEEP, cfg, ins, nullptr, nullptr, outs, workspace, workspace_bytes, stream);
+}
+
+cca_status_t cca_backward_saved(const cca_config_t* cfg, const void* x, const void* W_q, const void* W_k,
+                                const void* W_v, const void* convq_seq, const void* convq_chan, const void* convk_seq,
+                                const void* convk_chan, const void* W_o, const void* dy, float* dx, float* dW_q,
+                                float* dW_k, float* dW_v, float* dconvq_seq, float* dconvq_chan, float* dconvk_seq,
+                                float* dconvk_chan, float* dW_o, void* workspace, size_t workspace_bytes,
+                                void* stream) {
+  const void* ins[9] = {x, W_q, W_k, W_v, convq_seq, convq_chan, convk_seq, convk_chan, W_o};
+  float* g[9] = {dx, dW_q, dW_k, dW_v, dconvq_seq, dconvq_chan, dconvk_seq, dconvk_chan, dW_o};
+  return backward_call(BwdMode::SAVED, cfg, ins, dy, g, nullptr, workspace, workspace_bytes, stream);
 }
 
 cca_status_t cca_poll_device_status(void* stream) {

@@ -6,10 +6,11 @@
 //
 // Every step of the prefill runs for the one token in fp32 arithmetic (inputs, weights and cache in
 // the block's type). A step is bound by moving the weights and the cache once, and at batch 1 by
-// the latency of four dependent kernels. So each kernel first issues the loads that do not depend
-// on the kernel before it (weights, cache rows 0..t-1, the conv state), and only then waits for
-// that kernel (programmatic dependent launch: griddepcontrol.wait); each lets the next one launch
-// as soon as it starts (griddepcontrol.launch_dependents), so the four overlap:
+// the latency of four dependent kernels, launched one after the other on the stream. The kernels
+// can also run with programmatic dependent launch (each first issues the loads that do not depend
+// on the kernel before it, then waits for it with griddepcontrol.wait); that form is switched off
+// (kDecodePdl) because a run of the attention kernel under it produced a non-finite row whose cause
+// was not found. The four kernels:
 //   decode_down_kernel  z = x_t [W_q; W_k; W_v]^T: a warp per latent channel streams its weight row
 //                       once and serves up to kGemvBatch sequences
 //   decode_conv_kernel  a CTA per (head, KV group, sequence): the causal seq conv over the conv

@@ -356,6 +356,39 @@ cca_status_t cca_backward(const cca_config_t* cfg,
                           float* dconvk_seq, float* dconvk_chan, float* dW_o,
                           void* workspace, size_t workspace_bytes, void* stream);
 
+/*
+ * A training step's forward and backward without recomputing the forward:
+ * cca_prefill_train runs the block like cca_prefill (same inputs; y, k_cache
+ * and v_cache written) and keeps in `workspace` (>= cca_backward_workspace_size
+ * bytes, 256-byte aligned) the intermediates and each attention row's
+ * log-sum-exp that the backward reads. cca_backward_saved then computes the
+ * gradients of cca_backward from that workspace, skipping the forward: the
+ * caller passes the same cfg, inputs and workspace, and nothing may have
+ * written the workspace in between (the results are those of cca_backward).
+ * For bf16 blocks whose attention runs on the tensor cores (sm_100, head_dim
+ * 128); other blocks return CCA_ERR_UNSUPPORTED from both (use cca_prefill
+ * and cca_backward). Errors and pointer rules as cca_prefill / cca_backward;
+ * cca_prefill_train takes no conv state.
+ */
+cca_status_t cca_prefill_train(const cca_config_t* cfg,
+                               const void* x,
+                               const void* W_q, const void* W_k, const void* W_v,
+                               const void* convq_seq, const void* convq_chan,
+                               const void* convk_seq, const void* convk_chan,
+                               const void* W_o,
+                               void* y, void* k_cache, void* v_cache,
+                               void* workspace, size_t workspace_bytes, void* stream);
+cca_status_t cca_backward_saved(const cca_config_t* cfg,
+                                const void* x,
+                                const void* W_q, const void* W_k, const void* W_v,
+                                const void* convq_seq, const void* convq_chan,
+                                const void* convk_seq, const void* convk_chan,
+                                const void* W_o, const void* dy,
+                                float* dx, float* dW_q, float* dW_k, float* dW_v,
+                                float* dconvq_seq, float* dconvq_chan,
+                                float* dconvk_seq, float* dconvk_chan, float* dW_o,
+                                void* workspace, size_t workspace_bytes, void* stream);
+
 /* Synchronizes `stream`, then reports and clears the device error word:
  * CCA_ERR_DEVICE_TIMEOUT if a bounded wait in a kernel gave up since the last
  * poll, CCA_ERR_NUMERIC_RANGE if a finite fp16 intermediate overflowed (its

@@ -186,3 +186,35 @@ def test_backward_rejects_bad_arguments():
     too_long = cca.config_from_shape(shape.replace(conv_kernel=9))
     assert cca.backward_workspace_size(too_long) == 0
     torch.cuda.synchronize()
+
+
+@pytest.mark.parametrize("shape", [BF16_CASES[0], BF16_CASES[1], PLAIN_CASES[0]], ids=["ccgqa", "pre_mean", "plain_mha"])
+def test_backward_from_saved_forward(shape):
+    """prefill_train + backward(saved=True) gives prefill's outputs exactly and cca_backward's gradients
+    up to the order of fp32 atomic sums (dK / dV across key-tile chunks, K-split GEMM slices, dW_c
+    across row blocks), which can move a bf16 hi / lo split by one unit of the hi part (about 2^-16
+    of a value): the same kernels run on the same values, only the forward is not recomputed. A
+    saved path that read a wrong activation would differ by O(1)."""
+    inp = {k: v.cuda() for k, v in workloads.make_inputs(shape).items()}
+    dy = workloads.make_dy(shape).cuda()
+    cfg = cca.config_from_shape(shape)
+    ref_fwd = cca.prefill(cfg, inp)
+    ref = cca.backward(cfg, inp, dy)
+    fwd = cca.prefill_train(cfg, inp)
+    for k in ("y", "k_cache", "v_cache"):
+        assert torch.equal(fwd[k], ref_fwd[k]), k
+    got = cca.backward(cfg, inp, dy, workspace=fwd["workspace"], saved=True)
+    assert cca.poll_device_status() == cca.CCA_OK
+    for n in got:
+        a, b = got[n].double(), ref[n].double()
+        rms = b.pow(2).mean().sqrt().clamp_min(1e-30)
+        assert ((a - b).abs().max() / rms).item() <= 1e-3, n
+
+
+def test_saved_forward_unsupported_for_fp32():
+    shape = FP32_CASES[0]
+    inp = {k: v.cuda() for k, v in workloads.make_inputs(shape).items()}
+    cfg = cca.config_from_shape(shape)
+    with pytest.raises(cca.CcaError) as e:
+        cca.prefill_train(cfg, inp)
+    assert e.value.status == cca.CCA_ERR_UNSUPPORTED
