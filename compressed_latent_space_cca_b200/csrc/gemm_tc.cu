@@ -177,10 +177,17 @@ __device__ __forceinline__ bool store_row_chunk(const GemmParams& p, long long r
   return bad;
 }
 
-template <int MH, bool PAIR>
+// GEN: the general form (K slices, K-wrapped operands, MN-major operands). Without it those
+// parameters are compile-time off and the loops are the plain K-major ones: the forward's
+// projections are bound by the rate TMA copies and MMAs are issued at, and the general form's
+// runtime selections measured 15-20 % slower there.
+template <int MH, bool PAIR, bool GEN>
 __global__ void __launch_bounds__(Shape<MH, PAIR>::NUM_THREADS, 1)
     gemm_tc_kernel(const __grid_constant__ GemmMaps maps, const GemmParams p) {
   using T = Shape<MH, PAIR>;
+  const bool a_mn = GEN && p.a_mn, b_mn = GEN && p.b_mn;
+  const int a_kwrap = GEN ? p.a_kwrap : 0, b_kwrap = GEN ? p.b_kwrap : 0;
+  const int tiles = GEN ? p.tiles : p.num_tiles;
   constexpr int BM = T::BM, TM = T::TM, STAGES = T::STAGES, STAGE_BYTES = T::STAGE_BYTES, A_BYTES = T::A_BYTES;
   constexpr int ACC_BUFS = T::ACC_BUFS;
   extern __shared__ uint8_t smem_raw[];
@@ -237,8 +244,8 @@ __global__ void __launch_bounds__(Shape<MH, PAIR>::NUM_THREADS, 1)
       int stage = 0;
       uint32_t phase = 0;
       for (int t = unit; t < p.num_tiles; t += n_units) {
-        const int tile = t % p.tiles, kb0 = (t / p.tiles) * p.kb_slice;
-        const int kb1 = kb0 + p.kb_slice < kblocks ? kb0 + p.kb_slice : kblocks;
+        const int tile = GEN ? t % tiles : t, kb0 = GEN ? (t / tiles) * p.kb_slice : 0;
+        const int kb1 = GEN && kb0 + p.kb_slice < kblocks ? kb0 + p.kb_slice : kblocks;
         const int m0 = (tile / p.n_tiles_n) * TM + (int)rank * 128;  // this CTA's first row
         const int n0 = (tile % p.n_tiles_n) * BN;
         for (int kb = kb0; kb < kb1; ++kb) {
@@ -252,11 +259,11 @@ __global__ void __launch_bounds__(Shape<MH, PAIR>::NUM_THREADS, 1)
             mbar_arrive_expect_tx(fb, STAGE_BYTES);
           }
           uint8_t* sa = smem + stage * STAGE_BYTES;
-          const int ka = p.a_kwrap ? (kb * BK) % p.a_kwrap : kb * BK;
-          const int kbx = p.b_kwrap ? (kb * BK) % p.b_kwrap : kb * BK;
+          const int ka = a_kwrap ? (kb * BK) % a_kwrap : kb * BK;
+          const int kbx = b_kwrap ? (kb * BK) % b_kwrap : kb * BK;
 #pragma unroll
           for (int h = 0; h < MH; ++h) {
-            if (p.a_mn) {  // two 64-row chunks of M, each [64 K][64 M]
+            if (a_mn) {  // two 64-row chunks of M, each [64 K][64 M]
 #pragma unroll
               for (int c = 0; c < 2; ++c) {
                 const uint32_t dst = smem_u32(sa + h * A_HALF_BYTES + c * MN_CHUNK_BYTES);
@@ -277,7 +284,7 @@ __global__ void __launch_bounds__(Shape<MH, PAIR>::NUM_THREADS, 1)
               while (mi + 1 < p.nb && row >= p.row_start[mi + 1]) ++mi;
               r = row - p.row_start[mi];
             }
-            if (p.b_mn) {  // one B matrix stored [K][N]: two 64-column chunks of N, each [64 K][64 N]
+            if (b_mn) {  // one B matrix stored [K][N]: two 64-column chunks of N, each [64 K][64 N]
 #pragma unroll
               for (int c = 0; c < 2; ++c) {
                 const uint32_t dst = smem_u32(sa + A_BYTES + h * (128 * BK * 2) + c * MN_CHUNK_BYTES);
@@ -302,14 +309,14 @@ __global__ void __launch_bounds__(Shape<MH, PAIR>::NUM_THREADS, 1)
       // ------------------------------------------------------ MMA issuer --
       // Every lane runs this loop and its bounded waits; elect_one_sync picks the lane that issues
       // each tcgen05 instruction (issuing from a lane-divergent branch costs more per MMA).
-      const uint32_t idesc = idesc_f32acc(PAIR ? 256 : 128, BN, p.a_mn, p.b_mn, p.in_fmt);
+      const uint32_t idesc = idesc_f32acc(PAIR ? 256 : 128, BN, a_mn, b_mn, p.in_fmt);
       // descriptors built once; a stage step adds STAGE_BYTES / 16 to the start address, a K = 16 step 2
       // (K-major: 32 bytes along the row) or 128 (MN-major: 16 rows of 128 bytes); MN-major operands
       // carry LBO = the 64-wide chunk's bytes (it lives in the low word), SBO = 8 rows either way
       const uint32_t d_hi = desc_hi(smem_desc_sw128(smem_u32(smem), 16, 1024));
-      const uint32_t a_lo0 = desc_lo(smem_desc_sw128(smem_u32(smem), p.a_mn ? MN_CHUNK_BYTES : 16, 1024));
-      const uint32_t b_lo0 = desc_lo(smem_desc_sw128(smem_u32(smem + A_BYTES), p.b_mn ? MN_CHUNK_BYTES : 16, 1024));
-      const uint32_t a_kstep = p.a_mn ? 128 : 2, b_kstep = p.b_mn ? 128 : 2;
+      const uint32_t a_lo0 = desc_lo(smem_desc_sw128(smem_u32(smem), a_mn ? MN_CHUNK_BYTES : 16, 1024));
+      const uint32_t b_lo0 = desc_lo(smem_desc_sw128(smem_u32(smem + A_BYTES), b_mn ? MN_CHUNK_BYTES : 16, 1024));
+      const uint32_t a_kstep = a_mn ? 128 : 2, b_kstep = b_mn ? 128 : 2;
       int stage = 0;
       uint32_t phase = 0;
       int i = 0;
@@ -319,8 +326,8 @@ __global__ void __launch_bounds__(Shape<MH, PAIR>::NUM_THREADS, 1)
         if (!mbar_wait_bounded(smem_u32(&tempty[acc]), tph ^ 1, p.err, abort_flag, wait_site(kSiteGemm, 2, 2))) goto mma_done;
         tc_fence_after();
         const uint32_t d_tmem = tmem_base + acc * BN;
-        const int kb0 = (t / p.tiles) * p.kb_slice;
-        const int kb1 = kb0 + p.kb_slice < kblocks ? kb0 + p.kb_slice : kblocks;
+        const int kb0 = GEN ? (t / tiles) * p.kb_slice : 0;
+        const int kb1 = GEN && kb0 + p.kb_slice < kblocks ? kb0 + p.kb_slice : kblocks;
         for (int kb = kb0; kb < kb1; ++kb) {
           if (!mbar_wait_bounded(smem_u32(&full[stage]), phase, p.err, abort_flag, wait_site(kSiteGemm, 2, 3))) goto mma_done;
           tc_fence_after();
@@ -389,7 +396,7 @@ __global__ void __launch_bounds__(Shape<MH, PAIR>::NUM_THREADS, 1)
       const uint32_t tph = (i / ACC_BUFS) & 1;
       if (!mbar_wait_bounded(smem_u32(&tfull[acc]), tph, p.err, abort_flag, wait_site(kSiteGemm, 3, 4))) break;
       tc_fence_after();
-      const int tile = t % p.tiles;
+      const int tile = GEN ? t % tiles : t;
       const long long m0 = (long long)(tile / p.n_tiles_n) * TM + rank * 128;
       const int n0 = (tile % p.n_tiles_n) * BN;
       const long long row0 = m0 + half * T::HS + quad * 32;  // this warp's 32 rows
@@ -512,6 +519,17 @@ int gemm_tc_ksplit(long long M, int N, int K) {
   return ks < 1 ? 1 : (int)ks;
 }
 
+namespace {
+template <int MH, bool GEN>
+cudaError_t launch_single(int grid, const GemmMaps& maps, const GemmParams& p, cudaStream_t stream) {
+  cudaError_t e = cudaFuncSetAttribute(gemm_tc_kernel<MH, false, GEN>, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                                       (int)Shape<MH>::SMEM_BYTES);
+  if (e != cudaSuccess) return e;
+  gemm_tc_kernel<MH, false, GEN><<<grid, Shape<MH>::NUM_THREADS, Shape<MH>::SMEM_BYTES, stream>>>(maps, p);
+  return cudaGetLastError();
+}
+}  // namespace
+
 bool gemm_tc_supported(long long M, int N, int K) {
   return M >= 1 && M < (1ll << 31) && K >= BK && K % BK == 0 && N >= 128 && N % 128 == 0;
 }
@@ -535,7 +553,9 @@ void pair_config(cudaLaunchConfig_t& cfg, cudaLaunchAttribute* attr, int grid, c
 template <int MH>
 int pair_clusters() {
   static const int n = [] {
-    if (cudaFuncSetAttribute(gemm_tc_kernel<MH, true>, cudaFuncAttributeMaxDynamicSharedMemorySize,
+    if (cudaFuncSetAttribute(gemm_tc_kernel<MH, true, false>, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                             (int)Shape<MH, true>::SMEM_BYTES) != cudaSuccess ||
+        cudaFuncSetAttribute(gemm_tc_kernel<MH, true, true>, cudaFuncAttributeMaxDynamicSharedMemorySize,
                              (int)Shape<MH, true>::SMEM_BYTES) != cudaSuccess) {
       cudaGetLastError();
       return 0;
@@ -544,7 +564,7 @@ int pair_clusters() {
     cudaLaunchAttribute attr[1];
     pair_config<MH>(cfg, attr, 2 * (num_sms() / 2), nullptr);
     int c = 0;
-    if (cudaOccupancyMaxActiveClusters(&c, gemm_tc_kernel<MH, true>, &cfg) != cudaSuccess) {
+    if (cudaOccupancyMaxActiveClusters(&c, gemm_tc_kernel<MH, true, false>, &cfg) != cudaSuccess) {
       cudaGetLastError();
       return 0;
     }
@@ -656,27 +676,18 @@ cudaError_t launch_gemm_tc(const GemmTcArgs& a, cudaStream_t stream) {
   p.kb_slice = (kblocks + ks - 1) / ks;
   p.ksplit = (kblocks + p.kb_slice - 1) / p.kb_slice;  // no empty slice
   p.num_tiles = p.tiles * p.ksplit;
-  cudaError_t e;
+  const bool gen = p.ksplit > 1 || p.a_kwrap || p.b_kwrap || p.a_mn || p.b_mn;
   if (pair) {
     const int clusters = p.num_tiles < pair_clusters<1>() ? p.num_tiles : pair_clusters<1>();
     cudaLaunchConfig_t cfg = {};
     cudaLaunchAttribute attr[1];
     pair_config<1>(cfg, attr, 2 * clusters, stream);
-    return cudaLaunchKernelEx(&cfg, gemm_tc_kernel<1, true>, maps, p);
+    return gen ? cudaLaunchKernelEx(&cfg, gemm_tc_kernel<1, true, true>, maps, p)
+               : cudaLaunchKernelEx(&cfg, gemm_tc_kernel<1, true, false>, maps, p);
   }
   const int grid = p.num_tiles < num_sms() ? p.num_tiles : num_sms();
-  if (big) {
-    if ((e = cudaFuncSetAttribute(gemm_tc_kernel<2, false>, cudaFuncAttributeMaxDynamicSharedMemorySize,
-                                  (int)Shape<2>::SMEM_BYTES)) != cudaSuccess)
-      return e;
-    gemm_tc_kernel<2, false><<<grid, Shape<2>::NUM_THREADS, Shape<2>::SMEM_BYTES, stream>>>(maps, p);
-  } else {
-    if ((e = cudaFuncSetAttribute(gemm_tc_kernel<1, false>, cudaFuncAttributeMaxDynamicSharedMemorySize,
-                                  (int)Shape<1>::SMEM_BYTES)) != cudaSuccess)
-      return e;
-    gemm_tc_kernel<1, false><<<grid, Shape<1>::NUM_THREADS, Shape<1>::SMEM_BYTES, stream>>>(maps, p);
-  }
-  return cudaGetLastError();
+  if (big) return gen ? launch_single<2, true>(grid, maps, p, stream) : launch_single<2, false>(grid, maps, p, stream);
+  return gen ? launch_single<1, true>(grid, maps, p, stream) : launch_single<1, false>(grid, maps, p, stream);
 }
 
 }  // namespace cca
