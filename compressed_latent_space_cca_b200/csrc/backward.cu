@@ -466,72 +466,79 @@ __device__ __forceinline__ void store_dlat(const DlatOut& o, long long row, int 
 // ------------------------------------------------------------------ per-token backward --
 // Row t of one sequence: dq, dk turned back by RoPE; the QK-mean transpose gives dc (the
 // channel-mix outputs' gradient) and the latents' direct gradient dpre; dv goes through the value
-// shift's transpose (channels [vfrom, Lkv) take the next token's gradient). Thread = one pair
-// (i, i + d/2) of one head (q heads, then K heads), or one V channel.
+// shift's transpose (channels [vfrom, Lkv) take the next token's gradient). A block takes two rows,
+// 128 threads each. Thread = one pair (i, i + d/2) of one KV group g: the group's G query heads and
+// its K head are turned by the same angle t theta_i (one sincos), and the QK-mean terms of the
+// group's channels i and i + d/2 need only those heads. Then one V channel per thread and step.
 struct Theta64 {
   double v[64];  // base^(-2i/d)
 };
 
+__device__ __forceinline__ void rope_back(float& x1, float& x2, float cs, float sn) {
+  const float y1 = x1 * cs + x2 * sn, y2 = x2 * cs - x1 * sn;
+  x1 = y1;
+  x2 = y2;
+}
+
 __global__ void __launch_bounds__(256) token_bwd_kernel(const float* __restrict__ dq, const float* __restrict__ dk,
                                                         const float* __restrict__ dv, float* __restrict__ dc,
-                                                        float* __restrict__ dpre, const DlatOut dlat, int S,
-                                                        int nq, int nkv, int d, int mode, int vshift, int vfrom,
+                                                        float* __restrict__ dpre, const DlatOut dlat, long long T,
+                                                        int S, int nq, int nkv, int d, int mode, int vshift, int vfrom,
                                                         int use_rope, const __grid_constant__ Theta64 theta,
                                                         int plain) {
-  const long long row = blockIdx.x;  // b * S + t
+  const long long row = 2 * (long long)blockIdx.x + (threadIdx.x >> 7);  // b * S + t
+  if (row >= T) return;
+  const int lt = threadIdx.x & 127;
   const int t = (int)(row % S);
-  const int G = nq / nkv, Lq = nq * d, Lkv = nkv * d, half = d / 2, Nlat = Lq + 2 * Lkv;
+  const int G = nq / nkv, Lq = nq * d, Lkv = nkv * d, half = d / 2, W = Lq + Lkv;
   const float R = (mode & 1) ? 1.f : 0.f, P = (mode & 2) ? 1.f : 0.f;
-  extern __shared__ float ta[];  // dqa [Lq], dka [Lkv]
-  float* dqa = ta;
-  float* dka = ta + Lq;
-  for (int e = threadIdx.x; e < (nq + nkv) * half; e += blockDim.x) {
-    const int hh = e / half, i = e % half;
-    const bool isq = hh < nq;
-    const float* src = isq ? dq + row * Lq + hh * d : dk + row * Lkv + (hh - nq) * d;
-    float x1 = src[i], x2 = src[i + half];
+  const float* dqr = dq + row * Lq;
+  const float* dkr = dk + row * Lkv;
+  for (int e = lt; e < nkv * half; e += 128) {
+    const int g = e / half, i = e % half;
+    float cs = 1.f, sn = 0.f;
     if (use_rope) {  // turn back by t theta_i (angle reduced in fp64)
       const double a = (double)t * theta.v[i];
       const double kk = rint(a * 0.15915494309189535);
       double r = fma(-kk, 6.283185307179586, a);
       r = fma(-kk, 2.4492935982947064e-16, r);
-      float sn, cs;
       sincosf((float)r, &sn, &cs);
-      const float y1 = x1 * cs + x2 * sn, y2 = x2 * cs - x1 * sn;
-      x1 = y1;
-      x2 = y2;
     }
-    float* dst = isq ? dqa + hh * d : dka + (hh - nq) * d;
-    dst[i] = x1;
-    dst[i + half] = x2;
-  }
-  __syncthreads();
-  // QK-mean transpose: da_h = dqa_h / 2 + dka_g / (2G), db_g = sum_{h in g} dqa_h / 2 + dka_g / 2
-  for (int e = threadIdx.x; e < Lq + Lkv; e += blockDim.x) {
-    float a, bsum;
-    float direct;
-    if (e < Lq) {
-      const int h = e / d, i = e % d, g = h / G;
-      direct = dqa[e];
-      a = 0.5f * dqa[e] + (0.5f / (float)G) * dka[g * d + i];
-      bsum = a;
-    } else {
-      const int c = e - Lq, g = c / d, i = c % d;
-      direct = dka[c];
-      float s = 0.f;
-      for (int hh = 0; hh < G; ++hh) s += dqa[(g * G + hh) * d + i];
-      a = 0.5f * s + 0.5f * dka[c];
-      bsum = a;
+    float k1 = dkr[g * d + i], k2 = dkr[g * d + i + half];
+    if (use_rope) rope_back(k1, k2, cs, sn);
+    // QK-mean transpose: da_h = dqa_h / 2 + dka_g / (2G), db_g = sum_{h in g} dqa_h / 2 + dka_g / 2
+    float s1 = 0.f, s2 = 0.f;
+    for (int hh = 0; hh < G; ++hh) {
+      const int c = (g * G + hh) * d + i;
+      float q1 = dqr[c], q2 = dqr[c + half];
+      if (use_rope) rope_back(q1, q2, cs, sn);
+      s1 += q1;
+      s2 += q2;
+      const float a1 = 0.5f * q1 + (0.5f / (float)G) * k1, a2 = 0.5f * q2 + (0.5f / (float)G) * k2;
+      if (plain) {  // no convolutions: the attention inputs are the latents
+        store_dlat(dlat, row, c, q1);
+        store_dlat(dlat, row, c + half, q2);
+      } else {
+        dc[row * W + c] = q1 + P * a1;
+        dc[row * W + c + half] = q2 + P * a2;
+        dpre[row * W + c] = R * a1;
+        dpre[row * W + c + half] = R * a2;
+      }
     }
-    if (plain) {  // no convolutions: the attention inputs are the latents
-      store_dlat(dlat, row, e, direct);
+    const int c = Lq + g * d + i;
+    const float a1 = 0.5f * s1 + 0.5f * k1, a2 = 0.5f * s2 + 0.5f * k2;
+    if (plain) {
+      store_dlat(dlat, row, c, k1);
+      store_dlat(dlat, row, c + half, k2);
     } else {
-      dc[row * (Lq + Lkv) + e] = direct + P * bsum;
-      dpre[row * (Lq + Lkv) + e] = R * a;
+      dc[row * W + c] = k1 + P * a1;
+      dc[row * W + c + half] = k2 + P * a2;
+      dpre[row * W + c] = R * a1;
+      dpre[row * W + c + half] = R * a2;
     }
   }
   // value shift transpose
-  for (int c = threadIdx.x; c < Lkv; c += blockDim.x) {
+  for (int c = lt; c < Lkv; c += 128) {
     float val;
     if (vshift && c >= vfrom) val = (t + 1 < S) ? dv[(row + 1) * Lkv + c] : 0.f;
     else val = dv[row * Lkv + c];
@@ -690,62 +697,111 @@ __global__ void __launch_bounds__(256) chan_bwd_kernel(const float* __restrict__
   }
 }
 
-// Seq-conv transpose: dlat[t, c] = dpre[t, c] + sum_j w[c][j] ds[t + K-1-j, c] (within the sequence).
-template <typename Tc>
-__global__ void __launch_bounds__(256) seq_bwd_kernel(const float* __restrict__ ds, const float* __restrict__ dpre,
-                                                      const Tc* __restrict__ cq_seq, const Tc* __restrict__ ck_seq,
-                                                      const DlatOut dlat, int S, int nq, int nkv, int d, int K) {
-  const long long row = blockIdx.x;
-  const int t = (int)(row % S);
-  const int Lq = nq * d, Lkv = nkv * d, W = Lq + Lkv;
-  for (int e = threadIdx.x; e < W; e += blockDim.x) {
-    const bool isq = e < Lq;
-    const int c = isq ? e : e - Lq;
-    const Tc* w = (isq ? cq_seq : ck_seq) + (long long)c * K;
-    float acc = dpre[row * W + e];
+// Seq-conv transpose and tap gradients in one pass over ds (both within each sequence):
+//   dlat[t, c] = dpre[t, c] + sum_j w[c][j] ds[t + K-1-j, c]       (the q~ and k~ channels)
+//   dw[c][j]   = sum_t ds[t, c] z[t - K+1 + j, c]                    (z: the latents)
+// Thread = one channel over a slice of consecutive rows, with ds[t .. t+K-1] and z[t-K+1 .. t] in
+// registers (one new row of each per step); block = 32 channels x 8 slices; the slices' tap sums
+// reduce in shared memory, then atomically across blocks.
+constexpr int kSeqSliceRows = 32;
+template <int K, typename Tc, typename Tl>
+__global__ void __launch_bounds__(256) seq_tap_bwd_kernel(const float* __restrict__ ds, const float* __restrict__ dpre,
+                                                          const Tc* __restrict__ cq_seq, const Tc* __restrict__ ck_seq,
+                                                          const Tl* __restrict__ lat, const DlatOut dlat,
+                                                          float* __restrict__ dwq, float* __restrict__ dwk, long long T,
+                                                          int S, int Lq, int Lkv) {
+  __shared__ float red[8][32][K];
+  const int W = Lq + Lkv, Nlat = Lq + 2 * Lkv;
+  const int lane = threadIdx.x & 31, slice = threadIdx.x >> 5;
+  const int e = blockIdx.x * 32 + lane;  // latent column e (q~ channels, then k~)
+  const long long r0 = ((long long)blockIdx.y * 8 + slice) * kSeqSliceRows;
+  const long long r1 = r0 + kSeqSliceRows < T ? r0 + kSeqSliceRows : T;
+  float acc[K];
+#pragma unroll
+  for (int j = 0; j < K; ++j) acc[j] = 0.f;
+  if (e < W && r0 < T) {
+    const Tc* wp = e < Lq ? cq_seq + (long long)e * K : ck_seq + (long long)(e - Lq) * K;
+    float w[K], f[K], z[K];  // f[m] = ds[r + m], z[j] = z[r - K+1 + j]
+#pragma unroll
     for (int j = 0; j < K; ++j) {
-      const int tt = t + K - 1 - j;
-      if (tt < S) acc = fmaf(ld_f(w + j), ds[(row - t + tt) * W + e], acc);
+      w[j] = ld_f(wp + j);
+      f[j] = 0.f;
+      z[j] = 0.f;
     }
-    store_dlat(dlat, row, e, acc);
-  }
-}
-
-// Seq-conv tap gradients: dw[c][j] = sum over rows t of ds[t, c] z[t - K+1 + j, c] (within each
-// sequence). Block = 32 channels x 8 row slices; the slices reduce in shared memory, then atomically
-// across blocks of rows.
-template <typename Tl>
-__global__ void __launch_bounds__(256) tap_grad_kernel(const float* __restrict__ ds, const Tl* __restrict__ lat,
-                                                       float* __restrict__ dwq, float* __restrict__ dwk, int B, int S,
-                                                       int nq, int nkv, int d, int K, int rows_per_block) {
-  __shared__ float red[8][32][8];
-  const int Lq = nq * d, Lkv = nkv * d, Nlat = Lq + 2 * Lkv, W = Lq + Lkv;
-  const int e = blockIdx.x * 32 + (threadIdx.x & 31);
-  const int slice = threadIdx.x >> 5;
-  const long long T = (long long)B * S;
-  const long long r0 = (long long)blockIdx.y * rows_per_block;
-  float acc[8] = {};
-  if (e < W) {
-    const int col = e < Lq ? e : Lq + (e - Lq);
-    for (long long row = r0 + slice; row < r0 + rows_per_block && row < T; row += 8) {
-      const int t = (int)(row % S);
-      const float g = ds[row * W + e];
-      for (int j = 0; j < K && j < 8; ++j) {
-        const int src = t - (K - 1) + j;
-        if (src >= 0) acc[j] = fmaf(g, ld_f(lat + (row - t + src) * Nlat + col), acc[j]);
+#pragma unroll
+    for (int m = 0; m + 1 < K; ++m)
+      if (r0 + m < T) f[m] = ds[(r0 + m) * W + e];
+#pragma unroll
+    for (int j = 0; j + 1 < K; ++j) {
+      const long long src = r0 - (K - 1) + j;
+      if (src >= 0) z[j] = ld_f(lat + src * Nlat + e);
+    }
+    int t = (int)(r0 % S);
+#pragma unroll 1  // measured: unrolling 2 or 4 rows raised the registers and ran slower
+    for (long long r = r0; r < r1; ++r) {
+      f[K - 1] = r + K - 1 < T ? ds[(r + K - 1) * W + e] : 0.f;
+      z[K - 1] = ld_f(lat + r * Nlat + e);
+      float out = dpre[r * W + e];
+#pragma unroll
+      for (int j = 0; j < K; ++j)
+        if (t + K - 1 - j < S) out = fmaf(w[j], f[K - 1 - j], out);
+      store_dlat(dlat, r, e, out);
+      const float g = f[0];
+#pragma unroll
+      for (int j = 0; j < K; ++j)
+        if (t - (K - 1) + j >= 0) acc[j] = fmaf(g, z[j], acc[j]);
+#pragma unroll
+      for (int m = 0; m + 1 < K; ++m) {
+        f[m] = f[m + 1];
+        z[m] = z[m + 1];
       }
+      if (++t == S) t = 0;
     }
   }
 #pragma unroll
-  for (int j = 0; j < 8; ++j) red[slice][threadIdx.x & 31][j] = acc[j];
+  for (int j = 0; j < K; ++j) red[slice][lane][j] = acc[j];
   __syncthreads();
   if (slice == 0 && e < W) {
-    for (int j = 0; j < K && j < 8; ++j) {
-      float s = 0.f;
-      for (int sl = 0; sl < 8; ++sl) s += red[sl][threadIdx.x & 31][j];
+#pragma unroll
+    for (int j = 0; j < K; ++j) {
+      float sum = 0.f;
+      for (int sl = 0; sl < 8; ++sl) sum += red[sl][lane][j];
       float* dst = e < Lq ? dwq + (long long)e * K + j : dwk + (long long)(e - Lq) * K + j;
-      atomicAdd(dst, s);
+      atomicAdd(dst, sum);
     }
+  }
+}
+
+template <int K, typename Tc, typename Tl>
+cudaError_t launch_seq_tap_k(const float* ds, const float* dpre, const void* cq_seq, const void* ck_seq, const void* lat,
+                             const DlatOut& dlat, float* dwq, float* dwk, long long T, int S, int Lq, int Lkv,
+                             cudaStream_t stream) {
+  const dim3 grid((unsigned)((Lq + Lkv + 31) / 32), (unsigned)((T + 8 * kSeqSliceRows - 1) / (8 * kSeqSliceRows)));
+  seq_tap_bwd_kernel<K, Tc, Tl><<<grid, 256, 0, stream>>>(ds, dpre, static_cast<const Tc*>(cq_seq),
+                                                          static_cast<const Tc*>(ck_seq), static_cast<const Tl*>(lat),
+                                                          dlat, dwq, dwk, T, S, Lq, Lkv);
+  return cudaGetLastError();
+}
+
+template <typename Tc, typename Tl>
+cudaError_t launch_seq_tap(int K, const float* ds, const float* dpre, const void* cq_seq, const void* ck_seq,
+                           const void* lat, const DlatOut& dlat, float* dwq, float* dwk, long long T, int S, int Lq,
+                           int Lkv, cudaStream_t stream) {
+  switch (K) {
+#define CCA_SEQ_TAP_CASE(k) \
+  case k:                   \
+    return launch_seq_tap_k<k, Tc, Tl>(ds, dpre, cq_seq, ck_seq, lat, dlat, dwq, dwk, T, S, Lq, Lkv, stream);
+    CCA_SEQ_TAP_CASE(1)
+    CCA_SEQ_TAP_CASE(2)
+    CCA_SEQ_TAP_CASE(3)
+    CCA_SEQ_TAP_CASE(4)
+    CCA_SEQ_TAP_CASE(5)
+    CCA_SEQ_TAP_CASE(6)
+    CCA_SEQ_TAP_CASE(7)
+    CCA_SEQ_TAP_CASE(8)
+#undef CCA_SEQ_TAP_CASE
+    default:
+      return cudaErrorInvalidValue;
   }
 }
 
@@ -1108,8 +1164,8 @@ cudaError_t launch_backward(const BlockDims& dm, const BlockPtrs& p, const Backw
   {
     Theta64 th{};
     for (int i = 0; i < d / 2; ++i) th.v[i] = pow((double)dm.rope_base, -2.0 * (double)i / (double)d);
-    token_bwd_kernel<<<(unsigned)T, 256, sizeof(float) * W, stream>>>(
-        dq, dk, dv, dc, dpre, dlat_out, dm.S, dm.nq, dm.nkv, d, dm.qk_mean_mode, dm.value_shift, dm.vshift_from,
+    token_bwd_kernel<<<(unsigned)((T + 1) / 2), 256, 0, stream>>>(
+        dq, dk, dv, dc, dpre, dlat_out, T, dm.S, dm.nq, dm.nkv, d, dm.qk_mean_mode, dm.value_shift, dm.vshift_from,
         dm.use_rope, th, dm.K == 0);
     if ((e = cudaGetLastError()) != cudaSuccess) return e;
   }
@@ -1166,30 +1222,18 @@ cudaError_t launch_backward(const BlockDims& dm, const BlockPtrs& p, const Backw
                   d, d, T, dm.nkv, false, stream)) != cudaSuccess)
       return e;
   }
-  // 6. seq conv: dlat (q and k channels) and the tap gradients
-  if (it == DType::BF16)
-    seq_bwd_kernel<__nv_bfloat16><<<(unsigned)T, 256, 0, stream>>>(
-        ds, dpre, static_cast<const __nv_bfloat16*>(p.cq_seq), static_cast<const __nv_bfloat16*>(p.ck_seq), dlat_out,
-        dm.S, dm.nq, dm.nkv, d, dm.K);
-  else
-    seq_bwd_kernel<float><<<(unsigned)T, 256, 0, stream>>>(ds, dpre, static_cast<const float*>(p.cq_seq),
-                                                            static_cast<const float*>(p.ck_seq), dlat_out, dm.S, dm.nq,
-                                                            dm.nkv, d, dm.K);
-  if ((e = cudaGetLastError()) != cudaSuccess) return e;
+  // 6. seq conv: dlat (q and k channels) and the tap gradients, one pass
   if ((e = cudaMemsetAsync(g.dconvq_seq, 0, sizeof(float) * Lq * dm.K, stream)) != cudaSuccess ||
       (e = cudaMemsetAsync(g.dconvk_seq, 0, sizeof(float) * Lkv * dm.K, stream)) != cudaSuccess)
     return e;
-  {
-    const int rpb = 512;
-    const dim3 grid((W + 31) / 32, (unsigned)((T + rpb - 1) / rpb));
-    if (lt == DType::F16)
-      tap_grad_kernel<__half><<<grid, 256, 0, stream>>>(ds, static_cast<const __half*>(p.qkv_lat), g.dconvq_seq,
-                                                        g.dconvk_seq, dm.B, dm.S, dm.nq, dm.nkv, d, dm.K, rpb);
-    else
-      tap_grad_kernel<float><<<grid, 256, 0, stream>>>(ds, static_cast<const float*>(p.qkv_lat), g.dconvq_seq,
-                                                       g.dconvk_seq, dm.B, dm.S, dm.nq, dm.nkv, d, dm.K, rpb);
-    if ((e = cudaGetLastError()) != cudaSuccess) return e;
-  }
+  e = it == DType::BF16 && lt == DType::F16
+          ? launch_seq_tap<__nv_bfloat16, __half>(dm.K, ds, dpre, p.cq_seq, p.ck_seq, p.qkv_lat, dlat_out, g.dconvq_seq,
+                                                  g.dconvk_seq, T, dm.S, Lq, Lkv, stream)
+      : it == DType::F32 && lt == DType::F32
+          ? launch_seq_tap<float, float>(dm.K, ds, dpre, p.cq_seq, p.ck_seq, p.qkv_lat, dlat_out, g.dconvq_seq,
+                                         g.dconvk_seq, T, dm.S, Lq, Lkv, stream)
+          : cudaErrorInvalidValue;
+  if (e != cudaSuccess) return e;
   }  // convolutions
   // 7. down-projection: dx = dlat [W_q; W_k; W_v];  dW_* = dlat^T x
   const void* Ws[3] = {p.Wq, p.Wk, p.Wv};
