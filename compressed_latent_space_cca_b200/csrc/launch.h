@@ -122,8 +122,8 @@ struct GemmTcArgs {
   int a_kext, b_kext;
 };
 cudaError_t launch_gemm_tc(const GemmTcArgs& a, cudaStream_t stream);
-// K slices that give a GEMM with fewer 256 x 256 output tiles than the device has CTA pairs about
-// two rounds of work (1 otherwise), with slices of at least 256 along K
+// K slices for a GEMM with fewer 256 x 256 output tiles than the device has CTA pairs (1 otherwise):
+// the count whose items fill the rounds of pairs best, with slices of at least 256 along K
 int gemm_tc_ksplit(long long M, int N, int K);
 // dst[0, n) = fp16 copy of the bf16 src times scale (fp16 overflow reported as a range error)
 cudaError_t launch_convert_f16(const void* src, void* dst, long long n, unsigned* dev_err, cudaStream_t stream,
