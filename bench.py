@@ -95,15 +95,16 @@ def file_sha(path):
         return hashlib.sha256(f.read()).hexdigest()[:16]
 
 
-def traffic_record():
+def traffic_record(workload):
     """DRAM bytes per attention launch from the committed ncu summary, valid only
-    while the kernel source is unchanged since the counters were taken."""
+    for the workload it was captured on and while the kernel source is unchanged
+    since the counters were taken."""
     p = os.path.join(ROOT, "profiles", "traffic.json")
     if not os.path.exists(p) or not os.path.exists(ATTN_KERNEL_SRC):
         return None
     with open(p) as f:
         rec = json.load(f)
-    if rec.get("source_sha") != file_sha(ATTN_KERNEL_SRC):
+    if rec.get("source_sha") != file_sha(ATTN_KERNEL_SRC) or rec.get("workload") != workload:
         return None
     return rec
 
@@ -400,7 +401,7 @@ def run_ours(args, shape):
     attn_s = stage_ms[2] / 1e3
     attn_tflops = work["attention_flops"] / attn_s / 1e12
     peak = float(peaks.get("bf16_tflops", FALLBACK_PEAKS["bf16_tflops"]))
-    traffic = traffic_record()
+    traffic = traffic_record(args.workload)
     roofline = {
         "kernel": "attention (tcgen05)" if path_tensor else "attention (SIMT)",
         "bound": "tensor", "achieved": attn_tflops, "peak": peak, "unit": "TFLOP/s",

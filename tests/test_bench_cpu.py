@@ -59,3 +59,16 @@ def test_clock_samples_directory(monkeypatch, tmp_path):
     assert bench.ClockSampler(1).path == str(tmp_path / "cca_bench_clocks_rank1.csv")
     monkeypatch.delenv("CCA_BENCH_CLOCKS_DIR")
     assert bench.ClockSampler(0).path.startswith(tempfile.gettempdir())
+
+
+def test_traffic_record_only_for_its_workload_and_source():
+    """The committed DRAM traffic of the attention kernel is reported only for the workload it was
+    captured on, and only while the kernel source hashes as it did then."""
+    with open(os.path.join(ROOT, "profiles", "traffic.json")) as f:
+        rec = json.load(f)
+    current = rec["source_sha"] == bench.file_sha(bench.ATTN_KERNEL_SRC)
+    got = bench.traffic_record(rec["workload"])
+    assert (got is not None) == current
+    for name in workloads.WORKLOADS:
+        if name != rec["workload"]:
+            assert bench.traffic_record(name) is None
