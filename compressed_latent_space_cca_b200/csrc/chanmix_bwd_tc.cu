@@ -5,10 +5,11 @@
 // gradient dc of c:
 //   ds[t] = W_c^T dc[t]            (the gradient passed on to the sequence conv)
 //   dW_c  = sum_t dc[t] s[t]^T     (s recomputed from the latents by the sequence conv)
-// A CTA per (block of rows, head) walks 128-row tiles. Its 512 threads (a column and a quarter of the
-// rows each) load the tile's dc (fp32) and the latent rows, recompute s, and write both as bf16 pairs
-// hi = bf16(v),
-// lo = bf16(v - hi) into shared memory (128-byte swizzle). The dc tile serves twice: K-major (rows t,
+// A CTA per (block of rows, head) walks 128-row tiles. W_c arrives by asynchronous 16-byte copies
+// straight into its swizzled operand layout, and each tile's dc (fp32) is copied the same way into a
+// staging buffer while the previous tile's MMAs and ds rows run. Its 512 threads (a column and a
+// quarter of the rows each) read dc from there and the latent rows from global memory, recompute s,
+// and write both as bf16 pairs hi = bf16(v), lo = bf16(v - hi) into shared memory (128-byte swizzle). The dc tile serves twice: K-major (rows t,
 // k = i) as the A operand of ds, and read MN-major (m = i, k = t) as the A operand of dW_c. One
 // elected thread issues the MMAs:
 //   ds (TMEM columns 0..127)    = [dc_hi | dc_lo] x [W_c; W_c]       (K = 256 over the two segments)
@@ -28,12 +29,14 @@ constexpr int CT_RQ = CT_THREADS / CD;  // row quarters of a tile
 constexpr int CT_RROWS = CT / CT_RQ;    // rows of a tile per thread
 constexpr int HALF = CT * 128;  // 16 KB: 128 rows x 64 bf16 (one 128-byte swizzle span)
 // shared memory: W_c [2 column halves], dc [4 K chunks: hi i 0-63, hi i 64-127, lo, lo],
-// s [4: hi j 0-63, hi j 64-127, lo, lo], barrier
+// s [4: hi j 0-63, hi j 64-127, lo, lo], the next tile's dc (fp32 [128 rows][128]), barrier
 constexpr int OFF_W = 0;
 constexpr int OFF_DC = OFF_W + 2 * HALF;
 constexpr int OFF_S = OFF_DC + 4 * HALF;
-constexpr int OFF_BAR = OFF_S + 4 * HALF;
+constexpr int OFF_STG = OFF_S + 4 * HALF;
+constexpr int OFF_BAR = OFF_STG + CT * CD * 4;
 constexpr size_t CT_SMEM = OFF_BAR + 64 + 1024;
+static_assert(CT_SMEM <= 232448, "shared memory of one CTA");
 constexpr int CT_KMAX = 8;
 
 // byte offset of element (row, col) of a [rows][64-column half] bf16 tile with the 128-byte swizzle
@@ -45,7 +48,27 @@ __device__ __forceinline__ void st_bf16(uint8_t* base, uint32_t off, __nv_bfloat
   *reinterpret_cast<__nv_bfloat16*>(base + off) = v;
 }
 
-template <typename Tl, typename Tc>
+__device__ __forceinline__ void cp_async16(uint32_t dst, const void* src) {
+  asm volatile("cp.async.cg.shared.global [%0], [%1], 16;" ::"r"(dst), "l"(src) : "memory");
+}
+__device__ __forceinline__ void cp_async_commit() { asm volatile("cp.async.commit_group;" ::: "memory"); }
+__device__ __forceinline__ void cp_async_wait_all() { asm volatile("cp.async.wait_group 0;" ::: "memory"); }
+
+// rows [t0, t0 + 128) of this head's dc columns into the staging buffer, 16 bytes per copy (rows at
+// or past r_end are not copied: the tile's reads skip them)
+__device__ __forceinline__ void stage_dc(uint8_t* smem, const float* dc, long long t0, long long r_end, int W,
+                                         int ccol, int tid) {
+#pragma unroll
+  for (int u = 0; u < CT * CD / 4 / CT_THREADS; ++u) {
+    const int c = u * CT_THREADS + tid, r = c / (CD / 4), q = c % (CD / 4);
+    if (t0 + r < r_end) cp_async16(smem_u32(smem + OFF_STG + (r * CD + 4 * q) * 4), dc + (t0 + r) * W + ccol + 4 * q);
+  }
+  cp_async_commit();
+}
+
+// bf16 blocks: fp16 latents, bf16 weights (W_c is copied as it is: bf16 is the operand type)
+using Tl = __half;
+using Tc = __nv_bfloat16;
 __global__ void __launch_bounds__(CT_THREADS, 1)
     chanmix_bwd_tc_kernel(const float* __restrict__ dc, const Tl* __restrict__ lat, const Tc* __restrict__ cq_chan,
                           const Tc* __restrict__ ck_chan, const Tc* __restrict__ cq_seq, const Tc* __restrict__ ck_seq,
@@ -72,17 +95,21 @@ __global__ void __launch_bounds__(CT_THREADS, 1)
     tmem_alloc(smem_u32(tmem_slot), 256);
     tmem_relinquish();
   }
-  // W_c[i][j] as the MN-major B operand of ds (n = j contiguous, k = i rows): [2 j-halves][128 i][64]
-  for (int e = tid; e < CD * CD; e += CT_THREADS) {
-    const int i = e / CD, j = e % CD;
-    st_bf16(smem + OFF_W + (j >> 6) * HALF, sw_off(i, j & 63), __float2bfloat16_rn(ld_f(wsrc + e)));
+  // W_c[i][j] as the MN-major B operand of ds (n = j contiguous, k = i rows): [2 j-halves][128 i][64];
+  // 8 columns of a row per copy land in one 16-byte chunk of the swizzled row
+#pragma unroll
+  for (int u = 0; u < CD * CD / 8 / CT_THREADS; ++u) {
+    const int c = u * CT_THREADS + tid, i = c / (CD / 8), j0 = (c % (CD / 8)) * 8;
+    cp_async16(smem_u32(smem + OFF_W + (j0 >> 6) * HALF + sw_off(i, j0 & 63)), wsrc + (size_t)i * CD + j0);
   }
+  const long long r_begin = (long long)blockIdx.x * rows_per_cta;
+  const long long r_end = r_begin + rows_per_cta < T ? r_begin + rows_per_cta : T;
+  stage_dc(smem, dc, r_begin, r_end, W, ccol, tid);  // commits W_c's copies too
   // this thread's column j (and row quarter rq of each tile): its seq taps
   const int j = tid % CD, rq = tid / CD;
   float taps[CT_KMAX];
 #pragma unroll
   for (int k = 0; k < CT_KMAX; ++k) taps[k] = k < K ? ld_f(wseq + (size_t)j * K + k) : 0.f;
-  fence_async_smem();
   tc_fence_before();
   __syncthreads();
   tc_fence_after();
@@ -97,12 +124,13 @@ __global__ void __launch_bounds__(CT_THREADS, 1)
   const uint32_t w_lo = desc_lo(smem_desc_sw128(smem_u32(smem + OFF_W), HALF, 1024));
   const uint32_t s_lo = desc_lo(smem_desc_sw128(smem_u32(smem + OFF_S), HALF, 1024));
 
-  const long long r_begin = (long long)blockIdx.x * rows_per_cta;
-  const long long r_end = r_begin + rows_per_cta < T ? r_begin + rows_per_cta : T;
   bool ok = true;
   uint32_t phase = 0;
   int ntile = 0;
   for (long long t0 = r_begin; t0 < r_end; t0 += CT, ++ntile) {
+    // this tile's dc (and, for the first, W_c) in shared memory, from every thread's copies
+    cp_async_wait_all();
+    __syncthreads();
     // ---- operands of this tile: column j of dc and of s for rows t0 .. t0 + 127
     {
       // win[k] = latent of row t - (K-1) + k, k < K-1 (zero before row 0; taps that reach before a
@@ -123,7 +151,7 @@ __global__ void __launch_bounds__(CT_THREADS, 1)
         for (int u = 0; u < 8; ++u) {  // independent loads first
           const long long row = t0 + r0 + u;
           const bool in = row < r_end;
-          dv[u] = in ? dc[row * W + ccol + j] : 0.f;
+          dv[u] = in ? reinterpret_cast<const float*>(smem + OFF_STG)[(r0 + u) * CD + j] : 0.f;
           lv[u] = in ? ld_f(lat + row * Nlat + ccol + j) : 0.f;
         }
 #pragma unroll
@@ -146,10 +174,12 @@ __global__ void __launch_bounds__(CT_THREADS, 1)
         }
       }
     }
-    fence_async_smem();  // the generic-proxy stores above are read by the tensor core
+    fence_async_smem();  // the generic-proxy stores above (and W_c's copies) are read by the tensor core
     tc_fence_before();
     __syncthreads();
     tc_fence_after();
+    // the staging buffer has been read: the next tile's dc comes in while this tile's MMAs run
+    if (t0 + CT < r_end) stage_dc(smem, dc, t0 + CT, r_end, W, ccol, tid);
     if (warp == 0) {
       // ds = [dc_hi | dc_lo] [W_c; W_c]: 16 K steps; dc K-major (4 chunks of 64), W_c rows i by 16
 #pragma unroll
@@ -231,12 +261,18 @@ __global__ void __launch_bounds__(CT_THREADS, 1)
 
 }  // namespace
 
-bool chanmix_bwd_tc_supported(const BlockDims& dm) { return dm.d == CD && dm.K >= 1 && dm.K <= CT_KMAX; }
+bool chanmix_bwd_tc_supported(const BlockDims& dm) {
+  return dm.d == CD && dm.K >= 1 && dm.K <= CT_KMAX && dm.io == DType::BF16 && dm.lat == DType::F16;
+}
 
 cudaError_t launch_chanmix_bwd_tc(const BlockDims& dm, const float* dc, const void* lat, const void* cq_chan,
                                   const void* ck_chan, const void* cq_seq, const void* ck_seq, float* ds, float* dwq,
                                   float* dwk, unsigned* err, cudaStream_t stream) {
   if (!chanmix_bwd_tc_supported(dm)) return cudaErrorInvalidValue;
+  // W_c and dc arrive by 16-byte copies
+  if (((reinterpret_cast<uintptr_t>(cq_chan) | reinterpret_cast<uintptr_t>(ck_chan) |
+        reinterpret_cast<uintptr_t>(dc)) & 15) != 0)
+    return cudaErrorInvalidValue;
   const int heads = dm.nq + dm.nkv;
   // row blocks: about two CTAs per SM over all heads, whole tiles
   long long tiles = (dm.T + CT - 1) / CT;
@@ -245,25 +281,13 @@ cudaError_t launch_chanmix_bwd_tc(const BlockDims& dm, const float* dc, const vo
   const int rows = (int)(per * CT);
   const dim3 grid((unsigned)((dm.T + rows - 1) / rows), heads);
   cudaError_t e;
-  if (dm.lat == DType::F16 && dm.io == DType::BF16) {
-    auto k = chanmix_bwd_tc_kernel<__half, __nv_bfloat16>;
-    if ((e = cudaFuncSetAttribute(k, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)CT_SMEM)) != cudaSuccess)
-      return e;
-    k<<<grid, CT_THREADS, CT_SMEM, stream>>>(dc, static_cast<const __half*>(lat),
-                                             static_cast<const __nv_bfloat16*>(cq_chan),
-                                             static_cast<const __nv_bfloat16*>(ck_chan),
-                                             static_cast<const __nv_bfloat16*>(cq_seq),
-                                             static_cast<const __nv_bfloat16*>(ck_seq), ds, dwq, dwk, dm.T, dm.S, dm.nq,
-                                             dm.nkv, dm.K, rows, err);
-  } else {
-    auto k = chanmix_bwd_tc_kernel<float, float>;
-    if ((e = cudaFuncSetAttribute(k, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)CT_SMEM)) != cudaSuccess)
-      return e;
-    k<<<grid, CT_THREADS, CT_SMEM, stream>>>(dc, static_cast<const float*>(lat), static_cast<const float*>(cq_chan),
-                                             static_cast<const float*>(ck_chan), static_cast<const float*>(cq_seq),
-                                             static_cast<const float*>(ck_seq), ds, dwq, dwk, dm.T, dm.S, dm.nq,
-                                             dm.nkv, dm.K, rows, err);
-  }
+  if ((e = cudaFuncSetAttribute(chanmix_bwd_tc_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)CT_SMEM)) !=
+      cudaSuccess)
+    return e;
+  chanmix_bwd_tc_kernel<<<grid, CT_THREADS, CT_SMEM, stream>>>(
+      dc, static_cast<const __half*>(lat), static_cast<const __nv_bfloat16*>(cq_chan),
+      static_cast<const __nv_bfloat16*>(ck_chan), static_cast<const __nv_bfloat16*>(cq_seq),
+      static_cast<const __nv_bfloat16*>(ck_seq), ds, dwq, dwk, dm.T, dm.S, dm.nq, dm.nkv, dm.K, rows, err);
   return cudaGetLastError();
 }
 
