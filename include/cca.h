@@ -321,9 +321,15 @@ cca_status_t cca_decode(const cca_config_t* cfg, int cache_rows,
  * every weight, for the same inputs as cca_prefill.
  *
  * The forward's activations are recomputed first, by the forward's own
- * kernels (the path AUTO picks), into the workspace; the backward's kernels
- * then run in fp32 on the CUDA cores, reading the forward's 16-bit
- * intermediates where cfg->dtype is bf16.
+ * kernels (the path AUTO picks), into the workspace. Then, for bf16 blocks
+ * with head_dim 128 on sm_100, the attention backward, the channel-mix
+ * backward and the projection gradients run on the tensor cores: fp16 or
+ * bf16 operands, and fp32 values that bf16 does not hold exactly split into
+ * bf16 high and low parts, all accumulating in fp32. The remaining
+ * transposes (RoPE, QK-mean, value shift, sequence conv) run in fp32 on the
+ * CUDA cores. Other blocks run every step in fp32 on the CUDA cores. The
+ * reductions over tokens use atomic fp32 additions, so repeated calls agree
+ * to rounding, not bit for bit.
  *
  *   x ... W_o   as in cca_prefill, cfg->dtype
  *   dy          [B, S, E]              cfg->out_dtype
